@@ -1,0 +1,154 @@
+"""fp64 CPU oracle for the selective scan (S6) forward pass and state update.
+
+TEST INFRASTRUCTURE ONLY.  Only the test-suite, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py`` may import this package.  It shares
+no code with the CUDA library in ``selective_state_space_20_b200``; neither
+imports the other.
+
+The arithmetic lives in ``s6_oracle.c`` (a plain sequential fp64 loop, see
+its header for the equations and where each comes from).  This module only
+marshals numpy/torch CPU arrays into it:
+
+* :func:`scan` -- the whole forward scan (optionally from an initial state).
+* :func:`state_update` -- one recurrent step for every (batch, channel).
+* :func:`softplus`, :func:`silu` -- the pointwise functions the oracle uses.
+
+Inputs may be numpy arrays or CPU torch tensors of any float dtype; they are
+widened to fp32 (exact for bf16 and fp32 values) before the call, and all
+arithmetic happens in fp64 inside the C code.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load (building first if needed) an oracle shared library."""
+    lib = ctypes.CDLL(path or _build.build())
+    f32p = ctypes.POINTER(ctypes.c_float)
+    f64p = ctypes.POINTER(ctypes.c_double)
+    i64 = ctypes.c_int64
+    lib.s6_oracle_scan.restype = ctypes.c_int
+    lib.s6_oracle_scan.argtypes = [f32p, f32p, f32p, f32p, f32p, f32p, f32p,
+                                   f32p, ctypes.c_int, f64p, f64p, f64p,
+                                   i64, i64, i64, i64, ctypes.c_int]
+    lib.s6_oracle_state_update.restype = ctypes.c_int
+    lib.s6_oracle_state_update.argtypes = [f64p, f32p, f32p, f32p, f32p, f32p,
+                                           f32p, f32p, f32p, ctypes.c_int, f64p,
+                                           i64, i64, i64]
+    lib.s6_oracle_softplus.restype = ctypes.c_double
+    lib.s6_oracle_softplus.argtypes = [ctypes.c_double]
+    lib.s6_oracle_silu.restype = ctypes.c_double
+    lib.s6_oracle_silu.argtypes = [ctypes.c_double]
+    return lib
+
+
+def _get():
+    global _lib
+    if _lib is None:
+        _lib = load_library()
+    return _lib
+
+
+def _f32(x):
+    """Exact fp32 numpy copy of an array/tensor (None passes through)."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor
+        x = x.detach().to("cpu")
+        import torch
+        x = x.to(torch.float32).contiguous().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        import torch
+        x = x.detach().to("cpu").to(torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _p32(a):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+
+
+def _p64(a):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+         delta_softplus: bool = True, h0=None, nthreads: int = 0,
+         lib: Optional[ctypes.CDLL] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Selective scan forward in fp64.
+
+    Shapes: u, delta, z (batch, dim, L); B, C (batch, N, L); A (dim, N);
+    D, delta_bias (dim,); h0 (batch, dim, N).  Returns ``(out, last_state)``
+    as fp64 arrays of shapes (batch, dim, L) and (batch, dim, N).
+    """
+    lib = lib or _get()
+    u, delta, A, B, C = (_f32(t) for t in (u, delta, A, B, C))
+    D, z, delta_bias = _f32(D), _f32(z), _f32(delta_bias)
+    h0 = _f64(h0)
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    assert delta.shape == u.shape and (z is None or z.shape == u.shape)
+    assert A.shape == (dim, N) and B.shape == (batch, N, L) and C.shape == B.shape
+    assert D is None or D.shape == (dim,)
+    assert delta_bias is None or delta_bias.shape == (dim,)
+    assert h0 is None or h0.shape == (batch, dim, N)
+    out = np.empty((batch, dim, L), dtype=np.float64)
+    last = np.empty((batch, dim, N), dtype=np.float64)
+    rc = lib.s6_oracle_scan(_p32(u), _p32(delta), _p32(A), _p32(B), _p32(C),
+                            _p32(D), _p32(z), _p32(delta_bias),
+                            int(bool(delta_softplus)), _p64(h0), _p64(out),
+                            _p64(last), batch, dim, L, N, int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_scan failed with code {rc}")
+    return out, last
+
+
+def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                 delta_softplus: bool = True,
+                 lib: Optional[ctypes.CDLL] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """One recurrent step.  Returns ``(out, new_state)`` in fp64.
+
+    Shapes: state (batch, dim, N); u, delta, z (batch, dim); B, C (batch, N);
+    A (dim, N); D, delta_bias (dim,).  ``state`` is not modified.
+    """
+    lib = lib or _get()
+    st = _f64(state).copy()
+    u, delta, A, B, C = (_f32(t) for t in (u, delta, A, B, C))
+    D, z, delta_bias = _f32(D), _f32(z), _f32(delta_bias)
+    batch, dim = u.shape
+    N = A.shape[1]
+    assert st.shape == (batch, dim, N) and B.shape == (batch, N) and C.shape == B.shape
+    out = np.empty((batch, dim), dtype=np.float64)
+    rc = lib.s6_oracle_state_update(_p64(st), _p32(u), _p32(delta), _p32(A),
+                                    _p32(B), _p32(C), _p32(D), _p32(z),
+                                    _p32(delta_bias), int(bool(delta_softplus)),
+                                    _p64(out), batch, dim, N)
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_state_update failed with code {rc}")
+    return out, st
+
+
+def softplus(x: float, lib: Optional[ctypes.CDLL] = None) -> float:
+    return (lib or _get()).s6_oracle_softplus(float(x))
+
+
+def silu(x: float, lib: Optional[ctypes.CDLL] = None) -> float:
+    return (lib or _get()).s6_oracle_silu(float(x))
+
+
+def library_path() -> str:
+    return os.path.abspath(_build.LIB)

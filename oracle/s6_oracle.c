@@ -1,0 +1,227 @@
+/*
+ * s6_oracle.c -- plain fp64 CPU reference of the selective scan (S6) forward
+ * pass and of its one-token state update.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file; only the test-suite, the smoke check and the benchmark's CPU
+ * baseline use it.  It shares no code, header, table or constant with the CUDA
+ * library.
+ *
+ * What it computes (one independent recurrence per (batch b, channel d)):
+ *
+ *   delta_t = delta_raw[b,d,t] + bias[d]              (bias added before softplus:
+ *                                                      "Mamba SSM concept and
+ *                                                      implementation in Keras and
+ *                                                      TensorFlow", MambaBlock.ssm,
+ *                                                      where dt_proj carries the bias
+ *                                                      and softplus follows it)
+ *   delta_t = softplus(delta_t)   if the flag is set  (same page, MambaBlock.ssm)
+ *   Abar    = exp(delta_t * A[d,n])                   (zero-order hold of A; same page,
+ *                                                      "Going from continuous to discrete
+ *                                                      spaces" and selective_scan, "first
+ *                                                      step of A_bar = exp(dA)")
+ *   Bbar u  = delta_t * B[b,n,t] * u[b,d,t]           (the simplified B discretisation the
+ *                                                      same selective_scan uses for dB_u)
+ *   h_t[n]  = Abar * h_{t-1}[n] + Bbar u              (recurrent form, h_{-1} = h0, zero
+ *                                                      by default: same page, "assuming
+ *                                                      h0 = zero")
+ *   y_t     = sum_n C[b,n,t] * h_t[n] + D[d] * u[b,d,t]   (readout plus the D skip; same
+ *                                                      page, selective_scan "y + u * D")
+ *   out_t   = y_t * silu(z[b,d,t])    if z is given   (gate; same page, MambaBlock.call
+ *                                                      "y * swish(res)")
+ *   last_state[b,d,n] = h_{L-1}[n]
+ *
+ * Layouts (row-major, contiguous):
+ *   u, delta_raw, z, out : (batch, dim, seqlen)
+ *   B, C                 : (batch, dstate, seqlen)
+ *   A                    : (dim, dstate)
+ *   D, bias              : (dim)
+ *   h0, last_state, state: (batch, dim, dstate)
+ *
+ * Inputs arrive as fp32 arrays holding the exact values the device sees
+ * (bf16 values widen to fp32 exactly); every operation below is done in fp64,
+ * in the order written above, with no blocking, fusion or reordering.
+ * Time is strictly sequential; independent (b, d) rows are spread over
+ * POSIX threads, which does not change any result.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <unistd.h>
+
+/* softplus(x) = ln(1 + e^x), written in the overflow-free split form
+ * max(x, 0) + ln(1 + e^{-|x|}); the Keras/TensorFlow page applies
+ * tf.nn.softplus to the dt projection. */
+double s6_oracle_softplus(double x)
+{
+    if (x > 0.0)
+        return x + log1p(exp(-x));
+    return log1p(exp(x));
+}
+
+/* silu(z) = z * sigmoid(z) = z / (1 + e^{-z}) (the page's tf.nn.swish). */
+double s6_oracle_silu(double z)
+{
+    return z / (1.0 + exp(-z));
+}
+
+typedef struct {
+    const float *u, *delta, *A, *B, *C, *D, *z, *bias;
+    const double *h0;
+    int softplus;
+    double *out, *last_state;
+    int64_t dim, seqlen, dstate;
+    int64_t row_begin, row_end; /* rows are flattened (b * dim + d) */
+} scan_job_t;
+
+/* One (b, d) recurrence over the whole sequence. */
+static void scan_row(const scan_job_t *j, int64_t row, double *h)
+{
+    const int64_t L = j->seqlen, N = j->dstate;
+    const int64_t b = row / j->dim, d = row % j->dim;
+    const float *u = j->u + row * L;
+    const float *dr = j->delta + row * L;
+    const float *z = j->z ? j->z + row * L : NULL;
+    const float *Bb = j->B + b * N * L;
+    const float *Cb = j->C + b * N * L;
+    const float *Ad = j->A + d * N;
+    const double Dd = j->D ? (double)j->D[d] : 0.0;
+    const double bias = j->bias ? (double)j->bias[d] : 0.0;
+    double *out = j->out + row * L;
+
+    for (int64_t n = 0; n < N; ++n)
+        h[n] = j->h0 ? j->h0[row * N + n] : 0.0;
+
+    for (int64_t t = 0; t < L; ++t) {
+        double delta = (double)dr[t] + bias;
+        if (j->softplus)
+            delta = s6_oracle_softplus(delta);
+        const double ut = (double)u[t];
+        double y = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            const double Abar = exp(delta * (double)Ad[n]);
+            const double Bbar_u = delta * (double)Bb[n * L + t] * ut;
+            h[n] = Abar * h[n] + Bbar_u;
+            y += (double)Cb[n * L + t] * h[n];
+        }
+        y += Dd * ut;
+        if (z)
+            y *= s6_oracle_silu((double)z[t]);
+        out[t] = y;
+    }
+    if (j->last_state)
+        for (int64_t n = 0; n < N; ++n)
+            j->last_state[row * N + n] = h[n];
+}
+
+static void *scan_worker(void *arg)
+{
+    const scan_job_t *j = (const scan_job_t *)arg;
+    double *h = (double *)malloc(sizeof(double) * (size_t)j->dstate);
+    if (!h)
+        return (void *)1;
+    for (int64_t row = j->row_begin; row < j->row_end; ++row)
+        scan_row(j, row, h);
+    free(h);
+    return NULL;
+}
+
+/* Full scan over all (b, d) rows.  nthreads <= 0 uses every online core.
+ * Returns 0 on success, -1 on bad arguments, -2 on allocation failure. */
+int s6_oracle_scan(const float *u, const float *delta, const float *A,
+                   const float *B, const float *C, const float *D,
+                   const float *z, const float *delta_bias, int softplus,
+                   const double *h0, double *out, double *last_state,
+                   int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                   int nthreads)
+{
+    if (!u || !delta || !A || !B || !C || !out)
+        return -1;
+    if (batch <= 0 || dim <= 0 || seqlen <= 0 || dstate <= 0)
+        return -1;
+    const int64_t rows = batch * dim;
+    if (nthreads <= 0) {
+        long nc = sysconf(_SC_NPROCESSORS_ONLN);
+        nthreads = nc > 0 ? (int)nc : 1;
+    }
+    if (nthreads > rows)
+        nthreads = (int)rows;
+
+    scan_job_t base = {u, delta, A, B, C, D, z, delta_bias, h0, softplus,
+                       out, last_state, dim, seqlen, dstate, 0, rows};
+    if (nthreads == 1) {
+        return scan_worker(&base) ? -2 : 0;
+    }
+    scan_job_t *jobs = (scan_job_t *)malloc(sizeof(scan_job_t) * (size_t)nthreads);
+    pthread_t *tids = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!jobs || !tids) {
+        free(jobs);
+        free(tids);
+        return -2;
+    }
+    int rc = 0;
+    int started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i] = base;
+        jobs[i].row_begin = rows * i / nthreads;
+        jobs[i].row_end = rows * (i + 1) / nthreads;
+        if (pthread_create(&tids[i], NULL, scan_worker, &jobs[i]) != 0) {
+            /* run the remainder on this thread */
+            jobs[i].row_end = rows;
+            if (scan_worker(&jobs[i]))
+                rc = -2;
+            break;
+        }
+        ++started;
+    }
+    for (int i = 0; i < started; ++i) {
+        void *ret = NULL;
+        pthread_join(tids[i], &ret);
+        if (ret)
+            rc = -2;
+    }
+    free(jobs);
+    free(tids);
+    return rc;
+}
+
+/* One recurrent step for every (b, d): the same update as one iteration of
+ * the scan's time loop, applied to a state held by the caller (the decoding
+ * form that generation uses one token at a time).
+ *   state       : (batch, dim, dstate), read and overwritten
+ *   u, delta, z : (batch, dim);  B, C : (batch, dstate);  out : (batch, dim) */
+int s6_oracle_state_update(double *state, const float *u, const float *delta,
+                           const float *A, const float *B, const float *C,
+                           const float *D, const float *z,
+                           const float *delta_bias, int softplus, double *out,
+                           int64_t batch, int64_t dim, int64_t dstate)
+{
+    if (!state || !u || !delta || !A || !B || !C || !out)
+        return -1;
+    if (batch <= 0 || dim <= 0 || dstate <= 0)
+        return -1;
+    const int64_t N = dstate;
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < dim; ++d) {
+            const int64_t row = b * dim + d;
+            double delta_t = (double)delta[row] + (delta_bias ? (double)delta_bias[d] : 0.0);
+            if (softplus)
+                delta_t = s6_oracle_softplus(delta_t);
+            const double ut = (double)u[row];
+            double *h = state + row * N;
+            double y = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                const double Abar = exp(delta_t * (double)A[d * N + n]);
+                const double Bbar_u = delta_t * (double)B[b * N + n] * ut;
+                h[n] = Abar * h[n] + Bbar_u;
+                y += (double)C[b * N + n] * h[n];
+            }
+            y += (D ? (double)D[d] : 0.0) * ut;
+            if (z)
+                y *= s6_oracle_silu((double)z[row]);
+            out[row] = y;
+        }
+    }
+    return 0;
+}

@@ -1,0 +1,385 @@
+"""Pins for the fp64 oracle: checks against facts fixed by the mathematics,
+not by the oracle's own code.
+
+Each ``pin_*`` function takes an oracle library handle (the real one, or a
+copy of the oracle compiled with a planted mistake) and raises
+``AssertionError`` if the oracle disagrees with the independent fact.  The
+expected values are computed here by other means -- a closed form, a
+convolution, a library routine, an explicit product formula -- never by the
+oracle's recurrence.
+
+Sources of the facts (titles of the pages the method is described on):
+* recurrence, ZOH exponent, dB_u = delta*B*u, y + u*D and the swish gate:
+  "Mamba SSM concept and implementation in Keras and TensorFlow", sections
+  "Going from continuous to discrete spaces", the selective_scan listing and
+  MambaBlock.call/ssm;
+* convolutional (LTI) form with kernel K_k = C Abar^k Bbar: same page, the
+  convolutional-kernel discussion ("assuming h0 = zero");
+* the cumulative-sum (log-space) form: same page, selective_scan listing.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy import signal, special
+
+import oracle
+
+RTOL = 1e-11
+
+
+def _close(a, b, rtol=RTOL, scale=None, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, (what, a.shape, b.shape)
+    s = scale if scale is not None else max(1e-300, float(np.max(np.abs(b))))
+    err = float(np.max(np.abs(a - b))) / s if a.size else 0.0
+    assert err <= rtol, f"{what}: normwise error {err:.3e} > {rtol:.1e}"
+
+
+def _f32(x):
+    return np.asarray(x, dtype=np.float32)
+
+
+# ---------------------------------------------------------------- pointwise
+def pin_softplus_silu(lib):
+    """softplus against numpy's logaddexp(0, x) = ln(e^0 + e^x) and the
+    identity softplus(x) - softplus(-x) = x; silu against x * expit(x)."""
+    xs = [-40.0, -20.0, -9.21, -3.0, -0.5, 0.0, 1e-8, 0.3, 2.0, 15.0, 40.0]
+    for x in xs:
+        sp = oracle.softplus(x, lib=lib)
+        ref = float(np.logaddexp(0.0, x))
+        assert abs(sp - ref) <= 1e-15 * abs(ref), ("softplus", x, sp, ref)
+        assert abs((sp - oracle.softplus(-x, lib=lib)) - x) <= 1e-14 * max(1.0, abs(x))
+        si = oracle.silu(x, lib=lib)
+        ref = x * float(special.expit(x))
+        assert abs(si - ref) <= 1e-15 * max(1e-300, abs(ref)) + 1e-300, ("silu", x, si, ref)
+    assert abs(oracle.softplus(0.0, lib=lib) - math.log(2.0)) < 1e-16
+
+
+# ---------------------------------------------------------------- closed forms
+def _const_problem(L, N, softplus, raw, bias, u, Bv, Cv, Av, Dv, zv=None):
+    shape = (1, 1, L)
+    ins = dict(
+        u=np.full(shape, u, np.float32),
+        delta=np.full(shape, raw, np.float32),
+        A=_f32(np.asarray(Av).reshape(1, N)),
+        B=np.repeat(_f32(np.asarray(Bv).reshape(1, N, 1)), L, axis=2),
+        C=np.repeat(_f32(np.asarray(Cv).reshape(1, N, 1)), L, axis=2),
+        D=np.full((1,), Dv, np.float32),
+        z=None if zv is None else np.full(shape, zv, np.float32),
+        delta_bias=np.full((1,), bias, np.float32),
+        delta_softplus=softplus,
+    )
+    return ins
+
+
+def pin_geometric_series(lib):
+    """Constant inputs: h_t = b (1 - a^{t+1}) / (1 - a), a = e^{delta A},
+    b = delta B u; y_t = sum_n C_n h_t[n] + D u, times silu(z)."""
+    L, N = 300, 5
+    raw, bias = np.float32(-0.75), np.float32(-2.5)
+    delta = float(np.logaddexp(0.0, float(raw) + float(bias)))
+    u = np.float32(0.8125)
+    Av = _f32([-1.0, -2.0, -0.37, -5.5, -0.01])
+    Bv = _f32([0.5, -1.25, 2.0, 0.75, 1.5])
+    Cv = _f32([1.5, 0.25, -0.75, 1.0, -2.0])
+    Dv = np.float32(0.625)
+    zv = np.float32(-0.4375)
+    ins = _const_problem(L, N, True, raw, bias, u, Bv, Cv, Av, Dv, zv)
+    out, last = oracle.scan(**ins, lib=lib)
+    t = np.arange(L, dtype=np.float64)[:, None]
+    a = np.exp(delta * Av.astype(np.float64))[None, :]
+    b = (delta * Bv.astype(np.float64) * float(u))[None, :]
+    h = b * (1.0 - a ** (t + 1.0)) / (1.0 - a)
+    y = h @ Cv.astype(np.float64) + float(Dv) * float(u)
+    gate = float(zv) * float(special.expit(float(zv)))
+    _close(out[0, 0], y * gate, what="geometric series out")
+    _close(last[0, 0], h[-1], what="geometric series last_state")
+
+
+def pin_lti_convolution(lib):
+    """delta, B, C constant in time, u random: y = K * u + D u with
+    K_k = sum_n C_n Abar_n^k Bbar_n (Bbar_n = delta B_n), as an explicit
+    causal convolution (numpy.convolve); no gate."""
+    rng = np.random.default_rng(7)
+    L, N = 257, 6
+    raw, bias = np.float32(0.3), np.float32(-3.0)
+    delta = float(np.logaddexp(0.0, float(raw) + float(bias)))
+    Av = _f32(-rng.uniform(0.2, 6.0, N))
+    Bv = _f32(rng.normal(size=N))
+    Cv = _f32(rng.normal(size=N))
+    Dv = np.float32(1.375)
+    u = _f32(rng.normal(size=L))
+    ins = _const_problem(L, N, True, raw, bias, 0.0, Bv, Cv, Av, Dv)
+    ins["u"] = u.reshape(1, 1, L)
+    out, _ = oracle.scan(**ins, lib=lib)
+    k = np.arange(L, dtype=np.float64)[:, None]
+    Abar = np.exp(delta * Av.astype(np.float64))[None, :]
+    K = (Abar ** k) @ (Cv.astype(np.float64) * delta * Bv.astype(np.float64))
+    y = np.convolve(K, u.astype(np.float64))[:L] + float(Dv) * u.astype(np.float64)
+    _close(out[0, 0], y, rtol=1e-10, what="LTI convolution")
+
+
+def pin_first_order_iir(lib):
+    """N = 1 with constant delta and B: h is a first-order recursive filter,
+    h_t = a h_{t-1} + delta B u_t, which scipy.signal.lfilter computes."""
+    rng = np.random.default_rng(11)
+    L = 500
+    raw, bias = np.float32(0.0), np.float32(-1.0)
+    delta = float(np.logaddexp(0.0, -1.0))
+    Av, Bv, Cv, Dv = _f32([-0.7]), _f32([1.75]), _f32([-0.5]), np.float32(0.25)
+    u = _f32(rng.normal(size=L))
+    ins = _const_problem(L, 1, True, raw, bias, 0.0, Bv, Cv, Av, Dv)
+    ins["u"] = u.reshape(1, 1, L)
+    out, last = oracle.scan(**ins, lib=lib)
+    a = math.exp(delta * float(Av[0]))
+    h = signal.lfilter([delta * float(Bv[0])], [1.0, -a], u.astype(np.float64))
+    _close(out[0, 0], float(Cv[0]) * h + float(Dv) * u, rtol=1e-10, what="lfilter")
+    _close(last[0, 0, 0], h[-1], rtol=1e-10, what="lfilter last_state")
+
+
+def pin_zero_step_keeps_state(lib):
+    """delta = 0 (softplus off, zero raw delta and bias): Abar = 1 and
+    Bbar = 0, so the state never moves from h0 and y_t = C_t . h0 + D u_t."""
+    rng = np.random.default_rng(3)
+    Bt, Dm, L, N = 2, 3, 40, 4
+    u = _f32(rng.normal(size=(Bt, Dm, L)))
+    B = _f32(rng.normal(size=(Bt, N, L)))
+    C = _f32(rng.normal(size=(Bt, N, L)))
+    A = _f32(-rng.uniform(0.5, 3, size=(Dm, N)))
+    D = _f32(rng.normal(size=Dm))
+    h0 = rng.normal(size=(Bt, Dm, N))
+    out, last = oracle.scan(u, np.zeros_like(u), A, B, C, D=D, z=None,
+                            delta_bias=np.zeros(Dm, np.float32),
+                            delta_softplus=False, h0=h0, lib=lib)
+    y = np.einsum("bdn,bnl->bdl", h0, C.astype(np.float64)) + D[None, :, None].astype(np.float64) * u
+    _close(out, y, what="delta=0 readout")
+    assert np.array_equal(last, h0), "delta=0 must leave the state unchanged"
+
+
+def pin_memoryless_limit(lib):
+    """Large delta with A < 0: Abar underflows (e^{-60}), so h_t = delta B_t u_t
+    and y_t = delta u_t (B_t . C_t) + D u_t."""
+    rng = np.random.default_rng(5)
+    L, N = 64, 3
+    u = _f32(rng.normal(size=(1, 1, L)))
+    B = _f32(rng.normal(size=(1, N, L)))
+    C = _f32(rng.normal(size=(1, N, L)))
+    A = _f32([[-2.0, -3.0, -4.0]])
+    raw = np.full((1, 1, L), 30.0, np.float32)
+    out, _ = oracle.scan(u, raw, A, B, C, D=_f32([0.5]), z=None,
+                         delta_bias=_f32([0.0]), delta_softplus=True, lib=lib)
+    delta = float(np.logaddexp(0.0, 30.0))
+    u64 = u[0, 0].astype(np.float64)
+    y = delta * u64 * np.sum(B[0].astype(np.float64) * C[0], axis=0) + 0.5 * u64
+    _close(out[0, 0], y, rtol=1e-12, what="memoryless limit")
+
+
+# ---------------------------------------------------------------- brute force
+def _rand_problem(rng, Bt, Dm, L, N, gate=True, small_delta=False):
+    u = _f32(rng.normal(size=(Bt, Dm, L)))
+    delta = _f32(0.5 * rng.normal(size=(Bt, Dm, L)))
+    A = _f32(-rng.uniform(0.3, 4.0, size=(Dm, N)))
+    B = _f32(rng.normal(size=(Bt, N, L)))
+    C = _f32(rng.normal(size=(Bt, N, L)))
+    D = _f32(rng.uniform(0.5, 1.5, size=Dm))
+    z = _f32(rng.normal(size=(Bt, Dm, L))) if gate else None
+    lo, hi = (-6.0, -4.0) if small_delta else (-4.0, 0.0)
+    bias = _f32(rng.uniform(lo, hi, size=Dm))
+    return dict(u=u, delta=delta, A=A, B=B, C=C, D=D, z=z, delta_bias=bias)
+
+
+def pin_brute_force_products(lib):
+    """Tiny shapes, everything time-varying: the state written as the sum of
+    past inputs weighted by explicit products of the discretised decays,
+    h_t = sum_{s<=t} (prod_{k=s+1..t} Abar_k) Bbar_s u_s, in pure Python."""
+    rng = np.random.default_rng(1234)
+    Bt, Dm, L, N = 2, 3, 13, 4
+    p = _rand_problem(rng, Bt, Dm, L, N)
+    out, last = oracle.scan(**p, delta_softplus=True, lib=lib)
+    for b in range(Bt):
+        for d in range(Dm):
+            dl = [float(np.logaddexp(0.0, float(p["delta"][b, d, t]) + float(p["delta_bias"][d])))
+                  for t in range(L)]
+            for t in range(L):
+                y = 0.0
+                hT = []
+                for n in range(N):
+                    acc = 0.0
+                    for s in range(t + 1):
+                        w = 1.0
+                        for k in range(s + 1, t + 1):
+                            w *= math.exp(dl[k] * float(p["A"][d, n]))
+                        acc += w * dl[s] * float(p["B"][b, n, s]) * float(p["u"][b, d, s])
+                    hT.append(acc)
+                    y += float(p["C"][b, n, t]) * acc
+                y += float(p["D"][d]) * float(p["u"][b, d, t])
+                zt = float(p["z"][b, d, t])
+                y *= zt * float(special.expit(zt))
+                assert abs(out[b, d, t] - y) <= 1e-11 * max(1.0, abs(y)), (b, d, t, out[b, d, t], y)
+                if t == L - 1:
+                    _close(last[b, d], hT, rtol=1e-11, what="brute-force last_state")
+
+
+def pin_cumsum_form(lib):
+    """The cumulative-sum form of the scan: with P_t = sum_{k<=t} delta_k A,
+    h_t = e^{P_t} sum_{s<=t} e^{-P_s} Bbar_s u_s (vectorised with numpy
+    cumsum/einsum; valid while e^{-P} stays finite, so short L, small delta)."""
+    rng = np.random.default_rng(99)
+    Bt, Dm, L, N = 2, 4, 48, 5
+    p = _rand_problem(rng, Bt, Dm, L, N, small_delta=True)
+    out, last = oracle.scan(**p, delta_softplus=True, lib=lib)
+    dl = np.logaddexp(0.0, p["delta"].astype(np.float64) + p["delta_bias"][None, :, None])
+    dA = np.einsum("bdl,dn->bdln", dl, p["A"].astype(np.float64))
+    P = np.cumsum(dA, axis=2)
+    dBu = np.einsum("bdl,bnl,bdl->bdln", dl, p["B"].astype(np.float64), p["u"].astype(np.float64))
+    h = np.exp(P) * np.cumsum(np.exp(-P) * dBu, axis=2)
+    y = np.einsum("bdln,bnl->bdl", h, p["C"].astype(np.float64))
+    y = y + p["D"][None, :, None].astype(np.float64) * p["u"]
+    z = p["z"].astype(np.float64)
+    y = y * z * special.expit(z)
+    _close(out, y, rtol=1e-10, what="cumsum form")
+    _close(last, h[:, :, -1, :], rtol=1e-10, what="cumsum form last_state")
+
+
+# ---------------------------------------------------------------- invariants
+def pin_chunk_split(lib):
+    """Scanning [0, L1) then [L1, L) from the carried last_state equals one
+    scan over [0, L), bit for bit."""
+    rng = np.random.default_rng(21)
+    Bt, Dm, L, N = 2, 5, 97, 16
+    p = _rand_problem(rng, Bt, Dm, L, N)
+    full, last = oracle.scan(**p, delta_softplus=True, lib=lib)
+    for L1 in (1, 31, 64, 96):
+        def part(sl):
+            q = dict(p)
+            for k in ("u", "delta", "z", "B", "C"):
+                q[k] = np.ascontiguousarray(p[k][:, :, sl])
+            return q
+        o1, s1 = oracle.scan(**part(slice(0, L1)), delta_softplus=True, lib=lib)
+        o2, s2 = oracle.scan(**part(slice(L1, L)), delta_softplus=True, h0=s1, lib=lib)
+        assert np.array_equal(np.concatenate([o1, o2], axis=2), full), f"split at {L1}"
+        assert np.array_equal(s2, last), f"split at {L1}: last_state"
+
+
+def pin_steps_equal_scan(lib):
+    """L calls of the one-token state update reproduce the scan exactly."""
+    rng = np.random.default_rng(22)
+    Bt, Dm, L, N = 3, 4, 20, 16
+    p = _rand_problem(rng, Bt, Dm, L, N)
+    full, last = oracle.scan(**p, delta_softplus=True, lib=lib)
+    state = np.zeros((Bt, Dm, N))
+    for t in range(L):
+        o, state = oracle.state_update(state, p["u"][:, :, t], p["delta"][:, :, t],
+                                       p["A"], p["B"][:, :, t], p["C"][:, :, t],
+                                       D=p["D"], z=p["z"][:, :, t],
+                                       delta_bias=p["delta_bias"], delta_softplus=True,
+                                       lib=lib)
+        assert np.array_equal(o, full[:, :, t]), f"step {t}"
+    assert np.array_equal(state, last)
+
+
+def pin_causality(lib):
+    """Changing u at time t0 leaves every output before t0 bit-identical and
+    changes the output at t0."""
+    rng = np.random.default_rng(23)
+    p = _rand_problem(rng, 1, 2, 50, 8)
+    o1, _ = oracle.scan(**p, delta_softplus=True, lib=lib)
+    q = dict(p)
+    q["u"] = p["u"].copy()
+    q["u"][:, :, 30] += 1.0
+    o2, _ = oracle.scan(**q, delta_softplus=True, lib=lib)
+    assert np.array_equal(o1[:, :, :30], o2[:, :, :30])
+    assert np.all(o1[:, :, 30] != o2[:, :, 30])
+
+
+def pin_linearity(lib):
+    """With delta fixed and no gate, y is linear in u (and affine in B with
+    the D u term counted once): y(u1 + u2) = y(u1) + y(u2)."""
+    rng = np.random.default_rng(24)
+    p = _rand_problem(rng, 2, 3, 40, 6, gate=False)
+    u1 = _f32(rng.normal(size=p["u"].shape))
+    u2 = _f32(rng.normal(size=p["u"].shape))
+    y = {}
+    for name, uu in (("1", u1), ("2", u2), ("12", _f32(u1.astype(np.float64) + u2))):
+        q = dict(p)
+        q["u"] = uu
+        y[name], _ = oracle.scan(**q, delta_softplus=True, lib=lib)
+    # u1 + u2 is exactly representable only approximately in fp32: compare
+    # against the fp32-rounded sum's own linear combination bound.
+    _close(y["12"], y["1"] + y["2"], rtol=1e-6, what="linearity in u")
+    B1 = _f32(rng.normal(size=p["B"].shape))
+    q1, q2 = dict(p), dict(p)
+    q1["B"], q2["B"] = B1, _f32(-B1)
+    ya, _ = oracle.scan(**q1, delta_softplus=True, lib=lib)
+    yb, _ = oracle.scan(**q2, delta_softplus=True, lib=lib)
+    Du = p["D"][None, :, None].astype(np.float64) * p["u"]
+    _close(ya + yb, 2 * Du, rtol=1e-12, scale=float(np.max(np.abs(ya))), what="odd in B")
+
+
+def pin_shared_bc_and_independence(lib):
+    """B and C belong to a batch row and are shared by its channels; rows are
+    independent.  Changing B of batch 1 leaves batch 0 bit-identical, and
+    permuting channels (with A, D, bias) permutes the outputs."""
+    rng = np.random.default_rng(25)
+    p = _rand_problem(rng, 2, 5, 30, 4)
+    o, s = oracle.scan(**p, delta_softplus=True, lib=lib)
+    q = dict(p)
+    q["B"] = p["B"].copy()
+    q["B"][1] *= -2.0
+    o2, _ = oracle.scan(**q, delta_softplus=True, lib=lib)
+    assert np.array_equal(o[0], o2[0]) and not np.array_equal(o[1], o2[1])
+    perm = np.array([3, 0, 4, 1, 2])
+    r = dict(p)
+    for k in ("u", "delta", "z"):
+        r[k] = np.ascontiguousarray(p[k][:, perm])
+    r["A"] = np.ascontiguousarray(p["A"][perm])
+    r["D"] = np.ascontiguousarray(p["D"][perm])
+    r["delta_bias"] = np.ascontiguousarray(p["delta_bias"][perm])
+    o3, s3 = oracle.scan(**r, delta_softplus=True, lib=lib)
+    assert np.array_equal(o3, o[:, perm]) and np.array_equal(s3, s[:, perm])
+
+
+def pin_zero_b_or_c(lib):
+    """B = 0 or C = 0 removes the state's contribution: y = D u silu(z)."""
+    rng = np.random.default_rng(26)
+    p = _rand_problem(rng, 1, 3, 25, 4)
+    z = p["z"].astype(np.float64)
+    y = p["D"][None, :, None] * p["u"].astype(np.float64) * z * special.expit(z)
+    for key in ("B", "C"):
+        q = dict(p)
+        q[key] = np.zeros_like(p[key])
+        o, _ = oracle.scan(**q, delta_softplus=True, lib=lib)
+        _close(o, y, rtol=1e-15, what=f"{key} = 0")
+
+
+def pin_gate_and_softplus_flags(lib):
+    """z = None means no gate; softplus off means delta = raw + bias is used
+    as is (checked on one step against the closed form of a single update)."""
+    rng = np.random.default_rng(27)
+    p = _rand_problem(rng, 1, 2, 1, 3)
+    q = dict(p)
+    q["z"] = None
+    o_nogate, _ = oracle.scan(**q, delta_softplus=True, lib=lib)
+    o_gate, _ = oracle.scan(**p, delta_softplus=True, lib=lib)
+    z = p["z"].astype(np.float64)
+    _close(o_gate, o_nogate * z * special.expit(z), rtol=1e-15, what="gate")
+    # softplus off, one step from h = 0: h = (raw + bias) B u, y = C.h + D u
+    raw = np.abs(p["delta"]).astype(np.float32)
+    q["delta"] = raw
+    o, s = oracle.scan(**q, delta_softplus=False, lib=lib)
+    dl = raw[0, :, 0].astype(np.float64) + p["delta_bias"]
+    h = dl[:, None] * p["B"][0, :, 0].astype(np.float64)[None, :] * p["u"][0, :, 0].astype(np.float64)[:, None]
+    y = h @ p["C"][0, :, 0].astype(np.float64) + p["D"].astype(np.float64) * p["u"][0, :, 0]
+    _close(s[0], h, rtol=1e-15, what="softplus off state")
+    _close(o[0, :, 0], y, rtol=1e-14, what="softplus off out")
+
+
+ALL_PINS = [pin_softplus_silu, pin_geometric_series, pin_lti_convolution,
+            pin_first_order_iir, pin_zero_step_keeps_state, pin_memoryless_limit,
+            pin_brute_force_products, pin_cumsum_form, pin_chunk_split,
+            pin_steps_equal_scan, pin_causality, pin_linearity,
+            pin_shared_bc_and_independence, pin_zero_b_or_c,
+            pin_gate_and_softplus_flags]

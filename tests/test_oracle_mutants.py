@@ -1,0 +1,66 @@
+"""Planted mistakes: each test copies the oracle's C source, plants one
+plausible mistake (a dropped term, a wrong sign or index, a swapped operand),
+compiles the copy on the CPU and checks that at least one pin rejects it.
+This shows the pins are strong enough to catch such a mistake in the real
+oracle.  The real oracle source is never modified.
+"""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins
+from oracle import build as obuild
+
+SRC = open(obuild.SRC).read()
+
+# (id, text in the oracle, replacement)
+MUTANTS = [
+    ("input-term-sign", "h[n] = Abar * h[n] + Bbar_u;\n            y += (double)Cb",
+     "h[n] = Abar * h[n] - Bbar_u;\n            y += (double)Cb"),
+    ("decay-dropped", "h[n] = Abar * h[n] + Bbar_u;\n            y += (double)Cb",
+     "h[n] = h[n] + Bbar_u;\n            y += (double)Cb"),
+    ("update-decay-dropped", "h[n] = Abar * h[n] + Bbar_u;\n                y += (double)C[",
+     "h[n] = h[n] + Bbar_u;\n                y += (double)C["),
+    ("decay-exponent-sign", "exp(delta * (double)Ad[n])", "exp(-delta * (double)Ad[n])"),
+    ("A-index", "exp(delta * (double)Ad[n])", "exp(delta * (double)Ad[0])"),
+    ("D-skip-dropped", "y += Dd * ut;", "y += 0.0 * ut;"),
+    ("gate-dropped", "y *= s6_oracle_silu((double)z[t]);", "y *= 1.0;"),
+    ("B-C-swapped", "(double)Bb[n * L + t] * ut", "(double)Cb[n * L + t] * ut"),
+    ("B-time-lag", "(double)Bb[n * L + t] * ut", "(double)Bb[n * L + (t > 0 ? t - 1 : 0)] * ut"),
+    ("C-reads-old-state", "            h[n] = Abar * h[n] + Bbar_u;\n            y += (double)Cb[n * L + t] * h[n];",
+     "            y += (double)Cb[n * L + t] * h[n];\n            h[n] = Abar * h[n] + Bbar_u;"),
+    ("bias-after-softplus", "double delta = (double)dr[t] + bias;\n        if (j->softplus)\n            delta = s6_oracle_softplus(delta);",
+     "double delta = (double)dr[t];\n        if (j->softplus)\n            delta = s6_oracle_softplus(delta);\n        delta += bias;"),
+    ("softplus-dropped", "            delta = s6_oracle_softplus(delta);\n        const double ut",
+     "            delta = delta;\n        const double ut"),
+    ("Bbar-without-delta", "const double Bbar_u = delta * (double)Bb[n * L + t] * ut;",
+     "const double Bbar_u = (double)Bb[n * L + t] * ut;"),
+    ("B-batch-index", "const float *Bb = j->B + b * N * L;", "const float *Bb = j->B;"),
+    ("h0-ignored", "h[n] = j->h0 ? j->h0[row * N + n] : 0.0;", "h[n] = 0.0;"),
+    ("softplus-wrong-branch", "return log1p(exp(x));", "return log(exp(x));"),
+    ("silu-sigmoid-only", "return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));"),
+    ("state-update-C-lag", "y += (double)C[b * N + n] * h[n];", "y += (double)C[b * N + n] * (h[n] - Bbar_u);"),
+    ("last-state-off-by-one", "j->last_state[row * N + n] = h[n];", "j->last_state[row * N + n] = h[n] * 0.5;"),
+]
+
+
+def test_mutation_patterns_exist():
+    for mid, old, _ in MUTANTS:
+        assert SRC.count(old) == 1, f"mutant {mid}: pattern must occur exactly once"
+
+
+@pytest.mark.parametrize("mid,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(mid, old, new, tmp_path):
+    src = tmp_path / f"mutant_{mid}.c"
+    src.write_text(SRC.replace(old, new, 1))
+    so = str(tmp_path / f"libmutant_{mid}.so")
+    obuild.compile_source(str(src), so)
+    lib = oracle.load_library(so)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(lib)
+        except (AssertionError, RuntimeError, FloatingPointError, ValueError):
+            caught.append(pin.__name__)
+    assert caught, f"planted mistake {mid!r} passed every pin"
