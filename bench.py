@@ -1,0 +1,488 @@
+#!/usr/bin/env python3
+"""Benchmark of the selective-scan forward pass on B200.
+
+One "step" is one fused scan launch (softplus -> discretisation -> recurrence
+-> readout -> D skip -> silu gate -> last state) over the Mamba-2.8B layer
+shape: batch 4, 5120 channels (d_model 2560, expand 2), L = 4096, N = 16,
+bf16 activations, fp32 state and arithmetic.  Inputs are synthetic and
+seeded, resident in HBM, and larger than L2 (504 MB of u/delta/z), so no L2
+flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+prints one JSON line (rank 0).  For N > 1 (torchrun, one process per GPU) every
+rank runs its own problem of the same shape (weak scaling: the (batch,
+channel) recurrences are independent, there is no data-path collective); the
+time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_state_space_20_b200 import binding, inputs  # noqa: E402
+
+WORKLOAD = inputs.MAMBA_2_8B
+METRIC = "scan fwd Gelem/s (batch·dim·L) and % of HBM/MUFU roofline on 1 B200"
+UNIT = "Gelem/s"
+
+# Roofline denominators.  MUFU ex2 throughput is 16 results per clock per SM
+# (CUDA arithmetic-throughput table for compute capability 10.0); one ex2 per
+# (element, state) is the algorithmic exp count.  HBM peak is the measured copy
+# bandwidth of this GPU type.
+SM_COUNT = 148
+MUFU_PER_CLK_PER_SM = 16
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "sm_max_mhz": float(p["sm_max_mhz"]), "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def algorithmic_bytes(w) -> int:
+    """Bytes the scan must move at least once: u, delta, z read, out written
+    (act dtype), B and C read once, A/D/bias read, last_state written."""
+    es = 2 if w.dtype == "bf16" else 4
+    x = w.batch * w.dim * w.seqlen * es
+    bc = 2 * w.batch * w.dstate * w.seqlen * es
+    params = (w.dim * w.dstate + 2 * w.dim) * 4
+    state = w.batch * w.dim * w.dstate * 4
+    return 4 * x + bc + params + state
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_state_space_20_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(name.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel_key: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)
+        e = rec.get(kernel_key)
+        if e and e.get("source_hash") == source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.marks = {}
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, name):
+        self.marks[name] = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0=None, t1=None):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            rows.append((ts, parts))
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+        inside = [r for r in rows if (t0 is None or r[0] >= t0) and (t1 is None or r[0] <= t1)]
+        use = inside if inside else rows
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[1]) for _, p in use if num(p[1]) is not None]
+        mx = [num(p[2]) for _, p in use if num(p[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, p in use for i in range(4) if p[5 + i].lower() == "active"})
+        pw = [num(p[3]) for _, p in use if num(p[3]) is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(use),
+                "samples_in_timed_region": len(inside),
+                "power_w_max": max(pw) if pw else None}
+
+
+# ------------------------------------------------------------ distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ oracle timing
+def time_oracle_sample(w, seconds: float, rank_seed: int = 0):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the workload:
+    the first k channels of batch row 0 over the full sequence length, k sized
+    from a short calibration run for about `seconds` of CPU time."""
+    import oracle
+    cores = os.cpu_count() or 1
+    sub = inputs.custom(1, 64, w.seqlen, w.dstate, w.dtype, seed=w.seed + rank_seed,
+                        dt_min=w.dt_min, dt_max=w.dt_max, d_mode=w.d_mode)
+    cal = inputs.scan_inputs(sub)
+    t0 = time.perf_counter()
+    oracle.scan(cal["u"], cal["delta"], cal["A"], cal["B"], cal["C"], D=cal["D"], z=cal["z"],
+                delta_bias=cal["delta_bias"], nthreads=cores)
+    rate = 64 * w.seqlen / max(time.perf_counter() - t0, 1e-6)  # elements/s
+    k = int(max(cores, min(w.dim * w.batch, rate * seconds / w.seqlen)))
+    k = max(cores, (k // cores) * cores)
+    return k, rate
+
+
+def oracle_step(w, k, data=None):
+    import oracle
+    cores = os.cpu_count() or 1
+    if data is None:
+        sub = inputs.custom(1, k, w.seqlen, w.dstate, w.dtype, seed=w.seed, dt_min=w.dt_min,
+                            dt_max=w.dt_max, d_mode=w.d_mode)
+        data = inputs.scan_inputs(sub)
+    t0 = time.perf_counter()
+    oracle.scan(data["u"], data["delta"], data["A"], data["B"], data["C"], D=data["D"],
+                z=data["z"], delta_bias=data["delta_bias"], nthreads=cores)
+    return time.perf_counter() - t0, data
+
+
+def cpu_baseline(w, seconds=12.0):
+    cores = os.cpu_count() or 1
+    k, _ = time_oracle_sample(w, seconds)
+    dt, _ = oracle_step(w, k)
+    elems = k * w.seqlen
+    return {"value": elems / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"batch row 0, first {k} of {w.dim} channels, full L={w.seqlen}, N={w.dstate}: "
+                      f"{elems} elements in {dt:.2f} s (fp64 C loop, {cores} threads)"}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 oracle, as it stands, on the host cores."""
+    if rank != 0:
+        return 0
+    w = WORKLOAD
+    cores = os.cpu_count() or 1
+    total_budget = 150.0
+    per_step = max(0.05, total_budget / max(1, args.steps + args.warmup))
+    k, _ = time_oracle_sample(w, per_step)
+    data = None
+    for _ in range(args.warmup):
+        _, data = oracle_step(w, k, data)
+    times = []
+    for _ in range(args.steps):
+        dt, data = oracle_step(w, k, data)
+        times.append(dt)
+    tot = sum(times)
+    elems = k * w.seqlen * args.steps
+    value = elems / tot / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "dim": w.dim, "seqlen": w.seqlen,
+                       "dstate": w.dstate, "act_dtype": w.dtype,
+                       "sample_per_step": f"batch row 0, first {k} channels, full L"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{k} channels x L={w.seqlen} x N={w.dstate} per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ GPU timing
+_WS = {}
+
+
+def workspace_for(w, device):
+    key = (w.batch, w.dim, w.seqlen, w.dstate, w.dtype, str(device))
+    if key not in _WS:
+        n = binding.mamba_scan_workspace_size(w.batch, w.dim, w.seqlen, w.dstate, inputs.DTYPES[w.dtype])
+        _WS[key] = torch.empty(max(n, 16), device=device, dtype=torch.uint8)
+    return _WS[key]
+
+
+def scan_call(ins, out, last, ws=None):
+    binding.mamba_scan_fwd(ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"], D=ins["D"],
+                           z=ins["z"], delta_bias=ins["delta_bias"], out=out, last_state=last,
+                           workspace=ws)
+
+
+def time_device(w, ins, steps, warmup):
+    out = torch.empty_like(ins["u"])
+    last = torch.empty(w.batch, w.dim, w.dstate, device=ins["u"].device)
+    ws = workspace_for(w, ins["u"].device)
+    for _ in range(warmup):
+        scan_call(ins, out, last, ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    return out, last, starts, ends, stream
+
+
+def e2e_measure(w, dev_ins, steps):
+    """Same metric through the public API from pinned HOST buffers: every step
+    copies that step's inputs host->device, runs the scan, and reads the
+    output and final state back to the host."""
+    host = {k: (None if v is None else v.to("cpu").pin_memory()) for k, v in dev_ins.items()}
+    per_step = ("u", "delta", "z", "B", "C")
+    dev = {k: (None if v is None else torch.empty_like(v)) for k, v in dev_ins.items()}
+    for k in ("A", "D", "delta_bias"):
+        dev[k] = dev_ins[k]
+    out_h = torch.empty(dev_ins["u"].shape, dtype=dev_ins["u"].dtype).pin_memory()
+    last_h = torch.empty(w.batch, w.dim, w.dstate).pin_memory()
+    out_d = torch.empty_like(dev_ins["u"])
+    last_d = torch.empty(w.batch, w.dim, w.dstate, device=dev_ins["u"].device)
+    h2d = sum(host[k].numel() * host[k].element_size() for k in per_step if host[k] is not None)
+    d2h = out_h.numel() * out_h.element_size() + last_h.numel() * 4
+
+    def one():
+        for k in per_step:
+            if host[k] is not None:
+                dev[k].copy_(host[k], non_blocking=True)
+        scan_call(dev, out_d, last_d, workspace_for(w, out_d.device))
+        out_h.copy_(out_d, non_blocking=True)
+        last_h.copy_(last_d, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    return ms, h2d, d2h
+
+
+def decode_measure(steps=256):
+    """Per-token cost of mamba_state_update on the decoding shape (256 x 5120,
+    N = 16, fp32 state in HBM), captured in a CUDA graph of `steps` calls."""
+    w = inputs.DECODE
+    d = inputs.decode_inputs(w, device="cuda", steps=steps)
+    state = torch.zeros(w.batch, w.dim, w.dstate, device="cuda")
+    outs = torch.empty(steps, w.batch, w.dim, device="cuda", dtype=inputs.DTYPES[w.dtype])
+
+    def run():
+        for t in range(steps):
+            binding.mamba_state_update(state, d["u"][t], d["delta"][t], d["A"], d["B"][t], d["C"][t],
+                                       D=d["D"], z=d["z"][t], delta_bias=d["delta_bias"], out=outs[t])
+    run()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            run()
+    torch.cuda.current_stream().wait_stream(s)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 4
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * steps)
+    bytes_step = w.batch * w.dim * (2 * w.dstate * 4 + 4 * 2) + 2 * w.batch * w.dstate * 2 + w.dim * (w.dstate + 2) * 4
+    del g
+    return {"workload": w.name, "us_per_step": us, "Gelem_per_s": w.batch * w.dim / us / 1e3,
+            "GB_per_s": bytes_step / us / 1e3, "algorithmic_bytes_per_step": bytes_step,
+            "graph_of_steps": steps, "note": "state (84 MB) can stay L2-resident between steps"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        rc = run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+
+    w = WORKLOAD
+    dev = torch.device("cuda", torch.cuda.current_device())
+    binding.load_library()
+    ins = inputs.scan_inputs(dataclasses.replace(w, seed=w.seed + rank), device=dev)
+    out, last, starts, ends, stream = time_device(w, ins, args.steps, args.warmup)
+
+    clocks = ClockSampler(local)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    g0 = torch.cuda.Event(enable_timing=True)
+    g1 = torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    ws = workspace_for(w, dev)
+    for i in range(args.steps):
+        starts[i].record(stream)
+        scan_call(ins, out, last, ws)
+        ends[i].record(stream)
+    g1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    total_ms = g0.elapsed_time(g1)
+    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(total_ms, world)
+    clk = clocks.summary(t_wall0, t_wall1) if rank == 0 else None
+    clocks.stop()
+
+    ms_step = total_ms / args.steps
+    elems = w.elements
+    value = world * elems * args.steps / (total_ms * 1e-3) / 1e9
+    peaks = load_peaks()
+    avg_launch_ms = sum(launch_ms) / len(launch_ms)
+    mufu_peak_gelem = MUFU_PER_CLK_PER_SM * SM_COUNT * peaks["sm_max_mhz"] * 1e6 / w.dstate / 1e9
+    achieved = elems / (avg_launch_ms * 1e-3) / 1e9
+    alg_bytes = algorithmic_bytes(w)
+    lanes, threads, sched = binding.mamba_scan_plan(w.batch, w.dim, w.seqlen, w.dstate, inputs.DTYPES[w.dtype])
+    if binding.workspace_status(ws) != 0:
+        raise SystemExit("persistent scan reported a timeout")
+    roof = {"bound": "alu", "achieved": achieved, "peak": mufu_peak_gelem, "unit": UNIT,
+            "frac": achieved / mufu_peak_gelem,
+            "traffic": measured_traffic("scan_fwd_kernel mamba-2.8b"),
+            "peak_source": f"MUFU ex2 16/clk/SM x {SM_COUNT} SMs x {peaks['sm_max_mhz']:.0f} MHz "
+                           f"({peaks['source']} sm_max_mhz) / N={w.dstate} exps per element",
+            "kernel": "scan_fwd_kernel", "avg_launch_us": avg_launch_ms * 1e3,
+            "hbm": {"algorithmic_bytes_per_launch": alg_bytes,
+                    "achieved_gbs": alg_bytes / (avg_launch_ms * 1e-3) / 1e9,
+                    "peak_gbs": peaks["hbm_gbs"],
+                    "frac": alg_bytes / (avg_launch_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
+    if clk and clk.get("sm_mhz"):
+        roof["frac_at_sampled_clock"] = achieved / (mufu_peak_gelem * clk["sm_mhz"] / peaks["sm_max_mhz"])
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "dim": w.dim, "seqlen": w.seqlen,
+                       "dstate": w.dstate, "act_dtype": w.dtype, "state_dtype": "f32",
+                       "gate": True, "softplus": True, "emit_last_state": True,
+                       "l2": "inputs larger than L2 (3 x 168 MB act tensors), no flush",
+                       "launch": {"schedule": {1: "static", 2: "persistent"}.get(sched, sched),
+                                  "lanes_per_channel": lanes, "threads_per_block": threads},
+                       "per_rank": "independent problem of this shape (seed + rank)"},
+            "gpu_launches": args.steps, "roofline": roof, "clocks": clk}
+
+    if rank == 0 and not args.no_e2e:
+        e2e_steps = max(3, min(args.steps, 10))
+        ms_e2e, h2d, d2h = e2e_measure(w, ins, e2e_steps)
+        line["e2e"] = {"value": elems / (ms_e2e * 1e-3) / 1e9, "unit": UNIT,
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": ms_e2e, "steps": e2e_steps,
+                       "path": "pinned host -> device copies, mamba_scan_fwd, device -> host out + last_state"}
+    if rank == 0 and not args.no_decode:
+        line["decode"] = decode_measure()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world)
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,214 @@
+/*
+ * mamba_scan.h -- C ABI of the B200 (sm_100a) selective-scan library.
+ *
+ * The library computes the selective state-space (S6) layer of Mamba:
+ *
+ *   delta_t = softplus(delta_raw_t + delta_bias[d])        (softplus optional)
+ *   Abar    = exp(delta_t * A[d, n])                       (zero-order hold of A)
+ *   h_t[n]  = Abar * h_{t-1}[n] + delta_t * B[b, n, t] * u_t
+ *   y_t     = sum_n C[b, n, t] * h_t[n] + D[d] * u_t
+ *   out_t   = y_t * silu(z_t)                              (gate optional)
+ *
+ * Sources: "Mamba SSM concept and implementation in Keras and TensorFlow"
+ * (sections on the continuous SSM, its zero-order-hold discretisation and the
+ * recurrent form, the selective_scan listing with dA = delta*A,
+ * dB_u = delta*u*B and y + u*D, and MambaBlock.call, y * swish(res));
+ * "Mamba: Linear-Time Sequence Modeling with Selective State Spaces",
+ * Appendix E.5 (the scan fuses discretisation with the recurrence and does not
+ * write the expanded (batch, L, dim, N) parameters to HBM); the state-spaces
+ * mamba README (the selective-scan interface and the Mamba(d_model,
+ * d_state=16, d_conv=4, expand=2) block that wraps it).
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - Pointers are DEVICE pointers (cudaMalloc'd, managed, or mapped pinned host
+ *   memory) of the current CUDA device, except where stated.  Tensors are
+ *   dense, row-major and contiguous with the layouts given per function.
+ * - "act" tensors (u, delta, z, B, C, out) share one element type chosen by
+ *   `act_dtype` (MAMBA_F32 or MAMBA_BF16).  A, D, delta_bias, states are
+ *   always fp32.  All arithmetic is fp32.
+ * - The caller owns every buffer.  The library never allocates or frees, and
+ *   only mamba_scan_workspace_status synchronises: work is enqueued on
+ *   `stream` (0 = legacy default stream) and buffers must stay alive until
+ *   that work completes.
+ * - Argument validation is synchronous and happens before anything is
+ *   enqueued; a non-zero return means nothing was enqueued, except
+ *   MAMBA_ERR_CUDA, which reports a launch failure (cudaGetLastError).
+ * - Alignment never fails: 16-byte-aligned act pointers with seqlen a multiple
+ *   of the 16-byte vector width take the vectorised path, others a scalar path.
+ * - `out` may alias exactly one of u, delta or z (same pointer, in-place);
+ *   any other overlap between an output and an input is rejected.
+ * - The library holds no state; calls are reentrant and thread-safe.
+ */
+#ifndef MAMBA_SCAN_H
+#define MAMBA_SCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#ifndef __CUDA_RUNTIME_H__
+typedef struct CUstream_st *cudaStream_t; /* identical to the CUDA runtime's typedef */
+#endif
+
+typedef enum {
+    MAMBA_F32 = 0,  /* IEEE binary32 */
+    MAMBA_BF16 = 1  /* bfloat16; stores round to nearest even */
+} mamba_dtype_t;
+
+typedef enum {
+    MAMBA_OK = 0,
+    MAMBA_ERR_NULL = -1,        /* a required pointer is NULL */
+    MAMBA_ERR_SHAPE = -2,       /* a size is <= 0 or too large to index */
+    MAMBA_ERR_UNSUPPORTED = -3, /* dstate outside [1, 64], unknown dtype, bad tuning */
+    MAMBA_ERR_ALIGN = -4,       /* reserved (alignment selects a path, never fails) */
+    MAMBA_ERR_CUDA = -5,        /* the CUDA runtime reported an error at launch */
+    MAMBA_ERR_DEVICE = -6,      /* no usable CUDA device */
+    MAMBA_ERR_OVERLAP = -7,     /* an output partially overlaps an input */
+    MAMBA_ERR_WORKSPACE = -8,   /* workspace too small or misaligned */
+    MAMBA_ERR_TIMEOUT = -9      /* a persistent launch gave up waiting (see
+                                   mamba_scan_workspace_status) */
+} mamba_status_t;
+
+/* Launch schedules of the scan. */
+typedef enum {
+    MAMBA_SCHEDULE_AUTO = 0,
+    MAMBA_SCHEDULE_STATIC = 1,     /* one block per channel group walks the whole
+                                      sequence; no workspace */
+    MAMBA_SCHEDULE_PERSISTENT = 2  /* one thread per channel and all its states
+                                      (dstate <= 16); persistent workers take
+                                      (32-channel group, time chunk) units from a
+                                      ready queue and pass the state between
+                                      chunks through the workspace */
+} mamba_schedule_t;
+
+/* Optional launch tuning.  Zero fields mean "choose automatically".
+ *   lanes_per_channel : static schedule only: threads sharing one channel's
+ *                       states (1, 2, 4, 8 or 16; the padded dstate must be a
+ *                       multiple, and at most 16 states stay in one thread)
+ *   threads_per_block : static schedule only: 128 or 256
+ *   schedule          : a mamba_schedule_t
+ */
+typedef struct {
+    int lanes_per_channel;
+    int threads_per_block;
+    int schedule;
+} mamba_scan_tuning_t;
+
+/*
+ * mamba_scan_fwd -- fused selective scan forward over a whole sequence.
+ *
+ * Defining passage: the recurrent form of the discretised SSM and the
+ * selective_scan listing of "Mamba SSM concept and implementation in Keras
+ * and TensorFlow"; the fused, HBM-avoiding scan of Appendix E.5 of the Mamba
+ * paper.
+ *
+ *   u, delta, z  : act (batch, dim, seqlen).  delta is the raw step before the
+ *                  bias and softplus.  z may be NULL (no gate).
+ *   A            : fp32 (dim, dstate); the (usually negative) real diagonal A.
+ *   B, C         : act (batch, dstate, seqlen); shared by every channel of a
+ *                  batch row.
+ *   D            : fp32 (dim) or NULL (no skip term).
+ *   delta_bias   : fp32 (dim) or NULL (zero bias).
+ *   delta_softplus: non-zero applies softplus to delta_raw + delta_bias.
+ *   out          : act (batch, dim, seqlen), written.
+ *   last_state   : fp32 (batch, dim, dstate) or NULL; receives h_{seqlen-1}.
+ *   The state starts from zero.
+ *
+ * Returns MAMBA_OK or a mamba_status_t error.
+ */
+int mamba_scan_fwd(const void *u, const void *delta, const float *A,
+                   const void *B, const void *C, const float *D,
+                   const void *z, const float *delta_bias, int delta_softplus,
+                   void *out, float *last_state, int64_t batch, int64_t dim,
+                   int64_t seqlen, int64_t dstate, int act_dtype,
+                   cudaStream_t stream);
+
+/* mamba_scan_fwd with an explicit launch configuration (same results up to
+ * fp32 rounding order; NULL tuning is identical to mamba_scan_fwd).  Invalid
+ * tuning returns MAMBA_ERR_UNSUPPORTED. */
+int mamba_scan_fwd_tuned(const void *u, const void *delta, const float *A,
+                         const void *B, const void *C, const float *D,
+                         const void *z, const float *delta_bias,
+                         int delta_softplus, void *out, float *last_state,
+                         int64_t batch, int64_t dim, int64_t seqlen,
+                         int64_t dstate, int act_dtype,
+                         const mamba_scan_tuning_t *tuning,
+                         cudaStream_t stream);
+
+/* The launch configuration mamba_scan_fwd_ws would pick for these sizes on
+ * the current device, given a large enough workspace and 16-byte-aligned
+ * tensors (fields filled in `plan`), without launching anything.
+ * Returns MAMBA_OK or a validation error. */
+int mamba_scan_plan(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                    int act_dtype, mamba_scan_tuning_t *plan);
+
+/* Bytes of device workspace mamba_scan_fwd_ws may use for these sizes (an
+ * upper bound valid on every device); 0 when the persistent schedule never
+ * applies (dstate > 16).  Pure host arithmetic. */
+size_t mamba_scan_workspace_size(int64_t batch, int64_t dim, int64_t seqlen,
+                                 int64_t dstate, int act_dtype);
+
+/*
+ * mamba_scan_fwd_ws -- mamba_scan_fwd plus a caller-owned device workspace
+ * (at least mamba_scan_workspace_size bytes, 16-byte aligned) that enables
+ * the persistent, load-balanced schedule.  Same arguments and results as
+ * mamba_scan_fwd.  The workspace holds the work queue and the states carried
+ * between time chunks; its queue part is zeroed on `stream` before the
+ * launch, so one workspace must not be used by two launches that can run at
+ * the same time.  When the persistent schedule does not apply (dstate > 16,
+ * unaligned tensors, too few channel groups to fill the GPU) the static
+ * schedule runs and the workspace is not touched.  `tuning` may be NULL.
+ */
+int mamba_scan_fwd_ws(const void *u, const void *delta, const float *A,
+                      const void *B, const void *C, const float *D,
+                      const void *z, const float *delta_bias,
+                      int delta_softplus, void *out, float *last_state,
+                      int64_t batch, int64_t dim, int64_t seqlen,
+                      int64_t dstate, int act_dtype,
+                      const mamba_scan_tuning_t *tuning, void *workspace,
+                      size_t workspace_bytes, cudaStream_t stream);
+
+/* Synchronises `stream`, then reads the status a persistent launch left in
+ * `workspace`: MAMBA_OK, or MAMBA_ERR_TIMEOUT if a worker stopped waiting for
+ * a predecessor chunk (the outputs of that launch are then incomplete).
+ * This is the only entry point that synchronises. */
+int mamba_scan_workspace_status(const void *workspace, cudaStream_t stream);
+
+/*
+ * mamba_state_update -- one recurrent step (one token) for every channel,
+ * with the state held in HBM and updated in place: the decoding form used by
+ * generation, one token per call (mamba-jax sample.py; the generation
+ * benchmark of the state-spaces README).
+ *
+ *   state        : fp32 (batch, dim, dstate), read and overwritten.
+ *   u, delta, z  : act (batch, dim); z may be NULL.
+ *   A            : fp32 (dim, dstate).
+ *   B, C         : act (batch, dstate).
+ *   D, delta_bias: fp32 (dim) or NULL.
+ *   out          : act (batch, dim), written.
+ *
+ * One call equals one iteration of mamba_scan_fwd's time loop.
+ * Returns MAMBA_OK or a mamba_status_t error.
+ */
+int mamba_state_update(float *state, const void *u, const void *delta,
+                       const float *A, const void *B, const void *C,
+                       const float *D, const void *z, const float *delta_bias,
+                       int delta_softplus, void *out, int64_t batch,
+                       int64_t dim, int64_t dstate, int act_dtype,
+                       cudaStream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char *mamba_status_string(int status);
+
+/* Library ABI version, (major << 16) | minor. */
+int mamba_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBA_SCAN_H */

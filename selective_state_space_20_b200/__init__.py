@@ -8,7 +8,7 @@ there is no fallback path.
 """
 from __future__ import annotations
 
-__all__ = ["mamba_scan_fwd", "mamba_state_update", "load_library"]
+__all__ = ["mamba_scan_fwd", "mamba_state_update", "mamba_scan_plan", "load_library"]
 
 
 def __getattr__(name):

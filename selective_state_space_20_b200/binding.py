@@ -1,0 +1,250 @@
+"""ctypes binding of ``libmamba_scan.so`` (C ABI: ``include/mamba_scan.h``).
+
+Argument marshalling only: shapes and dtypes are checked, outputs are
+allocated with torch when the caller does not pass them, and raw device
+pointers plus the current CUDA stream are handed to the library.  Every step
+of the computation runs in the library's CUDA kernels; there is no host or
+PyTorch fallback, and a missing library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+from . import build as _build
+
+MAMBA_F32, MAMBA_BF16 = 0, 1
+_ACT = {torch.float32: MAMBA_F32, torch.bfloat16: MAMBA_BF16}
+
+MAMBA_OK = 0
+STATUS_NAMES = {0: "MAMBA_OK", -1: "MAMBA_ERR_NULL", -2: "MAMBA_ERR_SHAPE",
+                -3: "MAMBA_ERR_UNSUPPORTED", -4: "MAMBA_ERR_ALIGN",
+                -5: "MAMBA_ERR_CUDA", -6: "MAMBA_ERR_DEVICE", -7: "MAMBA_ERR_OVERLAP",
+                -8: "MAMBA_ERR_WORKSPACE", -9: "MAMBA_ERR_TIMEOUT"}
+SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT = 0, 1, 2
+
+# Every function include/mamba_scan.h declares.
+EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
+            "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
+            "mamba_state_update", "mamba_status_string", "mamba_abi_version")
+
+
+class MambaError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(code, code)} ({msg})")
+        self.code = code
+
+
+class Tuning(ctypes.Structure):
+    _fields_ = [("lanes_per_channel", ctypes.c_int), ("threads_per_block", ctypes.c_int),
+                ("schedule", ctypes.c_int)]
+
+
+_lock = threading.Lock()
+_lib: Optional[ctypes.CDLL] = None
+
+
+def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
+    vp, fp, i64, ci = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    scan_args = [vp, vp, fp, vp, vp, fp, vp, fp, ci, vp, fp, i64, i64, i64, i64, ci]
+    lib.mamba_scan_fwd.argtypes = scan_args + [vp]
+    lib.mamba_scan_fwd.restype = ci
+    lib.mamba_scan_fwd_tuned.argtypes = scan_args + [ctypes.POINTER(Tuning), vp]
+    lib.mamba_scan_fwd_tuned.restype = ci
+    lib.mamba_scan_fwd_ws.argtypes = scan_args + [ctypes.POINTER(Tuning), vp, ctypes.c_size_t, vp]
+    lib.mamba_scan_fwd_ws.restype = ci
+    lib.mamba_scan_plan.argtypes = [i64, i64, i64, i64, ci, ctypes.POINTER(Tuning)]
+    lib.mamba_scan_plan.restype = ci
+    lib.mamba_scan_workspace_size.argtypes = [i64, i64, i64, i64, ci]
+    lib.mamba_scan_workspace_size.restype = ctypes.c_size_t
+    lib.mamba_scan_workspace_status.argtypes = [vp, vp]
+    lib.mamba_scan_workspace_status.restype = ci
+    lib.mamba_state_update.argtypes = [fp, vp, vp, fp, vp, vp, fp, vp, fp, ci, vp,
+                                       i64, i64, i64, ci, vp]
+    lib.mamba_state_update.restype = ci
+    lib.mamba_status_string.argtypes = [ci]
+    lib.mamba_status_string.restype = ctypes.c_char_p
+    lib.mamba_abi_version.argtypes = []
+    lib.mamba_abi_version.restype = ci
+    return lib
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load the CUDA library, building it with nvcc first if it is missing or
+    older than its sources.  Raises if it cannot be built or loaded."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or _build.LIB
+        if path is None and not _build.up_to_date():
+            _build.build()
+        if not os.path.exists(p):
+            raise RuntimeError(f"CUDA library {p} is missing and could not be built")
+        lib = _declare(ctypes.CDLL(p))
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().mamba_status_string(code).decode()
+
+
+def _check(fn: str, code: int):
+    if code != MAMBA_OK:
+        raise MambaError(fn, code, status_string(code))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: Optional[torch.Tensor], name: str, device, dtype, shape):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def mamba_scan_fwd(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
+                   B: torch.Tensor, C: torch.Tensor, D: Optional[torch.Tensor] = None,
+                   z: Optional[torch.Tensor] = None,
+                   delta_bias: Optional[torch.Tensor] = None,
+                   delta_softplus: bool = True, out: Optional[torch.Tensor] = None,
+                   last_state: Optional[torch.Tensor] = None,
+                   return_last_state: bool = False, lanes_per_channel: int = 0,
+                   threads_per_block: int = 0, schedule: int = SCHEDULE_AUTO,
+                   workspace: Optional[torch.Tensor] = None):
+    """Selective scan forward on the current CUDA stream.
+
+    u, delta, z: (batch, dim, L); B, C: (batch, N, L) -- all one dtype,
+    float32 or bfloat16.  A: (dim, N) fp32; D, delta_bias: (dim,) fp32.
+    Returns ``out`` (batch, dim, L), or ``(out, last_state)`` when
+    ``return_last_state`` is set or ``last_state`` is passed.
+
+    A device workspace (``mamba_scan_workspace_size`` bytes, allocated here
+    with torch unless given) enables the persistent, load-balanced schedule;
+    ``schedule`` / ``lanes_per_channel`` / ``threads_per_block`` force a
+    launch configuration (0 = automatic).
+    """
+    if u.dim() != 3:
+        raise ValueError("u must be (batch, dim, seqlen)")
+    batch, dim, L = u.shape
+    if A.dim() != 2:
+        raise ValueError("A must be (dim, dstate)")
+    N = A.shape[1]
+    dev, act = u.device, u.dtype
+    if dev.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    if act not in _ACT:
+        raise TypeError(f"unsupported activation dtype {act}")
+    _need(u, "u", dev, act, (batch, dim, L))
+    _need(delta, "delta", dev, act, (batch, dim, L))
+    _need(z, "z", dev, act, (batch, dim, L))
+    _need(B, "B", dev, act, (batch, N, L))
+    _need(C, "C", dev, act, (batch, N, L))
+    _need(A, "A", dev, torch.float32, (dim, N))
+    _need(D, "D", dev, torch.float32, (dim,))
+    _need(delta_bias, "delta_bias", dev, torch.float32, (dim,))
+    if out is None:
+        out = torch.empty_like(u)
+    _need(out, "out", dev, act, (batch, dim, L))
+    want_state = return_last_state or last_state is not None
+    if want_state and last_state is None:
+        last_state = torch.empty((batch, dim, N), device=dev, dtype=torch.float32)
+    _need(last_state, "last_state", dev, torch.float32, (batch, dim, N))
+    lib = load_library()
+    if workspace is None and schedule != SCHEDULE_STATIC:
+        nbytes = lib.mamba_scan_workspace_size(batch, dim, L, N, _ACT[act])
+        if nbytes:
+            workspace = torch.empty(nbytes, device=dev, dtype=torch.uint8)
+    if workspace is not None and (workspace.device != dev or not workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous tensor on the input device")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    args = [_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+            _ptr(delta_bias), int(bool(delta_softplus)), _ptr(out), _ptr(last_state),
+            batch, dim, L, N, _ACT[act]]
+    tun = Tuning(int(lanes_per_channel), int(threads_per_block), int(schedule))
+    with torch.cuda.device(dev):
+        rc = lib.mamba_scan_fwd_ws(*args, ctypes.byref(tun), _ptr(workspace), ws_bytes,
+                                   _stream(dev))
+    _check("mamba_scan_fwd_ws", rc)
+    return (out, last_state) if want_state else out
+
+
+def workspace_status(workspace: torch.Tensor) -> int:
+    """Synchronise the current stream and return the status word a persistent
+    launch left in ``workspace`` (0 = ok, MAMBA_ERR_TIMEOUT otherwise)."""
+    with torch.cuda.device(workspace.device):
+        return load_library().mamba_scan_workspace_status(_ptr(workspace), _stream(workspace.device))
+
+
+def mamba_scan_workspace_size(batch: int, dim: int, seqlen: int, dstate: int,
+                              dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(load_library().mamba_scan_workspace_size(batch, dim, seqlen, dstate, _ACT[dtype]))
+
+
+def mamba_scan_plan(batch: int, dim: int, seqlen: int, dstate: int,
+                    dtype: torch.dtype = torch.bfloat16) -> Tuple[int, int, int]:
+    """(lanes_per_channel, threads_per_block, schedule) the library picks for a
+    shape on the current device (given a workspace and aligned tensors)."""
+    t = Tuning()
+    _check("mamba_scan_plan", load_library().mamba_scan_plan(batch, dim, seqlen, dstate,
+                                                            _ACT[dtype], ctypes.byref(t)))
+    return t.lanes_per_channel, t.threads_per_block, t.schedule
+
+
+def mamba_state_update(state: torch.Tensor, u: torch.Tensor, delta: torch.Tensor,
+                       A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+                       D: Optional[torch.Tensor] = None, z: Optional[torch.Tensor] = None,
+                       delta_bias: Optional[torch.Tensor] = None,
+                       delta_softplus: bool = True,
+                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One recurrent step, updating ``state`` (batch, dim, N) fp32 in place.
+
+    u, delta, z: (batch, dim); B, C: (batch, N) in one dtype.  Returns out
+    (batch, dim)."""
+    if state.dim() != 3:
+        raise ValueError("state must be (batch, dim, dstate)")
+    batch, dim, N = state.shape
+    dev, act = u.device, u.dtype
+    if dev.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    if act not in _ACT:
+        raise TypeError(f"unsupported activation dtype {act}")
+    _need(state, "state", dev, torch.float32, (batch, dim, N))
+    for name, t in (("u", u), ("delta", delta), ("z", z)):
+        _need(t, name, dev, act, (batch, dim))
+    _need(B, "B", dev, act, (batch, N))
+    _need(C, "C", dev, act, (batch, N))
+    _need(A, "A", dev, torch.float32, (dim, N))
+    _need(D, "D", dev, torch.float32, (dim,))
+    _need(delta_bias, "delta_bias", dev, torch.float32, (dim,))
+    if out is None:
+        out = torch.empty_like(u)
+    _need(out, "out", dev, act, (batch, dim))
+    lib = load_library()
+    with torch.cuda.device(dev):
+        rc = lib.mamba_state_update(_ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B),
+                                    _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+                                    int(bool(delta_softplus)), _ptr(out), batch, dim, N,
+                                    _ACT[act], _stream(dev))
+    _check("mamba_state_update", rc)
+    return out

@@ -1,0 +1,263 @@
+// api.cu -- the C ABI declared in include/mamba_scan.h: argument validation,
+// launch planning and dispatch.  No computation happens here and nothing is
+// allocated; only mamba_scan_workspace_status synchronises.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mamba_scan.h"
+#include "internal.h"
+
+namespace {
+
+constexpr int kMaxDstate = 64;
+constexpr int kMaxDevices = 64;
+
+int g_sm_count[kMaxDevices];  // 0 = not queried yet (benign races: same value)
+
+int current_sm_count(int *status) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { *status = MAMBA_ERR_DEVICE; return 0; }
+    if (dev >= 0 && dev < kMaxDevices && g_sm_count[dev] > 0) return g_sm_count[dev];
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+        *status = MAMBA_ERR_DEVICE;
+        return 0;
+    }
+    if (dev >= 0 && dev < kMaxDevices) g_sm_count[dev] = sms;
+    return sms;
+}
+
+size_t act_size(int act) { return act == MAMBA_BF16 ? 2 : 4; }
+
+bool overlaps(const void *a, size_t abytes, const void *b, size_t bbytes) {
+    if (!a || !b) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + bbytes && b0 < a0 + abytes;
+}
+
+// An output may coincide exactly with one same-shaped input (in place) but
+// must not otherwise overlap any input.
+bool bad_alias(const void *out, size_t obytes, const void *in, size_t ibytes, bool exact_ok) {
+    if (!overlaps(out, obytes, in, ibytes)) return false;
+    return !(exact_ok && out == in && obytes == ibytes);
+}
+
+// Largest element count a launch may index with int64 arithmetic.
+constexpr int64_t kMaxElems = (int64_t)1 << 50;
+
+int check_sizes(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate) {
+    if (batch <= 0 || dim <= 0 || seqlen <= 0 || dstate <= 0) return MAMBA_ERR_SHAPE;
+    if (dstate > kMaxDstate) return MAMBA_ERR_UNSUPPORTED;
+    if (batch > kMaxElems || dim > kMaxElems || seqlen > kMaxElems) return MAMBA_ERR_SHAPE;
+    if ((double)batch * (double)dim * (double)seqlen > (double)kMaxElems) return MAMBA_ERR_SHAPE;
+    if ((double)batch * (double)dstate * (double)seqlen > (double)kMaxElems) return MAMBA_ERR_SHAPE;
+    return MAMBA_OK;
+}
+
+int scan_impl(const void *u, const void *delta, const float *A, const void *B, const void *C,
+              const float *D, const void *z, const float *delta_bias, int delta_softplus,
+              void *out, float *last_state, int64_t batch, int64_t dim, int64_t seqlen,
+              int64_t dstate, int act_dtype, const mamba_scan_tuning_t *tuning,
+              void *workspace, size_t ws_bytes, cudaStream_t stream, bool launch,
+              mamba_scan_tuning_t *plan_out) {
+    if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
+    int rc = check_sizes(batch, dim, seqlen, dstate);
+    if (rc != MAMBA_OK) return rc;
+    if (launch) {
+        if (!u || !delta || !A || !B || !C || !out) return MAMBA_ERR_NULL;
+        const size_t es = act_size(act_dtype);
+        const size_t nx = (size_t)(batch * dim * seqlen) * es;
+        const size_t nbc = (size_t)(batch * dstate * seqlen) * es;
+        const size_t nA = (size_t)(dim * dstate) * 4, nd = (size_t)dim * 4;
+        const size_t nls = (size_t)(batch * dim * dstate) * 4;
+        // out may replace u, delta or z in place; nothing else may overlap.
+        if (bad_alias(out, nx, u, nx, true) || bad_alias(out, nx, delta, nx, true) ||
+            bad_alias(out, nx, z, nx, true) || bad_alias(out, nx, B, nbc, false) ||
+            bad_alias(out, nx, C, nbc, false) || bad_alias(out, nx, A, nA, false) ||
+            bad_alias(out, nx, D, nd, false) || bad_alias(out, nx, delta_bias, nd, false))
+            return MAMBA_ERR_OVERLAP;
+        if (last_state &&
+            (overlaps(last_state, nls, u, nx) || overlaps(last_state, nls, delta, nx) ||
+             overlaps(last_state, nls, z, nx) || overlaps(last_state, nls, B, nbc) ||
+             overlaps(last_state, nls, C, nbc) || overlaps(last_state, nls, A, nA) ||
+             overlaps(last_state, nls, D, nd) || overlaps(last_state, nls, delta_bias, nd) ||
+             overlaps(last_state, nls, out, nx)))
+            return MAMBA_ERR_OVERLAP;
+        if (workspace) {
+            if ((reinterpret_cast<uintptr_t>(workspace) & 15) != 0) return MAMBA_ERR_WORKSPACE;
+            const void *ins[] = {u, delta, z, B, C, A, D, delta_bias, out, last_state};
+            const size_t sz[] = {nx, nx, nx, nbc, nbc, nA, nd, nd, nx, nls};
+            for (int i = 0; i < 10; ++i)
+                if (overlaps(workspace, ws_bytes, ins[i], sz[i])) return MAMBA_ERR_OVERLAP;
+        }
+    }
+    int want_lanes = 0, want_threads = 0, want_sched = MAMBA_SCHEDULE_AUTO;
+    if (tuning) {
+        want_lanes = tuning->lanes_per_channel;
+        want_threads = tuning->threads_per_block;
+        want_sched = tuning->schedule;
+        if (want_lanes != 0 && want_lanes != 1 && want_lanes != 2 && want_lanes != 4 &&
+            want_lanes != 8 && want_lanes != 16)
+            return MAMBA_ERR_UNSUPPORTED;
+        if (want_threads != 0 && want_threads != 128 && want_threads != 256)
+            return MAMBA_ERR_UNSUPPORTED;
+        if (want_sched < MAMBA_SCHEDULE_AUTO || want_sched > MAMBA_SCHEDULE_PERSISTENT)
+            return MAMBA_ERR_UNSUPPORTED;
+    }
+    int status = MAMBA_OK;
+    const int sms = current_sm_count(&status);
+    if (status != MAMBA_OK) return status;
+
+    mscan::ScanArgs a;
+    a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.D = D; a.delta_bias = delta_bias; a.out = out; a.last_state = last_state;
+    a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = (int)dstate;
+    a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
+
+    // Persistent schedule: needs a workspace (when launching), dstate <= 16,
+    // aligned tensors and enough channel groups to occupy every worker.
+    const bool ws_ok = !launch || (workspace != nullptr &&
+                                   ws_bytes >= mscan::persistent_workspace_bound(
+                                                   batch, dim, seqlen, act_dtype));
+    const bool supported = mscan::persistent_supported(a);
+    bool persist = false;
+    if (want_sched == MAMBA_SCHEDULE_PERSISTENT) {
+        if (!supported) return MAMBA_ERR_UNSUPPORTED;
+        if (!ws_ok) return MAMBA_ERR_WORKSPACE;
+        persist = true;
+    } else if (want_sched == MAMBA_SCHEDULE_AUTO) {
+        persist = supported && ws_ok && mscan::persistent_preferred(a, sms) &&
+                  want_lanes == 0 && want_threads == 0;
+    }
+    if (persist) {
+        if (plan_out) {
+            plan_out->lanes_per_channel = 1;
+            plan_out->threads_per_block = 128;
+            plan_out->schedule = MAMBA_SCHEDULE_PERSISTENT;
+        }
+        if (!launch) return MAMBA_OK;
+        return mscan::launch_scan_fwd_persistent(a, workspace, ws_bytes, sms, stream) == cudaSuccess
+                   ? MAMBA_OK : MAMBA_ERR_CUDA;
+    }
+    mscan::ScanPlan pl;
+    if (mscan::make_scan_plan(a, want_lanes, want_threads, sms, &pl) != 0) return MAMBA_ERR_UNSUPPORTED;
+    if (plan_out) {
+        plan_out->lanes_per_channel = pl.lanes;
+        plan_out->threads_per_block = pl.threads;
+        plan_out->schedule = MAMBA_SCHEDULE_STATIC;
+    }
+    if (!launch) return MAMBA_OK;
+    return mscan::launch_scan_fwd(a, pl, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
+                   const void *C, const float *D, const void *z, const float *delta_bias,
+                   int delta_softplus, void *out, float *last_state, int64_t batch,
+                   int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
+                   cudaStream_t stream) {
+    return scan_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, last_state,
+                     batch, dim, seqlen, dstate, act_dtype, nullptr, nullptr, 0, stream, true,
+                     nullptr);
+}
+
+int mamba_scan_fwd_tuned(const void *u, const void *delta, const float *A, const void *B,
+                         const void *C, const float *D, const void *z,
+                         const float *delta_bias, int delta_softplus, void *out,
+                         float *last_state, int64_t batch, int64_t dim, int64_t seqlen,
+                         int64_t dstate, int act_dtype, const mamba_scan_tuning_t *tuning,
+                         cudaStream_t stream) {
+    return scan_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, last_state,
+                     batch, dim, seqlen, dstate, act_dtype, tuning, nullptr, 0, stream, true,
+                     nullptr);
+}
+
+int mamba_scan_fwd_ws(const void *u, const void *delta, const float *A, const void *B,
+                      const void *C, const float *D, const void *z, const float *delta_bias,
+                      int delta_softplus, void *out, float *last_state, int64_t batch,
+                      int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
+                      const mamba_scan_tuning_t *tuning, void *workspace,
+                      size_t workspace_bytes, cudaStream_t stream) {
+    return scan_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, last_state,
+                     batch, dim, seqlen, dstate, act_dtype, tuning, workspace, workspace_bytes,
+                     stream, true, nullptr);
+}
+
+size_t mamba_scan_workspace_size(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                                 int act_dtype) {
+    if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return 0;
+    if (check_sizes(batch, dim, seqlen, dstate) != MAMBA_OK || dstate > 16) return 0;
+    return mscan::persistent_workspace_bound(batch, dim, seqlen, act_dtype);
+}
+
+int mamba_scan_workspace_status(const void *workspace, cudaStream_t stream) {
+    if (!workspace) return MAMBA_ERR_NULL;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MAMBA_ERR_CUDA;
+    unsigned hdr[4] = {0, 0, 0, 0};
+    if (cudaMemcpy(hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MAMBA_ERR_CUDA;
+    return hdr[2] != 0 ? MAMBA_ERR_TIMEOUT : MAMBA_OK;
+}
+
+int mamba_scan_plan(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
+                    mamba_scan_tuning_t *plan) {
+    if (!plan) return MAMBA_ERR_NULL;
+    return scan_impl(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 1,
+                     nullptr, nullptr, batch, dim, seqlen, dstate, act_dtype, nullptr, nullptr, 0,
+                     nullptr, false, plan);
+}
+
+int mamba_state_update(float *state, const void *u, const void *delta, const float *A,
+                       const void *B, const void *C, const float *D, const void *z,
+                       const float *delta_bias, int delta_softplus, void *out, int64_t batch,
+                       int64_t dim, int64_t dstate, int act_dtype, cudaStream_t stream) {
+    if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
+    int rc = check_sizes(batch, dim, 1, dstate);
+    if (rc != MAMBA_OK) return rc;
+    if (!state || !u || !delta || !A || !B || !C || !out) return MAMBA_ERR_NULL;
+    const size_t es = act_size(act_dtype);
+    const size_t nx = (size_t)(batch * dim) * es, nbc = (size_t)(batch * dstate) * es;
+    const size_t ns = (size_t)(batch * dim * dstate) * 4, nA = (size_t)(dim * dstate) * 4;
+    const size_t nd = (size_t)dim * 4;
+    if (bad_alias(out, nx, u, nx, true) || bad_alias(out, nx, delta, nx, true) ||
+        bad_alias(out, nx, z, nx, true) || bad_alias(out, nx, B, nbc, false) ||
+        bad_alias(out, nx, C, nbc, false) || bad_alias(out, nx, A, nA, false) ||
+        bad_alias(out, nx, D, nd, false) || bad_alias(out, nx, delta_bias, nd, false) ||
+        overlaps(out, nx, state, ns))
+        return MAMBA_ERR_OVERLAP;
+    if (overlaps(state, ns, u, nx) || overlaps(state, ns, delta, nx) || overlaps(state, ns, z, nx) ||
+        overlaps(state, ns, B, nbc) || overlaps(state, ns, C, nbc) || overlaps(state, ns, A, nA) ||
+        overlaps(state, ns, D, nd) || overlaps(state, ns, delta_bias, nd))
+        return MAMBA_ERR_OVERLAP;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MAMBA_ERR_DEVICE;
+    mscan::StateUpdateArgs a;
+    a.state = state; a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.D = D; a.delta_bias = delta_bias; a.out = out;
+    a.batch = batch; a.dim = dim; a.dstate = (int)dstate;
+    a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
+    return mscan::launch_state_update(a, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
+const char *mamba_status_string(int status) {
+    switch (status) {
+        case MAMBA_OK: return "ok";
+        case MAMBA_ERR_NULL: return "a required pointer is NULL";
+        case MAMBA_ERR_SHAPE: return "a size is non-positive or too large";
+        case MAMBA_ERR_UNSUPPORTED: return "unsupported dstate, dtype or tuning";
+        case MAMBA_ERR_ALIGN: return "misaligned pointer";
+        case MAMBA_ERR_CUDA: return "CUDA runtime error at launch";
+        case MAMBA_ERR_DEVICE: return "no usable CUDA device";
+        case MAMBA_ERR_OVERLAP: return "an output overlaps an input or the workspace";
+        case MAMBA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+        case MAMBA_ERR_TIMEOUT: return "a persistent launch stopped waiting for a predecessor chunk";
+        default: return "unknown status";
+    }
+}
+
+int mamba_abi_version(void) { return (1 << 16) | 0; }
+
+}  // extern "C"

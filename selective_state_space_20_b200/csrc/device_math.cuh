@@ -1,0 +1,94 @@
+// device_math.cuh -- small device helpers for the scan kernels: element
+// conversion, 16-byte vectors, and the pointwise functions of the layer.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace mscan {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32).
+__device__ __forceinline__ float ex2_mufu(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// softplus(x) = ln(1 + e^x).  Above 20 the correction ln(1 + e^-x) < 2.1e-9
+// is below fp32 resolution of x, so x itself is returned.
+__device__ __forceinline__ float softplus_f(float x) {
+    return x > 20.f ? x : log1pf(__expf(x));
+}
+
+// silu(z) = z / (1 + e^-z); for z < -88 the denominator overflows and the
+// quotient is 0, which is the correctly rounded fp32 limit.
+__device__ __forceinline__ float silu_f(float z) {
+    return __fdividef(z, 1.f + __expf(-z));
+}
+
+// ---------------------------------------------------------------- elements
+template <typename T> struct Elem;
+
+template <> struct Elem<float> {
+    static constexpr int kVec = 4;  // elements per 16 bytes
+    __device__ __forceinline__ static float load(const float *p) { return __ldg(p); }
+    __device__ __forceinline__ static void store(float *p, float v) { *p = v; }
+    __device__ __forceinline__ static void unpack(const uint4 &w, float *f) {
+        f[0] = __uint_as_float(w.x); f[1] = __uint_as_float(w.y);
+        f[2] = __uint_as_float(w.z); f[3] = __uint_as_float(w.w);
+    }
+    __device__ __forceinline__ static uint4 pack(const float *f) {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]),
+                          __float_as_uint(f[2]), __float_as_uint(f[3]));
+    }
+};
+
+template <> struct Elem<__nv_bfloat16> {
+    static constexpr int kVec = 8;
+    __device__ __forceinline__ static float load(const __nv_bfloat16 *p) {
+        unsigned short s = __ldg(reinterpret_cast<const unsigned short *>(p));
+        return __uint_as_float(static_cast<uint32_t>(s) << 16);
+    }
+    __device__ __forceinline__ static void store(__nv_bfloat16 *p, float v) {
+        *p = __float2bfloat16_rn(v);
+    }
+    // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 bits.
+    __device__ __forceinline__ static void unpack2(uint32_t w, float &lo, float &hi) {
+        lo = __uint_as_float(w << 16);
+        hi = __uint_as_float(w & 0xffff0000u);
+    }
+    __device__ __forceinline__ static void unpack(const uint4 &w, float *f) {
+        unpack2(w.x, f[0], f[1]); unpack2(w.y, f[2], f[3]);
+        unpack2(w.z, f[4], f[5]); unpack2(w.w, f[6], f[7]);
+    }
+    __device__ __forceinline__ static uint32_t pack2(float lo, float hi) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // round to nearest even
+        return *reinterpret_cast<uint32_t *>(&v);
+    }
+    __device__ __forceinline__ static uint4 pack(const float *f) {
+        return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]),
+                          pack2(f[4], f[5]), pack2(f[6], f[7]));
+    }
+};
+
+__device__ __forceinline__ uint4 ldg16(const void *p) {
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+// Streaming 16-byte load: read once, do not keep in L1.
+__device__ __forceinline__ uint4 ldg16_stream(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+// Streaming 16-byte store (evict-first in L2: the output is not re-read).
+__device__ __forceinline__ void stg16_stream(void *p, const uint4 &v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};"
+                 :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+}  // namespace mscan

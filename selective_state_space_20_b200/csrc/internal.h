@@ -1,0 +1,62 @@
+// internal.h -- declarations shared by the C-ABI layer and the kernel files.
+// Not part of the public interface (that is include/mamba_scan.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mscan {
+
+enum ActType : int { kF32 = 0, kBF16 = 1 };
+
+struct ScanArgs {
+    const void *u, *delta, *B, *C, *z;
+    const float *A, *D, *delta_bias;
+    void *out;
+    float *last_state;
+    int64_t batch, dim, seqlen;
+    int dstate;
+    int softplus;
+    int act;  // ActType
+};
+
+struct ScanPlan {
+    int padded_dstate;      // dstate rounded up to 8, 16, 32 or 64
+    int lanes;              // threads per channel (R)
+    int threads;            // threads per block
+    int channels_per_block; // threads / lanes
+    int chunk;              // timesteps staged per pass
+    int vectorized;         // 16-byte loads/stores usable
+    int64_t blocks;
+    size_t smem_bytes;
+};
+
+struct StateUpdateArgs {
+    float *state;
+    const void *u, *delta, *B, *C, *z;
+    const float *A, *D, *delta_bias;
+    void *out;
+    int64_t batch, dim;
+    int dstate;
+    int softplus;
+    int act;
+};
+
+// Fills `plan` for the given sizes.  lanes/threads of 0 mean automatic.
+// Returns 0 if the configuration is valid, -1 otherwise.
+int make_scan_plan(const ScanArgs &a, int want_lanes, int want_threads,
+                   int sm_count, ScanPlan *plan);
+
+cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &plan,
+                            cudaStream_t stream);
+
+cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t stream);
+
+// Persistent, queue-balanced scan (one thread per channel, dstate <= 16).
+bool persistent_supported(const ScanArgs &a);
+bool persistent_preferred(const ScanArgs &a, int sm_count);
+size_t persistent_workspace_bound(int64_t batch, int64_t dim, int64_t seqlen, int act);
+cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, void *workspace, size_t ws_bytes,
+                                       int sm_count, cudaStream_t stream);
+
+}  // namespace mscan

@@ -1,0 +1,476 @@
+// scan_fwd.cu -- fused selective-scan (S6) forward kernel for sm_100a.
+//
+// What one launch computes (per batch row b and channel d, time in order):
+//   delta = softplus(delta_raw + bias[d]);  Abar = 2^(delta * A[d,n] * log2 e)
+//   h[n]  = Abar * h[n] + (delta * u) * B[b,n,t];   y = sum_n C[b,n,t] h[n]
+//   out   = (y + D[d] u) * silu(z)
+// following the recurrent form and the selective_scan / MambaBlock listings
+// of "Mamba SSM concept and implementation in Keras and TensorFlow", fused so
+// that nothing of size (batch, L, dim, N) ever reaches HBM (Mamba paper,
+// Appendix E.5).
+//
+// Work decomposition
+//   * A block owns one batch row and CG = THREADS / R consecutive channels and
+//     walks the whole sequence in chunks of TC timesteps, carrying the state
+//     h in registers from chunk to chunk (no inter-block communication).
+//   * Each channel's NP (padded) states are split over R consecutive lanes of
+//     one warp, S = NP / R states per thread.  R trades balance against
+//     overhead: more lanes per channel give more warps to spread over the 592
+//     SM sub-partitions but need a cross-lane sum of the readout.
+//   * Raw u / delta / z / B / C tiles are copied global -> shared with 16-byte
+//     cp.async into a double buffer, so the next chunk's loads overlap this
+//     chunk's scan.  B and C tiles are staged once per block and shared by all
+//     CG channels (they are per batch row, not per channel).
+//   * Prologue (one thread per 16-byte vector): delta = softplus(raw + bias)
+//     and delta*u are computed once per element into fp32 shared memory.
+//   * Scan: per thread, per state, per timestep: one ex2 (MUFU), one FMUL
+//     (delta*u*B), one FFMA (state), one FFMA (readout).  Partial readouts of
+//     the R lanes are summed with a transposed butterfly (log2 R shuffle
+//     rounds) so each lane ends up owning complete outputs.
+//   * Epilogue (one thread per 16-byte vector): out = (y + D u) silu(z),
+//     rounded to the activation type and stored with 16-byte stores.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "device_math.cuh"
+#include "internal.h"
+
+namespace mscan {
+
+struct KParams {
+    const void *u, *delta, *B, *C, *z;
+    const float *A, *D, *delta_bias;
+    void *out;
+    float *last_state;
+    int64_t dim, seqlen;
+    int64_t n_groups;  // channel groups per batch row
+    int dstate;
+    int softplus;
+    int vec;           // 16-byte path usable
+};
+
+// ------------------------------------------------------------ geometry
+template <typename T, int NP, int R, int THREADS>
+struct Geom {
+    static constexpr int S = NP / R;
+    static constexpr int CG = THREADS / R;
+    static constexpr int V = 16 / (int)sizeof(T);
+    static constexpr int RB = R > 4 ? R : 4;
+    static constexpr size_t smem_for(int tc) {
+        return (size_t)(2 * CG + 2 * NP) * (tc + 4) * 4 +
+               (size_t)2 * (3 * CG + 2 * NP) * tc * sizeof(T);
+    }
+    static constexpr bool tc_ok(int tc) {
+        return tc % (V * R) == 0 && tc % RB == 0;
+    }
+    // Largest chunk in {64, 32, 16, 8} that fits 56 KB (four blocks per SM),
+    // else the smallest legal chunk.
+    static constexpr int pick_tc() {
+        return (tc_ok(64) && smem_for(64) <= 56 * 1024) ? 64
+             : (tc_ok(32) && smem_for(32) <= 56 * 1024) ? 32
+             : (tc_ok(16) && smem_for(16) <= 56 * 1024) ? 16
+             : (tc_ok(8) && smem_for(8) <= 56 * 1024) ? 8
+             : tc_ok(8) ? 8 : tc_ok(16) ? 16 : tc_ok(32) ? 32 : tc_ok(64) ? 64 : 128;
+    }
+    static constexpr int TC = pick_tc();
+    static constexpr size_t SMEM = smem_for(TC);
+};
+
+// ------------------------------------------------------------ cp.async
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool pred) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    const int nbytes = pred ? 16 : 0;  // 0 -> zero-fill, nothing read
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                 :: "r"(s), "l"(gmem), "r"(nbytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// Sum v[] over the R lanes of a channel, transposed: afterwards lane r holds
+// the complete sums for indices [r * RB / R, (r + 1) * RB / R) in v[0 ..].
+// Round K (K = R/2, R/4, .., 1) halves the live values: the lane whose bit K
+// is set keeps the upper half and sends the lower half to its partner.
+template <int K, int CNT, int RB>
+struct TransposeReduce {
+    __device__ __forceinline__ static void run(float (&v)[RB], int r) {
+        constexpr int HALF = CNT / 2;
+        const bool upper = (r & K) != 0;
+#pragma unroll
+        for (int i = 0; i < HALF; ++i) {
+            const float send = upper ? v[i] : v[i + HALF];
+            const float keep = upper ? v[i + HALF] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, K);
+        }
+        TransposeReduce<K / 2, HALF, RB>::run(v, r);
+    }
+};
+template <int CNT, int RB>
+struct TransposeReduce<0, CNT, RB> {
+    __device__ __forceinline__ static void run(float (&)[RB], int) {}
+};
+
+template <int R, int RB>
+__device__ __forceinline__ void transpose_reduce(float (&v)[RB], int r) {
+    TransposeReduce<R / 2, RB, RB>::run(v, r);
+}
+
+template <typename T, int NP, int R, int THREADS>
+__global__ void __launch_bounds__(THREADS)
+scan_fwd_kernel(const KParams p) {
+    using G = Geom<T, NP, R, THREADS>;
+    constexpr int S = G::S, CG = G::CG, V = G::V, RB = G::RB, TC = G::TC;
+    constexpr int TCP = TC + 4;            // fp32 row pitch (16-byte multiple)
+    constexpr int VPR = TC / V;            // 16-byte vectors per row per chunk
+    constexpr int CH_VEC = CG * VPR;       // channel-tile vectors per tensor
+    constexpr int BC_VEC = NP * VPR;       // B (or C) tile vectors
+
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    float *sDelta = reinterpret_cast<float *>(smem_raw);  // delta, then y
+    float *sDu = sDelta + CG * TCP;                       // delta * u
+    float *sB = sDu + CG * TCP;
+    float *sC = sB + NP * TCP;
+    T *rawBase = reinterpret_cast<T *>(sC + NP * TCP);    // 2 stages
+    constexpr int STAGE = (3 * CG + 2 * NP) * TC;         // elements per stage
+
+    const int tid = threadIdx.x;
+    const int64_t grp = blockIdx.x % p.n_groups;
+    const int64_t b = blockIdx.x / p.n_groups;
+    const int64_t d0 = grp * CG;
+    const int64_t L = p.seqlen, Dm = p.dim;
+    const int N = p.dstate;
+    const bool has_z = p.z != nullptr;
+
+    const T *__restrict__ gu = static_cast<const T *>(p.u);
+    const T *__restrict__ gd = static_cast<const T *>(p.delta);
+    const T *__restrict__ gz = static_cast<const T *>(p.z);
+    const T *__restrict__ gB = static_cast<const T *>(p.B);
+    const T *__restrict__ gC = static_cast<const T *>(p.C);
+    T *__restrict__ gout = static_cast<T *>(p.out);
+    const int64_t row0 = (b * Dm + d0) * L;      // first element of this block's rows
+    const int64_t bc0 = (int64_t)b * N * L;      // first element of B[b] / C[b]
+
+    // ---- scan identity: channel c, lane r, states r*S .. r*S+S-1
+    const int c = tid / R, r = tid % R;
+    const int64_t d = d0 + c;
+    float h[S], A2[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+        const int n = r * S + s;
+        A2[s] = (d < Dm && n < N) ? __ldg(p.A + d * N + n) * kLog2e : 0.f;
+        h[s] = 0.f;
+    }
+
+    // ---- copy one chunk's raw tiles into stage `st`
+    auto issue_loads = [&](int64_t t0, int st) {
+        T *rU = rawBase + st * STAGE;
+        T *rD = rU + CG * TC;
+        T *rZ = rD + CG * TC;
+        T *rB = rZ + CG * TC;
+        T *rC = rB + NP * TC;
+        if (p.vec) {
+            for (int vi = tid; vi < CH_VEC; vi += THREADS) {
+                const int pc = vi / VPR, tv = vi % VPR;
+                const int64_t t = t0 + tv * V;
+                const bool ok = (d0 + pc < Dm) && (t < L);
+                const int64_t off = ok ? row0 + pc * L + t : 0;
+                cp_async16(rU + pc * TC + tv * V, gu + off, ok);
+                cp_async16(rD + pc * TC + tv * V, gd + off, ok);
+                if (has_z) cp_async16(rZ + pc * TC + tv * V, gz + off, ok);
+            }
+            for (int vi = tid; vi < 2 * BC_VEC; vi += THREADS) {
+                const int which = vi / BC_VEC, rem = vi % BC_VEC;
+                const int n = rem / VPR, tv = rem % VPR;
+                const int64_t t = t0 + tv * V;
+                const bool ok = (n < N) && (t < L);
+                const int64_t off = ok ? bc0 + (int64_t)n * L + t : 0;
+                cp_async16((which ? rC : rB) + n * TC + tv * V, (which ? gC : gB) + off, ok);
+            }
+            cp_async_commit();
+        } else {
+            // unaligned tensors: element loads, zero outside the problem
+            for (int e = tid; e < CG * TC; e += THREADS) {
+                const int pc = e / TC, tt = e % TC;
+                const int64_t t = t0 + tt;
+                const bool ok = (d0 + pc < Dm) && (t < L);
+                const int64_t off = row0 + pc * L + t;
+                rU[e] = ok ? gu[off] : T(0.f);
+                rD[e] = ok ? gd[off] : T(0.f);
+                if (has_z) rZ[e] = ok ? gz[off] : T(0.f);
+            }
+            for (int e = tid; e < 2 * NP * TC; e += THREADS) {
+                const int which = e / (NP * TC), rem = e % (NP * TC);
+                const int n = rem / TC, tt = rem % TC;
+                const int64_t t = t0 + tt;
+                const bool ok = (n < N) && (t < L);
+                const int64_t off = bc0 + (int64_t)n * L + t;
+                (which ? rC : rB)[rem] = ok ? (which ? gC : gB)[off] : T(0.f);
+            }
+        }
+    };
+
+    issue_loads(0, 0);
+
+    int stage = 0;
+#pragma unroll 1
+    for (int64_t t0 = 0; t0 < L; t0 += TC, stage ^= 1) {
+        const T *rU = rawBase + stage * STAGE;
+        const T *rD = rU + CG * TC;
+        const T *rZ = rD + CG * TC;
+        const T *rB = rZ + CG * TC;
+        const T *rC = rB + NP * TC;
+        const int tvalid = (L - t0) < TC ? (int)(L - t0) : TC;
+
+        if (p.vec) cp_async_wait_all();
+        __syncthreads();  // raw stage ready; previous epilogue finished
+
+        // ---- prologue: delta and delta*u for every element of the tile
+        for (int vi = tid; vi < CH_VEC; vi += THREADS) {
+            const int pc = vi / VPR, tv = vi % VPR;
+            const int64_t dd = d0 + pc;
+            const float bias = (dd < Dm && p.delta_bias) ? __ldg(p.delta_bias + dd) : 0.f;
+            float fu[V], fd[V];
+            Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + pc * TC + tv * V), fu);
+            Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rD + pc * TC + tv * V), fd);
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                float dl = fd[i] + bias;
+                if (p.softplus) dl = softplus_f(dl);
+                if (tv * V + i >= tvalid) dl = 0.f;  // past the end: Abar = 1, no input
+                fd[i] = dl;
+                fu[i] = dl * fu[i];
+            }
+            float *dst = sDelta + pc * TCP + tv * V;
+            float *dsu = sDu + pc * TCP + tv * V;
+#pragma unroll
+            for (int i = 0; i < V; i += 4) {
+                *reinterpret_cast<float4 *>(dst + i) = make_float4(fd[i], fd[i + 1], fd[i + 2], fd[i + 3]);
+                *reinterpret_cast<float4 *>(dsu + i) = make_float4(fu[i], fu[i + 1], fu[i + 2], fu[i + 3]);
+            }
+        }
+        for (int vi = tid; vi < 2 * BC_VEC; vi += THREADS) {
+            const int which = vi / BC_VEC, rem = vi % BC_VEC;
+            const int n = rem / VPR, tv = rem % VPR;
+            float f[V];
+            Elem<T>::unpack(*reinterpret_cast<const uint4 *>((which ? rC : rB) + n * TC + tv * V), f);
+            float *dst = (which ? sC : sB) + n * TCP + tv * V;
+#pragma unroll
+            for (int i = 0; i < V; i += 4)
+                *reinterpret_cast<float4 *>(dst + i) = make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
+        }
+
+        // next chunk's copies overlap this chunk's scan
+        if (t0 + TC < L) issue_loads(t0 + TC, stage ^ 1);
+        __syncthreads();
+
+        // ---- scan: thread (c, r) advances its S states through the chunk
+        {
+            float *dRow = sDelta + c * TCP;
+            const float *uRow = sDu + c * TCP;
+#pragma unroll 1
+            for (int tb = 0; tb < tvalid; tb += RB) {
+                float yp[RB];
+#pragma unroll
+                for (int q = 0; q < RB; q += 4) {
+                    const float4 dl = *reinterpret_cast<const float4 *>(dRow + tb + q);
+                    const float4 du = *reinterpret_cast<const float4 *>(uRow + tb + q);
+                    float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+#pragma unroll
+                    for (int s = 0; s < S; ++s) {
+                        const int n = r * S + s;
+                        const float4 bb = *reinterpret_cast<const float4 *>(sB + n * TCP + tb + q);
+                        const float4 cc = *reinterpret_cast<const float4 *>(sC + n * TCP + tb + q);
+                        float a;
+                        a = ex2_mufu(dl.x * A2[s]); h[s] = fmaf(a, h[s], du.x * bb.x); y0 = fmaf(cc.x, h[s], y0);
+                        a = ex2_mufu(dl.y * A2[s]); h[s] = fmaf(a, h[s], du.y * bb.y); y1 = fmaf(cc.y, h[s], y1);
+                        a = ex2_mufu(dl.z * A2[s]); h[s] = fmaf(a, h[s], du.z * bb.z); y2 = fmaf(cc.z, h[s], y2);
+                        a = ex2_mufu(dl.w * A2[s]); h[s] = fmaf(a, h[s], du.w * bb.w); y3 = fmaf(cc.w, h[s], y3);
+                    }
+                    yp[q] = y0; yp[q + 1] = y1; yp[q + 2] = y2; yp[q + 3] = y3;
+                }
+                if (R > 1) transpose_reduce<R, RB>(yp, r);
+                __syncwarp();  // every lane of the channel has read dRow[tb .. tb+RB)
+                constexpr int OWN = RB / R;  // outputs owned per lane
+                float *yo = dRow + tb + r * OWN;
+                if (OWN == 1) {
+                    yo[0] = yp[0];
+                } else if (OWN == 2) {
+                    *reinterpret_cast<float2 *>(yo) = make_float2(yp[0], yp[1]);
+                } else {
+                    *reinterpret_cast<float4 *>(yo) = make_float4(yp[0], yp[1], yp[2], yp[3]);
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- epilogue: out = (y + D u) * silu(z)
+        for (int vi = tid; vi < CH_VEC; vi += THREADS) {
+            const int pc = vi / VPR, tv = vi % VPR;
+            const int64_t dd = d0 + pc;
+            const int64_t t = t0 + tv * V;
+            if (dd >= Dm || tv * V >= tvalid) continue;
+            const float Dd = p.D ? __ldg(p.D + dd) : 0.f;
+            float fu[V], fz[V], y[V];
+            Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + pc * TC + tv * V), fu);
+            if (has_z) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rZ + pc * TC + tv * V), fz);
+            const float *ys = sDelta + pc * TCP + tv * V;
+#pragma unroll
+            for (int i = 0; i < V; i += 4) {
+                const float4 q = *reinterpret_cast<const float4 *>(ys + i);
+                y[i] = q.x; y[i + 1] = q.y; y[i + 2] = q.z; y[i + 3] = q.w;
+            }
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                float o = fmaf(Dd, fu[i], y[i]);
+                if (has_z) o *= silu_f(fz[i]);
+                y[i] = o;
+            }
+            T *dst = gout + row0 + pc * L + t;
+            if (p.vec) {
+                stg16_stream(dst, Elem<T>::pack(y));
+            } else {
+#pragma unroll
+                for (int i = 0; i < V; ++i)
+                    if (tv * V + i < tvalid) Elem<T>::store(dst + i, y[i]);
+            }
+        }
+    }
+
+    if (p.last_state != nullptr && d < Dm) {
+        float *ls = p.last_state + (b * Dm + d) * N;
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            const int n = r * S + s;
+            if (n < N) ls[n] = h[s];
+        }
+    }
+}
+
+// ------------------------------------------------------------ dispatch
+template <typename T, int NP, int R, int THREADS>
+static cudaError_t launch_impl(const KParams &kp, int64_t blocks, cudaStream_t st) {
+    using G = Geom<T, NP, R, THREADS>;
+    auto kern = scan_fwd_kernel<T, NP, R, THREADS>;
+    if (G::SMEM > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)G::SMEM);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<(unsigned)blocks, THREADS, G::SMEM, st>>>(kp);
+    return cudaGetLastError();
+}
+
+template <typename T, int NP, int R, int THREADS>
+static void geom_info(ScanPlan *pl) {
+    using G = Geom<T, NP, R, THREADS>;
+    pl->chunk = G::TC;
+    pl->channels_per_block = G::CG;
+    pl->smem_bytes = G::SMEM;
+}
+
+// Every (dtype, NP, R, THREADS) the library is built for.  R ranges over the
+// divisors of NP with at most 16 states per thread and at most 16 lanes.
+#define MSCAN_FOR_NP_R(X, T, TH) \
+    X(T, 8, 1, TH) X(T, 8, 2, TH) X(T, 8, 4, TH) X(T, 8, 8, TH) \
+    X(T, 16, 1, TH) X(T, 16, 2, TH) X(T, 16, 4, TH) X(T, 16, 8, TH) X(T, 16, 16, TH) \
+    X(T, 32, 2, TH) X(T, 32, 4, TH) X(T, 32, 8, TH) X(T, 32, 16, TH) \
+    X(T, 64, 4, TH) X(T, 64, 8, TH) X(T, 64, 16, TH)
+#define MSCAN_FOR_ALL(X) \
+    MSCAN_FOR_NP_R(X, float, 128) MSCAN_FOR_NP_R(X, float, 256) \
+    MSCAN_FOR_NP_R(X, __nv_bfloat16, 128) MSCAN_FOR_NP_R(X, __nv_bfloat16, 256)
+
+template <typename T> constexpr int act_of();
+template <> constexpr int act_of<float>() { return kF32; }
+template <> constexpr int act_of<__nv_bfloat16>() { return kBF16; }
+
+static bool lookup_geom(int act, int np, int r, int th, ScanPlan *pl) {
+#define X(T, NP_, R_, TH_) \
+    if (act == act_of<T>() && np == NP_ && r == R_ && th == TH_) { geom_info<T, NP_, R_, TH_>(pl); return true; }
+    MSCAN_FOR_ALL(X)
+#undef X
+    return false;
+}
+
+cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &pl, cudaStream_t st) {
+    KParams kp;
+    kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
+    kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias;
+    kp.out = a.out; kp.last_state = a.last_state;
+    kp.dim = a.dim; kp.seqlen = a.seqlen;
+    kp.n_groups = (a.dim + pl.channels_per_block - 1) / pl.channels_per_block;
+    kp.dstate = a.dstate; kp.softplus = a.softplus; kp.vec = pl.vectorized;
+#define X(T, NP_, R_, TH_) \
+    if (a.act == act_of<T>() && pl.padded_dstate == NP_ && pl.lanes == R_ && pl.threads == TH_) \
+        return launch_impl<T, NP_, R_, TH_>(kp, pl.blocks, st);
+    MSCAN_FOR_ALL(X)
+#undef X
+    return cudaErrorInvalidConfiguration;
+}
+
+// ------------------------------------------------------------ planning
+static int padded_dstate(int n) { return n <= 8 ? 8 : n <= 16 ? 16 : n <= 32 ? 32 : 64; }
+
+// Relative cost of one state-step for R lanes per channel (cross-lane readout
+// sums and duplicated delta reads grow with R).
+static double lane_overhead(int r) {
+    switch (r) {
+        case 1: return 1.00;
+        case 2: return 1.05;
+        case 4: return 1.12;
+        case 8: return 1.30;
+        default: return 1.60;
+    }
+}
+
+int make_scan_plan(const ScanArgs &a, int want_lanes, int want_threads, int sm_count,
+                   ScanPlan *pl) {
+    const int np = padded_dstate(a.dstate);
+    const int vbytes = 16;
+    const int esize = a.act == kBF16 ? 2 : 4;
+    const int vlen = vbytes / esize;
+    auto aligned = [](const void *ptr) { return ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
+    pl->vectorized = (a.seqlen % vlen == 0) && aligned(a.u) && aligned(a.delta) && aligned(a.z) &&
+                     aligned(a.B) && aligned(a.C) && aligned(a.out);
+    pl->padded_dstate = np;
+
+    int lanes = want_lanes;
+    if (lanes == 0) {
+        // Pick R minimising (warps on the busiest sub-partition) x (states per
+        // thread) x (per-state overhead): the scan is bound by per-SM-sub-
+        // partition MUFU throughput, so balance across the 4 x SM sub-
+        // partitions matters as much as the instruction count.
+        const double smsp = 4.0 * (sm_count > 0 ? sm_count : 148);
+        const double rows = (double)a.batch * (double)a.dim;
+        double best = 1e300;
+        for (int r = 1; r <= 16; r *= 2) {
+            if (np % r || np / r > 16) continue;
+            const double warps = rows * r / 32.0;
+            double per = warps / smsp;
+            double busiest = per <= 1.0 ? 1.0 : (double)(int64_t)(per + 0.999999);
+            const double cost = busiest * (np / r) * lane_overhead(r);
+            if (cost < best - 1e-9) { best = cost; lanes = r; }
+        }
+    }
+    int threads = want_threads;
+    if (threads == 0) {
+        threads = 256;
+        ScanPlan tmp;
+        if (lookup_geom(a.act, np, lanes, 256, &tmp)) {
+            const int64_t blocks256 = a.batch * ((a.dim + tmp.channels_per_block - 1) / tmp.channels_per_block);
+            if (blocks256 < 2LL * (sm_count > 0 ? sm_count : 148)) threads = 128;
+        }
+    }
+    if (!lookup_geom(a.act, np, lanes, threads, pl)) return -1;
+    pl->lanes = lanes;
+    pl->threads = threads;
+    pl->blocks = a.batch * ((a.dim + pl->channels_per_block - 1) / pl->channels_per_block);
+    if (pl->blocks <= 0 || pl->blocks > 0x7fffffffLL) return -1;
+    if (pl->smem_bytes > 227 * 1024) return -1;
+    return 0;
+}
+
+}  // namespace mscan

@@ -1,0 +1,425 @@
+// scan_fwd_persistent.cu -- the selective-scan (S6) forward pass as a
+// persistent, dynamically balanced kernel for sm_100a.
+//
+// Same result as scan_fwd.cu (one fused pass: softplus(delta + bias), the
+// zero-order-hold decay exp(delta A), the diagonal recurrence, the C readout,
+// the D skip and the silu(z) gate -- "Mamba SSM concept and implementation in
+// Keras and TensorFlow", recurrent form and selective_scan / MambaBlock; fused
+// without materialising (batch, L, dim, N) in HBM as in the Mamba paper,
+// Appendix E.5), organised for throughput on B200:
+//
+// * One thread owns one channel and all of its (<= 16) states, so the
+//   readout C.h needs no cross-lane sum and each element's softplus / gate is
+//   computed exactly once, by the thread that uses it.
+// * Each warp is an independent worker (its own shared-memory region, only
+//   warp-level synchronisation).  Work units are (group of 32 channels of one
+//   batch row, chunk of TU timesteps).  A unit needs the state its
+//   predecessor chunk ended with; that carry goes through global memory.
+// * Units are handed out by a ready queue: the first chunk of every group is
+//   ready at launch, and finishing chunk j of a group enqueues chunk j+1.  A
+//   worker always takes the oldest ready unit, so all SM sub-partitions stay
+//   busy until the queue drains, whatever the number of groups relative to
+//   the 4 x 148 sub-partitions -- the imbalance a static one-block-per-group
+//   launch suffers when the group count is not a multiple of the SM count.
+// * Inside a unit, sub-chunks of TC timesteps are double-buffered: raw
+//   u / delta / z rows and the per-batch-row B / C rows are copied global ->
+//   shared with 16-byte cp.async while the previous sub-chunk is computed;
+//   B and C are widened to fp32 once per sub-chunk and read as warp-wide
+//   broadcasts; outputs are packed to the activation type in a shared tile
+//   and stored with coalesced 16-byte stores.
+// * The state update runs on pairs of states with the packed fp32 x2
+//   instructions (FMUL2 / FFMA2), halving FP32 issue slots; the 16 ex2 per
+//   element go to the MUFU, which bounds the kernel.
+// * Every wait on another worker is bounded: on timeout the worker sets the
+//   error word in the workspace header and leaves; nothing spins forever.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "device_math.cuh"
+#include "internal.h"
+
+namespace mscan {
+
+namespace {
+
+constexpr int kWarps = 4;            // workers per block (one per SM sub-partition)
+constexpr int kNS = 16;              // states held per thread (dstate <= 16)
+constexpr unsigned kSpinLimit = 1u << 22;  // bounded wait (~4M polls, >1 s with backoff)
+
+struct PParams {
+    const void *u, *delta, *B, *C, *z;
+    const float *A, *D, *delta_bias;
+    void *out;
+    float *last_state;
+    int64_t dim, seqlen;
+    int dstate;
+    int softplus;
+    int groups_per_batch;  // ceil(dim / 32)
+    int n_groups;          // batch * groups_per_batch
+    int n_chunks;          // chunks per group
+    int chunk_len;         // TU, a multiple of kTC
+    unsigned *hdr;         // workspace: [head, pushed, error, pad]
+    unsigned *queue;       // workspace: n_groups * (n_chunks - 1) slots
+    float *carry;          // workspace: n_groups * 32 * 16 floats
+};
+
+template <typename T>
+struct WarpSmem {
+    static constexpr int kTC = 128 / (int)sizeof(T);       // timesteps per sub-chunk: 128-byte rows
+    static constexpr int V = 16 / (int)sizeof(T);        // elements per 16 bytes
+    static constexpr int ROWB = kTC * (int)sizeof(T) + 16;  // padded raw row (bytes)
+    static constexpr int RAW_ROWS = 3 * 32 + 2 * 16;       // u, delta, z, B, C rows
+    static constexpr int STAGE = RAW_ROWS * ROWB;
+    static constexpr int BC32 = 2 * kTC * kNS * 4;         // fp32 B and C, [t][n]
+    static constexpr int OUTB = 32 * ROWB;                 // packed output tile
+    static constexpr int BYTES = 2 * STAGE + BC32 + OUTB;
+};
+
+__device__ __forceinline__ void cp16(void *smem, const void *gmem, bool pred) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                 :: "r"(s), "l"(gmem), "r"(pred ? 16 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kWarps * 32, 1)
+scan_fwd_persistent_kernel(const PParams p) {
+    using W = WarpSmem<T>;
+    constexpr int V = W::V;
+    constexpr int kTC = W::kTC;
+    constexpr int CPR = kTC / V;  // 16-byte chunks per row per sub-chunk
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    unsigned char *base = smem + warp * W::BYTES;
+    unsigned char *stage_base = base;                       // 2 stages
+    float *bc32 = reinterpret_cast<float *>(base + 2 * W::STAGE);  // B: [t][16], then C
+    unsigned char *outt = base + 2 * W::STAGE + W::BC32;
+
+    const int64_t L = p.seqlen, Dm = p.dim;
+    const int N = p.dstate;
+    const int n_units = p.n_groups * p.n_chunks;
+    const T *gu = static_cast<const T *>(p.u);
+    const T *gd = static_cast<const T *>(p.delta);
+    const T *gz = static_cast<const T *>(p.z);
+    const T *gB = static_cast<const T *>(p.B);
+    const T *gC = static_cast<const T *>(p.C);
+    T *gout = static_cast<T *>(p.out);
+    const bool has_z = gz != nullptr;
+
+    int cur_group = -1;
+    float2 A2[kNS / 2];
+    float bias = 0.f, Dd = 0.f;
+
+#pragma unroll 1
+    while (true) {
+        // ---- take the next ready unit
+        unsigned unit = 0xffffffffu;
+        if (lane == 0) {
+            const unsigned s = atomicAdd(p.hdr + 0, 1u);
+            if ((int)s < n_units) {
+                if ((int)s < p.n_groups) {
+                    unit = s;  // chunk 0 of group s
+                } else {
+                    const unsigned *slot = p.queue + (s - p.n_groups);
+                    unsigned v = 0, spins = 0, ns = 32;
+                    while ((v = ld_acquire(slot)) == 0u) {
+                        if (++spins > kSpinLimit || ld_acquire(p.hdr + 2) != 0u) break;
+                        __nanosleep(ns);
+                        if (ns < 1024) ns <<= 1;
+                    }
+                    if (v == 0u) atomicOr(p.hdr + 2, 1u);
+                    unit = v == 0u ? 0xfffffffeu : v - 1u;
+                }
+            }
+        }
+        unit = __shfl_sync(0xffffffffu, unit, 0);
+        __syncwarp();  // order every lane's carry loads after lane 0's acquire
+        if (unit == 0xffffffffu || unit == 0xfffffffeu) break;
+        const int g = (int)(unit % (unsigned)p.n_groups);
+        const int j = (int)(unit / (unsigned)p.n_groups);
+        const int64_t b = g / p.groups_per_batch;
+        const int64_t d0 = (int64_t)(g % p.groups_per_batch) * 32;
+        const int64_t d = d0 + lane;
+        const bool dvalid = d < Dm;
+        const int nrows = (Dm - d0) < 32 ? (int)(Dm - d0) : 32;  // valid channel rows
+
+        if (g != cur_group) {
+            cur_group = g;
+#pragma unroll
+            for (int k = 0; k < kNS / 2; ++k) {
+                const int n0 = 2 * k, n1 = 2 * k + 1;
+                const float a0 = (dvalid && n0 < N) ? __ldg(p.A + d * N + n0) : 0.f;
+                const float a1 = (dvalid && n1 < N) ? __ldg(p.A + d * N + n1) : 0.f;
+                A2[k] = make_float2(a0 * kLog2e, a1 * kLog2e);
+            }
+            bias = (dvalid && p.delta_bias) ? __ldg(p.delta_bias + d) : 0.f;
+            Dd = (dvalid && p.D) ? __ldg(p.D + d) : 0.f;
+        }
+
+        // ---- carried state
+        float2 h[kNS / 2];
+        float *carry = p.carry + ((int64_t)g * 32 + lane) * kNS;
+        if (j == 0) {
+#pragma unroll
+            for (int k = 0; k < kNS / 2; ++k) h[k] = make_float2(0.f, 0.f);
+        } else {
+#pragma unroll
+            for (int k = 0; k < kNS / 4; ++k) {
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(carry) + k);
+                h[2 * k] = make_float2(v.x, v.y);
+                h[2 * k + 1] = make_float2(v.z, v.w);
+            }
+        }
+
+        const int64_t tb0 = (int64_t)j * p.chunk_len;
+        const int64_t tb1 = (tb0 + p.chunk_len) < L ? (tb0 + p.chunk_len) : L;
+        const int nsub = (int)((tb1 - tb0 + kTC - 1) / kTC);
+        const int64_t row0 = (b * Dm + d0) * L;  // element offset of this group's first row
+        const int64_t bc0 = b * (int64_t)N * L;
+
+        auto issue = [&](int sub, int st) {
+            unsigned char *sb = stage_base + st * W::STAGE;
+            const int64_t t0 = tb0 + (int64_t)sub * kTC;
+            // u, delta, z: 32 rows x CPR chunks each
+#pragma unroll
+            for (int i = lane; i < 32 * CPR; i += 32) {
+                const int r = i / CPR, c = i % CPR;
+                const int64_t t = t0 + c * V;
+                const bool ok = (r < nrows) && (t < L);
+                const int64_t off = ok ? row0 + r * L + t : 0;
+                cp16(sb + (0 * 32 + r) * W::ROWB + c * 16, gu + off, ok);
+                cp16(sb + (1 * 32 + r) * W::ROWB + c * 16, gd + off, ok);
+                if (has_z) cp16(sb + (2 * 32 + r) * W::ROWB + c * 16, gz + off, ok);
+            }
+            // B, C: 16 rows x CPR chunks each
+#pragma unroll
+            for (int i = lane; i < 2 * kNS * CPR; i += 32) {
+                const int which = i / (kNS * CPR), rem = i % (kNS * CPR);
+                const int n = rem / CPR, c = rem % CPR;
+                const int64_t t = t0 + c * V;
+                const bool ok = (n < N) && (t < L);
+                const int64_t off = ok ? bc0 + (int64_t)n * L + t : 0;
+                cp16(sb + (96 + which * 16 + n) * W::ROWB + c * 16, (which ? gC : gB) + off, ok);
+            }
+            cp_commit();
+        };
+
+        issue(0, 0);
+#pragma unroll 1
+        for (int sub = 0; sub < nsub; ++sub) {
+            const int st = sub & 1;
+            if (sub + 1 < nsub) {
+                issue(sub + 1, st ^ 1);
+                cp_wait<1>();
+            } else {
+                cp_wait<0>();
+            }
+            __syncwarp();
+            const unsigned char *sb = stage_base + st * W::STAGE;
+            const int64_t t0 = tb0 + (int64_t)sub * kTC;
+            const int tvalid = (L - t0) < kTC ? (int)(L - t0) : kTC;
+
+            // widen B and C to fp32, transposed to [t][n] for broadcast reads
+#pragma unroll
+            for (int i = lane; i < 2 * kNS * CPR; i += 32) {
+                const int which = i / (kNS * CPR), rem = i % (kNS * CPR);
+                const int n = rem / CPR, c = rem % CPR;
+                float f[V];
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sb + (96 + which * 16 + n) * W::ROWB + c * 16), f);
+                float *dst = bc32 + which * kTC * kNS;
+#pragma unroll
+                for (int e = 0; e < V; ++e) dst[(c * V + e) * kNS + n] = f[e];
+            }
+            __syncwarp();
+
+            const unsigned char *ru = sb + (0 * 32 + lane) * W::ROWB;
+            const unsigned char *rd = sb + (1 * 32 + lane) * W::ROWB;
+            const unsigned char *rz = sb + (2 * 32 + lane) * W::ROWB;
+            unsigned char *ro = outt + lane * W::ROWB;
+            const float *sBt = bc32;
+            const float *sCt = bc32 + kTC * kNS;
+#pragma unroll 1
+            for (int tv = 0; tv < tvalid; tv += V) {
+                float fu[V], fd[V], fz[V], fo[V];
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(ru + tv * sizeof(T)), fu);
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rd + tv * sizeof(T)), fd);
+                if (has_z) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rz + tv * sizeof(T)), fz);
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    const int t = tv + e;
+                    float dl = fd[e] + bias;
+                    if (p.softplus) dl = softplus_f(dl);
+                    if (t >= tvalid) dl = 0.f;  // past the end: Abar = 1, no input
+                    const float dlu = dl * fu[e];
+                    const float2 dl2 = make_float2(dl, dl);
+                    const float2 du2 = make_float2(dlu, dlu);
+                    const float4 *bq = reinterpret_cast<const float4 *>(sBt + t * kNS);
+                    const float4 *cq = reinterpret_cast<const float4 *>(sCt + t * kNS);
+                    float2 y2 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int q = 0; q < kNS / 4; ++q) {
+                        const float4 bb = bq[q];
+                        const float4 cc = cq[q];
+                        const float2 x0 = __fmul2_rn(dl2, A2[2 * q]);
+                        const float2 x1 = __fmul2_rn(dl2, A2[2 * q + 1]);
+                        const float2 a0 = make_float2(ex2_mufu(x0.x), ex2_mufu(x0.y));
+                        const float2 a1 = make_float2(ex2_mufu(x1.x), ex2_mufu(x1.y));
+                        const float2 bu0 = __fmul2_rn(du2, make_float2(bb.x, bb.y));
+                        const float2 bu1 = __fmul2_rn(du2, make_float2(bb.z, bb.w));
+                        h[2 * q] = __ffma2_rn(a0, h[2 * q], bu0);
+                        h[2 * q + 1] = __ffma2_rn(a1, h[2 * q + 1], bu1);
+                        y2 = __ffma2_rn(make_float2(cc.x, cc.y), h[2 * q], y2);
+                        y2 = __ffma2_rn(make_float2(cc.z, cc.w), h[2 * q + 1], y2);
+                    }
+                    float o = fmaf(Dd, fu[e], y2.x + y2.y);
+                    if (has_z) o *= silu_f(fz[e]);
+                    fo[e] = o;
+                }
+                *reinterpret_cast<uint4 *>(ro + tv * sizeof(T)) = Elem<T>::pack(fo);
+            }
+            __syncwarp();
+            // coalesced store of the packed tile
+#pragma unroll
+            for (int i = lane; i < 32 * CPR; i += 32) {
+                const int r = i / CPR, c = i % CPR;
+                const int64_t t = t0 + c * V;
+                if (r < nrows && t < L)
+                    stg16_stream(gout + row0 + r * L + t,
+                                 *reinterpret_cast<const uint4 *>(outt + r * W::ROWB + c * 16));
+            }
+            __syncwarp();
+        }
+
+        if (j + 1 < p.n_chunks) {
+#pragma unroll
+            for (int k = 0; k < kNS / 4; ++k)
+                __stcg(reinterpret_cast<float4 *>(carry) + k,
+                       make_float4(h[2 * k].x, h[2 * k].y, h[2 * k + 1].x, h[2 * k + 1].y));
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence();
+                const unsigned slot = atomicAdd(p.hdr + 1, 1u);
+                st_release(p.queue + slot, (unsigned)((j + 1) * p.n_groups + g) + 1u);
+            }
+        } else if (p.last_state != nullptr && dvalid) {
+            float *ls = p.last_state + (b * Dm + d) * N;
+#pragma unroll
+            for (int k = 0; k < kNS / 2; ++k) {
+                if (2 * k < N) ls[2 * k] = h[k].x;
+                if (2 * k + 1 < N) ls[2 * k + 1] = h[k].y;
+            }
+        }
+    }
+}
+
+}  // namespace
+
+// Workspace bytes for a persistent launch over these sizes (0 if the
+// persistent kernel does not apply).
+size_t persistent_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, int chunk_len) {
+    const int64_t gpb = (dim + 31) / 32;
+    const int64_t groups = batch * gpb;
+    const int64_t chunks = (seqlen + chunk_len - 1) / chunk_len;
+    const int64_t queue = groups * (chunks > 0 ? chunks - 1 : 0);
+    return 16 + (size_t)((queue * 4 + 255) / 256 * 256) + (size_t)(groups * 32 * kNS * 4);
+}
+
+// Upper bound of persistent_workspace_bytes over every device: the chunk
+// count never exceeds a quarter of the sub-chunk count (rounded up).
+size_t persistent_workspace_bound(int64_t batch, int64_t dim, int64_t seqlen, int act) {
+    const int kTC = act == kBF16 ? WarpSmem<__nv_bfloat16>::kTC : WarpSmem<float>::kTC;
+    const int64_t max_chunks = ((seqlen + kTC - 1) / kTC + 3) / 4;
+    const int64_t tu = ((seqlen + max_chunks - 1) / max_chunks + kTC - 1) / kTC * kTC;
+    return persistent_workspace_bytes(batch, dim, seqlen, (int)(tu < kTC ? kTC : tu)) +
+           (size_t)(batch * ((dim + 31) / 32)) * 4 + 256;
+}
+
+int persistent_chunk_len(int64_t batch, int64_t dim, int64_t seqlen, int sm_count, int act) {
+    const int kTC = act == kBF16 ? WarpSmem<__nv_bfloat16>::kTC : WarpSmem<float>::kTC;
+    // Aim for >= 16 units per worker so the drain at the end of the queue is
+    // short, but keep units >= 4 sub-chunks so per-unit costs stay small.
+    const int64_t groups = batch * ((dim + 31) / 32);
+    const int64_t workers = (int64_t)sm_count * kWarps;
+    const int64_t max_chunks = (seqlen + kTC - 1) / kTC;
+    int64_t want = (16 * workers + groups - 1) / groups;
+    int64_t lim = (max_chunks + 3) / 4;
+    if (lim < 1) lim = 1;
+    if (want > lim) want = lim;
+    if (want < 1) want = 1;
+    int64_t tu = (seqlen + want - 1) / want;
+    tu = (tu + kTC - 1) / kTC * kTC;
+    return (int)tu;
+}
+
+bool persistent_supported(const ScanArgs &a) {
+    if (a.dstate > kNS) return false;
+    const int es = a.act == kBF16 ? 2 : 4;
+    if (a.seqlen % (16 / es) != 0) return false;
+    auto al = [](const void *q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+    if (!(al(a.u) && al(a.delta) && al(a.z) && al(a.B) && al(a.C) && al(a.out))) return false;
+    const int64_t groups = a.batch * ((a.dim + 31) / 32);
+    const int64_t chunks = (a.seqlen + (128 / es) - 1) / (128 / es);
+    return groups * chunks < (int64_t)1 << 30;
+}
+
+bool persistent_preferred(const ScanArgs &a, int sm_count) {
+    // Enough channel groups to give every worker a chain of its own (minus
+    // 10 %); with fewer, the static schedule splits each channel's states
+    // over several lanes and keeps more warps busy.
+    const int64_t groups = a.batch * ((a.dim + 31) / 32);
+    return groups * 10 >= (int64_t)sm_count * kWarps * 9;
+}
+
+template <typename T>
+static cudaError_t launch_persistent_t(const PParams &kp, int sm_count, cudaStream_t st) {
+    const int smem = kWarps * WarpSmem<T>::BYTES;
+    cudaError_t e = cudaFuncSetAttribute(scan_fwd_persistent_kernel<T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int units = kp.n_groups * kp.n_chunks;
+    int grid = sm_count;
+    if (grid * kWarps > units) grid = (units + kWarps - 1) / kWarps;
+    scan_fwd_persistent_kernel<T><<<grid, kWarps * 32, smem, st>>>(kp);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, void *workspace, size_t ws_bytes,
+                                       int sm_count, cudaStream_t st) {
+    PParams kp;
+    kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
+    kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias;
+    kp.out = a.out; kp.last_state = a.last_state;
+    kp.dim = a.dim; kp.seqlen = a.seqlen; kp.dstate = a.dstate; kp.softplus = a.softplus;
+    kp.groups_per_batch = (int)((a.dim + 31) / 32);
+    kp.n_groups = (int)(a.batch * kp.groups_per_batch);
+    kp.chunk_len = persistent_chunk_len(a.batch, a.dim, a.seqlen, sm_count, a.act);
+    kp.n_chunks = (int)((a.seqlen + kp.chunk_len - 1) / kp.chunk_len);
+    const size_t need = persistent_workspace_bytes(a.batch, a.dim, a.seqlen, kp.chunk_len);
+    if (ws_bytes < need) return cudaErrorInvalidValue;
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    const int64_t qn = (int64_t)kp.n_groups * (kp.n_chunks - 1);
+    kp.hdr = reinterpret_cast<unsigned *>(w);
+    kp.queue = reinterpret_cast<unsigned *>(w + 16);
+    kp.carry = reinterpret_cast<float *>(w + 16 + (qn * 4 + 255) / 256 * 256);
+    // header and queue start at zero; carries are always written before read
+    cudaError_t e = cudaMemsetAsync(w, 0, 16 + (size_t)qn * 4, st);
+    if (e != cudaSuccess) return e;
+    if (a.act == kBF16) return launch_persistent_t<__nv_bfloat16>(kp, sm_count, st);
+    return launch_persistent_t<float>(kp, sm_count, st);
+}
+
+}  // namespace mscan

@@ -1,0 +1,115 @@
+"""The C-ABI library on the host, without a GPU: it loads, exports every
+function include/mamba_scan.h declares, and rejects bad arguments with the
+documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from selective_state_space_20_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mamba_scan.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(mamba_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_abi():
+    assert declared_functions() == sorted(binding.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} not exported"
+    out = os.popen(f"nm -D --defined-only {build.LIB}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}\b", out), f"{name} missing from dynamic symbol table"
+
+
+def test_library_is_built_for_sm100a_only():
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_status_strings_and_version(lib):
+    for code in list(binding.STATUS_NAMES) + [12345]:
+        s = lib.mamba_status_string(code)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert lib.mamba_abi_version() >> 16 == 1
+
+
+def _scan(lib, ptrs=None, batch=2, dim=4, L=8, N=16, dtype=1, softplus=1, last=None, tuning=None):
+    P = ptrs or {}
+    get = lambda k, default=0x10000: P.get(k, default)  # noqa: E731
+    args = [get("u", 0x100000), get("delta", 0x200000), get("A", 0x300000), get("B", 0x400000),
+            get("C", 0x500000), get("D", None), get("z", None), get("bias", None), softplus,
+            get("out", 0x600000), last, batch, dim, L, N, dtype]
+    args = [ctypes.c_void_p(a) if isinstance(a, int) and i not in (8, 11, 12, 13, 14, 15) else a
+            for i, a in enumerate(args)]
+    if tuning is not None:
+        return lib.mamba_scan_fwd_tuned(*args, ctypes.byref(tuning), None)
+    return lib.mamba_scan_fwd(*args, None)
+
+
+def test_null_pointers_rejected(lib):
+    for key in ("u", "delta", "A", "B", "C", "out"):
+        assert _scan(lib, {key: None}) == -1, key
+
+
+def test_bad_sizes_rejected(lib):
+    assert _scan(lib, batch=0) == -2
+    assert _scan(lib, dim=-3) == -2
+    assert _scan(lib, L=0) == -2
+    assert _scan(lib, N=0) == -2
+    assert _scan(lib, N=65) == -3
+    assert _scan(lib, dtype=7) == -3
+    assert _scan(lib, batch=1 << 40, dim=1 << 20) == -2
+
+
+def test_overlap_rejected(lib):
+    # out shifted into u by one element: partial overlap
+    assert _scan(lib, {"u": 0x100000, "out": 0x100002}) == -7
+    # out overlapping B
+    assert _scan(lib, {"B": 0x600000, "out": 0x600000}) == -7
+    # last_state overlapping out
+    assert _scan(lib, {"out": 0x600000}, last=ctypes.c_void_p(0x600010)) == -7
+
+
+def test_bad_tuning_rejected(lib):
+    assert _scan(lib, tuning=binding.Tuning(3, 0)) == -3
+    assert _scan(lib, tuning=binding.Tuning(0, 100)) == -3
+
+
+def test_state_update_validation(lib):
+    su = lib.mamba_state_update
+    vp = ctypes.c_void_p
+    ok = [vp(0x100000), vp(0x200000), vp(0x300000), vp(0x400000), vp(0x500000), vp(0x600000),
+          None, None, None, 1, vp(0x700000), 4, 8, 16, 1, None]
+    bad = list(ok)
+    bad[0] = None
+    assert su(*bad) == -1
+    bad = list(ok)
+    bad[11] = 0
+    assert su(*bad) == -2
+    bad = list(ok)
+    bad[13] = 100
+    assert su(*bad) == -3
+    bad = list(ok)
+    bad[10] = vp(0x100000 + 8)  # out inside the state
+    assert su(*bad) == -7
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 2, 8)
+    with pytest.raises(ValueError):
+        binding.mamba_scan_fwd(x, x, torch.zeros(2, 16), torch.zeros(1, 16, 8), torch.zeros(1, 16, 8))
