@@ -94,7 +94,7 @@ __device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
 }
 
-template <typename T>
+template <typename T, bool SP, bool GATE>
 __global__ void __launch_bounds__(kWarps * 32, 1)
 scan_fwd_persistent_kernel(const PParams p) {
     using W = WarpSmem<T>;
@@ -118,8 +118,6 @@ scan_fwd_persistent_kernel(const PParams p) {
     const T *gB = static_cast<const T *>(p.B);
     const T *gC = static_cast<const T *>(p.C);
     T *gout = static_cast<T *>(p.out);
-    const bool has_z = gz != nullptr;
-
     int cur_group = -1;
     float2 A2[kNS / 2];
     float bias = 0.f, Dd = 0.f;
@@ -203,7 +201,7 @@ scan_fwd_persistent_kernel(const PParams p) {
                 const int64_t off = ok ? row0 + r * L + t : 0;
                 cp16(sb + (0 * 32 + r) * W::ROWB + c * 16, gu + off, ok);
                 cp16(sb + (1 * 32 + r) * W::ROWB + c * 16, gd + off, ok);
-                if (has_z) cp16(sb + (2 * 32 + r) * W::ROWB + c * 16, gz + off, ok);
+                if (GATE) cp16(sb + (2 * 32 + r) * W::ROWB + c * 16, gz + off, ok);
             }
             // B, C: 16 rows x CPR chunks each
 #pragma unroll
@@ -254,26 +252,36 @@ scan_fwd_persistent_kernel(const PParams p) {
             const float *sCt = bc32 + kTC * kNS;
 #pragma unroll 1
             for (int tv = 0; tv < tvalid; tv += V) {
-                float fu[V], fd[V], fz[V], fo[V];
+                float fu[V], fd[V], fz[V];
                 Elem<T>::unpack(*reinterpret_cast<const uint4 *>(ru + tv * sizeof(T)), fu);
                 Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rd + tv * sizeof(T)), fd);
-                if (has_z) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rz + tv * sizeof(T)), fz);
+                if (GATE) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rz + tv * sizeof(T)), fz);
+                // per element, V independent chains: delta, delta*u, gate
+                float dl[V], du[V], gg[V];
 #pragma unroll
                 for (int e = 0; e < V; ++e) {
-                    const int t = tv + e;
-                    float dl = fd[e] + bias;
-                    if (p.softplus) dl = softplus_f(dl);
-                    if (t >= tvalid) dl = 0.f;  // past the end: Abar = 1, no input
-                    const float dlu = dl * fu[e];
-                    const float2 dl2 = make_float2(dl, dl);
-                    const float2 du2 = make_float2(dlu, dlu);
-                    const float4 *bq = reinterpret_cast<const float4 *>(sBt + t * kNS);
-                    const float4 *cq = reinterpret_cast<const float4 *>(sCt + t * kNS);
-                    float2 y2 = make_float2(0.f, 0.f);
+                    float x = fd[e] + bias;
+                    if (SP) x = softplus_f(x);
+                    dl[e] = (tv + e < tvalid) ? x : 0.f;  // past the end: Abar = 1, no input
+                    du[e] = dl[e] * fu[e];
+                    gg[e] = GATE ? silu_f(fz[e]) : 1.f;
+                }
+                // states: state pairs outer, timesteps inner.  Per pair the
+                // recurrence is a short FFMA2 chain through the V timesteps;
+                // the exponentials depend only on dl and can all be issued
+                // ahead; the V readout sums are independent accumulators.
+                float2 y2[V];
 #pragma unroll
-                    for (int q = 0; q < kNS / 4; ++q) {
-                        const float4 bb = bq[q];
-                        const float4 cc = cq[q];
+                for (int e = 0; e < V; ++e) y2[e] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int q = 0; q < kNS / 4; ++q) {
+#pragma unroll
+                    for (int e = 0; e < V; ++e) {
+                        const int t = tv + e;
+                        const float4 bb = *reinterpret_cast<const float4 *>(sBt + t * kNS + 4 * q);
+                        const float4 cc = *reinterpret_cast<const float4 *>(sCt + t * kNS + 4 * q);
+                        const float2 dl2 = make_float2(dl[e], dl[e]);
+                        const float2 du2 = make_float2(du[e], du[e]);
                         const float2 x0 = __fmul2_rn(dl2, A2[2 * q]);
                         const float2 x1 = __fmul2_rn(dl2, A2[2 * q + 1]);
                         const float2 a0 = make_float2(ex2_mufu(x0.x), ex2_mufu(x0.y));
@@ -282,13 +290,16 @@ scan_fwd_persistent_kernel(const PParams p) {
                         const float2 bu1 = __fmul2_rn(du2, make_float2(bb.z, bb.w));
                         h[2 * q] = __ffma2_rn(a0, h[2 * q], bu0);
                         h[2 * q + 1] = __ffma2_rn(a1, h[2 * q + 1], bu1);
-                        y2 = __ffma2_rn(make_float2(cc.x, cc.y), h[2 * q], y2);
-                        y2 = __ffma2_rn(make_float2(cc.z, cc.w), h[2 * q + 1], y2);
+                        y2[e] = __ffma2_rn(make_float2(cc.x, cc.y), h[2 * q], y2[e]);
+                        y2[e] = __ffma2_rn(make_float2(cc.z, cc.w), h[2 * q + 1], y2[e]);
                     }
-                    float o = fmaf(Dd, fu[e], y2.x + y2.y);
-                    if (has_z) o *= silu_f(fz[e]);
-                    fo[e] = o;
                 }
+                float yv[V];
+#pragma unroll
+                for (int e = 0; e < V; ++e) yv[e] = y2[e].x + y2[e].y;
+                float fo[V];
+#pragma unroll
+                for (int e = 0; e < V; ++e) fo[e] = fmaf(Dd, fu[e], yv[e]) * gg[e];
                 *reinterpret_cast<uint4 *>(ro + tv * sizeof(T)) = Elem<T>::pack(fo);
             }
             __syncwarp();
@@ -384,17 +395,27 @@ bool persistent_preferred(const ScanArgs &a, int sm_count) {
     return groups * 10 >= (int64_t)sm_count * kWarps * 9;
 }
 
-template <typename T>
+template <typename T, bool SP, bool GATE>
 static cudaError_t launch_persistent_t(const PParams &kp, int sm_count, cudaStream_t st) {
     const int smem = kWarps * WarpSmem<T>::BYTES;
-    cudaError_t e = cudaFuncSetAttribute(scan_fwd_persistent_kernel<T>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    auto kern = scan_fwd_persistent_kernel<T, SP, GATE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int units = kp.n_groups * kp.n_chunks;
     int grid = sm_count;
     if (grid * kWarps > units) grid = (units + kWarps - 1) / kWarps;
-    scan_fwd_persistent_kernel<T><<<grid, kWarps * 32, smem, st>>>(kp);
+    kern<<<grid, kWarps * 32, smem, st>>>(kp);
     return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_persistent_flags(const PParams &kp, int sm_count, cudaStream_t st) {
+    const bool gate = kp.z != nullptr;
+    if (kp.softplus)
+        return gate ? launch_persistent_t<T, true, true>(kp, sm_count, st)
+                    : launch_persistent_t<T, true, false>(kp, sm_count, st);
+    return gate ? launch_persistent_t<T, false, true>(kp, sm_count, st)
+                : launch_persistent_t<T, false, false>(kp, sm_count, st);
 }
 
 cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, void *workspace, size_t ws_bytes,
@@ -418,8 +439,8 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, void *workspace, size_
     // header and queue start at zero; carries are always written before read
     cudaError_t e = cudaMemsetAsync(w, 0, 16 + (size_t)qn * 4, st);
     if (e != cudaSuccess) return e;
-    if (a.act == kBF16) return launch_persistent_t<__nv_bfloat16>(kp, sm_count, st);
-    return launch_persistent_t<float>(kp, sm_count, st);
+    if (a.act == kBF16) return launch_persistent_flags<__nv_bfloat16>(kp, sm_count, st);
+    return launch_persistent_flags<float>(kp, sm_count, st);
 }
 
 }  // namespace mscan
