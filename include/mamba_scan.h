@@ -179,6 +179,41 @@ int mamba_scan_fwd_ws(const void *u, const void *delta, const float *A,
 int mamba_scan_workspace_status(const void *workspace, cudaStream_t stream);
 
 /*
+ * mamba_scan_fwd_noalloc -- mamba_scan_fwd for callers that cannot allocate
+ * device memory.  (No counterpart in the paper: this is an interface
+ * convenience, not part of the method.)
+ *
+ * Some callers have no way to obtain a device workspace to hand over: a
+ * plugin or foreign-language host that links only this library and is given
+ * just its input and output buffers, or a process whose device memory is
+ * owned by a pooling allocator that must not see extra cudaMalloc calls.
+ * For them this entry point runs the same computation as mamba_scan_fwd_ws
+ * (same arguments and results as mamba_scan_fwd) using a 4 MiB scratch area
+ * built into the library instead of a caller workspace, and calls no
+ * cudaMalloc, cudaFree or other allocating routine.  The caller still
+ * provides every input and output.
+ *
+ * - Every GPU that loads the library reserves the 4 MiB area until the
+ *   process exits.
+ * - Problems whose workspace (mamba_scan_workspace_size) exceeds 4 MiB are
+ *   rejected with MAMBA_ERR_WORKSPACE before anything is enqueued; that is
+ *   about 2,000 groups of 32 channels (batch * ceil(dim / 32)) at moderate
+ *   lengths.
+ * - The first call on each device looks up the area's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture begins.
+ * - All calls share the one area and each launch re-initialises the part
+ *   that must start at zero; calls whose GPU work can overlap (other streams,
+ *   other host threads) race on it and must be serialised by the caller.
+ */
+int mamba_scan_fwd_noalloc(const void *u, const void *delta, const float *A,
+                           const void *B, const void *C, const float *D,
+                           const void *z, const float *delta_bias,
+                           int delta_softplus, void *out, float *last_state,
+                           int64_t batch, int64_t dim, int64_t seqlen,
+                           int64_t dstate, int act_dtype, cudaStream_t stream);
+
+/*
  * mamba_state_update -- one recurrent step (one token) for every channel,
  * with the state held in HBM and updated in place: the decoding form used by
  * generation, one token per call (mamba-jax sample.py; the generation

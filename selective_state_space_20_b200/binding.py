@@ -30,7 +30,8 @@ SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT = 0, 1, 2
 # Every function include/mamba_scan.h declares.
 EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
-            "mamba_state_update", "mamba_status_string", "mamba_abi_version")
+            "mamba_scan_fwd_noalloc", "mamba_state_update", "mamba_status_string",
+            "mamba_abi_version")
 
 
 class MambaError(RuntimeError):
@@ -57,6 +58,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_fwd_tuned.restype = ci
     lib.mamba_scan_fwd_ws.argtypes = scan_args + [ctypes.POINTER(Tuning), vp, ctypes.c_size_t, vp]
     lib.mamba_scan_fwd_ws.restype = ci
+    lib.mamba_scan_fwd_noalloc.argtypes = scan_args + [vp]
+    lib.mamba_scan_fwd_noalloc.restype = ci
     lib.mamba_scan_plan.argtypes = [i64, i64, i64, i64, ci, ctypes.POINTER(Tuning)]
     lib.mamba_scan_plan.restype = ci
     lib.mamba_scan_workspace_size.argtypes = [i64, i64, i64, i64, ci]
