@@ -78,17 +78,18 @@ typedef enum {
     MAMBA_SCHEDULE_AUTO = 0,
     MAMBA_SCHEDULE_STATIC = 1,     /* one block per channel group walks the whole
                                       sequence; no workspace */
-    MAMBA_SCHEDULE_PERSISTENT = 2  /* one thread per channel and all its states
-                                      (dstate <= 16); persistent workers take
-                                      (32-channel group, time chunk) units from a
+    MAMBA_SCHEDULE_PERSISTENT = 2  /* dstate <= 16: persistent warps take
+                                      (channel group, time chunk) units from a
                                       ready queue and pass the state between
-                                      chunks through the workspace */
+                                      chunks through the workspace; one or two
+                                      lanes per channel */
 } mamba_schedule_t;
 
 /* Optional launch tuning.  Zero fields mean "choose automatically".
- *   lanes_per_channel : static schedule only: threads sharing one channel's
- *                       states (1, 2, 4, 8 or 16; the padded dstate must be a
- *                       multiple, and at most 16 states stay in one thread)
+ *   lanes_per_channel : threads sharing one channel's states.  Static
+ *                       schedule: 1, 2, 4, 8 or 16 (the padded dstate must be
+ *                       a multiple, and at most 16 states stay in one
+ *                       thread).  Persistent schedule: 1 or 2.
  *   threads_per_block : static schedule only: 128 or 256
  *   schedule          : a mamba_schedule_t
  */

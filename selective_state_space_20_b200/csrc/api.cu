@@ -121,22 +121,27 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
                                                    batch, dim, seqlen, act_dtype));
     const bool supported = mscan::persistent_supported(a);
     bool persist = false;
+    int persist_lanes = 0;
     if (want_sched == MAMBA_SCHEDULE_PERSISTENT) {
-        if (!supported) return MAMBA_ERR_UNSUPPORTED;
+        if (!supported || want_threads != 0 || (want_lanes != 0 && want_lanes != 1 && want_lanes != 2))
+            return MAMBA_ERR_UNSUPPORTED;
         if (!ws_ok) return MAMBA_ERR_WORKSPACE;
         persist = true;
-    } else if (want_sched == MAMBA_SCHEDULE_AUTO) {
-        persist = supported && ws_ok && mscan::persistent_preferred(a, sms) &&
-                  want_lanes == 0 && want_threads == 0;
+        persist_lanes = want_lanes != 0 ? want_lanes : mscan::persistent_choose_lanes(a, sms);
+        if (persist_lanes == 0) persist_lanes = 1;
+    } else if (want_sched == MAMBA_SCHEDULE_AUTO && want_lanes == 0 && want_threads == 0) {
+        persist_lanes = supported && ws_ok ? mscan::persistent_choose_lanes(a, sms) : 0;
+        persist = persist_lanes != 0;
     }
     if (persist) {
         if (plan_out) {
-            plan_out->lanes_per_channel = 1;
+            plan_out->lanes_per_channel = persist_lanes;
             plan_out->threads_per_block = 128;
             plan_out->schedule = MAMBA_SCHEDULE_PERSISTENT;
         }
         if (!launch) return MAMBA_OK;
-        return mscan::launch_scan_fwd_persistent(a, workspace, ws_bytes, sms, stream) == cudaSuccess
+        return mscan::launch_scan_fwd_persistent(a, persist_lanes, workspace, ws_bytes, sms,
+                                                 stream) == cudaSuccess
                    ? MAMBA_OK : MAMBA_ERR_CUDA;
     }
     mscan::ScanPlan pl;

@@ -52,11 +52,12 @@ cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &plan,
 
 cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t stream);
 
-// Persistent, queue-balanced scan (one thread per channel, dstate <= 16).
+// Persistent, queue-balanced scan (dstate <= 16), one or two lanes per channel.
 bool persistent_supported(const ScanArgs &a);
 bool persistent_preferred(const ScanArgs &a, int sm_count);
+int persistent_choose_lanes(const ScanArgs &a, int sm_count);  // 0 = not preferred
 size_t persistent_workspace_bound(int64_t batch, int64_t dim, int64_t seqlen, int act);
-cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, void *workspace, size_t ws_bytes,
-                                       int sm_count, cudaStream_t stream);
+cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, void *workspace,
+                                       size_t ws_bytes, int sm_count, cudaStream_t stream);
 
 }  // namespace mscan

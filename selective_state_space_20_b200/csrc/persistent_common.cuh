@@ -1,0 +1,108 @@
+// persistent_common.cuh -- pieces shared by the persistent scan kernels: the
+// launch parameters, the ready queue of (channel group, time chunk) units,
+// asynchronous global -> shared copies and acquire/release flags.
+//
+// Ready queue.  Unit u = j * n_groups + g is chunk j of channel group g.  All
+// chunk-0 units are ready at launch and occupy the first n_groups pop slots
+// implicitly.  Finishing chunk j < n_chunks - 1 of a group writes that
+// group's carried state, then appends unit (j + 1, g) to the queue (slot =
+// atomic counter, value released after the carry).  A pop at slot s >=
+// n_groups waits for queue entry s - n_groups.  Every popped unit is already
+// being run by a resident worker, so the entries a waiter needs are always
+// produced: the scheme cannot deadlock, whatever the residency.  Waits are
+// bounded all the same; a worker that gives up raises the error word, which
+// makes every other waiter give up too.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mscan {
+namespace persist {
+
+constexpr int kWarps = 4;                  // workers per block
+constexpr int kNS = 16;                    // max states per channel (dstate <= 16)
+constexpr unsigned kSpinLimit = 1u << 22;  // polls before a waiter gives up
+constexpr unsigned kUnitDone = 0xffffffffu;
+constexpr unsigned kUnitAbort = 0xfffffffeu;
+
+struct Params {
+    const void *u, *delta, *B, *C, *z;
+    const float *A, *D, *delta_bias;
+    void *out;
+    float *last_state;
+    int64_t dim, seqlen;
+    int dstate;
+    int softplus;
+    int group_channels;    // channels per unit: 32 (one lane per channel) or 16 (lane pairs)
+    int groups_per_batch;  // ceil(dim / group_channels)
+    int n_groups;          // batch * groups_per_batch
+    int n_chunks;          // chunks per group
+    int chunk_len;         // timesteps per chunk
+    unsigned *hdr;         // workspace: [pop counter, push counter, error, unused]
+    unsigned *queue;       // workspace: n_groups * (n_chunks - 1) entries
+    float *carry;          // workspace: n_groups * 32 lanes * states-per-lane floats
+};
+
+__device__ __forceinline__ void cp16(void *smem, const void *gmem, bool pred) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                 :: "r"(s), "l"(gmem), "r"(pred ? 16 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+
+// Next unit for this warp (call from all lanes; lane 0 talks to the queue).
+// Returns kUnitDone when the queue is drained, kUnitAbort after a timeout.
+// The trailing __syncwarp orders every lane's later carry loads after lane
+// 0's acquire.
+__device__ __forceinline__ unsigned pop_unit(const Params &p, int lane) {
+    const int n_units = p.n_groups * p.n_chunks;
+    unsigned unit = kUnitDone;
+    if (lane == 0) {
+        const unsigned s = atomicAdd(p.hdr + 0, 1u);
+        if ((int)s < n_units) {
+            if ((int)s < p.n_groups) {
+                unit = s;  // chunk 0 of group s
+            } else {
+                const unsigned *slot = p.queue + (s - p.n_groups);
+                unsigned v = 0, spins = 0, ns = 32;
+                while ((v = ld_acquire(slot)) == 0u) {
+                    if (++spins > kSpinLimit || ld_acquire(p.hdr + 2) != 0u) break;
+                    __nanosleep(ns);
+                    if (ns < 1024) ns <<= 1;
+                }
+                if (v == 0u) atomicOr(p.hdr + 2, 1u);
+                unit = v == 0u ? kUnitAbort : v - 1u;
+            }
+        }
+    }
+    unit = __shfl_sync(0xffffffffu, unit, 0);
+    __syncwarp();
+    return unit;
+}
+
+// Publish the successor of a finished unit.  Every lane must have written
+// its part of the carry before the call (the __syncwarp orders them before
+// lane 0's fence and release).
+__device__ __forceinline__ void push_unit(const Params &p, int lane, unsigned next_unit) {
+    __syncwarp();
+    if (lane == 0) {
+        __threadfence();
+        const unsigned slot = atomicAdd(p.hdr + 1, 1u);
+        st_release(p.queue + slot, next_unit + 1u);
+    }
+}
+
+}  // namespace persist
+}  // namespace mscan

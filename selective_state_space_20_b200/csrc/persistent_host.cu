@@ -1,0 +1,138 @@
+// persistent_host.cu -- planning for the persistent scan kernels: which
+// variant (one lane or two lanes per channel), chunk length, workspace
+// layout, grid size.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+#include "persistent_kernels.h"
+
+namespace mscan {
+
+namespace {
+
+int group_channels(int lanes) { return lanes == 2 ? 16 : 32; }
+int states_per_lane(int lanes) { return lanes == 2 ? 8 : 16; }
+int sub_chunk(int lanes, int act) {
+    return lanes == 2 ? persistent_lanes2_sub_chunk(act) : persistent_lanes1_sub_chunk(act);
+}
+int blocks_per_sm(int lanes) {
+    return lanes == 2 ? persistent_lanes2_blocks_per_sm() : persistent_lanes1_blocks_per_sm();
+}
+int64_t n_groups(int64_t batch, int64_t dim, int lanes) {
+    const int cw = group_channels(lanes);
+    return batch * ((dim + cw - 1) / cw);
+}
+
+// Timesteps per work unit: >= 16 units per worker so the queue drains with
+// little imbalance at the end, but >= 4 sub-chunks per unit so per-unit
+// costs (pop, carry, pipeline ramp) stay small.
+int chunk_len(int64_t groups, int64_t seqlen, int workers, int tc) {
+    const int64_t max_chunks = (seqlen + tc - 1) / tc;
+    int64_t want = (16LL * workers + groups - 1) / groups;
+    int64_t lim = (max_chunks + 3) / 4;
+    if (lim < 1) lim = 1;
+    if (want > lim) want = lim;
+    if (want < 1) want = 1;
+    int64_t tu = (seqlen + want - 1) / want;
+    tu = (tu + tc - 1) / tc * tc;
+    return (int)tu;
+}
+
+struct Layout {
+    int64_t groups, chunks;
+    size_t queue_off, carry_off, bytes;
+};
+
+Layout layout(int64_t batch, int64_t dim, int64_t seqlen, int lanes, int tu) {
+    Layout l;
+    l.groups = n_groups(batch, dim, lanes);
+    l.chunks = (seqlen + tu - 1) / tu;
+    const int64_t queue = l.groups * (l.chunks - 1);
+    l.queue_off = 16;
+    l.carry_off = 16 + (size_t)((queue * 4 + 255) / 256 * 256);
+    l.bytes = l.carry_off + (size_t)(l.groups * 32 * states_per_lane(lanes)) * 4;
+    return l;
+}
+
+// Largest workspace any device can need: the smallest unit (4 sub-chunks).
+size_t bound_for(int64_t batch, int64_t dim, int64_t seqlen, int lanes, int act) {
+    const int tc = sub_chunk(lanes, act);
+    const int64_t max_chunks = ((seqlen + tc - 1) / tc + 3) / 4;
+    int64_t tu = (seqlen + max_chunks - 1) / max_chunks;
+    tu = (tu + tc - 1) / tc * tc;
+    return layout(batch, dim, seqlen, lanes, (int)tu).bytes;
+}
+
+}  // namespace
+
+bool persistent_supported(const ScanArgs &a) {
+    if (a.dstate > persist::kNS) return false;
+    const int es = a.act == kBF16 ? 2 : 4;
+    if (a.seqlen % (16 / es) != 0) return false;
+    auto al = [](const void *q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+    if (!(al(a.u) && al(a.delta) && al(a.z) && al(a.B) && al(a.C) && al(a.out))) return false;
+    const int64_t units = n_groups(a.batch, a.dim, 2) * ((a.seqlen + 15) / 16);
+    return units < ((int64_t)1 << 30);
+}
+
+// 0 if neither variant has enough channel groups to give every worker a
+// chain of its own (minus 10 %), else the preferred lanes per channel: two
+// (two workers per SM sub-partition) when the groups suffice, else one.
+int persistent_choose_lanes(const ScanArgs &a, int sm_count) {
+    for (int lanes : {2, 1}) {
+        const int64_t workers = (int64_t)sm_count * blocks_per_sm(lanes) * persist::kWarps;
+        if (n_groups(a.batch, a.dim, lanes) * 10 >= workers * 9) return lanes;
+    }
+    return 0;
+}
+
+bool persistent_preferred(const ScanArgs &a, int sm_count) {
+    return persistent_choose_lanes(a, sm_count) != 0;
+}
+
+size_t persistent_workspace_bound(int64_t batch, int64_t dim, int64_t seqlen, int act) {
+    const size_t b1 = bound_for(batch, dim, seqlen, 1, act);
+    const size_t b2 = bound_for(batch, dim, seqlen, 2, act);
+    return b1 > b2 ? b1 : b2;
+}
+
+cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, void *workspace,
+                                       size_t ws_bytes, int sm_count, cudaStream_t st) {
+    if (lanes == 0) lanes = persistent_choose_lanes(a, sm_count);
+    if (lanes == 0) lanes = 1;
+    if (lanes != 1 && lanes != 2) return cudaErrorInvalidValue;
+    const int per_sm = blocks_per_sm(lanes);
+    const int64_t workers = (int64_t)sm_count * per_sm * persist::kWarps;
+    const int64_t groups = n_groups(a.batch, a.dim, lanes);
+    const int tu = chunk_len(groups, a.seqlen, (int)workers, sub_chunk(lanes, a.act));
+    const Layout l = layout(a.batch, a.dim, a.seqlen, lanes, tu);
+    if (ws_bytes < l.bytes) return cudaErrorInvalidValue;
+
+    persist::Params kp;
+    kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
+    kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias;
+    kp.out = a.out; kp.last_state = a.last_state;
+    kp.dim = a.dim; kp.seqlen = a.seqlen; kp.dstate = a.dstate; kp.softplus = a.softplus;
+    kp.group_channels = group_channels(lanes);
+    kp.groups_per_batch = (int)((a.dim + kp.group_channels - 1) / kp.group_channels);
+    kp.n_groups = (int)l.groups;
+    kp.n_chunks = (int)l.chunks;
+    kp.chunk_len = tu;
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    kp.hdr = reinterpret_cast<unsigned *>(w);
+    kp.queue = reinterpret_cast<unsigned *>(w + l.queue_off);
+    kp.carry = reinterpret_cast<float *>(w + l.carry_off);
+    // counters and queue entries start at zero; carries are written before read
+    cudaError_t e = cudaMemsetAsync(w, 0, l.queue_off + (size_t)(l.groups * (l.chunks - 1)) * 4, st);
+    if (e != cudaSuccess) return e;
+
+    const int64_t units = l.groups * l.chunks;
+    int64_t grid = (int64_t)sm_count * per_sm;
+    const int64_t need = (units + persist::kWarps - 1) / persist::kWarps;
+    if (grid > need) grid = need;
+    return lanes == 2 ? launch_persistent_lanes2(kp, a.act, (int)grid, st)
+                      : launch_persistent_lanes1(kp, a.act, (int)grid, st);
+}
+
+}  // namespace mscan

@@ -38,31 +38,15 @@
 
 #include "device_math.cuh"
 #include "internal.h"
+#include "persistent_common.cuh"
+#include "persistent_kernels.h"
 
 namespace mscan {
 
 namespace {
 
-constexpr int kWarps = 4;            // workers per block (one per SM sub-partition)
-constexpr int kNS = 16;              // states held per thread (dstate <= 16)
-constexpr unsigned kSpinLimit = 1u << 22;  // bounded wait (~4M polls, >1 s with backoff)
-
-struct PParams {
-    const void *u, *delta, *B, *C, *z;
-    const float *A, *D, *delta_bias;
-    void *out;
-    float *last_state;
-    int64_t dim, seqlen;
-    int dstate;
-    int softplus;
-    int groups_per_batch;  // ceil(dim / 32)
-    int n_groups;          // batch * groups_per_batch
-    int n_chunks;          // chunks per group
-    int chunk_len;         // TU, a multiple of kTC
-    unsigned *hdr;         // workspace: [head, pushed, error, pad]
-    unsigned *queue;       // workspace: n_groups * (n_chunks - 1) slots
-    float *carry;          // workspace: n_groups * 32 * 16 floats
-};
+using namespace persist;
+using PParams = persist::Params;
 
 template <typename T>
 struct WarpSmem {
@@ -75,24 +59,6 @@ struct WarpSmem {
     static constexpr int OUTB = 32 * ROWB;                 // packed output tile
     static constexpr int BYTES = 2 * STAGE + BC32 + OUTB;
 };
-
-__device__ __forceinline__ void cp16(void *smem, const void *gmem, bool pred) {
-    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-                 :: "r"(s), "l"(gmem), "r"(pred ? 16 : 0) : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
-
-__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
-}
 
 template <typename T, bool SP, bool GATE>
 __global__ void __launch_bounds__(kWarps * 32, 1)
@@ -111,7 +77,6 @@ scan_fwd_persistent_kernel(const PParams p) {
 
     const int64_t L = p.seqlen, Dm = p.dim;
     const int N = p.dstate;
-    const int n_units = p.n_groups * p.n_chunks;
     const T *gu = static_cast<const T *>(p.u);
     const T *gd = static_cast<const T *>(p.delta);
     const T *gz = static_cast<const T *>(p.z);
@@ -125,28 +90,8 @@ scan_fwd_persistent_kernel(const PParams p) {
 #pragma unroll 1
     while (true) {
         // ---- take the next ready unit
-        unsigned unit = 0xffffffffu;
-        if (lane == 0) {
-            const unsigned s = atomicAdd(p.hdr + 0, 1u);
-            if ((int)s < n_units) {
-                if ((int)s < p.n_groups) {
-                    unit = s;  // chunk 0 of group s
-                } else {
-                    const unsigned *slot = p.queue + (s - p.n_groups);
-                    unsigned v = 0, spins = 0, ns = 32;
-                    while ((v = ld_acquire(slot)) == 0u) {
-                        if (++spins > kSpinLimit || ld_acquire(p.hdr + 2) != 0u) break;
-                        __nanosleep(ns);
-                        if (ns < 1024) ns <<= 1;
-                    }
-                    if (v == 0u) atomicOr(p.hdr + 2, 1u);
-                    unit = v == 0u ? 0xfffffffeu : v - 1u;
-                }
-            }
-        }
-        unit = __shfl_sync(0xffffffffu, unit, 0);
-        __syncwarp();  // order every lane's carry loads after lane 0's acquire
-        if (unit == 0xffffffffu || unit == 0xfffffffeu) break;
+        const unsigned unit = pop_unit(p, lane);
+        if (unit == kUnitDone || unit == kUnitAbort) break;
         const int g = (int)(unit % (unsigned)p.n_groups);
         const int j = (int)(unit / (unsigned)p.n_groups);
         const int64_t b = g / p.groups_per_batch;
@@ -250,25 +195,36 @@ scan_fwd_persistent_kernel(const PParams p) {
             unsigned char *ro = outt + lane * W::ROWB;
             const float *sBt = bc32;
             const float *sCt = bc32 + kTC * kNS;
-#pragma unroll 1
-            for (int tv = 0; tv < tvalid; tv += V) {
+            // Per-element values of one vector of V timesteps.  The vector
+            // loop is software-pipelined: the next vector's values (smem
+            // loads, softplus, gate) are computed while the current
+            // vector's states update.  Reads one vector past the sub-chunk
+            // land in the row padding and are never used; timesteps past
+            // the end have delta = 0 (Abar = 1, no input) and are not stored.
+            struct Pre { float dl[V], du[V], gg[V], sk[V]; };
+            auto pre = [&](int tv, Pre &P) {
                 float fu[V], fd[V], fz[V];
                 Elem<T>::unpack(*reinterpret_cast<const uint4 *>(ru + tv * sizeof(T)), fu);
                 Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rd + tv * sizeof(T)), fd);
                 if (GATE) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rz + tv * sizeof(T)), fz);
-                // per element, V independent chains: delta, delta*u, gate
-                float dl[V], du[V], gg[V];
 #pragma unroll
                 for (int e = 0; e < V; ++e) {
                     float x = fd[e] + bias;
                     if (SP) x = softplus_f(x);
-                    dl[e] = (tv + e < tvalid) ? x : 0.f;  // past the end: Abar = 1, no input
-                    du[e] = dl[e] * fu[e];
-                    gg[e] = GATE ? silu_f(fz[e]) : 1.f;
+                    P.dl[e] = (tv + e < tvalid) ? x : 0.f;
+                    P.du[e] = P.dl[e] * fu[e];
+                    P.gg[e] = GATE ? silu_f(fz[e]) : 1.f;
+                    P.sk[e] = Dd * fu[e];
                 }
+            };
+            Pre cur, nxt;
+            pre(0, cur);
+#pragma unroll 2
+            for (int tv = 0; tv < kTC; tv += V) {
+                pre(tv + V, nxt);
                 // states: state pairs outer, timesteps inner.  Per pair the
                 // recurrence is a short FFMA2 chain through the V timesteps;
-                // the exponentials depend only on dl and can all be issued
+                // the exponentials depend only on delta and can all be issued
                 // ahead; the V readout sums are independent accumulators.
                 float2 y2[V];
 #pragma unroll
@@ -280,8 +236,8 @@ scan_fwd_persistent_kernel(const PParams p) {
                         const int t = tv + e;
                         const float4 bb = *reinterpret_cast<const float4 *>(sBt + t * kNS + 4 * q);
                         const float4 cc = *reinterpret_cast<const float4 *>(sCt + t * kNS + 4 * q);
-                        const float2 dl2 = make_float2(dl[e], dl[e]);
-                        const float2 du2 = make_float2(du[e], du[e]);
+                        const float2 dl2 = make_float2(cur.dl[e], cur.dl[e]);
+                        const float2 du2 = make_float2(cur.du[e], cur.du[e]);
                         const float2 x0 = __fmul2_rn(dl2, A2[2 * q]);
                         const float2 x1 = __fmul2_rn(dl2, A2[2 * q + 1]);
                         const float2 a0 = make_float2(ex2_mufu(x0.x), ex2_mufu(x0.y));
@@ -294,13 +250,11 @@ scan_fwd_persistent_kernel(const PParams p) {
                         y2[e] = __ffma2_rn(make_float2(cc.z, cc.w), h[2 * q + 1], y2[e]);
                     }
                 }
-                float yv[V];
-#pragma unroll
-                for (int e = 0; e < V; ++e) yv[e] = y2[e].x + y2[e].y;
                 float fo[V];
 #pragma unroll
-                for (int e = 0; e < V; ++e) fo[e] = fmaf(Dd, fu[e], yv[e]) * gg[e];
+                for (int e = 0; e < V; ++e) fo[e] = (y2[e].x + y2[e].y + cur.sk[e]) * cur.gg[e];
                 *reinterpret_cast<uint4 *>(ro + tv * sizeof(T)) = Elem<T>::pack(fo);
+                cur = nxt;
             }
             __syncwarp();
             // coalesced store of the packed tile
@@ -320,12 +274,7 @@ scan_fwd_persistent_kernel(const PParams p) {
             for (int k = 0; k < kNS / 4; ++k)
                 __stcg(reinterpret_cast<float4 *>(carry) + k,
                        make_float4(h[2 * k].x, h[2 * k].y, h[2 * k + 1].x, h[2 * k + 1].y));
-            __syncwarp();
-            if (lane == 0) {
-                __threadfence();
-                const unsigned slot = atomicAdd(p.hdr + 1, 1u);
-                st_release(p.queue + slot, (unsigned)((j + 1) * p.n_groups + g) + 1u);
-            }
+            push_unit(p, lane, (unsigned)((j + 1) * p.n_groups + g));
         } else if (p.last_state != nullptr && dvalid) {
             float *ls = p.last_state + (b * Dm + d) * N;
 #pragma unroll
@@ -339,108 +288,33 @@ scan_fwd_persistent_kernel(const PParams p) {
 
 }  // namespace
 
-// Workspace bytes for a persistent launch over these sizes (0 if the
-// persistent kernel does not apply).
-size_t persistent_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen, int chunk_len) {
-    const int64_t gpb = (dim + 31) / 32;
-    const int64_t groups = batch * gpb;
-    const int64_t chunks = (seqlen + chunk_len - 1) / chunk_len;
-    const int64_t queue = groups * (chunks > 0 ? chunks - 1 : 0);
-    return 16 + (size_t)((queue * 4 + 255) / 256 * 256) + (size_t)(groups * 32 * kNS * 4);
-}
-
-// Upper bound of persistent_workspace_bytes over every device: the chunk
-// count never exceeds a quarter of the sub-chunk count (rounded up).
-size_t persistent_workspace_bound(int64_t batch, int64_t dim, int64_t seqlen, int act) {
-    const int kTC = act == kBF16 ? WarpSmem<__nv_bfloat16>::kTC : WarpSmem<float>::kTC;
-    const int64_t max_chunks = ((seqlen + kTC - 1) / kTC + 3) / 4;
-    const int64_t tu = ((seqlen + max_chunks - 1) / max_chunks + kTC - 1) / kTC * kTC;
-    return persistent_workspace_bytes(batch, dim, seqlen, (int)(tu < kTC ? kTC : tu)) +
-           (size_t)(batch * ((dim + 31) / 32)) * 4 + 256;
-}
-
-int persistent_chunk_len(int64_t batch, int64_t dim, int64_t seqlen, int sm_count, int act) {
-    const int kTC = act == kBF16 ? WarpSmem<__nv_bfloat16>::kTC : WarpSmem<float>::kTC;
-    // Aim for >= 16 units per worker so the drain at the end of the queue is
-    // short, but keep units >= 4 sub-chunks so per-unit costs stay small.
-    const int64_t groups = batch * ((dim + 31) / 32);
-    const int64_t workers = (int64_t)sm_count * kWarps;
-    const int64_t max_chunks = (seqlen + kTC - 1) / kTC;
-    int64_t want = (16 * workers + groups - 1) / groups;
-    int64_t lim = (max_chunks + 3) / 4;
-    if (lim < 1) lim = 1;
-    if (want > lim) want = lim;
-    if (want < 1) want = 1;
-    int64_t tu = (seqlen + want - 1) / want;
-    tu = (tu + kTC - 1) / kTC * kTC;
-    return (int)tu;
-}
-
-bool persistent_supported(const ScanArgs &a) {
-    if (a.dstate > kNS) return false;
-    const int es = a.act == kBF16 ? 2 : 4;
-    if (a.seqlen % (16 / es) != 0) return false;
-    auto al = [](const void *q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
-    if (!(al(a.u) && al(a.delta) && al(a.z) && al(a.B) && al(a.C) && al(a.out))) return false;
-    const int64_t groups = a.batch * ((a.dim + 31) / 32);
-    const int64_t chunks = (a.seqlen + (128 / es) - 1) / (128 / es);
-    return groups * chunks < (int64_t)1 << 30;
-}
-
-bool persistent_preferred(const ScanArgs &a, int sm_count) {
-    // Enough channel groups to give every worker a chain of its own (minus
-    // 10 %); with fewer, the static schedule splits each channel's states
-    // over several lanes and keeps more warps busy.
-    const int64_t groups = a.batch * ((a.dim + 31) / 32);
-    return groups * 10 >= (int64_t)sm_count * kWarps * 9;
-}
-
 template <typename T, bool SP, bool GATE>
-static cudaError_t launch_persistent_t(const PParams &kp, int sm_count, cudaStream_t st) {
+static cudaError_t launch_t(const persist::Params &kp, int grid, cudaStream_t st) {
     const int smem = kWarps * WarpSmem<T>::BYTES;
     auto kern = scan_fwd_persistent_kernel<T, SP, GATE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    int units = kp.n_groups * kp.n_chunks;
-    int grid = sm_count;
-    if (grid * kWarps > units) grid = (units + kWarps - 1) / kWarps;
     kern<<<grid, kWarps * 32, smem, st>>>(kp);
     return cudaGetLastError();
 }
 
-template <typename T>
-static cudaError_t launch_persistent_flags(const PParams &kp, int sm_count, cudaStream_t st) {
-    const bool gate = kp.z != nullptr;
-    if (kp.softplus)
-        return gate ? launch_persistent_t<T, true, true>(kp, sm_count, st)
-                    : launch_persistent_t<T, true, false>(kp, sm_count, st);
-    return gate ? launch_persistent_t<T, false, true>(kp, sm_count, st)
-                : launch_persistent_t<T, false, false>(kp, sm_count, st);
+int persistent_lanes1_sub_chunk(int act) {
+    return act == kBF16 ? WarpSmem<__nv_bfloat16>::kTC : WarpSmem<float>::kTC;
 }
 
-cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, void *workspace, size_t ws_bytes,
-                                       int sm_count, cudaStream_t st) {
-    PParams kp;
-    kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
-    kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias;
-    kp.out = a.out; kp.last_state = a.last_state;
-    kp.dim = a.dim; kp.seqlen = a.seqlen; kp.dstate = a.dstate; kp.softplus = a.softplus;
-    kp.groups_per_batch = (int)((a.dim + 31) / 32);
-    kp.n_groups = (int)(a.batch * kp.groups_per_batch);
-    kp.chunk_len = persistent_chunk_len(a.batch, a.dim, a.seqlen, sm_count, a.act);
-    kp.n_chunks = (int)((a.seqlen + kp.chunk_len - 1) / kp.chunk_len);
-    const size_t need = persistent_workspace_bytes(a.batch, a.dim, a.seqlen, kp.chunk_len);
-    if (ws_bytes < need) return cudaErrorInvalidValue;
-    unsigned char *w = static_cast<unsigned char *>(workspace);
-    const int64_t qn = (int64_t)kp.n_groups * (kp.n_chunks - 1);
-    kp.hdr = reinterpret_cast<unsigned *>(w);
-    kp.queue = reinterpret_cast<unsigned *>(w + 16);
-    kp.carry = reinterpret_cast<float *>(w + 16 + (qn * 4 + 255) / 256 * 256);
-    // header and queue start at zero; carries are always written before read
-    cudaError_t e = cudaMemsetAsync(w, 0, 16 + (size_t)qn * 4, st);
-    if (e != cudaSuccess) return e;
-    if (a.act == kBF16) return launch_persistent_flags<__nv_bfloat16>(kp, sm_count, st);
-    return launch_persistent_flags<float>(kp, sm_count, st);
+int persistent_lanes1_blocks_per_sm() { return 1; }
+
+cudaError_t launch_persistent_lanes1(const persist::Params &kp, int act, int grid, cudaStream_t st) {
+    const bool gate = kp.z != nullptr;
+    if (act == kBF16) {
+        if (kp.softplus) return gate ? launch_t<__nv_bfloat16, true, true>(kp, grid, st)
+                                     : launch_t<__nv_bfloat16, true, false>(kp, grid, st);
+        return gate ? launch_t<__nv_bfloat16, false, true>(kp, grid, st)
+                    : launch_t<__nv_bfloat16, false, false>(kp, grid, st);
+    }
+    if (kp.softplus) return gate ? launch_t<float, true, true>(kp, grid, st)
+                                 : launch_t<float, true, false>(kp, grid, st);
+    return gate ? launch_t<float, false, true>(kp, grid, st) : launch_t<float, false, false>(kp, grid, st);
 }
 
 }  // namespace mscan

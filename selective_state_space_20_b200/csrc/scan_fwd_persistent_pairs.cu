@@ -1,0 +1,344 @@
+// scan_fwd_persistent_pairs.cu -- persistent selective-scan (S6) forward
+// with each channel's states split over a pair of lanes.
+//
+// Same computation as scan_fwd_persistent.cu (softplus(delta + bias), the
+// zero-order-hold decay exp(delta A), the diagonal recurrence, C readout, D
+// skip, silu gate; "Mamba SSM concept and implementation in Keras and
+// TensorFlow", recurrent form and selective_scan / MambaBlock; fused as in
+// the Mamba paper, Appendix E.5).  Splitting the 16 states of a channel over
+// two lanes doubles the number of warps a problem provides -- e.g. 1280
+// instead of 640 for the Mamba-2.8B layer -- so every SM sub-partition runs
+// two workers and one hides the other's dependency stalls; with one warp per
+// sub-partition the MUFU idles whenever that warp is in a non-exp stretch.
+//
+// Per (16-channel group, time chunk) unit, per sub-chunk of TC timesteps:
+//   1. cp.async stages the raw u / delta / z rows and the B / C rows of the
+//      next sub-chunk (double buffer) while this one is processed;
+//   2. prologue: B and C are widened to fp32 as [t][n] rows for broadcast
+//      reads; every element's delta = softplus(delta_raw + bias), delta * u,
+//      silu(z) and D * u are computed once (lane = channel & timestep half)
+//      into shared float2 arrays;
+//   3. scan: lane (channel c, half r) advances states 8r .. 8r+7 through
+//      blocks of 8 timesteps (state pairs on FMUL2 / FFMA2, 16 ex2 per lane
+//      per 2 timesteps on the MUFU); the two halves' readouts are combined
+//      with one transposed shuffle round, leaving each lane 4 consecutive
+//      complete outputs, which it gates and packs into the output tile;
+//   4. the tile is written with coalesced 16-byte stores.
+// Shared arrays are padded so that every quarter-warp access is free of bank
+// conflicts.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "device_math.cuh"
+#include "internal.h"
+#include "persistent_common.cuh"
+#include "persistent_kernels.h"
+
+namespace mscan {
+namespace {
+
+using namespace persist;
+
+template <typename T>
+struct PairSmem {
+    static constexpr int kTC = 64 / (int)sizeof(T);        // timesteps per sub-chunk (64-byte rows)
+    static constexpr int V = 16 / (int)sizeof(T);          // elements per 16 bytes
+    static constexpr int CPR = kTC / V;                    // 16-byte chunks per raw row
+    static constexpr int CW = 16;                          // channels per unit
+    static constexpr int ROWB = kTC * (int)sizeof(T) + 16;  // raw / output row pitch (bytes)
+    static constexpr int RAW_ROWS = 3 * CW + 2 * kNS;      // u, delta, z rows, then B, C rows
+    static constexpr int STAGE = RAW_ROWS * ROWB;
+    static constexpr int BC32 = 2 * kTC * kNS * 4;          // fp32 B then C, [t][n]
+    static constexpr int PAIRB = kTC * 8 + 16;              // float2 row pitch (bytes)
+    static constexpr int DDU = CW * PAIRB;                  // (delta, delta * u) [c][t]
+    static constexpr int GSK = CW * PAIRB;                  // (silu(z), D * u) [c][t]
+    static constexpr int OUTB = CW * ROWB;                  // packed outputs [c][t]
+    static constexpr int BYTES = 2 * STAGE + BC32 + DDU + GSK + OUTB;
+};
+
+template <typename T>
+__device__ __forceinline__ void store4(unsigned char *dst, const float *o);
+template <>
+__device__ __forceinline__ void store4<float>(unsigned char *dst, const float *o) {
+    *reinterpret_cast<float4 *>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(unsigned char *dst, const float *o) {
+    *reinterpret_cast<uint2 *>(dst) =
+        make_uint2(Elem<__nv_bfloat16>::pack2(o[0], o[1]), Elem<__nv_bfloat16>::pack2(o[2], o[3]));
+}
+
+template <typename T, bool SP, bool GATE>
+__global__ void __launch_bounds__(kWarps * 32, 2)
+scan_fwd_pairs_kernel(const Params p) {
+    using W = PairSmem<T>;
+    constexpr int kTC = W::kTC, V = W::V, CPR = W::CPR, CW = W::CW;
+    constexpr int S = kNS / 2;  // states per lane
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    unsigned char *base = smem + warp * W::BYTES;
+    float *bc32 = reinterpret_cast<float *>(base + 2 * W::STAGE);
+    unsigned char *ddu = base + 2 * W::STAGE + W::BC32;
+    unsigned char *gsk = ddu + W::DDU;
+    unsigned char *outt = gsk + W::GSK;
+
+    const int64_t L = p.seqlen, Dm = p.dim;
+    const int N = p.dstate;
+    const T *gu = static_cast<const T *>(p.u);
+    const T *gd = static_cast<const T *>(p.delta);
+    const T *gz = static_cast<const T *>(p.z);
+    const T *gB = static_cast<const T *>(p.B);
+    const T *gC = static_cast<const T *>(p.C);
+    T *gout = static_cast<T *>(p.out);
+
+    const int sc = lane >> 1, sr = lane & 1;  // scan: channel, state half
+    const int pc = lane & 15, ph = lane >> 4;  // prologue: channel, timestep half
+
+    int cur_group = -1;
+    float2 A2[S / 2];
+    float bias_p = 0.f, D_p = 0.f;
+
+#pragma unroll 1
+    while (true) {
+        const unsigned unit = pop_unit(p, lane);
+        if (unit == kUnitDone || unit == kUnitAbort) break;
+        const int g = (int)(unit % (unsigned)p.n_groups);
+        const int j = (int)(unit / (unsigned)p.n_groups);
+        const int64_t b = g / p.groups_per_batch;
+        const int64_t d0 = (int64_t)(g % p.groups_per_batch) * CW;
+        const int nrows = (Dm - d0) < CW ? (int)(Dm - d0) : CW;
+        const int64_t ds = d0 + sc, dp = d0 + pc;
+
+        if (g != cur_group) {
+            cur_group = g;
+#pragma unroll
+            for (int k = 0; k < S / 2; ++k) {
+                const int n0 = S * sr + 2 * k, n1 = n0 + 1;
+                const float a0 = (ds < Dm && n0 < N) ? __ldg(p.A + ds * N + n0) : 0.f;
+                const float a1 = (ds < Dm && n1 < N) ? __ldg(p.A + ds * N + n1) : 0.f;
+                A2[k] = make_float2(a0 * kLog2e, a1 * kLog2e);
+            }
+            bias_p = (dp < Dm && p.delta_bias) ? __ldg(p.delta_bias + dp) : 0.f;
+            D_p = (dp < Dm && p.D) ? __ldg(p.D + dp) : 0.f;
+        }
+
+        float2 h[S / 2];
+        float *carry = p.carry + ((int64_t)g * 32 + lane) * S;
+        if (j == 0) {
+#pragma unroll
+            for (int k = 0; k < S / 2; ++k) h[k] = make_float2(0.f, 0.f);
+        } else {
+#pragma unroll
+            for (int k = 0; k < S / 4; ++k) {
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(carry) + k);
+                h[2 * k] = make_float2(v.x, v.y);
+                h[2 * k + 1] = make_float2(v.z, v.w);
+            }
+        }
+
+        const int64_t tb0 = (int64_t)j * p.chunk_len;
+        const int64_t tb1 = (tb0 + p.chunk_len) < L ? (tb0 + p.chunk_len) : L;
+        const int nsub = (int)((tb1 - tb0 + kTC - 1) / kTC);
+        const int64_t row0 = (b * Dm + d0) * L;
+        const int64_t bc0 = b * (int64_t)N * L;
+
+        auto issue = [&](int sub, int st) {
+            unsigned char *sb = base + st * W::STAGE;
+            const int64_t t0 = tb0 + (int64_t)sub * kTC;
+#pragma unroll
+            for (int i = lane; i < CW * CPR; i += 32) {
+                const int r = i / CPR, c = i % CPR;
+                const int64_t t = t0 + c * V;
+                const bool ok = (r < nrows) && (t < L);
+                const int64_t off = ok ? row0 + r * L + t : 0;
+                cp16(sb + (0 * CW + r) * W::ROWB + c * 16, gu + off, ok);
+                cp16(sb + (1 * CW + r) * W::ROWB + c * 16, gd + off, ok);
+                if (GATE) cp16(sb + (2 * CW + r) * W::ROWB + c * 16, gz + off, ok);
+            }
+#pragma unroll
+            for (int i = lane; i < 2 * kNS * CPR; i += 32) {
+                const int which = i / (kNS * CPR), rem = i % (kNS * CPR);
+                const int n = rem / CPR, c = rem % CPR;
+                const int64_t t = t0 + c * V;
+                const bool ok = (n < N) && (t < L);
+                const int64_t off = ok ? bc0 + (int64_t)n * L + t : 0;
+                cp16(sb + (3 * CW + which * kNS + n) * W::ROWB + c * 16, (which ? gC : gB) + off, ok);
+            }
+            cp_commit();
+        };
+
+        issue(0, 0);
+#pragma unroll 1
+        for (int sub = 0; sub < nsub; ++sub) {
+            const int st = sub & 1;
+            if (sub + 1 < nsub) {
+                issue(sub + 1, st ^ 1);
+                cp_wait<1>();
+            } else {
+                cp_wait<0>();
+            }
+            __syncwarp();
+            const unsigned char *sb = base + st * W::STAGE;
+            const int64_t t0 = tb0 + (int64_t)sub * kTC;
+            const int tvalid = (L - t0) < kTC ? (int)(L - t0) : kTC;
+
+            // ---- prologue (a): B and C to fp32 [t][n]; a quarter-warp covers
+            // 8 consecutive rows of one chunk
+#pragma unroll
+            for (int i = lane; i < 2 * kNS * CPR; i += 32) {
+                const int c = i / (2 * kNS), rr = i % (2 * kNS);
+                float f[V];
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sb + (3 * CW + rr) * W::ROWB + c * 16), f);
+                float *dst = bc32 + (rr / kNS) * kTC * kNS + (rr % kNS);
+#pragma unroll
+                for (int e = 0; e < V; ++e) dst[(c * V + e) * kNS] = f[e];
+            }
+            // ---- prologue (b): per element, once: (delta, delta*u), (gate, D*u)
+#pragma unroll
+            for (int v = 0; v < kTC / 2; v += V) {
+                const int tt = ph * (kTC / 2) + v;
+                float fu[V], fd[V], fz[V];
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sb + (0 * CW + pc) * W::ROWB + tt * sizeof(T)), fu);
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sb + (1 * CW + pc) * W::ROWB + tt * sizeof(T)), fd);
+                if (GATE)
+                    Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sb + (2 * CW + pc) * W::ROWB + tt * sizeof(T)), fz);
+                float4 *dd = reinterpret_cast<float4 *>(ddu + pc * W::PAIRB + tt * 8);
+                float4 *gs = reinterpret_cast<float4 *>(gsk + pc * W::PAIRB + tt * 8);
+#pragma unroll
+                for (int e = 0; e < V; e += 2) {
+                    float x0 = fd[e] + bias_p, x1 = fd[e + 1] + bias_p;
+                    if (SP) { x0 = softplus_f(x0); x1 = softplus_f(x1); }
+                    x0 = (tt + e < tvalid) ? x0 : 0.f;  // past the end: Abar = 1, no input
+                    x1 = (tt + e + 1 < tvalid) ? x1 : 0.f;
+                    dd[e / 2] = make_float4(x0, x0 * fu[e], x1, x1 * fu[e + 1]);
+                    gs[e / 2] = make_float4(GATE ? silu_f(fz[e]) : 1.f, D_p * fu[e],
+                                            GATE ? silu_f(fz[e + 1]) : 1.f, D_p * fu[e + 1]);
+                }
+            }
+            __syncwarp();
+
+            // ---- scan: lane (sc, sr), blocks of 8 timesteps
+            {
+                const unsigned char *drow = ddu + sc * W::PAIRB;
+                const unsigned char *grow = gsk + sc * W::PAIRB;
+                unsigned char *orow = outt + sc * W::ROWB;
+                const float *sB = bc32 + S * sr;
+                const float *sC = bc32 + kTC * kNS + S * sr;
+#pragma unroll 1
+                for (int tb = 0; tb < kTC; tb += 8) {
+                    float dl[8], du[8];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float4 v = *reinterpret_cast<const float4 *>(drow + (tb + 2 * k) * 8);
+                        dl[2 * k] = v.x; du[2 * k] = v.y; dl[2 * k + 1] = v.z; du[2 * k + 1] = v.w;
+                    }
+                    float2 y2[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y2[e] = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int q = 0; q < S / 4; ++q) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int t = tb + e;
+                            const float4 bb = *reinterpret_cast<const float4 *>(sB + t * kNS + 4 * q);
+                            const float4 cc = *reinterpret_cast<const float4 *>(sC + t * kNS + 4 * q);
+                            const float2 dl2 = make_float2(dl[e], dl[e]);
+                            const float2 du2 = make_float2(du[e], du[e]);
+                            const float2 x0 = __fmul2_rn(dl2, A2[2 * q]);
+                            const float2 x1 = __fmul2_rn(dl2, A2[2 * q + 1]);
+                            const float2 a0 = make_float2(ex2_mufu(x0.x), ex2_mufu(x0.y));
+                            const float2 a1 = make_float2(ex2_mufu(x1.x), ex2_mufu(x1.y));
+                            const float2 bu0 = __fmul2_rn(du2, make_float2(bb.x, bb.y));
+                            const float2 bu1 = __fmul2_rn(du2, make_float2(bb.z, bb.w));
+                            h[2 * q] = __ffma2_rn(a0, h[2 * q], bu0);
+                            h[2 * q + 1] = __ffma2_rn(a1, h[2 * q + 1], bu1);
+                            y2[e] = __ffma2_rn(make_float2(cc.x, cc.y), h[2 * q], y2[e]);
+                            y2[e] = __ffma2_rn(make_float2(cc.z, cc.w), h[2 * q + 1], y2[e]);
+                        }
+                    }
+                    // combine the two halves, transposed: lane sr ends with the
+                    // complete outputs of timesteps tb + 4 sr .. tb + 4 sr + 3
+                    float yv[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float lo = y2[i].x + y2[i].y, hi = y2[i + 4].x + y2[i + 4].y;
+                        const float send = sr ? lo : hi;
+                        const float keep = sr ? hi : lo;
+                        yv[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                    }
+                    const int te = tb + 4 * sr;
+                    const float4 g01 = *reinterpret_cast<const float4 *>(grow + te * 8);
+                    const float4 g23 = *reinterpret_cast<const float4 *>(grow + (te + 2) * 8);
+                    float o[4];
+                    o[0] = (yv[0] + g01.y) * g01.x;
+                    o[1] = (yv[1] + g01.w) * g01.z;
+                    o[2] = (yv[2] + g23.y) * g23.x;
+                    o[3] = (yv[3] + g23.w) * g23.z;
+                    store4<T>(orow + te * sizeof(T), o);
+                }
+            }
+            __syncwarp();
+            // ---- coalesced store of the output tile
+#pragma unroll
+            for (int i = lane; i < CW * CPR; i += 32) {
+                const int r = i / CPR, c = i % CPR;
+                const int64_t t = t0 + c * V;
+                if (r < nrows && t < L)
+                    stg16_stream(gout + row0 + r * L + t,
+                                 *reinterpret_cast<const uint4 *>(outt + r * W::ROWB + c * 16));
+            }
+            __syncwarp();
+        }
+
+        if (j + 1 < p.n_chunks) {
+#pragma unroll
+            for (int k = 0; k < S / 4; ++k)
+                __stcg(reinterpret_cast<float4 *>(carry) + k,
+                       make_float4(h[2 * k].x, h[2 * k].y, h[2 * k + 1].x, h[2 * k + 1].y));
+            push_unit(p, lane, (unsigned)((j + 1) * p.n_groups + g));
+        } else if (p.last_state != nullptr && ds < Dm) {
+            float *ls = p.last_state + (b * Dm + ds) * N;
+#pragma unroll
+            for (int k = 0; k < S / 2; ++k) {
+                const int n0 = S * sr + 2 * k;
+                if (n0 < N) ls[n0] = h[k].x;
+                if (n0 + 1 < N) ls[n0 + 1] = h[k].y;
+            }
+        }
+    }
+}
+
+template <typename T, bool SP, bool GATE>
+cudaError_t launch_t(const Params &kp, int grid, cudaStream_t st) {
+    const int smem = kWarps * PairSmem<T>::BYTES;
+    auto kern = scan_fwd_pairs_kernel<T, SP, GATE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kWarps * 32, smem, st>>>(kp);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int persistent_lanes2_sub_chunk(int act) {
+    return act == kBF16 ? PairSmem<__nv_bfloat16>::kTC : PairSmem<float>::kTC;
+}
+
+int persistent_lanes2_blocks_per_sm() { return 2; }
+
+cudaError_t launch_persistent_lanes2(const Params &kp, int act, int grid, cudaStream_t st) {
+    const bool gate = kp.z != nullptr;
+    if (act == kBF16) {
+        if (kp.softplus) return gate ? launch_t<__nv_bfloat16, true, true>(kp, grid, st)
+                                     : launch_t<__nv_bfloat16, true, false>(kp, grid, st);
+        return gate ? launch_t<__nv_bfloat16, false, true>(kp, grid, st)
+                    : launch_t<__nv_bfloat16, false, false>(kp, grid, st);
+    }
+    if (kp.softplus) return gate ? launch_t<float, true, true>(kp, grid, st)
+                                 : launch_t<float, true, false>(kp, grid, st);
+    return gate ? launch_t<float, false, true>(kp, grid, st) : launch_t<float, false, false>(kp, grid, st);
+}
+
+}  // namespace mscan

@@ -159,7 +159,8 @@ def test_auto_plan_is_valid():
 @pytest.mark.parametrize("shape", [(1, 32, 64), (2, 70, 336), (3, 33, 1000), (1, 1, 8),
                                    (4, 100, 2048), (2, 64, 4096)])
 @pytest.mark.parametrize("dstate", [16, 5])
-def test_persistent_schedule(dtype, shape, dstate):
+@pytest.mark.parametrize("lanes", [1, 2])
+def test_persistent_schedule(dtype, shape, dstate, lanes):
     b, d, L = shape
     w = inputs.custom(b, d, L, dstate, dtype, seed=b * 1000 + d + L + dstate)
     cpu = inputs.scan_inputs(w)
@@ -167,22 +168,23 @@ def test_persistent_schedule(dtype, shape, dstate):
     nbytes = binding.mamba_scan_workspace_size(b, d, L, dstate, inputs.DTYPES[dtype])
     assert nbytes > 0
     ws = torch.full((nbytes,), 0x5A, device="cuda", dtype=torch.uint8)  # garbage-filled
-    out, last = run_scan(ins, schedule=binding.SCHEDULE_PERSISTENT, workspace=ws)
+    out, last = run_scan(ins, schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=lanes, workspace=ws)
     assert binding.workspace_status(ws) == 0
     ro, rs = oracle_full(cpu)
     tol = TOL[inputs.DTYPES[dtype]]
     e1, e2 = rel_err(to_np(out), ro), rel_err(to_np(last), rs)
-    record(f"persistent {w.name}", out=e1, state=e2)
+    record(f"persistent lanes={lanes} {w.name}", out=e1, state=e2)
     assert e1 <= tol and e2 <= tol, (e1, e2)
     # same workspace again (state of the previous launch must not leak in)
-    out2, last2 = run_scan(ins, schedule=binding.SCHEDULE_PERSISTENT, workspace=ws)
+    out2, last2 = run_scan(ins, schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=lanes, workspace=ws)
     assert torch.equal(out, out2) and torch.equal(last, last2)
 
 
-def test_persistent_matches_static_schedule():
+@pytest.mark.parametrize("lanes", [1, 2])
+def test_persistent_matches_static_schedule(lanes):
     w = inputs.custom(4, 640, 1024, 16, "bf16", seed=31)
     ins = dev_inputs(inputs.scan_inputs(w))
-    o1, s1 = run_scan(ins, schedule=binding.SCHEDULE_PERSISTENT)
+    o1, s1 = run_scan(ins, schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=lanes)
     o2, s2 = run_scan(ins, schedule=binding.SCHEDULE_STATIC)
     assert rel_err(to_np(o1), to_np(o2)) <= 2e-2
     assert rel_err(to_np(s1), to_np(s2)) <= 1e-4
