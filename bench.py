@@ -195,75 +195,63 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 # ------------------------------------------------------------ oracle timing
-def time_oracle_sample(w, seconds: float, rank_seed: int = 0):
-    """Time the fp64 oracle (as it stands) on a bounded sample of the workload:
-    the first k channels of batch row 0 over the full sequence length, k sized
-    from a short calibration run for about `seconds` of CPU time."""
+def _oracle_run(data, cores):
     import oracle
-    cores = os.cpu_count() or 1
-    sub = inputs.custom(1, 64, w.seqlen, w.dstate, w.dtype, seed=w.seed + rank_seed,
-                        dt_min=w.dt_min, dt_max=w.dt_max, d_mode=w.d_mode)
-    cal = inputs.scan_inputs(sub)
-    t0 = time.perf_counter()
-    oracle.scan(cal["u"], cal["delta"], cal["A"], cal["B"], cal["C"], D=cal["D"], z=cal["z"],
-                delta_bias=cal["delta_bias"], nthreads=cores)
-    rate = 64 * w.seqlen / max(time.perf_counter() - t0, 1e-6)  # elements/s
-    k = int(max(cores, min(w.dim * w.batch, rate * seconds / w.seqlen)))
-    k = max(cores, (k // cores) * cores)
-    return k, rate
-
-
-def oracle_step(w, k, data=None):
-    import oracle
-    cores = os.cpu_count() or 1
-    if data is None:
-        sub = inputs.custom(1, k, w.seqlen, w.dstate, w.dtype, seed=w.seed, dt_min=w.dt_min,
-                            dt_max=w.dt_max, d_mode=w.d_mode)
-        data = inputs.scan_inputs(sub)
     t0 = time.perf_counter()
     oracle.scan(data["u"], data["delta"], data["A"], data["B"], data["C"], D=data["D"],
                 z=data["z"], delta_bias=data["delta_bias"], nthreads=cores)
-    return time.perf_counter() - t0, data
+    return time.perf_counter() - t0
 
 
-def cpu_baseline(w, seconds=12.0):
+def oracle_sample(w, seconds: float):
+    """A sub-problem of the workload sized for about `seconds` of oracle time
+    on this host's cores: every batch row, the first k channels, full L (the
+    whole workload when it fits).  Returns (inputs, k)."""
     cores = os.cpu_count() or 1
-    k, _ = time_oracle_sample(w, seconds)
-    dt, _ = oracle_step(w, k)
-    elems = k * w.seqlen
+    probe = max(cores * 4, 64)
+    cal = inputs.scan_inputs(dataclasses.replace(w, batch=1, dim=min(probe, w.dim)))
+    rate = min(probe, w.dim) * w.seqlen / max(_oracle_run(cal, cores), 1e-6)  # elements/s
+    k = int(rate * seconds / (w.batch * w.seqlen))
+    k = max(1, min(w.dim, k))
+    return inputs.scan_inputs(dataclasses.replace(w, dim=k)), k
+
+
+def cpu_baseline(w, seconds=25.0):
+    cores = os.cpu_count() or 1
+    data, k = oracle_sample(w, seconds)
+    dt = _oracle_run(data, cores)
+    elems = w.batch * k * w.seqlen
+    what = "the whole workload" if k == w.dim else f"all {w.batch} batch rows, first {k} of {w.dim} channels"
     return {"value": elems / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"batch row 0, first {k} of {w.dim} channels, full L={w.seqlen}, N={w.dstate}: "
-                      f"{elems} elements in {dt:.2f} s (fp64 C loop, {cores} threads)"}
+            "sample": f"{what}, full L={w.seqlen}, N={w.dstate}: {elems} elements in {dt:.2f} s "
+                      f"(fp64 C loop over {cores} threads)"}
 
 
 def run_reference(args, world, rank):
-    """The reference arm: the fp64 oracle, as it stands, on the host cores."""
+    """The reference arm: the fp64 oracle, as it stands, on the host cores.
+    Each step runs a bounded sample of the workload (every batch row, the
+    first k channels, full L) sized so the whole run takes a few minutes."""
     if rank != 0:
         return 0
     w = WORKLOAD
     cores = os.cpu_count() or 1
-    total_budget = 150.0
-    per_step = max(0.05, total_budget / max(1, args.steps + args.warmup))
-    k, _ = time_oracle_sample(w, per_step)
-    data = None
+    per_step = max(0.05, 150.0 / max(1, args.steps + args.warmup))
+    data, k = oracle_sample(w, per_step)
     for _ in range(args.warmup):
-        _, data = oracle_step(w, k, data)
-    times = []
-    for _ in range(args.steps):
-        dt, data = oracle_step(w, k, data)
-        times.append(dt)
+        _oracle_run(data, cores)
+    times = [_oracle_run(data, cores) for _ in range(args.steps)]
     tot = sum(times)
-    elems = k * w.seqlen * args.steps
+    elems = w.batch * k * w.seqlen * args.steps
     value = elems / tot / 1e9
+    sample = f"all {w.batch} batch rows, first {k} of {w.dim} channels, full L={w.seqlen}, N={w.dstate} per step"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "dim": w.dim, "seqlen": w.seqlen,
-                       "dstate": w.dstate, "act_dtype": w.dtype,
-                       "sample_per_step": f"batch row 0, first {k} channels, full L"},
+                       "dstate": w.dstate, "act_dtype": w.dtype, "sample_per_step": sample},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"{k} channels x L={w.seqlen} x N={w.dstate} per step"},
+                             "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)

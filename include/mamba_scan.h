@@ -81,7 +81,7 @@ typedef enum {
     MAMBA_SCHEDULE_PERSISTENT = 2  /* dstate <= 16: persistent warps take
                                       (channel group, time chunk) units from a
                                       ready queue and pass the state between
-                                      chunks through the workspace; one or two
+                                      chunks through the workspace; 1, 2 or 4
                                       lanes per channel */
 } mamba_schedule_t;
 
@@ -89,14 +89,17 @@ typedef enum {
  *   lanes_per_channel : threads sharing one channel's states.  Static
  *                       schedule: 1, 2, 4, 8 or 16 (the padded dstate must be
  *                       a multiple, and at most 16 states stay in one
- *                       thread).  Persistent schedule: 1 or 2.
+ *                       thread).  Persistent schedule: 1, 2 or 4.
  *   threads_per_block : static schedule only: 128 or 256
  *   schedule          : a mamba_schedule_t
+ *   chunk_timesteps   : persistent schedule only: timesteps per work unit
+ *                       (rounded up to the kernel's staging granularity)
  */
 typedef struct {
     int lanes_per_channel;
     int threads_per_block;
     int schedule;
+    int chunk_timesteps;
 } mamba_scan_tuning_t;
 
 /*

@@ -42,7 +42,7 @@ class MambaError(RuntimeError):
 
 class Tuning(ctypes.Structure):
     _fields_ = [("lanes_per_channel", ctypes.c_int), ("threads_per_block", ctypes.c_int),
-                ("schedule", ctypes.c_int)]
+                ("schedule", ctypes.c_int), ("chunk_timesteps", ctypes.c_int)]
 
 
 _lock = threading.Lock()
@@ -134,7 +134,7 @@ def mamba_scan_fwd(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
                    last_state: Optional[torch.Tensor] = None,
                    return_last_state: bool = False, lanes_per_channel: int = 0,
                    threads_per_block: int = 0, schedule: int = SCHEDULE_AUTO,
-                   workspace: Optional[torch.Tensor] = None):
+                   workspace: Optional[torch.Tensor] = None, chunk_timesteps: int = 0):
     """Selective scan forward on the current CUDA stream.
 
     u, delta, z: (batch, dim, L); B, C: (batch, N, L) -- all one dtype,
@@ -184,7 +184,8 @@ def mamba_scan_fwd(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
     args = [_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
             _ptr(delta_bias), int(bool(delta_softplus)), _ptr(out), _ptr(last_state),
             batch, dim, L, N, _ACT[act]]
-    tun = Tuning(int(lanes_per_channel), int(threads_per_block), int(schedule))
+    tun = Tuning(int(lanes_per_channel), int(threads_per_block), int(schedule),
+                 int(chunk_timesteps))
     with torch.cuda.device(dev):
         rc = lib.mamba_scan_fwd_ws(*args, ctypes.byref(tun), _ptr(workspace), ws_bytes,
                                    _stream(dev))

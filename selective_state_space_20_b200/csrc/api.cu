@@ -4,7 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/mamba_scan.h"
+#include "mamba_scan.h"
 #include "internal.h"
 
 namespace {
@@ -91,11 +91,13 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
                 if (overlaps(workspace, ws_bytes, ins[i], sz[i])) return MAMBA_ERR_OVERLAP;
         }
     }
-    int want_lanes = 0, want_threads = 0, want_sched = MAMBA_SCHEDULE_AUTO;
+    int want_lanes = 0, want_threads = 0, want_sched = MAMBA_SCHEDULE_AUTO, want_chunk = 0;
     if (tuning) {
         want_lanes = tuning->lanes_per_channel;
         want_threads = tuning->threads_per_block;
         want_sched = tuning->schedule;
+        want_chunk = tuning->chunk_timesteps;
+        if (want_chunk < 0) return MAMBA_ERR_UNSUPPORTED;
         if (want_lanes != 0 && want_lanes != 1 && want_lanes != 2 && want_lanes != 4 &&
             want_lanes != 8 && want_lanes != 16)
             return MAMBA_ERR_UNSUPPORTED;
@@ -123,7 +125,8 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
     bool persist = false;
     int persist_lanes = 0;
     if (want_sched == MAMBA_SCHEDULE_PERSISTENT) {
-        if (!supported || want_threads != 0 || (want_lanes != 0 && want_lanes != 1 && want_lanes != 2))
+        if (!supported || want_threads != 0 ||
+            (want_lanes != 0 && want_lanes != 1 && want_lanes != 2 && want_lanes != 4))
             return MAMBA_ERR_UNSUPPORTED;
         if (!ws_ok) return MAMBA_ERR_WORKSPACE;
         persist = true;
@@ -138,10 +141,11 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
             plan_out->lanes_per_channel = persist_lanes;
             plan_out->threads_per_block = 128;
             plan_out->schedule = MAMBA_SCHEDULE_PERSISTENT;
+            plan_out->chunk_timesteps = want_chunk;
         }
         if (!launch) return MAMBA_OK;
-        return mscan::launch_scan_fwd_persistent(a, persist_lanes, workspace, ws_bytes, sms,
-                                                 stream) == cudaSuccess
+        return mscan::launch_scan_fwd_persistent(a, persist_lanes, want_chunk, workspace, ws_bytes,
+                                                 sms, stream) == cudaSuccess
                    ? MAMBA_OK : MAMBA_ERR_CUDA;
     }
     mscan::ScanPlan pl;
@@ -150,6 +154,7 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
         plan_out->lanes_per_channel = pl.lanes;
         plan_out->threads_per_block = pl.threads;
         plan_out->schedule = MAMBA_SCHEDULE_STATIC;
+        plan_out->chunk_timesteps = 0;
     }
     if (!launch) return MAMBA_OK;
     return mscan::launch_scan_fwd(a, pl, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;

@@ -57,7 +57,8 @@ bool persistent_supported(const ScanArgs &a);
 bool persistent_preferred(const ScanArgs &a, int sm_count);
 int persistent_choose_lanes(const ScanArgs &a, int sm_count);  // 0 = not preferred
 size_t persistent_workspace_bound(int64_t batch, int64_t dim, int64_t seqlen, int act);
-cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, void *workspace,
-                                       size_t ws_bytes, int sm_count, cudaStream_t stream);
+cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_timesteps,
+                                       void *workspace, size_t ws_bytes, int sm_count,
+                                       cudaStream_t stream);
 
 }  // namespace mscan

@@ -11,25 +11,26 @@ namespace mscan {
 
 namespace {
 
-int group_channels(int lanes) { return lanes == 2 ? 16 : 32; }
-int states_per_lane(int lanes) { return lanes == 2 ? 8 : 16; }
+int group_channels(int lanes) { return 32 / lanes; }
+int states_per_lane(int lanes) { return persist::kNS / lanes; }
 int sub_chunk(int lanes, int act) {
-    return lanes == 2 ? persistent_lanes2_sub_chunk(act) : persistent_lanes1_sub_chunk(act);
+    return lanes == 1 ? persistent_lanes1_sub_chunk(act) : persistent_split_sub_chunk(lanes, act);
 }
 int blocks_per_sm(int lanes) {
-    return lanes == 2 ? persistent_lanes2_blocks_per_sm() : persistent_lanes1_blocks_per_sm();
+    return lanes == 1 ? persistent_lanes1_blocks_per_sm() : persistent_split_blocks_per_sm(lanes);
 }
 int64_t n_groups(int64_t batch, int64_t dim, int lanes) {
     const int cw = group_channels(lanes);
     return batch * ((dim + cw - 1) / cw);
 }
 
-// Timesteps per work unit: >= 16 units per worker so the queue drains with
-// little imbalance at the end, but >= 4 sub-chunks per unit so per-unit
-// costs (pop, carry, pipeline ramp) stay small.
+// Timesteps per work unit: about 4 units per worker (measured best on B200
+// for the Mamba layer shapes: shorter units pay more per-unit costs -- pop,
+// carry, pipeline ramp -- longer ones leave a longer drain at the end), and
+// never fewer than 4 sub-chunks per unit.
 int chunk_len(int64_t groups, int64_t seqlen, int workers, int tc) {
     const int64_t max_chunks = (seqlen + tc - 1) / tc;
-    int64_t want = (16LL * workers + groups - 1) / groups;
+    int64_t want = (4LL * workers + groups - 1) / groups;
     int64_t lim = (max_chunks + 3) / 4;
     if (lim < 1) lim = 1;
     if (want > lim) want = lim;
@@ -72,18 +73,21 @@ bool persistent_supported(const ScanArgs &a) {
     if (a.seqlen % (16 / es) != 0) return false;
     auto al = [](const void *q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
     if (!(al(a.u) && al(a.delta) && al(a.z) && al(a.B) && al(a.C) && al(a.out))) return false;
-    const int64_t units = n_groups(a.batch, a.dim, 2) * ((a.seqlen + 15) / 16);
+    const int64_t units = n_groups(a.batch, a.dim, 4) * ((a.seqlen + 15) / 16);
     return units < ((int64_t)1 << 30);
 }
 
-// 0 if neither variant has enough channel groups to give every worker a
-// chain of its own (minus 10 %), else the preferred lanes per channel: two
-// (two workers per SM sub-partition) when the groups suffice, else one.
+// Preferred lanes per channel, or 0 when the static schedule should run.
+// Measured on B200 (Mamba layer shapes, N = 16): two lanes per channel is
+// fastest when its channel groups give every worker (2 blocks x 4 warps per
+// SM) a chain of its own, minus 10 %; with fewer groups, four lanes (3 blocks
+// per SM) as long as three quarters of its workers are busy; below that the
+// static schedule, which splits states further, keeps more warps busy.
 int persistent_choose_lanes(const ScanArgs &a, int sm_count) {
-    for (int lanes : {2, 1}) {
-        const int64_t workers = (int64_t)sm_count * blocks_per_sm(lanes) * persist::kWarps;
-        if (n_groups(a.batch, a.dim, lanes) * 10 >= workers * 9) return lanes;
-    }
+    const int64_t w2 = (int64_t)sm_count * blocks_per_sm(2) * persist::kWarps;
+    if (n_groups(a.batch, a.dim, 2) * 10 >= w2 * 9) return 2;
+    const int64_t w4 = (int64_t)sm_count * blocks_per_sm(4) * persist::kWarps;
+    if (n_groups(a.batch, a.dim, 4) * 4 >= w4 * 3) return 4;
     return 0;
 }
 
@@ -92,20 +96,34 @@ bool persistent_preferred(const ScanArgs &a, int sm_count) {
 }
 
 size_t persistent_workspace_bound(int64_t batch, int64_t dim, int64_t seqlen, int act) {
-    const size_t b1 = bound_for(batch, dim, seqlen, 1, act);
-    const size_t b2 = bound_for(batch, dim, seqlen, 2, act);
-    return b1 > b2 ? b1 : b2;
+    size_t m = 0;
+    for (int lanes : {1, 2, 4}) {
+        const size_t b = bound_for(batch, dim, seqlen, lanes, act);
+        if (b > m) m = b;
+    }
+    return m;
 }
 
-cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, void *workspace,
-                                       size_t ws_bytes, int sm_count, cudaStream_t st) {
+cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_timesteps,
+                                       void *workspace, size_t ws_bytes, int sm_count,
+                                       cudaStream_t st) {
     if (lanes == 0) lanes = persistent_choose_lanes(a, sm_count);
     if (lanes == 0) lanes = 1;
-    if (lanes != 1 && lanes != 2) return cudaErrorInvalidValue;
+    if (lanes != 1 && lanes != 2 && lanes != 4) return cudaErrorInvalidValue;
     const int per_sm = blocks_per_sm(lanes);
     const int64_t workers = (int64_t)sm_count * per_sm * persist::kWarps;
     const int64_t groups = n_groups(a.batch, a.dim, lanes);
-    const int tu = chunk_len(groups, a.seqlen, (int)workers, sub_chunk(lanes, a.act));
+    const int tc = sub_chunk(lanes, a.act);
+    int tu = chunk_len(groups, a.seqlen, (int)workers, tc);
+    if (chunk_timesteps > 0) {
+        // explicit unit length, but never shorter than the bound's units
+        // (4 sub-chunks or the whole sequence)
+        int64_t want = ((int64_t)chunk_timesteps + tc - 1) / tc * tc;
+        const int64_t min_tu = 4LL * tc < a.seqlen ? 4LL * tc : (a.seqlen + tc - 1) / tc * tc;
+        if (want < min_tu) want = min_tu;
+        if (want > a.seqlen) want = (a.seqlen + tc - 1) / tc * tc;
+        tu = (int)want;
+    }
     const Layout l = layout(a.batch, a.dim, a.seqlen, lanes, tu);
     if (ws_bytes < l.bytes) return cudaErrorInvalidValue;
 
@@ -131,8 +149,8 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, void *works
     int64_t grid = (int64_t)sm_count * per_sm;
     const int64_t need = (units + persist::kWarps - 1) / persist::kWarps;
     if (grid > need) grid = need;
-    return lanes == 2 ? launch_persistent_lanes2(kp, a.act, (int)grid, st)
-                      : launch_persistent_lanes1(kp, a.act, (int)grid, st);
+    return lanes == 1 ? launch_persistent_lanes1(kp, a.act, (int)grid, st)
+                      : launch_persistent_split(kp, lanes, a.act, (int)grid, st);
 }
 
 }  // namespace mscan

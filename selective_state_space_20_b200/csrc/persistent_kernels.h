@@ -13,9 +13,10 @@ int persistent_lanes1_sub_chunk(int act);
 int persistent_lanes1_blocks_per_sm();
 cudaError_t launch_persistent_lanes1(const persist::Params &kp, int act, int grid, cudaStream_t st);
 
-// Two lanes per channel, half of the states each; units of 16 channels.
-int persistent_lanes2_sub_chunk(int act);
-int persistent_lanes2_blocks_per_sm();
-cudaError_t launch_persistent_lanes2(const persist::Params &kp, int act, int grid, cudaStream_t st);
+// R = 2 or 4 lanes per channel, 16 / R states each; units of 32 / R channels.
+int persistent_split_sub_chunk(int lanes, int act);
+int persistent_split_blocks_per_sm(int lanes);
+cudaError_t launch_persistent_split(const persist::Params &kp, int lanes, int act, int grid,
+                                   cudaStream_t st);
 
 }  // namespace mscan

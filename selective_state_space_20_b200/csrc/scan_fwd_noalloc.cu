@@ -23,7 +23,7 @@
 
 #include <mutex>
 
-#include "../../include/mamba_scan.h"
+#include "mamba_scan.h"
 
 namespace {
 

@@ -208,13 +208,18 @@ scan_fwd_persistent_kernel(const PParams p) {
                 Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rd + tv * sizeof(T)), fd);
                 if (GATE) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rz + tv * sizeof(T)), fz);
 #pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    float x = fd[e] + bias;
-                    if (SP) x = softplus_f(x);
-                    P.dl[e] = (tv + e < tvalid) ? x : 0.f;
-                    P.du[e] = P.dl[e] * fu[e];
-                    P.gg[e] = GATE ? silu_f(fz[e]) : 1.f;
-                    P.sk[e] = Dd * fu[e];
+                for (int e = 0; e < V; e += 2) {  // element pairs on the packed x2 instructions
+                    float2 x = __fadd2_rn(f2(fd[e], fd[e + 1]), f2(bias, bias));
+                    if (SP) x = softplus2_f(x);
+                    P.dl[e] = (tv + e < tvalid) ? x.x : 0.f;
+                    P.dl[e + 1] = (tv + e + 1 < tvalid) ? x.y : 0.f;
+                    const float2 uu = f2(fu[e], fu[e + 1]);
+                    const float2 xu = __fmul2_rn(f2(P.dl[e], P.dl[e + 1]), uu);
+                    P.du[e] = xu.x; P.du[e + 1] = xu.y;
+                    const float2 gg = GATE ? silu2_f(f2(fz[e], fz[e + 1])) : f2(1.f, 1.f);
+                    P.gg[e] = gg.x; P.gg[e + 1] = gg.y;
+                    const float2 sk = __fmul2_rn(f2(Dd, Dd), uu);
+                    P.sk[e] = sk.x; P.sk[e + 1] = sk.y;
                 }
             };
             Pre cur, nxt;
@@ -257,6 +262,15 @@ scan_fwd_persistent_kernel(const PParams p) {
                 cur = nxt;
             }
             __syncwarp();
+            // the last sub-chunk's state is final: publish the successor unit
+            // before this tile's stores, so the release waits on less
+            if (sub + 1 == nsub && j + 1 < p.n_chunks) {
+#pragma unroll
+                for (int k = 0; k < kNS / 4; ++k)
+                    __stcg(reinterpret_cast<float4 *>(carry) + k,
+                           make_float4(h[2 * k].x, h[2 * k].y, h[2 * k + 1].x, h[2 * k + 1].y));
+                push_unit(p, lane, (unsigned)((j + 1) * p.n_groups + g));
+            }
             // coalesced store of the packed tile
 #pragma unroll
             for (int i = lane; i < 32 * CPR; i += 32) {
@@ -269,13 +283,7 @@ scan_fwd_persistent_kernel(const PParams p) {
             __syncwarp();
         }
 
-        if (j + 1 < p.n_chunks) {
-#pragma unroll
-            for (int k = 0; k < kNS / 4; ++k)
-                __stcg(reinterpret_cast<float4 *>(carry) + k,
-                       make_float4(h[2 * k].x, h[2 * k].y, h[2 * k + 1].x, h[2 * k + 1].y));
-            push_unit(p, lane, (unsigned)((j + 1) * p.n_groups + g));
-        } else if (p.last_state != nullptr && dvalid) {
+        if (j + 1 == p.n_chunks && p.last_state != nullptr && dvalid) {
             float *ls = p.last_state + (b * Dm + d) * N;
 #pragma unroll
             for (int k = 0; k < kNS / 2; ++k) {

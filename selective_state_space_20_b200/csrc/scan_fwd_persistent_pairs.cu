@@ -40,21 +40,20 @@ namespace {
 
 using namespace persist;
 
-template <typename T>
+template <typename T, int R>
 struct PairSmem {
     static constexpr int kTC = 64 / (int)sizeof(T);        // timesteps per sub-chunk (64-byte rows)
     static constexpr int V = 16 / (int)sizeof(T);          // elements per 16 bytes
     static constexpr int CPR = kTC / V;                    // 16-byte chunks per raw row
-    static constexpr int CW = 16;                          // channels per unit
+    static constexpr int CW = 32 / R;                      // channels per unit
     static constexpr int ROWB = kTC * (int)sizeof(T) + 16;  // raw / output row pitch (bytes)
     static constexpr int RAW_ROWS = 3 * CW + 2 * kNS;      // u, delta, z rows, then B, C rows
     static constexpr int STAGE = RAW_ROWS * ROWB;
     static constexpr int BC32 = 2 * kTC * kNS * 4;          // fp32 B then C, [t][n]
-    static constexpr int PAIRB = kTC * 8 + 16;              // float2 row pitch (bytes)
-    static constexpr int DDU = CW * PAIRB;                  // (delta, delta * u) [c][t]
-    static constexpr int GSK = CW * PAIRB;                  // (silu(z), D * u) [c][t]
+    static constexpr int QUADB = kTC * 16 + 16;             // float4 row pitch (bytes)
+    static constexpr int DDU = CW * QUADB;                  // (delta, delta, delta*u, delta*u) [c][t]
     static constexpr int OUTB = CW * ROWB;                  // packed outputs [c][t]
-    static constexpr int BYTES = 2 * STAGE + BC32 + DDU + GSK + OUTB;
+    static constexpr int BYTES = 2 * STAGE + BC32 + DDU + OUTB;
 };
 
 template <typename T>
@@ -68,21 +67,83 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(unsigned char *dst, const 
     *reinterpret_cast<uint2 *>(dst) =
         make_uint2(Elem<__nv_bfloat16>::pack2(o[0], o[1]), Elem<__nv_bfloat16>::pack2(o[2], o[3]));
 }
+template <typename T>
+__device__ __forceinline__ void store2(unsigned char *dst, const float *o);
+template <>
+__device__ __forceinline__ void store2<float>(unsigned char *dst, const float *o) {
+    *reinterpret_cast<float2 *>(dst) = make_float2(o[0], o[1]);
+}
+template <>
+__device__ __forceinline__ void store2<__nv_bfloat16>(unsigned char *dst, const float *o) {
+    *reinterpret_cast<uint32_t *>(dst) = Elem<__nv_bfloat16>::pack2(o[0], o[1]);
+}
 
-template <typename T, bool SP, bool GATE>
-__global__ void __launch_bounds__(kWarps * 32, 2)
+// OWN (2 or 4) consecutive activations from shared memory, widened to fp32.
+template <typename T, int OWN>
+__device__ __forceinline__ void load_small(const unsigned char *src, float *f);
+template <>
+__device__ __forceinline__ void load_small<float, 4>(const unsigned char *src, float *f) {
+    const float4 v = *reinterpret_cast<const float4 *>(src);
+    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void load_small<float, 2>(const unsigned char *src, float *f) {
+    const float2 v = *reinterpret_cast<const float2 *>(src);
+    f[0] = v.x; f[1] = v.y;
+}
+template <>
+__device__ __forceinline__ void load_small<__nv_bfloat16, 4>(const unsigned char *src, float *f) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(src);
+    Elem<__nv_bfloat16>::unpack2(v.x, f[0], f[1]);
+    Elem<__nv_bfloat16>::unpack2(v.y, f[2], f[3]);
+}
+template <>
+__device__ __forceinline__ void load_small<__nv_bfloat16, 2>(const unsigned char *src, float *f) {
+    Elem<__nv_bfloat16>::unpack2(*reinterpret_cast<const uint32_t *>(src), f[0], f[1]);
+}
+
+// Sum the 8 per-timestep partial readouts of a block over the R lanes of a
+// channel, transposed: afterwards lane r holds the complete outputs of
+// timesteps r * 8/R .. r * 8/R + 8/R - 1 in v[0 ..].  Round K halves the live
+// values: the lane with bit K set keeps the upper half, sends the lower.
+template <int K, int CNT>
+struct LaneReduce {
+    __device__ __forceinline__ static void run(float (&v)[8], int r) {
+        constexpr int HALF = CNT / 2;
+        const bool upper = (r & K) != 0;
+#pragma unroll
+        for (int i = 0; i < HALF; ++i) {
+            const float send = upper ? v[i] : v[i + HALF];
+            const float keep = upper ? v[i + HALF] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, K);
+        }
+        LaneReduce<K / 2, HALF>::run(v, r);
+    }
+};
+template <int CNT>
+struct LaneReduce<0, CNT> {
+    __device__ __forceinline__ static void run(float (&)[8], int) {}
+};
+
+template <int R> struct LanesOccupancy;
+template <> struct LanesOccupancy<2> { static constexpr int kBlocks = 2; };
+template <> struct LanesOccupancy<4> { static constexpr int kBlocks = 3; };
+
+template <typename T, int R, bool SP, bool GATE>
+__global__ void __launch_bounds__(kWarps * 32, LanesOccupancy<R>::kBlocks)
 scan_fwd_pairs_kernel(const Params p) {
-    using W = PairSmem<T>;
+    using W = PairSmem<T, R>;
     constexpr int kTC = W::kTC, V = W::V, CPR = W::CPR, CW = W::CW;
-    constexpr int S = kNS / 2;  // states per lane
+    constexpr int S = kNS / R;   // states per lane
+    constexpr int OWN = 8 / R;   // outputs per lane per block of 8 timesteps
+    constexpr int PT = kTC / R;  // prologue timesteps per lane
     extern __shared__ __align__(16) unsigned char smem[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     unsigned char *base = smem + warp * W::BYTES;
     float *bc32 = reinterpret_cast<float *>(base + 2 * W::STAGE);
     unsigned char *ddu = base + 2 * W::STAGE + W::BC32;
-    unsigned char *gsk = ddu + W::DDU;
-    unsigned char *outt = gsk + W::GSK;
+    unsigned char *outt = ddu + W::DDU;
 
     const int64_t L = p.seqlen, Dm = p.dim;
     const int N = p.dstate;
@@ -93,12 +154,12 @@ scan_fwd_pairs_kernel(const Params p) {
     const T *gC = static_cast<const T *>(p.C);
     T *gout = static_cast<T *>(p.out);
 
-    const int sc = lane >> 1, sr = lane & 1;  // scan: channel, state half
-    const int pc = lane & 15, ph = lane >> 4;  // prologue: channel, timestep half
+    const int sc = lane / R, sr = lane % R;    // scan: channel, state slice
+    const int pc = lane % CW, ph = lane / CW;  // prologue: channel, timestep slice
 
     int cur_group = -1;
     float2 A2[S / 2];
-    float bias_p = 0.f, D_p = 0.f;
+    float bias_p = 0.f, D_s = 0.f;
 
 #pragma unroll 1
     while (true) {
@@ -121,7 +182,7 @@ scan_fwd_pairs_kernel(const Params p) {
                 A2[k] = make_float2(a0 * kLog2e, a1 * kLog2e);
             }
             bias_p = (dp < Dm && p.delta_bias) ? __ldg(p.delta_bias + dp) : 0.f;
-            D_p = (dp < Dm && p.D) ? __ldg(p.D + dp) : 0.f;
+            D_s = (ds < Dm && p.D) ? __ldg(p.D + ds) : 0.f;
         }
 
         float2 h[S / 2];
@@ -132,7 +193,7 @@ scan_fwd_pairs_kernel(const Params p) {
         } else {
 #pragma unroll
             for (int k = 0; k < S / 4; ++k) {
-                const float4 v = __ldcg(reinterpret_cast<const float4 *>(carry) + k);
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(carry) + k);  // S/4 float4
                 h[2 * k] = make_float2(v.x, v.y);
                 h[2 * k + 1] = make_float2(v.z, v.w);
             }
@@ -195,45 +256,43 @@ scan_fwd_pairs_kernel(const Params p) {
 #pragma unroll
                 for (int e = 0; e < V; ++e) dst[(c * V + e) * kNS] = f[e];
             }
-            // ---- prologue (b): per element, once: (delta, delta*u), (gate, D*u)
+            // ---- prologue (b): per element, once: delta and delta*u, stored
+            // duplicated as (delta, delta, delta*u, delta*u) so the scan reads
+            // both packed operand pairs with one 16-byte load
 #pragma unroll
-            for (int v = 0; v < kTC / 2; v += V) {
-                const int tt = ph * (kTC / 2) + v;
-                float fu[V], fd[V], fz[V];
+            for (int v = 0; v < PT; v += V) {
+                const int tt = ph * PT + v;
+                float fu[V], fd[V];
                 Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sb + (0 * CW + pc) * W::ROWB + tt * sizeof(T)), fu);
                 Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sb + (1 * CW + pc) * W::ROWB + tt * sizeof(T)), fd);
-                if (GATE)
-                    Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sb + (2 * CW + pc) * W::ROWB + tt * sizeof(T)), fz);
-                float4 *dd = reinterpret_cast<float4 *>(ddu + pc * W::PAIRB + tt * 8);
-                float4 *gs = reinterpret_cast<float4 *>(gsk + pc * W::PAIRB + tt * 8);
+                float4 *dd = reinterpret_cast<float4 *>(ddu + pc * W::QUADB + tt * 16);
 #pragma unroll
-                for (int e = 0; e < V; e += 2) {
-                    float x0 = fd[e] + bias_p, x1 = fd[e + 1] + bias_p;
-                    if (SP) { x0 = softplus_f(x0); x1 = softplus_f(x1); }
-                    x0 = (tt + e < tvalid) ? x0 : 0.f;  // past the end: Abar = 1, no input
-                    x1 = (tt + e + 1 < tvalid) ? x1 : 0.f;
-                    dd[e / 2] = make_float4(x0, x0 * fu[e], x1, x1 * fu[e + 1]);
-                    gs[e / 2] = make_float4(GATE ? silu_f(fz[e]) : 1.f, D_p * fu[e],
-                                            GATE ? silu_f(fz[e + 1]) : 1.f, D_p * fu[e + 1]);
+                for (int e = 0; e < V; e += 2) {  // element pairs on the packed x2 instructions
+                    float2 x = __fadd2_rn(f2(fd[e], fd[e + 1]), f2(bias_p, bias_p));
+                    if (SP) x = softplus2_f(x);
+                    x.x = (tt + e < tvalid) ? x.x : 0.f;  // past the end: Abar = 1, no input
+                    x.y = (tt + e + 1 < tvalid) ? x.y : 0.f;
+                    const float2 xu = __fmul2_rn(x, f2(fu[e], fu[e + 1]));
+                    dd[e] = make_float4(x.x, x.x, xu.x, xu.x);
+                    dd[e + 1] = make_float4(x.y, x.y, xu.y, xu.y);
                 }
             }
             __syncwarp();
 
             // ---- scan: lane (sc, sr), blocks of 8 timesteps
             {
-                const unsigned char *drow = ddu + sc * W::PAIRB;
-                const unsigned char *grow = gsk + sc * W::PAIRB;
+                const unsigned char *drow = ddu + sc * W::QUADB;
+                const unsigned char *urow = sb + (0 * CW + sc) * W::ROWB;
+                const unsigned char *zrow = sb + (2 * CW + sc) * W::ROWB;
                 unsigned char *orow = outt + sc * W::ROWB;
                 const float *sB = bc32 + S * sr;
                 const float *sC = bc32 + kTC * kNS + S * sr;
 #pragma unroll 1
                 for (int tb = 0; tb < kTC; tb += 8) {
-                    float dl[8], du[8];
+                    float4 dq[8];  // (delta, delta, delta*u, delta*u) per timestep
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float4 v = *reinterpret_cast<const float4 *>(drow + (tb + 2 * k) * 8);
-                        dl[2 * k] = v.x; du[2 * k] = v.y; dl[2 * k + 1] = v.z; du[2 * k + 1] = v.w;
-                    }
+                    for (int e = 0; e < 8; ++e)
+                        dq[e] = *reinterpret_cast<const float4 *>(drow + (tb + e) * 16);
                     float2 y2[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) y2[e] = make_float2(0.f, 0.f);
@@ -244,8 +303,8 @@ scan_fwd_pairs_kernel(const Params p) {
                             const int t = tb + e;
                             const float4 bb = *reinterpret_cast<const float4 *>(sB + t * kNS + 4 * q);
                             const float4 cc = *reinterpret_cast<const float4 *>(sC + t * kNS + 4 * q);
-                            const float2 dl2 = make_float2(dl[e], dl[e]);
-                            const float2 du2 = make_float2(du[e], du[e]);
+                            const float2 dl2 = make_float2(dq[e].x, dq[e].y);
+                            const float2 du2 = make_float2(dq[e].z, dq[e].w);
                             const float2 x0 = __fmul2_rn(dl2, A2[2 * q]);
                             const float2 x1 = __fmul2_rn(dl2, A2[2 * q + 1]);
                             const float2 a0 = make_float2(ex2_mufu(x0.x), ex2_mufu(x0.y));
@@ -258,28 +317,40 @@ scan_fwd_pairs_kernel(const Params p) {
                             y2[e] = __ffma2_rn(make_float2(cc.z, cc.w), h[2 * q + 1], y2[e]);
                         }
                     }
-                    // combine the two halves, transposed: lane sr ends with the
-                    // complete outputs of timesteps tb + 4 sr .. tb + 4 sr + 3
-                    float yv[4];
+                    // combine the R slices, transposed: lane sr ends with the
+                    // complete outputs of timesteps tb + OWN sr .. + OWN - 1
+                    float yv[8];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float lo = y2[i].x + y2[i].y, hi = y2[i + 4].x + y2[i + 4].y;
-                        const float send = sr ? lo : hi;
-                        const float keep = sr ? hi : lo;
-                        yv[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                    for (int e = 0; e < 8; ++e) yv[e] = y2[e].x + y2[e].y;
+                    LaneReduce<R / 2, 8>::run(yv, sr);
+                    // epilogue of this lane's outputs: out = (y + D u) * silu(z),
+                    // u and z read from the staged raw rows
+                    const int te = tb + OWN * sr;
+                    float fu[OWN], fz[OWN], o[OWN];
+                    load_small<T, OWN>(urow + te * sizeof(T), fu);
+                    if (GATE) load_small<T, OWN>(zrow + te * sizeof(T), fz);
+#pragma unroll
+                    for (int i = 0; i < OWN; i += 2) {
+                        const float2 uu = f2(fu[i], fu[i + 1]);
+                        const float2 yy = __ffma2_rn(f2(D_s, D_s), uu, f2(yv[i], yv[i + 1]));
+                        const float2 oo = GATE ? __fmul2_rn(yy, silu2_f(f2(fz[i], fz[i + 1]))) : yy;
+                        o[i] = oo.x;
+                        o[i + 1] = oo.y;
                     }
-                    const int te = tb + 4 * sr;
-                    const float4 g01 = *reinterpret_cast<const float4 *>(grow + te * 8);
-                    const float4 g23 = *reinterpret_cast<const float4 *>(grow + (te + 2) * 8);
-                    float o[4];
-                    o[0] = (yv[0] + g01.y) * g01.x;
-                    o[1] = (yv[1] + g01.w) * g01.z;
-                    o[2] = (yv[2] + g23.y) * g23.x;
-                    o[3] = (yv[3] + g23.w) * g23.z;
-                    store4<T>(orow + te * sizeof(T), o);
+                    if (OWN == 4) store4<T>(orow + te * sizeof(T), o);
+                    else store2<T>(orow + te * sizeof(T), o);
                 }
             }
             __syncwarp();
+            // the last sub-chunk's state is final: publish the successor unit
+            // before this tile's stores, so the release waits on less
+            if (sub + 1 == nsub && j + 1 < p.n_chunks) {
+#pragma unroll
+                for (int k = 0; k < S / 4; ++k)
+                    __stcg(reinterpret_cast<float4 *>(carry) + k,
+                           make_float4(h[2 * k].x, h[2 * k].y, h[2 * k + 1].x, h[2 * k + 1].y));
+                push_unit(p, lane, (unsigned)((j + 1) * p.n_groups + g));
+            }
             // ---- coalesced store of the output tile
 #pragma unroll
             for (int i = lane; i < CW * CPR; i += 32) {
@@ -292,13 +363,7 @@ scan_fwd_pairs_kernel(const Params p) {
             __syncwarp();
         }
 
-        if (j + 1 < p.n_chunks) {
-#pragma unroll
-            for (int k = 0; k < S / 4; ++k)
-                __stcg(reinterpret_cast<float4 *>(carry) + k,
-                       make_float4(h[2 * k].x, h[2 * k].y, h[2 * k + 1].x, h[2 * k + 1].y));
-            push_unit(p, lane, (unsigned)((j + 1) * p.n_groups + g));
-        } else if (p.last_state != nullptr && ds < Dm) {
+        if (j + 1 == p.n_chunks && p.last_state != nullptr && ds < Dm) {
             float *ls = p.last_state + (b * Dm + ds) * N;
 #pragma unroll
             for (int k = 0; k < S / 2; ++k) {
@@ -310,35 +375,44 @@ scan_fwd_pairs_kernel(const Params p) {
     }
 }
 
-template <typename T, bool SP, bool GATE>
+template <typename T, int R, bool SP, bool GATE>
 cudaError_t launch_t(const Params &kp, int grid, cudaStream_t st) {
-    const int smem = kWarps * PairSmem<T>::BYTES;
-    auto kern = scan_fwd_pairs_kernel<T, SP, GATE>;
+    const int smem = kWarps * PairSmem<T, R>::BYTES;
+    auto kern = scan_fwd_pairs_kernel<T, R, SP, GATE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kWarps * 32, smem, st>>>(kp);
     return cudaGetLastError();
 }
 
-}  // namespace
-
-int persistent_lanes2_sub_chunk(int act) {
-    return act == kBF16 ? PairSmem<__nv_bfloat16>::kTC : PairSmem<float>::kTC;
-}
-
-int persistent_lanes2_blocks_per_sm() { return 2; }
-
-cudaError_t launch_persistent_lanes2(const Params &kp, int act, int grid, cudaStream_t st) {
+template <int R>
+cudaError_t launch_r(const Params &kp, int act, int grid, cudaStream_t st) {
     const bool gate = kp.z != nullptr;
     if (act == kBF16) {
-        if (kp.softplus) return gate ? launch_t<__nv_bfloat16, true, true>(kp, grid, st)
-                                     : launch_t<__nv_bfloat16, true, false>(kp, grid, st);
-        return gate ? launch_t<__nv_bfloat16, false, true>(kp, grid, st)
-                    : launch_t<__nv_bfloat16, false, false>(kp, grid, st);
+        if (kp.softplus) return gate ? launch_t<__nv_bfloat16, R, true, true>(kp, grid, st)
+                                     : launch_t<__nv_bfloat16, R, true, false>(kp, grid, st);
+        return gate ? launch_t<__nv_bfloat16, R, false, true>(kp, grid, st)
+                    : launch_t<__nv_bfloat16, R, false, false>(kp, grid, st);
     }
-    if (kp.softplus) return gate ? launch_t<float, true, true>(kp, grid, st)
-                                 : launch_t<float, true, false>(kp, grid, st);
-    return gate ? launch_t<float, false, true>(kp, grid, st) : launch_t<float, false, false>(kp, grid, st);
+    if (kp.softplus) return gate ? launch_t<float, R, true, true>(kp, grid, st)
+                                 : launch_t<float, R, true, false>(kp, grid, st);
+    return gate ? launch_t<float, R, false, true>(kp, grid, st) : launch_t<float, R, false, false>(kp, grid, st);
+}
+
+}  // namespace
+
+int persistent_split_sub_chunk(int lanes, int act) {
+    (void)lanes;
+    return act == kBF16 ? PairSmem<__nv_bfloat16, 2>::kTC : PairSmem<float, 2>::kTC;
+}
+
+int persistent_split_blocks_per_sm(int lanes) {
+    return lanes == 4 ? LanesOccupancy<4>::kBlocks : LanesOccupancy<2>::kBlocks;
+}
+
+cudaError_t launch_persistent_split(const Params &kp, int lanes, int act, int grid, cudaStream_t st) {
+    if (lanes == 4) return launch_r<4>(kp, act, grid, st);
+    return launch_r<2>(kp, act, grid, st);
 }
 
 }  // namespace mscan

@@ -85,8 +85,10 @@ def test_overlap_rejected(lib):
 
 
 def test_bad_tuning_rejected(lib):
-    assert _scan(lib, tuning=binding.Tuning(3, 0)) == -3
-    assert _scan(lib, tuning=binding.Tuning(0, 100)) == -3
+    assert _scan(lib, tuning=binding.Tuning(3, 0, 0, 0)) == -3
+    assert _scan(lib, tuning=binding.Tuning(0, 100, 0, 0)) == -3
+    assert _scan(lib, tuning=binding.Tuning(0, 0, 7, 0)) == -3
+    assert _scan(lib, tuning=binding.Tuning(0, 0, 0, -5)) == -3
 
 
 def test_state_update_validation(lib):

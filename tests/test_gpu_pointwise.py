@@ -17,6 +17,7 @@ pytestmark = pytest.mark.gpu
 
 SCHEDULES = [dict(schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=1),
              dict(schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=2),
+             dict(schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=4),
              dict(schedule=binding.SCHEDULE_STATIC, lanes_per_channel=1),
              dict(schedule=binding.SCHEDULE_STATIC, lanes_per_channel=8),
              dict(schedule=binding.SCHEDULE_STATIC, lanes_per_channel=4, threads_per_block=256)]

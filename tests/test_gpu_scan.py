@@ -159,7 +159,7 @@ def test_auto_plan_is_valid():
 @pytest.mark.parametrize("shape", [(1, 32, 64), (2, 70, 336), (3, 33, 1000), (1, 1, 8),
                                    (4, 100, 2048), (2, 64, 4096)])
 @pytest.mark.parametrize("dstate", [16, 5])
-@pytest.mark.parametrize("lanes", [1, 2])
+@pytest.mark.parametrize("lanes", [1, 2, 4])
 def test_persistent_schedule(dtype, shape, dstate, lanes):
     b, d, L = shape
     w = inputs.custom(b, d, L, dstate, dtype, seed=b * 1000 + d + L + dstate)
@@ -180,7 +180,7 @@ def test_persistent_schedule(dtype, shape, dstate, lanes):
     assert torch.equal(out, out2) and torch.equal(last, last2)
 
 
-@pytest.mark.parametrize("lanes", [1, 2])
+@pytest.mark.parametrize("lanes", [1, 2, 4])
 def test_persistent_matches_static_schedule(lanes):
     w = inputs.custom(4, 640, 1024, 16, "bf16", seed=31)
     ins = dev_inputs(inputs.scan_inputs(w))
