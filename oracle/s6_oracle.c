@@ -7,28 +7,28 @@
  * baseline use it.  It shares no code, header, table or constant with the CUDA
  * library.
  *
- * What it computes (one independent recurrence per (batch b, channel d)):
+ * What it computes (one independent recurrence per (batch b, channel d)).
+ * Sources are sections of the page "Mamba SSM concept and implementation in
+ * Keras and TensorFlow":
  *
- *   delta_t = delta_raw[b,d,t] + bias[d]              (bias added before softplus:
- *                                                      "Mamba SSM concept and
- *                                                      implementation in Keras and
- *                                                      TensorFlow", MambaBlock.ssm,
- *                                                      where dt_proj carries the bias
- *                                                      and softplus follows it)
- *   delta_t = softplus(delta_t)   if the flag is set  (same page, MambaBlock.ssm)
- *   Abar    = exp(delta_t * A[d,n])                   (zero-order hold of A; same page,
- *                                                      "Going from continuous to discrete
- *                                                      spaces" and selective_scan, "first
- *                                                      step of A_bar = exp(dA)")
- *   Bbar u  = delta_t * B[b,n,t] * u[b,d,t]           (the simplified B discretisation the
- *                                                      same selective_scan uses for dB_u)
- *   h_t[n]  = Abar * h_{t-1}[n] + Bbar u              (recurrent form, h_{-1} = h0, zero
- *                                                      by default: same page, "assuming
- *                                                      h0 = zero")
- *   y_t     = sum_n C[b,n,t] * h_t[n] + D[d] * u[b,d,t]   (readout plus the D skip; same
- *                                                      page, selective_scan "y + u * D")
- *   out_t   = y_t * silu(z[b,d,t])    if z is given   (gate; same page, MambaBlock.call
- *                                                      "y * swish(res)")
+ *   delta_t = delta_raw[b,d,t] + bias[d]              the bias belongs to the dt
+ *                                                     projection and is applied
+ *                                                     before softplus (MambaBlock.ssm)
+ *   delta_t = softplus(delta_t)   if the flag is set  (MambaBlock.ssm)
+ *   Abar    = exp(delta_t * A[d,n])                   zero-order hold of A ("Going from
+ *                                                     continuous to discrete spaces";
+ *                                                     the selective_scan listing forms
+ *                                                     delta*A and exponentiates it)
+ *   Bbar u  = delta_t * B[b,n,t] * u[b,d,t]           the simplified B discretisation of
+ *                                                     the selective_scan listing
+ *   h_t[n]  = Abar * h_{t-1}[n] + Bbar u              recurrent form; h_{-1} = h0, zero
+ *                                                     by default (the page unrolls the
+ *                                                     recurrence from a zero state)
+ *   y_t     = sum_n C[b,n,t] * h_t[n] + D[d] * u[b,d,t]   readout plus the D skip
+ *                                                     connection (selective_scan)
+ *   out_t   = y_t * silu(z[b,d,t])    if z is given   the gate of MambaBlock.call (swish of
+ *                                                     the residual half of the input
+ *                                                     projection)
  *   last_state[b,d,n] = h_{L-1}[n]
  *
  * Layouts (row-major, contiguous):

@@ -14,7 +14,7 @@ Sources of the facts (titles of the pages the method is described on):
   "Going from continuous to discrete spaces", the selective_scan listing and
   MambaBlock.call/ssm;
 * convolutional (LTI) form with kernel K_k = C Abar^k Bbar: same page, the
-  convolutional-kernel discussion ("assuming h0 = zero");
+  convolutional-kernel discussion (derived from a zero initial state);
 * the cumulative-sum (log-space) form: same page, selective_scan listing.
 """
 from __future__ import annotations
