@@ -427,12 +427,16 @@ def main():
     lanes, threads, sched = binding.mamba_scan_plan(w.batch, w.dim, w.seqlen, w.dstate, inputs.DTYPES[w.dtype])
     if binding.workspace_status(ws) != 0:
         raise SystemExit("persistent scan reported a timeout")
+    if sched == binding.SCHEDULE_PERSISTENT:
+        kernel = "scan_fwd_pairs_kernel" if lanes > 1 else "scan_fwd_persistent_kernel"
+    else:
+        kernel = "scan_fwd_kernel"
     roof = {"bound": "alu", "achieved": achieved, "peak": mufu_peak_gelem, "unit": UNIT,
             "frac": achieved / mufu_peak_gelem,
-            "traffic": measured_traffic("scan_fwd_kernel mamba-2.8b"),
+            "traffic": measured_traffic(f"{kernel} {w.name}"),
             "peak_source": f"MUFU ex2 16/clk/SM x {SM_COUNT} SMs x {peaks['sm_max_mhz']:.0f} MHz "
                            f"({peaks['source']} sm_max_mhz) / N={w.dstate} exps per element",
-            "kernel": "scan_fwd_kernel", "avg_launch_us": avg_launch_ms * 1e3,
+            "kernel": kernel, "avg_launch_us": avg_launch_ms * 1e3,
             "hbm": {"algorithmic_bytes_per_launch": alg_bytes,
                     "achieved_gbs": alg_bytes / (avg_launch_ms * 1e-3) / 1e9,
                     "peak_gbs": peaks["hbm_gbs"],
