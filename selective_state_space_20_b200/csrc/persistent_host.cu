@@ -14,10 +14,11 @@ namespace {
 int group_channels(int lanes) { return 32 / lanes; }
 int states_per_lane(int lanes) { return persist::kNS / lanes; }
 int sub_chunk(int lanes, int act) {
-    return lanes == 1 ? persistent_lanes1_sub_chunk(act) : persistent_split_sub_chunk(lanes, act);
+    return lanes == 1 ? persistent_spec_sub_chunk() : persistent_split_sub_chunk(lanes, act);
 }
 int blocks_per_sm(int lanes) {
-    return lanes == 1 ? persistent_lanes1_blocks_per_sm() : persistent_split_blocks_per_sm(lanes);
+    // blocks of kWarps workers; the one-lane kernel runs one block of kWarps pairs
+    return lanes == 1 ? persistent_spec_pairs_per_sm() / persist::kWarps : persistent_split_blocks_per_sm(lanes);
 }
 int64_t n_groups(int64_t batch, int64_t dim, int lanes) {
     const int cw = group_channels(lanes);
@@ -78,12 +79,16 @@ bool persistent_supported(const ScanArgs &a) {
 }
 
 // Preferred lanes per channel, or 0 when the static schedule should run.
-// Measured on B200 (Mamba layer shapes, N = 16): two lanes per channel is
-// fastest when its channel groups give every worker (2 blocks x 4 warps per
-// SM) a chain of its own, minus 10 %; with fewer groups, four lanes (3 blocks
-// per SM) as long as three quarters of its workers are busy; below that the
-// static schedule, which splits states further, keeps more warps busy.
+// Measured on B200 (Mamba layer shapes, N = 16): one lane per channel (the
+// warp-specialised kernel, 4 scan warps per SM) is fastest when its channel
+// groups give every scan warp a chain of its own, minus 10 %; then two lanes
+// per channel under the same rule (2 blocks x 4 warps per SM); with fewer
+// groups, four lanes (3 blocks per SM) as long as three quarters of its
+// workers are busy; below that the static schedule, which splits states
+// further, keeps more warps busy.
 int persistent_choose_lanes(const ScanArgs &a, int sm_count) {
+    const int64_t w1 = (int64_t)sm_count * persistent_spec_pairs_per_sm();
+    if (n_groups(a.batch, a.dim, 1) * 10 >= w1 * 9) return 1;
     const int64_t w2 = (int64_t)sm_count * blocks_per_sm(2) * persist::kWarps;
     if (n_groups(a.batch, a.dim, 2) * 10 >= w2 * 9) return 2;
     const int64_t w4 = (int64_t)sm_count * blocks_per_sm(4) * persist::kWarps;
@@ -149,7 +154,7 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
     int64_t grid = (int64_t)sm_count * per_sm;
     const int64_t need = (units + persist::kWarps - 1) / persist::kWarps;
     if (grid > need) grid = need;
-    return lanes == 1 ? launch_persistent_lanes1(kp, a.act, (int)grid, st)
+    return lanes == 1 ? launch_persistent_spec(kp, a.act, (int)grid, st)
                       : launch_persistent_split(kp, lanes, a.act, (int)grid, st);
 }
 

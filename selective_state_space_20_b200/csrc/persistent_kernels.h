@@ -8,10 +8,11 @@
 
 namespace mscan {
 
-// One lane per channel, all states in one thread; units of 32 channels.
-int persistent_lanes1_sub_chunk(int act);
-int persistent_lanes1_blocks_per_sm();
-cudaError_t launch_persistent_lanes1(const persist::Params &kp, int act, int grid, cudaStream_t st);
+// One lane per channel, all states in one thread; units of 32 channels; each
+// scan warp paired with a helper warp (blocks of four pairs, one per SM).
+int persistent_spec_sub_chunk();
+int persistent_spec_pairs_per_sm();
+cudaError_t launch_persistent_spec(const persist::Params &kp, int act, int grid, cudaStream_t st);
 
 // R = 2 or 4 lanes per channel, 16 / R states each; units of 32 / R channels.
 int persistent_split_sub_chunk(int lanes, int act);

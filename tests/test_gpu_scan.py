@@ -29,6 +29,10 @@ def check_full(w: inputs.ScanWorkload, softplus=True, drop=(), **kw):
     cpu = inputs.scan_inputs(w)
     for k in drop:
         cpu[k] = None
+    if not softplus:  # the raw projections are negative; keep delta positive
+        cpu["delta"] = cpu["delta"].abs() * 0.1
+        if cpu["delta_bias"] is not None:
+            cpu["delta_bias"] = cpu["delta_bias"].abs() * 0.01
     ins = dev_inputs(cpu)
     out, last = run_scan(ins, softplus=softplus, **kw)
     torch.cuda.synchronize()
@@ -188,6 +192,24 @@ def test_persistent_matches_static_schedule(lanes):
     o2, s2 = run_scan(ins, schedule=binding.SCHEDULE_STATIC)
     assert rel_err(to_np(o1), to_np(o2)) <= 2e-2
     assert rel_err(to_np(s1), to_np(s2)) <= 1e-4
+
+
+@pytest.mark.parametrize("lanes", [1, 2, 4])
+@pytest.mark.parametrize("drop,softplus", [(("z",), True), (("D", "delta_bias"), True), ((), False),
+                                           (("z", "D", "delta_bias"), False)])
+def test_persistent_optional_inputs(lanes, drop, softplus):
+    for dtype in ("fp32", "bf16"):
+        check_full(inputs.custom(2, 33, 152, 16, dtype, seed=17), softplus=softplus, drop=drop,
+                   schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=lanes)
+
+
+@pytest.mark.parametrize("lanes", [1, 2, 4])
+@pytest.mark.parametrize("chunk", [64, 200, 4096])
+def test_persistent_short_units(lanes, chunk):
+    # few channel groups and many short time chunks: most claimed units are
+    # not ready when claimed, so the workers mostly wait on one another
+    check_full(inputs.custom(2, 96, 2048, 16, "bf16", seed=chunk + lanes),
+               schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=lanes, chunk_timesteps=chunk)
 
 
 def test_persistent_rejects_unsupported():
