@@ -1,6 +1,7 @@
 // persistent_common.cuh -- pieces shared by the persistent scan kernels: the
-// launch parameters, the ready queue of (channel group, time chunk) units,
-// asynchronous global -> shared copies and acquire/release flags.
+// launch parameters, the two schedules (a ready queue of (channel group, time
+// chunk) units, and a balanced static split of the sub-chunks over the
+// workers), asynchronous global -> shared copies and acquire/release flags.
 //
 // Ready queue.  Unit u = j * n_groups + g is chunk j of channel group g.  All
 // chunk-0 units are ready at launch and occupy the first n_groups pop slots
@@ -40,7 +41,9 @@ struct Params {
     int n_chunks;          // chunks per group
     int chunk_len;         // timesteps per chunk
     unsigned *hdr;         // workspace: [pop counter, push counter, error, unused]
-    unsigned *queue;       // workspace: n_groups * (n_chunks - 1) entries
+    unsigned *queue;       // ready-queue schedule: n_groups * (n_chunks - 1) entries
+    unsigned *progress;    // balanced schedule: per group, sub-chunks whose carry is out
+    int subs_per_chain;    // balanced schedule: sub-chunks per group (ceil(seqlen / TC))
     float *carry;          // workspace: n_groups * 32 lanes * states-per-lane floats
 };
 
@@ -101,6 +104,91 @@ __device__ __forceinline__ void push_unit(const Params &p, int lane, unsigned ne
         __threadfence();
         const unsigned slot = atomicAdd(p.hdr + 1, 1u);
         st_release(p.queue + slot, next_unit + 1u);
+    }
+}
+
+// ------------------------------------------------------ balanced schedule
+// The (group, sub-chunk) grid, flattened group-major into T = n_groups * S
+// sub-chunks, is cut into one contiguous range per worker, w * T / P ..
+// (w + 1) * T / P.  A range holds at most three kinds of piece: the start of
+// the group where it ends (from sub-chunk 0), whole groups, and the rest of
+// the group where it starts.  A worker runs them in that order.  Only the
+// last kind depends on another worker -- the one before it, which cut that
+// group and runs its part first -- so every wait points to a lower worker
+// and is over almost as soon as it begins.  The carried state of a group
+// passes through one workspace slot: its producer writes it, then publishes
+// the sub-chunk position in progress[g]; the consumer waits until progress[g]
+// reaches its first sub-chunk.  Pieces of one group run strictly one after
+// the other, so the slot is never overwritten before it has been read.
+struct Piece {
+    int g;       // group
+    int sb, se;  // sub-chunks [sb, se) of the group
+};
+
+// One worker's range, run in field order: head, whole groups, tail.
+struct Range {
+    Piece head;          // the group where the range ends, from sub-chunk 0 (se == 0: none)
+    int full_b, full_e;  // whole groups [full_b, full_e)
+    Piece tail;          // the group where the range starts (se == 0: none); its
+                         // sb > 0 means it continues another worker's piece
+};
+
+__device__ __forceinline__ Range worker_range(const Params &p, long long w, long long P) {
+    const long long S = p.subs_per_chain;
+    const long long T = (long long)p.n_groups * S;
+    const long long s = w * T / P, e = (w + 1) * T / P;
+    Range r;
+    r.head = Piece{0, 0, 0};
+    r.tail = Piece{0, 0, 0};
+    r.full_b = r.full_e = 0;
+    if (s >= e) return r;
+    const int cs = (int)(s / S), os = (int)(s % S);
+    const int ce = (int)(e / S), oe = (int)(e % S);
+    if (cs == ce) {  // inside one group
+        r.tail = Piece{cs, os, oe};
+        return r;
+    }
+    if (oe > 0) r.head = Piece{ce, 0, oe};
+    r.full_b = os > 0 ? cs + 1 : cs;
+    r.full_e = ce;
+    if (os > 0) r.tail = Piece{cs, os, (int)S};
+    return r;
+}
+
+// Wait (lane 0 polls, bounded in time) until group g's carry covers sub-chunk
+// position `pos`; false after a timeout or when another worker gave up.
+__device__ __forceinline__ bool wait_progress(const Params &p, int lane, int g, int pos) {
+    unsigned ok = 1;
+    if (lane == 0) {
+        const unsigned *f = p.progress + g;
+        if (ld_acquire(f) < (unsigned)pos) {
+            unsigned long long t0, t;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+            unsigned ns = 32;
+            while (ld_acquire(f) < (unsigned)pos) {
+                asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+                if (ld_acquire(p.hdr + 2) != 0u || t - t0 > 2000000000ull) {
+                    atomicOr(p.hdr + 2, 1u);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(ns);
+                if (ns < 1024) ns <<= 1;
+            }
+        }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();  // every lane's carry loads come after lane 0's acquire
+    return ok != 0;
+}
+
+// Publish that group g's carry now covers sub-chunk position `pos`.  Every
+// lane must have written its part of the carry before the call.
+__device__ __forceinline__ void publish_progress(const Params &p, int lane, int g, int pos) {
+    __syncwarp();
+    if (lane == 0) {
+        __threadfence();
+        st_release(p.progress + g, (unsigned)pos);
     }
 }
 

@@ -57,8 +57,22 @@ Layout layout(int64_t batch, int64_t dim, int64_t seqlen, int lanes, int tu) {
     return l;
 }
 
-// Largest workspace any device can need: the smallest unit (4 sub-chunks).
+// Balanced split (lanes 2 and 4): header, one progress word per group, one
+// carried state per group.  Independent of the device.
+Layout balanced_layout(int64_t batch, int64_t dim, int lanes) {
+    Layout l;
+    l.groups = n_groups(batch, dim, lanes);
+    l.chunks = 1;
+    l.queue_off = 16;  // progress words
+    l.carry_off = 16 + (size_t)((l.groups * 4 + 255) / 256 * 256);
+    l.bytes = l.carry_off + (size_t)(l.groups * 32 * states_per_lane(lanes)) * 4;
+    return l;
+}
+
+// Largest workspace any device can need.  Queue schedule (one lane): the
+// smallest unit (4 sub-chunks).
 size_t bound_for(int64_t batch, int64_t dim, int64_t seqlen, int lanes, int act) {
+    if (lanes != 1) return balanced_layout(batch, dim, lanes).bytes;
     const int tc = sub_chunk(lanes, act);
     const int64_t max_chunks = ((seqlen + tc - 1) / tc + 3) / 4;
     int64_t tu = (seqlen + max_chunks - 1) / max_chunks;
@@ -79,16 +93,14 @@ bool persistent_supported(const ScanArgs &a) {
 }
 
 // Preferred lanes per channel, or 0 when the static schedule should run.
-// Measured on B200 (Mamba layer shapes, N = 16): one lane per channel (the
-// warp-specialised kernel, 4 scan warps per SM) is fastest when its channel
-// groups give every scan warp a chain of its own, minus 10 %; then two lanes
-// per channel under the same rule (2 blocks x 4 warps per SM); with fewer
-// groups, four lanes (3 blocks per SM) as long as three quarters of its
-// workers are busy; below that the static schedule, which splits states
-// further, keeps more warps busy.
+// Measured on B200 (Mamba layer shapes, N = 16): two lanes per channel is
+// fastest when its channel groups give every worker (2 blocks x 4 warps per
+// SM) a chain of its own, minus 10 %; with fewer groups, four lanes (3 blocks
+// per SM) as long as three quarters of its workers are busy; below that the
+// static schedule, which splits states further, keeps more warps busy.  One
+// lane per channel (the warp-specialised kernel) is never preferred: it
+// measured slower than two lanes on every Mamba shape; it runs on request.
 int persistent_choose_lanes(const ScanArgs &a, int sm_count) {
-    const int64_t w1 = (int64_t)sm_count * persistent_spec_pairs_per_sm();
-    if (n_groups(a.batch, a.dim, 1) * 10 >= w1 * 9) return 1;
     const int64_t w2 = (int64_t)sm_count * blocks_per_sm(2) * persist::kWarps;
     if (n_groups(a.batch, a.dim, 2) * 10 >= w2 * 9) return 2;
     const int64_t w4 = (int64_t)sm_count * blocks_per_sm(4) * persist::kWarps;
@@ -119,6 +131,33 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
     const int64_t workers = (int64_t)sm_count * per_sm * persist::kWarps;
     const int64_t groups = n_groups(a.batch, a.dim, lanes);
     const int tc = sub_chunk(lanes, a.act);
+
+    persist::Params kp;
+    kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
+    kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias;
+    kp.out = a.out; kp.last_state = a.last_state;
+    kp.dim = a.dim; kp.seqlen = a.seqlen; kp.dstate = a.dstate; kp.softplus = a.softplus;
+    kp.group_channels = group_channels(lanes);
+    kp.groups_per_batch = (int)((a.dim + kp.group_channels - 1) / kp.group_channels);
+    kp.n_groups = (int)groups;
+    kp.subs_per_chain = (int)((a.seqlen + tc - 1) / tc);
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    kp.hdr = reinterpret_cast<unsigned *>(w);
+
+    if (lanes != 1) {
+        // balanced split over every resident worker; chunk_timesteps does not apply
+        const Layout l = balanced_layout(a.batch, a.dim, lanes);
+        if (ws_bytes < l.bytes) return cudaErrorInvalidValue;
+        kp.n_chunks = 1;
+        kp.chunk_len = (int)a.seqlen;
+        kp.queue = nullptr;
+        kp.progress = reinterpret_cast<unsigned *>(w + l.queue_off);
+        kp.carry = reinterpret_cast<float *>(w + l.carry_off);
+        cudaError_t e = cudaMemsetAsync(w, 0, l.queue_off + (size_t)groups * 4, st);
+        if (e != cudaSuccess) return e;
+        return launch_persistent_split(kp, lanes, a.act, sm_count, st);
+    }
+
     int tu = chunk_len(groups, a.seqlen, (int)workers, tc);
     if (chunk_timesteps > 0) {
         // explicit unit length, but never shorter than the bound's units
@@ -131,20 +170,10 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
     }
     const Layout l = layout(a.batch, a.dim, a.seqlen, lanes, tu);
     if (ws_bytes < l.bytes) return cudaErrorInvalidValue;
-
-    persist::Params kp;
-    kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
-    kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias;
-    kp.out = a.out; kp.last_state = a.last_state;
-    kp.dim = a.dim; kp.seqlen = a.seqlen; kp.dstate = a.dstate; kp.softplus = a.softplus;
-    kp.group_channels = group_channels(lanes);
-    kp.groups_per_batch = (int)((a.dim + kp.group_channels - 1) / kp.group_channels);
-    kp.n_groups = (int)l.groups;
     kp.n_chunks = (int)l.chunks;
     kp.chunk_len = tu;
-    unsigned char *w = static_cast<unsigned char *>(workspace);
-    kp.hdr = reinterpret_cast<unsigned *>(w);
     kp.queue = reinterpret_cast<unsigned *>(w + l.queue_off);
+    kp.progress = nullptr;
     kp.carry = reinterpret_cast<float *>(w + l.carry_off);
     // counters and queue entries start at zero; carries are written before read
     cudaError_t e = cudaMemsetAsync(w, 0, l.queue_off + (size_t)(l.groups * (l.chunks - 1)) * 4, st);
@@ -154,8 +183,7 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
     int64_t grid = (int64_t)sm_count * per_sm;
     const int64_t need = (units + persist::kWarps - 1) / persist::kWarps;
     if (grid > need) grid = need;
-    return lanes == 1 ? launch_persistent_spec(kp, a.act, (int)grid, st)
-                      : launch_persistent_split(kp, lanes, a.act, (int)grid, st);
+    return launch_persistent_spec(kp, a.act, (int)grid, st);
 }
 
 }  // namespace mscan

@@ -14,10 +14,12 @@ int persistent_spec_sub_chunk();
 int persistent_spec_pairs_per_sm();
 cudaError_t launch_persistent_spec(const persist::Params &kp, int act, int grid, cudaStream_t st);
 
-// R = 2 or 4 lanes per channel, 16 / R states each; units of 32 / R channels.
+// R = 2 or 4 lanes per channel, 16 / R states each; groups of 32 / R
+// channels; the balanced split over every worker that fits on the device
+// (launched cooperatively, all resident).
 int persistent_split_sub_chunk(int lanes, int act);
 int persistent_split_blocks_per_sm(int lanes);
-cudaError_t launch_persistent_split(const persist::Params &kp, int lanes, int act, int grid,
+cudaError_t launch_persistent_split(const persist::Params &kp, int lanes, int act, int sm_count,
                                    cudaStream_t st);
 
 }  // namespace mscan

@@ -1,28 +1,31 @@
 // scan_fwd_persistent_pairs.cu -- persistent selective-scan (S6) forward
-// with each channel's states split over a pair of lanes.
+// with each channel's states split over R = 2 or 4 lanes.
 //
-// Same computation as scan_fwd_persistent.cu (softplus(delta + bias), the
-// zero-order-hold decay exp(delta A), the diagonal recurrence, C readout, D
-// skip, silu gate; "Mamba SSM concept and implementation in Keras and
-// TensorFlow", recurrent form and selective_scan / MambaBlock; fused as in
-// the Mamba paper, Appendix E.5).  Splitting the 16 states of a channel over
-// two lanes doubles the number of warps a problem provides -- e.g. 1280
-// instead of 640 for the Mamba-2.8B layer -- so every SM sub-partition runs
-// two workers and one hides the other's dependency stalls; with one warp per
-// sub-partition the MUFU idles whenever that warp is in a non-exp stretch.
+// Computes softplus(delta + bias), the zero-order-hold decay exp(delta A),
+// the diagonal recurrence, the C readout, the D skip and the silu gate ("Mamba
+// SSM concept and implementation in Keras and TensorFlow", recurrent form and
+// selective_scan / MambaBlock; fused as in the Mamba paper, Appendix E.5).
+// Splitting the 16 states of a channel over R lanes multiplies the number of
+// warps a problem provides -- e.g. 1280 instead of 640 for the Mamba-2.8B
+// layer at R = 2 -- so every SM sub-partition runs two or more workers and one
+// hides the other's dependency stalls; with one warp per sub-partition the
+// MUFU idles whenever that warp is in a non-exp stretch.
 //
-// Per (16-channel group, time chunk) unit, per sub-chunk of TC timesteps:
+// Work: the balanced split of persistent_common.cuh -- each warp runs a
+// contiguous share of the (channel group, sub-chunk) grid, at most three
+// pieces.  Per piece, per sub-chunk of TC timesteps:
 //   1. cp.async stages the raw u / delta / z rows and the B / C rows of the
 //      next sub-chunk (double buffer) while this one is processed;
 //   2. prologue: B and C are widened to fp32 as [t][n] rows for broadcast
-//      reads; every element's delta = softplus(delta_raw + bias), delta * u,
-//      silu(z) and D * u are computed once (lane = channel & timestep half)
-//      into shared float2 arrays;
-//   3. scan: lane (channel c, half r) advances states 8r .. 8r+7 through
-//      blocks of 8 timesteps (state pairs on FMUL2 / FFMA2, 16 ex2 per lane
-//      per 2 timesteps on the MUFU); the two halves' readouts are combined
-//      with one transposed shuffle round, leaving each lane 4 consecutive
-//      complete outputs, which it gates and packs into the output tile;
+//      reads; every element's delta = softplus(delta_raw + bias) and delta * u
+//      are computed once (lane = channel & timestep slice) into shared
+//      (delta, delta, delta u, delta u) quads;
+//   3. scan: lane (channel c, slice r) advances states (16/R) r .. through
+//      blocks of 8 timesteps (state pairs on FMUL2 / FFMA2, the decays on the
+//      MUFU); the R slices' readouts are combined with transposed shuffle
+//      rounds, leaving each lane 8/R consecutive complete outputs, which it
+//      gates -- (y + D u) * silu(z) from the staged raw rows -- and packs into
+//      the output tile;
 //   4. the tile is written with coalesced 16-byte stores.
 // Shared arrays are padded so that every quarter-warp access is free of bank
 // conflicts.
@@ -49,7 +52,8 @@ struct PairSmem {
     static constexpr int ROWB = kTC * (int)sizeof(T) + 16;  // raw / output row pitch (bytes)
     static constexpr int RAW_ROWS = 3 * CW + 2 * kNS;      // u, delta, z rows, then B, C rows
     static constexpr int STAGE = RAW_ROWS * ROWB;
-    static constexpr int BC32 = 2 * kTC * kNS * 4;          // fp32 B then C, [t][n]
+    static constexpr int CPAD = 16;                         // C starts 64 bytes after B's end
+    static constexpr int BC32 = (2 * kTC * kNS + CPAD) * 4;  // fp32 B then C, [t][n]
     static constexpr int QUADB = kTC * 16 + 16;             // float4 row pitch (bytes)
     static constexpr int DDU = CW * QUADB;                  // (delta, delta, delta*u, delta*u) [c][t]
     static constexpr int OUTB = CW * ROWB;                  // packed outputs [c][t]
@@ -161,12 +165,22 @@ scan_fwd_pairs_kernel(const Params p) {
     float2 A2[S / 2];
     float bias_p = 0.f, D_s = 0.f;
 
+    // This worker's share of the balanced split: head, whole groups, tail.
+    // Piece: sub-chunks [sb, se) of group g, carried state in from sub-chunk
+    // sb and out at se (or the final state when se is the group's end).
+    const Range rg = worker_range(p, (long long)blockIdx.x * kWarps + warp, (long long)gridDim.x * kWarps);
+    const int has_head = rg.head.se > 0 ? 1 : 0;
+    const int n_pieces = has_head + (rg.full_e - rg.full_b) + (rg.tail.se > 0 ? 1 : 0);
 #pragma unroll 1
-    while (true) {
-        const unsigned unit = pop_unit(p, lane);
-        if (unit == kUnitDone || unit == kUnitAbort) break;
-        const int g = (int)(unit % (unsigned)p.n_groups);
-        const int j = (int)(unit / (unsigned)p.n_groups);
+    for (int pi = 0; pi < n_pieces; ++pi) {
+        int g, sb, se;
+        if (pi < has_head) {
+            g = rg.head.g; sb = 0; se = rg.head.se;
+        } else if (pi - has_head < rg.full_e - rg.full_b) {
+            g = rg.full_b + (pi - has_head); sb = 0; se = p.subs_per_chain;
+        } else {
+            g = rg.tail.g; sb = rg.tail.sb; se = rg.tail.se;
+        }
         const int64_t b = g / p.groups_per_batch;
         const int64_t d0 = (int64_t)(g % p.groups_per_batch) * CW;
         const int nrows = (Dm - d0) < CW ? (int)(Dm - d0) : CW;
@@ -187,10 +201,11 @@ scan_fwd_pairs_kernel(const Params p) {
 
         float2 h[S / 2];
         float *carry = p.carry + ((int64_t)g * 32 + lane) * S;
-        if (j == 0) {
+        if (sb == 0) {
 #pragma unroll
             for (int k = 0; k < S / 2; ++k) h[k] = make_float2(0.f, 0.f);
         } else {
+            if (!wait_progress(p, lane, g, sb)) return;
 #pragma unroll
             for (int k = 0; k < S / 4; ++k) {
                 const float4 v = __ldcg(reinterpret_cast<const float4 *>(carry) + k);  // S/4 float4
@@ -199,14 +214,13 @@ scan_fwd_pairs_kernel(const Params p) {
             }
         }
 
-        const int64_t tb0 = (int64_t)j * p.chunk_len;
-        const int64_t tb1 = (tb0 + p.chunk_len) < L ? (tb0 + p.chunk_len) : L;
-        const int nsub = (int)((tb1 - tb0 + kTC - 1) / kTC);
+        const int64_t tb0 = (int64_t)sb * kTC;
+        const int nsub = se - sb;
         const int64_t row0 = (b * Dm + d0) * L;
         const int64_t bc0 = b * (int64_t)N * L;
 
         auto issue = [&](int sub, int st) {
-            unsigned char *sb = base + st * W::STAGE;
+            unsigned char *sbuf = base + st * W::STAGE;
             const int64_t t0 = tb0 + (int64_t)sub * kTC;
 #pragma unroll
             for (int i = lane; i < CW * CPR; i += 32) {
@@ -214,9 +228,9 @@ scan_fwd_pairs_kernel(const Params p) {
                 const int64_t t = t0 + c * V;
                 const bool ok = (r < nrows) && (t < L);
                 const int64_t off = ok ? row0 + r * L + t : 0;
-                cp16(sb + (0 * CW + r) * W::ROWB + c * 16, gu + off, ok);
-                cp16(sb + (1 * CW + r) * W::ROWB + c * 16, gd + off, ok);
-                if (GATE) cp16(sb + (2 * CW + r) * W::ROWB + c * 16, gz + off, ok);
+                cp16(sbuf + (0 * CW + r) * W::ROWB + c * 16, gu + off, ok);
+                cp16(sbuf + (1 * CW + r) * W::ROWB + c * 16, gd + off, ok);
+                if (GATE) cp16(sbuf + (2 * CW + r) * W::ROWB + c * 16, gz + off, ok);
             }
 #pragma unroll
             for (int i = lane; i < 2 * kNS * CPR; i += 32) {
@@ -225,7 +239,7 @@ scan_fwd_pairs_kernel(const Params p) {
                 const int64_t t = t0 + c * V;
                 const bool ok = (n < N) && (t < L);
                 const int64_t off = ok ? bc0 + (int64_t)n * L + t : 0;
-                cp16(sb + (3 * CW + which * kNS + n) * W::ROWB + c * 16, (which ? gC : gB) + off, ok);
+                cp16(sbuf + (3 * CW + which * kNS + n) * W::ROWB + c * 16, (which ? gC : gB) + off, ok);
             }
             cp_commit();
         };
@@ -241,7 +255,7 @@ scan_fwd_pairs_kernel(const Params p) {
                 cp_wait<0>();
             }
             __syncwarp();
-            const unsigned char *sb = base + st * W::STAGE;
+            const unsigned char *sbuf = base + st * W::STAGE;
             const int64_t t0 = tb0 + (int64_t)sub * kTC;
             const int tvalid = (L - t0) < kTC ? (int)(L - t0) : kTC;
 
@@ -251,8 +265,8 @@ scan_fwd_pairs_kernel(const Params p) {
             for (int i = lane; i < 2 * kNS * CPR; i += 32) {
                 const int c = i / (2 * kNS), rr = i % (2 * kNS);
                 float f[V];
-                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sb + (3 * CW + rr) * W::ROWB + c * 16), f);
-                float *dst = bc32 + (rr / kNS) * kTC * kNS + (rr % kNS);
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sbuf + (3 * CW + rr) * W::ROWB + c * 16), f);
+                float *dst = bc32 + (rr / kNS) * (kTC * kNS + W::CPAD) + (rr % kNS);
 #pragma unroll
                 for (int e = 0; e < V; ++e) dst[(c * V + e) * kNS] = f[e];
             }
@@ -263,8 +277,8 @@ scan_fwd_pairs_kernel(const Params p) {
             for (int v = 0; v < PT; v += V) {
                 const int tt = ph * PT + v;
                 float fu[V], fd[V];
-                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sb + (0 * CW + pc) * W::ROWB + tt * sizeof(T)), fu);
-                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sb + (1 * CW + pc) * W::ROWB + tt * sizeof(T)), fd);
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sbuf + (0 * CW + pc) * W::ROWB + tt * sizeof(T)), fu);
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sbuf + (1 * CW + pc) * W::ROWB + tt * sizeof(T)), fd);
                 float4 *dd = reinterpret_cast<float4 *>(ddu + pc * W::QUADB + tt * 16);
 #pragma unroll
                 for (int e = 0; e < V; e += 2) {  // element pairs on the packed x2 instructions
@@ -282,11 +296,11 @@ scan_fwd_pairs_kernel(const Params p) {
             // ---- scan: lane (sc, sr), blocks of 8 timesteps
             {
                 const unsigned char *drow = ddu + sc * W::QUADB;
-                const unsigned char *urow = sb + (0 * CW + sc) * W::ROWB;
-                const unsigned char *zrow = sb + (2 * CW + sc) * W::ROWB;
+                const unsigned char *urow = sbuf + (0 * CW + sc) * W::ROWB;
+                const unsigned char *zrow = sbuf + (2 * CW + sc) * W::ROWB;
                 unsigned char *orow = outt + sc * W::ROWB;
                 const float *sB = bc32 + S * sr;
-                const float *sC = bc32 + kTC * kNS + S * sr;
+                const float *sC = bc32 + kTC * kNS + W::CPAD + S * sr;
 #pragma unroll 1
                 for (int tb = 0; tb < kTC; tb += 8) {
                     float4 dq[8];  // (delta, delta, delta*u, delta*u) per timestep
@@ -342,14 +356,14 @@ scan_fwd_pairs_kernel(const Params p) {
                 }
             }
             __syncwarp();
-            // the last sub-chunk's state is final: publish the successor unit
+            // the piece's last sub-chunk leaves the carried state: publish it
             // before this tile's stores, so the release waits on less
-            if (sub + 1 == nsub && j + 1 < p.n_chunks) {
+            if (sub + 1 == nsub && se < p.subs_per_chain) {
 #pragma unroll
                 for (int k = 0; k < S / 4; ++k)
                     __stcg(reinterpret_cast<float4 *>(carry) + k,
                            make_float4(h[2 * k].x, h[2 * k].y, h[2 * k + 1].x, h[2 * k + 1].y));
-                push_unit(p, lane, (unsigned)((j + 1) * p.n_groups + g));
+                publish_progress(p, lane, g, se);
             }
             // ---- coalesced store of the output tile
 #pragma unroll
@@ -363,7 +377,7 @@ scan_fwd_pairs_kernel(const Params p) {
             __syncwarp();
         }
 
-        if (j + 1 == p.n_chunks && p.last_state != nullptr && ds < Dm) {
+        if (se == p.subs_per_chain && p.last_state != nullptr && ds < Dm) {
             float *ls = p.last_state + (b * Dm + ds) * N;
 #pragma unroll
             for (int k = 0; k < S / 2; ++k) {
@@ -376,27 +390,43 @@ scan_fwd_pairs_kernel(const Params p) {
 }
 
 template <typename T, int R, bool SP, bool GATE>
-cudaError_t launch_t(const Params &kp, int grid, cudaStream_t st) {
+cudaError_t launch_t(const Params &kp, int sm_count, cudaStream_t st) {
     const int smem = kWarps * PairSmem<T, R>::BYTES;
     auto kern = scan_fwd_pairs_kernel<T, R, SP, GATE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kWarps * 32, smem, st>>>(kp);
-    return cudaGetLastError();
+    static const int per_sm = [&] {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kWarps * 32, smem) != cudaSuccess) n = 0;
+        return n < LanesOccupancy<R>::kBlocks ? n : LanesOccupancy<R>::kBlocks;
+    }();
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    // a worker may wait on the one before it: launch them all resident at once
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sm_count * per_sm));
+    cfg.blockDim = dim3(kWarps * 32);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, kp);
 }
 
 template <int R>
-cudaError_t launch_r(const Params &kp, int act, int grid, cudaStream_t st) {
+cudaError_t launch_r(const Params &kp, int act, int sm_count, cudaStream_t st) {
     const bool gate = kp.z != nullptr;
     if (act == kBF16) {
-        if (kp.softplus) return gate ? launch_t<__nv_bfloat16, R, true, true>(kp, grid, st)
-                                     : launch_t<__nv_bfloat16, R, true, false>(kp, grid, st);
-        return gate ? launch_t<__nv_bfloat16, R, false, true>(kp, grid, st)
-                    : launch_t<__nv_bfloat16, R, false, false>(kp, grid, st);
+        if (kp.softplus) return gate ? launch_t<__nv_bfloat16, R, true, true>(kp, sm_count, st)
+                                     : launch_t<__nv_bfloat16, R, true, false>(kp, sm_count, st);
+        return gate ? launch_t<__nv_bfloat16, R, false, true>(kp, sm_count, st)
+                    : launch_t<__nv_bfloat16, R, false, false>(kp, sm_count, st);
     }
-    if (kp.softplus) return gate ? launch_t<float, R, true, true>(kp, grid, st)
-                                 : launch_t<float, R, true, false>(kp, grid, st);
-    return gate ? launch_t<float, R, false, true>(kp, grid, st) : launch_t<float, R, false, false>(kp, grid, st);
+    if (kp.softplus) return gate ? launch_t<float, R, true, true>(kp, sm_count, st)
+                                 : launch_t<float, R, true, false>(kp, sm_count, st);
+    return gate ? launch_t<float, R, false, true>(kp, sm_count, st) : launch_t<float, R, false, false>(kp, sm_count, st);
 }
 
 }  // namespace
@@ -410,9 +440,9 @@ int persistent_split_blocks_per_sm(int lanes) {
     return lanes == 4 ? LanesOccupancy<4>::kBlocks : LanesOccupancy<2>::kBlocks;
 }
 
-cudaError_t launch_persistent_split(const Params &kp, int lanes, int act, int grid, cudaStream_t st) {
-    if (lanes == 4) return launch_r<4>(kp, act, grid, st);
-    return launch_r<2>(kp, act, grid, st);
+cudaError_t launch_persistent_split(const Params &kp, int lanes, int act, int sm_count, cudaStream_t st) {
+    if (lanes == 4) return launch_r<4>(kp, act, sm_count, st);
+    return launch_r<2>(kp, act, sm_count, st);
 }
 
 }  // namespace mscan

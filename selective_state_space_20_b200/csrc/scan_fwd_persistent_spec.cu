@@ -50,12 +50,18 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // give up a wait after 2 s
 
 constexpr unsigned kFirst = 1u, kLast = 2u, kEnd = 4u, kSkip = 8u;
 
+// One sub-chunk of a unit, as the helper hands it along (48 bytes).
 struct Desc {
     unsigned unit;
-    int sub;
+    int sub;           // sub-chunk within the unit
     unsigned flags;
-    int tvalid;
+    int tvalid;        // timesteps of the sub-chunk inside the sequence
+    int g, j;          // channel group, time chunk
+    int b, d0;         // batch, first channel of the group
+    long long rowidx;  // b * dim + d0: row of the group's first channel
+    long long t0;      // first timestep
 };
+static_assert(sizeof(Desc) == 48, "descriptor layout");
 
 template <typename T>
 struct SpecSmem {
@@ -64,18 +70,21 @@ struct SpecSmem {
     static constexpr int ROWB = kTC * (int)sizeof(T) + 16;  // raw row pitch
     static constexpr int ROW_U = 0, ROW_D = 32, ROW_Z = 64, ROW_B = 96, ROW_C = 112;
     static constexpr int RAW_ROWS = 128;
-    static constexpr int RAW = 16 + RAW_ROWS * ROWB;      // descriptor, then rows
+    static constexpr int HDR = (int)sizeof(Desc);
+    static constexpr int RAW = HDR + RAW_ROWS * ROWB;     // descriptor, then rows
     static constexpr int NRAW = sizeof(T) == 2 ? 4 : 3;   // raw slots in flight
     static constexpr int DLB = kTC * 8 + 16;              // (delta, delta u) row pitch
-    static constexpr int DL_OFF = 16;                     // after the descriptor
+    static constexpr int DL_OFF = HDR;
     static constexpr int BC_OFF = DL_OFF + kChannels * DLB;
     static constexpr int C_FLOATS = kTC * kNS + 16;       // C starts 64 bytes after B's end
+    static constexpr int PROC = BC_OFF + (kTC * kNS + C_FLOATS) * 4;
     static constexpr int YB = kTC * 4 + 16;               // readout row pitch
-    static constexpr int Y_OFF = BC_OFF + (kTC * kNS + C_FLOATS) * 4;
-    static constexpr int PROC = Y_OFF + kChannels * YB;
-    static constexpr int BAR_OFF = NRAW * RAW + 2 * PROC;  // 4 mbarriers
+    static constexpr int Y = kChannels * YB;
+    static constexpr int PROC_OFF = NRAW * RAW;
+    static constexpr int Y_OFF = PROC_OFF + 2 * PROC;     // three readout slots
+    static constexpr int BAR_OFF = Y_OFF + 3 * Y;         // 4 mbarriers
     static constexpr int PAIR = BAR_OFF + 32;
-    static_assert(RAW % 16 == 0 && PROC % 16 == 0 && BAR_OFF % 16 == 0, "16-byte alignment");
+    static_assert(RAW % 16 == 0 && PROC % 16 == 0 && Y % 16 == 0 && BAR_OFF % 16 == 0, "16-byte alignment");
     static_assert(ROW_C == ROW_B + kNS && ROW_C + kNS == RAW_ROWS, "B rows, then C rows");
 };
 
@@ -135,30 +144,42 @@ struct Helper {
     const Params &p;
     unsigned char *pair;  // this pair's shared memory
     int lane;
-    // unit generator
-    unsigned unit;        // current unit, or kUnitDone when a new one is needed
-    int sub, nsub;
+    // unit generator (all lanes hold the same values)
+    unsigned unit;        // unit being handed out, or kUnitDone when a new one is needed
+    int sub, nsub, g, j, b, d0;
+    long long rowidx;
     long long pending;    // claimed queue slot not yet ready, or -1
     bool finished;
-    uint64_t skip_since;
+    uint64_t skip_since;  // lane 0: when the pending slot was first found empty
+    // per-lane source offsets of this lane's 16-byte copies (elements, before
+    // the sub-chunk's first timestep is added)
+    long long off_x[W::CPR], off_bc[W::CPR];
+    int row_x[W::CPR], n_bc[W::CPR], c_x;
 
     __device__ Helper(const Params &p_, unsigned char *pair_, int lane_)
-        : p(p_), pair(pair_), lane(lane_), unit(kUnitDone), sub(0), nsub(0), pending(-1),
-          finished(false), skip_since(0) {}
+        : p(p_), pair(pair_), lane(lane_), unit(kUnitDone), sub(0), nsub(0), g(0), j(0), b(0), d0(0),
+          rowidx(0), pending(-1), finished(false), skip_since(0) {
+        // copy i = lane + 32 it covers row i / CPR, 16-byte chunk i % CPR
+        c_x = lane % W::CPR;
+#pragma unroll
+        for (int it = 0; it < W::CPR; ++it) {
+            const int i = lane + 32 * it;
+            row_x[it] = i / W::CPR;
+            off_x[it] = (long long)row_x[it] * p.seqlen + c_x * W::V;
+            const int rem = i % (kNS * W::CPR);
+            n_bc[it] = rem / W::CPR;
+            off_bc[it] = (long long)n_bc[it] * p.seqlen + c_x * W::V;
+        }
+    }
 
     __device__ unsigned char *raw(int k) const { return pair + (k % W::NRAW) * W::RAW; }
-    __device__ unsigned char *proc(int k) const { return pair + W::NRAW * W::RAW + (k & 1) * W::PROC; }
-
-    __device__ int unit_subs(unsigned u) const {
-        const int j = (int)(u / (unsigned)p.n_groups);
-        const int64_t t0 = (int64_t)j * p.chunk_len;
-        const int64_t len = (p.seqlen - t0) < p.chunk_len ? (p.seqlen - t0) : p.chunk_len;
-        return (int)((len + kTC - 1) / kTC);
-    }
+    __device__ unsigned char *proc(int k) const { return pair + W::PROC_OFF + (k & 1) * W::PROC; }
+    __device__ unsigned char *ybuf(int k) const { return pair + W::Y_OFF + (k % 3) * W::Y; }
 
     // Descriptor of the next sub-chunk in this pair's stream.
     __device__ Desc next() {
-        Desc d{0u, 0, kEnd, 0};
+        Desc d{};
+        d.flags = kEnd;
         if (finished) return d;
         if (unit == kUnitDone) {
             const unsigned n_units = (unsigned)p.n_groups * (unsigned)p.n_chunks;
@@ -196,15 +217,23 @@ struct Helper {
                 pending = -1;
                 skip_since = 0;
             }
+            g = (int)(unit % (unsigned)p.n_groups);
+            j = (int)(unit / (unsigned)p.n_groups);
+            b = g / p.groups_per_batch;
+            d0 = (g % p.groups_per_batch) * kChannels;
+            rowidx = (long long)b * p.dim + d0;
+            const long long ts = (long long)j * p.chunk_len;
+            const long long len = (p.seqlen - ts) < p.chunk_len ? (p.seqlen - ts) : p.chunk_len;
             sub = 0;
-            nsub = unit_subs(unit);
+            nsub = (int)((len + kTC - 1) / kTC);
         }
         d.unit = unit;
         d.sub = sub;
         d.flags = (sub == 0 ? kFirst : 0u) | (sub + 1 == nsub ? kLast : 0u);
-        const int j = (int)(unit / (unsigned)p.n_groups);
-        const int64_t t0 = (int64_t)j * p.chunk_len + (int64_t)sub * kTC;
-        d.tvalid = (p.seqlen - t0) < kTC ? (int)(p.seqlen - t0) : kTC;
+        d.g = g; d.j = j; d.b = b; d.d0 = d0;
+        d.rowidx = rowidx;
+        d.t0 = (long long)j * p.chunk_len + (long long)sub * kTC;
+        d.tvalid = (p.seqlen - d.t0) < kTC ? (int)(p.seqlen - d.t0) : kTC;
         if (++sub == nsub) unit = kUnitDone;
         return d;
     }
@@ -214,39 +243,31 @@ struct Helper {
         unsigned char *rb = raw(k);
         if (lane == 0) *reinterpret_cast<Desc *>(rb) = d;
         if ((d.flags & (kEnd | kSkip)) == 0) {
-            const int g = (int)(d.unit % (unsigned)p.n_groups);
-            const int j = (int)(d.unit / (unsigned)p.n_groups);
-            const int64_t b = g / p.groups_per_batch;
-            const int64_t d0 = (int64_t)(g % p.groups_per_batch) * kChannels;
-            const int nrows = (p.dim - d0) < kChannels ? (int)(p.dim - d0) : kChannels;
-            const int64_t L = p.seqlen;
-            const int64_t t0 = (int64_t)j * p.chunk_len + (int64_t)d.sub * kTC;
-            const int64_t row0 = (b * p.dim + d0) * L;
-            const int64_t bc0 = b * (int64_t)p.dstate * L;
+            const long long L = p.seqlen;
+            const long long base_x = d.rowidx * L + d.t0;
+            const long long base_bc = (long long)d.b * p.dstate * L + d.t0;
+            const int nrows = (p.dim - d.d0) < kChannels ? (int)(p.dim - d.d0) : kChannels;
+            const bool tok = d.t0 + c_x * W::V < L;
             const T *gu = static_cast<const T *>(p.u);
             const T *gd = static_cast<const T *>(p.delta);
             const T *gz = static_cast<const T *>(p.z);
             const T *gB = static_cast<const T *>(p.B);
             const T *gC = static_cast<const T *>(p.C);
-            unsigned char *rows = rb + 16;
+            unsigned char *rows = rb + W::HDR + c_x * 16;
 #pragma unroll
-            for (int i = lane; i < kChannels * W::CPR; i += 32) {
-                const int r = i / W::CPR, c = i % W::CPR;
-                const int64_t t = t0 + c * W::V;
-                const bool ok = r < nrows && t < L;
-                const int64_t off = ok ? row0 + r * L + t : 0;
-                cp16(rows + (W::ROW_U + r) * W::ROWB + c * 16, gu + off, ok);
-                cp16(rows + (W::ROW_D + r) * W::ROWB + c * 16, gd + off, ok);
-                if (gz) cp16(rows + (W::ROW_Z + r) * W::ROWB + c * 16, gz + off, ok);
+            for (int it = 0; it < W::CPR; ++it) {
+                const bool ok = tok && row_x[it] < nrows;
+                const long long off = ok ? base_x + off_x[it] : 0;
+                cp16(rows + (W::ROW_U + row_x[it]) * W::ROWB, gu + off, ok);
+                cp16(rows + (W::ROW_D + row_x[it]) * W::ROWB, gd + off, ok);
+                if (gz) cp16(rows + (W::ROW_Z + row_x[it]) * W::ROWB, gz + off, ok);
             }
 #pragma unroll
-            for (int i = lane; i < 2 * kNS * W::CPR; i += 32) {
-                const int which = i / (kNS * W::CPR), rem = i % (kNS * W::CPR);
-                const int n = rem / W::CPR, c = rem % W::CPR;
-                const int64_t t = t0 + c * W::V;
-                const bool ok = n < p.dstate && t < L;
-                const int64_t off = ok ? bc0 + (int64_t)n * L + t : 0;
-                cp16(rows + (W::ROW_B + which * kNS + n) * W::ROWB + c * 16, (which ? gC : gB) + off, ok);
+            for (int it = 0; it < W::CPR; ++it) {
+                const int which = (lane + 32 * it) / (kNS * W::CPR);
+                const bool ok = tok && n_bc[it] < p.dstate;
+                const long long off = ok ? base_bc + off_bc[it] : 0;
+                cp16(rows + (W::ROW_B + which * kNS + n_bc[it]) * W::ROWB, (which ? gC : gB) + off, ok);
             }
         }
         cp_commit();
@@ -259,10 +280,8 @@ struct Helper {
         unsigned char *pb = proc(k);
         if (lane == 0) *reinterpret_cast<Desc *>(pb) = d;
         if (d.flags & (kEnd | kSkip)) return;
-        const unsigned char *rows = raw(k) + 16;
-        const int g = (int)(d.unit % (unsigned)p.n_groups);
-        const int64_t d0 = (int64_t)(g % p.groups_per_batch) * kChannels;
-        const int64_t dc = d0 + lane;
+        const unsigned char *rows = raw(k) + W::HDR;
+        const int dc = d.d0 + lane;
         const float bias = (dc < p.dim && p.delta_bias) ? __ldg(p.delta_bias + dc) : 0.f;
         float fu[kTC], fd[kTC];
         unpack_row<T>(rows + (W::ROW_U + lane) * W::ROWB, fu);
@@ -289,19 +308,14 @@ struct Helper {
     template <bool GATE>
     __device__ void epilogue(int k, const Desc &d) {
         if (d.flags & (kEnd | kSkip)) return;
-        const unsigned char *rows = raw(k) + 16;
-        const unsigned char *pb = proc(k);
-        const int g = (int)(d.unit % (unsigned)p.n_groups);
-        const int j = (int)(d.unit / (unsigned)p.n_groups);
-        const int64_t b = g / p.groups_per_batch;
-        const int64_t d0 = (int64_t)(g % p.groups_per_batch) * kChannels;
-        const int64_t dc = d0 + lane;
+        const int dc = d.d0 + lane;
         if (dc >= p.dim) return;
+        const unsigned char *rows = raw(k) + W::HDR;
         const float Dd = p.D ? __ldg(p.D + dc) : 0.f;
         float fu[kTC], fz[kTC], y[kTC];
         unpack_row<T>(rows + (W::ROW_U + lane) * W::ROWB, fu);
         if (GATE) unpack_row<T>(rows + (W::ROW_Z + lane) * W::ROWB, fz);
-        const float4 *yr = reinterpret_cast<const float4 *>(pb + W::Y_OFF + lane * W::YB);
+        const float4 *yr = reinterpret_cast<const float4 *>(ybuf(k) + lane * W::YB);
 #pragma unroll
         for (int i = 0; i < kTC / 4; ++i) {
             const float4 v = yr[i];
@@ -315,9 +329,7 @@ struct Helper {
             o[t] = oo.x;
             o[t + 1] = oo.y;
         }
-        T *gout = static_cast<T *>(p.out);
-        const int64_t t0 = (int64_t)j * p.chunk_len + (int64_t)d.sub * kTC;
-        T *dst = gout + (b * p.dim + dc) * p.seqlen + t0;
+        T *dst = static_cast<T *>(p.out) + (d.rowidx + lane) * p.seqlen + d.t0;
 #pragma unroll
         for (int c = 0; c < W::CPR; ++c)
             if (c * W::V < d.tvalid) stg16_stream(dst + c * W::V, Elem<T>::pack(o + c * W::V));
@@ -344,9 +356,11 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
     __syncthreads();
 
     if (is_helper) {
+        // Iteration k (the scan warp runs sub-chunk k): once the scan is done
+        // with k-1, prepare k+1 in its processed slot and hand it over; then
+        // finish k-1 and refill k-1's raw slot with sub-chunk k + NRAW - 1.
         Helper<T> h(p, pair, lane);
         constexpr int NR = W::NRAW;
-        // fill the pipeline: sub-chunks 0 .. NR-2 staged, 0 prepared
         for (int k = 0; k < NR - 1; ++k) h.issue(k, h.next());
         cp_wait<NR - 2>();
         __syncwarp();
@@ -355,22 +369,25 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
         __syncwarp();
         if (lane == 0) mbar_arrive(full + 0);
         bool ok = true;
-        Desc dprev{0u, 0, kSkip, 0};
+        Desc dprev{};
+        dprev.flags = kSkip;
         int k = 0;
         while (!(dcur.flags & kEnd)) {
-            // the scan runs sub-chunk k; finish k-1, then prepare k+1
-            if (k >= 1) {
-                if (!mbar_wait(done + ((k - 1) & 1), ((k - 1) >> 1) & 1, err)) { ok = false; break; }
-                h.template epilogue<GATE>(k - 1, dprev);
-                __syncwarp();  // raw slot of k-1 is read before it is refilled
+            if (k >= 1 && !mbar_wait(done + ((k - 1) & 1), ((k - 1) >> 1) & 1, err)) {
+                ok = false;
+                break;
             }
-            h.issue(k + NR - 1, h.next());
-            cp_wait<NR - 2>();
+            cp_wait<NR - 3>();  // sub-chunk k+1's rows have landed
             __syncwarp();
             const Desc dnext = *reinterpret_cast<const Desc *>(h.raw(k + 1));
             h.template prologue<SP>(k + 1, dnext);
             __syncwarp();
             if (lane == 0) mbar_arrive(full + ((k + 1) & 1));
+            if (k >= 1) {
+                h.template epilogue<GATE>(k - 1, dprev);
+                __syncwarp();  // k-1's raw rows are read before the slot is refilled
+            }
+            h.issue(k + NR - 1, h.next());
             dprev = dcur;
             dcur = dnext;
             ++k;
@@ -390,29 +407,25 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
     for (int q = 0; q < kNS / 2; ++q) { A2[q] = f2(0.f, 0.f); hs[q] = f2(0.f, 0.f); }
     const int N = p.dstate;
     for (int k = 0;; ++k) {
-        uint64_t *bar = full + (k & 1);
-        if (!mbar_wait(bar, (k >> 1) & 1, err)) return;
-        unsigned char *pb = pair + W::NRAW * W::RAW + (k & 1) * W::PROC;
+        if (!mbar_wait(full + (k & 1), (k >> 1) & 1, err)) return;
+        const unsigned char *pb = pair + W::PROC_OFF + (k & 1) * W::PROC;
         const Desc d = *reinterpret_cast<const Desc *>(pb);
         if (d.flags & kEnd) return;
         if (!(d.flags & kSkip)) {
-            const int g = (int)(d.unit % (unsigned)p.n_groups);
-            const int j = (int)(d.unit / (unsigned)p.n_groups);
-            const int64_t b = g / p.groups_per_batch;
-            const int64_t dc = (int64_t)(g % p.groups_per_batch) * kChannels + lane;
-            float *carry = p.carry + ((int64_t)g * 32 + lane) * kNS;
+            const int dc = d.d0 + lane;
+            float *carry = p.carry + ((int64_t)d.g * 32 + lane) * kNS;
             if (d.flags & kFirst) {
-                if (g != cur_group) {
-                    cur_group = g;
+                if (d.g != cur_group) {
+                    cur_group = d.g;
 #pragma unroll
                     for (int q = 0; q < kNS / 2; ++q) {
                         const int n0 = 2 * q, n1 = 2 * q + 1;
-                        const float a0 = (dc < p.dim && n0 < N) ? __ldg(p.A + dc * N + n0) : 0.f;
-                        const float a1 = (dc < p.dim && n1 < N) ? __ldg(p.A + dc * N + n1) : 0.f;
+                        const float a0 = (dc < p.dim && n0 < N) ? __ldg(p.A + (int64_t)dc * N + n0) : 0.f;
+                        const float a1 = (dc < p.dim && n1 < N) ? __ldg(p.A + (int64_t)dc * N + n1) : 0.f;
                         A2[q] = f2(a0 * kLog2e, a1 * kLog2e);
                     }
                 }
-                if (j == 0) {
+                if (d.j == 0) {
 #pragma unroll
                     for (int q = 0; q < kNS / 2; ++q) hs[q] = f2(0.f, 0.f);
                 } else {
@@ -427,7 +440,7 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
             const float4 *dlrow = reinterpret_cast<const float4 *>(pb + W::DL_OFF + lane * W::DLB);
             const float *sB = reinterpret_cast<const float *>(pb + W::BC_OFF);
             const float *sC = sB + kTC * kNS + 16;
-            float4 *yrow = reinterpret_cast<float4 *>(pb + W::Y_OFF + lane * W::YB);
+            float4 *yrow = reinterpret_cast<float4 *>(pair + W::Y_OFF + (k % 3) * W::Y + lane * W::YB);
 #pragma unroll 1
             for (int tb = 0; tb < kTC; tb += 8) {
                 float4 dd[4];  // (delta_t, delta_t u_t, delta_t+1, delta_t+1 u_t+1)
@@ -464,14 +477,14 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
                                                y2[7].x + y2[7].y);
             }
             if (d.flags & kLast) {
-                if (j + 1 < p.n_chunks) {
+                if (d.j + 1 < p.n_chunks) {
 #pragma unroll
                     for (int q = 0; q < kNS / 4; ++q)
                         __stcg(reinterpret_cast<float4 *>(carry) + q,
                                make_float4(hs[2 * q].x, hs[2 * q].y, hs[2 * q + 1].x, hs[2 * q + 1].y));
-                    push_unit(p, lane, (unsigned)((j + 1) * p.n_groups + g));
+                    push_unit(p, lane, (unsigned)((d.j + 1) * p.n_groups + d.g));
                 } else if (p.last_state != nullptr && dc < p.dim) {
-                    float *ls = p.last_state + (b * p.dim + dc) * N;
+                    float *ls = p.last_state + (d.rowidx + lane) * N;
 #pragma unroll
                     for (int q = 0; q < kNS / 2; ++q) {
                         if (2 * q < N) ls[2 * q] = hs[q].x;
