@@ -52,8 +52,12 @@ struct PairSmem {
     static constexpr int ROWB = kTC * (int)sizeof(T) + 16;  // raw / output row pitch (bytes)
     static constexpr int RAW_ROWS = 3 * CW + 2 * kNS;      // u, delta, z rows, then B, C rows
     static constexpr int STAGE = RAW_ROWS * ROWB;
-    static constexpr int CPAD = 16;                         // C starts 64 bytes after B's end
-    static constexpr int BC32 = (2 * kTC * kNS + CPAD) * 4;  // fp32 B then C, [t][n]
+    // fp32 B then C as [t][n] rows of 64 bytes; every V rows (one staged
+    // 16-byte chunk of timesteps) are followed by 32 bytes of padding, which
+    // makes the transposing 16-byte stores free of bank conflicts
+    static constexpr int BLKB = V * kNS * 4 + 32;
+    static constexpr int BARR = (kTC / V) * BLKB;          // one of B, C
+    static constexpr int BC32 = 2 * BARR;
     static constexpr int QUADB = kTC * 16 + 16;             // float4 row pitch (bytes)
     static constexpr int DDU = CW * QUADB;                  // (delta, delta, delta*u, delta*u) [c][t]
     static constexpr int OUTB = CW * ROWB;                  // packed outputs [c][t]
@@ -219,27 +223,45 @@ scan_fwd_pairs_kernel(const Params p) {
         const int64_t row0 = (b * Dm + d0) * L;
         const int64_t bc0 = b * (int64_t)N * L;
 
-        auto issue = [&](int sub, int st) {
-            unsigned char *sbuf = base + st * W::STAGE;
-            const int64_t t0 = tb0 + (int64_t)sub * kTC;
+        // this lane's 16-byte copies: chunk cx of rows (lane + 32 i) / CPR
+        constexpr int NX = (CW * CPR + 31) / 32, NB = 2 * kNS * CPR / 32;
+        const int cx = lane % CPR;
+        int64_t xoff[NX], boff[NB];
+        bool xok[NX], bok[NB];
 #pragma unroll
-            for (int i = lane; i < CW * CPR; i += 32) {
-                const int r = i / CPR, c = i % CPR;
-                const int64_t t = t0 + c * V;
-                const bool ok = (r < nrows) && (t < L);
-                const int64_t off = ok ? row0 + r * L + t : 0;
-                cp16(sbuf + (0 * CW + r) * W::ROWB + c * 16, gu + off, ok);
-                cp16(sbuf + (1 * CW + r) * W::ROWB + c * 16, gd + off, ok);
-                if (GATE) cp16(sbuf + (2 * CW + r) * W::ROWB + c * 16, gz + off, ok);
+        for (int i = 0; i < NX; ++i) {
+            const int r = (lane + 32 * i) / CPR;
+            xok[i] = lane + 32 * i < CW * CPR && r < nrows;
+            xoff[i] = row0 + r * L + cx * V;
+        }
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+            const int n = ((lane + 32 * i) % (kNS * CPR)) / CPR;
+            bok[i] = n < N;
+            boff[i] = bc0 + (int64_t)n * L + cx * V;
+        }
+        auto issue = [&](int sub, int st) {
+            unsigned char *sbuf = base + st * W::STAGE + cx * 16;
+            const int64_t t0 = tb0 + (int64_t)sub * kTC;
+            const bool tok = t0 + cx * V < L;
+#pragma unroll
+            for (int i = 0; i < NX; ++i) {
+                const int r = (lane + 32 * i) / CPR;
+                if (lane + 32 * i < CW * CPR) {
+                    const bool ok = xok[i] && tok;
+                    const int64_t off = ok ? xoff[i] + t0 : 0;
+                    cp16(sbuf + (0 * CW + r) * W::ROWB, gu + off, ok);
+                    cp16(sbuf + (1 * CW + r) * W::ROWB, gd + off, ok);
+                    if (GATE) cp16(sbuf + (2 * CW + r) * W::ROWB, gz + off, ok);
+                }
             }
 #pragma unroll
-            for (int i = lane; i < 2 * kNS * CPR; i += 32) {
-                const int which = i / (kNS * CPR), rem = i % (kNS * CPR);
-                const int n = rem / CPR, c = rem % CPR;
-                const int64_t t = t0 + c * V;
-                const bool ok = (n < N) && (t < L);
-                const int64_t off = ok ? bc0 + (int64_t)n * L + t : 0;
-                cp16(sbuf + (3 * CW + which * kNS + n) * W::ROWB + c * 16, (which ? gC : gB) + off, ok);
+            for (int i = 0; i < NB; ++i) {
+                const int which = (lane + 32 * i) / (kNS * CPR);
+                const int n = ((lane + 32 * i) % (kNS * CPR)) / CPR;
+                const bool ok = bok[i] && tok;
+                const int64_t off = ok ? boff[i] + t0 : 0;
+                cp16(sbuf + (3 * CW + which * kNS + n) * W::ROWB, (which ? gC : gB) + off, ok);
             }
             cp_commit();
         };
@@ -259,16 +281,22 @@ scan_fwd_pairs_kernel(const Params p) {
             const int64_t t0 = tb0 + (int64_t)sub * kTC;
             const int tvalid = (L - t0) < kTC ? (int)(L - t0) : kTC;
 
-            // ---- prologue (a): B and C to fp32 [t][n]; a quarter-warp covers
-            // 8 consecutive rows of one chunk
+            // ---- prologue (a): B and C to fp32 [t][n].  Lane (which, q, c)
+            // reads states 4q .. 4q+3 of B (which 0) or C (which 1) in chunk c
+            // and writes them back as one 16-byte [t][4q .. 4q+3] piece per
+            // timestep
+            {
+                static_assert(CPR == 4, "four chunks of timesteps per sub-chunk");
+                const int which = lane >> 4, q = (lane >> 2) & 3, c = lane & 3;
+                float f[4][V];
 #pragma unroll
-            for (int i = lane; i < 2 * kNS * CPR; i += 32) {
-                const int c = i / (2 * kNS), rr = i % (2 * kNS);
-                float f[V];
-                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sbuf + (3 * CW + rr) * W::ROWB + c * 16), f);
-                float *dst = bc32 + (rr / kNS) * (kTC * kNS + W::CPAD) + (rr % kNS);
+                for (int k = 0; k < 4; ++k)
+                    Elem<T>::unpack(*reinterpret_cast<const uint4 *>(
+                                        sbuf + (3 * CW + which * kNS + 4 * q + k) * W::ROWB + c * 16), f[k]);
+                unsigned char *dst = reinterpret_cast<unsigned char *>(bc32) + which * W::BARR + c * W::BLKB + 16 * q;
 #pragma unroll
-                for (int e = 0; e < V; ++e) dst[(c * V + e) * kNS] = f[e];
+                for (int e = 0; e < V; ++e)
+                    *reinterpret_cast<float4 *>(dst + e * kNS * 4) = make_float4(f[0][e], f[1][e], f[2][e], f[3][e]);
             }
             // ---- prologue (b): per element, once: delta and delta*u, stored
             // duplicated as (delta, delta, delta*u, delta*u) so the scan reads
@@ -284,8 +312,10 @@ scan_fwd_pairs_kernel(const Params p) {
                 for (int e = 0; e < V; e += 2) {  // element pairs on the packed x2 instructions
                     float2 x = __fadd2_rn(f2(fd[e], fd[e + 1]), f2(bias_p, bias_p));
                     if (SP) x = softplus2_f(x);
-                    x.x = (tt + e < tvalid) ? x.x : 0.f;  // past the end: Abar = 1, no input
-                    x.y = (tt + e + 1 < tvalid) ? x.y : 0.f;
+                    if (tvalid < kTC) {  // past the end: Abar = 1, no input
+                        x.x = (tt + e < tvalid) ? x.x : 0.f;
+                        x.y = (tt + e + 1 < tvalid) ? x.y : 0.f;
+                    }
                     const float2 xu = __fmul2_rn(x, f2(fu[e], fu[e + 1]));
                     dd[e] = make_float4(x.x, x.x, xu.x, xu.x);
                     dd[e + 1] = make_float4(x.y, x.y, xu.y, xu.y);
@@ -299,10 +329,11 @@ scan_fwd_pairs_kernel(const Params p) {
                 const unsigned char *urow = sbuf + (0 * CW + sc) * W::ROWB;
                 const unsigned char *zrow = sbuf + (2 * CW + sc) * W::ROWB;
                 unsigned char *orow = outt + sc * W::ROWB;
-                const float *sB = bc32 + S * sr;
-                const float *sC = bc32 + kTC * kNS + W::CPAD + S * sr;
+                const float *sB0 = bc32 + S * sr;
 #pragma unroll 1
                 for (int tb = 0; tb < kTC; tb += 8) {
+                    const float *sB = sB0 + (tb / V) * (W::BLKB / 4);
+                    const float *sC = sB + W::BARR / 4;
                     float4 dq[8];  // (delta, delta, delta*u, delta*u) per timestep
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
@@ -314,9 +345,9 @@ scan_fwd_pairs_kernel(const Params p) {
                     for (int q = 0; q < S / 4; ++q) {
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            const int t = tb + e;
-                            const float4 bb = *reinterpret_cast<const float4 *>(sB + t * kNS + 4 * q);
-                            const float4 cc = *reinterpret_cast<const float4 *>(sC + t * kNS + 4 * q);
+                            const int to = (e / V) * (W::BLKB / 4) + (e % V) * kNS + 4 * q;
+                            const float4 bb = *reinterpret_cast<const float4 *>(sB + to);
+                            const float4 cc = *reinterpret_cast<const float4 *>(sC + to);
                             const float2 dl2 = make_float2(dq[e].x, dq[e].y);
                             const float2 du2 = make_float2(dq[e].z, dq[e].w);
                             const float2 x0 = __fmul2_rn(dl2, A2[2 * q]);
