@@ -428,7 +428,7 @@ def main():
     if binding.workspace_status(ws) != 0:
         raise SystemExit("persistent scan reported a timeout")
     if sched == binding.SCHEDULE_PERSISTENT:
-        kernel = "scan_fwd_pairs_kernel" if lanes > 1 else "scan_fwd_persistent_kernel"
+        kernel = "scan_fwd_pairs_kernel" if lanes > 1 else "scan_fwd_spec_kernel"
     else:
         kernel = "scan_fwd_kernel"
     roof = {"bound": "alu", "achieved": achieved, "peak": mufu_peak_gelem, "unit": UNIT,
