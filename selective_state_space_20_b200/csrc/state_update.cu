@@ -5,10 +5,13 @@
 // form; mamba-jax sample.py generation loop).
 //
 // The step is bound by HBM traffic: 2 * 4 * N bytes of state per channel
-// against ~N exponentials.  One thread owns one (batch, channel) row and
-// streams its N states with 16-byte loads and stores; A rows are re-read by
+// against ~N exponentials.  The main kernel gives each (batch, channel) row
+// N / 4 consecutive lanes, one 16-byte slice of the state each, so a warp's
+// state loads and stores cover whole contiguous 512-byte spans; the row's
+// readout is summed over its lanes with shuffles.  A rows are re-read by
 // every batch row and stay in L2, B and C rows are shared by all channels of a
-// batch row and stay in L1.
+// batch row and stay in L1.  Other state sizes and unaligned tensors take a
+// thread-per-row kernel.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -79,8 +82,75 @@ state_update_kernel(const SUParams p) {
     Elem<T>::store(static_cast<T *>(p.out) + row, y);
 }
 
+// Four states per lane: bf16 / fp32 loads of four consecutive B or C values.
+template <typename T> struct Quad;
+template <> struct Quad<float> {
+    __device__ __forceinline__ static float4 load(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
+};
+template <> struct Quad<__nv_bfloat16> {
+    __device__ __forceinline__ static float4 load(const __nv_bfloat16 *p) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2 *>(p));
+        float4 f;
+        Elem<__nv_bfloat16>::unpack2(w.x, f.x, f.y);
+        Elem<__nv_bfloat16>::unpack2(w.y, f.z, f.w);
+        return f;
+    }
+};
+
+// NV / 4 lanes per row (NV = dstate, a multiple of 4 up to 128); lane q of a
+// row owns states 4q .. 4q + 3.
+template <typename T, int NV>
+__global__ void __launch_bounds__(256)
+state_update_lanes_kernel(const SUParams p) {
+    constexpr int Q = NV / 4;
+    static_assert(Q >= 1 && Q <= 32 && (Q & (Q - 1)) == 0, "lanes per row: a power of two");
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool live = gid / Q < p.rows;
+    const int64_t row = live ? gid / Q : p.rows - 1;  // idle lanes still join the shuffles
+    const int qi = (int)(gid % Q);
+    const int64_t b = row / p.dim, d = row % p.dim;
+    const T *gu = static_cast<const T *>(p.u);
+    const T *gd = static_cast<const T *>(p.delta);
+    const T *gz = static_cast<const T *>(p.z);
+
+    float dl = Elem<T>::load(gd + row) + (p.delta_bias ? __ldg(p.delta_bias + d) : 0.f);
+    if (p.softplus) dl = softplus_f(dl);
+    const float ut = Elem<T>::load(gu + row);
+    const float du = dl * ut;
+    const float dl2 = dl * kLog2e;
+    float4 *st = reinterpret_cast<float4 *>(p.state + row * NV) + qi;
+    const float4 h4 = *st;
+    const float4 a4 = __ldg(reinterpret_cast<const float4 *>(p.A + d * NV) + qi);
+    const float4 b4 = Quad<T>::load(static_cast<const T *>(p.B) + b * NV + 4 * qi);
+    const float4 c4 = Quad<T>::load(static_cast<const T *>(p.C) + b * NV + 4 * qi);
+    float4 hn;
+    hn.x = fmaf(ex2_mufu(dl2 * a4.x), h4.x, du * b4.x);
+    hn.y = fmaf(ex2_mufu(dl2 * a4.y), h4.y, du * b4.y);
+    hn.z = fmaf(ex2_mufu(dl2 * a4.z), h4.z, du * b4.z);
+    hn.w = fmaf(ex2_mufu(dl2 * a4.w), h4.w, du * b4.w);
+    float y = fmaf(c4.x, hn.x, fmaf(c4.y, hn.y, fmaf(c4.z, hn.z, c4.w * hn.w)));
+#pragma unroll
+    for (int o = Q / 2; o >= 1; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
+    if (!live) return;
+    *st = hn;
+    if (qi == 0) {
+        if (p.D) y = fmaf(__ldg(p.D + d), ut, y);
+        if (gz) y *= silu_f(Elem<T>::load(gz + row));
+        Elem<T>::store(static_cast<T *>(p.out) + row, y);
+    }
+}
+
+template <typename T, int NV>
+static cudaError_t launch_lanes(const SUParams &kp, cudaStream_t st) {
+    const int threads = 256;
+    const int64_t blocks = (kp.rows * (NV / 4) + threads - 1) / threads;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    state_update_lanes_kernel<T, NV><<<(unsigned)blocks, threads, 0, st>>>(kp);
+    return cudaGetLastError();
+}
+
 template <typename T>
-static cudaError_t launch_typed(const SUParams &kp, cudaStream_t st) {
+static cudaError_t launch_rows(const SUParams &kp, cudaStream_t st) {
     const int threads = 256;
     const int64_t blocks = (kp.rows + threads - 1) / threads;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
@@ -97,6 +167,20 @@ static cudaError_t launch_typed(const SUParams &kp, cudaStream_t st) {
     else
         state_update_kernel<T, 0><<<(unsigned)blocks, threads, 0, st>>>(kp);
     return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_typed(const SUParams &kp, cudaStream_t st) {
+    auto al = [](const void *q, uintptr_t m) { return (reinterpret_cast<uintptr_t>(q) & (m - 1)) == 0; };
+    const uintptr_t bc_align = 4 * sizeof(T);  // four B / C values per lane
+    if (al(kp.state, 16) && al(kp.A, 16) && al(kp.B, bc_align) && al(kp.C, bc_align)) {
+        if (kp.dstate == 16) return launch_lanes<T, 16>(kp, st);
+        if (kp.dstate == 8) return launch_lanes<T, 8>(kp, st);
+        if (kp.dstate == 32) return launch_lanes<T, 32>(kp, st);
+        if (kp.dstate == 64) return launch_lanes<T, 64>(kp, st);
+        if (kp.dstate == 4) return launch_lanes<T, 4>(kp, st);
+    }
+    return launch_rows<T>(kp, st);
 }
 
 cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t st) {

@@ -104,3 +104,19 @@ def test_decode_workload_1024_steps():
     record("decode 1024 steps, sampled rows", out=e_out, state=e_st, scan_vs_decode=diff / scale,
            state_vs_scan=e_state)
     assert e_out <= 2e-2 and e_st <= 2e-2
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_misaligned_b_c_take_row_kernel(dtype):
+    # aligned state and A, B / C rows starting off their 16-byte grid
+    cpu = step_inputs(3, 40, 16, dtype, seed=8)
+    dev = {k: v.cuda() for k, v in cpu.items()}
+    for k in ("B", "C"):
+        buf = torch.empty(dev[k].numel() + 1, device="cuda", dtype=dev[k].dtype)
+        t = buf[1:].view(dev[k].shape)
+        t.copy_(dev[k])
+        dev[k] = t
+    out, st = run_step(dev)
+    ro, rs = oracle.state_update(cpu["state"], cpu["u"], cpu["delta"], cpu["A"], cpu["B"], cpu["C"],
+                                 D=cpu["D"], z=cpu["z"], delta_bias=cpu["delta_bias"])
+    assert rel_err(to_np(out), ro) <= TOL[inputs.DTYPES[dtype]] and rel_err(to_np(st), rs) <= 1e-4
