@@ -96,15 +96,22 @@ bool persistent_supported(const ScanArgs &a) {
 // Measured on B200 (Mamba layer shapes, N = 16): two lanes per channel is
 // fastest when its channel groups give every worker (2 blocks x 4 warps per
 // SM) a chain of its own, minus 10 %; with fewer groups, four lanes (3 blocks
-// per SM) as long as three quarters of its workers are busy; below that the
-// static schedule, which splits states further, keeps more warps busy.  One
-// lane per channel (the warp-specialised kernel) is never preferred: it
-// measured slower than two lanes on every Mamba shape; it runs on request.
+// per SM) as long as three quarters of its workers are busy.  With fewer
+// groups still, long sequences (at least 8 sub-chunks per worker) go back to
+// two lanes, where the balanced split cuts each group into pieces that run
+// at once (two-phase pieces; the long-context layer, 1 x 2048 x 262144:
+// 6.0 ms against 7.9 ms for the static schedule).  Below that the static
+// schedule, which splits states further, keeps more warps busy.  One lane
+// per channel (the warp-specialised kernel) is never preferred: it measured
+// slower than two lanes on every Mamba shape; it runs on request.
 int persistent_choose_lanes(const ScanArgs &a, int sm_count) {
     const int64_t w2 = (int64_t)sm_count * blocks_per_sm(2) * persist::kWarps;
-    if (n_groups(a.batch, a.dim, 2) * 10 >= w2 * 9) return 2;
+    const int64_t g2 = n_groups(a.batch, a.dim, 2);
+    if (g2 * 10 >= w2 * 9) return 2;
     const int64_t w4 = (int64_t)sm_count * blocks_per_sm(4) * persist::kWarps;
     if (n_groups(a.batch, a.dim, 4) * 4 >= w4 * 3) return 4;
+    const int tc = sub_chunk(2, a.act);
+    if (g2 * ((a.seqlen + tc - 1) / tc) >= 8 * w2) return 2;
     return 0;
 }
 

@@ -172,7 +172,12 @@ scan_fwd_pairs_kernel(const Params p) {
     // This worker's share of the balanced split: head, whole groups, tail.
     // Piece: sub-chunks [sb, se) of group g, carried state in from sub-chunk
     // sb and out at se (or the final state when se is the group's end).
-    const Range rg = worker_range(p, (long long)blockIdx.x * kWarps + warp, (long long)gridDim.x * kWarps);
+    const long long n_workers = (long long)gridDim.x * kWarps;
+    const Range rg = worker_range(p, (long long)blockIdx.x * kWarps + warp, n_workers);
+    // Shares shorter than ~0.55 of a group: waiting for the piece before
+    // would chain a group's pieces end to end (the group's full length); the
+    // two-phase pieces below cost ~1.8x their length but all run at once.
+    const bool two_phase = 20LL * p.n_groups < 11LL * n_workers;
     const int has_head = rg.head.se > 0 ? 1 : 0;
     const int n_pieces = has_head + (rg.full_e - rg.full_b) + (rg.tail.se > 0 ? 1 : 0);
 #pragma unroll 1
@@ -203,20 +208,21 @@ scan_fwd_pairs_kernel(const Params p) {
             D_s = (ds < Dm && p.D) ? __ldg(p.D + ds) : 0.f;
         }
 
-        float2 h[S / 2];
         float *carry = p.carry + ((int64_t)g * 32 + lane) * S;
-        if (sb == 0) {
-#pragma unroll
-            for (int k = 0; k < S / 2; ++k) h[k] = make_float2(0.f, 0.f);
-        } else {
-            if (!wait_progress(p, lane, g, sb)) return;
+        auto load_carry = [&](float2 (&hh)[S / 2]) {
 #pragma unroll
             for (int k = 0; k < S / 4; ++k) {
                 const float4 v = __ldcg(reinterpret_cast<const float4 *>(carry) + k);  // S/4 float4
-                h[2 * k] = make_float2(v.x, v.y);
-                h[2 * k + 1] = make_float2(v.z, v.w);
+                hh[2 * k] = make_float2(v.x, v.y);
+                hh[2 * k + 1] = make_float2(v.z, v.w);
             }
-        }
+        };
+        auto store_carry = [&](const float2 (&hh)[S / 2]) {
+#pragma unroll
+            for (int k = 0; k < S / 4; ++k)
+                __stcg(reinterpret_cast<float4 *>(carry) + k,
+                       make_float4(hh[2 * k].x, hh[2 * k].y, hh[2 * k + 1].x, hh[2 * k + 1].y));
+        };
 
         const int64_t tb0 = (int64_t)sb * kTC;
         const int nsub = se - sb;
@@ -266,6 +272,10 @@ scan_fwd_pairs_kernel(const Params p) {
             cp_commit();
         };
 
+        // The piece's sub-chunks.  State-only (SO) runs do the recurrence alone
+        // -- no C rows, readout, gate or stores -- and sum delta into dsum;
+        // full runs publish the carried state at the end when `publish_end`.
+        auto run_subs = [&](const bool SO, float2 (&h)[S / 2], double &dsum, bool publish_end) {
         issue(0, 0);
 #pragma unroll 1
         for (int sub = 0; sub < nsub; ++sub) {
@@ -285,7 +295,7 @@ scan_fwd_pairs_kernel(const Params p) {
             // reads states 4q .. 4q+3 of B (which 0) or C (which 1) in chunk c
             // and writes them back as one 16-byte [t][4q .. 4q+3] piece per
             // timestep
-            {
+            if (!SO || lane < 16) {  // C rows only feed the readout
                 static_assert(CPR == 4, "four chunks of timesteps per sub-chunk");
                 const int which = lane >> 4, q = (lane >> 2) & 3, c = lane & 3;
                 float f[4][V];
@@ -338,6 +348,12 @@ scan_fwd_pairs_kernel(const Params p) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         dq[e] = *reinterpret_cast<const float4 *>(drow + (tb + e) * 16);
+                    if (SO) {
+                        float s8 = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) s8 += dq[e].x;
+                        dsum += (double)s8;
+                    }
                     float2 y2[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) y2[e] = make_float2(0.f, 0.f);
@@ -347,7 +363,6 @@ scan_fwd_pairs_kernel(const Params p) {
                         for (int e = 0; e < 8; ++e) {
                             const int to = (e / V) * (W::BLKB / 4) + (e % V) * kNS + 4 * q;
                             const float4 bb = *reinterpret_cast<const float4 *>(sB + to);
-                            const float4 cc = *reinterpret_cast<const float4 *>(sC + to);
                             const float2 dl2 = make_float2(dq[e].x, dq[e].y);
                             const float2 du2 = make_float2(dq[e].z, dq[e].w);
                             const float2 x0 = __fmul2_rn(dl2, A2[2 * q]);
@@ -358,10 +373,14 @@ scan_fwd_pairs_kernel(const Params p) {
                             const float2 bu1 = __fmul2_rn(du2, make_float2(bb.z, bb.w));
                             h[2 * q] = __ffma2_rn(a0, h[2 * q], bu0);
                             h[2 * q + 1] = __ffma2_rn(a1, h[2 * q + 1], bu1);
-                            y2[e] = __ffma2_rn(make_float2(cc.x, cc.y), h[2 * q], y2[e]);
-                            y2[e] = __ffma2_rn(make_float2(cc.z, cc.w), h[2 * q + 1], y2[e]);
+                            if (!SO) {
+                                const float4 cc = *reinterpret_cast<const float4 *>(sC + to);
+                                y2[e] = __ffma2_rn(make_float2(cc.x, cc.y), h[2 * q], y2[e]);
+                                y2[e] = __ffma2_rn(make_float2(cc.z, cc.w), h[2 * q + 1], y2[e]);
+                            }
                         }
                     }
+                    if (SO) continue;
                     // combine the R slices, transposed: lane sr ends with the
                     // complete outputs of timesteps tb + OWN sr .. + OWN - 1
                     float yv[8];
@@ -387,13 +406,11 @@ scan_fwd_pairs_kernel(const Params p) {
                 }
             }
             __syncwarp();
+            if (SO) continue;
             // the piece's last sub-chunk leaves the carried state: publish it
             // before this tile's stores, so the release waits on less
-            if (sub + 1 == nsub && se < p.subs_per_chain) {
-#pragma unroll
-                for (int k = 0; k < S / 4; ++k)
-                    __stcg(reinterpret_cast<float4 *>(carry) + k,
-                           make_float4(h[2 * k].x, h[2 * k].y, h[2 * k + 1].x, h[2 * k + 1].y));
+            if (publish_end && sub + 1 == nsub && se < p.subs_per_chain) {
+                store_carry(h);
                 publish_progress(p, lane, g, se);
             }
             // ---- coalesced store of the output tile
@@ -406,6 +423,47 @@ scan_fwd_pairs_kernel(const Params p) {
                                  *reinterpret_cast<const uint4 *>(outt + r * W::ROWB + c * 16));
             }
             __syncwarp();
+        }
+        };
+
+        float2 h[S / 2];
+#pragma unroll
+        for (int k = 0; k < S / 2; ++k) h[k] = make_float2(0.f, 0.f);
+        double dsum = 0.0;
+        if (two_phase && se < p.subs_per_chain) {
+            // The piece ends inside its group and other workers' pieces of the
+            // group wait for its end state.  Get that state first with a
+            // state-only run from a zero start, while the worker before it is
+            // still busy; then, with that worker's carry h_in (none when the
+            // piece starts the group): end = exp(A sum(delta)) h_in + local
+            // end, published at once.  The pieces of a group thus finish their
+            // waits one after the other in a few steps instead of running one
+            // after the other; the output run follows from h_in.
+            run_subs(true, h, dsum, false);
+            float2 hin[S / 2];
+#pragma unroll
+            for (int k = 0; k < S / 2; ++k) hin[k] = make_float2(0.f, 0.f);
+            if (sb > 0) {
+                if (!wait_progress(p, lane, g, sb)) return;
+                load_carry(hin);
+            }
+            float2 hend[S / 2];
+#pragma unroll
+            for (int k = 0; k < S / 2; ++k) {
+                const float2 decay = f2(ex2_mufu((float)((double)A2[k].x * dsum)),
+                                        ex2_mufu((float)((double)A2[k].y * dsum)));
+                hend[k] = __ffma2_rn(decay, hin[k], h[k]);
+                h[k] = hin[k];
+            }
+            store_carry(hend);
+            publish_progress(p, lane, g, se);
+            run_subs(false, h, dsum, false);
+        } else {
+            if (sb > 0) {
+                if (!wait_progress(p, lane, g, sb)) return;
+                load_carry(h);
+            }
+            run_subs(false, h, dsum, true);
         }
 
         if (se == p.subs_per_chain && p.last_state != nullptr && ds < Dm) {

@@ -156,6 +156,9 @@ def test_auto_plan_is_valid():
     # the Mamba-2.8B layer has enough channel groups for the persistent schedule
     w = inputs.MAMBA_2_8B
     assert binding.mamba_scan_plan(w.batch, w.dim, w.seqlen, w.dstate)[2] == binding.SCHEDULE_PERSISTENT
+    # the long-context layer has few groups but long sequences: two-phase pieces
+    w = inputs.LONG_CONTEXT
+    assert binding.mamba_scan_plan(w.batch, w.dim, w.seqlen, w.dstate)[:3:2] == (2, binding.SCHEDULE_PERSISTENT)
 
 
 # ------------------------------------------------------------ persistent schedule
@@ -210,6 +213,18 @@ def test_persistent_short_units(lanes, chunk):
     # not ready when claimed, so the workers mostly wait on one another
     check_full(inputs.custom(2, 96, 2048, 16, "bf16", seed=chunk + lanes),
                schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=lanes, chunk_timesteps=chunk)
+
+
+@pytest.mark.parametrize("lanes", [2, 4])
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("shape", [(1, 64, 16384), (1, 16, 16384), (2, 40, 6000)])
+def test_persistent_few_groups_long_sequences(lanes, dtype, shape):
+    # fewer channel groups than workers: every group is cut into many pieces
+    # that run at once (each from its own end state, then corrected by the
+    # carry of the piece before it)
+    b, d, L = shape
+    check_full(inputs.custom(b, d, L, 16, dtype, seed=d + L), schedule=binding.SCHEDULE_PERSISTENT,
+               lanes_per_channel=lanes)
 
 
 def test_persistent_rejects_unsupported():
