@@ -246,6 +246,7 @@ scan_fwd_pairs_kernel(const Params p) {
             bok[i] = n < N;
             boff[i] = bc0 + (int64_t)n * L + cx * V;
         }
+        bool so_stage = false;  // state-only run: no z or C rows to stage
         auto issue = [&](int sub, int st) {
             unsigned char *sbuf = base + st * W::STAGE + cx * 16;
             const int64_t t0 = tb0 + (int64_t)sub * kTC;
@@ -258,7 +259,7 @@ scan_fwd_pairs_kernel(const Params p) {
                     const int64_t off = ok ? xoff[i] + t0 : 0;
                     cp16(sbuf + (0 * CW + r) * W::ROWB, gu + off, ok);
                     cp16(sbuf + (1 * CW + r) * W::ROWB, gd + off, ok);
-                    if (GATE) cp16(sbuf + (2 * CW + r) * W::ROWB, gz + off, ok);
+                    if (GATE && !so_stage) cp16(sbuf + (2 * CW + r) * W::ROWB, gz + off, ok);
                 }
             }
 #pragma unroll
@@ -267,7 +268,7 @@ scan_fwd_pairs_kernel(const Params p) {
                 const int n = ((lane + 32 * i) % (kNS * CPR)) / CPR;
                 const bool ok = bok[i] && tok;
                 const int64_t off = ok ? boff[i] + t0 : 0;
-                cp16(sbuf + (3 * CW + which * kNS + n) * W::ROWB, (which ? gC : gB) + off, ok);
+                if (!(so_stage && which)) cp16(sbuf + (3 * CW + which * kNS + n) * W::ROWB, (which ? gC : gB) + off, ok);
             }
             cp_commit();
         };
@@ -276,6 +277,7 @@ scan_fwd_pairs_kernel(const Params p) {
         // -- no C rows, readout, gate or stores -- and sum delta into dsum;
         // full runs publish the carried state at the end when `publish_end`.
         auto run_subs = [&](const bool SO, float2 (&h)[S / 2], double &dsum, bool publish_end) {
+        so_stage = SO;
         issue(0, 0);
 #pragma unroll 1
         for (int sub = 0; sub < nsub; ++sub) {
@@ -368,7 +370,12 @@ scan_fwd_pairs_kernel(const Params p) {
                             const float2 x0 = __fmul2_rn(dl2, A2[2 * q]);
                             const float2 x1 = __fmul2_rn(dl2, A2[2 * q + 1]);
                             const float2 a0 = make_float2(ex2_mufu(x0.x), ex2_mufu(x0.y));
-                            const float2 a1 = make_float2(ex2_mufu(x1.x), ex2_mufu(x1.y));
+                            // state-only runs lean harder on the MUFU (no readout or
+                            // gate work beside it): one decay pair in eight goes
+                            // to the FMA-pipe exp2 there
+                            float2 a1;
+                            if (SO && q == S / 4 - 1 && (e & 1) == 0) a1 = ex2_poly2(x1);
+                            else a1 = make_float2(ex2_mufu(x1.x), ex2_mufu(x1.y));
                             const float2 bu0 = __fmul2_rn(du2, make_float2(bb.x, bb.y));
                             const float2 bu1 = __fmul2_rn(du2, make_float2(bb.z, bb.w));
                             h[2 * q] = __ffma2_rn(a0, h[2 * q], bu0);
