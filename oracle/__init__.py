@@ -11,6 +11,8 @@ marshals numpy/torch CPU arrays into it:
 
 * :func:`scan` -- the whole forward scan (optionally from an initial state).
 * :func:`state_update` -- one recurrent step for every (batch, channel).
+* :func:`conv1d`, :func:`conv1d_update` -- the causal depthwise convolution
+  (+ bias, + silu) that feeds the scan, whole-sequence and one token.
 * :func:`softplus`, :func:`silu` -- the pointwise functions the oracle uses.
 
 Inputs may be numpy arrays or CPU torch tensors of any float dtype; they are
@@ -44,6 +46,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.s6_oracle_state_update.argtypes = [f64p, f32p, f32p, f32p, f32p, f32p,
                                            f32p, f32p, f32p, ctypes.c_int, f64p,
                                            i64, i64, i64]
+    lib.s6_oracle_conv1d.restype = ctypes.c_int
+    lib.s6_oracle_conv1d.argtypes = [f32p, f32p, f32p, ctypes.c_int, f64p, i64, i64, i64, i64, i64]
+    lib.s6_oracle_conv1d_update.restype = ctypes.c_int
+    lib.s6_oracle_conv1d_update.argtypes = [f64p, f32p, f32p, f32p, ctypes.c_int, f64p, i64, i64, i64]
     lib.s6_oracle_softplus.restype = ctypes.c_double
     lib.s6_oracle_softplus.argtypes = [ctypes.c_double]
     lib.s6_oracle_silu.restype = ctypes.c_double
@@ -139,6 +145,47 @@ def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
                                     _p64(out), batch, dim, N)
     if rc != 0:
         raise RuntimeError(f"s6_oracle_state_update failed with code {rc}")
+    return out, st
+
+
+def conv1d(x, weight, bias=None, silu: bool = True, dim: Optional[int] = None,
+           lib: Optional[ctypes.CDLL] = None) -> np.ndarray:
+    """Causal depthwise convolution + bias (+ silu) in fp64.
+
+    x: (batch, C, L) with C >= dim (the first ``dim`` channel rows are used,
+    as when x is the x half of a (batch, 2 * dim, L) projection output);
+    weight (dim, K); bias (dim,).  Returns (batch, dim, L) fp64.
+    """
+    lib = lib or _get()
+    x, weight, bias = _f32(x), _f32(weight), _f32(bias)
+    batch, C, L = x.shape
+    dim = dim or C
+    K = weight.shape[1]
+    assert weight.shape == (dim, K) and C >= dim and (bias is None or bias.shape == (dim,))
+    out = np.empty((batch, dim, L), dtype=np.float64)
+    rc = lib.s6_oracle_conv1d(_p32(x), _p32(weight), _p32(bias), int(bool(silu)), _p64(out),
+                              batch, dim, L, K, C * L)
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_conv1d failed with code {rc}")
+    return out
+
+
+def conv1d_update(state, x, weight, bias=None, silu: bool = True,
+                  lib: Optional[ctypes.CDLL] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """One token of :func:`conv1d`.  state (batch, dim, K-1), oldest input
+    first; x (batch, dim).  Returns ``(out, new_state)`` in fp64; ``state`` is
+    not modified."""
+    lib = lib or _get()
+    st = _f64(state).copy()
+    x, weight, bias = _f32(x), _f32(weight), _f32(bias)
+    batch, dim = x.shape
+    K = weight.shape[1]
+    assert st.shape == (batch, dim, K - 1) and weight.shape == (dim, K)
+    out = np.empty((batch, dim), dtype=np.float64)
+    rc = lib.s6_oracle_conv1d_update(_p64(st), _p32(x), _p32(weight), _p32(bias), int(bool(silu)),
+                                     _p64(out), batch, dim, K)
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_conv1d_update failed with code {rc}")
     return out, st
 
 

@@ -31,6 +31,10 @@
  *                                                     projection)
  *   last_state[b,d,n] = h_{L-1}[n]
  *
+ * and, for the step before the scan in the same block, the causal depthwise
+ * convolution with bias and silu that produces u (s6_oracle_conv1d, and its
+ * one-token form s6_oracle_conv1d_update; equations beside them).
+ *
  * Layouts (row-major, contiguous):
  *   u, delta_raw, z, out : (batch, dim, seqlen)
  *   B, C                 : (batch, dstate, seqlen)
@@ -184,6 +188,76 @@ int s6_oracle_scan(const float *u, const float *delta, const float *A,
     free(jobs);
     free(tids);
     return rc;
+}
+
+/* Causal depthwise convolution over time with bias and optional silu: the
+ * step before the scan in the block of the page "Mamba SSM concept and
+ * implementation in Keras and TensorFlow" (MambaBlock: a Conv1D with one
+ * group per channel, channels-first, causal padding, bias, cut to the input
+ * length, then swish):
+ *   v[b,d,t]   = bias[d] + sum_{k=0}^{K-1} w[d,k] * x[b,d,t-(K-1)+k],
+ *                x[b,d,t] = 0 for t < 0 (the causal padding)
+ *   out[b,d,t] = silu(v[b,d,t]) if the flag is set, else v[b,d,t]
+ * x rows of batch row b start at b * x_batch_stride (dim * seqlen for a
+ * contiguous tensor; larger when x is the first part of a wider tensor, as
+ * the x half of the input projection's output is); w is (dim, K) row-major;
+ * out is contiguous (batch, dim, seqlen).  The sum starts from the bias and
+ * adds k = 0 .. K-1 in order. */
+int s6_oracle_conv1d(const float *x, const float *w, const float *bias, int silu,
+                     double *out, int64_t batch, int64_t dim, int64_t seqlen,
+                     int64_t width, int64_t x_batch_stride)
+{
+    if (!x || !w || !out || batch <= 0 || dim <= 0 || seqlen <= 0 || width <= 0)
+        return -1;
+    if (x_batch_stride < dim * seqlen)
+        return -1;
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < dim; ++d) {
+            const float *xr = x + b * x_batch_stride + d * seqlen;
+            const float *wr = w + d * width;
+            double *o = out + (b * dim + d) * seqlen;
+            for (int64_t t = 0; t < seqlen; ++t) {
+                double v = bias ? (double)bias[d] : 0.0;
+                for (int64_t k = 0; k < width; ++k) {
+                    const int64_t s = t - (width - 1) + k;
+                    if (s >= 0)
+                        v += (double)wr[k] * (double)xr[s];
+                }
+                o[t] = silu ? s6_oracle_silu(v) : v;
+            }
+        }
+    }
+    return 0;
+}
+
+/* One token of the same convolution, for decoding.  state (batch, dim, K-1)
+ * holds each row's last K-1 inputs, oldest first (zeros before the sequence
+ * starts); the token's input x[b,d] is the newest.  The output is formed as
+ * in s6_oracle_conv1d (bias, then k = 0 .. K-1 over the K inputs oldest
+ * first), then the state drops its oldest input and appends x[b,d]. */
+int s6_oracle_conv1d_update(double *state, const float *x, const float *w,
+                            const float *bias, int silu, double *out,
+                            int64_t batch, int64_t dim, int64_t width)
+{
+    if (!state || !x || !w || !out || batch <= 0 || dim <= 0 || width <= 0)
+        return -1;
+    const int64_t S = width - 1;
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < dim; ++d) {
+            double *st = state + (b * dim + d) * S;
+            const float *wr = w + d * width;
+            const double xt = (double)x[b * dim + d];
+            double v = bias ? (double)bias[d] : 0.0;
+            for (int64_t k = 0; k < width; ++k)
+                v += (double)wr[k] * (k < S ? st[k] : xt);
+            out[b * dim + d] = silu ? s6_oracle_silu(v) : v;
+            for (int64_t k = 0; k + 1 < S; ++k)
+                st[k] = st[k + 1];
+            if (S > 0)
+                st[S - 1] = xt;
+        }
+    }
+    return 0;
 }
 
 /* One recurrent step for every (b, d): the same update as one iteration of

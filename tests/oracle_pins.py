@@ -377,9 +377,104 @@ def pin_gate_and_softplus_flags(lib):
     _close(o[0, :, 0], y, rtol=1e-14, what="softplus off out")
 
 
+# ------------------------------------------------------------ convolution
+# The causal depthwise Conv1D (+ bias, + swish) of MambaBlock on the same
+# page: channels-first, one group per channel, causal padding.
+
+def _conv_inputs(rng, batch, dim, L, K):
+    x = rng.standard_normal((batch, dim, L)).astype(np.float32)
+    w = rng.standard_normal((dim, K)).astype(np.float32)
+    bias = rng.standard_normal(dim).astype(np.float32)
+    return x, w, bias
+
+
+def pin_conv_numpy(lib):
+    """silu off: every row is numpy.convolve of the row with the reversed
+    kernel (causal padding = the first L terms of the full convolution) plus
+    the bias."""
+    rng = np.random.default_rng(101)
+    for K in (1, 2, 3, 4):
+        x, w, bias = _conv_inputs(rng, 2, 5, 37, K)
+        got = oracle.conv1d(x, w, bias, silu=False, lib=lib)
+        exp = np.empty_like(got)
+        for b in range(2):
+            for d in range(5):
+                full = np.convolve(x[b, d].astype(np.float64), w[d, ::-1].astype(np.float64))
+                exp[b, d] = full[:37] + float(bias[d])
+        _close(got, exp, rtol=1e-14, what=f"conv vs numpy K={K}")
+
+
+def pin_conv_impulse(lib):
+    """A unit impulse at t0 gives back the kernel, newest tap first, on top of
+    the bias, and only the bias elsewhere."""
+    K, L, t0 = 4, 12, 5
+    x = np.zeros((1, 3, L), dtype=np.float32)
+    x[:, :, t0] = 1.0
+    w = (np.arange(12, dtype=np.float32).reshape(3, 4) + 1.0) * 0.25
+    bias = np.array([0.5, -1.0, 2.0], dtype=np.float32)
+    got = oracle.conv1d(x, w, bias, silu=False, lib=lib)
+    exp = np.repeat(bias.astype(np.float64)[:, None], L, axis=1)[None]
+    for d in range(3):
+        for j in range(K):
+            exp[0, d, t0 + j] += w[d, K - 1 - j]
+    assert np.array_equal(got, exp), "impulse response"
+
+
+def pin_conv_silu(lib):
+    """silu on: z * expit(z) of the silu-off result (scipy)."""
+    rng = np.random.default_rng(102)
+    x, w, bias = _conv_inputs(rng, 2, 4, 29, 4)
+    v = oracle.conv1d(x, w, bias, silu=False, lib=lib)
+    got = oracle.conv1d(x, w, bias, silu=True, lib=lib)
+    _close(got, v * special.expit(v), rtol=1e-14, what="conv silu")
+
+
+def pin_conv_wide_input(lib):
+    """x as the first dim channel rows of a (batch, 2 dim, L) tensor (the x
+    half of the input projection) gives the same as a contiguous x."""
+    rng = np.random.default_rng(103)
+    xz, w, bias = _conv_inputs(rng, 3, 8, 21, 3)
+    w, bias = w[:4], bias[:4]
+    got = oracle.conv1d(xz, w, bias, silu=True, dim=4, lib=lib)
+    ref = oracle.conv1d(np.ascontiguousarray(xz[:, :4]), w, bias, silu=True, lib=lib)
+    assert np.array_equal(got, ref), "wide input"
+    # and the other rows do matter when they are the ones selected
+    other = oracle.conv1d(np.ascontiguousarray(xz[:, 4:]), w, bias, silu=True, lib=lib)
+    assert not np.allclose(got, other)
+
+
+def pin_conv_update_stream(lib):
+    """One-token updates from a zero state reproduce the whole-sequence
+    convolution bit for bit (same summation order)."""
+    rng = np.random.default_rng(104)
+    for K in (1, 2, 4):
+        x, w, bias = _conv_inputs(rng, 2, 3, 15, K)
+        ref = oracle.conv1d(x, w, bias, silu=True, lib=lib)
+        st = np.zeros((2, 3, K - 1))
+        for t in range(15):
+            o, st = oracle.conv1d_update(st, x[:, :, t], w, bias, silu=True, lib=lib)
+            assert np.array_equal(o, ref[:, :, t]), f"step {t}, K={K}"
+        if K > 1:
+            assert np.array_equal(st, x[:, :, 15 - (K - 1):].astype(np.float64)), "final state"
+
+
+def pin_conv_causality(lib):
+    """Changing x at t* changes no output before t* and the output at t*."""
+    rng = np.random.default_rng(105)
+    x, w, bias = _conv_inputs(rng, 1, 4, 20, 4)
+    a = oracle.conv1d(x, w, bias, silu=True, lib=lib)
+    x2 = x.copy()
+    x2[:, :, 11] += 3.0
+    b = oracle.conv1d(x2, w, bias, silu=True, lib=lib)
+    assert np.array_equal(a[:, :, :11], b[:, :, :11])
+    assert np.all(a[:, :, 11] != b[:, :, 11])
+
+
 ALL_PINS = [pin_softplus_silu, pin_geometric_series, pin_lti_convolution,
             pin_first_order_iir, pin_zero_step_keeps_state, pin_memoryless_limit,
             pin_brute_force_products, pin_cumsum_form, pin_chunk_split,
             pin_steps_equal_scan, pin_causality, pin_linearity,
             pin_shared_bc_and_independence, pin_zero_b_or_c,
-            pin_gate_and_softplus_flags]
+            pin_gate_and_softplus_flags,
+            pin_conv_numpy, pin_conv_impulse, pin_conv_silu, pin_conv_wide_input,
+            pin_conv_update_stream, pin_conv_causality]

@@ -42,6 +42,19 @@ MUTANTS = [
     ("silu-sigmoid-only", "return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));"),
     ("state-update-C-lag", "y += (double)C[b * N + n] * h[n];", "y += (double)C[b * N + n] * (h[n] - Bbar_u);"),
     ("last-state-off-by-one", "j->last_state[row * N + n] = h[n];", "j->last_state[row * N + n] = h[n] * 0.5;"),
+    # causal depthwise convolution
+    ("conv-kernel-flipped", "v += (double)wr[k] * (double)xr[s];", "v += (double)wr[width - 1 - k] * (double)xr[s];"),
+    ("conv-off-by-one", "const int64_t s = t - (width - 1) + k;", "const int64_t s = t - width + k;"),
+    ("conv-centred-padding", "const int64_t s = t - (width - 1) + k;\n                    if (s >= 0)",
+     "const int64_t s = t - (width - 1) / 2 + k;\n                    if (s >= 0 && s < seqlen)"),
+    ("conv-bias-dropped", "double v = bias ? (double)bias[d] : 0.0;\n                for",
+     "double v = 0.0;\n                for"),
+    ("conv-silu-dropped", "o[t] = silu ? s6_oracle_silu(v) : v;", "o[t] = v;"),
+    ("conv-stride-ignored", "const float *xr = x + b * x_batch_stride + d * seqlen;",
+     "const float *xr = x + b * dim * seqlen + d * seqlen;"),
+    ("conv-update-no-shift", "st[k] = st[k + 1];", "st[k] = st[k];"),
+    ("conv-update-newest-first", "v += (double)wr[k] * (k < S ? st[k] : xt);",
+     "v += (double)wr[k] * (k == 0 ? xt : st[k - 1]);"),
 ]
 
 
