@@ -384,6 +384,36 @@ def decode_measure(steps=256):
                                    "timed alone with events (includes launch latency)"}}
 
 
+def conv1d_measure(reps=20):
+    """The causal depthwise conv1d (+ bias + silu) that produces u, on the
+    benchmark layer's shape: x = the first 5120 channel rows of a
+    (4, 10240, 4096) bf16 projection output, width 4.  HBM-bound stream:
+    x read once (168 MB) and out written once (168 MB) per call."""
+    w = inputs.MAMBA_2_8B
+    K = 4
+    d = inputs.conv_inputs(w.batch, w.dim, w.seqlen, K, w.dtype, seed=44, device="cuda")
+    out = torch.empty(w.batch, w.dim, w.seqlen, device="cuda", dtype=inputs.DTYPES[w.dtype])
+    run = lambda: binding.mamba_conv1d_fwd(d["xz"], d["weight"], d["bias"], dim=w.dim, out=out)  # noqa: E731
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    es = 2 if w.dtype == "bf16" else 4
+    nbytes = 2 * w.batch * w.dim * w.seqlen * es + w.dim * (K + 1) * 4
+    hbm = load_peaks()["hbm_gbs"]
+    return {"workload": f"conv1d K={K} {w.batch}x{w.dim}x{w.seqlen} {w.dtype} (x half of a 2x-wide input)",
+            "us_per_call": us, "Gelem_per_s": w.elements / us / 1e3,
+            "roofline": {"bound": "hbm", "achieved": nbytes / us / 1e3, "peak": hbm, "unit": "GB/s",
+                         "frac": nbytes / us / 1e3 / hbm, "algorithmic_bytes": nbytes},
+            "reps": reps, "l2": "inputs larger than L2, no flush"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -393,6 +423,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-conv", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -486,6 +517,8 @@ def main():
                        "path": "pinned host -> device copies, mamba_scan_fwd, device -> host out + last_state"}
     if rank == 0 and not args.no_decode:
         line["decode"] = decode_measure()
+    if rank == 0 and not args.no_conv:
+        line["conv1d"] = conv1d_measure()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:

@@ -240,6 +240,59 @@ int mamba_state_update(float *state, const void *u, const void *delta,
                        int64_t dim, int64_t dstate, int act_dtype,
                        cudaStream_t stream);
 
+/*
+ * mamba_conv1d_fwd -- the step that produces the scan's input u: a causal
+ * depthwise convolution over time with a bias, then silu ("Mamba SSM concept
+ * and implementation in Keras and TensorFlow", MambaBlock: a Conv1D with one
+ * group per channel, channels-first, causal padding and a bias, cut to the
+ * input length, then swish).  With K = width:
+ *
+ *   v[b,d,t]   = bias[d] + sum_{k=0}^{K-1} weight[d,k] * x[b,d,t-(K-1)+k],
+ *                x[b,d,t] = 0 for t < 0
+ *   out[b,d,t] = silu(v) if apply_silu, else v
+ *
+ *   x            : act; channel d of batch row b is the seqlen-long row at
+ *                  x + b * x_batch_stride + d * seqlen (elements).
+ *                  x_batch_stride = 0 means dim * seqlen (contiguous); a
+ *                  larger stride takes x as the first dim channel rows of a
+ *                  wider tensor, such as the x half of the input
+ *                  projection's (batch, 2 dim, seqlen) output.
+ *   weight       : fp32 (dim, width), width 1 .. 4.
+ *   bias         : fp32 (dim) or NULL.
+ *   out          : act (batch, dim, seqlen), contiguous, written; must not
+ *                  overlap x.
+ *
+ * 16-byte-aligned x / out with seqlen and x_batch_stride multiples of 8
+ * (bf16) or 4 (fp32) take the vector path; anything else a scalar one.
+ * Returns MAMBA_OK or a mamba_status_t error (MAMBA_ERR_UNSUPPORTED for a
+ * width outside 1 .. 4, MAMBA_ERR_SHAPE for a stride below dim * seqlen).
+ */
+int mamba_conv1d_fwd(const void *x, const float *weight, const float *bias,
+                     int apply_silu, void *out, int64_t batch, int64_t dim,
+                     int64_t seqlen, int64_t width, int64_t x_batch_stride,
+                     int act_dtype, cudaStream_t stream);
+
+/*
+ * mamba_conv1d_update -- one token of mamba_conv1d_fwd, for decoding.
+ *
+ *   conv_state   : fp32 (batch, dim, width - 1): each row's last width - 1
+ *                  inputs, oldest first (zeros before the sequence starts);
+ *                  read, then shifted by one with the token's input
+ *                  appended.  Unused (may be NULL) when width is 1.
+ *   x            : act (batch, dim); row b at x + b * x_batch_stride
+ *                  (0 means dim).
+ *   weight, bias : as for mamba_conv1d_fwd.
+ *   out          : act (batch, dim), written; must not overlap x or the state.
+ *
+ * A run of calls from a zero state equals mamba_conv1d_fwd over the tokens.
+ * Returns MAMBA_OK or a mamba_status_t error.
+ */
+int mamba_conv1d_update(float *conv_state, const void *x, const float *weight,
+                        const float *bias, int apply_silu, void *out,
+                        int64_t batch, int64_t dim, int64_t width,
+                        int64_t x_batch_stride, int act_dtype,
+                        cudaStream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char *mamba_status_string(int status);
 

@@ -30,8 +30,8 @@ SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT = 0, 1, 2
 # Every function include/mamba_scan.h declares.
 EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
-            "mamba_scan_fwd_noalloc", "mamba_state_update", "mamba_status_string",
-            "mamba_abi_version")
+            "mamba_scan_fwd_noalloc", "mamba_state_update", "mamba_conv1d_fwd",
+            "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version")
 
 
 class MambaError(RuntimeError):
@@ -69,6 +69,10 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_state_update.argtypes = [fp, vp, vp, fp, vp, vp, fp, vp, fp, ci, vp,
                                        i64, i64, i64, ci, vp]
     lib.mamba_state_update.restype = ci
+    lib.mamba_conv1d_fwd.argtypes = [vp, fp, fp, ci, vp, i64, i64, i64, i64, i64, ci, vp]
+    lib.mamba_conv1d_fwd.restype = ci
+    lib.mamba_conv1d_update.argtypes = [fp, vp, fp, fp, ci, vp, i64, i64, i64, i64, ci, vp]
+    lib.mamba_conv1d_update.restype = ci
     lib.mamba_status_string.argtypes = [ci]
     lib.mamba_status_string.restype = ctypes.c_char_p
     lib.mamba_abi_version.argtypes = []
@@ -251,4 +255,75 @@ def mamba_state_update(state: torch.Tensor, u: torch.Tensor, delta: torch.Tensor
                                     int(bool(delta_softplus)), _ptr(out), batch, dim, N,
                                     _ACT[act], _stream(dev))
     _check("mamba_state_update", rc)
+    return out
+
+
+def mamba_conv1d_fwd(x: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                     apply_silu: bool = True, dim: Optional[int] = None,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Causal depthwise conv1d + bias (+ silu) on the current CUDA stream.
+
+    x: contiguous (batch, C, L) with C >= dim; the first ``dim`` channel rows
+    are convolved (``dim`` defaults to C), so the x half of a (batch, 2 dim, L)
+    projection output can be passed as is.  weight: (dim, K) fp32, K <= 4;
+    bias: (dim,) fp32.  Returns out (batch, dim, L) in x's dtype."""
+    if x.dim() != 3:
+        raise ValueError("x must be (batch, channels, L)")
+    batch, C, L = x.shape
+    dim = C if dim is None else int(dim)
+    dev, act = x.device, x.dtype
+    if dev.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    if act not in _ACT:
+        raise TypeError(f"unsupported activation dtype {act}")
+    if not x.is_contiguous() or dim > C:
+        raise ValueError("x must be contiguous with at least dim channel rows")
+    if weight.dim() != 2:
+        raise ValueError("weight must be (dim, width)")
+    K = weight.shape[1]
+    _need(weight, "weight", dev, torch.float32, (dim, K))
+    _need(bias, "bias", dev, torch.float32, (dim,))
+    if out is None:
+        out = torch.empty(batch, dim, L, device=dev, dtype=act)
+    _need(out, "out", dev, act, (batch, dim, L))
+    lib = load_library()
+    with torch.cuda.device(dev):
+        rc = lib.mamba_conv1d_fwd(_ptr(x), _ptr(weight), _ptr(bias), int(bool(apply_silu)), _ptr(out),
+                                  batch, dim, L, K, C * L, _ACT[act], _stream(dev))
+    _check("mamba_conv1d_fwd", rc)
+    return out
+
+
+def mamba_conv1d_update(conv_state: Optional[torch.Tensor], x: torch.Tensor, weight: torch.Tensor,
+                        bias: Optional[torch.Tensor] = None, apply_silu: bool = True,
+                        out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One token of :func:`mamba_conv1d_fwd`.  conv_state: (batch, dim, K-1)
+    fp32, oldest input first, updated in place (None when K is 1); x:
+    (batch, dim).  Returns out (batch, dim)."""
+    if x.dim() != 2:
+        raise ValueError("x must be (batch, dim)")
+    batch, dim = x.shape
+    dev, act = x.device, x.dtype
+    if dev.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    if act not in _ACT:
+        raise TypeError(f"unsupported activation dtype {act}")
+    if weight.dim() != 2:
+        raise ValueError("weight must be (dim, width)")
+    K = weight.shape[1]
+    _need(x, "x", dev, act, (batch, dim))
+    _need(weight, "weight", dev, torch.float32, (dim, K))
+    _need(bias, "bias", dev, torch.float32, (dim,))
+    if K > 1 and conv_state is None:
+        raise ValueError("conv_state is required for width > 1")
+    _need(conv_state, "conv_state", dev, torch.float32, (batch, dim, K - 1))
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, "out", dev, act, (batch, dim))
+    lib = load_library()
+    with torch.cuda.device(dev):
+        rc = lib.mamba_conv1d_update(_ptr(conv_state), _ptr(x), _ptr(weight), _ptr(bias),
+                                     int(bool(apply_silu)), _ptr(out), batch, dim, K, dim,
+                                     _ACT[act], _stream(dev))
+    _check("mamba_conv1d_update", rc)
     return out

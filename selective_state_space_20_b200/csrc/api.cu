@@ -252,6 +252,60 @@ int mamba_state_update(float *state, const void *u, const void *delta, const flo
     return mscan::launch_state_update(a, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 
+int mamba_conv1d_fwd(const void *x, const float *weight, const float *bias, int apply_silu,
+                     void *out, int64_t batch, int64_t dim, int64_t seqlen, int64_t width,
+                     int64_t x_batch_stride, int act_dtype, cudaStream_t stream) {
+    if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
+    int rc = check_sizes(batch, dim, seqlen, 1);
+    if (rc != MAMBA_OK) return rc;
+    if (width < 1 || width > 4) return MAMBA_ERR_UNSUPPORTED;
+    if (!x || !weight || !out) return MAMBA_ERR_NULL;
+    if (x_batch_stride == 0) x_batch_stride = dim * seqlen;
+    if (x_batch_stride < dim * seqlen || x_batch_stride > kMaxElems) return MAMBA_ERR_SHAPE;
+    if ((double)batch * (double)x_batch_stride > (double)kMaxElems) return MAMBA_ERR_SHAPE;
+    const size_t es = act_size(act_dtype);
+    const size_t nout = (size_t)(batch * dim * seqlen) * es;
+    const size_t nx = (size_t)((batch - 1) * x_batch_stride + dim * seqlen) * es;
+    if (overlaps(out, nout, x, nx) || overlaps(out, nout, weight, (size_t)(dim * width) * 4) ||
+        overlaps(out, nout, bias, (size_t)dim * 4))
+        return MAMBA_ERR_OVERLAP;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MAMBA_ERR_DEVICE;
+    mscan::Conv1dArgs a;
+    a.x = x; a.weight = weight; a.bias = bias; a.out = out;
+    a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.x_batch_stride = x_batch_stride;
+    a.width = (int)width; a.silu = apply_silu ? 1 : 0; a.act = act_dtype;
+    return mscan::launch_conv1d_fwd(a, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
+int mamba_conv1d_update(float *conv_state, const void *x, const float *weight, const float *bias,
+                        int apply_silu, void *out, int64_t batch, int64_t dim, int64_t width,
+                        int64_t x_batch_stride, int act_dtype, cudaStream_t stream) {
+    if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
+    int rc = check_sizes(batch, dim, 1, 1);
+    if (rc != MAMBA_OK) return rc;
+    if (width < 1 || width > 4) return MAMBA_ERR_UNSUPPORTED;
+    if (!x || !weight || !out || (width > 1 && !conv_state)) return MAMBA_ERR_NULL;
+    if (x_batch_stride == 0) x_batch_stride = dim;
+    if (x_batch_stride < dim || x_batch_stride > kMaxElems) return MAMBA_ERR_SHAPE;
+    const size_t es = act_size(act_dtype);
+    const size_t nout = (size_t)(batch * dim) * es;
+    const size_t nx = (size_t)((batch - 1) * x_batch_stride + dim) * es;
+    const size_t ns = (size_t)(batch * dim * (width - 1)) * 4;
+    if (overlaps(out, nout, x, nx) || overlaps(out, nout, conv_state, ns) ||
+        overlaps(out, nout, weight, (size_t)(dim * width) * 4) || overlaps(out, nout, bias, (size_t)dim * 4) ||
+        overlaps(conv_state, ns, x, nx) || overlaps(conv_state, ns, weight, (size_t)(dim * width) * 4) ||
+        overlaps(conv_state, ns, bias, (size_t)dim * 4))
+        return MAMBA_ERR_OVERLAP;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MAMBA_ERR_DEVICE;
+    mscan::Conv1dUpdateArgs a;
+    a.state = conv_state; a.x = x; a.weight = weight; a.bias = bias; a.out = out;
+    a.batch = batch; a.dim = dim; a.x_batch_stride = x_batch_stride;
+    a.width = (int)width; a.silu = apply_silu ? 1 : 0; a.act = act_dtype;
+    return mscan::launch_conv1d_update(a, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
 const char *mamba_status_string(int status) {
     switch (status) {
         case MAMBA_OK: return "ok";
@@ -268,6 +322,6 @@ const char *mamba_status_string(int status) {
     }
 }
 
-int mamba_abi_version(void) { return (1 << 16) | 0; }
+int mamba_abi_version(void) { return (1 << 16) | 1; }
 
 }  // extern "C"

@@ -1,0 +1,204 @@
+// conv1d.cu -- causal depthwise convolution over time, plus bias and silu:
+// the step that turns the x half of the input projection into the scan's
+// input u ("Mamba SSM concept and implementation in Keras and TensorFlow",
+// MambaBlock: a Conv1D with one group per channel, channels-first, causal
+// padding and a bias, cut to the input length, then swish):
+//   v[b,d,t]   = bias[d] + sum_{k<K} w[d,k] * x[b,d,t-(K-1)+k],  x = 0 for t < 0
+//   out[b,d,t] = silu(v) if requested, else v
+// and its one-token form for decoding, which keeps each row's last K-1
+// inputs as a state.
+//
+// The sequence kernel is a pure stream: 2 (bf16) or 4 (fp32) bytes read and
+// written per element, so it is bound by HBM.  A warp covers four tiles of
+// 32 consecutive 16-byte chunks of one row (1024 bf16 / 512 fp32 timesteps)
+// with one load and one store per lane and tile; the K-1 inputs before a
+// lane's chunk come from the lane before it by shuffle (at the span's start
+// lane 0 reads them from memory), so every input byte is read once.  Rows that are not 16-byte aligned or whose length is not a
+// whole number of chunks take a one-thread-per-output kernel.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "device_math.cuh"
+#include "internal.h"
+
+namespace mscan {
+namespace {
+
+struct ConvParams {
+    const void *x;
+    const float *w, *bias;
+    void *out;
+    int64_t batch, dim, seqlen, x_batch_stride;
+    int width, silu;
+};
+
+template <typename T>
+__device__ __forceinline__ float load_elem(const T *p) { return Elem<T>::load(p); }
+
+// One warp per NT consecutive 32-chunk tiles of one row: every lane issues
+// its NT 16-byte loads first (NT x 512 bytes in flight per warp), then the
+// tiles are finished in order, each taking the inputs before a lane's chunk
+// from the lane before it, and lane 0 from lane 31 of the previous tile.
+template <typename T, int K, int NT>
+__global__ void __launch_bounds__(256) conv1d_tiles_kernel(const ConvParams p) {
+    constexpr int V = 16 / (int)sizeof(T);  // elements per 16-byte chunk
+    constexpr int TILE = 32 * V;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t spans_per_row = (p.seqlen + NT * TILE - 1) / (NT * TILE);
+    const int64_t row = warp / spans_per_row;
+    if (row >= p.batch * p.dim) return;  // whole warp leaves together
+    const int64_t b = row / p.dim, d = row % p.dim;
+    const int64_t span0 = (warp % spans_per_row) * (NT * TILE);
+    const T *xr = static_cast<const T *>(p.x) + b * p.x_batch_stride + d * p.seqlen;
+    T *orow = static_cast<T *>(p.out) + row * p.seqlen;
+
+    uint4 raw[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        const int64_t t0 = span0 + j * TILE + (int64_t)lane * V;
+        raw[j] = t0 < p.seqlen ? ldg16_stream(xr + t0) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float carry[K];  // lane 0: the K-1 inputs before the span
+#pragma unroll
+    for (int k = 0; k < K - 1; ++k) {
+        const int64_t s = span0 - (K - 1) + k;
+        carry[k] = (lane == 0 && s >= 0) ? load_elem(xr + s) : 0.f;
+    }
+    float wk[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) wk[k] = __ldg(p.w + d * K + k);
+    const float bias = p.bias ? __ldg(p.bias + d) : 0.f;
+
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        const int64_t t0 = span0 + j * TILE + (int64_t)lane * V;
+        float f[V + K - 1];  // K-1 earlier inputs, then this chunk
+        Elem<T>::unpack(raw[j], f + K - 1);
+#pragma unroll
+        for (int k = 0; k < K - 1; ++k) {
+            const float prev = __shfl_up_sync(0xffffffffu, f[V + k], 1);
+            const float last = __shfl_sync(0xffffffffu, f[V + k], 31);  // for the next tile
+            f[k] = lane > 0 ? prev : carry[k];
+            carry[k] = last;
+        }
+        if (t0 < p.seqlen) {  // seqlen is a whole number of chunks
+            float o[V];
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                float v = bias;
+#pragma unroll
+                for (int k = 0; k < K; ++k) v = fmaf(wk[k], f[i + k], v);
+                o[i] = p.silu ? silu_f(v) : v;
+            }
+            stg16_stream(orow + t0, Elem<T>::pack(o));
+        }
+    }
+}
+
+// Any alignment and length: one thread per output.
+template <typename T>
+__global__ void __launch_bounds__(256) conv1d_scalar_kernel(const ConvParams p) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= p.batch * p.dim * p.seqlen) return;
+    const int64_t t = i % p.seqlen, row = i / p.seqlen;
+    const int64_t b = row / p.dim, d = row % p.dim;
+    const T *xr = static_cast<const T *>(p.x) + b * p.x_batch_stride + d * p.seqlen;
+    float v = p.bias ? __ldg(p.bias + d) : 0.f;
+    for (int k = 0; k < p.width; ++k) {
+        const int64_t s = t - (p.width - 1) + k;
+        if (s >= 0) v = fmaf(__ldg(p.w + d * p.width + k), load_elem(xr + s), v);
+    }
+    Elem<T>::store(static_cast<T *>(p.out) + i, p.silu ? silu_f(v) : v);
+}
+
+struct ConvUpdateParams {
+    float *state;
+    const void *x;
+    const float *w, *bias;
+    void *out;
+    int64_t batch, dim, x_batch_stride;
+    int width, silu;
+};
+
+// One thread per (batch, channel): read the K-1 kept inputs and the token,
+// emit the output, shift the kept inputs.
+template <typename T, int K>
+__global__ void __launch_bounds__(256) conv1d_update_kernel(const ConvUpdateParams p) {
+    const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (row >= p.batch * p.dim) return;
+    const int64_t b = row / p.dim, d = row % p.dim;
+    constexpr int S = K - 1;
+    float *st = p.state + row * S;
+    float in[K];
+#pragma unroll
+    for (int k = 0; k < S; ++k) in[k] = st[k];
+    in[S] = load_elem(static_cast<const T *>(p.x) + b * p.x_batch_stride + d);
+    float v = p.bias ? __ldg(p.bias + d) : 0.f;
+#pragma unroll
+    for (int k = 0; k < K; ++k) v = fmaf(__ldg(p.w + d * K + k), in[k], v);
+    Elem<T>::store(static_cast<T *>(p.out) + row, p.silu ? silu_f(v) : v);
+#pragma unroll
+    for (int k = 0; k < S; ++k) st[k] = in[k + 1];
+}
+
+template <typename T>
+cudaError_t launch_fwd_typed(const ConvParams &p, cudaStream_t st) {
+    constexpr int V = 16 / (int)sizeof(T);
+    const auto aligned = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+    const bool tiles = aligned(p.x) && aligned(p.out) && p.seqlen % V == 0 && p.x_batch_stride % V == 0;
+    const int threads = 256;
+    if (tiles) {
+        constexpr int TILE = 32 * V, NT = 4;
+        const int64_t warps = p.batch * p.dim * ((p.seqlen + NT * TILE - 1) / (NT * TILE));
+        const int64_t blocks = (warps * 32 + threads - 1) / threads;
+        if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+        switch (p.width) {
+            case 1: conv1d_tiles_kernel<T, 1, NT><<<(unsigned)blocks, threads, 0, st>>>(p); break;
+            case 2: conv1d_tiles_kernel<T, 2, NT><<<(unsigned)blocks, threads, 0, st>>>(p); break;
+            case 3: conv1d_tiles_kernel<T, 3, NT><<<(unsigned)blocks, threads, 0, st>>>(p); break;
+            default: conv1d_tiles_kernel<T, 4, NT><<<(unsigned)blocks, threads, 0, st>>>(p); break;
+        }
+        return cudaGetLastError();
+    }
+    const int64_t blocks = (p.batch * p.dim * p.seqlen + threads - 1) / threads;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    conv1d_scalar_kernel<T><<<(unsigned)blocks, threads, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_update_typed(const ConvUpdateParams &p, unsigned blocks, cudaStream_t st) {
+    switch (p.width) {
+        case 1: conv1d_update_kernel<T, 1><<<blocks, 256, 0, st>>>(p); break;
+        case 2: conv1d_update_kernel<T, 2><<<blocks, 256, 0, st>>>(p); break;
+        case 3: conv1d_update_kernel<T, 3><<<blocks, 256, 0, st>>>(p); break;
+        default: conv1d_update_kernel<T, 4><<<blocks, 256, 0, st>>>(p); break;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_conv1d_fwd(const Conv1dArgs &a, cudaStream_t st) {
+    ConvParams p;
+    p.x = a.x; p.w = a.weight; p.bias = a.bias; p.out = a.out;
+    p.batch = a.batch; p.dim = a.dim; p.seqlen = a.seqlen; p.x_batch_stride = a.x_batch_stride;
+    p.width = a.width; p.silu = a.silu;
+    return a.act == kBF16 ? launch_fwd_typed<__nv_bfloat16>(p, st) : launch_fwd_typed<float>(p, st);
+}
+
+cudaError_t launch_conv1d_update(const Conv1dUpdateArgs &a, cudaStream_t st) {
+    ConvUpdateParams p;
+    p.state = a.state; p.x = a.x; p.w = a.weight; p.bias = a.bias; p.out = a.out;
+    p.batch = a.batch; p.dim = a.dim; p.x_batch_stride = a.x_batch_stride;
+    p.width = a.width; p.silu = a.silu;
+    const int threads = 256;
+    const int64_t blocks = (a.batch * a.dim + threads - 1) / threads;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    return a.act == kBF16 ? launch_update_typed<__nv_bfloat16>(p, (unsigned)blocks, st)
+                          : launch_update_typed<float>(p, (unsigned)blocks, st);
+}
+
+}  // namespace mscan

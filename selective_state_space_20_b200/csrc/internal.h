@@ -52,6 +52,26 @@ cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &plan,
 
 cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t stream);
 
+// Causal depthwise conv1d (+ bias, + silu) producing u; width 1 .. 4.
+struct Conv1dArgs {
+    const void *x;           // row (b, d) at x + b * x_batch_stride + d * seqlen
+    const float *weight;     // (dim, width)
+    const float *bias;       // (dim) or null
+    void *out;               // (batch, dim, seqlen)
+    int64_t batch, dim, seqlen, x_batch_stride;
+    int width, silu, act;
+};
+struct Conv1dUpdateArgs {
+    float *state;            // (batch, dim, width - 1), oldest input first
+    const void *x;           // (batch, dim): row b at x + b * x_batch_stride
+    const float *weight, *bias;
+    void *out;               // (batch, dim)
+    int64_t batch, dim, x_batch_stride;
+    int width, silu, act;
+};
+cudaError_t launch_conv1d_fwd(const Conv1dArgs &a, cudaStream_t stream);
+cudaError_t launch_conv1d_update(const Conv1dUpdateArgs &a, cudaStream_t stream);
+
 // Persistent, queue-balanced scan (dstate <= 16), one or two lanes per channel.
 bool persistent_supported(const ScanArgs &a);
 bool persistent_preferred(const ScanArgs &a, int sm_count);

@@ -19,6 +19,12 @@ dt initialisation of the mamba-jax ``train.py`` flags and the Keras/TensorFlow
   initialised to target a range of step sizes.
 * ``u, B, C, z ~ N(0, 1)``.
 * ``D = 1`` or ``D ~ U(0.5, 1.5)`` depending on the workload.
+
+Convolution inputs (the causal depthwise conv1d that produces u): the x half
+of the input projection's output ``xz ~ N(0, 1)`` of shape (batch, 2 dim, L)
+(x = the first dim channel rows), conv weight and bias ``~ U(-1/sqrt(K),
+1/sqrt(K))`` -- the default uniform initialisation bound of a convolution
+with fan-in K (one input channel per group, K taps).
 """
 from __future__ import annotations
 
@@ -187,3 +193,18 @@ def decode_as_scan(d: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]:
     for k in ("B", "C"):
         out[k] = d[k].permute(1, 2, 0).contiguous()
     return out
+
+
+def conv_inputs(batch: int, dim: int, seqlen: int, width: int = 4, dtype: str = "bf16",
+                seed: int = 40, device="cpu", wide: bool = True) -> Dict[str, torch.Tensor]:
+    """Inputs of the causal depthwise conv1d: ``xz`` (batch, 2 dim, L) in the
+    activation dtype when ``wide`` (the projection output; x = xz[:, :dim]),
+    else ``x`` (batch, dim, L); ``weight`` (dim, width) and ``bias`` (dim,)
+    fp32."""
+    g = _gen(seed, device)
+    bound = 1.0 / math.sqrt(width)
+    weight = ((torch.rand(dim, width, generator=g, device=device) * 2 - 1) * bound).contiguous()
+    bias = ((torch.rand(dim, generator=g, device=device) * 2 - 1) * bound).contiguous()
+    rows = 2 * dim if wide else dim
+    x = _normal((batch, rows, seqlen), g, device, DTYPES[dtype])
+    return {"xz" if wide else "x": x, "weight": weight, "bias": bias}

@@ -115,3 +115,37 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 2, 8)
     with pytest.raises(ValueError):
         binding.mamba_scan_fwd(x, x, torch.zeros(2, 16), torch.zeros(1, 16, 8), torch.zeros(1, 16, 8))
+
+
+def test_conv1d_validation(lib):
+    vp = ctypes.c_void_p
+    cf = lib.mamba_conv1d_fwd
+    # x, weight, bias, silu, out, batch, dim, L, width, stride, dtype, stream
+    ok = [vp(0x100000), vp(0x200000), None, 1, vp(0x800000), 2, 4, 64, 4, 0, 1, None]
+
+    def call(**kw):
+        a = list(ok)
+        names = ["x", "w", "bias", "silu", "out", "batch", "dim", "L", "width", "stride", "dtype"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return cf(*a)
+    assert call(x=None) == -1 and call(w=None) == -1 and call(out=None) == -1
+    assert call(batch=0) == -2 and call(L=-1) == -2
+    assert call(width=0) == -3 and call(width=5) == -3 and call(dtype=3) == -3
+    assert call(stride=4 * 64 - 1) == -2  # rows of one batch row would overlap the next
+    assert call(out=vp(0x100000 + 64)) == -7  # out inside x
+    cu = lib.mamba_conv1d_update
+    # state, x, weight, bias, silu, out, batch, dim, width, stride, dtype, stream
+    okc = [vp(0x100000), vp(0x200000), vp(0x300000), None, 1, vp(0x400000), 2, 4, 4, 0, 1, None]
+    bad = list(okc)
+    bad[0] = None
+    assert cu(*bad) == -1  # width 4 needs a state
+    bad = list(okc)
+    bad[0], bad[8] = None, 1
+    assert cu(*bad) != -1  # width 1 keeps no state (fails later only for want of a device)
+    bad = list(okc)
+    bad[8] = 9
+    assert cu(*bad) == -3
+    bad = list(okc)
+    bad[5] = vp(0x100000 + 4)  # out inside the state
+    assert cu(*bad) == -7
