@@ -69,10 +69,22 @@ def algorithmic_bytes(w) -> int:
     return 4 * x + bc + params + state
 
 
-def source_hash() -> str:
+# The sources each benchmarked kernel is built from (its file, the headers it
+# includes and the host code that plans its launch): a committed DRAM-traffic
+# record stays valid until one of them changes.
+KERNEL_SOURCES = {
+    "scan_fwd_pairs_kernel": ("scan_fwd_persistent_pairs.cu", "persistent_common.cuh", "persistent_kernels.h",
+                              "persistent_host.cu", "device_math.cuh", "internal.h"),
+    "scan_fwd_spec_kernel": ("scan_fwd_persistent_spec.cu", "persistent_common.cuh", "persistent_kernels.h",
+                             "persistent_host.cu", "device_math.cuh", "internal.h"),
+    "scan_fwd_kernel": ("scan_fwd.cu", "device_math.cuh", "internal.h"),
+}
+
+
+def source_hash(kernel: str = "scan_fwd_pairs_kernel") -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_state_space_20_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(KERNEL_SOURCES[kernel]):
         with open(os.path.join(csrc, name), "rb") as fh:
             h.update(name.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -86,7 +98,7 @@ def measured_traffic(kernel_key: str):
         with open(path) as fh:
             rec = json.load(fh)
         e = rec.get(kernel_key)
-        if e and e.get("source_hash") == source_hash():
+        if e and e.get("source_hash") == source_hash(kernel_key.split(" ")[0]):
             return float(e["dram_bytes_per_launch"])
     except Exception:
         pass
