@@ -10,6 +10,7 @@ its header for the equations and where each comes from).  This module only
 marshals numpy/torch CPU arrays into it:
 
 * :func:`scan` -- the whole forward scan (optionally from an initial state).
+* :func:`scan_bwd` -- gradients of the forward scan (reverse mode).
 * :func:`state_update` -- one recurrent step for every (batch, channel).
 * :func:`conv1d`, :func:`conv1d_update` -- the causal depthwise convolution
   (+ bias, + silu) that feeds the scan, whole-sequence and one token.
@@ -50,6 +51,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.s6_oracle_conv1d.argtypes = [f32p, f32p, f32p, ctypes.c_int, f64p, i64, i64, i64, i64, i64]
     lib.s6_oracle_conv1d_update.restype = ctypes.c_int
     lib.s6_oracle_conv1d_update.argtypes = [f64p, f32p, f32p, f32p, ctypes.c_int, f64p, i64, i64, i64]
+    lib.s6_oracle_scan_bwd.restype = ctypes.c_int
+    lib.s6_oracle_scan_bwd.argtypes = [f32p, f32p, f32p, f32p, f32p, f32p, f32p, f32p, ctypes.c_int,
+                                       f64p, f64p, f64p, f64p, f64p, f64p, f64p, f64p, f64p, f64p,
+                                       f64p, f64p, i64, i64, i64, i64, ctypes.c_int]
     lib.s6_oracle_softplus.restype = ctypes.c_double
     lib.s6_oracle_softplus.argtypes = [ctypes.c_double]
     lib.s6_oracle_silu.restype = ctypes.c_double
@@ -121,6 +126,37 @@ def scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     if rc != 0:
         raise RuntimeError(f"s6_oracle_scan failed with code {rc}")
     return out, last
+
+
+def scan_bwd(dout, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+             delta_softplus: bool = True, h0=None, dlast=None, nthreads: int = 0,
+             lib: Optional[ctypes.CDLL] = None) -> dict:
+    """Gradients of :func:`scan` in fp64 for dL/dout = ``dout`` (batch, dim,
+    L) and optionally dL/dlast_state = ``dlast`` (batch, dim, N).
+
+    Returns a dict with du, ddelta, dz (batch, dim, L; dz None without z),
+    dA (dim, N), dB, dC (batch, N, L), dD, ddelta_bias (dim,) and dh0
+    (batch, dim, N)."""
+    lib = lib or _get()
+    u, delta, A, B, C = (_f32(t) for t in (u, delta, A, B, C))
+    D, z, delta_bias = _f32(D), _f32(z), _f32(delta_bias)
+    h0, dout, dlast = _f64(h0), _f64(dout), _f64(dlast)
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    assert dout.shape == u.shape and (dlast is None or dlast.shape == (batch, dim, N))
+    r = {k: np.empty(s, dtype=np.float64) for k, s in (
+        ("du", (batch, dim, L)), ("ddelta", (batch, dim, L)), ("dA", (dim, N)),
+        ("dB", (batch, N, L)), ("dC", (batch, N, L)), ("dD", (dim,)),
+        ("ddelta_bias", (dim,)), ("dh0", (batch, dim, N)))}
+    r["dz"] = np.empty((batch, dim, L), dtype=np.float64) if z is not None else None
+    rc = lib.s6_oracle_scan_bwd(_p32(u), _p32(delta), _p32(A), _p32(B), _p32(C), _p32(D), _p32(z),
+                                _p32(delta_bias), int(bool(delta_softplus)), _p64(h0), _p64(dout),
+                                _p64(dlast), _p64(r["du"]), _p64(r["ddelta"]), _p64(r["dA"]),
+                                _p64(r["dB"]), _p64(r["dC"]), _p64(r["dD"]), _p64(r["dz"]),
+                                _p64(r["ddelta_bias"]), _p64(r["dh0"]), batch, dim, L, N, int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_scan_bwd failed with code {rc}")
+    return r
 
 
 def state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,

@@ -299,3 +299,207 @@ int s6_oracle_state_update(double *state, const float *u, const float *delta,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ backward
+ * Gradients of the forward scan above for a loss L with dL/dout = dout and
+ * (optionally) dL/dlast_state = dlast: reverse-mode differentiation of the
+ * recurrence written out (the scan is differentiated as a whole sequence;
+ * the training path the pages describe back-propagates through it, and the
+ * Mamba paper's hardware-aware algorithm recomputes the states in the
+ * backward pass instead of storing them -- this plain loop stores them).
+ *
+ * Per (b, d), with g[n] = dL/dh_t[n] carried backwards from g = dlast:
+ *   y_t  = sum_n C[n,t] h_t[n] + D u_t            (recomputed from stored h)
+ *   dz_t = dout_t * y_t * silu'(z_t),  silu'(z) = s (1 + z (1 - s)), s = 1/(1+e^-z)
+ *   dy_t = dout_t * silu(z_t)  (dout_t without a gate)
+ *   dD  += dy_t u_t;  du_t = dy_t D;  dC[b,n,t] += dy_t h_t[n];  g[n] += dy_t C[n,t]
+ *   with hp = h_{t-1}[n] (h0 or 0 at t = 0) and Abar = exp(delta_t A[n]):
+ *   ddelta_t += g[n] (hp Abar A[n] + B[n,t] u_t)
+ *   dA[d,n]  += g[n] hp Abar delta_t
+ *   dB[b,n,t]+= g[n] delta_t u_t
+ *   du_t     += g[n] delta_t B[n,t]
+ *   g[n]      = g[n] Abar                        (dL/dh_{t-1}[n])
+ *   ddelta_raw_t = ddelta_t * sigmoid(delta_raw_t + bias[d]) with softplus,
+ *   ddelta_t itself without;  dbias[d] += ddelta_raw_t
+ *   dh0 = g after t = 0.
+ * Outputs: du, ddelta, dz (batch, dim, L); dA (dim, N); dB, dC (batch, N, L);
+ * dD, ddelta_bias (dim); dh0 (batch, dim, N) -- all fp64; dz, dD,
+ * ddelta_bias, dh0 may be NULL when not wanted (dz must be NULL without z).
+ * Channel rows are spread over POSIX threads; the sums over channels (dA,
+ * dB, dC, dD, dbias) are accumulated per thread and added in thread order,
+ * so results do not depend on timing. */
+typedef struct {
+    const float *u, *delta, *A, *B, *C, *D, *z, *bias;
+    const double *h0, *dout, *dlast;
+    int softplus;
+    double *du, *ddelta, *dz, *dh0;
+    double *dA, *dB, *dC, *dD, *dbias; /* this thread's partial sums */
+    int64_t batch, dim, seqlen, dstate;
+    int64_t row_begin, row_end;
+    int status;
+} bwd_job_t;
+
+static double s6_oracle_sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+static void *bwd_worker(void *arg)
+{
+    bwd_job_t *j = (bwd_job_t *)arg;
+    const int64_t L = j->seqlen, N = j->dstate;
+    double *hs = (double *)malloc(sizeof(double) * (size_t)((L + 1) * N));
+    double *g = (double *)malloc(sizeof(double) * (size_t)N);
+    if (!hs || !g) {
+        free(hs);
+        free(g);
+        j->status = -2;
+        return NULL;
+    }
+    for (int64_t row = j->row_begin; row < j->row_end; ++row) {
+        const int64_t b = row / j->dim, d = row % j->dim;
+        const float *u = j->u + row * L;
+        const float *dr = j->delta + row * L;
+        const float *z = j->z ? j->z + row * L : NULL;
+        const float *Bw = j->B + b * N * L;
+        const float *Cw = j->C + b * N * L;
+        const float *Aw = j->A + d * N;
+        const double Dd = j->D ? (double)j->D[d] : 0.0;
+        const double bias = j->bias ? (double)j->bias[d] : 0.0;
+        const double *dout = j->dout + row * L;
+        /* forward, keeping every state: hs[(t + 1) N + n] = h_t[n], hs[n] = h_{-1} */
+        for (int64_t n = 0; n < N; ++n)
+            hs[n] = j->h0 ? j->h0[row * N + n] : 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            double delta = (double)dr[t] + bias;
+            if (j->softplus)
+                delta = s6_oracle_softplus(delta);
+            for (int64_t n = 0; n < N; ++n)
+                hs[(t + 1) * N + n] = exp((double)Aw[n] * delta) * hs[t * N + n] +
+                                      delta * (double)Bw[n * L + t] * (double)u[t];
+        }
+        for (int64_t n = 0; n < N; ++n)
+            g[n] = j->dlast ? j->dlast[row * N + n] : 0.0;
+        for (int64_t t = L - 1; t >= 0; --t) {
+            const double draw = (double)dr[t] + bias;
+            const double delta = j->softplus ? s6_oracle_softplus(draw) : draw;
+            const double ut = (double)u[t];
+            const double *h = hs + (t + 1) * N, *hp = hs + t * N;
+            double y = Dd * ut;
+            for (int64_t n = 0; n < N; ++n)
+                y += (double)Cw[n * L + t] * h[n];
+            double dy = dout[t];
+            if (z) {
+                const double zt = (double)z[t], s = s6_oracle_sigmoid(zt);
+                if (j->dz)
+                    j->dz[row * L + t] = dout[t] * y * s * (1.0 + zt * (1.0 - s));
+                dy = dout[t] * s6_oracle_silu(zt);
+            }
+            j->dD[d] += dy * ut;
+            double du = dy * Dd, ddelta = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                j->dC[b * N * L + n * L + t] += dy * h[n];
+                g[n] += dy * (double)Cw[n * L + t];
+                const double Abar = exp((double)Aw[n] * delta);
+                ddelta += g[n] * (hp[n] * Abar * (double)Aw[n] + (double)Bw[n * L + t] * ut);
+                j->dA[d * N + n] += g[n] * hp[n] * Abar * delta;
+                j->dB[b * N * L + n * L + t] += g[n] * delta * ut;
+                du += g[n] * delta * (double)Bw[n * L + t];
+                g[n] *= Abar;
+            }
+            const double ddraw = j->softplus ? ddelta * s6_oracle_sigmoid(draw) : ddelta;
+            j->du[row * L + t] = du;
+            j->ddelta[row * L + t] = ddraw;
+            j->dbias[d] += ddraw;
+        }
+        if (j->dh0)
+            for (int64_t n = 0; n < N; ++n)
+                j->dh0[row * N + n] = g[n];
+    }
+    free(hs);
+    free(g);
+    return NULL;
+}
+
+int s6_oracle_scan_bwd(const float *u, const float *delta, const float *A,
+                       const float *B, const float *C, const float *D,
+                       const float *z, const float *delta_bias, int softplus,
+                       const double *h0, const double *dout, const double *dlast,
+                       double *du, double *ddelta, double *dA, double *dB,
+                       double *dC, double *dD, double *dz, double *ddelta_bias,
+                       double *dh0, int64_t batch, int64_t dim, int64_t seqlen,
+                       int64_t dstate, int nthreads)
+{
+    if (!u || !delta || !A || !B || !C || !dout || !du || !ddelta || !dA || !dB || !dC)
+        return -1;
+    if (batch <= 0 || dim <= 0 || seqlen <= 0 || dstate <= 0 || (dz && !z))
+        return -1;
+    const int64_t rows = batch * dim, N = dstate, L = seqlen;
+    if (nthreads <= 0) {
+        long nc = sysconf(_SC_NPROCESSORS_ONLN);
+        nthreads = nc > 0 ? (int)nc : 1;
+    }
+    if (nthreads > rows)
+        nthreads = (int)rows;
+    const size_t nA = (size_t)(dim * N), nBC = (size_t)(batch * N * L), nd = (size_t)dim;
+    const size_t per = 2 * nBC + nA + 2 * nd; /* dB, dC, dA, dD, dbias */
+    double *acc = (double *)calloc((size_t)nthreads * per, sizeof(double));
+    bwd_job_t *jobs = (bwd_job_t *)malloc(sizeof(bwd_job_t) * (size_t)nthreads);
+    pthread_t *tids = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!acc || !jobs || !tids) {
+        free(acc);
+        free(jobs);
+        free(tids);
+        return -2;
+    }
+    int started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        double *a = acc + (size_t)i * per;
+        bwd_job_t jb = {u, delta, A, B, C, D, z, delta_bias, h0, dout, dlast, softplus,
+                        du, ddelta, dz, dh0, a + 2 * nBC, a, a + nBC, a + 2 * nBC + nA,
+                        a + 2 * nBC + nA + nd, batch, dim, seqlen, dstate,
+                        rows * i / nthreads, rows * (i + 1) / nthreads, 0};
+        jobs[i] = jb;
+    }
+    for (int i = 0; i < nthreads; ++i) {
+        if (nthreads == 1 || pthread_create(&tids[i], NULL, bwd_worker, &jobs[i]) != 0) {
+            for (int k = i; k < nthreads; ++k) /* run the rest on this thread */
+                bwd_worker(&jobs[k]);
+            break;
+        }
+        ++started;
+    }
+    for (int i = 0; i < started; ++i)
+        pthread_join(tids[i], NULL);
+    int rc = 0;
+    for (size_t k = 0; k < nBC; ++k) {
+        dB[k] = 0.0;
+        dC[k] = 0.0;
+    }
+    for (size_t k = 0; k < nA; ++k)
+        dA[k] = 0.0;
+    for (size_t k = 0; k < nd; ++k) {
+        if (dD)
+            dD[k] = 0.0;
+        if (ddelta_bias)
+            ddelta_bias[k] = 0.0;
+    }
+    for (int i = 0; i < nthreads; ++i) {
+        if (jobs[i].status)
+            rc = jobs[i].status;
+        const double *a = acc + (size_t)i * per;
+        for (size_t k = 0; k < nBC; ++k) {
+            dB[k] += a[k];
+            dC[k] += a[nBC + k];
+        }
+        for (size_t k = 0; k < nA; ++k)
+            dA[k] += a[2 * nBC + k];
+        for (size_t k = 0; k < nd; ++k) {
+            if (dD)
+                dD[k] += a[2 * nBC + nA + k];
+            if (ddelta_bias)
+                ddelta_bias[k] += a[2 * nBC + nA + nd + k];
+        }
+    }
+    free(acc);
+    free(jobs);
+    free(tids);
+    return rc;
+}

@@ -470,6 +470,94 @@ def pin_conv_causality(lib):
     assert np.all(a[:, :, 11] != b[:, :, 11])
 
 
+# ------------------------------------------------------------ backward
+# Gradients of the scan: against torch.autograd on an fp64 forward written
+# here with torch tensor ops (a different program from the oracle's loop),
+# and against central finite differences of the oracle's own (pinned)
+# forward.
+
+def _bwd_problem(seed, batch=2, dim=3, L=9, N=4, gate=True):
+    rng = np.random.default_rng(seed)
+    f = lambda *s, scale=1.0: (rng.standard_normal(s) * scale).astype(np.float32)  # noqa: E731
+    p = dict(u=f(batch, dim, L), delta=f(batch, dim, L, scale=0.5),
+             A=-np.abs(f(dim, N)) - 0.2, B=f(batch, N, L), C=f(batch, N, L),
+             D=f(dim), z=f(batch, dim, L) if gate else None, delta_bias=f(dim, scale=0.3))
+    h0 = f(batch, dim, N).astype(np.float64)
+    dout = f(batch, dim, L).astype(np.float64)
+    dlast = f(batch, dim, N).astype(np.float64)
+    return p, h0, dout, dlast
+
+
+def _torch_scan(u, delta, A, B, C, D, z, bias, h0, softplus=True):
+    import torch
+    dl = delta + bias[None, :, None]
+    if softplus:
+        dl = torch.logaddexp(dl, torch.zeros_like(dl))
+    h, ys = h0, []
+    for t in range(u.shape[-1]):
+        h = torch.exp(dl[..., t, None] * A) * h + dl[..., t, None] * B[:, None, :, t] * u[..., t, None]
+        y = (h * C[:, None, :, t]).sum(-1) + D * u[..., t]
+        if z is not None:
+            y = y * z[..., t] * torch.sigmoid(z[..., t])
+        ys.append(y)
+    return torch.stack(ys, -1), h
+
+
+def pin_bwd_autograd(lib):
+    """Every gradient equals torch.autograd's through an fp64 forward written
+    with torch ops, with and without the gate and softplus."""
+    import torch
+    for seed, gate, sp in ((301, True, True), (302, False, True), (303, True, False)):
+        p, h0, dout, dlast = _bwd_problem(seed, gate=gate)
+        if not sp:
+            p["delta"] = np.abs(p["delta"])
+            p["delta_bias"] = np.abs(p["delta_bias"])
+        names = ["u", "delta", "A", "B", "C", "D", "z", "delta_bias"]
+        t = {k: (None if p[k] is None else torch.tensor(p[k], dtype=torch.float64, requires_grad=True))
+             for k in names}
+        th0 = torch.tensor(h0, requires_grad=True)
+        out, last = _torch_scan(t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"],
+                                t["delta_bias"], th0, softplus=sp)
+        loss = (out * torch.tensor(dout)).sum() + (last * torch.tensor(dlast)).sum()
+        wrt = [t[k] for k in names if t[k] is not None] + [th0]
+        grads = dict(zip([k for k in names if t[k] is not None] + ["h0"], torch.autograd.grad(loss, wrt)))
+        r = oracle.scan_bwd(dout, **p, delta_softplus=sp, h0=h0, dlast=dlast, lib=lib)
+        pairs = [("du", "u"), ("ddelta", "delta"), ("dA", "A"), ("dB", "B"), ("dC", "C"),
+                 ("dD", "D"), ("ddelta_bias", "delta_bias"), ("dh0", "h0")] + ([("dz", "z")] if gate else [])
+        for mine, theirs in pairs:
+            _close(r[mine], grads[theirs].numpy(), rtol=1e-11, what=f"{mine} vs autograd (seed {seed})")
+
+
+def pin_bwd_finite_differences(lib):
+    """Central differences of the oracle's forward loss at a few entries of
+    every input; the perturbed values are fp32 numbers, and the divisor is
+    their exact difference."""
+    p, h0, dout, dlast = _bwd_problem(304, L=6, N=3)
+    r = oracle.scan_bwd(dout, **p, h0=h0, dlast=dlast, lib=lib)
+
+    def loss(q, hh):
+        o, s = oracle.scan(**q, h0=hh, lib=lib)
+        return float(np.sum(o * dout) + np.sum(s * dlast))
+    rng = np.random.default_rng(305)
+    for name, gname in (("u", "du"), ("delta", "ddelta"), ("A", "dA"), ("B", "dB"), ("C", "dC"),
+                        ("D", "dD"), ("z", "dz"), ("delta_bias", "ddelta_bias"), ("h0", "dh0")):
+        base = h0 if name == "h0" else p[name]
+        for _ in range(3):
+            idx = tuple(int(rng.integers(0, n)) for n in base.shape)
+            x = float(base[idx])
+            step = 1e-3 * max(abs(x), 1.0)
+            vals = []
+            for sgn in (1, -1):
+                q = {k: (None if v is None else v.copy()) for k, v in p.items()}
+                hh = h0.copy()
+                tgt = hh if name == "h0" else q[name]
+                tgt[idx] = np.float32(x + sgn * step)
+                vals.append((loss(q, hh), float(np.float32(x + sgn * step))))
+            fd = (vals[0][0] - vals[1][0]) / (vals[0][1] - vals[1][1])
+            g = float(r[gname][idx])
+            assert abs(fd - g) <= 2e-5 * max(1.0, abs(g)), f"{gname}{idx}: fd {fd} vs {g}"
+
+
 ALL_PINS = [pin_softplus_silu, pin_geometric_series, pin_lti_convolution,
             pin_first_order_iir, pin_zero_step_keeps_state, pin_memoryless_limit,
             pin_brute_force_products, pin_cumsum_form, pin_chunk_split,
@@ -477,4 +565,5 @@ ALL_PINS = [pin_softplus_silu, pin_geometric_series, pin_lti_convolution,
             pin_shared_bc_and_independence, pin_zero_b_or_c,
             pin_gate_and_softplus_flags,
             pin_conv_numpy, pin_conv_impulse, pin_conv_silu, pin_conv_wide_input,
-            pin_conv_update_stream, pin_conv_causality]
+            pin_conv_update_stream, pin_conv_causality,
+            pin_bwd_autograd, pin_bwd_finite_differences]

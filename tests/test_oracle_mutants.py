@@ -55,6 +55,22 @@ MUTANTS = [
     ("conv-update-no-shift", "st[k] = st[k + 1];", "st[k] = st[k];"),
     ("conv-update-newest-first", "v += (double)wr[k] * (k < S ? st[k] : xt);",
      "v += (double)wr[k] * (k == 0 ? xt : st[k - 1]);"),
+    # backward
+    ("bwd-ddelta-decay-term-dropped", "ddelta += g[n] * (hp[n] * Abar * (double)Aw[n] + (double)Bw[n * L + t] * ut);",
+     "ddelta += g[n] * ((double)Bw[n * L + t] * ut);"),
+    ("bwd-carry-without-decay", "g[n] *= Abar;", "g[n] *= 1.0;"),
+    ("bwd-dC-uses-previous-state", "j->dC[b * N * L + n * L + t] += dy * h[n];",
+     "j->dC[b * N * L + n * L + t] += dy * hp[n];"),
+    ("bwd-softplus-derivative-dropped", "const double ddraw = j->softplus ? ddelta * s6_oracle_sigmoid(draw) : ddelta;",
+     "const double ddraw = ddelta;"),
+    ("bwd-silu-derivative-wrong", "s * (1.0 + zt * (1.0 - s))", "s"),
+    ("bwd-dlast-ignored", "g[n] = j->dlast ? j->dlast[row * N + n] : 0.0;", "g[n] = 0.0;"),
+    ("bwd-dA-without-delta", "j->dA[d * N + n] += g[n] * hp[n] * Abar * delta;",
+     "j->dA[d * N + n] += g[n] * hp[n] * Abar;"),
+    ("bwd-du-input-term-dropped", "du += g[n] * delta * (double)Bw[n * L + t];", "du += 0.0;"),
+    ("bwd-dB-without-u", "j->dB[b * N * L + n * L + t] += g[n] * delta * ut;",
+     "j->dB[b * N * L + n * L + t] += g[n] * delta;"),
+    ("bwd-dD-without-gate", "j->dD[d] += dy * ut;", "j->dD[d] += dout[t] * ut;"),
 ]
 
 
