@@ -241,6 +241,51 @@ int mamba_state_update(float *state, const void *u, const void *delta,
                        cudaStream_t stream);
 
 /*
+ * mamba_scan_bwd -- gradients of mamba_scan_fwd with respect to every input,
+ * for a loss L given dL/dout and optionally dL/dlast_state: reverse-mode
+ * differentiation of the recurrence ("Mamba SSM concept and implementation
+ * in Keras and TensorFlow", recurrent form, differentiated through the whole
+ * sequence for training; recomputing the states in the backward pass, as the
+ * Mamba paper's hardware-aware algorithm does, Section 3.3).  With
+ * g = dL/dh_t carried backwards from dlast:
+ *   dy = dout silu(z), dz = dout y silu'(z), dD += dy u, du = dy D,
+ *   dC[n,t] += dy h_t[n], g[n] += dy C[n,t],
+ *   ddelta += g[n] (h_{t-1}[n] Abar A[n] + B[n,t] u), dA[n] += g[n] h_{t-1}[n] Abar delta,
+ *   dB[n,t] += g[n] delta u, du += g[n] delta B[n,t], g[n] *= Abar,
+ *   ddelta_raw = ddelta sigmoid(delta_raw + bias) with softplus, dbias += ddelta_raw.
+ *
+ *   inputs       : exactly those of mamba_scan_fwd (same layouts and dtypes).
+ *   dout         : act (batch, dim, seqlen).
+ *   dlast_state  : fp32 (batch, dim, dstate) or NULL (no loss on the final state).
+ *   du, ddelta   : act (batch, dim, seqlen), written.
+ *   dz           : act (batch, dim, seqlen), written; required iff z is given.
+ *   dA           : fp32 (dim, dstate); dB, dC: fp32 (batch, dstate, seqlen);
+ *   dD, ddelta_bias : fp32 (dim) or NULL -- all zeroed on `stream`, then
+ *                  accumulated (sums over batch rows, channels and time).
+ *   workspace    : at least mamba_scan_bwd_workspace_size bytes, 16-byte
+ *                  aligned, caller-owned (the states checkpointed every 16
+ *                  timesteps).
+ *
+ * dstate <= 16.  The sums over channels use floating-point atomics, so dA,
+ * dB, dC, dD and ddelta_bias may differ in the last bits between runs; du,
+ * ddelta and dz do not.  Returns MAMBA_OK or a mamba_status_t error.
+ */
+int mamba_scan_bwd(const void *u, const void *delta, const float *A,
+                   const void *B, const void *C, const float *D,
+                   const void *z, const float *delta_bias, int delta_softplus,
+                   const void *dout, const float *dlast_state,
+                   void *du, void *ddelta, float *dA, float *dB, float *dC,
+                   float *dD, void *dz, float *ddelta_bias,
+                   int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                   int act_dtype, void *workspace, size_t workspace_bytes,
+                   cudaStream_t stream);
+
+/* Bytes of workspace mamba_scan_bwd needs for these sizes (0 when dstate > 16
+ * or the sizes are invalid).  Pure host arithmetic. */
+size_t mamba_scan_bwd_workspace_size(int64_t batch, int64_t dim, int64_t seqlen,
+                                     int64_t dstate);
+
+/*
  * mamba_conv1d_fwd -- the step that produces the scan's input u: a causal
  * depthwise convolution over time with a bias, then silu ("Mamba SSM concept
  * and implementation in Keras and TensorFlow", MambaBlock: a Conv1D with one

@@ -30,7 +30,8 @@ SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT = 0, 1, 2
 # Every function include/mamba_scan.h declares.
 EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
-            "mamba_scan_fwd_noalloc", "mamba_state_update", "mamba_conv1d_fwd",
+            "mamba_scan_fwd_noalloc", "mamba_scan_bwd", "mamba_scan_bwd_workspace_size",
+            "mamba_state_update", "mamba_conv1d_fwd",
             "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version")
 
 
@@ -69,6 +70,11 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_state_update.argtypes = [fp, vp, vp, fp, vp, vp, fp, vp, fp, ci, vp,
                                        i64, i64, i64, ci, vp]
     lib.mamba_state_update.restype = ci
+    lib.mamba_scan_bwd.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, ci, vp, fp, vp, vp, fp, fp, fp, fp,
+                                   vp, fp, i64, i64, i64, i64, ci, vp, ctypes.c_size_t, vp]
+    lib.mamba_scan_bwd.restype = ci
+    lib.mamba_scan_bwd_workspace_size.argtypes = [i64, i64, i64, i64]
+    lib.mamba_scan_bwd_workspace_size.restype = ctypes.c_size_t
     lib.mamba_conv1d_fwd.argtypes = [vp, fp, fp, ci, vp, i64, i64, i64, i64, i64, ci, vp]
     lib.mamba_conv1d_fwd.restype = ci
     lib.mamba_conv1d_update.argtypes = [fp, vp, fp, fp, ci, vp, i64, i64, i64, i64, ci, vp]
@@ -327,3 +333,53 @@ def mamba_conv1d_update(conv_state: Optional[torch.Tensor], x: torch.Tensor, wei
                                      _ACT[act], _stream(dev))
     _check("mamba_conv1d_update", rc)
     return out
+
+
+def mamba_scan_bwd(dout: torch.Tensor, u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
+                   B: torch.Tensor, C: torch.Tensor, D: Optional[torch.Tensor] = None,
+                   z: Optional[torch.Tensor] = None, delta_bias: Optional[torch.Tensor] = None,
+                   delta_softplus: bool = True, dlast_state: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None) -> dict:
+    """Gradients of :func:`mamba_scan_fwd` for dL/dout = ``dout`` (and
+    dL/dlast_state = ``dlast_state``).  Returns a dict: du, ddelta, dz (act
+    dtype, like u; dz None without z), dA (dim, N), dB, dC (batch, N, L),
+    dD, ddelta_bias (dim,) -- fp32 (dD / ddelta_bias None when D / the bias
+    are not given)."""
+    if u.dim() != 3:
+        raise ValueError("u must be (batch, dim, L)")
+    batch, dim, L = u.shape
+    N = A.shape[-1]
+    dev, act = u.device, u.dtype
+    if dev.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    if act not in _ACT:
+        raise TypeError(f"unsupported activation dtype {act}")
+    for name, t in (("u", u), ("delta", delta), ("z", z), ("dout", dout)):
+        _need(t, name, dev, act, (batch, dim, L))
+    _need(B, "B", dev, act, (batch, N, L))
+    _need(C, "C", dev, act, (batch, N, L))
+    _need(A, "A", dev, torch.float32, (dim, N))
+    _need(D, "D", dev, torch.float32, (dim,))
+    _need(delta_bias, "delta_bias", dev, torch.float32, (dim,))
+    _need(dlast_state, "dlast_state", dev, torch.float32, (batch, dim, N))
+    lib = load_library()
+    need = lib.mamba_scan_bwd_workspace_size(batch, dim, L, N)
+    if need == 0:
+        raise MambaError("mamba_scan_bwd", -3, "unsupported sizes (dstate <= 16)")
+    if workspace is None:
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    f32 = dict(device=dev, dtype=torch.float32)
+    r = {"du": torch.empty_like(u), "ddelta": torch.empty_like(u),
+         "dz": torch.empty_like(u) if z is not None else None,
+         "dA": torch.empty(dim, N, **f32), "dB": torch.empty(batch, N, L, **f32),
+         "dC": torch.empty(batch, N, L, **f32),
+         "dD": torch.empty(dim, **f32) if D is not None else None,
+         "ddelta_bias": torch.empty(dim, **f32) if delta_bias is not None else None}
+    with torch.cuda.device(dev):
+        rc = lib.mamba_scan_bwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                                _ptr(delta_bias), int(bool(delta_softplus)), _ptr(dout), _ptr(dlast_state),
+                                _ptr(r["du"]), _ptr(r["ddelta"]), _ptr(r["dA"]), _ptr(r["dB"]), _ptr(r["dC"]),
+                                _ptr(r["dD"]), _ptr(r["dz"]), _ptr(r["ddelta_bias"]), batch, dim, L, N,
+                                _ACT[act], _ptr(workspace), workspace.numel(), _stream(dev))
+    _check("mamba_scan_bwd", rc)
+    return r

@@ -252,6 +252,53 @@ int mamba_state_update(float *state, const void *u, const void *delta, const flo
     return mscan::launch_state_update(a, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 
+size_t mamba_scan_bwd_workspace_size(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate) {
+    if (check_sizes(batch, dim, seqlen, dstate) != MAMBA_OK || dstate > 16) return 0;
+    return mscan::scan_bwd_workspace_bytes(batch, dim, seqlen);
+}
+
+int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                   const float *D, const void *z, const float *delta_bias, int delta_softplus,
+                   const void *dout, const float *dlast_state, void *du, void *ddelta, float *dA,
+                   float *dB, float *dC, float *dD, void *dz, float *ddelta_bias, int64_t batch,
+                   int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype, void *workspace,
+                   size_t workspace_bytes, cudaStream_t stream) {
+    if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
+    int rc = check_sizes(batch, dim, seqlen, dstate);
+    if (rc != MAMBA_OK) return rc;
+    if (dstate > 16) return MAMBA_ERR_UNSUPPORTED;
+    if (!u || !delta || !A || !B || !C || !dout || !du || !ddelta || !dA || !dB || !dC) return MAMBA_ERR_NULL;
+    if ((z != nullptr) != (dz != nullptr)) return MAMBA_ERR_NULL;
+    const size_t need = mscan::scan_bwd_workspace_bytes(batch, dim, seqlen);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15))
+        return MAMBA_ERR_WORKSPACE;
+    const size_t es = act_size(act_dtype);
+    const size_t nx = (size_t)(batch * dim * seqlen) * es, nbc = (size_t)(batch * dstate * seqlen) * es;
+    const size_t nbc32 = (size_t)(batch * dstate * seqlen) * 4, nA = (size_t)(dim * dstate) * 4;
+    const size_t nd = (size_t)dim * 4, ns = (size_t)(batch * dim * dstate) * 4;
+    const void *ins[] = {u, delta, z, dout, B, C, A, D, delta_bias, dlast_state, workspace};
+    const size_t inb[] = {nx, nx, nx, nx, nbc, nbc, nA, nd, nd, ns, need};
+    void *outs[] = {du, ddelta, dz, dA, dB, dC, dD, ddelta_bias};
+    const size_t outb[] = {nx, nx, nx, nA, nbc32, nbc32, nd, nd};
+    for (int i = 0; i < 8; ++i) {
+        for (int k = 0; k < 11; ++k)
+            if (overlaps(outs[i], outb[i], ins[k], inb[k])) return MAMBA_ERR_OVERLAP;
+        for (int k = 0; k < i; ++k)
+            if (overlaps(outs[i], outb[i], outs[k], outb[k])) return MAMBA_ERR_OVERLAP;
+    }
+    int status = MAMBA_OK;
+    const int sms = current_sm_count(&status);
+    if (status != MAMBA_OK) return status;
+    mscan::ScanBwdArgs a;
+    a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z; a.dout = dout;
+    a.A = A; a.D = D; a.delta_bias = delta_bias; a.dlast = dlast_state;
+    a.du = du; a.ddelta = ddelta; a.dz = dz;
+    a.dA = dA; a.dB = dB; a.dC = dC; a.dD = dD; a.ddelta_bias = ddelta_bias;
+    a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = (int)dstate;
+    a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
+    return mscan::launch_scan_bwd(a, workspace, sms, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
 int mamba_conv1d_fwd(const void *x, const float *weight, const float *bias, int apply_silu,
                      void *out, int64_t batch, int64_t dim, int64_t seqlen, int64_t width,
                      int64_t x_batch_stride, int act_dtype, cudaStream_t stream) {
@@ -322,6 +369,6 @@ const char *mamba_status_string(int status) {
     }
 }
 
-int mamba_abi_version(void) { return (1 << 16) | 1; }
+int mamba_abi_version(void) { return (1 << 16) | 2; }
 
 }  // extern "C"

@@ -69,6 +69,18 @@ struct Conv1dUpdateArgs {
     int64_t batch, dim, x_batch_stride;
     int width, silu, act;
 };
+// Backward of the scan (dstate <= 16): every input gradient.
+struct ScanBwdArgs {
+    const void *u, *delta, *B, *C, *z, *dout;
+    const float *A, *D, *delta_bias, *dlast;
+    void *du, *ddelta, *dz;                          // act (batch, dim, L)
+    float *dA, *dB, *dC, *dD, *ddelta_bias;          // fp32, accumulated from zero
+    int64_t batch, dim, seqlen;
+    int dstate, softplus, act;
+};
+size_t scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen);
+cudaError_t launch_scan_bwd(const ScanBwdArgs &a, void *workspace, int sm_count, cudaStream_t stream);
+
 cudaError_t launch_conv1d_fwd(const Conv1dArgs &a, cudaStream_t stream);
 cudaError_t launch_conv1d_update(const Conv1dUpdateArgs &a, cudaStream_t stream);
 

@@ -149,3 +149,26 @@ def test_conv1d_validation(lib):
     bad = list(okc)
     bad[5] = vp(0x100000 + 4)  # out inside the state
     assert cu(*bad) == -7
+
+
+def test_scan_bwd_validation(lib):
+    vp = ctypes.c_void_p
+    assert lib.mamba_scan_bwd_workspace_size(2, 40, 100, 16) > 0
+    assert lib.mamba_scan_bwd_workspace_size(2, 40, 100, 17) == 0
+    ws_n = lib.mamba_scan_bwd_workspace_size(2, 8, 64, 16)
+    P = [vp(0x100000 * (i + 1)) for i in range(20)]
+    # u delta A B C D z bias sp dout dlast du ddelta dA dB dC dD dz dbias b d L N act ws wsb stream
+    ok = [P[0], P[1], P[2], P[3], P[4], None, None, None, 1, P[5], None, P[6], P[7], P[8], P[9], P[10],
+          None, None, None, 2, 8, 64, 16, 1, P[11], ws_n, None]
+
+    def call(**kw):
+        a = list(ok)
+        idx = {"u": 0, "z": 6, "dout": 9, "du": 11, "dz": 17, "N": 22, "ws": 24, "wsb": 25, "dB": 14}
+        for k, v in kw.items():
+            a[idx[k]] = v
+        return lib.mamba_scan_bwd(*a)
+    assert call(u=None) == -1 and call(dout=None) == -1 and call(du=None) == -1
+    assert call(z=P[12]) == -1  # a gate needs dz
+    assert call(N=32) == -3
+    assert call(ws=None) == -8 and call(wsb=ws_n - 1) == -8 and call(ws=vp(0x1000008)) == -8
+    assert call(dB=vp(0x400000 + 64)) == -7  # dB inside B
