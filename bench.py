@@ -426,6 +426,41 @@ def conv1d_measure(reps=20):
             "reps": reps, "l2": "inputs larger than L2, no flush"}
 
 
+def backward_measure(reps=5):
+    """The scan's backward pass on the benchmark layer (Mamba-2.8B shape,
+    bf16): every input gradient for a random dL/dout and dL/dlast_state.
+    The roof counts the decays the gradients need at least once (16 per
+    element, N = 16) on the MUFU; this kernel evaluates them three times
+    (checkpoint pass, segment recompute, reverse pass)."""
+    w = inputs.MAMBA_2_8B
+    d = inputs.scan_inputs(w, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(7)
+    dout = torch.randn(w.batch, w.dim, w.seqlen, generator=g, device="cuda").to(inputs.DTYPES[w.dtype])
+    dlast = torch.randn(w.batch, w.dim, w.dstate, generator=g, device="cuda")
+    ws = torch.empty(binding.load_library().mamba_scan_bwd_workspace_size(w.batch, w.dim, w.seqlen, w.dstate),
+                     device="cuda", dtype=torch.uint8)
+    run = lambda: binding.mamba_scan_bwd(dout, d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"],  # noqa: E731
+                                         z=d["z"], delta_bias=d["delta_bias"], dlast_state=dlast,
+                                         workspace=ws)
+    run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    peak = MUFU_PER_CLK_PER_SM * SM_COUNT * load_peaks()["sm_max_mhz"] * 1e6 / w.dstate / 1e9
+    achieved = w.elements / us / 1e3
+    return {"workload": w.name, "us_per_call": us, "Gelem_per_s": achieved,
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Gelem/s",
+                         "frac": achieved / peak,
+                         "note": "peak = 16 decays per element once on the MUFU; the kernel evaluates them 3x "
+                                 "(checkpoint sweep, segment recompute, reverse sweep)"},
+            "reps": reps}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -436,6 +471,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-conv", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -531,6 +567,8 @@ def main():
         line["decode"] = decode_measure()
     if rank == 0 and not args.no_conv:
         line["conv1d"] = conv1d_measure()
+    if rank == 0 and not args.no_bwd:
+        line["backward"] = backward_measure()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:

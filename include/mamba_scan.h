@@ -260,15 +260,16 @@ int mamba_state_update(float *state, const void *u, const void *delta,
  *   du, ddelta   : act (batch, dim, seqlen), written.
  *   dz           : act (batch, dim, seqlen), written; required iff z is given.
  *   dA           : fp32 (dim, dstate); dB, dC: fp32 (batch, dstate, seqlen);
- *   dD, ddelta_bias : fp32 (dim) or NULL -- all zeroed on `stream`, then
- *                  accumulated (sums over batch rows, channels and time).
+ *   dD, ddelta_bias : fp32 (dim) or NULL -- written (sums over batch rows,
+ *                  channels and time).
  *   workspace    : at least mamba_scan_bwd_workspace_size bytes, 16-byte
  *                  aligned, caller-owned (the states checkpointed every 16
- *                  timesteps).
+ *                  timesteps, and per-32-channel partial sums of dB and dC).
  *
- * dstate <= 16.  The sums over channels use floating-point atomics, so dA,
- * dB, dC, dD and ddelta_bias may differ in the last bits between runs; du,
- * ddelta and dz do not.  Returns MAMBA_OK or a mamba_status_t error.
+ * dstate <= 16.  dA, dD and ddelta_bias add per-channel-group sums with
+ * floating-point atomics, so they may differ in the last bits between runs;
+ * du, ddelta, dz, dB and dC do not.  Returns MAMBA_OK or a mamba_status_t
+ * error.
  */
 int mamba_scan_bwd(const void *u, const void *delta, const float *A,
                    const void *B, const void *C, const float *D,
