@@ -176,6 +176,29 @@ int mamba_scan_fwd_ws(const void *u, const void *delta, const float *A,
                       const mamba_scan_tuning_t *tuning, void *workspace,
                       size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * mamba_scan_fwd_init -- mamba_scan_fwd_ws from a given initial state
+ * instead of zeros: the recurrence starts from h_{-1} = h0 (the pages unroll
+ * it from a zero state; a nonzero start continues an earlier scan -- pass
+ * that scan's last_state -- without replaying it).
+ *
+ *   h0           : fp32 (batch, dim, dstate), required; read only.  It may
+ *                  be the same buffer as last_state (exactly), which then
+ *                  advances in place; any other overlap with an output is
+ *                  rejected.
+ *
+ * All other arguments, results and errors as mamba_scan_fwd_ws (workspace
+ * may be NULL: static schedule).
+ */
+int mamba_scan_fwd_init(const void *u, const void *delta, const float *A,
+                        const void *B, const void *C, const float *D,
+                        const void *z, const float *delta_bias,
+                        int delta_softplus, const float *h0, void *out,
+                        float *last_state, int64_t batch, int64_t dim,
+                        int64_t seqlen, int64_t dstate, int act_dtype,
+                        const mamba_scan_tuning_t *tuning, void *workspace,
+                        size_t workspace_bytes, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads the status a persistent launch left in
  * `workspace`: MAMBA_OK, or MAMBA_ERR_TIMEOUT if a worker stopped waiting for
  * a predecessor chunk (the outputs of that launch are then incomplete).
@@ -263,7 +286,7 @@ int mamba_state_update(float *state, const void *u, const void *delta,
  *   dD, ddelta_bias : fp32 (dim) or NULL -- written (sums over batch rows,
  *                  channels and time).
  *   workspace    : at least mamba_scan_bwd_workspace_size bytes, 16-byte
- *                  aligned, caller-owned (the states checkpointed every 16
+ *                  aligned, caller-owned (the states checkpointed every 8
  *                  timesteps, and per-32-channel partial sums of dB and dC).
  *
  * dstate <= 16.  dA, dD and ddelta_bias add per-channel-group sums with
@@ -280,6 +303,29 @@ int mamba_scan_bwd(const void *u, const void *delta, const float *A,
                    int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
                    int act_dtype, void *workspace, size_t workspace_bytes,
                    cudaStream_t stream);
+
+/*
+ * mamba_scan_bwd_init -- mamba_scan_bwd for a forward that started from the
+ * state h0 (mamba_scan_fwd_init), which also returns the gradient with
+ * respect to that state: dh0 = dL/dh_{-1}, the carried g after timestep 0
+ * (g times that step's Abar).
+ *
+ *   h0           : fp32 (batch, dim, dstate), required; read only.
+ *   dh0          : fp32 (batch, dim, dstate), written, or NULL; must not
+ *                  overlap any other argument.
+ *
+ * All other arguments, results and errors as mamba_scan_bwd.
+ */
+int mamba_scan_bwd_init(const void *u, const void *delta, const float *A,
+                        const void *B, const void *C, const float *D,
+                        const void *z, const float *delta_bias,
+                        int delta_softplus, const float *h0, const void *dout,
+                        const float *dlast_state, void *du, void *ddelta,
+                        float *dA, float *dB, float *dC, float *dD, void *dz,
+                        float *ddelta_bias, float *dh0, int64_t batch,
+                        int64_t dim, int64_t seqlen, int64_t dstate,
+                        int act_dtype, void *workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
 
 /* Bytes of workspace mamba_scan_bwd needs for these sizes (0 when dstate > 16
  * or the sizes are invalid).  Pure host arithmetic. */

@@ -30,7 +30,8 @@ SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT = 0, 1, 2
 # Every function include/mamba_scan.h declares.
 EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
-            "mamba_scan_fwd_noalloc", "mamba_scan_bwd", "mamba_scan_bwd_workspace_size",
+            "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_bwd", "mamba_scan_bwd_init",
+            "mamba_scan_bwd_workspace_size",
             "mamba_state_update", "mamba_conv1d_fwd",
             "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version")
 
@@ -59,6 +60,9 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_fwd_tuned.restype = ci
     lib.mamba_scan_fwd_ws.argtypes = scan_args + [ctypes.POINTER(Tuning), vp, ctypes.c_size_t, vp]
     lib.mamba_scan_fwd_ws.restype = ci
+    lib.mamba_scan_fwd_init.argtypes = scan_args[:9] + [fp] + scan_args[9:] + [
+        ctypes.POINTER(Tuning), vp, ctypes.c_size_t, vp]
+    lib.mamba_scan_fwd_init.restype = ci
     lib.mamba_scan_fwd_noalloc.argtypes = scan_args + [vp]
     lib.mamba_scan_fwd_noalloc.restype = ci
     lib.mamba_scan_plan.argtypes = [i64, i64, i64, i64, ci, ctypes.POINTER(Tuning)]
@@ -73,6 +77,9 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_bwd.argtypes = [vp, vp, fp, vp, vp, fp, vp, fp, ci, vp, fp, vp, vp, fp, fp, fp, fp,
                                    vp, fp, i64, i64, i64, i64, ci, vp, ctypes.c_size_t, vp]
     lib.mamba_scan_bwd.restype = ci
+    bwd = lib.mamba_scan_bwd.argtypes
+    lib.mamba_scan_bwd_init.argtypes = bwd[:9] + [fp] + bwd[9:19] + [fp] + bwd[19:]
+    lib.mamba_scan_bwd_init.restype = ci
     lib.mamba_scan_bwd_workspace_size.argtypes = [i64, i64, i64, i64]
     lib.mamba_scan_bwd_workspace_size.restype = ctypes.c_size_t
     lib.mamba_conv1d_fwd.argtypes = [vp, fp, fp, ci, vp, i64, i64, i64, i64, i64, ci, vp]
@@ -144,7 +151,8 @@ def mamba_scan_fwd(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
                    last_state: Optional[torch.Tensor] = None,
                    return_last_state: bool = False, lanes_per_channel: int = 0,
                    threads_per_block: int = 0, schedule: int = SCHEDULE_AUTO,
-                   workspace: Optional[torch.Tensor] = None, chunk_timesteps: int = 0):
+                   workspace: Optional[torch.Tensor] = None, chunk_timesteps: int = 0,
+                   h0: Optional[torch.Tensor] = None):
     """Selective scan forward on the current CUDA stream.
 
     u, delta, z: (batch, dim, L); B, C: (batch, N, L) -- all one dtype,
@@ -156,6 +164,9 @@ def mamba_scan_fwd(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
     with torch unless given) enables the persistent, load-balanced schedule;
     ``schedule`` / ``lanes_per_channel`` / ``threads_per_block`` force a
     launch configuration (0 = automatic).
+
+    ``h0`` (batch, dim, N) fp32 starts every row's recurrence from that
+    state instead of zeros (it may be ``last_state`` itself).
     """
     if u.dim() != 3:
         raise ValueError("u must be (batch, dim, seqlen)")
@@ -183,6 +194,7 @@ def mamba_scan_fwd(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
     if want_state and last_state is None:
         last_state = torch.empty((batch, dim, N), device=dev, dtype=torch.float32)
     _need(last_state, "last_state", dev, torch.float32, (batch, dim, N))
+    _need(h0, "h0", dev, torch.float32, (batch, dim, N))
     lib = load_library()
     if workspace is None and schedule != SCHEDULE_STATIC:
         nbytes = lib.mamba_scan_workspace_size(batch, dim, L, N, _ACT[act])
@@ -197,9 +209,15 @@ def mamba_scan_fwd(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
     tun = Tuning(int(lanes_per_channel), int(threads_per_block), int(schedule),
                  int(chunk_timesteps))
     with torch.cuda.device(dev):
-        rc = lib.mamba_scan_fwd_ws(*args, ctypes.byref(tun), _ptr(workspace), ws_bytes,
-                                   _stream(dev))
-    _check("mamba_scan_fwd_ws", rc)
+        if h0 is None:
+            fn = "mamba_scan_fwd_ws"
+            rc = lib.mamba_scan_fwd_ws(*args, ctypes.byref(tun), _ptr(workspace), ws_bytes,
+                                       _stream(dev))
+        else:
+            fn = "mamba_scan_fwd_init"
+            rc = lib.mamba_scan_fwd_init(*args[:9], _ptr(h0), *args[9:], ctypes.byref(tun),
+                                         _ptr(workspace), ws_bytes, _stream(dev))
+    _check(fn, rc)
     return (out, last_state) if want_state else out
 
 
@@ -339,12 +357,14 @@ def mamba_scan_bwd(dout: torch.Tensor, u: torch.Tensor, delta: torch.Tensor, A: 
                    B: torch.Tensor, C: torch.Tensor, D: Optional[torch.Tensor] = None,
                    z: Optional[torch.Tensor] = None, delta_bias: Optional[torch.Tensor] = None,
                    delta_softplus: bool = True, dlast_state: Optional[torch.Tensor] = None,
-                   workspace: Optional[torch.Tensor] = None) -> dict:
+                   workspace: Optional[torch.Tensor] = None,
+                   h0: Optional[torch.Tensor] = None) -> dict:
     """Gradients of :func:`mamba_scan_fwd` for dL/dout = ``dout`` (and
     dL/dlast_state = ``dlast_state``).  Returns a dict: du, ddelta, dz (act
     dtype, like u; dz None without z), dA (dim, N), dB, dC (batch, N, L),
     dD, ddelta_bias (dim,) -- fp32 (dD / ddelta_bias None when D / the bias
-    are not given)."""
+    are not given) -- and dh0 (batch, dim, N) fp32 when the forward started
+    from the state ``h0`` (else None)."""
     if u.dim() != 3:
         raise ValueError("u must be (batch, dim, L)")
     batch, dim, L = u.shape
@@ -362,6 +382,7 @@ def mamba_scan_bwd(dout: torch.Tensor, u: torch.Tensor, delta: torch.Tensor, A: 
     _need(D, "D", dev, torch.float32, (dim,))
     _need(delta_bias, "delta_bias", dev, torch.float32, (dim,))
     _need(dlast_state, "dlast_state", dev, torch.float32, (batch, dim, N))
+    _need(h0, "h0", dev, torch.float32, (batch, dim, N))
     lib = load_library()
     need = lib.mamba_scan_bwd_workspace_size(batch, dim, L, N)
     if need == 0:
@@ -374,12 +395,19 @@ def mamba_scan_bwd(dout: torch.Tensor, u: torch.Tensor, delta: torch.Tensor, A: 
          "dA": torch.empty(dim, N, **f32), "dB": torch.empty(batch, N, L, **f32),
          "dC": torch.empty(batch, N, L, **f32),
          "dD": torch.empty(dim, **f32) if D is not None else None,
-         "ddelta_bias": torch.empty(dim, **f32) if delta_bias is not None else None}
+         "ddelta_bias": torch.empty(dim, **f32) if delta_bias is not None else None,
+         "dh0": torch.empty(batch, dim, N, **f32) if h0 is not None else None}
+    head = [_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+            int(bool(delta_softplus))]
+    grads = [_ptr(dout), _ptr(dlast_state), _ptr(r["du"]), _ptr(r["ddelta"]), _ptr(r["dA"]),
+             _ptr(r["dB"]), _ptr(r["dC"]), _ptr(r["dD"]), _ptr(r["dz"]), _ptr(r["ddelta_bias"])]
+    tail = [batch, dim, L, N, _ACT[act], _ptr(workspace), workspace.numel(), _stream(dev)]
     with torch.cuda.device(dev):
-        rc = lib.mamba_scan_bwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
-                                _ptr(delta_bias), int(bool(delta_softplus)), _ptr(dout), _ptr(dlast_state),
-                                _ptr(r["du"]), _ptr(r["ddelta"]), _ptr(r["dA"]), _ptr(r["dB"]), _ptr(r["dC"]),
-                                _ptr(r["dD"]), _ptr(r["dz"]), _ptr(r["ddelta_bias"]), batch, dim, L, N,
-                                _ACT[act], _ptr(workspace), workspace.numel(), _stream(dev))
-    _check("mamba_scan_bwd", rc)
+        if h0 is None:
+            fn = "mamba_scan_bwd"
+            rc = lib.mamba_scan_bwd(*head, *grads, *tail)
+        else:
+            fn = "mamba_scan_bwd_init"
+            rc = lib.mamba_scan_bwd_init(*head, _ptr(h0), *grads, _ptr(r["dh0"]), *tail)
+    _check(fn, rc)
     return r

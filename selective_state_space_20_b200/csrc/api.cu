@@ -56,7 +56,7 @@ int check_sizes(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate) {
 
 int scan_impl(const void *u, const void *delta, const float *A, const void *B, const void *C,
               const float *D, const void *z, const float *delta_bias, int delta_softplus,
-              void *out, float *last_state, int64_t batch, int64_t dim, int64_t seqlen,
+              const float *h0, void *out, float *last_state, int64_t batch, int64_t dim, int64_t seqlen,
               int64_t dstate, int act_dtype, const mamba_scan_tuning_t *tuning,
               void *workspace, size_t ws_bytes, cudaStream_t stream, bool launch,
               mamba_scan_tuning_t *plan_out) {
@@ -83,11 +83,14 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
              overlaps(last_state, nls, D, nd) || overlaps(last_state, nls, delta_bias, nd) ||
              overlaps(last_state, nls, out, nx)))
             return MAMBA_ERR_OVERLAP;
+        // the initial state may be the final-state output itself (in place)
+        if (h0 && (overlaps(h0, nls, out, nx) || bad_alias(last_state, nls, h0, nls, true)))
+            return MAMBA_ERR_OVERLAP;
         if (workspace) {
             if ((reinterpret_cast<uintptr_t>(workspace) & 15) != 0) return MAMBA_ERR_WORKSPACE;
-            const void *ins[] = {u, delta, z, B, C, A, D, delta_bias, out, last_state};
-            const size_t sz[] = {nx, nx, nx, nbc, nbc, nA, nd, nd, nx, nls};
-            for (int i = 0; i < 10; ++i)
+            const void *ins[] = {u, delta, z, B, C, A, D, delta_bias, out, last_state, h0};
+            const size_t sz[] = {nx, nx, nx, nbc, nbc, nA, nd, nd, nx, nls, nls};
+            for (int i = 0; i < 11; ++i)
                 if (overlaps(workspace, ws_bytes, ins[i], sz[i])) return MAMBA_ERR_OVERLAP;
         }
     }
@@ -112,7 +115,7 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
 
     mscan::ScanArgs a;
     a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z;
-    a.A = A; a.D = D; a.delta_bias = delta_bias; a.out = out; a.last_state = last_state;
+    a.A = A; a.D = D; a.delta_bias = delta_bias; a.out = out; a.last_state = last_state; a.h0 = h0;
     a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = (int)dstate;
     a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
 
@@ -169,7 +172,7 @@ int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void 
                    int delta_softplus, void *out, float *last_state, int64_t batch,
                    int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
                    cudaStream_t stream) {
-    return scan_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, last_state,
+    return scan_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, out, last_state,
                      batch, dim, seqlen, dstate, act_dtype, nullptr, nullptr, 0, stream, true,
                      nullptr);
 }
@@ -180,7 +183,7 @@ int mamba_scan_fwd_tuned(const void *u, const void *delta, const float *A, const
                          float *last_state, int64_t batch, int64_t dim, int64_t seqlen,
                          int64_t dstate, int act_dtype, const mamba_scan_tuning_t *tuning,
                          cudaStream_t stream) {
-    return scan_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, last_state,
+    return scan_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, out, last_state,
                      batch, dim, seqlen, dstate, act_dtype, tuning, nullptr, 0, stream, true,
                      nullptr);
 }
@@ -191,7 +194,19 @@ int mamba_scan_fwd_ws(const void *u, const void *delta, const float *A, const vo
                       int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
                       const mamba_scan_tuning_t *tuning, void *workspace,
                       size_t workspace_bytes, cudaStream_t stream) {
-    return scan_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, last_state,
+    return scan_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, out, last_state,
+                     batch, dim, seqlen, dstate, act_dtype, tuning, workspace, workspace_bytes,
+                     stream, true, nullptr);
+}
+
+int mamba_scan_fwd_init(const void *u, const void *delta, const float *A, const void *B,
+                        const void *C, const float *D, const void *z, const float *delta_bias,
+                        int delta_softplus, const float *h0, void *out, float *last_state,
+                        int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
+                        const mamba_scan_tuning_t *tuning, void *workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+    if (!h0) return MAMBA_ERR_NULL;
+    return scan_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, out, last_state,
                      batch, dim, seqlen, dstate, act_dtype, tuning, workspace, workspace_bytes,
                      stream, true, nullptr);
 }
@@ -216,7 +231,7 @@ int mamba_scan_plan(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate, 
                     mamba_scan_tuning_t *plan) {
     if (!plan) return MAMBA_ERR_NULL;
     return scan_impl(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 1,
-                     nullptr, nullptr, batch, dim, seqlen, dstate, act_dtype, nullptr, nullptr, 0,
+                     nullptr, nullptr, nullptr, batch, dim, seqlen, dstate, act_dtype, nullptr, nullptr, 0,
                      nullptr, false, plan);
 }
 
@@ -257,12 +272,14 @@ size_t mamba_scan_bwd_workspace_size(int64_t batch, int64_t dim, int64_t seqlen,
     return mscan::scan_bwd_workspace_bytes(batch, dim, seqlen);
 }
 
-int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void *B, const void *C,
-                   const float *D, const void *z, const float *delta_bias, int delta_softplus,
-                   const void *dout, const float *dlast_state, void *du, void *ddelta, float *dA,
-                   float *dB, float *dC, float *dD, void *dz, float *ddelta_bias, int64_t batch,
-                   int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype, void *workspace,
-                   size_t workspace_bytes, cudaStream_t stream) {
+namespace {
+int scan_bwd_impl(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                  const float *D, const void *z, const float *delta_bias, int delta_softplus,
+                  const float *h0, const void *dout, const float *dlast_state, void *du,
+                  void *ddelta, float *dA, float *dB, float *dC, float *dD, void *dz,
+                  float *ddelta_bias, float *dh0, int64_t batch, int64_t dim, int64_t seqlen,
+                  int64_t dstate, int act_dtype, void *workspace, size_t workspace_bytes,
+                  cudaStream_t stream) {
     if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
     int rc = check_sizes(batch, dim, seqlen, dstate);
     if (rc != MAMBA_OK) return rc;
@@ -276,12 +293,12 @@ int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void 
     const size_t nx = (size_t)(batch * dim * seqlen) * es, nbc = (size_t)(batch * dstate * seqlen) * es;
     const size_t nbc32 = (size_t)(batch * dstate * seqlen) * 4, nA = (size_t)(dim * dstate) * 4;
     const size_t nd = (size_t)dim * 4, ns = (size_t)(batch * dim * dstate) * 4;
-    const void *ins[] = {u, delta, z, dout, B, C, A, D, delta_bias, dlast_state, workspace};
-    const size_t inb[] = {nx, nx, nx, nx, nbc, nbc, nA, nd, nd, ns, need};
-    void *outs[] = {du, ddelta, dz, dA, dB, dC, dD, ddelta_bias};
-    const size_t outb[] = {nx, nx, nx, nA, nbc32, nbc32, nd, nd};
-    for (int i = 0; i < 8; ++i) {
-        for (int k = 0; k < 11; ++k)
+    const void *ins[] = {u, delta, z, dout, B, C, A, D, delta_bias, dlast_state, workspace, h0};
+    const size_t inb[] = {nx, nx, nx, nx, nbc, nbc, nA, nd, nd, ns, need, ns};
+    void *outs[] = {du, ddelta, dz, dA, dB, dC, dD, ddelta_bias, dh0};
+    const size_t outb[] = {nx, nx, nx, nA, nbc32, nbc32, nd, nd, ns};
+    for (int i = 0; i < 9; ++i) {
+        for (int k = 0; k < 12; ++k)
             if (overlaps(outs[i], outb[i], ins[k], inb[k])) return MAMBA_ERR_OVERLAP;
         for (int k = 0; k < i; ++k)
             if (overlaps(outs[i], outb[i], outs[k], outb[k])) return MAMBA_ERR_OVERLAP;
@@ -291,12 +308,37 @@ int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void 
     if (status != MAMBA_OK) return status;
     mscan::ScanBwdArgs a;
     a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z; a.dout = dout;
-    a.A = A; a.D = D; a.delta_bias = delta_bias; a.dlast = dlast_state;
+    a.A = A; a.D = D; a.delta_bias = delta_bias; a.dlast = dlast_state; a.h0 = h0;
     a.du = du; a.ddelta = ddelta; a.dz = dz;
-    a.dA = dA; a.dB = dB; a.dC = dC; a.dD = dD; a.ddelta_bias = ddelta_bias;
+    a.dA = dA; a.dB = dB; a.dC = dC; a.dD = dD; a.ddelta_bias = ddelta_bias; a.dh0 = dh0;
     a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = (int)dstate;
     a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
     return mscan::launch_scan_bwd(a, workspace, sms, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+}  // namespace
+
+int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                   const float *D, const void *z, const float *delta_bias, int delta_softplus,
+                   const void *dout, const float *dlast_state, void *du, void *ddelta, float *dA,
+                   float *dB, float *dC, float *dD, void *dz, float *ddelta_bias, int64_t batch,
+                   int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype, void *workspace,
+                   size_t workspace_bytes, cudaStream_t stream) {
+    return scan_bwd_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, nullptr, dout,
+                         dlast_state, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, nullptr, batch,
+                         dim, seqlen, dstate, act_dtype, workspace, workspace_bytes, stream);
+}
+
+int mamba_scan_bwd_init(const void *u, const void *delta, const float *A, const void *B,
+                        const void *C, const float *D, const void *z, const float *delta_bias,
+                        int delta_softplus, const float *h0, const void *dout,
+                        const float *dlast_state, void *du, void *ddelta, float *dA, float *dB,
+                        float *dC, float *dD, void *dz, float *ddelta_bias, float *dh0,
+                        int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
+                        void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (!h0) return MAMBA_ERR_NULL;
+    return scan_bwd_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, dout,
+                         dlast_state, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, dh0, batch,
+                         dim, seqlen, dstate, act_dtype, workspace, workspace_bytes, stream);
 }
 
 int mamba_conv1d_fwd(const void *x, const float *weight, const float *bias, int apply_silu,
@@ -369,6 +411,6 @@ const char *mamba_status_string(int status) {
     }
 }
 
-int mamba_abi_version(void) { return (1 << 16) | 2; }
+int mamba_abi_version(void) { return (1 << 16) | 3; }
 
 }  // extern "C"

@@ -14,6 +14,7 @@ struct ScanArgs {
     const float *A, *D, *delta_bias;
     void *out;
     float *last_state;
+    const float *h0;  // initial state (batch, dim, dstate) or null (zeros)
     int64_t batch, dim, seqlen;
     int dstate;
     int softplus;
@@ -73,8 +74,10 @@ struct Conv1dUpdateArgs {
 struct ScanBwdArgs {
     const void *u, *delta, *B, *C, *z, *dout;
     const float *A, *D, *delta_bias, *dlast;
+    const float *h0;                                 // initial state (batch, dim, N) or null (zeros)
     void *du, *ddelta, *dz;                          // act (batch, dim, L)
     float *dA, *dB, *dC, *dD, *ddelta_bias;          // fp32, accumulated from zero
+    float *dh0;                                      // fp32 (batch, dim, N) or null
     int64_t batch, dim, seqlen;
     int dstate, softplus, act;
 };

@@ -32,6 +32,7 @@ struct Params {
     const float *A, *D, *delta_bias;
     void *out;
     float *last_state;
+    const float *h0;       // initial state (batch, dim, dstate) or null (zeros)
     int64_t dim, seqlen;
     int dstate;
     int softplus;

@@ -142,7 +142,7 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
     persist::Params kp;
     kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
     kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias;
-    kp.out = a.out; kp.last_state = a.last_state;
+    kp.out = a.out; kp.last_state = a.last_state; kp.h0 = a.h0;
     kp.dim = a.dim; kp.seqlen = a.seqlen; kp.dstate = a.dstate; kp.softplus = a.softplus;
     kp.group_channels = group_channels(lanes);
     kp.groups_per_batch = (int)((a.dim + kp.group_channels - 1) / kp.group_channels);

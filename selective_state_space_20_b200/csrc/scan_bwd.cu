@@ -11,6 +11,7 @@
 //   ddelta += g[n] (h_{t-1}[n] Abar A[n] + B[n,t] u);  dA[n] += g[n] h_{t-1}[n] Abar delta
 //   dB[n,t] += g[n] delta u;  du += g[n] delta B[n,t];  g[n] *= Abar
 //   ddelta_raw = ddelta sigmoid(delta_raw + bias) (softplus);  dbias += ddelta_raw
+// and, when the forward started from a given state h0, dh0 = g after t = 0.
 //
 // Design.  One lane per channel with all (<= 16) states in registers; a warp
 // takes a group of 32 channels of one batch row through the whole sequence,
@@ -41,9 +42,9 @@ constexpr int kWarpsBwd = 4;  // warps per block
 
 struct BwdParams {
     const void *u, *delta, *B, *C, *z, *dout;
-    const float *A, *D, *delta_bias, *dlast;
+    const float *A, *D, *delta_bias, *dlast, *h0;
     void *du, *ddelta, *dz;
-    float *dA, *dB, *dC, *dD, *dbias;
+    float *dA, *dB, *dC, *dD, *dbias, *dh0;
     float *ckpt;  // workspace: n_groups x n_segs x 32 lanes x kNS checkpointed states
     float *part;  // workspace: n_groups x seqlen x 32 partial dB (lanes 0-15) / dC (16-31) sums
     int vec;      // rows 16-byte aligned and a whole number of 16-byte chunks
@@ -206,10 +207,10 @@ __global__ void __launch_bounds__(kWarpsBwd * 32) scan_bwd_kernel(const BwdParam
             }
         };
 
-        // ---- forward: checkpoints every kSeg timesteps (state before the segment)
+        // ---- forward from h0 (or zeros): checkpoints every kSeg timesteps (state before the segment)
         float h[kNS];
 #pragma unroll
-        for (int n = 0; n < kNS; ++n) h[n] = 0.f;
+        for (int n = 0; n < kNS; ++n) h[n] = (valid && p.h0 && n < N) ? __ldg(p.h0 + (b * p.dim + dc) * N + n) : 0.f;
         for (int seg = 0; seg < p.n_segs; ++seg) {
             const int64_t t0 = (int64_t)seg * kSeg;
             const int tn = (L - t0) < kSeg ? (int)(L - t0) : kSeg;
@@ -322,8 +323,10 @@ __global__ void __launch_bounds__(kWarpsBwd * 32) scan_bwd_kernel(const BwdParam
         }
         if (valid) {
 #pragma unroll
-            for (int n = 0; n < kNS; ++n)
+            for (int n = 0; n < kNS; ++n) {
                 if (n < N) atomicAdd(p.dA + dc * N + n, dA_acc[n]);
+                if (n < N && p.dh0) p.dh0[(b * p.dim + dc) * N + n] = g[n];  // dL/dh_{-1}
+            }
             if (p.dD) atomicAdd(p.dD + dc, dD_acc);
             if (p.dbias) atomicAdd(p.dbias + dc, dbias_acc);
         }
@@ -398,9 +401,9 @@ size_t scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen) {
 cudaError_t launch_scan_bwd(const ScanBwdArgs &a, void *workspace, int sm_count, cudaStream_t st) {
     BwdParams p;
     p.u = a.u; p.delta = a.delta; p.B = a.B; p.C = a.C; p.z = a.z; p.dout = a.dout;
-    p.A = a.A; p.D = a.D; p.delta_bias = a.delta_bias; p.dlast = a.dlast;
+    p.A = a.A; p.D = a.D; p.delta_bias = a.delta_bias; p.dlast = a.dlast; p.h0 = a.h0;
     p.du = a.du; p.ddelta = a.ddelta; p.dz = a.dz;
-    p.dA = a.dA; p.dB = a.dB; p.dC = a.dC; p.dD = a.dD; p.dbias = a.ddelta_bias;
+    p.dA = a.dA; p.dB = a.dB; p.dC = a.dC; p.dD = a.dD; p.dbias = a.ddelta_bias; p.dh0 = a.dh0;
     p.ckpt = static_cast<float *>(workspace);
     p.part = p.ckpt + (size_t)((a.batch * ((a.dim + 31) / 32)) * ((a.seqlen + kSeg - 1) / kSeg)) * 32 * kNS;
     {

@@ -43,6 +43,7 @@ struct KParams {
     const float *A, *D, *delta_bias;
     void *out;
     float *last_state;
+    const float *h0;
     int64_t dim, seqlen;
     int64_t n_groups;  // channel groups per batch row
     int dstate;
@@ -162,7 +163,7 @@ scan_fwd_kernel(const KParams p) {
     for (int s = 0; s < S; ++s) {
         const int n = r * S + s;
         A2[s] = (d < Dm && n < N) ? __ldg(p.A + d * N + n) * kLog2e : 0.f;
-        h[s] = 0.f;
+        h[s] = (p.h0 && d < Dm && n < N) ? __ldcg(p.h0 + (b * Dm + d) * N + n) : 0.f;
     }
 
     // ---- copy one chunk's raw tiles into stage `st`
@@ -399,7 +400,7 @@ cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &pl, cudaStream_t 
     KParams kp;
     kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
     kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias;
-    kp.out = a.out; kp.last_state = a.last_state;
+    kp.out = a.out; kp.last_state = a.last_state; kp.h0 = a.h0;
     kp.dim = a.dim; kp.seqlen = a.seqlen;
     kp.n_groups = (a.dim + pl.channels_per_block - 1) / pl.channels_per_block;
     kp.dstate = a.dstate; kp.softplus = a.softplus; kp.vec = pl.vectorized;

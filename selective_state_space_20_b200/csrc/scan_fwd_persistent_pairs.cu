@@ -433,6 +433,17 @@ scan_fwd_pairs_kernel(const Params p) {
         }
         };
 
+        // the state before sub-chunk 0: the initial state, or zeros
+        auto load_h0 = [&](float2 (&hh)[S / 2]) {
+#pragma unroll
+            for (int k = 0; k < S / 2; ++k) {
+                const int n0 = S * sr + 2 * k;
+                const float *src = p.h0 + (b * Dm + ds) * N;
+                hh[k] = (p.h0 && ds < Dm) ? make_float2(n0 < N ? __ldcg(src + n0) : 0.f,
+                                                        n0 + 1 < N ? __ldcg(src + n0 + 1) : 0.f)
+                                          : make_float2(0.f, 0.f);
+            }
+        };
         float2 h[S / 2];
 #pragma unroll
         for (int k = 0; k < S / 2; ++k) h[k] = make_float2(0.f, 0.f);
@@ -448,11 +459,11 @@ scan_fwd_pairs_kernel(const Params p) {
             // after the other; the output run follows from h_in.
             run_subs(true, h, dsum, false);
             float2 hin[S / 2];
-#pragma unroll
-            for (int k = 0; k < S / 2; ++k) hin[k] = make_float2(0.f, 0.f);
             if (sb > 0) {
                 if (!wait_progress(p, lane, g, sb)) return;
                 load_carry(hin);
+            } else {
+                load_h0(hin);
             }
             float2 hend[S / 2];
 #pragma unroll
@@ -469,6 +480,8 @@ scan_fwd_pairs_kernel(const Params p) {
             if (sb > 0) {
                 if (!wait_progress(p, lane, g, sb)) return;
                 load_carry(h);
+            } else {
+                load_h0(h);
             }
             run_subs(false, h, dsum, true);
         }

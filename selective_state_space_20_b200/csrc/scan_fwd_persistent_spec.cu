@@ -425,9 +425,13 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
                         A2[q] = f2(a0 * kLog2e, a1 * kLog2e);
                     }
                 }
-                if (d.j == 0) {
+                if (d.j == 0) {  // the initial state, or zeros
+                    const float *src = p.h0 + (d.rowidx + lane) * N;
 #pragma unroll
-                    for (int q = 0; q < kNS / 2; ++q) hs[q] = f2(0.f, 0.f);
+                    for (int q = 0; q < kNS / 2; ++q)
+                        hs[q] = (p.h0 && dc < p.dim) ? f2(2 * q < N ? __ldcg(src + 2 * q) : 0.f,
+                                                          2 * q + 1 < N ? __ldcg(src + 2 * q + 1) : 0.f)
+                                                     : f2(0.f, 0.f);
                 } else {
 #pragma unroll
                     for (int q = 0; q < kNS / 4; ++q) {

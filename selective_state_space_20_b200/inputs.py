@@ -208,3 +208,13 @@ def conv_inputs(batch: int, dim: int, seqlen: int, width: int = 4, dtype: str = 
     rows = 2 * dim if wide else dim
     x = _normal((batch, rows, seqlen), g, device, DTYPES[dtype])
     return {"xz" if wide else "x": x, "weight": weight, "bias": bias}
+
+
+def initial_state(batch: int, dim: int, dstate: int, seed: int = 50, device="cpu",
+                  scale: float = 0.25) -> torch.Tensor:
+    """A seeded fp32 state (batch, dim, dstate) to start a scan from: normal
+    values times ``scale``.  The default is about the spread of the states a
+    scan of unit-variance inputs leaves behind: h_t = a h_{t-1} + delta B u
+    with a = exp(delta A) settles at variance delta^2 / (1 - a^2), close to
+    delta / (2 |A|) = 0.05 for delta = 0.1, A = -1."""
+    return _normal((batch, dim, dstate), _gen(seed, device), device, torch.float32, scale)

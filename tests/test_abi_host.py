@@ -84,6 +84,20 @@ def test_overlap_rejected(lib):
     assert _scan(lib, {"out": 0x600000}, last=ctypes.c_void_p(0x600010)) == -7
 
 
+def test_initial_state_validation(lib):
+    vp = ctypes.c_void_p
+    tun = binding.Tuning(0, 0, 0, 0)
+
+    def init(h0, last=None):
+        args = [vp(0x100000), vp(0x200000), vp(0x300000), vp(0x400000), vp(0x500000), None, None,
+                None, 1, h0, vp(0x600000), last, 2, 4, 8, 16, 1]
+        return lib.mamba_scan_fwd_init(*args, ctypes.byref(tun), None, 0, None)
+
+    assert init(None) == -1                                   # h0 is required
+    assert init(vp(0x600000 + 4)) == -7                       # h0 inside out
+    assert init(vp(0x700000), last=vp(0x700000 + 16)) == -7   # partly overlaps last_state
+
+
 def test_bad_tuning_rejected(lib):
     assert _scan(lib, tuning=binding.Tuning(3, 0, 0, 0)) == -3
     assert _scan(lib, tuning=binding.Tuning(0, 100, 0, 0)) == -3
@@ -172,3 +186,11 @@ def test_scan_bwd_validation(lib):
     assert call(N=32) == -3
     assert call(ws=None) == -8 and call(wsb=ws_n - 1) == -8 and call(ws=vp(0x1000008)) == -8
     assert call(dB=vp(0x400000 + 64)) == -7  # dB inside B
+
+    # the initial-state form: h0 after the softplus flag, dh0 after dbias
+    def call_init(h0, dh0):
+        a = ok[:9] + [h0] + ok[9:19] + [dh0] + ok[19:]
+        return lib.mamba_scan_bwd_init(*a)
+    assert call_init(None, None) == -1                     # h0 is required
+    assert call_init(P[13], vp(0x600000 + 128)) == -7      # dh0 inside dout
+    assert call_init(P[13], P[13]) == -7                   # dh0 over h0

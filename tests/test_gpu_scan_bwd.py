@@ -16,7 +16,7 @@ FP32_GRADS = ("dA", "dB", "dC", "dD", "ddelta_bias")
 ACT_GRADS = ("du", "ddelta", "dz")
 
 
-def check_bwd(batch, dim, L, N, dtype, seed, gate=True, softplus=True, dlast=True, drop=()):
+def check_bwd(batch, dim, L, N, dtype, seed, gate=True, softplus=True, dlast=True, drop=(), h0=False):
     w = inputs.custom(batch, dim, L, N, dtype, seed=seed)
     cpu = inputs.scan_inputs(w)
     if not gate:
@@ -30,19 +30,21 @@ def check_bwd(batch, dim, L, N, dtype, seed, gate=True, softplus=True, dlast=Tru
     g = torch.Generator().manual_seed(seed + 1)
     dout = torch.randn(batch, dim, L, generator=g).to(inputs.DTYPES[dtype])
     dl = torch.randn(batch, dim, N, generator=g) if dlast else None
+    hs = inputs.initial_state(batch, dim, N, seed=seed + 2) if h0 else None
     dev = {k: (None if v is None else v.cuda()) for k, v in cpu.items()}
     got = binding.mamba_scan_bwd(dout.cuda(), dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"],
                                  D=dev["D"], z=dev["z"], delta_bias=dev["delta_bias"],
-                                 delta_softplus=softplus, dlast_state=None if dl is None else dl.cuda())
+                                 delta_softplus=softplus, dlast_state=None if dl is None else dl.cuda(),
+                                 h0=None if hs is None else hs.cuda())
     ref = oracle.scan_bwd(dout, cpu["u"], cpu["delta"], cpu["A"], cpu["B"], cpu["C"], D=cpu["D"], z=cpu["z"],
-                          delta_bias=cpu["delta_bias"], delta_softplus=softplus,
+                          delta_bias=cpu["delta_bias"], delta_softplus=softplus, h0=hs,
                           dlast=None if dl is None else dl.double())
     errs = {}
-    for k in FP32_GRADS + ACT_GRADS:
+    for k in FP32_GRADS + ACT_GRADS + (("dh0",) if h0 else ()):
         if got.get(k) is None:
             continue
         errs[k] = rel_err(to_np(got[k]), ref[k])
-    record(f"scan_bwd {batch}x{dim}x{L} N{N} {dtype} gate={gate} sp={softplus} dlast={dlast}", **errs)
+    record(f"scan_bwd {batch}x{dim}x{L} N{N} {dtype} gate={gate} sp={softplus} dlast={dlast} h0={h0}", **errs)
     for k, e in errs.items():
         tol = TOL[inputs.DTYPES[dtype]] if k in ACT_GRADS else 1e-3
         assert e <= tol, (k, e, errs)
@@ -60,6 +62,14 @@ def test_bwd_matches_oracle(dtype, shape):
 def test_bwd_flags(gate, softplus, dlast):
     for dtype in ("fp32", "bf16"):
         check_bwd(2, 40, 80, 16, dtype, seed=7, gate=gate, softplus=softplus, dlast=dlast)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("shape", [(2, 37, 100, 16), (3, 20, 33, 5), (1, 64, 257, 16)])
+@pytest.mark.parametrize("dlast", [True, False])
+def test_bwd_from_an_initial_state(dtype, shape, dlast):
+    """The forward started from h0: every gradient, and dh0 = dL/dh_{-1}."""
+    check_bwd(*shape, dtype, seed=sum(shape) + 3, dlast=dlast, h0=True)
 
 
 def test_bwd_without_D_and_bias():
