@@ -199,6 +199,58 @@ int mamba_scan_fwd_init(const void *u, const void *delta, const float *A,
                         const mamba_scan_tuning_t *tuning, void *workspace,
                         size_t workspace_bytes, cudaStream_t stream);
 
+/* Element strides of one sequence tensor: along the batch, along its rows
+ * (channels for u / delta / z / out, states for B / C) and along time. */
+typedef struct {
+    int64_t batch;
+    int64_t row;
+    int64_t time;
+} mamba_stride3_t;
+
+typedef struct {
+    mamba_stride3_t u, delta, z, out, B, C;
+} mamba_scan_strides_t;
+
+/*
+ * mamba_scan_fwd_strided -- mamba_scan_fwd_init with every sequence tensor
+ * given by its own element strides instead of the dense (batch, dim, seqlen)
+ * / (batch, dstate, seqlen) layout.  This reads a model's activations where
+ * they already are: the (batch, seqlen, dim) layout the pages' Keras listing
+ * uses (channels contiguous, "b l d"), slices of a wider projection output
+ * (x and z as the two halves of one (batch, seqlen, 2 dim) tensor; B and C as
+ * columns of one (batch, seqlen, R + 2 dstate) tensor), B or C shared by
+ * every batch row (batch stride 0), or the dense layout itself.
+ *
+ *   strides      : element strides (>= 0) of u, delta, z, out, B and C;
+ *                  NULL means dense.  z's entry is ignored when z is NULL.
+ *   h0           : fp32 (batch, dim, dstate) or NULL (zeros); as for
+ *                  mamba_scan_fwd_init.
+ *   out          : its strides must not map two elements to one address.
+ *                  out may be u, delta or z in place only with the same
+ *                  pointer and strides; any other overlap of out, last_state
+ *                  or h0 with an input is rejected (MAMBA_ERR_OVERLAP, judged
+ *                  on each tensor's address span).
+ *   tuning       : NULL, or schedule AUTO / STATIC with optional lanes and
+ *                  threads (the persistent schedule needs the dense layout).
+ *
+ * Uses the static schedule.  16-byte copies are used where a tensor allows
+ * them: channel-contiguous u / delta / z / out (row stride 1) with 16-byte-
+ * aligned pointers, batch and time strides multiples of 8 (bf16) or 4 (fp32)
+ * elements and dim a multiple of the same; time-contiguous ones likewise
+ * with the row stride and seqlen; B and C likewise along time or along
+ * states.  Anything else is read and written element by element (correct,
+ * slower).  Other arguments, results and errors as mamba_scan_fwd.
+ */
+int mamba_scan_fwd_strided(const void *u, const void *delta, const float *A,
+                           const void *B, const void *C, const float *D,
+                           const void *z, const float *delta_bias,
+                           int delta_softplus, const float *h0, void *out,
+                           float *last_state, int64_t batch, int64_t dim,
+                           int64_t seqlen, int64_t dstate, int act_dtype,
+                           const mamba_scan_strides_t *strides,
+                           const mamba_scan_tuning_t *tuning,
+                           cudaStream_t stream);
+
 /* Synchronises `stream`, then reads the status a persistent launch left in
  * `workspace`: MAMBA_OK, or MAMBA_ERR_TIMEOUT if a worker stopped waiting for
  * a predecessor chunk (the outputs of that launch are then incomplete).

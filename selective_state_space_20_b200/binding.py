@@ -30,7 +30,7 @@ SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT = 0, 1, 2
 # Every function include/mamba_scan.h declares.
 EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
-            "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_bwd", "mamba_scan_bwd_init",
+            "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_fwd_strided", "mamba_scan_bwd", "mamba_scan_bwd_init",
             "mamba_scan_bwd_workspace_size",
             "mamba_state_update", "mamba_conv1d_fwd",
             "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version")
@@ -45,6 +45,15 @@ class MambaError(RuntimeError):
 class Tuning(ctypes.Structure):
     _fields_ = [("lanes_per_channel", ctypes.c_int), ("threads_per_block", ctypes.c_int),
                 ("schedule", ctypes.c_int), ("chunk_timesteps", ctypes.c_int)]
+
+
+class Stride3(ctypes.Structure):
+    """Element strides of one sequence tensor (batch, row, time)."""
+    _fields_ = [("batch", ctypes.c_int64), ("row", ctypes.c_int64), ("time", ctypes.c_int64)]
+
+
+class ScanStrides(ctypes.Structure):
+    _fields_ = [(k, Stride3) for k in ("u", "delta", "z", "out", "B", "C")]
 
 
 _lock = threading.Lock()
@@ -63,6 +72,9 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_fwd_init.argtypes = scan_args[:9] + [fp] + scan_args[9:] + [
         ctypes.POINTER(Tuning), vp, ctypes.c_size_t, vp]
     lib.mamba_scan_fwd_init.restype = ci
+    lib.mamba_scan_fwd_strided.argtypes = scan_args[:9] + [fp] + scan_args[9:] + [
+        ctypes.POINTER(ScanStrides), ctypes.POINTER(Tuning), vp]
+    lib.mamba_scan_fwd_strided.restype = ci
     lib.mamba_scan_fwd_noalloc.argtypes = scan_args + [vp]
     lib.mamba_scan_fwd_noalloc.restype = ci
     lib.mamba_scan_plan.argtypes = [i64, i64, i64, i64, ci, ctypes.POINTER(Tuning)]
@@ -218,6 +230,77 @@ def mamba_scan_fwd(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
             rc = lib.mamba_scan_fwd_init(*args[:9], _ptr(h0), *args[9:], ctypes.byref(tun),
                                          _ptr(workspace), ws_bytes, _stream(dev))
     _check(fn, rc)
+    return (out, last_state) if want_state else out
+
+
+def _need_strided(t: Optional[torch.Tensor], name: str, device, dtype, shape):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _stride3(t: Optional[torch.Tensor]) -> Stride3:
+    return Stride3(0, 0, 0) if t is None else Stride3(*t.stride())
+
+
+def mamba_scan_fwd_strided(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
+                           B: torch.Tensor, C: torch.Tensor, D: Optional[torch.Tensor] = None,
+                           z: Optional[torch.Tensor] = None,
+                           delta_bias: Optional[torch.Tensor] = None,
+                           delta_softplus: bool = True, out: Optional[torch.Tensor] = None,
+                           last_state: Optional[torch.Tensor] = None,
+                           return_last_state: bool = False, h0: Optional[torch.Tensor] = None,
+                           lanes_per_channel: int = 0, threads_per_block: int = 0):
+    """:func:`mamba_scan_fwd` on tensors with any strides: u, delta, z (and
+    out) of logical shape (batch, dim, L) and B, C of (batch, N, L), each
+    laid out however it is -- e.g. ``x.transpose(1, 2)`` of a (batch, L, dim)
+    activation, or a slice of a wider projection output.  ``out`` is
+    allocated channel-contiguous like u when u is.  Static schedule."""
+    if u.dim() != 3:
+        raise ValueError("u must be (batch, dim, seqlen)")
+    batch, dim, L = u.shape
+    if A.dim() != 2:
+        raise ValueError("A must be (dim, dstate)")
+    N = A.shape[1]
+    dev, act = u.device, u.dtype
+    if dev.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    if act not in _ACT:
+        raise TypeError(f"unsupported activation dtype {act}")
+    for name, t in (("u", u), ("delta", delta), ("z", z)):
+        _need_strided(t, name, dev, act, (batch, dim, L))
+    _need_strided(B, "B", dev, act, (batch, N, L))
+    _need_strided(C, "C", dev, act, (batch, N, L))
+    _need(A, "A", dev, torch.float32, (dim, N))
+    _need(D, "D", dev, torch.float32, (dim,))
+    _need(delta_bias, "delta_bias", dev, torch.float32, (dim,))
+    if out is None:
+        if u.stride(1) == 1 and L > 1:
+            out = torch.empty((batch, L, dim), device=dev, dtype=act).transpose(1, 2)
+        else:
+            out = torch.empty((batch, dim, L), device=dev, dtype=act)
+    _need_strided(out, "out", dev, act, (batch, dim, L))
+    want_state = return_last_state or last_state is not None
+    if want_state and last_state is None:
+        last_state = torch.empty((batch, dim, N), device=dev, dtype=torch.float32)
+    _need(last_state, "last_state", dev, torch.float32, (batch, dim, N))
+    _need(h0, "h0", dev, torch.float32, (batch, dim, N))
+    st = ScanStrides(_stride3(u), _stride3(delta), _stride3(z), _stride3(out), _stride3(B), _stride3(C))
+    tun = Tuning(int(lanes_per_channel), int(threads_per_block), SCHEDULE_STATIC, 0)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        rc = lib.mamba_scan_fwd_strided(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                                        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(h0), _ptr(out),
+                                        _ptr(last_state), batch, dim, L, N, _ACT[act], ctypes.byref(st),
+                                        ctypes.byref(tun), _stream(dev))
+    _check("mamba_scan_fwd_strided", rc)
     return (out, last_state) if want_state else out
 
 

@@ -116,6 +116,7 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
     mscan::ScanArgs a;
     a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z;
     a.A = A; a.D = D; a.delta_bias = delta_bias; a.out = out; a.last_state = last_state; a.h0 = h0;
+    a.strides = nullptr;
     a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = (int)dstate;
     a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
 
@@ -163,9 +164,130 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
     return mscan::launch_scan_fwd(a, pl, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 
+// A strided tensor: its first byte and the bytes up to its last element
+// (strides >= 0); false when an offset would not fit the int64 indexing.
+struct Span {
+    uintptr_t lo;
+    size_t bytes;
+};
+bool strided_span(const void *p, const mamba_stride3_t &s, int64_t nb, int64_t nr, int64_t nt,
+                  size_t es, Span *out) {
+    if (s.batch < 0 || s.row < 0 || s.time < 0) return false;
+    const double last = (double)(nb - 1) * (double)s.batch + (double)(nr - 1) * (double)s.row +
+                        (double)(nt - 1) * (double)s.time;
+    if (last > (double)kMaxElems) return false;
+    out->lo = reinterpret_cast<uintptr_t>(p);
+    out->bytes = p ? (size_t)((nb - 1) * s.batch + (nr - 1) * s.row + (nt - 1) * s.time + 1) * es : 0;
+    return true;
+}
+bool spans_overlap(const Span &a, const Span &b) {
+    if (!a.bytes || !b.bytes) return false;
+    return a.lo < b.lo + b.bytes && b.lo < a.lo + a.bytes;
+}
+// No two elements at one address: ordered by stride, each extent's step
+// clears everything the smaller strides reach (extents of 1 are ignored).
+bool injective(const mamba_stride3_t &s, int64_t nb, int64_t nr, int64_t nt) {
+    int64_t st[3] = {s.batch, s.row, s.time}, ex[3] = {nb, nr, nt};
+    for (int i = 0; i < 3; ++i)
+        for (int j = i + 1; j < 3; ++j)
+            if (ex[j] > 1 && (ex[i] <= 1 || st[j] < st[i])) {
+                int64_t t = st[i]; st[i] = st[j]; st[j] = t;
+                t = ex[i]; ex[i] = ex[j]; ex[j] = t;
+            }
+    int64_t reach = 0;  // largest offset reachable with the smaller strides
+    for (int i = 0; i < 3; ++i) {
+        if (ex[i] <= 1) continue;
+        if (st[i] <= reach) return false;
+        reach += (ex[i] - 1) * st[i];
+    }
+    return true;
+}
+bool same_stride(const mamba_stride3_t &a, const mamba_stride3_t &b) {
+    return a.batch == b.batch && a.row == b.row && a.time == b.time;
+}
+
 }  // namespace
 
 extern "C" {
+
+int mamba_scan_fwd_strided(const void *u, const void *delta, const float *A, const void *B,
+                           const void *C, const float *D, const void *z, const float *delta_bias,
+                           int delta_softplus, const float *h0, void *out, float *last_state,
+                           int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                           int act_dtype, const mamba_scan_strides_t *strides,
+                           const mamba_scan_tuning_t *tuning, cudaStream_t stream) {
+    if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
+    int rc = check_sizes(batch, dim, seqlen, dstate);
+    if (rc != MAMBA_OK) return rc;
+    if (!u || !delta || !A || !B || !C || !out) return MAMBA_ERR_NULL;
+    int want_lanes = 0, want_threads = 0;
+    if (tuning) {
+        if (tuning->schedule != MAMBA_SCHEDULE_AUTO && tuning->schedule != MAMBA_SCHEDULE_STATIC)
+            return MAMBA_ERR_UNSUPPORTED;
+        want_lanes = tuning->lanes_per_channel;
+        want_threads = tuning->threads_per_block;
+        if (want_lanes != 0 && want_lanes != 1 && want_lanes != 2 && want_lanes != 4 &&
+            want_lanes != 8 && want_lanes != 16)
+            return MAMBA_ERR_UNSUPPORTED;
+        if (want_threads != 0 && want_threads != 128 && want_threads != 256)
+            return MAMBA_ERR_UNSUPPORTED;
+    }
+    mamba_scan_strides_t st;
+    if (strides) {
+        st = *strides;
+    } else {
+        const mamba_stride3_t x{dim * seqlen, seqlen, 1}, bc{dstate * seqlen, seqlen, 1};
+        st.u = st.delta = st.z = st.out = x;
+        st.B = st.C = bc;
+    }
+    const size_t es = act_size(act_dtype);
+    Span su, sd, sz, so, sb, sc;
+    if (!strided_span(u, st.u, batch, dim, seqlen, es, &su) ||
+        !strided_span(delta, st.delta, batch, dim, seqlen, es, &sd) ||
+        !strided_span(z, st.z, batch, dim, seqlen, es, &sz) ||
+        !strided_span(out, st.out, batch, dim, seqlen, es, &so) ||
+        !strided_span(B, st.B, batch, dstate, seqlen, es, &sb) ||
+        !strided_span(C, st.C, batch, dstate, seqlen, es, &sc))
+        return MAMBA_ERR_SHAPE;
+    if (!injective(st.out, batch, dim, seqlen)) return MAMBA_ERR_SHAPE;
+    const Span sA{reinterpret_cast<uintptr_t>(A), (size_t)(dim * dstate) * 4};
+    const Span sD{reinterpret_cast<uintptr_t>(D), D ? (size_t)dim * 4 : 0};
+    const Span sbias{reinterpret_cast<uintptr_t>(delta_bias), delta_bias ? (size_t)dim * 4 : 0};
+    const size_t nls = (size_t)(batch * dim * dstate) * 4;
+    const Span sls{reinterpret_cast<uintptr_t>(last_state), last_state ? nls : 0};
+    const Span sh0{reinterpret_cast<uintptr_t>(h0), h0 ? nls : 0};
+    // out: in place over u, delta or z with the same map, else apart from every input
+    auto in_place = [&](const void *in, const mamba_stride3_t &s) {
+        return in == out && same_stride(s, st.out);
+    };
+    if ((spans_overlap(so, su) && !in_place(u, st.u)) ||
+        (spans_overlap(so, sd) && !in_place(delta, st.delta)) ||
+        (spans_overlap(so, sz) && !in_place(z, st.z)) || spans_overlap(so, sb) ||
+        spans_overlap(so, sc) || spans_overlap(so, sA) || spans_overlap(so, sD) ||
+        spans_overlap(so, sbias) || spans_overlap(so, sh0))
+        return MAMBA_ERR_OVERLAP;
+    const Span ins[] = {su, sd, sz, sb, sc, sA, sD, sbias, so};
+    for (const Span &x : ins)
+        if (spans_overlap(sls, x)) return MAMBA_ERR_OVERLAP;
+    if (h0 && last_state && spans_overlap(sls, sh0) && h0 != last_state) return MAMBA_ERR_OVERLAP;
+
+    int status = MAMBA_OK;
+    const int sms = current_sm_count(&status);
+    if (status != MAMBA_OK) return status;
+    mscan::ScanStrides ks;
+    auto cvt = [](const mamba_stride3_t &s) { return mscan::Stride3{s.batch, s.row, s.time}; };
+    ks.u = cvt(st.u); ks.delta = cvt(st.delta); ks.z = cvt(st.z); ks.out = cvt(st.out);
+    ks.B = cvt(st.B); ks.C = cvt(st.C);
+    mscan::ScanArgs a;
+    a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.D = D; a.delta_bias = delta_bias; a.out = out; a.last_state = last_state; a.h0 = h0;
+    a.strides = &ks;
+    a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = (int)dstate;
+    a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
+    mscan::ScanPlan pl;
+    if (mscan::make_scan_plan(a, want_lanes, want_threads, sms, &pl) != 0) return MAMBA_ERR_UNSUPPORTED;
+    return mscan::launch_scan_fwd(a, pl, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
 
 int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
                    const void *C, const float *D, const void *z, const float *delta_bias,
@@ -411,6 +533,6 @@ const char *mamba_status_string(int status) {
     }
 }
 
-int mamba_abi_version(void) { return (1 << 16) | 3; }
+int mamba_abi_version(void) { return (1 << 16) | 4; }
 
 }  // extern "C"

@@ -98,7 +98,8 @@ template <typename T> struct Elem;
 
 template <> struct Elem<float> {
     static constexpr int kVec = 4;  // elements per 16 bytes
-    __device__ __forceinline__ static float load(const float *p) { return __ldg(p); }
+    __device__ __forceinline__ static float load(const float *p) { return __ldg(p); }  // global only
+    __device__ __forceinline__ static float to_f(float v) { return v; }
     __device__ __forceinline__ static void store(float *p, float v) { *p = v; }
     __device__ __forceinline__ static void unpack(const uint4 &w, float *f) {
         f[0] = __uint_as_float(w.x); f[1] = __uint_as_float(w.y);
@@ -112,10 +113,11 @@ template <> struct Elem<float> {
 
 template <> struct Elem<__nv_bfloat16> {
     static constexpr int kVec = 8;
-    __device__ __forceinline__ static float load(const __nv_bfloat16 *p) {
+    __device__ __forceinline__ static float load(const __nv_bfloat16 *p) {  // global only
         unsigned short s = __ldg(reinterpret_cast<const unsigned short *>(p));
         return __uint_as_float(static_cast<uint32_t>(s) << 16);
     }
+    __device__ __forceinline__ static float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
     __device__ __forceinline__ static void store(__nv_bfloat16 *p, float v) {
         *p = __float2bfloat16_rn(v);
     }

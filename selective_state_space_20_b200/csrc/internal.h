@@ -9,12 +9,23 @@ namespace mscan {
 
 enum ActType : int { kF32 = 0, kBF16 = 1 };
 
+// Element strides of one (batch, channel or state, time) tensor.
+struct Stride3 {
+    int64_t b, d, t;
+};
+// Strides of every sequence tensor of a scan; u, delta, z, out are (batch,
+// channel, time) and B, C (batch, state, time).
+struct ScanStrides {
+    Stride3 u, delta, z, out, B, C;
+};
+
 struct ScanArgs {
     const void *u, *delta, *B, *C, *z;
     const float *A, *D, *delta_bias;
     void *out;
     float *last_state;
     const float *h0;  // initial state (batch, dim, dstate) or null (zeros)
+    const ScanStrides *strides;  // null: dense (batch, dim, L) / (batch, N, L), L contiguous
     int64_t batch, dim, seqlen;
     int dstate;
     int softplus;

@@ -29,6 +29,17 @@
 //     rounds) so each lane ends up owning complete outputs.
 //   * Epilogue (one thread per 16-byte vector): out = (y + D u) silu(z),
 //     rounded to the activation type and stored with 16-byte stores.
+//
+// Layouts.  Every sequence tensor has its own (batch, channel or state, time)
+// element strides.  The kernel comes in two orientations: time-contiguous
+// (CL = false: u / delta / z / out rows of consecutive timesteps, the dense
+// (batch, dim, L) layout among them) and channel-contiguous (CL = true: the
+// (batch, L, dim) layout of a sequence model's activations, possibly a slice
+// of a wider projection output).  Both stage a tile in the orientation it
+// has in memory -- [channel][time] or [time][channel] -- so the copies stay
+// 16-byte and coalesced, and read it transposed on chip.  B and C are staged
+// as [state][time] or [time][state] the same way, independently.  Tensors
+// that fit neither vector form take element copies with any strides.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -44,11 +55,13 @@ struct KParams {
     void *out;
     float *last_state;
     const float *h0;
+    ScanStrides st;    // element strides of u, delta, z, out, B, C
     int64_t dim, seqlen;
     int64_t n_groups;  // channel groups per batch row
     int dstate;
     int softplus;
-    int vec;           // 16-byte path usable
+    int vec;           // u / delta / z / out: 16-byte vectors along the kernel's contiguous axis
+    int bc_mode;       // B / C: 0 element copies, 1 vectors along time, 2 vectors along states
 };
 
 // ------------------------------------------------------------ geometry
@@ -120,7 +133,7 @@ __device__ __forceinline__ void transpose_reduce(float (&v)[RB], int r) {
     TransposeReduce<R / 2, RB, RB>::run(v, r);
 }
 
-template <typename T, int NP, int R, int THREADS>
+template <typename T, int NP, int R, int THREADS, bool CL>
 __global__ void __launch_bounds__(THREADS)
 scan_fwd_kernel(const KParams p) {
     using G = Geom<T, NP, R, THREADS>;
@@ -129,6 +142,8 @@ scan_fwd_kernel(const KParams p) {
     constexpr int VPR = TC / V;            // 16-byte vectors per row per chunk
     constexpr int CH_VEC = CG * VPR;       // channel-tile vectors per tensor
     constexpr int BC_VEC = NP * VPR;       // B (or C) tile vectors
+    constexpr int CVR = CG / V;            // channel-contiguous: vectors per timestep row
+    constexpr int NVR = NP / V;            // state-contiguous B / C: vectors per timestep row
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
     float *sDelta = reinterpret_cast<float *>(smem_raw);  // delta, then y
@@ -152,8 +167,7 @@ scan_fwd_kernel(const KParams p) {
     const T *__restrict__ gB = static_cast<const T *>(p.B);
     const T *__restrict__ gC = static_cast<const T *>(p.C);
     T *__restrict__ gout = static_cast<T *>(p.out);
-    const int64_t row0 = (b * Dm + d0) * L;      // first element of this block's rows
-    const int64_t bc0 = (int64_t)b * N * L;      // first element of B[b] / C[b]
+    const Stride3 su = p.st.u, sdl = p.st.delta, sz = p.st.z, so = p.st.out, sBs = p.st.B, sCs = p.st.C;
 
     // ---- scan identity: channel c, lane r, states r*S .. r*S+S-1
     const int c = tid / R, r = tid % R;
@@ -166,7 +180,9 @@ scan_fwd_kernel(const KParams p) {
         h[s] = (p.h0 && d < Dm && n < N) ? __ldcg(p.h0 + (b * Dm + d) * N + n) : 0.f;
     }
 
-    // ---- copy one chunk's raw tiles into stage `st`
+    // ---- copy one chunk's raw tiles into stage `st`: u / delta / z as
+    // [channel][time] (CL = false) or [time][channel] (CL = true); B / C as
+    // [state][time], or [time][state] when they are state-contiguous
     auto issue_loads = [&](int64_t t0, int st) {
         T *rU = rawBase + st * STAGE;
         T *rD = rU + CG * TC;
@@ -174,44 +190,67 @@ scan_fwd_kernel(const KParams p) {
         T *rB = rZ + CG * TC;
         T *rC = rB + NP * TC;
         if (p.vec) {
-            for (int vi = tid; vi < CH_VEC; vi += THREADS) {
-                const int pc = vi / VPR, tv = vi % VPR;
-                const int64_t t = t0 + tv * V;
-                const bool ok = (d0 + pc < Dm) && (t < L);
-                const int64_t off = ok ? row0 + pc * L + t : 0;
-                cp_async16(rU + pc * TC + tv * V, gu + off, ok);
-                cp_async16(rD + pc * TC + tv * V, gd + off, ok);
-                if (has_z) cp_async16(rZ + pc * TC + tv * V, gz + off, ok);
+            if (!CL) {
+                for (int vi = tid; vi < CH_VEC; vi += THREADS) {
+                    const int pc = vi / VPR, tv = vi % VPR;
+                    const int64_t t = t0 + tv * V, dd = d0 + pc;
+                    const bool ok = (dd < Dm) && (t < L);
+                    cp_async16(rU + pc * TC + tv * V, gu + (ok ? b * su.b + dd * su.d + t : 0), ok);
+                    cp_async16(rD + pc * TC + tv * V, gd + (ok ? b * sdl.b + dd * sdl.d + t : 0), ok);
+                    if (has_z) cp_async16(rZ + pc * TC + tv * V, gz + (ok ? b * sz.b + dd * sz.d + t : 0), ok);
+                }
+            } else {
+                for (int vi = tid; vi < TC * CVR; vi += THREADS) {
+                    const int tt = vi / CVR, cv = vi % CVR;
+                    const int64_t t = t0 + tt, dd = d0 + cv * V;
+                    const bool ok = (dd < Dm) && (t < L);  // dim is a whole number of vectors
+                    cp_async16(rU + tt * CG + cv * V, gu + (ok ? b * su.b + t * su.t + dd : 0), ok);
+                    cp_async16(rD + tt * CG + cv * V, gd + (ok ? b * sdl.b + t * sdl.t + dd : 0), ok);
+                    if (has_z) cp_async16(rZ + tt * CG + cv * V, gz + (ok ? b * sz.b + t * sz.t + dd : 0), ok);
+                }
             }
+        } else {
+            // any strides: element copies, zero outside the problem
+            for (int e = tid; e < CG * TC; e += THREADS) {
+                const int pc = CL ? e % CG : e / TC, tt = CL ? e / CG : e % TC;
+                const int64_t t = t0 + tt, dd = d0 + pc;
+                const bool ok = (dd < Dm) && (t < L);
+                rU[e] = ok ? gu[b * su.b + dd * su.d + t * su.t] : T(0.f);
+                rD[e] = ok ? gd[b * sdl.b + dd * sdl.d + t * sdl.t] : T(0.f);
+                if (has_z) rZ[e] = ok ? gz[b * sz.b + dd * sz.d + t * sz.t] : T(0.f);
+            }
+        }
+        if (p.bc_mode == 1) {
             for (int vi = tid; vi < 2 * BC_VEC; vi += THREADS) {
                 const int which = vi / BC_VEC, rem = vi % BC_VEC;
                 const int n = rem / VPR, tv = rem % VPR;
                 const int64_t t = t0 + tv * V;
                 const bool ok = (n < N) && (t < L);
-                const int64_t off = ok ? bc0 + (int64_t)n * L + t : 0;
+                const Stride3 &sx = which ? sCs : sBs;
+                const int64_t off = ok ? b * sx.b + n * sx.d + t : 0;
                 cp_async16((which ? rC : rB) + n * TC + tv * V, (which ? gC : gB) + off, ok);
             }
-            cp_async_commit();
-        } else {
-            // unaligned tensors: element loads, zero outside the problem
-            for (int e = tid; e < CG * TC; e += THREADS) {
-                const int pc = e / TC, tt = e % TC;
+        } else if (p.bc_mode == 2) {
+            for (int vi = tid; vi < 2 * TC * NVR; vi += THREADS) {
+                const int which = vi / (TC * NVR), rem = vi % (TC * NVR);
+                const int tt = rem / NVR, n = (rem % NVR) * V;
                 const int64_t t = t0 + tt;
-                const bool ok = (d0 + pc < Dm) && (t < L);
-                const int64_t off = row0 + pc * L + t;
-                rU[e] = ok ? gu[off] : T(0.f);
-                rD[e] = ok ? gd[off] : T(0.f);
-                if (has_z) rZ[e] = ok ? gz[off] : T(0.f);
+                const bool ok = (n < N) && (t < L);  // dstate is a whole number of vectors
+                const Stride3 &sx = which ? sCs : sBs;
+                const int64_t off = ok ? b * sx.b + t * sx.t + n : 0;
+                cp_async16((which ? rC : rB) + tt * NP + n, (which ? gC : gB) + off, ok);
             }
+        } else {
             for (int e = tid; e < 2 * NP * TC; e += THREADS) {
                 const int which = e / (NP * TC), rem = e % (NP * TC);
                 const int n = rem / TC, tt = rem % TC;
                 const int64_t t = t0 + tt;
                 const bool ok = (n < N) && (t < L);
-                const int64_t off = bc0 + (int64_t)n * L + t;
-                (which ? rC : rB)[rem] = ok ? (which ? gC : gB)[off] : T(0.f);
+                const Stride3 &sx = which ? sCs : sBs;
+                (which ? rC : rB)[rem] = ok ? (which ? gC : gB)[b * sx.b + n * sx.d + t * sx.t] : T(0.f);
             }
         }
+        cp_async_commit();  // an empty group when everything was copied by hand
     };
 
     issue_loads(0, 0);
@@ -226,17 +265,25 @@ scan_fwd_kernel(const KParams p) {
         const T *rC = rB + NP * TC;
         const int tvalid = (L - t0) < TC ? (int)(L - t0) : TC;
 
-        if (p.vec) cp_async_wait_all();
+        cp_async_wait_all();
         __syncthreads();  // raw stage ready; previous epilogue finished
 
         // ---- prologue: delta and delta*u for every element of the tile
         for (int vi = tid; vi < CH_VEC; vi += THREADS) {
-            const int pc = vi / VPR, tv = vi % VPR;
+            const int pc = CL ? vi % CG : vi / VPR, tv = CL ? vi / CG : vi % VPR;
             const int64_t dd = d0 + pc;
             const float bias = (dd < Dm && p.delta_bias) ? __ldg(p.delta_bias + dd) : 0.f;
             float fu[V], fd[V];
-            Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + pc * TC + tv * V), fu);
-            Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rD + pc * TC + tv * V), fd);
+            if (!CL) {
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + pc * TC + tv * V), fu);
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rD + pc * TC + tv * V), fd);
+            } else {  // a column of the [time][channel] tile
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    fu[i] = Elem<T>::to_f(rU[(tv * V + i) * CG + pc]);
+                    fd[i] = Elem<T>::to_f(rD[(tv * V + i) * CG + pc]);
+                }
+            }
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 float dl = fd[i] + bias;
@@ -255,9 +302,16 @@ scan_fwd_kernel(const KParams p) {
         }
         for (int vi = tid; vi < 2 * BC_VEC; vi += THREADS) {
             const int which = vi / BC_VEC, rem = vi % BC_VEC;
-            const int n = rem / VPR, tv = rem % VPR;
+            const bool by_state = p.bc_mode == 2;
+            const int n = by_state ? rem % NP : rem / VPR, tv = by_state ? rem / NP : rem % VPR;
+            const T *raw = which ? rC : rB;
             float f[V];
-            Elem<T>::unpack(*reinterpret_cast<const uint4 *>((which ? rC : rB) + n * TC + tv * V), f);
+            if (!by_state) {
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(raw + n * TC + tv * V), f);
+            } else {  // a column of the [time][state] tile
+#pragma unroll
+                for (int i = 0; i < V; ++i) f[i] = Elem<T>::to_f(raw[(tv * V + i) * NP + n]);
+            }
             float *dst = (which ? sC : sB) + n * TCP + tv * V;
 #pragma unroll
             for (int i = 0; i < V; i += 4)
@@ -309,34 +363,61 @@ scan_fwd_kernel(const KParams p) {
         __syncthreads();
 
         // ---- epilogue: out = (y + D u) * silu(z)
-        for (int vi = tid; vi < CH_VEC; vi += THREADS) {
-            const int pc = vi / VPR, tv = vi % VPR;
-            const int64_t dd = d0 + pc;
-            const int64_t t = t0 + tv * V;
-            if (dd >= Dm || tv * V >= tvalid) continue;
-            const float Dd = p.D ? __ldg(p.D + dd) : 0.f;
-            float fu[V], fz[V], y[V];
-            Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + pc * TC + tv * V), fu);
-            if (has_z) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rZ + pc * TC + tv * V), fz);
-            const float *ys = sDelta + pc * TCP + tv * V;
+        if (!CL) {
+            for (int vi = tid; vi < CH_VEC; vi += THREADS) {
+                const int pc = vi / VPR, tv = vi % VPR;
+                const int64_t dd = d0 + pc;
+                const int64_t t = t0 + tv * V;
+                if (dd >= Dm || tv * V >= tvalid) continue;
+                const float Dd = p.D ? __ldg(p.D + dd) : 0.f;
+                float fu[V], fz[V], y[V];
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + pc * TC + tv * V), fu);
+                if (has_z) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rZ + pc * TC + tv * V), fz);
+                const float *ys = sDelta + pc * TCP + tv * V;
 #pragma unroll
-            for (int i = 0; i < V; i += 4) {
-                const float4 q = *reinterpret_cast<const float4 *>(ys + i);
-                y[i] = q.x; y[i + 1] = q.y; y[i + 2] = q.z; y[i + 3] = q.w;
+                for (int i = 0; i < V; i += 4) {
+                    const float4 q = *reinterpret_cast<const float4 *>(ys + i);
+                    y[i] = q.x; y[i + 1] = q.y; y[i + 2] = q.z; y[i + 3] = q.w;
+                }
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    float o = fmaf(Dd, fu[i], y[i]);
+                    if (has_z) o *= silu_f(fz[i]);
+                    y[i] = o;
+                }
+                T *dst = gout + b * so.b + dd * so.d + t * so.t;
+                if (p.vec) {
+                    stg16_stream(dst, Elem<T>::pack(y));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < V; ++i)
+                        if (tv * V + i < tvalid) Elem<T>::store(dst + i * so.t, y[i]);
+                }
             }
+        } else {  // one thread per V channels of one timestep
+            for (int vi = tid; vi < TC * CVR; vi += THREADS) {
+                const int tt = vi / CVR, cv = vi % CVR;
+                const int64_t dd = d0 + cv * V;
+                const int64_t t = t0 + tt;
+                if (dd >= Dm || tt >= tvalid) continue;
+                float fu[V], fz[V], y[V];
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + tt * CG + cv * V), fu);
+                if (has_z) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rZ + tt * CG + cv * V), fz);
 #pragma unroll
-            for (int i = 0; i < V; ++i) {
-                float o = fmaf(Dd, fu[i], y[i]);
-                if (has_z) o *= silu_f(fz[i]);
-                y[i] = o;
-            }
-            T *dst = gout + row0 + pc * L + t;
-            if (p.vec) {
-                stg16_stream(dst, Elem<T>::pack(y));
-            } else {
+                for (int i = 0; i < V; ++i) {
+                    const float Dd = (p.D && dd + i < Dm) ? __ldg(p.D + dd + i) : 0.f;
+                    float o = fmaf(Dd, fu[i], sDelta[(cv * V + i) * TCP + tt]);
+                    if (has_z) o *= silu_f(fz[i]);
+                    y[i] = o;
+                }
+                T *dst = gout + b * so.b + t * so.t + dd * so.d;
+                if (p.vec) {
+                    stg16_stream(dst, Elem<T>::pack(y));
+                } else {
 #pragma unroll
-                for (int i = 0; i < V; ++i)
-                    if (tv * V + i < tvalid) Elem<T>::store(dst + i, y[i]);
+                    for (int i = 0; i < V; ++i)
+                        if (dd + i < Dm) Elem<T>::store(dst + i * so.d, y[i]);
+                }
             }
         }
     }
@@ -352,10 +433,10 @@ scan_fwd_kernel(const KParams p) {
 }
 
 // ------------------------------------------------------------ dispatch
-template <typename T, int NP, int R, int THREADS>
+template <typename T, int NP, int R, int THREADS, bool CL>
 static cudaError_t launch_impl(const KParams &kp, int64_t blocks, cudaStream_t st) {
     using G = Geom<T, NP, R, THREADS>;
-    auto kern = scan_fwd_kernel<T, NP, R, THREADS>;
+    auto kern = scan_fwd_kernel<T, NP, R, THREADS, CL>;
     if (G::SMEM > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)G::SMEM);
@@ -396,6 +477,45 @@ static bool lookup_geom(int act, int np, int r, int th, ScanPlan *pl) {
     return false;
 }
 
+// How the static kernel reads and writes the sequence tensors: the
+// orientation (channel-contiguous when u is), whether u / delta / z / out all
+// allow 16-byte vectors along it, and the form of the B / C copies.
+struct StaticLayout {
+    ScanStrides st;
+    bool cl;
+    int vec, bc_mode;
+};
+
+static StaticLayout static_layout(const ScanArgs &a) {
+    StaticLayout r;
+    const int64_t Dm = a.dim, L = a.seqlen, N = a.dstate;
+    if (a.strides) {
+        r.st = *a.strides;
+    } else {
+        r.st.u = r.st.delta = r.st.z = r.st.out = Stride3{Dm * L, L, 1};
+        r.st.B = r.st.C = Stride3{N * L, L, 1};
+    }
+    const int64_t V = a.act == kBF16 ? 8 : 4;
+    auto al = [](const void *q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+    r.cl = r.st.u.d == 1 && r.st.u.t != 1 && L > 1;
+    auto x_ok = [&](const void *q, const Stride3 &s) {
+        if (q == nullptr) return true;
+        if (!al(q) || s.b % V != 0) return false;
+        return r.cl ? (s.d == 1 && s.t % V == 0) : (s.t == 1 && s.d % V == 0);
+    };
+    const bool len_ok = r.cl ? Dm % V == 0 : L % V == 0;
+    r.vec = len_ok && x_ok(a.u, r.st.u) && x_ok(a.delta, r.st.delta) && x_ok(a.z, r.st.z) &&
+            x_ok(a.out, r.st.out);
+    auto bc_ok = [&](int mode, const void *q, const Stride3 &s) {
+        if (!al(q) || s.b % V != 0) return false;
+        return mode == 1 ? (s.t == 1 && s.d % V == 0) : (s.d == 1 && s.t % V == 0);
+    };
+    if (L % V == 0 && bc_ok(1, a.B, r.st.B) && bc_ok(1, a.C, r.st.C)) r.bc_mode = 1;
+    else if (N % V == 0 && bc_ok(2, a.B, r.st.B) && bc_ok(2, a.C, r.st.C)) r.bc_mode = 2;
+    else r.bc_mode = 0;
+    return r;
+}
+
 cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &pl, cudaStream_t st) {
     KParams kp;
     kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
@@ -403,10 +523,13 @@ cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &pl, cudaStream_t 
     kp.out = a.out; kp.last_state = a.last_state; kp.h0 = a.h0;
     kp.dim = a.dim; kp.seqlen = a.seqlen;
     kp.n_groups = (a.dim + pl.channels_per_block - 1) / pl.channels_per_block;
-    kp.dstate = a.dstate; kp.softplus = a.softplus; kp.vec = pl.vectorized;
+    kp.dstate = a.dstate; kp.softplus = a.softplus;
+    const StaticLayout lay = static_layout(a);
+    kp.st = lay.st; kp.vec = lay.vec; kp.bc_mode = lay.bc_mode;
 #define X(T, NP_, R_, TH_) \
     if (a.act == act_of<T>() && pl.padded_dstate == NP_ && pl.lanes == R_ && pl.threads == TH_) \
-        return launch_impl<T, NP_, R_, TH_>(kp, pl.blocks, st);
+        return lay.cl ? launch_impl<T, NP_, R_, TH_, true>(kp, pl.blocks, st)   \
+                      : launch_impl<T, NP_, R_, TH_, false>(kp, pl.blocks, st);
     MSCAN_FOR_ALL(X)
 #undef X
     return cudaErrorInvalidConfiguration;
@@ -434,8 +557,9 @@ int make_scan_plan(const ScanArgs &a, int want_lanes, int want_threads, int sm_c
     const int esize = a.act == kBF16 ? 2 : 4;
     const int vlen = vbytes / esize;
     auto aligned = [](const void *ptr) { return ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
-    pl->vectorized = (a.seqlen % vlen == 0) && aligned(a.u) && aligned(a.delta) && aligned(a.z) &&
-                     aligned(a.B) && aligned(a.C) && aligned(a.out);
+    pl->vectorized = a.strides == nullptr && (a.seqlen % vlen == 0) && aligned(a.u) &&
+                     aligned(a.delta) && aligned(a.z) && aligned(a.B) && aligned(a.C) &&
+                     aligned(a.out);
     pl->padded_dstate = np;
 
     int lanes = want_lanes;
