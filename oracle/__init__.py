@@ -10,6 +10,7 @@ its header for the equations and where each comes from).  This module only
 marshals numpy/torch CPU arrays into it:
 
 * :func:`scan` -- the whole forward scan (optionally from an initial state).
+* :func:`scan_complex` -- the forward scan with complex A, B, C.
 * :func:`scan_bwd` -- gradients of the forward scan (reverse mode).
 * :func:`state_update` -- one recurrent step for every (batch, channel).
 * :func:`conv1d`, :func:`conv1d_update` -- the causal depthwise convolution
@@ -55,6 +56,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.s6_oracle_scan_bwd.argtypes = [f32p, f32p, f32p, f32p, f32p, f32p, f32p, f32p, ctypes.c_int,
                                        f64p, f64p, f64p, f64p, f64p, f64p, f64p, f64p, f64p, f64p,
                                        f64p, f64p, i64, i64, i64, i64, ctypes.c_int]
+    lib.s6_oracle_scan_complex.restype = ctypes.c_int
+    lib.s6_oracle_scan_complex.argtypes = lib.s6_oracle_scan.argtypes
     lib.s6_oracle_softplus.restype = ctypes.c_double
     lib.s6_oracle_softplus.argtypes = [ctypes.c_double]
     lib.s6_oracle_silu.restype = ctypes.c_double
@@ -126,6 +129,54 @@ def scan(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     if rc != 0:
         raise RuntimeError(f"s6_oracle_scan failed with code {rc}")
     return out, last
+
+
+def _pairs(x):
+    """A complex array, or a real one whose last axis holds (re, im), as an
+    fp32 (..., 2) array (exact for bf16 / fp32 parts)."""
+    if x is None:
+        return None
+    if hasattr(x, "detach") and x.is_complex():
+        x = x.detach().to("cpu").numpy()
+    if isinstance(x, np.ndarray) and np.iscomplexobj(x):
+        return np.ascontiguousarray(np.stack([x.real, x.imag], axis=-1).astype(np.float32))
+    return _f32(x)
+
+
+def scan_complex(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                 delta_softplus: bool = True, h0=None, nthreads: int = 0,
+                 lib: Optional[ctypes.CDLL] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Complex-mode selective scan in fp64.
+
+    u, delta, z (batch, dim, L) real; A (dim, N), B, C (batch, N, L) and
+    h0 (batch, dim, N) complex -- complex arrays, or real ones with a
+    trailing (re, im) axis.  Returns ``(out, last_state)``: out (batch, dim,
+    L) fp64 and last_state (batch, dim, N) complex128.
+    """
+    lib = lib or _get()
+    u, delta, D, z, delta_bias = _f32(u), _f32(delta), _f32(D), _f32(z), _f32(delta_bias)
+    A, B, C = _pairs(A), _pairs(B), _pairs(C)
+    if h0 is not None:
+        h0 = np.asarray(h0.detach().cpu().numpy() if hasattr(h0, "detach") else h0)
+        if np.iscomplexobj(h0):
+            h0 = np.stack([h0.real, h0.imag], axis=-1)
+        h0 = np.ascontiguousarray(h0, dtype=np.float64)
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    assert delta.shape == u.shape and (z is None or z.shape == u.shape)
+    assert A.shape == (dim, N, 2) and B.shape == (batch, N, L, 2) and C.shape == B.shape
+    assert D is None or D.shape == (dim,)
+    assert delta_bias is None or delta_bias.shape == (dim,)
+    assert h0 is None or h0.shape == (batch, dim, N, 2)
+    out = np.empty((batch, dim, L), dtype=np.float64)
+    last = np.empty((batch, dim, N, 2), dtype=np.float64)
+    rc = lib.s6_oracle_scan_complex(_p32(u), _p32(delta), _p32(A), _p32(B), _p32(C),
+                                    _p32(D), _p32(z), _p32(delta_bias),
+                                    int(bool(delta_softplus)), _p64(h0), _p64(out),
+                                    _p64(last), batch, dim, L, N, int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_scan_complex failed with code {rc}")
+    return out, last[..., 0] + 1j * last[..., 1]
 
 
 def scan_bwd(dout, u, delta, A, B, C, D=None, z=None, delta_bias=None,

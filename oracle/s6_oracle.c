@@ -503,3 +503,137 @@ int s6_oracle_scan_bwd(const float *u, const float *delta, const float *A,
     free(tids);
     return rc;
 }
+
+/*
+ * Complex-valued mode: the same recurrence with a complex diagonal A and
+ * complex, input-dependent B and C (the complex SSM the Mamba paper compares
+ * with the real one on audio, Appendix E.4.1, and the "complex number mode"
+ * on the roadmap of the "Mamba x JAX" page).  The pages give no formulas for
+ * it; this is the real recurrence above read over the complex numbers, with
+ * the output taken as the real part of the readout:
+ *
+ *   delta_t = softplus(delta_raw + bias)          (real, as above)
+ *   Abar    = exp(delta_t * A[d,n])                complex exponential
+ *   Bbar u  = delta_t * B[b,n,t] * u[b,d,t]        complex
+ *   h_t[n]  = Abar * h_{t-1}[n] + Bbar u           complex state
+ *   y_t     = Re(sum_n C[b,n,t] * h_t[n]) + D[d] * u[b,d,t]
+ *   out_t   = y_t * silu(z[b,d,t])    if z is given
+ *
+ * Complex arrays are interleaved (real, imaginary) pairs of the real layouts:
+ *   A (dim, dstate, 2); B, C (batch, dstate, seqlen, 2);
+ *   h0, last_state (batch, dim, dstate, 2).
+ */
+#include <complex.h>
+
+typedef struct {
+    const float *u, *delta, *A, *B, *C, *D, *z, *bias;
+    const double *h0;
+    int softplus;
+    double *out, *last_state;
+    int64_t dim, seqlen, dstate;
+    int64_t row_begin, row_end;
+} cscan_job_t;
+
+static void *cscan_worker(void *arg)
+{
+    const cscan_job_t *j = (const cscan_job_t *)arg;
+    const int64_t L = j->seqlen, N = j->dstate;
+    double complex *h = (double complex *)malloc(sizeof(double complex) * (size_t)N);
+    if (!h)
+        return (void *)1;
+    for (int64_t row = j->row_begin; row < j->row_end; ++row) {
+        const int64_t b = row / j->dim, d = row % j->dim;
+        const float *u = j->u + row * L;
+        const float *dr = j->delta + row * L;
+        const float *z = j->z ? j->z + row * L : NULL;
+        const float *Bb = j->B + b * N * L * 2;
+        const float *Cb = j->C + b * N * L * 2;
+        const float *Ad = j->A + d * N * 2;
+        const double Dd = j->D ? (double)j->D[d] : 0.0;
+        const double bias = j->bias ? (double)j->bias[d] : 0.0;
+        double *out = j->out + row * L;
+
+        for (int64_t n = 0; n < N; ++n)
+            h[n] = j->h0 ? j->h0[(row * N + n) * 2] + I * j->h0[(row * N + n) * 2 + 1] : 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            double delta = (double)dr[t] + bias;
+            if (j->softplus)
+                delta = s6_oracle_softplus(delta);
+            const double ut = (double)u[t];
+            double y = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                const double complex An = (double)Ad[2 * n] + I * (double)Ad[2 * n + 1];
+                const double complex Bn = (double)Bb[(n * L + t) * 2] + I * (double)Bb[(n * L + t) * 2 + 1];
+                const double complex Cn = (double)Cb[(n * L + t) * 2] + I * (double)Cb[(n * L + t) * 2 + 1];
+                const double complex Abar = cexp(delta * An);
+                const double complex Bbar_u = delta * Bn * ut;
+                h[n] = Abar * h[n] + Bbar_u;
+                y += creal(Cn * h[n]);
+            }
+            y += Dd * (double)u[t];
+            if (z)
+                y = y * s6_oracle_silu((double)z[t]);
+            out[t] = y;
+        }
+        if (j->last_state)
+            for (int64_t n = 0; n < N; ++n) {
+                j->last_state[(row * N + n) * 2] = creal(h[n]);
+                j->last_state[(row * N + n) * 2 + 1] = cimag(h[n]);
+            }
+    }
+    free(h);
+    return NULL;
+}
+
+/* Complex-mode scan over all (b, d) rows; threads and return codes as
+ * s6_oracle_scan. */
+int s6_oracle_scan_complex(const float *u, const float *delta, const float *A,
+                           const float *B, const float *C, const float *D,
+                           const float *z, const float *delta_bias, int softplus,
+                           const double *h0, double *out, double *last_state,
+                           int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                           int nthreads)
+{
+    if (!u || !delta || !A || !B || !C || !out)
+        return -1;
+    if (batch <= 0 || dim <= 0 || seqlen <= 0 || dstate <= 0)
+        return -1;
+    const int64_t rows = batch * dim;
+    if (nthreads <= 0) {
+        long nc = sysconf(_SC_NPROCESSORS_ONLN);
+        nthreads = nc > 0 ? (int)nc : 1;
+    }
+    if (nthreads > rows)
+        nthreads = (int)rows;
+    cscan_job_t base = {u, delta, A, B, C, D, z, delta_bias, h0, softplus,
+                        out, last_state, dim, seqlen, dstate, 0, rows};
+    cscan_job_t *jobs = (cscan_job_t *)malloc(sizeof(cscan_job_t) * (size_t)nthreads);
+    pthread_t *tids = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!jobs || !tids) {
+        free(jobs);
+        free(tids);
+        return -2;
+    }
+    int rc = 0, started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i] = base;
+        jobs[i].row_begin = rows * i / nthreads;
+        jobs[i].row_end = rows * (i + 1) / nthreads;
+        if (pthread_create(&tids[i], NULL, cscan_worker, &jobs[i]) != 0) {
+            jobs[i].row_end = rows;
+            if (cscan_worker(&jobs[i]))
+                rc = -2;
+            break;
+        }
+        ++started;
+    }
+    for (int i = 0; i < started; ++i) {
+        void *ret = NULL;
+        pthread_join(tids[i], &ret);
+        if (ret)
+            rc = -2;
+    }
+    free(jobs);
+    free(tids);
+    return rc;
+}

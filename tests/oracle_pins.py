@@ -558,6 +558,161 @@ def pin_bwd_finite_differences(lib):
             assert abs(fd - g) <= 2e-5 * max(1.0, abs(g)), f"{gname}{idx}: fd {fd} vs {g}"
 
 
+# ---------------------------------------------------------------- complex mode
+def _cplx32(rng, shape, scale=1.0):
+    """Complex values whose real and imaginary parts are fp32-exact."""
+    re = _f32(rng.normal(size=shape) * scale).astype(np.float64)
+    im = _f32(rng.normal(size=shape) * scale).astype(np.float64)
+    return re + 1j * im
+
+
+def _cplx_problem(rng, Bt, Dm, L, N, gate=True):
+    A = (-_f32(rng.uniform(0.1, 2.0, (Dm, N))).astype(np.float64)
+         + 1j * _f32(rng.uniform(-6.0, 6.0, (Dm, N))).astype(np.float64))
+    return dict(u=_f32(rng.normal(size=(Bt, Dm, L))), delta=_f32(0.5 * rng.normal(size=(Bt, Dm, L))),
+                A=A, B=_cplx32(rng, (Bt, N, L)), C=_cplx32(rng, (Bt, N, L)),
+                D=_f32(rng.uniform(0.5, 1.5, Dm)), z=_f32(rng.normal(size=(Bt, Dm, L))) if gate else None,
+                delta_bias=_f32(rng.uniform(-3.0, -1.0, Dm)))
+
+
+def pin_complex_real_case(lib):
+    """Imaginary parts zero: the complex mode is the real scan (the real
+    oracle is pinned on its own), outputs and states bit for bit."""
+    rng = np.random.default_rng(41)
+    p = _rand_problem(rng, 2, 3, 37, 5)
+    pc = dict(p, A=p["A"].astype(np.complex128), B=p["B"].astype(np.complex128),
+              C=p["C"].astype(np.complex128))
+    o_r, s_r = oracle.scan(**p, lib=lib)
+    o_c, s_c = oracle.scan_complex(**pc, lib=lib)
+    assert np.array_equal(o_r, o_c), "complex mode with real inputs differs from the real scan"
+    assert np.array_equal(s_r, s_c.real) and not np.any(s_c.imag)
+
+
+def pin_complex_geometric_series(lib):
+    """Constant inputs: h_t = b (1 - a^{t+1}) / (1 - a) over the complex
+    numbers, a = e^{delta A}, b = delta B u; y_t = Re(sum_n C_n h_t[n]) + D u,
+    times silu(z)."""
+    rng = np.random.default_rng(42)
+    L, N = 200, 4
+    raw, bias = np.float32(-0.5), np.float32(-2.0)
+    delta = float(np.logaddexp(0.0, float(raw) + float(bias)))
+    A = -_f32([0.5, 0.05, 1.3, 0.2]).astype(np.float64) + 1j * _f32([3.0, -1.5, 0.25, 9.0]).astype(np.float64)
+    Bv, Cv = _cplx32(rng, N), _cplx32(rng, N)
+    u, Dv, zv = np.float32(0.75), np.float32(0.5), np.float32(0.8125)
+    ins = dict(u=np.full((1, 1, L), u, np.float32), delta=np.full((1, 1, L), raw, np.float32),
+               A=A.reshape(1, N), B=np.repeat(Bv.reshape(1, N, 1), L, axis=2),
+               C=np.repeat(Cv.reshape(1, N, 1), L, axis=2), D=np.full((1,), Dv, np.float32),
+               z=np.full((1, 1, L), zv, np.float32), delta_bias=np.full((1,), bias, np.float32))
+    out, last = oracle.scan_complex(**ins, lib=lib)
+    t = np.arange(L, dtype=np.float64)[:, None]
+    a = np.exp(delta * A)[None, :]
+    b = (delta * Bv * float(u))[None, :]
+    h = b * (1.0 - a ** (t + 1.0)) / (1.0 - a)
+    y = (h @ Cv).real + float(Dv) * float(u)
+    gate = float(zv) * float(special.expit(float(zv)))
+    _close(out[0, 0], y * gate, what="complex geometric series out")
+    _close(np.abs(last[0, 0] - h[-1]), np.zeros(N), scale=float(np.max(np.abs(h[-1]))),
+           what="complex geometric series last_state")
+
+
+def pin_complex_lti_convolution(lib):
+    """delta, B, C constant in time: y = K * u + D u with the real kernel
+    K_k = Re(sum_n C_n Abar_n^k delta B_n) (numpy.convolve)."""
+    rng = np.random.default_rng(43)
+    L, N = 181, 5
+    raw, bias = np.float32(0.2), np.float32(-2.5)
+    delta = float(np.logaddexp(0.0, float(raw) + float(bias)))
+    A = (-_f32(rng.uniform(0.2, 3.0, N)).astype(np.float64)
+         + 1j * _f32(rng.uniform(-8.0, 8.0, N)).astype(np.float64))
+    Bv, Cv = _cplx32(rng, N), _cplx32(rng, N)
+    u = _f32(rng.normal(size=L))
+    Dv = np.float32(1.25)
+    ins = dict(u=u.reshape(1, 1, L), delta=np.full((1, 1, L), raw, np.float32), A=A.reshape(1, N),
+               B=np.repeat(Bv.reshape(1, N, 1), L, axis=2), C=np.repeat(Cv.reshape(1, N, 1), L, axis=2),
+               D=np.full((1,), Dv, np.float32), z=None, delta_bias=np.full((1,), bias, np.float32))
+    out, _ = oracle.scan_complex(**ins, lib=lib)
+    k = np.arange(L, dtype=np.float64)[:, None]
+    K = ((np.exp(delta * A)[None, :] ** k) @ (Cv * delta * Bv)).real
+    y = np.convolve(K, u.astype(np.float64))[:L] + float(Dv) * u.astype(np.float64)
+    _close(out[0, 0], y, rtol=1e-10, what="complex LTI convolution")
+
+
+def pin_complex_iir(lib):
+    """One state, delta constant, B and u varying: the state is the output
+    of the complex first-order filter h_t = a h_{t-1} + x_t
+    (scipy.signal.lfilter with a complex pole), started from h0."""
+    rng = np.random.default_rng(44)
+    L = 150
+    raw, bias = np.float32(-1.0), np.float32(0.25)
+    delta = float(np.logaddexp(0.0, float(raw) + float(bias)))
+    A = complex(-_f32(0.3), _f32(2.5))
+    Bs = _cplx32(rng, L)
+    u = _f32(rng.normal(size=L))
+    h0 = complex(0.75, -1.5)
+    ins = dict(u=u.reshape(1, 1, L), delta=np.full((1, 1, L), raw, np.float32), A=np.array([[A]]),
+               B=Bs.reshape(1, 1, L), C=np.ones((1, 1, L), np.complex128), D=None, z=None,
+               delta_bias=np.full((1,), bias, np.float32), h0=np.array([[[h0]]]))
+    out, last = oracle.scan_complex(**ins, lib=lib)
+    a = np.exp(delta * A)
+    x = delta * Bs * u.astype(np.float64)
+    h, _ = signal.lfilter([1.0], [1.0, -a], x, zi=[a * h0])
+    _close(out[0, 0], h.real, what="complex IIR (real part readout)")
+    assert abs(last[0, 0, 0] - h[-1]) <= 1e-11 * abs(h[-1])
+
+
+def pin_complex_brute_force(lib):
+    """Tiny shapes: h_t = sum_{s<=t} (prod_{r=s+1..t} Abar_r) Bbar_s u_s
+    with Python complex arithmetic (cmath), no recurrence; y as defined."""
+    import cmath
+    rng = np.random.default_rng(45)
+    Bt, Dm, L, N = 2, 2, 9, 3
+    p = _cplx_problem(rng, Bt, Dm, L, N)
+    out, last = oracle.scan_complex(**p, lib=lib)
+    for b in range(Bt):
+        for d in range(Dm):
+            dl = [float(np.logaddexp(0.0, float(p["delta"][b, d, t]) + float(p["delta_bias"][d]))) for t in range(L)]
+            for t in range(L):
+                y = 0.0
+                for n in range(N):
+                    hs = 0j
+                    for s_ in range(t + 1):
+                        prod = 1 + 0j
+                        for r in range(s_ + 1, t + 1):
+                            prod *= cmath.exp(dl[r] * complex(p["A"][d, n]))
+                        hs += prod * dl[s_] * complex(p["B"][b, n, s_]) * float(p["u"][b, d, s_])
+                    y += (complex(p["C"][b, n, t]) * hs).real
+                    if t == L - 1:
+                        assert abs(last[b, d, n] - hs) <= 1e-12 * max(1.0, abs(hs))
+                y += float(p["D"][d]) * float(p["u"][b, d, t])
+                zt = float(p["z"][b, d, t])
+                y *= zt / (1.0 + math.exp(-zt))
+                assert abs(out[b, d, t] - y) <= 1e-12 * max(1.0, abs(y)), (b, d, t, out[b, d, t], y)
+
+
+def pin_complex_phase_invariance(lib):
+    """Rotating state n by e^{i phi_n} -- B times e^{i phi_n}, C times
+    e^{-i phi_n}, h0 times e^{i phi_n} -- leaves every output unchanged and
+    rotates the final state; conjugating A, B, C and h0 leaves the outputs
+    unchanged and conjugates the state."""
+    rng = np.random.default_rng(46)
+    Bt, Dm, L, N = 2, 3, 64, 4
+    p = _cplx_problem(rng, Bt, Dm, L, N)
+    h0 = _cplx32(rng, (Bt, Dm, N), 0.3)
+    o1, s1 = oracle.scan_complex(**p, h0=h0, lib=lib)
+    rot = np.exp(1j * rng.uniform(0, 2 * np.pi, N))
+    q = dict(p, B=p["B"] * rot[None, :, None], C=p["C"] * np.conj(rot)[None, :, None])
+    # the rotated inputs are rounded to fp32 on the way in: compare at that level
+    o2, s2 = oracle.scan_complex(**q, h0=h0 * rot[None, None, :], lib=lib)
+    _close(o2, o1, rtol=2e-6, what="phase rotation: outputs")
+    _close(np.abs(s2 - s1 * rot[None, None, :]), np.zeros(s1.shape), scale=float(np.max(np.abs(s1))),
+           rtol=2e-6, what="phase rotation: state")
+    c = dict(p, A=np.conj(p["A"]), B=np.conj(p["B"]), C=np.conj(p["C"]))
+    o3, s3 = oracle.scan_complex(**c, h0=np.conj(h0), lib=lib)
+    _close(o3, o1, rtol=1e-13, what="conjugation: outputs")
+    _close(np.abs(s3 - np.conj(s1)), np.zeros(s1.shape), scale=float(np.max(np.abs(s1))), rtol=1e-13,
+           what="conjugation: state")
+
+
 ALL_PINS = [pin_softplus_silu, pin_geometric_series, pin_lti_convolution,
             pin_first_order_iir, pin_zero_step_keeps_state, pin_memoryless_limit,
             pin_brute_force_products, pin_cumsum_form, pin_chunk_split,
@@ -566,4 +721,6 @@ ALL_PINS = [pin_softplus_silu, pin_geometric_series, pin_lti_convolution,
             pin_gate_and_softplus_flags,
             pin_conv_numpy, pin_conv_impulse, pin_conv_silu, pin_conv_wide_input,
             pin_conv_update_stream, pin_conv_causality,
-            pin_bwd_autograd, pin_bwd_finite_differences]
+            pin_bwd_autograd, pin_bwd_finite_differences,
+            pin_complex_real_case, pin_complex_geometric_series, pin_complex_lti_convolution,
+            pin_complex_iir, pin_complex_brute_force, pin_complex_phase_invariance]

@@ -71,6 +71,25 @@ MUTANTS = [
     ("bwd-dB-without-u", "j->dB[b * N * L + n * L + t] += g[n] * delta * ut;",
      "j->dB[b * N * L + n * L + t] += g[n] * delta;"),
     ("bwd-dD-without-gate", "j->dD[d] += dy * ut;", "j->dD[d] += dout[t] * ut;"),
+    # complex mode
+    ("cplx-readout-conjugated", "y += creal(Cn * h[n]);", "y += creal(conj(Cn) * h[n]);"),
+    ("cplx-readout-magnitude", "y += creal(Cn * h[n]);", "y += cabs(Cn * h[n]);"),
+    ("cplx-rotation-reversed", "cexp(delta * An)", "cexp(delta * conj(An))"),
+    ("cplx-rotation-dropped", "cexp(delta * An)", "exp(delta * creal(An))"),
+    ("cplx-B-imag-dropped", "(double)Bb[(n * L + t) * 2] + I * (double)Bb[(n * L + t) * 2 + 1]",
+     "(double)Bb[(n * L + t) * 2]"),
+    ("cplx-B-parts-swapped", "(double)Bb[(n * L + t) * 2] + I * (double)Bb[(n * L + t) * 2 + 1]",
+     "(double)Bb[(n * L + t) * 2 + 1] + I * (double)Bb[(n * L + t) * 2]"),
+    ("cplx-C-time-lag", "(double)Cb[(n * L + t) * 2] + I * (double)Cb[(n * L + t) * 2 + 1]",
+     "(double)Cb[(n * L + (t > 0 ? t - 1 : 0)) * 2] + I * (double)Cb[(n * L + (t > 0 ? t - 1 : 0)) * 2 + 1]"),
+    ("cplx-h0-imag-dropped", "h[n] = j->h0 ? j->h0[(row * N + n) * 2] + I * j->h0[(row * N + n) * 2 + 1] : 0.0;",
+     "h[n] = j->h0 ? j->h0[(row * N + n) * 2] : 0.0;"),
+    ("cplx-last-state-conjugated", "j->last_state[(row * N + n) * 2 + 1] = cimag(h[n]);",
+     "j->last_state[(row * N + n) * 2 + 1] = -cimag(h[n]);"),
+    ("cplx-D-dropped", "y += Dd * (double)u[t];", "y += 0.0 * (double)u[t];"),
+    ("cplx-gate-dropped", "y = y * s6_oracle_silu((double)z[t]);", "y = y * 1.0;"),
+    ("cplx-A-index", "const double complex An = (double)Ad[2 * n] + I * (double)Ad[2 * n + 1];",
+     "const double complex An = (double)Ad[0] + I * (double)Ad[1];"),
 ]
 
 
