@@ -78,6 +78,7 @@ KERNEL_SOURCES = {
     "scan_fwd_spec_kernel": ("scan_fwd_persistent_spec.cu", "persistent_common.cuh", "persistent_kernels.h",
                              "persistent_host.cu", "device_math.cuh", "internal.h"),
     "scan_fwd_kernel": ("scan_fwd.cu", "device_math.cuh", "internal.h"),
+    "scan_fwd_complex_kernel": ("scan_fwd_complex.cu", "device_math.cuh", "internal.h"),
 }
 
 
@@ -461,6 +462,38 @@ def backward_measure(reps=5):
             "reps": reps}
 
 
+def complex_measure(reps=10):
+    """Complex-valued mode on the benchmark layer's shape (4 x 5120 x 4096,
+    N = 16 complex states, bf16 activations; A = -1/2 + i pi n).  Each
+    state-step takes three special-function ops (ex2, sin, cos), so the roof
+    is the MUFU rate over 3 N ops per element."""
+    w = inputs.MAMBA_2_8B
+    d = inputs.complex_inputs(w.batch, w.dim, w.seqlen, w.dstate, w.dtype, device="cuda")
+    out = torch.empty_like(d["u"])
+    last = torch.empty(w.batch, w.dim, w.dstate, 2, device="cuda")
+    run = lambda: binding.mamba_scan_fwd_complex(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"],  # noqa: E731
+                                                 z=d["z"], delta_bias=d["delta_bias"], out=out,
+                                                 last_state=last)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    peak = MUFU_PER_CLK_PER_SM * SM_COUNT * load_peaks()["sm_max_mhz"] * 1e6 / (3 * w.dstate) / 1e9
+    achieved = w.elements / us / 1e3
+    return {"workload": f"complex mode {w.batch}x{w.dim}x{w.seqlen} N{w.dstate} {w.dtype}",
+            "us_per_call": us, "Gelem_per_s": achieved,
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Gelem/s",
+                         "frac": achieved / peak,
+                         "note": "peak = MUFU ops/s over 3 N (ex2, sin, cos per complex state-step)"},
+            "reps": reps, "l2": "inputs larger than L2, no flush"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -472,6 +505,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-conv", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--no-complex", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -569,6 +603,8 @@ def main():
         line["conv1d"] = conv1d_measure()
     if rank == 0 and not args.no_bwd:
         line["backward"] = backward_measure()
+    if rank == 0 and not args.no_complex:
+        line["complex"] = complex_measure()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:

@@ -251,6 +251,40 @@ int mamba_scan_fwd_strided(const void *u, const void *delta, const float *A,
                            const mamba_scan_tuning_t *tuning,
                            cudaStream_t stream);
 
+/*
+ * mamba_scan_fwd_complex -- the scan in complex-valued mode: a complex
+ * diagonal A and complex, input-dependent B and C (the complex SSM the Mamba
+ * paper compares with the real one on audio, Appendix E.4.1; the "complex
+ * number mode" on the roadmap of the "Mamba x JAX" page).  The pages give no
+ * formulas for it; this is the real recurrence over the complex numbers with
+ * the real part of the readout as output:
+ *
+ *   delta = softplus(delta_raw + delta_bias[d])            (real)
+ *   Abar  = exp(delta A[d,n])                               (complex)
+ *   h[n]  = Abar h[n] + delta B[b,n,t] u[b,d,t]             (complex)
+ *   y     = Re(sum_n C[b,n,t] h[n]) + D[d] u[b,d,t];  out = y silu(z)
+ *
+ *   u, delta, z, out : act (batch, dim, seqlen), as mamba_scan_fwd.
+ *   A            : fp32 (dim, dstate, 2): (re, im) pairs.
+ *   B, C         : act (batch, dstate, seqlen, 2): (re, im) pairs.
+ *   h0           : fp32 (batch, dim, dstate, 2) or NULL (zeros); may be
+ *                  last_state exactly.
+ *   last_state   : fp32 (batch, dim, dstate, 2) or NULL.
+ *   tuning       : NULL or schedule AUTO / STATIC with lanes_per_channel
+ *                  0 (auto), 1, 2 or 4; other fields 0.
+ *
+ * dstate <= 16.  Each state-step takes three special-function ops (ex2, sin,
+ * cos).  Aliasing rules and errors as mamba_scan_fwd.
+ */
+int mamba_scan_fwd_complex(const void *u, const void *delta, const float *A,
+                           const void *B, const void *C, const float *D,
+                           const void *z, const float *delta_bias,
+                           int delta_softplus, const float *h0, void *out,
+                           float *last_state, int64_t batch, int64_t dim,
+                           int64_t seqlen, int64_t dstate, int act_dtype,
+                           const mamba_scan_tuning_t *tuning,
+                           cudaStream_t stream);
+
 /* Synchronises `stream`, then reads the status a persistent launch left in
  * `workspace`: MAMBA_OK, or MAMBA_ERR_TIMEOUT if a worker stopped waiting for
  * a predecessor chunk (the outputs of that launch are then incomplete).

@@ -30,7 +30,8 @@ SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT = 0, 1, 2
 # Every function include/mamba_scan.h declares.
 EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
-            "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_fwd_strided", "mamba_scan_bwd", "mamba_scan_bwd_init",
+            "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_fwd_strided",
+            "mamba_scan_fwd_complex", "mamba_scan_bwd", "mamba_scan_bwd_init",
             "mamba_scan_bwd_workspace_size",
             "mamba_state_update", "mamba_conv1d_fwd",
             "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version")
@@ -75,6 +76,9 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_fwd_strided.argtypes = scan_args[:9] + [fp] + scan_args[9:] + [
         ctypes.POINTER(ScanStrides), ctypes.POINTER(Tuning), vp]
     lib.mamba_scan_fwd_strided.restype = ci
+    lib.mamba_scan_fwd_complex.argtypes = scan_args[:9] + [fp] + scan_args[9:] + [
+        ctypes.POINTER(Tuning), vp]
+    lib.mamba_scan_fwd_complex.restype = ci
     lib.mamba_scan_fwd_noalloc.argtypes = scan_args + [vp]
     lib.mamba_scan_fwd_noalloc.restype = ci
     lib.mamba_scan_plan.argtypes = [i64, i64, i64, i64, ci, ctypes.POINTER(Tuning)]
@@ -301,6 +305,55 @@ def mamba_scan_fwd_strided(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor
                                         _ptr(last_state), batch, dim, L, N, _ACT[act], ctypes.byref(st),
                                         ctypes.byref(tun), _stream(dev))
     _check("mamba_scan_fwd_strided", rc)
+    return (out, last_state) if want_state else out
+
+
+def mamba_scan_fwd_complex(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
+                           B: torch.Tensor, C: torch.Tensor, D: Optional[torch.Tensor] = None,
+                           z: Optional[torch.Tensor] = None,
+                           delta_bias: Optional[torch.Tensor] = None,
+                           delta_softplus: bool = True, out: Optional[torch.Tensor] = None,
+                           last_state: Optional[torch.Tensor] = None,
+                           return_last_state: bool = False, h0: Optional[torch.Tensor] = None,
+                           lanes_per_channel: int = 0):
+    """Complex-valued mode.  u, delta, z: (batch, dim, L) in the activation
+    dtype; A: (dim, N, 2) fp32 (re, im); B, C: (batch, N, L, 2) in the
+    activation dtype; h0 / last_state: (batch, dim, N, 2) fp32.  Returns
+    ``out`` or ``(out, last_state)``."""
+    if u.dim() != 3:
+        raise ValueError("u must be (batch, dim, seqlen)")
+    batch, dim, L = u.shape
+    if A.dim() != 3 or A.shape[2] != 2:
+        raise ValueError("A must be (dim, dstate, 2)")
+    N = A.shape[1]
+    dev, act = u.device, u.dtype
+    if dev.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    if act not in _ACT:
+        raise TypeError(f"unsupported activation dtype {act}")
+    for name, t in (("u", u), ("delta", delta), ("z", z)):
+        _need(t, name, dev, act, (batch, dim, L))
+    _need(B, "B", dev, act, (batch, N, L, 2))
+    _need(C, "C", dev, act, (batch, N, L, 2))
+    _need(A, "A", dev, torch.float32, (dim, N, 2))
+    _need(D, "D", dev, torch.float32, (dim,))
+    _need(delta_bias, "delta_bias", dev, torch.float32, (dim,))
+    if out is None:
+        out = torch.empty_like(u)
+    _need(out, "out", dev, act, (batch, dim, L))
+    want_state = return_last_state or last_state is not None
+    if want_state and last_state is None:
+        last_state = torch.empty((batch, dim, N, 2), device=dev, dtype=torch.float32)
+    _need(last_state, "last_state", dev, torch.float32, (batch, dim, N, 2))
+    _need(h0, "h0", dev, torch.float32, (batch, dim, N, 2))
+    tun = Tuning(int(lanes_per_channel), 0, SCHEDULE_AUTO, 0)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        rc = lib.mamba_scan_fwd_complex(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                                        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(h0), _ptr(out),
+                                        _ptr(last_state), batch, dim, L, N, _ACT[act], ctypes.byref(tun),
+                                        _stream(dev))
+    _check("mamba_scan_fwd_complex", rc)
     return (out, last_state) if want_state else out
 
 

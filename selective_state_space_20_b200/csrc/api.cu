@@ -289,6 +289,57 @@ int mamba_scan_fwd_strided(const void *u, const void *delta, const float *A, con
     return mscan::launch_scan_fwd(a, pl, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 
+int mamba_scan_fwd_complex(const void *u, const void *delta, const float *A, const void *B,
+                           const void *C, const float *D, const void *z, const float *delta_bias,
+                           int delta_softplus, const float *h0, void *out, float *last_state,
+                           int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                           int act_dtype, const mamba_scan_tuning_t *tuning, cudaStream_t stream) {
+    if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
+    int rc = check_sizes(batch, dim, seqlen, dstate);
+    if (rc != MAMBA_OK) return rc;
+    if (dstate > 16) return MAMBA_ERR_UNSUPPORTED;
+    if ((double)batch * (double)dstate * (double)seqlen * 2.0 > (double)kMaxElems) return MAMBA_ERR_SHAPE;
+    if (!u || !delta || !A || !B || !C || !out) return MAMBA_ERR_NULL;
+    int lanes = 0;
+    if (tuning) {
+        if (tuning->schedule != MAMBA_SCHEDULE_AUTO && tuning->schedule != MAMBA_SCHEDULE_STATIC)
+            return MAMBA_ERR_UNSUPPORTED;
+        if (tuning->threads_per_block != 0 || tuning->chunk_timesteps != 0) return MAMBA_ERR_UNSUPPORTED;
+        lanes = tuning->lanes_per_channel;
+        if (lanes != 0 && lanes != 1 && lanes != 2 && lanes != 4) return MAMBA_ERR_UNSUPPORTED;
+    }
+    const size_t es = act_size(act_dtype);
+    const size_t nx = (size_t)(batch * dim * seqlen) * es;
+    const size_t nbc = (size_t)(batch * dstate * seqlen) * 2 * es;
+    const size_t nA = (size_t)(dim * dstate) * 8, nd = (size_t)dim * 4;
+    const size_t nls = (size_t)(batch * dim * dstate) * 8;
+    if (bad_alias(out, nx, u, nx, true) || bad_alias(out, nx, delta, nx, true) ||
+        bad_alias(out, nx, z, nx, true) || bad_alias(out, nx, B, nbc, false) ||
+        bad_alias(out, nx, C, nbc, false) || bad_alias(out, nx, A, nA, false) ||
+        bad_alias(out, nx, D, nd, false) || bad_alias(out, nx, delta_bias, nd, false))
+        return MAMBA_ERR_OVERLAP;
+    if (last_state &&
+        (overlaps(last_state, nls, u, nx) || overlaps(last_state, nls, delta, nx) ||
+         overlaps(last_state, nls, z, nx) || overlaps(last_state, nls, B, nbc) ||
+         overlaps(last_state, nls, C, nbc) || overlaps(last_state, nls, A, nA) ||
+         overlaps(last_state, nls, D, nd) || overlaps(last_state, nls, delta_bias, nd) ||
+         overlaps(last_state, nls, out, nx)))
+        return MAMBA_ERR_OVERLAP;
+    if (h0 && (overlaps(h0, nls, out, nx) || bad_alias(last_state, nls, h0, nls, true)))
+        return MAMBA_ERR_OVERLAP;
+    int status = MAMBA_OK;
+    const int sms = current_sm_count(&status);
+    if (status != MAMBA_OK) return status;
+    if (lanes == 0) lanes = mscan::complex_scan_lanes(batch, dim, sms);
+    mscan::ScanArgs a;
+    a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.D = D; a.delta_bias = delta_bias; a.out = out; a.last_state = last_state; a.h0 = h0;
+    a.strides = nullptr;
+    a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = (int)dstate;
+    a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
+    return mscan::launch_scan_fwd_complex(a, lanes, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
 int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
                    const void *C, const float *D, const void *z, const float *delta_bias,
                    int delta_softplus, void *out, float *last_state, int64_t batch,
@@ -533,6 +584,6 @@ const char *mamba_status_string(int status) {
     }
 }
 
-int mamba_abi_version(void) { return (1 << 16) | 4; }
+int mamba_abi_version(void) { return (1 << 16) | 5; }
 
 }  // extern "C"

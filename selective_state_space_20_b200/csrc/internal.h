@@ -103,6 +103,11 @@ bool persistent_supported(const ScanArgs &a);
 bool persistent_preferred(const ScanArgs &a, int sm_count);
 int persistent_choose_lanes(const ScanArgs &a, int sm_count);  // 0 = not preferred
 size_t persistent_workspace_bound(int64_t batch, int64_t dim, int64_t seqlen, int act);
+// Complex-valued mode (dstate <= 16): A (dim, N, 2), B / C (batch, N, L, 2),
+// h0 / last_state (batch, dim, N, 2); lanes 1, 2 or 4 per channel.
+int complex_scan_lanes(int64_t batch, int64_t dim, int sm_count);
+cudaError_t launch_scan_fwd_complex(const ScanArgs &a, int lanes, cudaStream_t stream);
+
 cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_timesteps,
                                        void *workspace, size_t ws_bytes, int sm_count,
                                        cudaStream_t stream);

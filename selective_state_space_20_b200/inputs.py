@@ -218,3 +218,27 @@ def initial_state(batch: int, dim: int, dstate: int, seed: int = 50, device="cpu
     with a = exp(delta A) settles at variance delta^2 / (1 - a^2), close to
     delta / (2 |A|) = 0.05 for delta = 0.1, A = -1."""
     return _normal((batch, dim, dstate), _gen(seed, device), device, torch.float32, scale)
+
+
+def complex_inputs(batch: int, dim: int, seqlen: int, dstate: int = 16, dtype: str = "bf16",
+                   seed: int = 60, device="cpu", dt_min: float = 0.001, dt_max: float = 0.1,
+                   gate: bool = True) -> Dict[str, torch.Tensor]:
+    """Inputs of one complex-mode scan.  u, delta, z (batch, dim, L) as in
+    :func:`scan_inputs`; A (dim, N, 2) fp32 with real part -1/2 and
+    imaginary part pi n (the usual complex diagonal initialisation with
+    linearly spaced frequencies); B, C (batch, N, L, 2) with N(0, 1/2) real
+    and imaginary parts (unit mean square magnitude); D ~ U(0.5, 1.5) and the
+    dt bias as in :func:`scan_inputs`."""
+    dt = DTYPES[dtype]
+    g = _gen(seed, device)
+    _, D, bias = _params(dim, dstate, dt_min, dt_max, 1e-4, "uniform", g, device)
+    n = torch.arange(dstate, dtype=torch.float32, device=device)
+    A = torch.stack([torch.full((dim, dstate), -0.5, device=device),
+                     (math.pi * n).expand(dim, dstate)], dim=-1).contiguous()
+    shp = (batch, dim, seqlen)
+    u = _normal(shp, g, device, dt)
+    delta = _normal(shp, g, device, dt, 0.5)
+    z = _normal(shp, g, device, dt) if gate else None
+    B = _normal((batch, dstate, seqlen, 2), g, device, dt, math.sqrt(0.5))
+    C = _normal((batch, dstate, seqlen, 2), g, device, dt, math.sqrt(0.5))
+    return {"u": u, "delta": delta, "A": A, "B": B, "C": C, "D": D, "z": z, "delta_bias": bias}
