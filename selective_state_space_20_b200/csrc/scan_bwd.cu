@@ -13,19 +13,23 @@
 //   ddelta_raw = ddelta sigmoid(delta_raw + bias) (softplus);  dbias += ddelta_raw
 // and, when the forward started from a given state h0, dh0 = g after t = 0.
 //
-// Design.  One lane per channel with all (<= 16) states in registers; a warp
-// takes a group of 32 channels of one batch row through the whole sequence,
-// twice: forward, storing the state every kSeg timesteps in the workspace
-// (the checkpoints), then backward segment by segment from the end: each
-// segment's inputs are staged in shared memory (B and C widened to fp32
-// [t][n] for broadcast reads, the lane's own u, delta, sigmoid, z and dout),
-// its states recomputed from the checkpoint into shared memory and consumed
-// in reverse.  dB and dC are sums over all channels of a batch row: each warp
-// sums its 32 channels with a transposed shuffle reduction that leaves lane l
-// the total for one (B or C, state) pair and stores it as the group's partial
-// sum; a second kernel adds the groups of each batch row in a fixed order.
-// dA, dD and dbias are summed over a group's whole sequence in registers and
-// added once per group with atomics.
+// Design.  A block of four warps takes a group of 32 channels of one batch
+// row through the whole sequence, twice: forward, storing the state every
+// kSeg timesteps in the workspace (the checkpoints), then backward segment
+// by segment from the end: each segment's inputs are staged once for the
+// block in shared memory (B and C widened to fp32 [t][n] for broadcast
+// reads; u, delta, sigmoid, z and dout per channel), its states recomputed
+// from the checkpoint into shared memory and consumed in reverse.  Four
+// lanes share a channel, four states each, so a group is four warps and
+// each SM sub-partition holds several -- the reverse sweep is a long chain of
+// dependent steps, and the warps hide each other's latency.  Per-channel
+// sums over states (the readout, ddelta, du) are shuffles among a channel's
+// lanes.  dB and dC are sums over all channels of a batch row: each warp sums
+// its 8 channels with a transposed shuffle reduction, the block adds its
+// warps in a fixed order and stores the group's partial sum; a second kernel
+// adds the groups of each batch row in a fixed order.  dA, dD and dbias are
+// summed over a group's whole sequence in registers and added once per
+// group with atomics.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -36,7 +40,7 @@
 namespace mscan {
 namespace {
 
-constexpr int kNS = 16;       // states per lane (dstate <= 16)
+constexpr int kNS = 16;       // padded states per channel (dstate <= 16)
 constexpr int kSeg = 8;       // timesteps between checkpoints
 constexpr int kWarpsBwd = 4;  // warps per block
 
@@ -53,11 +57,44 @@ struct BwdParams {
     int groups_per_batch, n_groups, n_segs;
 };
 
-// Sum v[i] over the 32 lanes, transposed: afterwards v[0] of lane l holds the
-// warp total of the lanes' original v[l].
+// Lane layout.  A block of kWarpsBwd warps owns one group of 32 channels of
+// one batch row; in a warp, lane = 4 c + r takes channel c (of the warp's 8)
+// and states 4 r .. 4 r + 3.  Sums over a channel's states are shuffles
+// among its 4 lanes; sums over channels (dB, dC) are shuffles among the 8
+// lanes with the same r, then shared memory across the block's warps.
+constexpr int kCPW = 8;  // channels per warp
+constexpr int kSPL = 4;  // states per lane
+
+// Shared memory per block (floats): per warp the recomputed states after
+// each step of the segment [step][lane][4 states]; the segment's B and C rows
+// widened to fp32 [t][state] (C 16 floats after B's end, so the widening
+// stores are free of bank conflicts); per warp the channels' per-timestep
+// values [quantity][t][channel]; per warp the dB / dC partial sums [t][32].
+enum { X_U, X_DL, X_SIG, X_Z, X_DOUT, X_SGZ, X_N };  // X_SIG: sigmoid(delta_raw + bias), X_SGZ: sigmoid(z)
+constexpr int kHistW = (kSeg + 1) * 32 * kSPL;
+constexpr int kBC = 2 * kSeg * kNS + 16;
+constexpr int kXW = X_N * kSeg * kCPW;
+constexpr int kRedW = kSeg * 32;
+constexpr int kOutW = 3 * kSeg * kCPW;  // per warp: du, ddelta_raw, dz [q][t][channel]
+// raw rows in flight, per stage: 32 B / C rows and 32 x 4 (channel, quantity)
+// rows of kSeg elements, sized for fp32 (bf16 uses half)
+constexpr int kRawRows = 32 + kWarpsBwd * 32;
+constexpr int kRawStage = kRawRows * kSeg;  // elements of T per stage (room reserved as floats)
+constexpr int kBlockFloats = kWarpsBwd * (kHistW + kXW + kRedW + kOutW) + kBC + 2 * kRawStage;
+
+__device__ __forceinline__ void cp16_async(void *smem, const void *gmem, bool pred) {
+    const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                 :: "r"(sa), "l"(gmem), "r"(pred ? 16 : 0) : "memory");
+}
+
+// Sum v[] over the 8 lanes that share lane & 3, transposed: afterwards
+// v[0] of lane 4 c + r holds the total of the lanes' original v[c].  Round K
+// (lane bit 16, 8, 4) halves the live values; the lane with bit K set keeps
+// the upper half.
 template <int K, int CNT>
-struct WarpTranspose {
-    __device__ __forceinline__ static void run(float (&v)[32], int lane) {
+struct ChannelTranspose {
+    __device__ __forceinline__ static void run(float (&v)[8], int lane) {
         constexpr int HALF = CNT / 2;
         const bool upper = (lane & K) != 0;
 #pragma unroll
@@ -66,46 +103,33 @@ struct WarpTranspose {
             const float keep = upper ? v[i + HALF] : v[i];
             v[i] = keep + __shfl_xor_sync(0xffffffffu, send, K);
         }
-        WarpTranspose<K / 2, HALF>::run(v, lane);
+        ChannelTranspose<K / 2, HALF>::run(v, lane);
     }
 };
 template <int CNT>
-struct WarpTranspose<0, CNT> {
-    __device__ __forceinline__ static void run(float (&)[32], int) {}
+struct ChannelTranspose<2, CNT> {
+    __device__ __forceinline__ static void run(float (&)[8], int) {}
 };
 
-// Per-warp shared memory (floats): recomputed states [step][state][lane],
-// the segment's B and C rows widened to fp32 [t][state] (C 16 floats after
-// B's end, so the widening stores are free of bank conflicts), and this
-// lane's per-timestep values [quantity][t][lane].
-constexpr int kHist = (kSeg + 1) * kNS * 32;
-constexpr int kBC = 2 * kSeg * kNS + 16;
-enum { X_U, X_DL, X_SIG, X_Z, X_DOUT, X_N };
-constexpr int kX = X_N * kSeg * 32;
-constexpr int kWarpFloats = kHist + kBC + kX;
-
-template <typename T>
-__device__ __forceinline__ void load_row16(const T *src, int tn, float (&f)[kSeg]) {
-    constexpr int V = 16 / (int)sizeof(T);
-#pragma unroll
-    for (int c = 0; c < kSeg / V; ++c) {
-        if (c * V < tn) Elem<T>::unpack(ldg16(src + c * V), f + c * V);
-        else {
-#pragma unroll
-            for (int e = 0; e < V; ++e) f[c * V + e] = 0.f;
-        }
-    }
+__device__ __forceinline__ float quad_sum(float x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    return x + __shfl_xor_sync(0xffffffffu, x, 2);
 }
 
 template <typename T, bool SP, bool GATE>
-__global__ void __launch_bounds__(kWarpsBwd * 32) scan_bwd_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(kWarpsBwd * 32, 5) scan_bwd_kernel(const BwdParams p) {
     extern __shared__ __align__(16) float bwd_smem[];
-    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-    float *wsm = bwd_smem + wib * kWarpFloats;
-    float(*hist)[kNS][32] = reinterpret_cast<float(*)[kNS][32]>(wsm);
-    float *sB = wsm + kHist;                   // [t][n]
-    float *sC = sB + kSeg * kNS + 16;          // [t][n]
-    float(*sx)[kSeg][32] = reinterpret_cast<float(*)[kSeg][32]>(wsm + kHist + kBC);
+    const int tid = threadIdx.x, lane = tid & 31, wib = tid >> 5;
+    const int c = lane >> 2, r = lane & 3;
+    float4 *hist = reinterpret_cast<float4 *>(bwd_smem + wib * kHistW);       // [kSeg + 1][32]
+    float *sB = bwd_smem + kWarpsBwd * kHistW;                                 // [t][n]
+    float *sC = sB + kSeg * kNS + 16;                                          // [t][n]
+    float *sxAll = sB + kBC;                                                   // [warp][q][t][c]
+    float *redAll = sxAll + kWarpsBwd * kXW;                                   // [warp][t][32]
+    float *sx = sxAll + wib * kXW;
+    float *red = redAll + wib * kRedW;
+    float *so = redAll + kWarpsBwd * kRedW + wib * kOutW;                      // [q][t][c]
+    T *rawBase = reinterpret_cast<T *>(redAll + kWarpsBwd * (kRedW + kOutW));  // [2][kRawRows][kSeg]
     const int64_t L = p.seqlen;
     const int N = p.dstate;
     const T *gu = static_cast<const T *>(p.u);
@@ -117,219 +141,252 @@ __global__ void __launch_bounds__(kWarpsBwd * 32) scan_bwd_kernel(const BwdParam
     T *gdu = static_cast<T *>(p.du);
     T *gdd = static_cast<T *>(p.ddelta);
     T *gdz = static_cast<T *>(p.dz);
-    const int64_t total_warps = (int64_t)gridDim.x * kWarpsBwd;
-    const bool vec = p.vec != 0;  // 16-byte row loads (aligned rows, whole chunks)
+    const bool vec = p.vec != 0;
 
-    for (int64_t grp = (int64_t)blockIdx.x * kWarpsBwd + wib; grp < p.n_groups; grp += total_warps) {
+    for (int64_t grp = blockIdx.x; grp < p.n_groups; grp += gridDim.x) {
         const int64_t b = grp / p.groups_per_batch;
-        const int64_t dc = (grp % p.groups_per_batch) * 32 + lane;
+        const int64_t d0 = (grp % p.groups_per_batch) * 32;
+        const int64_t dc = d0 + wib * kCPW + c;  // this lane's channel
         const bool valid = dc < p.dim;
-        const int64_t row = (b * p.dim + (valid ? dc : 0)) * L;  // this lane's channel row
-        float A2[kNS], Ar[kNS];
+        const int64_t row = (b * p.dim + (valid ? dc : 0)) * L;
+        float A2[kSPL], Ar[kSPL];
 #pragma unroll
-        for (int n = 0; n < kNS; ++n) {
-            Ar[n] = (valid && n < N) ? __ldg(p.A + dc * N + n) : 0.f;
-            A2[n] = Ar[n] * kLog2e;
+        for (int i = 0; i < kSPL; ++i) {
+            const int n = kSPL * r + i;
+            Ar[i] = (valid && n < N) ? __ldg(p.A + dc * N + n) : 0.f;
+            A2[i] = Ar[i] * kLog2e;
         }
         const float bias = (valid && p.delta_bias) ? __ldg(p.delta_bias + dc) : 0.f;
         const float Dd = (valid && p.D) ? __ldg(p.D + dc) : 0.f;
-        float *ck = p.ckpt + grp * (int64_t)p.n_segs * 32 * kNS + lane * kNS;
+        // checkpoints: [group][segment][32 channels][16 states]; this lane's 4 states
+        float *ck = p.ckpt + grp * (int64_t)p.n_segs * 32 * kNS + (wib * kCPW + c) * kNS + kSPL * r;
 
-        // Stage segment [t0, t0 + tn): B (and C) widened into [t][n]; this
-        // lane's u, delta (after softplus), sigmoid(delta_raw) and, for the
-        // backward, z and dout, into sx[.][t][lane].
-        auto stage = [&](int64_t t0, int tn, bool full) {
-            __syncwarp();
-            {
-                const int which = lane >> 4, n = lane & 15;  // lanes 0-15: B, 16-31: C
-                float f[kSeg];
-                if (n < N && (full || which == 0)) {
-                    const T *src = (which ? gC : gB) + (b * N + n) * L + t0;
-                    if (vec) load_row16<T>(src, tn, f);
-                    else {
+        // Staging of segment [t0, t0 + tn) for the whole block, in two halves.
+        // fetch: the raw rows go to a double-buffered shared area with 16-byte
+        // cp.async (element copies when rows are not 16-byte aligned), issued
+        // one segment ahead so the copies overlap the current segment's work:
+        // threads 0-31 copy a B (0-15) or C (16-31) row, every thread one
+        // (channel, quantity) row -- 0 u, 1 delta, 2 dout, 3 z.  convert: each
+        // thread, once its own copies have landed, widens its rows to fp32:
+        // B / C into [t][n], u / delta (softplus, sigmoid) / dout / z into
+        // each warp's sx[q][t][c].
+        const int fch = tid & 31, fq = tid >> 5;
+        const int64_t fd = d0 + fch;
+        const bool fok = fd < p.dim;
+        const T *fsrc = (fq == 0 ? gu : fq == 1 ? gd : fq == 2 ? go : gz) + (b * p.dim + (fok ? fd : 0)) * L;
+        const float fbias = (fok && p.delta_bias) ? __ldg(p.delta_bias + fd) : 0.f;
+        const int bwhich = tid >> 4, bn = tid & 15;
+        const T *bsrc = (bwhich ? gC : gB) + (b * N + (bn < N ? bn : 0)) * L;
+        auto fetch = [&](int64_t t0, int tn, bool full, int buf) {
+            T *raw = rawBase + buf * kRawStage;
+            auto copy_row = [&](T *dst, const T *src, bool ok) {
+                if (vec) {
+                    constexpr int V = 16 / (int)sizeof(T);
 #pragma unroll
-                        for (int s = 0; s < kSeg; ++s) f[s] = s < tn ? Elem<T>::load(src + s) : 0.f;
+                    for (int q = 0; q < kSeg / V; ++q) {
+                        const bool in = ok && q * V < tn;
+                        cp16_async(dst + q * V, in ? src + q * V : src, in);
                     }
                 } else {
 #pragma unroll
-                    for (int s = 0; s < kSeg; ++s) f[s] = 0.f;
+                    for (int s = 0; s < kSeg; ++s) dst[s] = (ok && s < tn) ? src[s] : T(0.f);
                 }
-                float *dst = (which ? sC : sB) + n;
+            };
+            if (tid < 32) copy_row(raw + tid * kSeg, bsrc + t0, bn < N && (full || bwhich == 0));
+            if (fq < (full ? (GATE ? 4 : 3) : 2)) copy_row(raw + (32 + tid) * kSeg, fsrc + t0, fok);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+        auto convert = [&](bool full, int buf) {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");  // this thread's copies
+            const T *raw = rawBase + buf * kRawStage;
+            float f[kSeg];
+            if (tid < 32) {
+                const T *row = raw + tid * kSeg;
+#pragma unroll
+                for (int s = 0; s < kSeg; ++s) f[s] = Elem<T>::to_f(row[s]);
+                float *dst = (bwhich ? sC : sB) + bn;
 #pragma unroll
                 for (int s = 0; s < kSeg; ++s) dst[s * kNS] = f[s];
             }
-            float fu[kSeg], fd[kSeg];
-            const bool ok = valid;
-            auto load_own = [&](const T *base, float (&f)[kSeg]) {
-                if (ok && vec) load_row16<T>(base + row + t0, tn, f);
-                else {
+            if (fq < (full ? (GATE ? 4 : 3) : 2)) {
+                const T *row = raw + (32 + tid) * kSeg;
 #pragma unroll
-                    for (int s = 0; s < kSeg; ++s) f[s] = (ok && s < tn) ? Elem<T>::load(base + row + t0 + s) : 0.f;
-                }
-            };
-            load_own(gu, fu);
-            load_own(gd, fd);
+                for (int s = 0; s < kSeg; ++s) f[s] = Elem<T>::to_f(row[s]);
+                float *dst = sxAll + (fch >> 3) * kXW + (fch & 7);
+                if (fq == 1) {
 #pragma unroll
-            for (int s = 0; s < kSeg; ++s) {
-                const float x = fd[s] + bias;
-                sx[X_U][s][lane] = fu[s];
-                sx[X_DL][s][lane] = SP ? softplus_f(x) : x;
-                if (full) sx[X_SIG][s][lane] = SP ? __fdividef(1.f, 1.f + __expf(-x)) : 1.f;
-            }
-            if (full) {
-                load_own(go, fu);
+                    for (int s = 0; s < kSeg; ++s) {
+                        const float x = f[s] + fbias;
+                        dst[(X_DL * kSeg + s) * kCPW] = SP ? softplus_f(x) : x;
+                        if (full) dst[(X_SIG * kSeg + s) * kCPW] = SP ? __fdividef(1.f, 1.f + __expf(-x)) : 1.f;
+                    }
+                } else {
+                    const int X = fq == 0 ? X_U : fq == 2 ? X_DOUT : X_Z;
 #pragma unroll
-                for (int s = 0; s < kSeg; ++s) sx[X_DOUT][s][lane] = fu[s];
-                if (GATE) {
-                    load_own(gz, fu);
+                    for (int s = 0; s < kSeg; ++s) dst[(X * kSeg + s) * kCPW] = f[s];
+                    if (fq == 3) {
 #pragma unroll
-                    for (int s = 0; s < kSeg; ++s) sx[X_Z][s][lane] = fu[s];
-                }
-            }
-            __syncwarp();
-        };
-        // h <- the states after `tn` steps of the staged segment; into hist[1..] when asked
-        auto advance = [&](float (&h)[kNS], int tn, bool keep) {
-            for (int s = 0; s < tn; ++s) {
-                const float dl = sx[X_DL][s][lane];
-                const float du = dl * sx[X_U][s][lane];
-#pragma unroll
-                for (int q = 0; q < kNS / 4; ++q) {
-                    const float4 bb = *reinterpret_cast<const float4 *>(sB + s * kNS + 4 * q);
-                    const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int n = 4 * q + i;
-                        h[n] = fmaf(ex2_mufu(dl * A2[n]), h[n], du * bv[i]);
-                        if (keep) hist[s + 1][n][lane] = h[n];
+                        for (int s = 0; s < kSeg; ++s) dst[(X_SGZ * kSeg + s) * kCPW] = __fdividef(1.f, 1.f + __expf(-f[s]));
                     }
                 }
+            }
+        };
+        // h <- the states after `tn` steps of the staged segment; into hist[1..] when asked
+        auto advance = [&](float (&h)[kSPL], int tn, bool keep) {
+            for (int s = 0; s < tn; ++s) {
+                const float dl = sx[(X_DL * kSeg + s) * kCPW + c];
+                const float du = dl * sx[(X_U * kSeg + s) * kCPW + c];
+                const float4 bb = *reinterpret_cast<const float4 *>(sB + s * kNS + kSPL * r);
+                const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                for (int i = 0; i < kSPL; ++i) h[i] = fmaf(ex2_mufu(dl * A2[i]), h[i], du * bv[i]);
+                if (keep) hist[(s + 1) * 32 + lane] = make_float4(h[0], h[1], h[2], h[3]);
             }
         };
 
         // ---- forward from h0 (or zeros): checkpoints every kSeg timesteps (state before the segment)
-        float h[kNS];
+        float h[kSPL];
 #pragma unroll
-        for (int n = 0; n < kNS; ++n) h[n] = (valid && p.h0 && n < N) ? __ldg(p.h0 + (b * p.dim + dc) * N + n) : 0.f;
-        for (int seg = 0; seg < p.n_segs; ++seg) {
+        for (int i = 0; i < kSPL; ++i) {
+            const int n = kSPL * r + i;
+            h[i] = (valid && p.h0 && n < N) ? __ldg(p.h0 + (b * p.dim + dc) * N + n) : 0.f;
+        }
+        auto seg_len = [&](int seg) {
             const int64_t t0 = (int64_t)seg * kSeg;
-            const int tn = (L - t0) < kSeg ? (int)(L - t0) : kSeg;
-            float4 *dst = reinterpret_cast<float4 *>(ck + seg * 32 * kNS);
-#pragma unroll
-            for (int q = 0; q < kNS / 4; ++q) __stcg(dst + q, make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]));
-            stage(t0, tn, false);
-            advance(h, tn, false);
+            return (L - t0) < kSeg ? (int)(L - t0) : kSeg;
+        };
+        fetch(0, seg_len(0), false, 0);
+        for (int seg = 0; seg < p.n_segs; ++seg) {
+            __stcg(reinterpret_cast<float4 *>(ck + (int64_t)seg * 32 * kNS), make_float4(h[0], h[1], h[2], h[3]));
+            __syncthreads();  // the previous segment's staging is consumed
+            convert(false, seg & 1);
+            if (seg + 1 < p.n_segs) fetch((int64_t)(seg + 1) * kSeg, seg_len(seg + 1), false, (seg + 1) & 1);
+            __syncthreads();
+            advance(h, seg_len(seg), false);
         }
 
-        // ---- backward, segment by segment from the end
-        float g[kNS], dA_acc[kNS];
+        // ---- reverse sweep, segment by segment from the end
+        float g[kSPL], dA_acc[kSPL];
 #pragma unroll
-        for (int n = 0; n < kNS; ++n) {
-            g[n] = (valid && p.dlast && n < N) ? p.dlast[(b * p.dim + dc) * N + n] : 0.f;
-            dA_acc[n] = 0.f;
+        for (int i = 0; i < kSPL; ++i) {
+            const int n = kSPL * r + i;
+            g[i] = (valid && p.dlast && n < N) ? p.dlast[(b * p.dim + dc) * N + n] : 0.f;
+            dA_acc[i] = 0.f;
         }
         float dD_acc = 0.f, dbias_acc = 0.f;
-        float *part = p.part + grp * L * 32 + lane;  // this lane's (B or C, state) partial sums
+        // this lane's slot of the warp's channel-summed dB / dC: lanes c < 4
+        // hold dB of state 4 r + c, lanes c >= 4 dC of state 4 r + c - 4
+        const int kslot = (c < 4 ? 0 : 16) + kSPL * r + (c & 3);
+        fetch((int64_t)(p.n_segs - 1) * kSeg, seg_len(p.n_segs - 1), true, (p.n_segs - 1) & 1);
         for (int seg = p.n_segs - 1; seg >= 0; --seg) {
             const int64_t t0 = (int64_t)seg * kSeg;
-            const int tn = (L - t0) < kSeg ? (int)(L - t0) : kSeg;
-            stage(t0, tn, true);
-            const float4 *src = reinterpret_cast<const float4 *>(ck + seg * 32 * kNS);
-#pragma unroll
-            for (int q = 0; q < kNS / 4; ++q) {
-                const float4 v = __ldcg(src + q);
-                h[4 * q] = v.x; h[4 * q + 1] = v.y; h[4 * q + 2] = v.z; h[4 * q + 3] = v.w;
+            const int tn = seg_len(seg);
+            __syncthreads();  // staging, hist and red of the previous segment are consumed
+            convert(true, seg & 1);
+            if (seg > 0) fetch(t0 - kSeg, seg_len(seg - 1), true, (seg - 1) & 1);
+            {
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(ck + (int64_t)seg * 32 * kNS));
+                h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
             }
-#pragma unroll
-            for (int n = 0; n < kNS; ++n) hist[0][n][lane] = h[n];
+            __syncthreads();
+            hist[lane] = make_float4(h[0], h[1], h[2], h[3]);
             advance(h, tn, true);
-            float o_du[kSeg], o_dd[kSeg], o_dz[kSeg];
-#pragma unroll
-            for (int s = 0; s < kSeg; ++s) { o_du[s] = 0.f; o_dd[s] = 0.f; o_dz[s] = 0.f; }
+            __syncwarp();
+            float4 hc4 = make_float4(h[0], h[1], h[2], h[3]);  // the state after the segment's last step
 #pragma unroll
             for (int s = kSeg - 1; s >= 0; --s) {
                 if (s >= tn) continue;
-                const float dl = sx[X_DL][s][lane];
-                const float ut = sx[X_U][s][lane];
-                const float dout = sx[X_DOUT][s][lane];
-                float y = Dd * ut;
+                const float dl = sx[(X_DL * kSeg + s) * kCPW + c];
+                const float ut = sx[(X_U * kSeg + s) * kCPW + c];
+                const float dout = sx[(X_DOUT * kSeg + s) * kCPW + c];
+                const float4 hp4 = hist[s * 32 + lane];
+                const float4 bb = *reinterpret_cast<const float4 *>(sB + s * kNS + kSPL * r);
+                const float4 cc = *reinterpret_cast<const float4 *>(sC + s * kNS + kSPL * r);
+                const float hcur[4] = {hc4.x, hc4.y, hc4.z, hc4.w}, hp[4] = {hp4.x, hp4.y, hp4.z, hp4.w};
+                const float bv[4] = {bb.x, bb.y, bb.z, bb.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
+                float yp = 0.f;
 #pragma unroll
-                for (int q = 0; q < kNS / 4; ++q) {
-                    const float4 cc = *reinterpret_cast<const float4 *>(sC + s * kNS + 4 * q);
-                    y = fmaf(cc.x, hist[s + 1][4 * q][lane], y);
-                    y = fmaf(cc.y, hist[s + 1][4 * q + 1][lane], y);
-                    y = fmaf(cc.z, hist[s + 1][4 * q + 2][lane], y);
-                    y = fmaf(cc.w, hist[s + 1][4 * q + 3][lane], y);
-                }
+                for (int i = 0; i < kSPL; ++i) yp = fmaf(cv[i], hcur[i], yp);
+                const float y = fmaf(Dd, ut, quad_sum(yp));
                 float dy = dout;
                 if (GATE) {
-                    const float zt = sx[X_Z][s][lane];
-                    const float sg = __fdividef(1.f, 1.f + __expf(-zt));
-                    o_dz[s] = dout * y * sg * fmaf(zt, 1.f - sg, 1.f);
+                    const float zt = sx[(X_Z * kSeg + s) * kCPW + c];
+                    const float sg = sx[(X_SGZ * kSeg + s) * kCPW + c];
+                    if (r == 0) so[(2 * kSeg + s) * kCPW + c] = dout * y * sg * fmaf(zt, 1.f - sg, 1.f);
                     dy = dout * zt * sg;
                 }
                 dD_acc = fmaf(dy, ut, dD_acc);
-                float dut = dy * Dd, ddelta = 0.f;
-                float v[32];  // this lane's dB (states 0-15) and dC (16-31) terms
+                float dut_p = 0.f, ddelta_p = 0.f;
+                float v[8];  // dB (0-3) and dC (4-7) terms of this lane's states
 #pragma unroll
-                for (int q = 0; q < kNS / 4; ++q) {
-                    const float4 bb = *reinterpret_cast<const float4 *>(sB + s * kNS + 4 * q);
-                    const float4 cc = *reinterpret_cast<const float4 *>(sC + s * kNS + 4 * q);
-                    const float bv[4] = {bb.x, bb.y, bb.z, bb.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int n = 4 * q + i;
-                        const float hcur = hist[s + 1][n][lane], hp = hist[s][n][lane];
-                        v[16 + n] = dy * hcur;
-                        g[n] = fmaf(dy, cv[i], g[n]);
-                        const float ab = ex2_mufu(dl * A2[n]);
-                        const float gha = g[n] * hp * ab;
-                        ddelta = fmaf(gha, Ar[n], fmaf(g[n], bv[i] * ut, ddelta));
-                        dA_acc[n] = fmaf(gha, dl, dA_acc[n]);
-                        v[n] = g[n] * dl * ut;
-                        dut = fmaf(g[n] * dl, bv[i], dut);
-                        g[n] *= ab;
-                    }
+                for (int i = 0; i < kSPL; ++i) {
+                    v[4 + i] = dy * hcur[i];
+                    g[i] = fmaf(dy, cv[i], g[i]);
+                    const float ab = ex2_mufu(dl * A2[i]);
+                    const float gha = g[i] * hp[i] * ab;
+                    ddelta_p = fmaf(gha, Ar[i], fmaf(g[i], bv[i] * ut, ddelta_p));
+                    dA_acc[i] = fmaf(gha, dl, dA_acc[i]);
+                    v[i] = g[i] * dl * ut;
+                    dut_p = fmaf(g[i] * dl, bv[i], dut_p);
+                    g[i] *= ab;
                 }
-                WarpTranspose<16, 32>::run(v, lane);
-                __stcg(part + (t0 + s) * 32, v[0]);
-                const float ddraw = ddelta * sx[X_SIG][s][lane];
+                ChannelTranspose<16, 8>::run(v, lane);
+                red[s * 32 + kslot] = v[0];
+                const float ddelta = quad_sum(ddelta_p);
+                const float ddraw = ddelta * sx[(X_SIG * kSeg + s) * kCPW + c];
                 dbias_acc += ddraw;
-                o_du[s] = dut;
-                o_dd[s] = ddraw;
+                const float dut = fmaf(dy, Dd, quad_sum(dut_p));
+                if (r == 0) {
+                    so[(0 * kSeg + s) * kCPW + c] = dut;
+                    so[(1 * kSeg + s) * kCPW + c] = ddraw;
+                }
+                hc4 = hp4;
             }
-            // this lane's row of the segment, 16 bytes at a time where possible
-            if (valid) {
+            // this channel's rows of the segment: lane r = 0 du, 1 ddelta_raw,
+            // 2 dz, 16 bytes at a time where possible
+            __syncwarp();
+            if (valid && r < (GATE ? 3 : 2)) {
                 constexpr int V = 16 / (int)sizeof(T);
+                T *dst = (r == 0 ? gdu : r == 1 ? gdd : gdz) + row + t0;
+                float f[kSeg];
 #pragma unroll
-                for (int c = 0; c < kSeg / V; ++c) {
-                    if (vec && (c + 1) * V <= tn) {
-                        *reinterpret_cast<uint4 *>(gdu + row + t0 + c * V) = Elem<T>::pack(o_du + c * V);
-                        *reinterpret_cast<uint4 *>(gdd + row + t0 + c * V) = Elem<T>::pack(o_dd + c * V);
-                        if (GATE) *reinterpret_cast<uint4 *>(gdz + row + t0 + c * V) = Elem<T>::pack(o_dz + c * V);
+                for (int s = 0; s < kSeg; ++s) f[s] = so[(r * kSeg + s) * kCPW + c];
+#pragma unroll
+                for (int q = 0; q < kSeg / V; ++q) {
+                    if (vec && (q + 1) * V <= tn) {
+                        *reinterpret_cast<uint4 *>(dst + q * V) = Elem<T>::pack(f + q * V);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < V; ++e) {
-                            const int s = c * V + e;
-                            if (s < tn) {
-                                Elem<T>::store(gdu + row + t0 + s, o_du[s]);
-                                Elem<T>::store(gdd + row + t0 + s, o_dd[s]);
-                                if (GATE) Elem<T>::store(gdz + row + t0 + s, o_dz[s]);
-                            }
-                        }
+                        for (int e = 0; e < V; ++e)
+                            if (q * V + e < tn) Elem<T>::store(dst + q * V + e, f[q * V + e]);
                     }
                 }
+            }
+            // the block's dB / dC partial sums: the warps' sums added in warp order
+            __syncthreads();
+            float *part = p.part + (grp * L + t0) * 32;
+            for (int idx = tid; idx < tn * 32; idx += kWarpsBwd * 32) {
+                float acc = 0.f;
+#pragma unroll
+                for (int w = 0; w < kWarpsBwd; ++w) acc += redAll[w * kRedW + idx];
+                __stcg(part + idx, acc);
             }
         }
         if (valid) {
 #pragma unroll
-            for (int n = 0; n < kNS; ++n) {
-                if (n < N) atomicAdd(p.dA + dc * N + n, dA_acc[n]);
-                if (n < N && p.dh0) p.dh0[(b * p.dim + dc) * N + n] = g[n];  // dL/dh_{-1}
+            for (int i = 0; i < kSPL; ++i) {
+                const int n = kSPL * r + i;
+                if (n < N) {
+                    atomicAdd(p.dA + dc * N + n, dA_acc[i]);
+                    if (p.dh0) p.dh0[(b * p.dim + dc) * N + n] = g[i];  // dL/dh_{-1}
+                }
             }
-            if (p.dD) atomicAdd(p.dD + dc, dD_acc);
-            if (p.dbias) atomicAdd(p.dbias + dc, dbias_acc);
+            if (r == 0) {
+                if (p.dD) atomicAdd(p.dD + dc, dD_acc);
+                if (p.dbias) atomicAdd(p.dbias + dc, dbias_acc);
+            }
         }
+        __syncthreads();  // before the next group reuses shared memory
     }
 }
 
@@ -364,16 +421,15 @@ __global__ void __launch_bounds__(256) bwd_reduce_bc_kernel(const BwdParams p) {
 template <typename T, bool SP, bool GATE>
 cudaError_t launch_t(const BwdParams &p, int sm_count, cudaStream_t st) {
     auto kern = scan_bwd_kernel<T, SP, GATE>;
-    const int smem = kWarpsBwd * kWarpFloats * 4;
+    const int smem = kBlockFloats * 4;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarpsBwd * 32, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
-    int64_t grid = (int64_t)sm_count * per_sm;
-    const int64_t need = (p.n_groups + kWarpsBwd - 1) / kWarpsBwd;
-    if (grid > need) grid = need;
+    int64_t grid = (int64_t)sm_count * per_sm;  // one block per channel group, grid-strided
+    if (grid > p.n_groups) grid = p.n_groups;
     kern<<<(unsigned)grid, kWarpsBwd * 32, smem, st>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
