@@ -79,6 +79,7 @@ KERNEL_SOURCES = {
                              "persistent_host.cu", "device_math.cuh", "internal.h"),
     "scan_fwd_kernel": ("scan_fwd.cu", "device_math.cuh", "internal.h"),
     "scan_fwd_complex_kernel": ("scan_fwd_complex.cu", "device_math.cuh", "internal.h"),
+    "scan_bwd_kernel": ("scan_bwd.cu", "device_math.cuh", "internal.h"),
 }
 
 
@@ -457,6 +458,7 @@ def backward_measure(reps=5):
     return {"workload": w.name, "us_per_call": us, "Gelem_per_s": achieved,
             "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Gelem/s",
                          "frac": achieved / peak,
+                         "traffic": measured_traffic(f"scan_bwd_kernel {w.name}"),
                          "note": "peak = 16 decays per element once on the MUFU; the kernel evaluates them 3x "
                                  "(checkpoint sweep, segment recompute, reverse sweep)"},
             "reps": reps}
@@ -490,6 +492,8 @@ def complex_measure(reps=10):
             "us_per_call": us, "Gelem_per_s": achieved,
             "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Gelem/s",
                          "frac": achieved / peak,
+                         "traffic": measured_traffic(f"scan_fwd_complex_kernel complex mode {w.batch}x{w.dim}x{w.seqlen} "
+                                                     f"N{w.dstate} {w.dtype}"),
                          "note": "peak = MUFU ops/s over 3 N (ex2, sin, cos per complex state-step)"},
             "reps": reps, "l2": "inputs larger than L2, no flush"}
 
