@@ -108,3 +108,29 @@ def test_bwd_full_size_layer():
     for k in ACT_GRADS:
         e = rel_err(to_np(got[k][b:b + 1, chans]), r[k])
         assert e <= 2e-2, (k, e)
+
+
+def test_bwd_benchmark_layer_sampled():
+    """The layer the bench times the backward on (Mamba-2.8B, 4 x 5120 x 4096,
+    bf16, with dL/dlast_state): du, ddelta, dz on sampled channels of two batch
+    rows, and dA, dD, dbias of sampled channels (sums over all four batch
+    rows) against the oracle run on exactly those rows."""
+    w = inputs.MAMBA_2_8B
+    dev = inputs.scan_inputs(w, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(7)
+    dout = torch.randn(w.batch, w.dim, w.seqlen, generator=g, device="cuda").to(torch.bfloat16)
+    dlast = torch.randn(w.batch, w.dim, w.dstate, generator=g, device="cuda")
+    got = binding.mamba_scan_bwd(dout, dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],
+                                 z=dev["z"], delta_bias=dev["delta_bias"], dlast_state=dlast)
+    torch.cuda.synchronize()
+    chans = [0, 31, 32, 2047, 4096, 5119]
+    cpu = lambda t: t.detach().to("cpu")  # noqa: E731
+    r = oracle.scan_bwd(cpu(dout[:, chans]), cpu(dev["u"][:, chans]), cpu(dev["delta"][:, chans]),
+                        cpu(dev["A"][chans]), cpu(dev["B"]), cpu(dev["C"]), D=cpu(dev["D"][chans]),
+                        z=cpu(dev["z"][:, chans]), delta_bias=cpu(dev["delta_bias"][chans]),
+                        dlast=cpu(dlast[:, chans]).double())
+    errs = {k: rel_err(to_np(got[k][:, chans]), r[k]) for k in ACT_GRADS}
+    errs.update({k: rel_err(to_np(got[k][chans]), r[k]) for k in ("dA", "dD", "ddelta_bias")})
+    record("scan_bwd mamba-2.8b layer sampled channels", **errs)
+    for k, e in errs.items():
+        assert e <= (TOL[torch.bfloat16] if k in ACT_GRADS else 1e-3), (k, e, errs)

@@ -114,3 +114,25 @@ def test_complex_rejects_bad_arguments():
     dev = {k: (None if v is None else v.cuda()) for k, v in big.items()}
     with pytest.raises(binding.MambaError):  # dstate > 16
         _run(dev)
+
+
+def test_complex_benchmark_shape_sampled():
+    """The shape the bench times complex mode on (4 x 5120 x 4096, N = 16,
+    bf16), sampled rows against the oracle run on each row alone."""
+    b, d, L, N = 4, 5120, 4096, 16
+    dev = {k: (None if v is None else v.cuda()) for k, v in inputs.complex_inputs(b, d, L, N, "bf16", device="cuda").items()}
+    out, last = _run(dev)
+    torch.cuda.synchronize()
+    rows = [(0, 0), (0, 5119), (1, 777), (2, 2048), (3, 0), (3, 5119)]
+    cpu = lambda t: None if t is None else t.detach().to("cpu")  # noqa: E731
+    errs = []
+    for bi, di in rows:
+        ro, rs = oracle.scan_complex(cpu(dev["u"][bi:bi + 1, di:di + 1]), cpu(dev["delta"][bi:bi + 1, di:di + 1]),
+                                     cpu(dev["A"][di:di + 1]), cpu(dev["B"][bi:bi + 1]), cpu(dev["C"][bi:bi + 1]),
+                                     D=cpu(dev["D"][di:di + 1]), z=cpu(dev["z"][bi:bi + 1, di:di + 1]),
+                                     delta_bias=cpu(dev["delta_bias"][di:di + 1]), nthreads=1)
+        errs.append((rel_err(to_np(out[bi, di]), ro[0, 0]),
+                     rel_err(to_np(last[bi, di]), np.stack([rs.real, rs.imag], -1)[0, 0])))
+    e_out, e_state = max(e[0] for e in errs), max(e[1] for e in errs)
+    record("complex 4x5120x4096 N16 bf16 sampled", out=e_out, state=e_state)
+    assert e_out <= TOL[torch.bfloat16] and e_state <= TOL[torch.bfloat16], errs
