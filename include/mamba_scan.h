@@ -285,6 +285,43 @@ int mamba_scan_fwd_complex(const void *u, const void *delta, const float *A,
                            const mamba_scan_tuning_t *tuning,
                            cudaStream_t stream);
 
+/*
+ * Splitting one sequence across GPUs.  The recurrence is affine in the state
+ * and its decays are diagonal, so a shard of timesteps maps an initial state
+ * h to exp(A * S) (.) h + h_local, where S is the shard's sum of delta
+ * (after bias and softplus) per (batch, channel) and h_local its final state
+ * from a zero start (the recurrent form of "Mamba SSM concept and
+ * implementation in Keras and TensorFlow", unrolled over the shard).  Rank r
+ * scans its shard from zero (mamba_scan_fwd with last_state -> h_local),
+ * sums delta (mamba_delta_sum -> S), exchanges (S, h_local) with the other
+ * ranks, folds the summaries of ranks 0 .. r-1 into its true initial state
+ * (mamba_state_fold) and scans its shard again from it (mamba_scan_fwd_init).
+ *
+ * mamba_delta_sum -- S[b, d] = sum_t softplus(delta[b, d, t] + delta_bias[d])
+ * (without softplus when delta_softplus is 0), accumulated in fp64.
+ *   delta        : act (batch, dim, seqlen); delta_bias: fp32 (dim) or NULL.
+ *   out          : fp64 (batch, dim), written.
+ */
+int mamba_delta_sum(const void *delta, const float *delta_bias, int delta_softplus,
+                    double *out, int64_t batch, int64_t dim, int64_t seqlen, int act_dtype,
+                    cudaStream_t stream);
+
+/*
+ * mamba_state_fold -- h_out = the state after `count` shards starting from
+ * h_init (NULL: zeros): for k = 0 .. count - 1,
+ *   h <- exp(A[d, n] * delta_sums[k][b, d]) * h + h_local[k][b, d, n]
+ * evaluated in fp64, rounded to fp32 once.
+ *   h_init       : fp32 (batch, dim, dstate) or NULL.
+ *   delta_sums   : fp64 (count, batch, dim); h_local: fp32 (count, batch, dim, dstate).
+ *   A            : fp32 (dim, dstate).
+ *   h_out        : fp32 (batch, dim, dstate), written; may be h_init or one of
+ *                  the h_local slices exactly.
+ * count may be 0 (h_out = h_init, or zeros).
+ */
+int mamba_state_fold(const float *h_init, const double *delta_sums, const float *A,
+                     const float *h_local, float *h_out, int64_t batch, int64_t dim,
+                     int64_t dstate, int64_t count, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads the status a persistent launch left in
  * `workspace`: MAMBA_OK, or MAMBA_ERR_TIMEOUT if a worker stopped waiting for
  * a predecessor chunk (the outputs of that launch are then incomplete).

@@ -31,7 +31,7 @@ SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT = 0, 1, 2
 EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
             "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_fwd_strided",
-            "mamba_scan_fwd_complex", "mamba_scan_bwd", "mamba_scan_bwd_init",
+            "mamba_scan_fwd_complex", "mamba_delta_sum", "mamba_state_fold", "mamba_scan_bwd", "mamba_scan_bwd_init",
             "mamba_scan_bwd_workspace_size",
             "mamba_state_update", "mamba_conv1d_fwd",
             "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version")
@@ -79,6 +79,11 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_fwd_complex.argtypes = scan_args[:9] + [fp] + scan_args[9:] + [
         ctypes.POINTER(Tuning), vp]
     lib.mamba_scan_fwd_complex.restype = ci
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.mamba_delta_sum.argtypes = [vp, fp, ci, dp, i64, i64, i64, ci, vp]
+    lib.mamba_delta_sum.restype = ci
+    lib.mamba_state_fold.argtypes = [fp, dp, fp, fp, fp, i64, i64, i64, i64, vp]
+    lib.mamba_state_fold.restype = ci
     lib.mamba_scan_fwd_noalloc.argtypes = scan_args + [vp]
     lib.mamba_scan_fwd_noalloc.restype = ci
     lib.mamba_scan_plan.argtypes = [i64, i64, i64, i64, ci, ctypes.POINTER(Tuning)]
@@ -355,6 +360,54 @@ def mamba_scan_fwd_complex(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor
                                         _stream(dev))
     _check("mamba_scan_fwd_complex", rc)
     return (out, last_state) if want_state else out
+
+
+def mamba_delta_sum(delta: torch.Tensor, delta_bias: Optional[torch.Tensor] = None,
+                    delta_softplus: bool = True) -> torch.Tensor:
+    """Per-row sum over time of delta after bias and softplus: (batch, dim)
+    fp64."""
+    if delta.dim() != 3:
+        raise ValueError("delta must be (batch, dim, seqlen)")
+    batch, dim, L = delta.shape
+    dev, act = delta.device, delta.dtype
+    if dev.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    if act not in _ACT:
+        raise TypeError(f"unsupported activation dtype {act}")
+    _need(delta, "delta", dev, act, (batch, dim, L))
+    _need(delta_bias, "delta_bias", dev, torch.float32, (dim,))
+    out = torch.empty((batch, dim), device=dev, dtype=torch.float64)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        rc = lib.mamba_delta_sum(_ptr(delta), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(out),
+                                 batch, dim, L, _ACT[act], _stream(dev))
+    _check("mamba_delta_sum", rc)
+    return out
+
+
+def mamba_state_fold(A: torch.Tensor, delta_sums: torch.Tensor, h_local: torch.Tensor,
+                     h_init: Optional[torch.Tensor] = None,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The state after ``count`` shards from ``h_init`` (zeros if None):
+    delta_sums (count, batch, dim) fp64, h_local (count, batch, dim, N)
+    fp32; returns (batch, dim, N) fp32."""
+    if h_local.dim() != 4:
+        raise ValueError("h_local must be (count, batch, dim, dstate)")
+    count, batch, dim, N = h_local.shape
+    dev = A.device
+    _need(A, "A", dev, torch.float32, (dim, N))
+    _need(delta_sums, "delta_sums", dev, torch.float64, (count, batch, dim))
+    _need(h_local, "h_local", dev, torch.float32, (count, batch, dim, N))
+    _need(h_init, "h_init", dev, torch.float32, (batch, dim, N))
+    if out is None:
+        out = torch.empty((batch, dim, N), device=dev, dtype=torch.float32)
+    _need(out, "out", dev, torch.float32, (batch, dim, N))
+    lib = load_library()
+    with torch.cuda.device(dev):
+        rc = lib.mamba_state_fold(_ptr(h_init), _ptr(delta_sums), _ptr(A), _ptr(h_local), _ptr(out),
+                                  batch, dim, N, count, _stream(dev))
+    _check("mamba_state_fold", rc)
+    return out
 
 
 def workspace_status(workspace: torch.Tensor) -> int:

@@ -340,6 +340,44 @@ int mamba_scan_fwd_complex(const void *u, const void *delta, const float *A, con
     return mscan::launch_scan_fwd_complex(a, lanes, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 
+int mamba_delta_sum(const void *delta, const float *delta_bias, int delta_softplus,
+                    double *out, int64_t batch, int64_t dim, int64_t seqlen, int act_dtype,
+                    cudaStream_t stream) {
+    if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
+    int rc = check_sizes(batch, dim, seqlen, 1);
+    if (rc != MAMBA_OK) return rc;
+    if (!delta || !out) return MAMBA_ERR_NULL;
+    const size_t nx = (size_t)(batch * dim * seqlen) * act_size(act_dtype);
+    if (overlaps(out, (size_t)(batch * dim) * 8, delta, nx) ||
+        overlaps(out, (size_t)(batch * dim) * 8, delta_bias, (size_t)dim * 4))
+        return MAMBA_ERR_OVERLAP;
+    return mscan::launch_delta_sum(delta, delta_bias, delta_softplus ? 1 : 0, out, batch, dim, seqlen,
+                                   act_dtype, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
+int mamba_state_fold(const float *h_init, const double *delta_sums, const float *A,
+                     const float *h_local, float *h_out, int64_t batch, int64_t dim,
+                     int64_t dstate, int64_t count, cudaStream_t stream) {
+    int rc = check_sizes(batch, dim, 1, dstate);
+    if (rc != MAMBA_OK) return rc;
+    if (count < 0 || count > (1 << 20)) return MAMBA_ERR_SHAPE;
+    if (!A || !h_out || (count > 0 && (!delta_sums || !h_local))) return MAMBA_ERR_NULL;
+    const size_t ns = (size_t)(batch * dim * dstate) * 4;
+    if ((double)count * (double)ns > (double)kMaxElems) return MAMBA_ERR_SHAPE;
+    const size_t nsum = (size_t)count * (size_t)(batch * dim) * 8;
+    // h_out may be h_init or one of the h_local slices exactly; nothing else
+    if (h_init && overlaps(h_out, ns, h_init, ns) && h_out != h_init) return MAMBA_ERR_OVERLAP;
+    if (count > 0 && overlaps(h_out, ns, h_local, (size_t)count * ns)) {
+        const uintptr_t off = reinterpret_cast<uintptr_t>(h_out) - reinterpret_cast<uintptr_t>(h_local);
+        if (reinterpret_cast<uintptr_t>(h_out) < reinterpret_cast<uintptr_t>(h_local) || off % ns != 0)
+            return MAMBA_ERR_OVERLAP;
+    }
+    if (overlaps(h_out, ns, delta_sums, nsum) || overlaps(h_out, ns, A, (size_t)(dim * dstate) * 4))
+        return MAMBA_ERR_OVERLAP;
+    return mscan::launch_state_fold(h_init, delta_sums, A, h_local, h_out, batch, dim, dstate, (int)count,
+                                    stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
 int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
                    const void *C, const float *D, const void *z, const float *delta_bias,
                    int delta_softplus, void *out, float *last_state, int64_t batch,
@@ -584,6 +622,6 @@ const char *mamba_status_string(int status) {
     }
 }
 
-int mamba_abi_version(void) { return (1 << 16) | 5; }
+int mamba_abi_version(void) { return (1 << 16) | 6; }
 
 }  // extern "C"

@@ -103,6 +103,14 @@ bool persistent_supported(const ScanArgs &a);
 bool persistent_preferred(const ScanArgs &a, int sm_count);
 int persistent_choose_lanes(const ScanArgs &a, int sm_count);  // 0 = not preferred
 size_t persistent_workspace_bound(int64_t batch, int64_t dim, int64_t seqlen, int act);
+// Sequence split across GPUs: per-row sums of delta, and the fold of shard
+// summaries into an initial state (seqpar.cu).
+cudaError_t launch_delta_sum(const void *delta, const float *bias, int softplus, double *out,
+                             int64_t batch, int64_t dim, int64_t seqlen, int act, cudaStream_t stream);
+cudaError_t launch_state_fold(const float *h_init, const double *sums, const float *A,
+                              const float *h_local, float *h_out, int64_t batch, int64_t dim,
+                              int64_t dstate, int count, cudaStream_t stream);
+
 // Complex-valued mode (dstate <= 16): A (dim, N, 2), B / C (batch, N, L, 2),
 // h0 / last_state (batch, dim, N, 2); lanes 1, 2 or 4 per channel.
 int complex_scan_lanes(int64_t batch, int64_t dim, int sm_count);
