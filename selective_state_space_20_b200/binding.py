@@ -79,7 +79,7 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_fwd_complex.argtypes = scan_args[:9] + [fp] + scan_args[9:] + [
         ctypes.POINTER(Tuning), vp]
     lib.mamba_scan_fwd_complex.restype = ci
-    dp = ctypes.POINTER(ctypes.c_double)
+    dp = vp  # double *
     lib.mamba_delta_sum.argtypes = [vp, fp, ci, dp, i64, i64, i64, ci, vp]
     lib.mamba_delta_sum.restype = ci
     lib.mamba_state_fold.argtypes = [fp, dp, fp, fp, fp, i64, i64, i64, i64, vp]

@@ -194,3 +194,23 @@ def test_scan_bwd_validation(lib):
     assert call_init(None, None) == -1                     # h0 is required
     assert call_init(P[13], vp(0x600000 + 128)) == -7      # dh0 inside dout
     assert call_init(P[13], P[13]) == -7                   # dh0 over h0
+
+
+def test_sequence_split_validation(lib):
+    vp = ctypes.c_void_p
+    # argument marshalling as the binding passes it, rejected before any device work
+    assert lib.mamba_delta_sum(vp(0x100000), vp(0x200000), 1, vp(0x300000), 0, 4, 8, 1, None) == -2
+    assert lib.mamba_delta_sum(None, None, 1, vp(0x300000), 2, 4, 8, 1, None) == -1
+    assert lib.mamba_delta_sum(vp(0x100000), None, 1, vp(0x100000 + 8), 2, 4, 8, 1, None) == -7
+    assert lib.mamba_state_fold(vp(0x100000), vp(0x200000), vp(0x300000), vp(0x400000), vp(0x500000),
+                                2, 4, 16, -1, None) == -2
+    assert lib.mamba_state_fold(None, None, vp(0x300000), None, vp(0x500000), 2, 4, 16, 3, None) == -1
+    # the output partly over the initial state
+    assert lib.mamba_state_fold(vp(0x500000), vp(0x200000), vp(0x300000), vp(0x400000), vp(0x500000 + 4),
+                                2, 4, 16, 1, None) == -7
+    # the output over the second h_local slice exactly is allowed; mid-slice is not
+    ns = 2 * 4 * 16 * 4
+    assert lib.mamba_state_fold(None, vp(0x200000), vp(0x300000), vp(0x400000), vp(0x400000 + 12),
+                                2, 4, 16, 2, None) == -7
+    assert lib.mamba_state_fold(None, vp(0x200000), vp(0x300000), vp(0x400000), vp(0x400000 + ns + 16),
+                                2, 4, 16, 2, None) == -7
