@@ -286,6 +286,50 @@ int mamba_scan_fwd_complex(const void *u, const void *delta, const float *A,
                            cudaStream_t stream);
 
 /*
+ * mamba_scan_fwd_conv -- the causal depthwise conv1d + silu fused into the
+ * scan's prologue: the step before the scan in the Mamba block ("Mamba SSM
+ * concept and implementation in Keras and TensorFlow", MambaBlock: Conv1D
+ * with one group per channel, causal padding, bias, then swish) computed
+ * where the scan loads u, so u never makes a round trip through HBM:
+ *
+ *   u[b,d,t] = silu(conv_bias[d] + sum_{k<K} conv_weight[d,k] x[b,d,t-(K-1)+k]),
+ *              x = 0 before the sequence, u rounded to the activation type,
+ *   then the scan of mamba_scan_fwd_init on that u, softplus on.
+ *
+ * The result equals mamba_conv1d_fwd followed by mamba_scan_fwd_ws bit for
+ * bit.
+ *
+ *   x            : act; channel d of batch row b is the seqlen-long row at
+ *                  x + b * x_batch_stride + d * seqlen (0: dim * seqlen) --
+ *                  e.g. the x half of the in-projection's (batch, 2 dim,
+ *                  seqlen) output.
+ *   conv_weight  : fp32 (dim, conv_width), conv_width 1 .. 4; conv_bias:
+ *                  fp32 (dim) or NULL.
+ *   z            : act or NULL, rows at z + b * z_batch_stride + d * seqlen
+ *                  (0: dim * seqlen) -- e.g. the other half of the same
+ *                  output; x and z may share one buffer.
+ *   u_out        : act (batch, dim, seqlen) or NULL: the u it formed (what a
+ *                  backward pass needs).
+ *   h0           : fp32 (batch, dim, dstate) or NULL; may be last_state.
+ *   other arguments as mamba_scan_fwd_ws; the workspace is required.
+ *
+ * The fused prologue lives in the persistent lane-split kernel, so the
+ * call needs its layout: dstate <= 16, 16-byte-aligned tensors, seqlen and
+ * both batch strides multiples of 8 (bf16) or 4 (fp32) elements; otherwise
+ * MAMBA_ERR_UNSUPPORTED (run the two calls instead).  out, u_out and
+ * last_state must not overlap any input (h0 == last_state excepted) or
+ * each other.
+ */
+int mamba_scan_fwd_conv(const void *x, const float *conv_weight, const float *conv_bias,
+                        int64_t conv_width, int64_t x_batch_stride, const void *delta,
+                        const float *A, const void *B, const void *C, const float *D,
+                        const void *z, int64_t z_batch_stride, const float *delta_bias,
+                        const float *h0, void *out, float *last_state, void *u_out,
+                        int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                        int act_dtype, void *workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
+/*
  * Splitting one sequence across GPUs.  The recurrence is affine in the state
  * and its decays are diagonal, so a shard of timesteps maps an initial state
  * h to exp(A * S) (.) h + h_local, where S is the shard's sum of delta

@@ -31,7 +31,7 @@ SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT = 0, 1, 2
 EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
             "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_fwd_strided",
-            "mamba_scan_fwd_complex", "mamba_delta_sum", "mamba_state_fold", "mamba_scan_bwd", "mamba_scan_bwd_init",
+            "mamba_scan_fwd_complex", "mamba_delta_sum", "mamba_state_fold", "mamba_scan_fwd_conv", "mamba_scan_bwd", "mamba_scan_bwd_init",
             "mamba_scan_bwd_workspace_size",
             "mamba_state_update", "mamba_conv1d_fwd",
             "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version")
@@ -80,6 +80,9 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         ctypes.POINTER(Tuning), vp]
     lib.mamba_scan_fwd_complex.restype = ci
     dp = vp  # double *
+    lib.mamba_scan_fwd_conv.argtypes = [vp, fp, fp, i64, i64, vp, fp, vp, vp, fp, vp, i64, fp, fp, vp, fp, vp,
+                                        i64, i64, i64, i64, ci, vp, ctypes.c_size_t, vp]
+    lib.mamba_scan_fwd_conv.restype = ci
     lib.mamba_delta_sum.argtypes = [vp, fp, ci, dp, i64, i64, i64, ci, vp]
     lib.mamba_delta_sum.restype = ci
     lib.mamba_state_fold.argtypes = [fp, dp, fp, fp, fp, i64, i64, i64, i64, vp]
@@ -360,6 +363,80 @@ def mamba_scan_fwd_complex(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor
                                         _stream(dev))
     _check("mamba_scan_fwd_complex", rc)
     return (out, last_state) if want_state else out
+
+
+def _rows(t: Optional[torch.Tensor], name: str, device, dtype, batch: int, dim: int, L: int) -> int:
+    """Batch stride of a (batch, >= dim, L) tensor whose rows are dense."""
+    if t is None:
+        return 0
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if t.dim() != 3 or t.shape[0] != batch or t.shape[1] < dim or t.shape[2] != L:
+        raise ValueError(f"{name} must be (batch, >= {dim}, {L}), got {tuple(t.shape)}")
+    if t.stride(2) != 1 or (t.shape[1] > 1 and t.stride(1) != L):
+        raise ValueError(f"{name} rows must be dense (strides (*, L, 1))")
+    return int(t.stride(0)) if batch > 1 else int(t.shape[1]) * L
+
+
+def mamba_scan_fwd_conv(x: torch.Tensor, conv_weight: torch.Tensor, conv_bias: Optional[torch.Tensor],
+                        delta: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+                        D: Optional[torch.Tensor] = None, z: Optional[torch.Tensor] = None,
+                        delta_bias: Optional[torch.Tensor] = None, h0: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, last_state: Optional[torch.Tensor] = None,
+                        return_last_state: bool = False, return_u: bool = False,
+                        workspace: Optional[torch.Tensor] = None):
+    """Causal depthwise conv1d + silu fused into the scan (softplus on).
+
+    x: (batch, >= dim, L) -- the first ``dim`` channel rows are the conv
+    input (so the in-projection's (batch, 2 dim, L) output can be passed
+    whole); z: None or (batch, >= dim, L) likewise (e.g. ``xz[:, dim:]``);
+    dim = delta.shape[1].  conv_weight (dim, K <= 4), conv_bias (dim,) fp32.
+    Returns out, plus last_state and / or u when asked, in that order."""
+    if delta.dim() != 3:
+        raise ValueError("delta must be (batch, dim, seqlen)")
+    batch, dim, L = delta.shape
+    N = A.shape[1]
+    dev, act = delta.device, delta.dtype
+    if dev.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    if act not in _ACT:
+        raise TypeError(f"unsupported activation dtype {act}")
+    xbs = _rows(x, "x", dev, act, batch, dim, L)
+    zbs = _rows(z, "z", dev, act, batch, dim, L)
+    if conv_weight.dim() != 2 or conv_weight.shape[0] != dim:
+        raise ValueError("conv_weight must be (dim, width)")
+    K = conv_weight.shape[1]
+    _need(conv_weight, "conv_weight", dev, torch.float32, (dim, K))
+    _need(conv_bias, "conv_bias", dev, torch.float32, (dim,))
+    _need(delta, "delta", dev, act, (batch, dim, L))
+    _need(B, "B", dev, act, (batch, N, L))
+    _need(C, "C", dev, act, (batch, N, L))
+    _need(A, "A", dev, torch.float32, (dim, N))
+    _need(D, "D", dev, torch.float32, (dim,))
+    _need(delta_bias, "delta_bias", dev, torch.float32, (dim,))
+    _need(h0, "h0", dev, torch.float32, (batch, dim, N))
+    if out is None:
+        out = torch.empty_like(delta)
+    _need(out, "out", dev, act, (batch, dim, L))
+    want_state = return_last_state or last_state is not None
+    if want_state and last_state is None:
+        last_state = torch.empty((batch, dim, N), device=dev, dtype=torch.float32)
+    _need(last_state, "last_state", dev, torch.float32, (batch, dim, N))
+    u = torch.empty_like(delta) if return_u else None
+    lib = load_library()
+    if workspace is None:
+        workspace = torch.empty(max(1, lib.mamba_scan_workspace_size(batch, dim, L, N, _ACT[act])),
+                                device=dev, dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        rc = lib.mamba_scan_fwd_conv(_ptr(x), _ptr(conv_weight), _ptr(conv_bias), K, xbs, _ptr(delta), _ptr(A),
+                                     _ptr(B), _ptr(C), _ptr(D), _ptr(z), zbs, _ptr(delta_bias), _ptr(h0),
+                                     _ptr(out), _ptr(last_state), _ptr(u), batch, dim, L, N, _ACT[act],
+                                     _ptr(workspace), workspace.numel(), _stream(dev))
+    _check("mamba_scan_fwd_conv", rc)
+    res = (out,) + ((last_state,) if want_state else ()) + ((u,) if return_u else ())
+    return res[0] if len(res) == 1 else res
 
 
 def mamba_delta_sum(delta: torch.Tensor, delta_bias: Optional[torch.Tensor] = None,

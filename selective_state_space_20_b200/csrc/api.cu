@@ -340,6 +340,76 @@ int mamba_scan_fwd_complex(const void *u, const void *delta, const float *A, con
     return mscan::launch_scan_fwd_complex(a, lanes, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 
+int mamba_scan_fwd_conv(const void *x, const float *conv_weight, const float *conv_bias,
+                        int64_t conv_width, int64_t x_batch_stride, const void *delta,
+                        const float *A, const void *B, const void *C, const float *D, const void *z,
+                        int64_t z_batch_stride, const float *delta_bias, const float *h0, void *out,
+                        float *last_state, void *u_out, int64_t batch, int64_t dim, int64_t seqlen,
+                        int64_t dstate, int act_dtype, void *workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+    if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
+    int rc = check_sizes(batch, dim, seqlen, dstate);
+    if (rc != MAMBA_OK) return rc;
+    if (conv_width < 1 || conv_width > 4) return MAMBA_ERR_UNSUPPORTED;
+    if (!x || !conv_weight || !delta || !A || !B || !C || !out) return MAMBA_ERR_NULL;
+    const int64_t dense = dim * seqlen;
+    if (x_batch_stride == 0) x_batch_stride = dense;
+    if (z_batch_stride == 0) z_batch_stride = dense;
+    if (x_batch_stride < dense || z_batch_stride < dense) return MAMBA_ERR_SHAPE;
+    if ((double)batch * (double)x_batch_stride > (double)kMaxElems ||
+        (double)batch * (double)z_batch_stride > (double)kMaxElems)
+        return MAMBA_ERR_SHAPE;
+    const size_t es = act_size(act_dtype);
+    const int64_t V = 16 / (int64_t)es;
+    auto al = [](const void *q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+    // the fused prologue lives in the persistent lane-split kernel: its layout rules
+    if (dstate > 16 || seqlen % V != 0 || x_batch_stride % V != 0 || z_batch_stride % V != 0 ||
+        !al(x) || !al(delta) || !al(z) || !al(B) || !al(C) || !al(out) || !al(u_out))
+        return MAMBA_ERR_UNSUPPORTED;
+    const size_t nx = (size_t)(batch * dense) * es;
+    const size_t nxs = (size_t)((batch - 1) * x_batch_stride + dense) * es;
+    const size_t nzs = (size_t)((batch - 1) * z_batch_stride + dense) * es;
+    const size_t nbc = (size_t)(batch * dstate * seqlen) * es;
+    const size_t nA = (size_t)(dim * dstate) * 4, nd = (size_t)dim * 4;
+    const size_t nls = (size_t)(batch * dim * dstate) * 4, nw = (size_t)(dim * conv_width) * 4;
+    // outputs apart from every input and from each other (a worker reads the
+    // conv inputs just before its piece while another writes outputs)
+    const void *ins[] = {x, delta, z, B, C, A, D, delta_bias, conv_weight, conv_bias, h0};
+    const size_t insz[] = {nxs, nx, nzs, nbc, nbc, nA, nd, nd, nw, nd, nls};
+    void *outs[] = {out, u_out, last_state};
+    const size_t outsz[] = {nx, nx, nls};
+    for (int i = 0; i < 3; ++i) {
+        for (int k = 0; k < 11; ++k) {
+            if (i == 2 && k == 10 && h0 == last_state) continue;  // the state may advance in place
+            if (overlaps(outs[i], outsz[i], ins[k], insz[k])) return MAMBA_ERR_OVERLAP;
+        }
+        for (int k = 0; k < i; ++k)
+            if (overlaps(outs[i], outsz[i], outs[k], outsz[k])) return MAMBA_ERR_OVERLAP;
+    }
+    const size_t need = mscan::persistent_workspace_bound(batch, dim, seqlen, act_dtype);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15) != 0)
+        return MAMBA_ERR_WORKSPACE;
+    for (int k = 0; k < 11; ++k)
+        if (overlaps(workspace, workspace_bytes, ins[k], insz[k])) return MAMBA_ERR_OVERLAP;
+    for (int i = 0; i < 3; ++i)
+        if (overlaps(workspace, workspace_bytes, outs[i], outsz[i])) return MAMBA_ERR_OVERLAP;
+    int status = MAMBA_OK;
+    const int sms = current_sm_count(&status);
+    if (status != MAMBA_OK) return status;
+    mscan::ScanArgs a;
+    a.u = x; a.delta = delta; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.D = D; a.delta_bias = delta_bias; a.out = out; a.last_state = last_state; a.h0 = h0;
+    a.strides = nullptr;
+    a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = (int)dstate;
+    a.softplus = 1; a.act = act_dtype;
+    a.conv_w = conv_weight; a.conv_b = conv_bias; a.conv_k = (int)conv_width; a.u_out = u_out;
+    a.u_bstride = x_batch_stride; a.z_bstride = z_batch_stride;
+    int lanes = mscan::persistent_choose_lanes(a, sms);
+    if (lanes != 2 && lanes != 4) lanes = 2;  // the balanced split covers any shape
+    return mscan::launch_scan_fwd_persistent(a, lanes, 0, workspace, workspace_bytes, sms, stream) == cudaSuccess
+               ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
 int mamba_delta_sum(const void *delta, const float *delta_bias, int delta_softplus,
                     double *out, int64_t batch, int64_t dim, int64_t seqlen, int act_dtype,
                     cudaStream_t stream) {
@@ -622,6 +692,6 @@ const char *mamba_status_string(int status) {
     }
 }
 
-int mamba_abi_version(void) { return (1 << 16) | 6; }
+int mamba_abi_version(void) { return (1 << 16) | 7; }
 
 }  // extern "C"

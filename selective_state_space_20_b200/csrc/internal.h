@@ -26,6 +26,15 @@ struct ScanArgs {
     float *last_state;
     const float *h0;  // initial state (batch, dim, dstate) or null (zeros)
     const ScanStrides *strides;  // null: dense (batch, dim, L) / (batch, N, L), L contiguous
+    // fused causal conv1d prologue (persistent lane-split kernel only): when
+    // conv_w is set, u holds x, the conv input, and the kernel forms
+    // u = silu(conv_b + sum_k conv_w[k] x[t - (conv_k - 1) + k]) itself
+    const float *conv_w = nullptr;  // (dim, conv_k), conv_k <= 4
+    const float *conv_b = nullptr;  // (dim) or null
+    int conv_k = 0;
+    void *u_out = nullptr;          // (batch, dim, L) act or null: the u it formed
+    int64_t u_bstride = 0;          // batch stride of x when conv_w is set (elements); 0: dim * L
+    int64_t z_bstride = 0;          // batch stride of z when conv_w is set; 0: dim * L
     int64_t batch, dim, seqlen;
     int dstate;
     int softplus;

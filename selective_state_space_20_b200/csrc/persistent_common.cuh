@@ -33,6 +33,12 @@ struct Params {
     void *out;
     float *last_state;
     const float *h0;       // initial state (batch, dim, dstate) or null (zeros)
+    // fused conv1d prologue (lane-split kernel): u holds x; weights
+    // right-aligned to 4 taps on load; u_out optional; batch strides of x, z
+    const float *conv_w, *conv_b;
+    int conv_k;
+    void *u_out;
+    int64_t u_bstride, z_bstride;
     int64_t dim, seqlen;
     int dstate;
     int softplus;

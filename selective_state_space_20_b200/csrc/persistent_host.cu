@@ -143,6 +143,10 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
     kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
     kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias;
     kp.out = a.out; kp.last_state = a.last_state; kp.h0 = a.h0;
+    kp.conv_w = a.conv_w; kp.conv_b = a.conv_b; kp.conv_k = a.conv_k; kp.u_out = a.u_out;
+    kp.u_bstride = a.u_bstride > 0 ? a.u_bstride : a.dim * a.seqlen;
+    kp.z_bstride = a.z_bstride > 0 ? a.z_bstride : a.dim * a.seqlen;
+    if (a.conv_w && (lanes == 1 || !a.softplus)) return cudaErrorInvalidValue;  // lane-split kernel, softplus on
     kp.dim = a.dim; kp.seqlen = a.seqlen; kp.dstate = a.dstate; kp.softplus = a.softplus;
     kp.group_channels = group_channels(lanes);
     kp.groups_per_batch = (int)((a.dim + kp.group_channels - 1) / kp.group_channels);

@@ -137,7 +137,7 @@ template <int R> struct LanesOccupancy;
 template <> struct LanesOccupancy<2> { static constexpr int kBlocks = 2; };
 template <> struct LanesOccupancy<4> { static constexpr int kBlocks = 3; };
 
-template <typename T, int R, bool SP, bool GATE>
+template <typename T, int R, bool SP, bool GATE, bool CONV>
 __global__ void __launch_bounds__(kWarps * 32, LanesOccupancy<R>::kBlocks)
 scan_fwd_pairs_kernel(const Params p) {
     using W = PairSmem<T, R>;
@@ -168,6 +168,7 @@ scan_fwd_pairs_kernel(const Params p) {
     int cur_group = -1;
     float2 A2[S / 2];
     float bias_p = 0.f, D_s = 0.f;
+    float cw[4] = {0.f, 0.f, 0.f, 0.f}, cb_p = 0.f;  // CONV: the prologue channel's conv taps and bias
 
     // This worker's share of the balanced split: head, whole groups, tail.
     // Piece: sub-chunks [sb, se) of group g, carried state in from sub-chunk
@@ -206,6 +207,13 @@ scan_fwd_pairs_kernel(const Params p) {
             }
             bias_p = (dp < Dm && p.delta_bias) ? __ldg(p.delta_bias + dp) : 0.f;
             D_s = (ds < Dm && p.D) ? __ldg(p.D + ds) : 0.f;
+            if (CONV) {  // taps right-aligned to 4: a shorter kernel sees zeros before it
+                const int K = p.conv_k;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    cw[j] = (dp < Dm && j >= 4 - K) ? __ldg(p.conv_w + dp * K + (j - (4 - K))) : 0.f;
+                cb_p = (dp < Dm && p.conv_b) ? __ldg(p.conv_b + dp) : 0.f;
+            }
         }
 
         float *carry = p.carry + ((int64_t)g * 32 + lane) * S;
@@ -232,13 +240,15 @@ scan_fwd_pairs_kernel(const Params p) {
         // this lane's 16-byte copies: chunk cx of rows (lane + 32 i) / CPR
         constexpr int NX = (CW * CPR + 31) / 32, NB = 2 * kNS * CPR / 32;
         const int cx = lane % CPR;
-        int64_t xoff[NX], boff[NB];
+        int64_t xoff[NX], boff[NB], uoff[NX], zoff[NX];
         bool xok[NX], bok[NB];
 #pragma unroll
         for (int i = 0; i < NX; ++i) {
             const int r = (lane + 32 * i) / CPR;
             xok[i] = lane + 32 * i < CW * CPR && r < nrows;
             xoff[i] = row0 + r * L + cx * V;
+            uoff[i] = CONV ? b * p.u_bstride + (d0 + r) * L + cx * V : xoff[i];
+            zoff[i] = CONV ? b * p.z_bstride + (d0 + r) * L + cx * V : xoff[i];
         }
 #pragma unroll
         for (int i = 0; i < NB; ++i) {
@@ -257,9 +267,9 @@ scan_fwd_pairs_kernel(const Params p) {
                 if (lane + 32 * i < CW * CPR) {
                     const bool ok = xok[i] && tok;
                     const int64_t off = ok ? xoff[i] + t0 : 0;
-                    cp16(sbuf + (0 * CW + r) * W::ROWB, gu + off, ok);
+                    cp16(sbuf + (0 * CW + r) * W::ROWB, gu + (ok ? uoff[i] + t0 : 0), ok);
                     cp16(sbuf + (1 * CW + r) * W::ROWB, gd + off, ok);
-                    if (GATE && !so_stage) cp16(sbuf + (2 * CW + r) * W::ROWB, gz + off, ok);
+                    if (GATE && !so_stage) cp16(sbuf + (2 * CW + r) * W::ROWB, gz + (ok ? zoff[i] + t0 : 0), ok);
                 }
             }
 #pragma unroll
@@ -279,6 +289,16 @@ scan_fwd_pairs_kernel(const Params p) {
         auto run_subs = [&](const bool SO, float2 (&h)[S / 2], double &dsum, bool publish_end) {
         so_stage = SO;
         issue(0, 0);
+        if (CONV && ph == 0) {
+            // the conv inputs before sub-chunk 0 (zeros before the sequence),
+            // kept in the padding of the channel's x row of stage 0
+            T *halo = reinterpret_cast<T *>(base + (0 * CW + pc) * W::ROWB + kTC * sizeof(T));
+#pragma unroll
+            for (int k = 0; k < 3; ++k) {
+                const int64_t t = tb0 - 3 + k;
+                halo[k] = (t >= 0 && pc < nrows) ? gu[b * p.u_bstride + (d0 + pc) * L + t] : T(0.f);
+            }
+        }
 #pragma unroll 1
         for (int sub = 0; sub < nsub; ++sub) {
             const int st = sub & 1;
@@ -293,6 +313,40 @@ scan_fwd_pairs_kernel(const Params p) {
             const int64_t t0 = tb0 + (int64_t)sub * kTC;
             const int tvalid = (L - t0) < kTC ? (int)(L - t0) : kTC;
 
+            // ---- prologue (0), fused conv1d: this lane's PT inputs of its
+            // channel and the 3 before them (from the row, or from the
+            // padding where the previous sub-chunk left its last 3) become
+            // u = silu(conv_b + sum_k w_k x), rounded to the activation type
+            // and written over the inputs, so everything below reads u
+            if (CONV) {
+                unsigned char *urw = base + st * W::STAGE + (0 * CW + pc) * W::ROWB;
+                float xs[PT + 3];
+#pragma unroll
+                for (int k = 0; k < 3; ++k)
+                    xs[k] = Elem<T>::to_f(ph == 0 ? reinterpret_cast<const T *>(urw + kTC * sizeof(T))[k]
+                                                  : reinterpret_cast<const T *>(urw)[ph * PT - 3 + k]);
+#pragma unroll
+                for (int v = 0; v < PT; v += V)
+                    Elem<T>::unpack(*reinterpret_cast<const uint4 *>(urw + (ph * PT + v) * sizeof(T)), xs + 3 + v);
+                __syncwarp();  // every lane holds its inputs before any u is written over them
+                if (ph == R - 1) {  // the next sub-chunk's 3 inputs before it
+                    T *nh = reinterpret_cast<T *>(base + (st ^ 1) * W::STAGE + (0 * CW + pc) * W::ROWB + kTC * sizeof(T));
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) Elem<T>::store(nh + k, xs[PT + k]);
+                }
+#pragma unroll
+                for (int v = 0; v < PT; v += V) {
+                    float uo[V];
+#pragma unroll
+                    for (int e = 0; e < V; ++e) {
+                        float acc = cb_p;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) acc = fmaf(cw[k], xs[v + e + k], acc);
+                        uo[e] = silu_f(acc);
+                    }
+                    *reinterpret_cast<uint4 *>(urw + (ph * PT + v) * sizeof(T)) = Elem<T>::pack(uo);
+                }
+            }
             // ---- prologue (a): B and C to fp32 [t][n].  Lane (which, q, c)
             // reads states 4q .. 4q+3 of B (which 0) or C (which 1) in chunk c
             // and writes them back as one 16-byte [t][4q .. 4q+3] piece per
@@ -334,6 +388,16 @@ scan_fwd_pairs_kernel(const Params p) {
                 }
             }
             __syncwarp();
+            if (CONV && !SO && p.u_out) {  // the u it formed, for a backward pass
+                T *gu_out = static_cast<T *>(p.u_out);
+#pragma unroll
+                for (int i = lane; i < CW * CPR; i += 32) {
+                    const int r = i / CPR, c = i % CPR;
+                    const int64_t t = t0 + c * V;
+                    if (r < nrows && t < L)
+                        stg16_stream(gu_out + row0 + r * L + t, *reinterpret_cast<const uint4 *>(sbuf + (0 * CW + r) * W::ROWB + c * 16));
+                }
+            }
 
             // ---- scan: lane (sc, sr), blocks of 8 timesteps
             {
@@ -498,10 +562,10 @@ scan_fwd_pairs_kernel(const Params p) {
     }
 }
 
-template <typename T, int R, bool SP, bool GATE>
+template <typename T, int R, bool SP, bool GATE, bool CONV = false>
 cudaError_t launch_t(const Params &kp, int sm_count, cudaStream_t st) {
     const int smem = kWarps * PairSmem<T, R>::BYTES;
-    auto kern = scan_fwd_pairs_kernel<T, R, SP, GATE>;
+    auto kern = scan_fwd_pairs_kernel<T, R, SP, GATE, CONV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     static const int per_sm = [&] {
@@ -527,6 +591,12 @@ cudaError_t launch_t(const Params &kp, int sm_count, cudaStream_t st) {
 template <int R>
 cudaError_t launch_r(const Params &kp, int act, int sm_count, cudaStream_t st) {
     const bool gate = kp.z != nullptr;
+    if (kp.conv_w) {  // fused conv1d prologue: softplus on (checked by the caller)
+        if (act == kBF16) return gate ? launch_t<__nv_bfloat16, R, true, true, true>(kp, sm_count, st)
+                                      : launch_t<__nv_bfloat16, R, true, false, true>(kp, sm_count, st);
+        return gate ? launch_t<float, R, true, true, true>(kp, sm_count, st)
+                    : launch_t<float, R, true, false, true>(kp, sm_count, st);
+    }
     if (act == kBF16) {
         if (kp.softplus) return gate ? launch_t<__nv_bfloat16, R, true, true>(kp, sm_count, st)
                                      : launch_t<__nv_bfloat16, R, true, false>(kp, sm_count, st);

@@ -214,3 +214,20 @@ def test_sequence_split_validation(lib):
                                 2, 4, 16, 2, None) == -7
     assert lib.mamba_state_fold(None, vp(0x200000), vp(0x300000), vp(0x400000), vp(0x400000 + ns + 16),
                                 2, 4, 16, 2, None) == -7
+
+
+def test_fused_conv_scan_validation(lib):
+    vp = ctypes.c_void_p
+    P = [vp(0x100000 * (i + 1)) for i in range(16)]
+
+    def call(x=P[0], width=4, xbs=0, ws=P[12], wsb=1 << 20, dstate=16, L=64, out=P[8], z=None, zbs=0):
+        return lib.mamba_scan_fwd_conv(x, P[1], None, width, xbs, P[2], P[3], P[4], P[5], None, z, zbs, None,
+                                       None, out, None, None, 2, 8, L, dstate, 1, ws, wsb, None)
+    assert call(x=None) == -1
+    assert call(width=5) == -3 and call(width=0) == -3
+    assert call(dstate=32) == -3              # the lane-split kernel holds 16 states
+    assert call(L=60) == -3                   # whole 16-byte chunks of timesteps
+    assert call(x=vp(0x100000 + 2)) == -3     # 16-byte alignment
+    assert call(xbs=8 * 64 - 8) == -2         # rows would overlap
+    assert call(out=vp(0x100000 + 64)) == -7  # out over x
+    assert call(ws=None) == -8 and call(wsb=16) == -8
