@@ -421,10 +421,47 @@ def conv1d_measure(reps=20):
     es = 2 if w.dtype == "bf16" else 4
     nbytes = 2 * w.batch * w.dim * w.seqlen * es + w.dim * (K + 1) * 4
     hbm = load_peaks()["hbm_gbs"]
+
+    # the same conv fused into the scan's prologue (x and z read from the
+    # projection output), against the conv kernel followed by the scan
+    s = inputs.scan_inputs(w, device="cuda")
+    xz = d["xz"]
+    xz[:, w.dim:] = s["z"]
+    z = xz[:, w.dim:]
+    ws = torch.empty(binding.mamba_scan_workspace_size(w.batch, w.dim, w.seqlen, w.dstate), device="cuda",
+                     dtype=torch.uint8)
+    y = torch.empty_like(out)
+    last = torch.empty(w.batch, w.dim, w.dstate, device="cuda")
+
+    def fused():
+        binding.mamba_scan_fwd_conv(xz, d["weight"], d["bias"], s["delta"], s["A"], s["B"], s["C"], D=s["D"],
+                                    z=z, delta_bias=s["delta_bias"], out=y, last_state=last, workspace=ws)
+
+    def separate():
+        binding.mamba_conv1d_fwd(xz, d["weight"], d["bias"], dim=w.dim, out=out)
+        binding.mamba_scan_fwd(out, s["delta"], s["A"], s["B"], s["C"], D=s["D"], z=s["z"],
+                               delta_bias=s["delta_bias"], out=y, last_state=last, workspace=ws)
+
+    def time_us(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        c.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(c) * 1e3 / reps
+
+    us_fused, us_sep = time_us(fused), time_us(separate)
     return {"workload": f"conv1d K={K} {w.batch}x{w.dim}x{w.seqlen} {w.dtype} (x half of a 2x-wide input)",
             "us_per_call": us, "Gelem_per_s": w.elements / us / 1e3,
             "roofline": {"bound": "hbm", "achieved": nbytes / us / 1e3, "peak": hbm, "unit": "GB/s",
                          "frac": nbytes / us / 1e3 / hbm, "algorithmic_bytes": nbytes},
+            "fused_with_scan": {"us_per_call": us_fused, "Gelem_per_s": w.elements / us_fused / 1e3,
+                                "separate_conv_then_scan_us": us_sep,
+                                "note": "mamba_scan_fwd_conv: u formed in the scan's prologue, never stored"},
             "reps": reps, "l2": "inputs larger than L2, no flush"}
 
 
