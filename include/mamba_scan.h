@@ -286,6 +286,39 @@ int mamba_scan_fwd_complex(const void *u, const void *delta, const float *A,
                            cudaStream_t stream);
 
 /*
+ * mamba_scan_fwd_host -- mamba_scan_fwd_init for sequences in HOST memory:
+ * the scan of a model whose activations do not stay on the GPU, or of a
+ * problem larger than the device.  The (batch, channel) rows are cut into
+ * chunks (channel ranges of one batch row); for each chunk the inputs are
+ * copied host -> device on an internal stream, the scan runs on `stream`,
+ * and the outputs are copied back on a second internal stream, through two
+ * device slots, so both copy directions and the scans overlap.
+ *
+ *   u, delta, z, B, C : HOST, layouts of mamba_scan_fwd (z may be NULL).
+ *                  Page-locked (pinned) memory lets the copies run
+ *                  asynchronously; pageable memory works but serialises them.
+ *   out          : HOST act (batch, dim, seqlen), written.
+ *   last_state   : HOST fp32 (batch, dim, dstate) or NULL.
+ *   A, D, delta_bias, h0 : DEVICE, as for mamba_scan_fwd_init (h0 may be NULL).
+ *   scratch      : DEVICE, at least mamba_scan_host_scratch_size bytes,
+ *                  16-byte aligned, caller-owned; must not overlap A, D,
+ *                  delta_bias or h0.
+ *
+ * Stream-ordered like the other entry points: the copies start after the
+ * work already queued on `stream`, and `stream` waits for the last copy
+ * back; host buffers must stay valid (and out unread) until then.  Returns
+ * MAMBA_OK or a mamba_status_t error (MAMBA_ERR_WORKSPACE for a missing or
+ * small scratch; an error of a chunk's scan is returned as is).
+ */
+size_t mamba_scan_host_scratch_size(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                                    int act_dtype);
+int mamba_scan_fwd_host(const void *u, const void *delta, const float *A, const void *B,
+                        const void *C, const float *D, const void *z, const float *delta_bias,
+                        int delta_softplus, const float *h0, void *out, float *last_state,
+                        int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
+                        void *scratch, size_t scratch_bytes, cudaStream_t stream);
+
+/*
  * mamba_scan_fwd_conv -- the causal depthwise conv1d + silu fused into the
  * scan's prologue: the step before the scan in the Mamba block ("Mamba SSM
  * concept and implementation in Keras and TensorFlow", MambaBlock: Conv1D

@@ -31,7 +31,8 @@ SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT = 0, 1, 2
 EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
             "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_fwd_strided",
-            "mamba_scan_fwd_complex", "mamba_delta_sum", "mamba_state_fold", "mamba_scan_fwd_conv", "mamba_scan_bwd", "mamba_scan_bwd_init",
+            "mamba_scan_fwd_complex", "mamba_delta_sum", "mamba_state_fold", "mamba_scan_fwd_conv",
+            "mamba_scan_host_scratch_size", "mamba_scan_fwd_host", "mamba_scan_bwd", "mamba_scan_bwd_init",
             "mamba_scan_bwd_workspace_size",
             "mamba_state_update", "mamba_conv1d_fwd",
             "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version")
@@ -83,6 +84,10 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_fwd_conv.argtypes = [vp, fp, fp, i64, i64, vp, fp, vp, vp, fp, vp, i64, fp, fp, vp, fp, vp,
                                         i64, i64, i64, i64, ci, vp, ctypes.c_size_t, vp]
     lib.mamba_scan_fwd_conv.restype = ci
+    lib.mamba_scan_host_scratch_size.argtypes = [i64, i64, i64, i64, ci]
+    lib.mamba_scan_host_scratch_size.restype = ctypes.c_size_t
+    lib.mamba_scan_fwd_host.argtypes = scan_args[:9] + [fp] + scan_args[9:] + [vp, ctypes.c_size_t, vp]
+    lib.mamba_scan_fwd_host.restype = ci
     lib.mamba_delta_sum.argtypes = [vp, fp, ci, dp, i64, i64, i64, ci, vp]
     lib.mamba_delta_sum.restype = ci
     lib.mamba_state_fold.argtypes = [fp, dp, fp, fp, fp, i64, i64, i64, i64, vp]
@@ -437,6 +442,54 @@ def mamba_scan_fwd_conv(x: torch.Tensor, conv_weight: torch.Tensor, conv_bias: O
     _check("mamba_scan_fwd_conv", rc)
     res = (out,) + ((last_state,) if want_state else ()) + ((u,) if return_u else ())
     return res[0] if len(res) == 1 else res
+
+
+def mamba_scan_fwd_host(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                        C: torch.Tensor, D: Optional[torch.Tensor] = None, z: Optional[torch.Tensor] = None,
+                        delta_bias: Optional[torch.Tensor] = None, delta_softplus: bool = True,
+                        h0: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                        last_state: Optional[torch.Tensor] = None, return_last_state: bool = False,
+                        scratch: Optional[torch.Tensor] = None):
+    """The scan on sequences in host memory (ideally pinned): u, delta, z, B,
+    C on the CPU; A, D, delta_bias (and h0) on the GPU.  Returns host
+    ``out`` (and host ``last_state``).  Runs on the current stream of A's
+    device; the results are ready once that stream has reached this point."""
+    if u.dim() != 3:
+        raise ValueError("u must be (batch, dim, seqlen)")
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    dev, act = A.device, u.dtype
+    if dev.type != "cuda":
+        raise ValueError("A, D, delta_bias must be on a CUDA device")
+    if act not in _ACT:
+        raise TypeError(f"unsupported activation dtype {act}")
+    cpu = torch.device("cpu")
+    for name, t in (("u", u), ("delta", delta), ("z", z)):
+        _need(t, name, cpu, act, (batch, dim, L))
+    _need(B, "B", cpu, act, (batch, N, L))
+    _need(C, "C", cpu, act, (batch, N, L))
+    _need(A, "A", dev, torch.float32, (dim, N))
+    _need(D, "D", dev, torch.float32, (dim,))
+    _need(delta_bias, "delta_bias", dev, torch.float32, (dim,))
+    _need(h0, "h0", dev, torch.float32, (batch, dim, N))
+    if out is None:
+        out = torch.empty((batch, dim, L), dtype=act, pin_memory=u.is_pinned())
+    _need(out, "out", cpu, act, (batch, dim, L))
+    want_state = return_last_state or last_state is not None
+    if want_state and last_state is None:
+        last_state = torch.empty((batch, dim, N), dtype=torch.float32, pin_memory=u.is_pinned())
+    _need(last_state, "last_state", cpu, torch.float32, (batch, dim, N))
+    lib = load_library()
+    if scratch is None:
+        scratch = torch.empty(lib.mamba_scan_host_scratch_size(batch, dim, L, N, _ACT[act]), device=dev,
+                              dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        rc = lib.mamba_scan_fwd_host(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                                     _ptr(delta_bias), int(bool(delta_softplus)), _ptr(h0), _ptr(out),
+                                     _ptr(last_state), batch, dim, L, N, _ACT[act], _ptr(scratch),
+                                     scratch.numel(), _stream(dev))
+    _check("mamba_scan_fwd_host", rc)
+    return (out, last_state) if want_state else out
 
 
 def mamba_delta_sum(delta: torch.Tensor, delta_bias: Optional[torch.Tensor] = None,

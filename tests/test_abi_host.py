@@ -231,3 +231,19 @@ def test_fused_conv_scan_validation(lib):
     assert call(xbs=8 * 64 - 8) == -2         # rows would overlap
     assert call(out=vp(0x100000 + 64)) == -7  # out over x
     assert call(ws=None) == -8 and call(wsb=16) == -8
+
+
+def test_host_memory_scan_validation(lib):
+    vp = ctypes.c_void_p
+    need = lib.mamba_scan_host_scratch_size(4, 5120, 4096, 16, 1)
+    assert need > 0 and lib.mamba_scan_host_scratch_size(0, 8, 8, 16, 1) == 0
+    args = [vp(0x100000), vp(0x200000), vp(0x300000), vp(0x400000), vp(0x500000), None, None, None, 1, None,
+            vp(0x600000), None, 2, 4, 64, 16, 1]
+    assert lib.mamba_scan_fwd_host(*args, None, 0, None) == -8                      # no scratch
+    assert lib.mamba_scan_fwd_host(*args, vp(0x1000000), 16, None) == -8            # too small
+    bad = list(args)
+    bad[0] = None
+    assert lib.mamba_scan_fwd_host(*bad, vp(0x1000000), 1 << 30, None) == -1
+    bad = list(args)
+    bad[15] = 65
+    assert lib.mamba_scan_fwd_host(*bad, vp(0x1000000), 1 << 30, None) == -3
