@@ -52,22 +52,19 @@ def test_host_scan_from_a_state_without_gate():
     assert rel_err(to_np(out), ro) <= 2e-2 and rel_err(to_np(last), rs) <= 2e-2
 
 
-def test_host_scan_benchmark_layer_equals_device_scan_rows():
-    """The Mamba-2.8B layer from pinned host memory: every row equal to the
-    device scan of the same chunk layout (a batch row's channel range runs
-    as its own problem, so it is compared with the device scan of that
-    range)."""
+def test_host_scan_benchmark_layer_matches_device_scan():
+    """The Mamba-2.8B layer from pinned host memory against the device scan
+    of the whole problem (the chunks run as their own problems, so lane
+    splits, and with them summation orders, may differ: compared within the
+    bf16 tolerance)."""
     wl = inputs.MAMBA_2_8B
     dev = inputs.scan_inputs(wl, device="cuda")
     h = {k: dev[k].cpu().pin_memory() for k in ("u", "delta", "z", "B", "C")}
     out, last = binding.mamba_scan_fwd_host(h["u"], h["delta"], dev["A"], h["B"], h["C"], D=dev["D"], z=h["z"],
                                             delta_bias=dev["delta_bias"], return_last_state=True)
+    o2, s2 = binding.mamba_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"],
+                                    delta_bias=dev["delta_bias"], return_last_state=True)
     torch.cuda.current_stream().synchronize()
-    # batch row 1, channels 2560 .. 5119 (the second chunk of that row)
-    b, d0, d1 = 1, 2560, 5120
-    sub = lambda t: t[b:b + 1, d0:d1].contiguous()  # noqa: E731
-    o2, s2 = binding.mamba_scan_fwd(sub(dev["u"]), sub(dev["delta"]), dev["A"][d0:d1].contiguous(),
-                                    dev["B"][b:b + 1].contiguous(), dev["C"][b:b + 1].contiguous(),
-                                    D=dev["D"][d0:d1].contiguous(), z=sub(dev["z"]),
-                                    delta_bias=dev["delta_bias"][d0:d1].contiguous(), return_last_state=True)
-    assert torch.equal(out[b:b + 1, d0:d1], o2.cpu()) and torch.equal(last[b:b + 1, d0:d1], s2.cpu())
+    e1, e2 = rel_err(to_np(out), to_np(o2)), rel_err(to_np(last), to_np(s2))
+    record("host-memory scan mamba-2.8b vs device scan", out=e1, state=e2)
+    assert e1 <= 2e-2 and e2 <= 1e-4, (e1, e2)
