@@ -297,3 +297,62 @@ def test_scan_then_steps_continue_the_sequence():
     assert rel_err(to_np(tail), ro[..., L1:]) <= 2e-2
     assert rel_err(to_np(state), rs) <= 2e-2
     assert rel_err(to_np(tail), to_np(full[..., L1:])) <= 2e-2
+
+
+def test_past_32_bit_indexing():
+    """4 x 5120 x 131072 bf16: 2.7 G elements per tensor, past 2^31, so every
+    row offset of the lane-split kernel needs 64-bit arithmetic; sampled rows
+    at both ends of the address range against the oracle."""
+    w = inputs.custom(4, 5120, 131072, 16, "bf16", seed=61, name="4x5120x131072 bf16")
+    assert w.batch * w.dim * w.seqlen > 2 ** 31
+    dev = inputs.scan_inputs(w, device="cuda")
+    out, last = run_scan(dev)
+    torch.cuda.synchronize()
+    rows = [0, 1, 5119, 5120 * 2 + 77, 5120 * 3, 5120 * 4 - 1]
+    cpu = {k: (None if v is None else v) for k, v in dev.items()}
+    ro, rs = oracle_rows(cpu, rows)
+    flat_out = out.view(w.batch * w.dim, w.seqlen)
+    flat_st = last.view(w.batch * w.dim, w.dstate)
+    idx = torch.tensor(rows, device=out.device)
+    e_out = rel_err(to_np(flat_out.index_select(0, idx)), ro)
+    e_state = rel_err(to_np(flat_st.index_select(0, idx)), rs)
+    record("4x5120x131072 bf16 sampled rows", out=e_out, state=e_state)
+    assert e_out <= TOL[torch.bfloat16] and e_state <= TOL[torch.bfloat16]
+
+
+@pytest.mark.parametrize("sched", [binding.SCHEDULE_STATIC, binding.SCHEDULE_PERSISTENT])
+def test_zero_step_keeps_the_state(sched):
+    """delta = 0 (softplus off, no bias): Abar = 1 and no input, so the state
+    stays h0 bit for bit and y_t = C_t . h0 + D u_t (the oracle's pin, on
+    the GPU)."""
+    w = inputs.custom(2, 48, 256, 16, "fp32", seed=62)
+    cpu = inputs.scan_inputs(w)
+    cpu["delta"] = torch.zeros_like(cpu["delta"])
+    cpu["delta_bias"] = None
+    cpu["z"] = None
+    dev = dev_inputs(cpu)
+    h0 = inputs.initial_state(2, 48, 16, seed=5)
+    out, last = binding.mamba_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],
+                                       delta_softplus=False, return_last_state=True, h0=h0.cuda(), schedule=sched)
+    torch.cuda.synchronize()
+    assert torch.equal(last.cpu(), h0)
+    y = torch.einsum("bdn,bnl->bdl", h0.double(), cpu["C"].double()) + cpu["D"].double()[None, :, None] * cpu["u"].double()
+    assert rel_err(to_np(out), y.numpy()) <= 1e-5
+
+
+def test_memoryless_limit():
+    """A very negative: Abar underflows to 0 and h_t = delta_t B_t u_t, so
+    y_t = delta_t u_t (C_t . B_t) + D u_t -- a closed form without the
+    recurrence."""
+    w = inputs.custom(2, 40, 200, 16, "fp32", seed=63)
+    cpu = inputs.scan_inputs(w)
+    cpu["A"] = torch.full_like(cpu["A"], -1e7)  # delta A log2 e < -126 for every delta
+    cpu["z"] = None
+    dev = dev_inputs(cpu)
+    out, last = binding.mamba_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],
+                                       delta_bias=dev["delta_bias"], return_last_state=True)
+    torch.cuda.synchronize()
+    dl = torch.nn.functional.softplus(cpu["delta"].double() + cpu["delta_bias"].double()[None, :, None])
+    cb = (cpu["C"].double() * cpu["B"].double()).sum(1)  # (batch, L)
+    y = dl * cpu["u"].double() * cb[:, None, :] + cpu["D"].double()[None, :, None] * cpu["u"].double()
+    assert rel_err(to_np(out), y.numpy()) <= 1e-4
