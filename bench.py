@@ -230,6 +230,36 @@ def oracle_sample(w, seconds: float):
     return inputs.scan_inputs(dataclasses.replace(w, dim=k)), k
 
 
+def oracle_beside(kind: str, w, k: int = 32):
+    """The fp64 oracle of one section timed on this host's cores on a fixed
+    sample (every batch row, the first k channels, full L), for the section's
+    line: Gelem/s as the section counts elements."""
+    import oracle
+    cores = os.cpu_count() or 1
+    sw = dataclasses.replace(w, dim=min(k, w.dim))
+    elems = sw.batch * sw.dim * sw.seqlen
+    if kind == "backward":
+        d = inputs.scan_inputs(sw)
+        g = torch.Generator().manual_seed(7)
+        dout = torch.randn(sw.batch, sw.dim, sw.seqlen, generator=g)
+        t0 = time.perf_counter()
+        oracle.scan_bwd(dout, d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                        delta_bias=d["delta_bias"], nthreads=cores)
+    elif kind == "complex":
+        d = inputs.complex_inputs(sw.batch, sw.dim, sw.seqlen, sw.dstate, sw.dtype)
+        t0 = time.perf_counter()
+        oracle.scan_complex(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                            delta_bias=d["delta_bias"], nthreads=cores)
+    else:  # conv1d
+        d = inputs.conv_inputs(sw.batch, sw.dim, sw.seqlen, 4, sw.dtype, wide=False)
+        t0 = time.perf_counter()
+        oracle.conv1d(d["x"], d["weight"], d["bias"])
+    dt = time.perf_counter() - t0
+    return {"value": elems / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"all {sw.batch} batch rows, first {sw.dim} channels, full L={sw.seqlen}: "
+                      f"{elems} elements in {dt:.2f} s"}
+
+
 def cpu_baseline(w, seconds=25.0):
     cores = os.cpu_count() or 1
     data, k = oracle_sample(w, seconds)
@@ -642,6 +672,10 @@ def main():
         line["backward"] = backward_measure()
     if rank == 0 and not args.no_complex:
         line["complex"] = complex_measure()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        for key, kind in (("conv1d", "conv1d"), ("backward", "backward"), ("complex", "complex")):
+            if key in line:
+                line[key]["cpu_oracle"] = oracle_beside(kind, w, k={"conv1d": 1024}.get(kind, 256))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
