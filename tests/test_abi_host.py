@@ -36,6 +36,41 @@ def test_library_exports_every_declared_symbol(lib):
         assert re.search(rf"\bT {name}\b", out), f"{name} missing from dynamic symbol table"
 
 
+def _prototypes():
+    """{name: [parameter type strings]} parsed from the header."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = {}
+    for m in re.finditer(r"^\s*(?:const\s+)?\w+\s*\*?\s*(mamba_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.M | re.S):
+        params = [p.strip() for p in m.group(2).replace("\n", " ").split(",")]
+        protos[m.group(1)] = [] if params == ["void"] else params
+    return protos
+
+
+def test_binding_argtypes_match_the_header(lib):
+    """Every declared function has ctypes argtypes of the header's arity and
+    kind: pointers as void pointers (the binding passes c_void_p for every
+    buffer), int64_t, int, size_t and the stream as a pointer."""
+    import ctypes as C
+    protos = _prototypes()
+    assert sorted(protos) == sorted(binding.EXPORTED)
+    for name, params in protos.items():
+        fn = getattr(lib, name)
+        types = fn.argtypes or []
+        assert len(types) == len(params), (name, len(types), len(params))
+        for p, t in zip(params, types):
+            if "*" in p or p.startswith("cudaStream_t"):
+                want = (C.c_void_p, C.POINTER(binding.Tuning), C.POINTER(binding.ScanStrides))
+                assert t in want, (name, p, t)
+            elif p.startswith("int64_t"):
+                assert t is C.c_int64, (name, p, t)
+            elif p.startswith("size_t"):
+                assert t is C.c_size_t, (name, p, t)
+            elif p.startswith("int "):
+                assert t is C.c_int, (name, p, t)
+            else:
+                raise AssertionError((name, p))
+
+
 def test_library_is_built_for_sm100a_only():
     assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
 
