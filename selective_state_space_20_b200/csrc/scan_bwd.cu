@@ -233,7 +233,9 @@ __global__ void __launch_bounds__(kWarpsBwd * 32, 5) scan_bwd_kernel(const BwdPa
         };
         // h <- the states after `tn` steps of the staged segment; into hist[1..] when asked
         auto advance = [&](float (&h)[kSPL], int tn, bool keep) {
-            for (int s = 0; s < tn; ++s) {
+#pragma unroll
+            for (int s = 0; s < kSeg; ++s) {
+                if (s >= tn) break;
                 const float dl = sx[(X_DL * kSeg + s) * kCPW + c];
                 const float du = dl * sx[(X_U * kSeg + s) * kCPW + c];
                 const float4 bb = *reinterpret_cast<const float4 *>(sB + s * kNS + kSPL * r);
