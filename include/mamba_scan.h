@@ -399,6 +399,16 @@ int mamba_state_fold(const float *h_init, const double *delta_sums, const float 
                      const float *h_local, float *h_out, int64_t batch, int64_t dim,
                      int64_t dstate, int64_t count, cudaStream_t stream);
 
+/* Test hook for the failure-detection path: from the next launch on, the
+ * persistent lane-split kernel's pieces of channel group `group` no longer
+ * publish their carried state, so the piece after them waits until its time
+ * limit (2 s) runs out, raises the workspace's error word and stops, and the
+ * other pieces of the group stop on the error word; every other group
+ * completes.  mamba_scan_workspace_status then reports MAMBA_ERR_TIMEOUT.
+ * No wait is unbounded and nothing faults.  group < 0 turns the hook off
+ * (the default).  Process-wide; returns the previous setting. */
+int mamba_debug_stall_group(int group);
+
 /* Synchronises `stream`, then reads the status a persistent launch left in
  * `workspace`: MAMBA_OK, or MAMBA_ERR_TIMEOUT if a worker stopped waiting for
  * a predecessor chunk (the outputs of that launch are then incomplete).

@@ -25,6 +25,7 @@ STATUS_NAMES = {0: "MAMBA_OK", -1: "MAMBA_ERR_NULL", -2: "MAMBA_ERR_SHAPE",
                 -3: "MAMBA_ERR_UNSUPPORTED", -4: "MAMBA_ERR_ALIGN",
                 -5: "MAMBA_ERR_CUDA", -6: "MAMBA_ERR_DEVICE", -7: "MAMBA_ERR_OVERLAP",
                 -8: "MAMBA_ERR_WORKSPACE", -9: "MAMBA_ERR_TIMEOUT"}
+MAMBA_ERR_TIMEOUT = -9
 SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT = 0, 1, 2
 
 # Every function include/mamba_scan.h declares.
@@ -32,7 +33,7 @@ EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
             "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_fwd_strided",
             "mamba_scan_fwd_complex", "mamba_delta_sum", "mamba_state_fold", "mamba_scan_fwd_conv",
-            "mamba_scan_host_scratch_size", "mamba_scan_fwd_host", "mamba_scan_bwd", "mamba_scan_bwd_init",
+            "mamba_scan_host_scratch_size", "mamba_scan_fwd_host", "mamba_debug_stall_group", "mamba_scan_bwd", "mamba_scan_bwd_init",
             "mamba_scan_bwd_workspace_size",
             "mamba_state_update", "mamba_conv1d_fwd",
             "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version")
@@ -84,6 +85,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_fwd_conv.argtypes = [vp, fp, fp, i64, i64, vp, fp, vp, vp, fp, vp, i64, fp, fp, vp, fp, vp,
                                         i64, i64, i64, i64, ci, vp, ctypes.c_size_t, vp]
     lib.mamba_scan_fwd_conv.restype = ci
+    lib.mamba_debug_stall_group.argtypes = [ci]
+    lib.mamba_debug_stall_group.restype = ci
     lib.mamba_scan_host_scratch_size.argtypes = [i64, i64, i64, i64, ci]
     lib.mamba_scan_host_scratch_size.restype = ctypes.c_size_t
     lib.mamba_scan_fwd_host.argtypes = scan_args[:9] + [fp] + scan_args[9:] + [vp, ctypes.c_size_t, vp]

@@ -692,6 +692,8 @@ const char *mamba_status_string(int status) {
     }
 }
 
-int mamba_abi_version(void) { return (1 << 16) | 7; }
+int mamba_debug_stall_group(int group) { return mscan::set_stall_group(group < 0 ? -1 : group); }
+
+int mamba_abi_version(void) { return (1 << 16) | 8; }
 
 }  // extern "C"

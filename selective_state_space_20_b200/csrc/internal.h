@@ -109,6 +109,10 @@ cudaError_t launch_conv1d_update(const Conv1dUpdateArgs &a, cudaStream_t stream)
 
 // Persistent, queue-balanced scan (dstate <= 16), one or two lanes per channel.
 bool persistent_supported(const ScanArgs &a);
+// Test hook: the lane-split kernel's pieces of this channel group stop
+// publishing their carried state, so the next piece's bounded wait runs out
+// (-1 turns it off).  Returns the previous value.
+int set_stall_group(int group);
 bool persistent_preferred(const ScanArgs &a, int sm_count);
 int persistent_choose_lanes(const ScanArgs &a, int sm_count);  // 0 = not preferred
 size_t persistent_workspace_bound(int64_t batch, int64_t dim, int64_t seqlen, int act);

@@ -51,6 +51,7 @@ struct Params {
     unsigned *queue;       // ready-queue schedule: n_groups * (n_chunks - 1) entries
     unsigned *progress;    // balanced schedule: per group, sub-chunks whose carry is out
     int subs_per_chain;    // balanced schedule: sub-chunks per group (ceil(seqlen / TC))
+    int stall_group;       // test hook: this group's pieces never publish their carry (-1: none)
     float *carry;          // workspace: n_groups * 32 lanes * states-per-lane floats
 };
 

@@ -82,6 +82,16 @@ size_t bound_for(int64_t batch, int64_t dim, int64_t seqlen, int lanes, int act)
 
 }  // namespace
 
+namespace {
+int g_stall_group = -1;  // test hook (mamba_debug_stall_group)
+}  // namespace
+
+int set_stall_group(int group) {
+    const int prev = g_stall_group;
+    g_stall_group = group;
+    return prev;
+}
+
 bool persistent_supported(const ScanArgs &a) {
     if (a.dstate > persist::kNS) return false;
     const int es = a.act == kBF16 ? 2 : 4;
@@ -152,6 +162,7 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
     kp.groups_per_batch = (int)((a.dim + kp.group_channels - 1) / kp.group_channels);
     kp.n_groups = (int)groups;
     kp.subs_per_chain = (int)((a.seqlen + tc - 1) / tc);
+    kp.stall_group = g_stall_group;
     unsigned char *w = static_cast<unsigned char *>(workspace);
     kp.hdr = reinterpret_cast<unsigned *>(w);
 

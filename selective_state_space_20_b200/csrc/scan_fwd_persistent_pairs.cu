@@ -482,7 +482,7 @@ scan_fwd_pairs_kernel(const Params p) {
             // before this tile's stores, so the release waits on less
             if (publish_end && sub + 1 == nsub && se < p.subs_per_chain) {
                 store_carry(h);
-                publish_progress(p, lane, g, se);
+                if (g != p.stall_group) publish_progress(p, lane, g, se);
             }
             // ---- coalesced store of the output tile
 #pragma unroll
@@ -538,7 +538,7 @@ scan_fwd_pairs_kernel(const Params p) {
                 h[k] = hin[k];
             }
             store_carry(hend);
-            publish_progress(p, lane, g, se);
+            if (g != p.stall_group) publish_progress(p, lane, g, se);
             run_subs(false, h, dsum, false);
         } else {
             if (sb > 0) {
