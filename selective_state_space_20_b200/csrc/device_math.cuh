@@ -45,13 +45,15 @@ __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b
 
 // 2^x for two values on the FMA pipe, leaving the MUFU free for other work.
 // Cody-Waite split x = j + f, j = rint(x) (adding and subtracting 1.5 * 2^23
-// rounds to the nearest integer), f in [-1/2, 1/2]; 2^f = Q(f), Q the degree-5
-// Chebyshev interpolant of 2^f (coefficients from fit_exp2_poly.py in this
-// directory; relative error in fp32 <= 2.2e-7, the same order as ex2.approx);
-// 2^j is added into the exponent field of Q(f) (the low bits of x + 1.5 * 2^23
-// hold j, so (bits << 23) is j << 23).  x is clamped to [-125, 127] so the
-// exponent field cannot wrap: below -125 the result is 2^-125 instead of a
-// denormal or 0, above 127 it stays finite.
+// rounds to the nearest integer), f in [-1/2, 1/2]; 2^f = Q(f) = 1 + f P(f),
+// P the degree-4 Chebyshev interpolant of (2^f - 1) / f (coefficients from
+// fit_exp2_poly.py in this directory; relative error of Q in fp32 <= 2.6e-7,
+// the order of ex2.approx, and Q(0) = 1 exactly, so a decay near 1 carries no
+// fixed bias into the many steps a slow state remembers); 2^j is added into
+// the exponent field of Q(f) (the low bits of x + 1.5 * 2^23 hold j, so
+// (bits << 23) is j << 23).  x is clamped to [-125, 127] so the exponent field
+// cannot wrap: below -125 the result is 2^-125 instead of a denormal or 0,
+// above 127 it stays finite.
 __device__ __forceinline__ float2 ex2_poly2(float2 x) {
     x.x = fminf(fmaxf(x.x, -125.f), 127.f);
     x.y = fminf(fmaxf(x.y, -125.f), 127.f);
@@ -59,11 +61,11 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
     const float2 t = __fadd2_rn(x, f2(kRound, kRound));
     const float2 j = __fadd2_rn(t, f2(-kRound, -kRound));
     const float2 f = __ffma2_rn(j, f2(-1.f, -1.f), x);
-    float2 q = __ffma2_rn(f2(1.339086331e-03f, 1.339086331e-03f), f, f2(9.676031768e-03f, 9.676031768e-03f));
-    q = __ffma2_rn(q, f, f2(5.550356954e-02f, 5.550356954e-02f));
-    q = __ffma2_rn(q, f, f2(2.402210683e-01f, 2.402210683e-01f));
+    float2 q = __ffma2_rn(f2(1.338130212e-03f, 1.338130212e-03f), f, f2(9.666368365e-03f, 9.666368365e-03f));
+    q = __ffma2_rn(q, f, f2(5.550381169e-02f, 5.550381169e-02f));
+    q = __ffma2_rn(q, f, f2(2.402234972e-01f, 2.402234972e-01f));
     q = __ffma2_rn(q, f, f2(6.931471825e-01f, 6.931471825e-01f));
-    q = __ffma2_rn(q, f, f2(1.000000119e+00f, 1.000000119e+00f));
+    q = __ffma2_rn(q, f, f2(1.f, 1.f));  // Q(f) = 1 + f P(f)
     return f2(__uint_as_float(__float_as_uint(t.x) * 8388608u + __float_as_uint(q.x)),
               __uint_as_float(__float_as_uint(t.y) * 8388608u + __float_as_uint(q.y)));
 }

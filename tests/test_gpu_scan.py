@@ -320,8 +320,9 @@ def test_past_32_bit_indexing():
     assert e_out <= TOL[torch.bfloat16] and e_state <= TOL[torch.bfloat16]
 
 
-@pytest.mark.parametrize("sched", [binding.SCHEDULE_STATIC, binding.SCHEDULE_PERSISTENT])
-def test_zero_step_keeps_the_state(sched):
+@pytest.mark.parametrize("sched,lanes", [(binding.SCHEDULE_STATIC, 0), (binding.SCHEDULE_PERSISTENT, 1),
+                                         (binding.SCHEDULE_PERSISTENT, 2), (binding.SCHEDULE_PERSISTENT, 4)])
+def test_zero_step_keeps_the_state(sched, lanes):
     """delta = 0 (softplus off, no bias): Abar = 1 and no input, so the state
     stays h0 bit for bit and y_t = C_t . h0 + D u_t (the oracle's pin, on
     the GPU)."""
@@ -333,7 +334,8 @@ def test_zero_step_keeps_the_state(sched):
     dev = dev_inputs(cpu)
     h0 = inputs.initial_state(2, 48, 16, seed=5)
     out, last = binding.mamba_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],
-                                       delta_softplus=False, return_last_state=True, h0=h0.cuda(), schedule=sched)
+                                       delta_softplus=False, return_last_state=True, h0=h0.cuda(), schedule=sched,
+                                       lanes_per_channel=lanes)
     torch.cuda.synchronize()
     assert torch.equal(last.cpu(), h0)
     y = torch.einsum("bdn,bnl->bdl", h0.double(), cpu["C"].double()) + cpu["D"].double()[None, :, None] * cpu["u"].double()
