@@ -57,6 +57,14 @@ def test_shapes_span_tiles_and_ragged_tails(dtype, shape):
     check_full(inputs.custom(b, d, L, 16, dtype, seed=hash(shape) % 1000))
 
 
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("L", [1, 3, 7, 9])
+@pytest.mark.parametrize("dstate", [1, 2])
+def test_tiny_odd_lengths_and_states(dtype, L, dstate):
+    # every schedule the planner may pick for these (static, and persistent where L allows)
+    check_full(inputs.custom(2, 33, L, dstate, dtype, seed=L * 10 + dstate))
+
+
 @pytest.mark.parametrize("dstate", [1, 2, 3, 5, 8, 13, 16, 17, 24, 32, 33, 40, 64])
 def test_every_dstate(dstate):
     check_full(inputs.custom(2, 19, 100, dstate, "fp32", seed=dstate))
