@@ -399,6 +399,15 @@ int mamba_state_fold(const float *h_init, const double *delta_sums, const float 
                      const float *h_local, float *h_out, int64_t batch, int64_t dim,
                      int64_t dstate, int64_t count, cudaStream_t stream);
 
+/* The device-side status of this process's work on the current device:
+ * synchronises `stream`, then returns MAMBA_ERR_CUDA if the stream or the
+ * context reports an error, MAMBA_ERR_TIMEOUT if the last persistent launch
+ * on this device (any entry point that was given a workspace) gave up a
+ * bounded wait -- the error word in its workspace, which must still be
+ * allocated -- else MAMBA_OK.  No device code traps; this and
+ * mamba_scan_workspace_status are how failures surface. */
+int mamba_get_device_status(cudaStream_t stream);
+
 /* Test hook for the failure-detection path: from the next launch on, the
  * persistent lane-split kernel's pieces of channel group `group` no longer
  * publish their carried state, so the piece after them waits until its time

@@ -33,7 +33,8 @@ EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
             "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_fwd_strided",
             "mamba_scan_fwd_complex", "mamba_delta_sum", "mamba_state_fold", "mamba_scan_fwd_conv",
-            "mamba_scan_host_scratch_size", "mamba_scan_fwd_host", "mamba_debug_stall_group", "mamba_scan_bwd", "mamba_scan_bwd_init",
+            "mamba_scan_host_scratch_size", "mamba_scan_fwd_host", "mamba_debug_stall_group",
+            "mamba_get_device_status", "mamba_scan_bwd", "mamba_scan_bwd_init",
             "mamba_scan_bwd_workspace_size",
             "mamba_state_update", "mamba_conv1d_fwd",
             "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version")
@@ -85,6 +86,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_fwd_conv.argtypes = [vp, fp, fp, i64, i64, vp, fp, vp, vp, fp, vp, i64, fp, fp, vp, fp, vp,
                                         i64, i64, i64, i64, ci, vp, ctypes.c_size_t, vp]
     lib.mamba_scan_fwd_conv.restype = ci
+    lib.mamba_get_device_status.argtypes = [vp]
+    lib.mamba_get_device_status.restype = ci
     lib.mamba_debug_stall_group.argtypes = [ci]
     lib.mamba_debug_stall_group.restype = ci
     lib.mamba_scan_host_scratch_size.argtypes = [i64, i64, i64, i64, ci]
@@ -541,6 +544,15 @@ def mamba_state_fold(A: torch.Tensor, delta_sums: torch.Tensor, h_local: torch.T
                                   batch, dim, N, count, _stream(dev))
     _check("mamba_state_fold", rc)
     return out
+
+
+def device_status(device=None) -> int:
+    """Synchronise the current stream and return the library's device status
+    (0 = ok, MAMBA_ERR_TIMEOUT after a bounded wait gave up, MAMBA_ERR_CUDA
+    after a CUDA error)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return load_library().mamba_get_device_status(_stream(dev))
 
 
 def workspace_status(workspace: torch.Tensor) -> int:

@@ -13,6 +13,13 @@ constexpr int kMaxDstate = 64;
 constexpr int kMaxDevices = 64;
 
 int g_sm_count[kMaxDevices];  // 0 = not queried yet (benign races: same value)
+// workspace of the last persistent launch per device (mamba_get_device_status)
+const void *g_last_workspace[kMaxDevices];
+
+void note_workspace(const void *ws) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) g_last_workspace[dev] = ws;
+}
 
 int current_sm_count(int *status) {
     int dev = 0;
@@ -148,6 +155,7 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
             plan_out->chunk_timesteps = want_chunk;
         }
         if (!launch) return MAMBA_OK;
+        note_workspace(workspace);
         return mscan::launch_scan_fwd_persistent(a, persist_lanes, want_chunk, workspace, ws_bytes,
                                                  sms, stream) == cudaSuccess
                    ? MAMBA_OK : MAMBA_ERR_CUDA;
@@ -406,6 +414,7 @@ int mamba_scan_fwd_conv(const void *x, const float *conv_weight, const float *co
     a.u_bstride = x_batch_stride; a.z_bstride = z_batch_stride;
     int lanes = mscan::persistent_choose_lanes(a, sms);
     if (lanes != 2 && lanes != 4) lanes = 2;  // the balanced split covers any shape
+    note_workspace(workspace);
     return mscan::launch_scan_fwd_persistent(a, lanes, 0, workspace, workspace_bytes, sms, stream) == cudaSuccess
                ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
@@ -505,6 +514,19 @@ int mamba_scan_workspace_status(const void *workspace, cudaStream_t stream) {
     unsigned hdr[4] = {0, 0, 0, 0};
     if (cudaMemcpy(hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost) != cudaSuccess)
         return MAMBA_ERR_CUDA;
+    return hdr[2] != 0 ? MAMBA_ERR_TIMEOUT : MAMBA_OK;
+}
+
+int mamba_get_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MAMBA_ERR_CUDA;
+    const cudaError_t sticky = cudaPeekAtLastError();
+    if (sticky != cudaSuccess) return MAMBA_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MAMBA_ERR_DEVICE;
+    const void *ws = (dev >= 0 && dev < kMaxDevices) ? g_last_workspace[dev] : nullptr;
+    if (!ws) return MAMBA_OK;
+    unsigned hdr[4] = {0, 0, 0, 0};
+    if (cudaMemcpy(hdr, ws, sizeof(hdr), cudaMemcpyDeviceToHost) != cudaSuccess) return MAMBA_ERR_CUDA;
     return hdr[2] != 0 ? MAMBA_ERR_TIMEOUT : MAMBA_OK;
 }
 

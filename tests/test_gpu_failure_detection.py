@@ -36,12 +36,13 @@ def test_stalled_carry_times_out_and_is_reported():
     try:
         run()
         status = binding.workspace_status(ws)
+        device_status = binding.device_status()
     finally:
         lib.mamba_debug_stall_group(prev)
-    assert status == binding.MAMBA_ERR_TIMEOUT
+    assert status == binding.MAMBA_ERR_TIMEOUT and device_status == binding.MAMBA_ERR_TIMEOUT
     # the context and the workspace are fine: the next launch is complete and correct
     out, last = run()
-    assert binding.workspace_status(ws) == 0
+    assert binding.workspace_status(ws) == 0 and binding.device_status() == 0
     rows = [0, 17, 63]
     cpu = {k: v for k, v in dev.items()}
     from parity import oracle_rows
