@@ -137,8 +137,14 @@ int mamba_scan_fwd_host(const void *u, const void *delta, const float *A, const 
     }
     if (ok && last_state)
         ok = cu(cudaMemcpyAsync(last_state, ls_dev, (size_t)(batch * dim * dstate) * 4, cudaMemcpyDeviceToHost, s_out));
-    // the caller's stream continues after every copy back
-    if (ok) ok = cu(cudaEventRecord(start, s_out)) && cu(cudaStreamWaitEvent(stream, start, 0));
+    // the caller's stream continues after everything this call enqueued --
+    // also after an error, so that synchronising it still covers every copy
+    if (s_in && s_out && ev[0] && ev[1]) {
+        cu(cudaEventRecord(ev[0], s_out));
+        cu(cudaStreamWaitEvent(stream, ev[0], 0));
+        cu(cudaEventRecord(ev[1], s_in));
+        cu(cudaStreamWaitEvent(stream, ev[1], 0));
+    }
     for (int i = 0; i < 7; ++i)
         if (ev[i]) cudaEventDestroy(ev[i]);
     if (s_in) cudaStreamDestroy(s_in);
