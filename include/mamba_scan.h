@@ -19,18 +19,36 @@
  * mamba README (the selective-scan interface and the Mamba(d_model,
  * d_state=16, d_conv=4, expand=2) block that wraps it).
  *
+ * Entry points
+ * ------------
+ *   forward scan      mamba_scan_fwd, _tuned, _ws (workspace: persistent
+ *                     schedule), _noalloc, _init (from a given state),
+ *                     _strided (any strides), _complex (complex mode),
+ *                     _conv (causal conv1d + silu fused in), _host (sequences
+ *                     in host memory); mamba_scan_plan, mamba_scan_workspace_size,
+ *                     mamba_scan_host_scratch_size
+ *   decoding          mamba_state_update (one token), mamba_conv1d_update
+ *   conv1d            mamba_conv1d_fwd
+ *   backward          mamba_scan_bwd, mamba_scan_bwd_init, mamba_scan_bwd_workspace_size
+ *   sequence split    mamba_delta_sum, mamba_state_fold
+ *   status            mamba_scan_workspace_status, mamba_get_device_status,
+ *                     mamba_status_string, mamba_abi_version;
+ *                     mamba_debug_stall_group (test hook)
+ *
  * Conventions for every entry point
  * ---------------------------------
  * - Pointers are DEVICE pointers (cudaMalloc'd, managed, or mapped pinned host
  *   memory) of the current CUDA device, except where stated.  Tensors are
- *   dense, row-major and contiguous with the layouts given per function.
+ *   dense, row-major and contiguous with the layouts given per function,
+ *   except where strides are given.
  * - "act" tensors (u, delta, z, B, C, out) share one element type chosen by
  *   `act_dtype` (MAMBA_F32 or MAMBA_BF16).  A, D, delta_bias, states are
  *   always fp32.  All arithmetic is fp32.
- * - The caller owns every buffer.  The library never allocates or frees, and
- *   only mamba_scan_workspace_status synchronises: work is enqueued on
- *   `stream` (0 = legacy default stream) and buffers must stay alive until
- *   that work completes.
+ * - The caller owns every buffer.  The library allocates no memory (the
+ *   host-memory scan creates and releases two streams and seven events per
+ *   call) and only mamba_scan_workspace_status and mamba_get_device_status
+ *   synchronise: work is enqueued on `stream` (0 = legacy default stream) and
+ *   buffers must stay alive until that work completes.
  * - Argument validation is synchronous and happens before anything is
  *   enqueued; a non-zero return means nothing was enqueued, except
  *   MAMBA_ERR_CUDA, which reports a launch failure (cudaGetLastError).
@@ -38,7 +56,10 @@
  *   of the 16-byte vector width take the vectorised path, others a scalar path.
  * - `out` may alias exactly one of u, delta or z (same pointer, in-place);
  *   any other overlap between an output and an input is rejected.
- * - The library holds no state; calls are reentrant and thread-safe.
+ * - Calls are reentrant and thread-safe.  Library state: per device, the
+ *   workspace pointer of the last persistent launch (for
+ *   mamba_get_device_status) and the scratch area of mamba_scan_fwd_noalloc;
+ *   process-wide, the mamba_debug_stall_group test hook (off by default).
  */
 #ifndef MAMBA_SCAN_H
 #define MAMBA_SCAN_H
@@ -78,11 +99,13 @@ typedef enum {
     MAMBA_SCHEDULE_AUTO = 0,
     MAMBA_SCHEDULE_STATIC = 1,     /* one block per channel group walks the whole
                                       sequence; no workspace */
-    MAMBA_SCHEDULE_PERSISTENT = 2  /* dstate <= 16: persistent warps take
-                                      (channel group, time chunk) units from a
-                                      ready queue and pass the state between
-                                      chunks through the workspace; 1, 2 or 4
-                                      lanes per channel */
+    MAMBA_SCHEDULE_PERSISTENT = 2  /* dstate <= 16: persistent warps, all
+                                      resident; 2 or 4 lanes per channel split
+                                      the (channel group, sub-chunk) grid into
+                                      equal contiguous shares, 1 lane per
+                                      channel takes (group, time chunk) units
+                                      from a ready queue; states pass between
+                                      pieces through the workspace */
 } mamba_schedule_t;
 
 /* Optional launch tuning.  Zero fields mean "choose automatically".
