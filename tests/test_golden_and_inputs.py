@@ -101,3 +101,27 @@ def test_distribution_moments():
     dt = np.logaddexp(0.0, a["delta_bias"].double().numpy())
     # log-uniform: log(dt) spread over [log 1e-3, log 1e-1]
     assert math.log(1e-3) - 1e-6 <= np.log(dt).min() and np.log(dt).max() <= math.log(1e-1) + 1e-6
+
+
+def test_complex_conv_and_state_recipes():
+    """The generators of the further rows: shapes, dtypes and the stated
+    distributions (complex A = -1/2 + i pi n, B and C with unit mean square
+    magnitude; conv taps within +-1/sqrt(K); initial states with spread 1/4);
+    deterministic under a seed."""
+    import math
+    import torch
+    from selective_state_space_20_b200 import inputs
+    c = inputs.complex_inputs(2, 8, 512, 16, "bf16", seed=3)
+    assert c["A"].shape == (8, 16, 2) and c["A"].dtype == torch.float32
+    assert torch.all(c["A"][..., 0] == -0.5)
+    assert torch.allclose(c["A"][0, :, 1], math.pi * torch.arange(16, dtype=torch.float32))
+    assert c["B"].shape == (2, 16, 512, 2) and c["B"].dtype == torch.bfloat16
+    ms = (c["B"].float() ** 2).sum(-1).mean().item()
+    assert 0.9 < ms < 1.1
+    c2 = inputs.complex_inputs(2, 8, 512, 16, "bf16", seed=3)
+    assert all(torch.equal(c[k], c2[k]) for k in ("u", "delta", "B", "C", "A"))
+    k = inputs.conv_inputs(2, 8, 64, width=3, dtype="fp32", seed=4)
+    assert k["xz"].shape == (2, 16, 64) and k["weight"].shape == (8, 3)
+    assert k["weight"].abs().max().item() <= 1 / math.sqrt(3)
+    h = inputs.initial_state(4, 256, 16, seed=5)
+    assert h.shape == (4, 256, 16) and 0.22 < h.std().item() < 0.28
