@@ -108,9 +108,6 @@ def test_complex_conv_and_state_recipes():
     distributions (complex A = -1/2 + i pi n, B and C with unit mean square
     magnitude; conv taps within +-1/sqrt(K); initial states with spread 1/4);
     deterministic under a seed."""
-    import math
-    import torch
-    from selective_state_space_20_b200 import inputs
     c = inputs.complex_inputs(2, 8, 512, 16, "bf16", seed=3)
     assert c["A"].shape == (8, 16, 2) and c["A"].dtype == torch.float32
     assert torch.all(c["A"][..., 0] == -0.5)
