@@ -85,3 +85,16 @@ def test_fused_benchmark_layer():
     _, out2, last2 = _two_calls(ins, x, cw, cb, w.dim, lanes)
     torch.cuda.synchronize()
     assert torch.equal(out, out2) and torch.equal(last, last2)
+
+
+@pytest.mark.parametrize("K", [1, 3])
+def test_fused_short_kernels_without_bias(K):
+    b, d, L = 2, 64, 512
+    ins, x, w, cb = _problem(b, d, L, 16, "bf16", K, seed=40 + K)
+    out, last, u = binding.mamba_scan_fwd_conv(x, w, None, ins["delta"], ins["A"], ins["B"], ins["C"], D=ins["D"],
+                                               z=ins["z"], delta_bias=ins["delta_bias"], return_last_state=True,
+                                               return_u=True)
+    lanes = _plan_lanes(b, d, L, 16, torch.bfloat16)
+    u2, out2, last2 = _two_calls(ins, x, w, None, d, lanes)
+    torch.cuda.synchronize()
+    assert torch.equal(u, u2) and torch.equal(out, out2) and torch.equal(last, last2)
