@@ -71,6 +71,16 @@ MUTANTS = [
     ("bwd-dB-without-u", "j->dB[b * N * L + n * L + t] += g[n] * delta * ut;",
      "j->dB[b * N * L + n * L + t] += g[n] * delta;"),
     ("bwd-dD-without-gate", "j->dD[d] += dy * ut;", "j->dD[d] += dout[t] * ut;"),
+    ("bwd-dbias-without-softplus-derivative", "j->dbias[d] += ddraw;", "j->dbias[d] += ddelta;"),
+    ("bwd-dh0-missing-first-decay", "                g[n] *= Abar;\n            }\n            const double ddraw",
+     "                if (t > 0)\n                    g[n] *= Abar;\n            }\n            const double ddraw"),
+    ("bwd-du-skip-term-dropped", "double du = dy * Dd, ddelta = 0.0;", "double du = 0.0, ddelta = 0.0;"),
+    ("bwd-dz-without-skip", "double y = Dd * ut;\n            for (int64_t n = 0; n < N; ++n)\n                y += (double)Cw",
+     "double y = 0.0;\n            for (int64_t n = 0; n < N; ++n)\n                y += (double)Cw"),
+    # one-token state update
+    ("update-gate-dropped", "y *= s6_oracle_silu((double)z[row]);", "y *= 1.0;"),
+    ("update-skip-dropped", "y += (D ? (double)D[d] : 0.0) * ut;", "y += 0.0 * ut;"),
+    ("update-softplus-dropped", "delta_t = s6_oracle_softplus(delta_t);", "delta_t = delta_t;"),
     # complex mode
     ("cplx-readout-conjugated", "y += creal(Cn * h[n]);", "y += creal(conj(Cn) * h[n]);"),
     ("cplx-readout-magnitude", "y += creal(Cn * h[n]);", "y += cabs(Cn * h[n]);"),
