@@ -260,15 +260,35 @@ def oracle_beside(kind: str, w, k: int = 32):
                       f"{elems} elements in {dt:.2f} s"}
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(w, seconds=25.0):
     cores = os.cpu_count() or 1
     data, k = oracle_sample(w, seconds)
     dt = _oracle_run(data, cores)
     elems = w.batch * k * w.seqlen
     what = "the whole workload" if k == w.dim else f"all {w.batch} batch rows, first {k} of {w.dim} channels"
+    # one thread on a small fixed sample (best of 3), for the per-core rate
+    k1 = min(64, w.dim)
+    one = inputs.scan_inputs(dataclasses.replace(w, batch=1, dim=k1))
+    dt1 = min(_oracle_run(one, 1) for _ in range(3))
     return {"value": elems / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{what}, full L={w.seqlen}, N={w.dstate}: {elems} elements in {dt:.2f} s "
-                      f"(fp64 C loop over {cores} threads)"}
+                      f"(fp64 C loop over {cores} threads)",
+            "cpu_model": cpu_model(),
+            "single_thread": {"value": k1 * w.seqlen / dt1 / 1e9, "unit": UNIT,
+                              "sample": f"1 batch row, first {k1} channels, full L={w.seqlen}, "
+                                        f"best of 3 runs on 1 thread"}}
 
 
 def run_reference(args, world, rank):
@@ -295,7 +315,7 @@ def run_reference(args, world, rank):
             "config": {"workload": w.name, "batch": w.batch, "dim": w.dim, "seqlen": w.seqlen,
                        "dstate": w.dstate, "act_dtype": w.dtype, "sample_per_step": sample},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
