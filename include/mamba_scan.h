@@ -56,7 +56,9 @@
  *   of the 16-byte vector width take the vectorised path, others a scalar path.
  * - `out` may alias exactly one of u, delta or z (same pointer, in-place);
  *   any other overlap between an output and an input is rejected.
- * - Calls are reentrant and thread-safe.  Library state: per device, the
+ * - Calls are reentrant and thread-safe, with one exception:
+ *   mamba_scan_fwd_noalloc calls share one scratch area per device, so the
+ *   caller must serialise them (see there).  Library state: per device, the
  *   workspace pointer of the last persistent launch (for
  *   mamba_get_device_status) and the scratch area of mamba_scan_fwd_noalloc;
  *   process-wide, the mamba_debug_stall_group test hook (off by default).
@@ -462,15 +464,18 @@ int mamba_scan_workspace_status(const void *workspace, cudaStream_t stream);
  * cudaMalloc, cudaFree or other allocating routine.  The caller still
  * provides every input and output.
  *
- * - Every GPU that loads the library reserves the 4 MiB area until the
- *   process exits.
+ * - The 4 MiB area is reserved on a device when the library's device code
+ *   is loaded there, and held until the process exits.  With lazily loaded
+ *   modules (CUDA_MODULE_LOADING=LAZY, the CUDA default) that happens at the
+ *   first call on each device, which can then fail with MAMBA_ERR_CUDA if
+ *   the device is out of memory: make the first call early, and before any
+ *   stream capture begins.
  * - Problems whose workspace (mamba_scan_workspace_size) exceeds 4 MiB are
  *   rejected with MAMBA_ERR_WORKSPACE before anything is enqueued; that is
  *   about 2,000 groups of 32 channels (batch * ceil(dim / 32)) at moderate
  *   lengths.
- * - The first call on each device looks up the area's device address
- *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call before any stream capture begins.
+ * - Every call looks the area's device address up in the current context
+ *   (cudaGetSymbolAddress); nothing is cached between calls.
  * - All calls share the one area and each launch re-initialises the part
  *   that must start at zero; calls whose GPU work can overlap (other streams,
  *   other host threads) race on it and must be serialised by the caller.

@@ -1,5 +1,6 @@
-"""Coefficients of the e^x - 1 polynomial used by the complex-mode scan's
-fp32 path.
+"""Coefficients of the e^x - 1 polynomial (expm1_f in device_math.cuh) that
+the fp32-activation paths of every scan kernel, real and complex, use for
+their decays.
 
 For x in [-1, 1], e^x - 1 = x + x^2 P(x), P the degree-DEG Chebyshev
 interpolant of (e^x - 1 - x) / x^2 on [-1, 1] (a near-minimax fit, computed

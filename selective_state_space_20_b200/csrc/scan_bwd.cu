@@ -29,7 +29,9 @@
 // warps in a fixed order and stores the group's partial sum; a second kernel
 // adds the groups of each batch row in a fixed order.  dA, dD and dbias are
 // summed over a group's whole sequence in registers and added once per
-// group with atomics.
+// group with atomics.  fp32 activations take the accurate decay, softplus and
+// sigmoid (Decay<true> of device_math.cuh: the state and the adjoint advance
+// by (Abar - 1) x + b, Abar - 1 on the FMA pipe), bf16 ones one ex2 per decay.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -111,6 +113,14 @@ struct ChannelTranspose<2, CNT> {
     __device__ __forceinline__ static void run(float (&)[8], int) {}
 };
 
+// 1 / (1 + e^-x): the MUFU form for bf16 activations, CUDA's full-precision
+// expf and division for fp32 ones.
+template <bool ACC>
+__device__ __forceinline__ float sigmoid(float x) {
+    if (ACC) return 1.f / (1.f + expf(-x));
+    return __fdividef(1.f, 1.f + __expf(-x));
+}
+
 __device__ __forceinline__ float quad_sum(float x) {
     x += __shfl_xor_sync(0xffffffffu, x, 1);
     return x + __shfl_xor_sync(0xffffffffu, x, 2);
@@ -118,6 +128,8 @@ __device__ __forceinline__ float quad_sum(float x) {
 
 template <typename T, bool SP, bool GATE>
 __global__ void __launch_bounds__(kWarpsBwd * 32, 5) scan_bwd_kernel(const BwdParams p) {
+    constexpr bool ACC = sizeof(T) == 4;
+    using Dk = Decay<ACC>;
     extern __shared__ __align__(16) float bwd_smem[];
     const int tid = threadIdx.x, lane = tid & 31, wib = tid >> 5;
     const int c = lane >> 2, r = lane & 3;
@@ -154,7 +166,7 @@ __global__ void __launch_bounds__(kWarpsBwd * 32, 5) scan_bwd_kernel(const BwdPa
         for (int i = 0; i < kSPL; ++i) {
             const int n = kSPL * r + i;
             Ar[i] = (valid && n < N) ? __ldg(p.A + dc * N + n) : 0.f;
-            A2[i] = Ar[i] * kLog2e;
+            A2[i] = Ar[i] * Dk::kScale;
         }
         const float bias = (valid && p.delta_bias) ? __ldg(p.delta_bias + dc) : 0.f;
         const float Dd = (valid && p.D) ? __ldg(p.D + dc) : 0.f;
@@ -217,8 +229,8 @@ __global__ void __launch_bounds__(kWarpsBwd * 32, 5) scan_bwd_kernel(const BwdPa
 #pragma unroll
                     for (int s = 0; s < kSeg; ++s) {
                         const float x = f[s] + fbias;
-                        dst[(X_DL * kSeg + s) * kCPW] = SP ? softplus_f(x) : x;
-                        if (full) dst[(X_SIG * kSeg + s) * kCPW] = SP ? __fdividef(1.f, 1.f + __expf(-x)) : 1.f;
+                        dst[(X_DL * kSeg + s) * kCPW] = SP ? Dk::softplus(x) : x;
+                        if (full) dst[(X_SIG * kSeg + s) * kCPW] = SP ? sigmoid<ACC>(x) : 1.f;
                     }
                 } else {
                     const int X = fq == 0 ? X_U : fq == 2 ? X_DOUT : X_Z;
@@ -226,7 +238,7 @@ __global__ void __launch_bounds__(kWarpsBwd * 32, 5) scan_bwd_kernel(const BwdPa
                     for (int s = 0; s < kSeg; ++s) dst[(X * kSeg + s) * kCPW] = f[s];
                     if (fq == 3) {
 #pragma unroll
-                        for (int s = 0; s < kSeg; ++s) dst[(X_SGZ * kSeg + s) * kCPW] = __fdividef(1.f, 1.f + __expf(-f[s]));
+                        for (int s = 0; s < kSeg; ++s) dst[(X_SGZ * kSeg + s) * kCPW] = sigmoid<ACC>(f[s]);
                     }
                 }
             }
@@ -241,7 +253,7 @@ __global__ void __launch_bounds__(kWarpsBwd * 32, 5) scan_bwd_kernel(const BwdPa
                 const float4 bb = *reinterpret_cast<const float4 *>(sB + s * kNS + kSPL * r);
                 const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
-                for (int i = 0; i < kSPL; ++i) h[i] = fmaf(ex2_mufu(dl * A2[i]), h[i], du * bv[i]);
+                for (int i = 0; i < kSPL; ++i) h[i] = Dk::step(dl * A2[i], h[i], du * bv[i]);
                 if (keep) hist[(s + 1) * 32 + lane] = make_float4(h[0], h[1], h[2], h[3]);
             }
         };
@@ -324,13 +336,14 @@ __global__ void __launch_bounds__(kWarpsBwd * 32, 5) scan_bwd_kernel(const BwdPa
                 for (int i = 0; i < kSPL; ++i) {
                     v[4 + i] = dy * hcur[i];
                     g[i] = fmaf(dy, cv[i], g[i]);
-                    const float ab = ex2_mufu(dl * A2[i]);
+                    const float xa = dl * A2[i];
+                    const float ab = Dk::abar(xa);
                     const float gha = g[i] * hp[i] * ab;
                     ddelta_p = fmaf(gha, Ar[i], fmaf(g[i], bv[i] * ut, ddelta_p));
                     dA_acc[i] = fmaf(gha, dl, dA_acc[i]);
                     v[i] = g[i] * dl * ut;
                     dut_p = fmaf(g[i] * dl, bv[i], dut_p);
-                    g[i] *= ab;
+                    g[i] = ACC ? Dk::scale(xa, g[i]) : g[i] * ab;
                 }
                 ChannelTranspose<16, 8>::run(v, lane);
                 red[s * 32 + kslot] = v[0];

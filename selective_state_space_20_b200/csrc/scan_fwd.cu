@@ -1,7 +1,7 @@
 // scan_fwd.cu -- fused selective-scan (S6) forward kernel for sm_100a.
 //
 // What one launch computes (per batch row b and channel d, time in order):
-//   delta = softplus(delta_raw + bias[d]);  Abar = 2^(delta * A[d,n] * log2 e)
+//   delta = softplus(delta_raw + bias[d]);  Abar = exp(delta * A[d,n])
 //   h[n]  = Abar * h[n] + (delta * u) * B[b,n,t];   y = sum_n C[b,n,t] h[n]
 //   out   = (y + D[d] u) * silu(z)
 // following the recurrent form and the selective_scan / MambaBlock listings
@@ -24,7 +24,9 @@
 //   * Prologue (one thread per 16-byte vector): delta = softplus(raw + bias)
 //     and delta*u are computed once per element into fp32 shared memory.
 //   * Scan: per thread, per state, per timestep: one ex2 (MUFU), one FMUL
-//     (delta*u*B), one FFMA (state), one FFMA (readout).  Partial readouts of
+//     (delta*u*B), one FFMA (state), one FFMA (readout).  fp32 activations
+//     take the accurate decay of device_math.cuh (Decay<true>: the state
+//     advances by (Abar - 1) h + b with Abar - 1 on the FMA pipe).  Partial readouts of
 //     the R lanes are summed with a transposed butterfly (log2 R shuffle
 //     rounds) so each lane ends up owning complete outputs.
 //   * Epilogue (one thread per 16-byte vector): out = (y + D u) silu(z),
@@ -137,6 +139,7 @@ template <typename T, int NP, int R, int THREADS, bool CL>
 __global__ void __launch_bounds__(THREADS)
 scan_fwd_kernel(const KParams p) {
     using G = Geom<T, NP, R, THREADS>;
+    using Dk = Decay<sizeof(T) == 4>;
     constexpr int S = G::S, CG = G::CG, V = G::V, RB = G::RB, TC = G::TC;
     constexpr int TCP = TC + 4;            // fp32 row pitch (16-byte multiple)
     constexpr int VPR = TC / V;            // 16-byte vectors per row per chunk
@@ -176,7 +179,7 @@ scan_fwd_kernel(const KParams p) {
 #pragma unroll
     for (int s = 0; s < S; ++s) {
         const int n = r * S + s;
-        A2[s] = (d < Dm && n < N) ? __ldg(p.A + d * N + n) * kLog2e : 0.f;
+        A2[s] = (d < Dm && n < N) ? __ldg(p.A + d * N + n) * Dk::kScale : 0.f;
         h[s] = (p.h0 && d < Dm && n < N) ? __ldcg(p.h0 + (b * Dm + d) * N + n) : 0.f;
     }
 
@@ -287,7 +290,7 @@ scan_fwd_kernel(const KParams p) {
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 float dl = fd[i] + bias;
-                if (p.softplus) dl = softplus_f(dl);
+                if (p.softplus) dl = Dk::softplus(dl);
                 if (tv * V + i >= tvalid) dl = 0.f;  // past the end: Abar = 1, no input
                 fd[i] = dl;
                 fu[i] = dl * fu[i];
@@ -339,11 +342,10 @@ scan_fwd_kernel(const KParams p) {
                         const int n = r * S + s;
                         const float4 bb = *reinterpret_cast<const float4 *>(sB + n * TCP + tb + q);
                         const float4 cc = *reinterpret_cast<const float4 *>(sC + n * TCP + tb + q);
-                        float a;
-                        a = ex2_mufu(dl.x * A2[s]); h[s] = fmaf(a, h[s], du.x * bb.x); y0 = fmaf(cc.x, h[s], y0);
-                        a = ex2_mufu(dl.y * A2[s]); h[s] = fmaf(a, h[s], du.y * bb.y); y1 = fmaf(cc.y, h[s], y1);
-                        a = ex2_mufu(dl.z * A2[s]); h[s] = fmaf(a, h[s], du.z * bb.z); y2 = fmaf(cc.z, h[s], y2);
-                        a = ex2_mufu(dl.w * A2[s]); h[s] = fmaf(a, h[s], du.w * bb.w); y3 = fmaf(cc.w, h[s], y3);
+                        h[s] = Dk::step(dl.x * A2[s], h[s], du.x * bb.x); y0 = fmaf(cc.x, h[s], y0);
+                        h[s] = Dk::step(dl.y * A2[s], h[s], du.y * bb.y); y1 = fmaf(cc.y, h[s], y1);
+                        h[s] = Dk::step(dl.z * A2[s], h[s], du.z * bb.z); y2 = fmaf(cc.z, h[s], y2);
+                        h[s] = Dk::step(dl.w * A2[s], h[s], du.w * bb.w); y3 = fmaf(cc.w, h[s], y3);
                     }
                     yp[q] = y0; yp[q + 1] = y1; yp[q + 2] = y2; yp[q + 3] = y3;
                 }

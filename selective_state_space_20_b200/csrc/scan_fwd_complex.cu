@@ -122,37 +122,24 @@ __device__ __forceinline__ void sincos_cm1(float t, float &s, float &c, float &c
     cm1 = (qi & 3u) == 0 ? cm1r : c - 1.f;
 }
 
-// softplus with CUDA's full-precision expf and log1pf (errors of an ulp or
-// two).  A relative error e in delta turns the rotation of a state with
-// frequency Im A by e * delta * Im A per step, and over the ~1 / (delta |Re
-// A|) steps the state remembers by e * Im A / |Re A| -- a factor of ~100 for
-// the highest frequencies of the usual complex initialisation.  The one-op
-// softplus of the real kernels has e up to 8.5e-7 for very negative inputs
-// (its exponent x log2 e is rounded to fp32), enough to show at fp32
-// tolerance; this one keeps e near 1e-7.
-__device__ __forceinline__ float softplus_precise(float x) {
-    return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));
-}
+// The fp32 path's softplus is softplus_precise (device_math.cuh): a relative
+// error e in delta turns the rotation of a state with frequency Im A by
+// e * delta * Im A per step, and over the ~1 / (delta |Re A|) steps the state
+// remembers by e * Im A / |Re A| -- a factor of ~100 for the highest
+// frequencies of the usual complex initialisation.  The one-op softplus_f has
+// e up to 8.5e-7 for very negative inputs, enough to show at fp32 tolerance;
+// softplus_precise keeps e near 1e-7.
 
 // Abar - 1 for x = delta Re A, t = delta Im A, as (re, im):
 //   e^x cos t - 1 = em1 cos t + (cos t - 1),   e^x sin t = (1 + em1) sin t,
-// em1 = e^x - 1 = x + x^2 P(x) on |x| <= 1 (P the degree-6 Chebyshev fit from
-// fit_expm1_poly.py in this directory; relative error <= 1.6e-7 in fp32),
-// else e^x - 1 directly.  The state then advances as h + (Abar - 1) h: a
+// em1 = e^x - 1 from expm1_f (device_math.cuh: accurate relative to its own
+// size near x = 0).  The state then advances as h + (Abar - 1) h: a
 // step's error is relative to the small change of h, not to h.  A decay
 // rounded to fp32 near 1 would carry the same relative error, 2^-24 or more,
 // into h at every step, and those errors add up over the ~1 / (delta |Re A|)
 // steps a state remembers -- the limit of the plain form in fp32.
 __device__ __forceinline__ void abar_minus_one(float x, float t, float &dr, float &di) {
-    float p = 2.528843470e-05f;
-    p = fmaf(p, x, 2.032904158e-04f);
-    p = fmaf(p, x, 1.388644800e-03f);
-    p = fmaf(p, x, 8.330886252e-03f);
-    p = fmaf(p, x, 4.166669771e-02f);
-    p = fmaf(p, x, 1.666669697e-01f);
-    p = fmaf(p, x, 5.000000000e-01f);
-    float em1 = fmaf(x * x, p, x);
-    if (fabsf(x) > 1.f) em1 = __expf(x) - 1.f;
+    const float em1 = expm1_f(x);
     float s, c, cm1;
     sincos_cm1(t, s, c, cm1);
     dr = fmaf(em1, c, cm1);

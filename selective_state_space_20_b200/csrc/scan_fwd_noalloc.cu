@@ -11,44 +11,36 @@
 //   exits.  Problems whose workspace would exceed it are rejected with
 //   MAMBA_ERR_WORKSPACE before anything is enqueued.
 // * A __device__ variable's name in host code is only a host-side stand-in,
-//   not a device address.  The device address is looked up with
-//   cudaGetSymbolAddress, once per device, with that device current, the
-//   first time the entry point runs on it, and cached for later calls.
+//   not a device address.  Every call looks the device address up with
+//   cudaGetSymbolAddress on the current device and context (cheap once the
+//   module is loaded), so a reset device or another context on the same
+//   device never sees a stale address.  With lazily loaded modules (the
+//   CUDA default) the first lookup on a device loads the module and thereby
+//   reserves the array; that first call may fail with MAMBA_ERR_CUDA when
+//   device memory is short, and it should come before any stream capture.
 // * Every call shares the array.  mamba_scan_fwd_ws zeroes the part that
-//   must start at zero (queue counters and slots) on the caller's stream
+//   must start at zero (header and progress words) on the caller's stream
 //   before each launch; calls whose work overlaps on the GPU (different
 //   streams, or different host threads) race on the array and must not run
 //   concurrently.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "mamba_scan.h"
 
 namespace {
 
 constexpr size_t kScratchBytes = size_t(4) << 20;  // 4 MiB per device
-constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_scan_scratch[kScratchBytes];
 
-std::mutex g_setup_mutex;
-void *g_scratch_addr[kMaxDevices];  // device address of g_scan_scratch, per device
-
-// Device address of the scratch array on the current device (set-up on the
-// first call per device).
+// Device address of the scratch array in the current context.
 int scratch_address(void **addr) {
     int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-        return MAMBA_ERR_DEVICE;
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (g_scratch_addr[dev] == nullptr) {
-        void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_scan_scratch);
-        if (e != cudaSuccess || p == nullptr) return MAMBA_ERR_CUDA;
-        g_scratch_addr[dev] = p;
-    }
-    *addr = g_scratch_addr[dev];
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return MAMBA_ERR_DEVICE;
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_scan_scratch);
+    if (e != cudaSuccess || p == nullptr) return MAMBA_ERR_CUDA;
+    *addr = p;
     return MAMBA_OK;
 }
 

@@ -28,7 +28,8 @@
 //      the output tile;
 //   4. the tile is written with coalesced 16-byte stores.
 // Shared arrays are padded so that every quarter-warp access is free of bank
-// conflicts.
+// conflicts.  fp32 activations take the accurate decay and softplus of
+// device_math.cuh (Decay<true>) in place of the MUFU ones.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -141,6 +142,8 @@ template <typename T, int R, bool SP, bool GATE, bool CONV>
 __global__ void __launch_bounds__(kWarps * 32, LanesOccupancy<R>::kBlocks)
 scan_fwd_pairs_kernel(const Params p) {
     using W = PairSmem<T, R>;
+    constexpr bool ACC = sizeof(T) == 4;
+    using Dk = Decay<ACC>;
     constexpr int kTC = W::kTC, V = W::V, CPR = W::CPR, CW = W::CW;
     constexpr int S = kNS / R;   // states per lane
     constexpr int OWN = 8 / R;   // outputs per lane per block of 8 timesteps
@@ -203,7 +206,7 @@ scan_fwd_pairs_kernel(const Params p) {
                 const int n0 = S * sr + 2 * k, n1 = n0 + 1;
                 const float a0 = (ds < Dm && n0 < N) ? __ldg(p.A + ds * N + n0) : 0.f;
                 const float a1 = (ds < Dm && n1 < N) ? __ldg(p.A + ds * N + n1) : 0.f;
-                A2[k] = make_float2(a0 * kLog2e, a1 * kLog2e);
+                A2[k] = make_float2(a0 * Dk::kScale, a1 * Dk::kScale);
             }
             bias_p = (dp < Dm && p.delta_bias) ? __ldg(p.delta_bias + dp) : 0.f;
             D_s = (ds < Dm && p.D) ? __ldg(p.D + ds) : 0.f;
@@ -377,7 +380,7 @@ scan_fwd_pairs_kernel(const Params p) {
 #pragma unroll
                 for (int e = 0; e < V; e += 2) {  // element pairs on the packed x2 instructions
                     float2 x = __fadd2_rn(f2(fd[e], fd[e + 1]), f2(bias_p, bias_p));
-                    if (SP) x = softplus2_f(x);
+                    if (SP) x = Dk::softplus2(x);
                     if (tvalid < kTC) {  // past the end: Abar = 1, no input
                         x.x = (tt + e < tvalid) ? x.x : 0.f;
                         x.y = (tt + e + 1 < tvalid) ? x.y : 0.f;
@@ -433,17 +436,22 @@ scan_fwd_pairs_kernel(const Params p) {
                             const float2 du2 = make_float2(dq[e].z, dq[e].w);
                             const float2 x0 = __fmul2_rn(dl2, A2[2 * q]);
                             const float2 x1 = __fmul2_rn(dl2, A2[2 * q + 1]);
-                            const float2 a0 = make_float2(ex2_mufu(x0.x), ex2_mufu(x0.y));
-                            // state-only runs lean harder on the MUFU (no readout or
-                            // gate work beside it): one decay pair in eight goes
-                            // to the FMA-pipe exp2 there
-                            float2 a1;
-                            if (SO && q == S / 4 - 1 && (e & 1) == 0) a1 = ex2_poly2(x1);
-                            else a1 = make_float2(ex2_mufu(x1.x), ex2_mufu(x1.y));
                             const float2 bu0 = __fmul2_rn(du2, make_float2(bb.x, bb.y));
                             const float2 bu1 = __fmul2_rn(du2, make_float2(bb.z, bb.w));
-                            h[2 * q] = __ffma2_rn(a0, h[2 * q], bu0);
-                            h[2 * q + 1] = __ffma2_rn(a1, h[2 * q + 1], bu1);
+                            if (ACC) {
+                                h[2 * q] = Dk::step2(x0, h[2 * q], bu0);
+                                h[2 * q + 1] = Dk::step2(x1, h[2 * q + 1], bu1);
+                            } else {
+                                const float2 a0 = make_float2(ex2_mufu(x0.x), ex2_mufu(x0.y));
+                                // state-only runs lean harder on the MUFU (no readout or
+                                // gate work beside it): one decay pair in eight goes
+                                // to the FMA-pipe exp2 there
+                                float2 a1;
+                                if (SO && q == S / 4 - 1 && (e & 1) == 0) a1 = ex2_poly2(x1);
+                                else a1 = make_float2(ex2_mufu(x1.x), ex2_mufu(x1.y));
+                                h[2 * q] = __ffma2_rn(a0, h[2 * q], bu0);
+                                h[2 * q + 1] = __ffma2_rn(a1, h[2 * q + 1], bu1);
+                            }
                             if (!SO) {
                                 const float4 cc = *reinterpret_cast<const float4 *>(sC + to);
                                 y2[e] = __ffma2_rn(make_float2(cc.x, cc.y), h[2 * q], y2[e]);
@@ -532,8 +540,10 @@ scan_fwd_pairs_kernel(const Params p) {
             float2 hend[S / 2];
 #pragma unroll
             for (int k = 0; k < S / 2; ++k) {
-                const float2 decay = f2(ex2_mufu((float)((double)A2[k].x * dsum)),
-                                        ex2_mufu((float)((double)A2[k].y * dsum)));
+                // exp(A sum(delta)): fp64 for fp32 activations, else one ex2 each
+                const float2 decay = ACC ? f2((float)exp((double)A2[k].x * dsum), (float)exp((double)A2[k].y * dsum))
+                                         : f2(ex2_mufu((float)((double)A2[k].x * dsum)),
+                                              ex2_mufu((float)((double)A2[k].y * dsum)));
                 hend[k] = __ffma2_rn(decay, hin[k], h[k]);
                 h[k] = hin[k];
             }

@@ -20,6 +20,8 @@
 //     rows that the scan reads with broadcast loads;
 //   * epilogue: out = (y + D u) * silu(z) from the scan's fp32 readouts and the
 //     staged u / z rows, packed and stored to global memory.
+// fp32 activations take the accurate decay and softplus of device_math.cuh
+// (Decay<true>) for all 16 states instead.
 // The pair hands sub-chunks back and forth through two processed-data slots,
 // each guarded by a pair of mbarriers (full: helper -> scan, done: scan ->
 // helper).  Every wait is bounded in time; a timeout raises the error word.
@@ -290,7 +292,7 @@ struct Helper {
 #pragma unroll
         for (int t = 0; t < kTC; t += 2) {
             float2 x = __fadd2_rn(f2(fd[t], fd[t + 1]), f2(bias, bias));
-            if (SP) x = softplus2_f(x);
+            if (SP) x = Decay<sizeof(T) == 4>::softplus2(x);
             x.x = t < d.tvalid ? x.x : 0.f;  // past the end: decay 1, no input
             x.y = t + 1 < d.tvalid ? x.y : 0.f;
             const float2 xu = __fmul2_rn(x, f2(fu[t], fu[t + 1]));
@@ -422,7 +424,7 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
                         const int n0 = 2 * q, n1 = 2 * q + 1;
                         const float a0 = (dc < p.dim && n0 < N) ? __ldg(p.A + (int64_t)dc * N + n0) : 0.f;
                         const float a1 = (dc < p.dim && n1 < N) ? __ldg(p.A + (int64_t)dc * N + n1) : 0.f;
-                        A2[q] = f2(a0 * kLog2e, a1 * kLog2e);
+                        A2[q] = f2(a0 * Decay<sizeof(T) == 4>::kScale, a1 * Decay<sizeof(T) == 4>::kScale);
                     }
                 }
                 if (d.j == 0) {  // the initial state, or zeros
@@ -464,13 +466,18 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
                         const float4 cc = *reinterpret_cast<const float4 *>(sC + t * kNS + 4 * q);
                         const float2 x0 = __fmul2_rn(f2(dl, dl), A2[2 * q]);
                         const float2 x1 = __fmul2_rn(f2(dl, dl), A2[2 * q + 1]);
-                        const float2 a0 = f2(ex2_mufu(x0.x), ex2_mufu(x0.y));
-                        // states 14 and 15 on the FMA pipe
-                        const float2 a1 = q == kNS / 4 - 1 ? ex2_poly2(x1) : f2(ex2_mufu(x1.x), ex2_mufu(x1.y));
                         const float2 bu0 = __fmul2_rn(f2(du, du), f2(bb.x, bb.y));
                         const float2 bu1 = __fmul2_rn(f2(du, du), f2(bb.z, bb.w));
-                        hs[2 * q] = __ffma2_rn(a0, hs[2 * q], bu0);
-                        hs[2 * q + 1] = __ffma2_rn(a1, hs[2 * q + 1], bu1);
+                        if (sizeof(T) == 4) {  // fp32 activations: the accurate decay
+                            hs[2 * q] = Decay<true>::step2(x0, hs[2 * q], bu0);
+                            hs[2 * q + 1] = Decay<true>::step2(x1, hs[2 * q + 1], bu1);
+                        } else {
+                            const float2 a0 = f2(ex2_mufu(x0.x), ex2_mufu(x0.y));
+                            // states 14 and 15 on the FMA pipe
+                            const float2 a1 = q == kNS / 4 - 1 ? ex2_poly2(x1) : f2(ex2_mufu(x1.x), ex2_mufu(x1.y));
+                            hs[2 * q] = __ffma2_rn(a0, hs[2 * q], bu0);
+                            hs[2 * q + 1] = __ffma2_rn(a1, hs[2 * q + 1], bu1);
+                        }
                         y2[e] = __ffma2_rn(f2(cc.x, cc.y), hs[2 * q], y2[e]);
                         y2[e] = __ffma2_rn(f2(cc.z, cc.w), hs[2 * q + 1], y2[e]);
                     }

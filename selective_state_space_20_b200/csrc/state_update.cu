@@ -11,7 +11,8 @@
 // readout is summed over its lanes with shuffles.  A rows are re-read by
 // every batch row and stay in L2, B and C rows are shared by all channels of a
 // batch row and stay in L1.  Other state sizes and unaligned tensors take a
-// thread-per-row kernel.
+// thread-per-row kernel.  fp32 activations take the accurate decay of
+// device_math.cuh (Decay<true>), bf16 ones one ex2 per state.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -46,12 +47,13 @@ state_update_kernel(const SUParams p) {
     const T *gB = static_cast<const T *>(p.B) + b * N;
     const T *gC = static_cast<const T *>(p.C) + b * N;
     const float *Ad = p.A + d * N;
+    using Dk = Decay<sizeof(T) == 4>;
 
     float dl = Elem<T>::load(gd + row) + (p.delta_bias ? __ldg(p.delta_bias + d) : 0.f);
-    if (p.softplus) dl = softplus_f(dl);
+    if (p.softplus) dl = Dk::softplus(dl);
     const float ut = Elem<T>::load(gu + row);
     const float du = dl * ut;
-    const float dl2 = dl * kLog2e;
+    const float dl2 = dl * Dk::kScale;
     float *st = p.state + row * N;
     float y = 0.f;
     if (NV > 0) {
@@ -63,16 +65,14 @@ state_update_kernel(const SUParams p) {
             const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float a = ex2_mufu(dl2 * av[i]);
-                hv[i] = fmaf(a, hv[i], du * Elem<T>::load(gB + n + i));
+                hv[i] = Dk::step(dl2 * av[i], hv[i], du * Elem<T>::load(gB + n + i));
                 y = fmaf(Elem<T>::load(gC + n + i), hv[i], y);
             }
             *reinterpret_cast<float4 *>(st + n) = make_float4(hv[0], hv[1], hv[2], hv[3]);
         }
     } else {
         for (int n = 0; n < N; ++n) {
-            const float a = ex2_mufu(dl2 * __ldg(Ad + n));
-            const float hn = fmaf(a, st[n], du * Elem<T>::load(gB + n));
+            const float hn = Dk::step(dl2 * __ldg(Ad + n), st[n], du * Elem<T>::load(gB + n));
             st[n] = hn;
             y = fmaf(Elem<T>::load(gC + n), hn, y);
         }
@@ -112,22 +112,23 @@ state_update_lanes_kernel(const SUParams p) {
     const T *gu = static_cast<const T *>(p.u);
     const T *gd = static_cast<const T *>(p.delta);
     const T *gz = static_cast<const T *>(p.z);
+    using Dk = Decay<sizeof(T) == 4>;
 
     float dl = Elem<T>::load(gd + row) + (p.delta_bias ? __ldg(p.delta_bias + d) : 0.f);
-    if (p.softplus) dl = softplus_f(dl);
+    if (p.softplus) dl = Dk::softplus(dl);
     const float ut = Elem<T>::load(gu + row);
     const float du = dl * ut;
-    const float dl2 = dl * kLog2e;
+    const float dl2 = dl * Dk::kScale;
     float4 *st = reinterpret_cast<float4 *>(p.state + row * NV) + qi;
     const float4 h4 = *st;
     const float4 a4 = __ldg(reinterpret_cast<const float4 *>(p.A + d * NV) + qi);
     const float4 b4 = Quad<T>::load(static_cast<const T *>(p.B) + b * NV + 4 * qi);
     const float4 c4 = Quad<T>::load(static_cast<const T *>(p.C) + b * NV + 4 * qi);
     float4 hn;
-    hn.x = fmaf(ex2_mufu(dl2 * a4.x), h4.x, du * b4.x);
-    hn.y = fmaf(ex2_mufu(dl2 * a4.y), h4.y, du * b4.y);
-    hn.z = fmaf(ex2_mufu(dl2 * a4.z), h4.z, du * b4.z);
-    hn.w = fmaf(ex2_mufu(dl2 * a4.w), h4.w, du * b4.w);
+    hn.x = Dk::step(dl2 * a4.x, h4.x, du * b4.x);
+    hn.y = Dk::step(dl2 * a4.y, h4.y, du * b4.y);
+    hn.z = Dk::step(dl2 * a4.z, h4.z, du * b4.z);
+    hn.w = Dk::step(dl2 * a4.w, h4.w, du * b4.w);
     float y = fmaf(c4.x, hn.x, fmaf(c4.y, hn.y, fmaf(c4.z, hn.z, c4.w * hn.w)));
 #pragma unroll
     for (int o = Q / 2; o >= 1; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);

@@ -4,32 +4,35 @@ Accepted error: max relative error <= 1e-4 for fp32 inputs and <= 2e-2 for
 bf16 inputs with fp32 accumulation.  A plain max |y - r| / |r| is undefined
 where the reference crosses zero (y_t = sum_n C_n h_n + D u is a sum of ~17
 terms of either sign and cancels freely), so the relative error of each
-element is taken against max(|r|, FLOOR * rms(r)) with FLOOR = 0.1: an element
-below a tenth of the typical magnitude is judged by its absolute error at
-that level.  A smaller floor would fail exact fp32 arithmetic itself: a
-correctly rounded fp32 evaluation of the recurrence (every product, sum and
-exp rounded once) already shows absolute errors of ~5e-7 * rms on outputs
-near zero, i.e. 5e-5 at a 1e-2 floor, and the 2^-22 relative error of a
-hardware exp2 lifts that to ~2e-4.
+element is taken against max(|r|, FLOOR * rms(r)) with FLOOR = 1e-2: an
+element below a hundredth of the typical magnitude is judged by its absolute
+error at that level.  A correctly rounded fp32 evaluation of the recurrence
+(every product, sum and exponential rounded once) measures up to ~5e-5 on
+this metric for the tiny fp32 workload and N up to 64, so the fp32 kernels
+take an unbiased decay (Abar - 1 on the FMA pipe) rather than the special
+function unit's exp2, whose 2^-22 error alone lifts the same runs to ~2e-4.
+
+``rel_err(got, ref, floor=0.1)`` gives the same metric at a tenth of the
+typical magnitude; the tests record it beside the gated figure.
 """
 from __future__ import annotations
 
 import numpy as np
 import torch
 
-FLOOR = 0.1
+FLOOR = 1e-2
 TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
 
 
-def rel_err(got, ref) -> float:
-    """max_i |got_i - ref_i| / max(|ref_i|, FLOOR * rms(ref))."""
+def rel_err(got, ref, floor: float = FLOOR) -> float:
+    """max_i |got_i - ref_i| / max(|ref_i|, floor * rms(ref))."""
     g = np.asarray(got, dtype=np.float64)
     r = np.asarray(ref, dtype=np.float64)
     assert g.shape == r.shape, (g.shape, r.shape)
     if r.size == 0:
         return 0.0
     rms = float(np.sqrt(np.mean(r * r)))
-    den = np.maximum(np.abs(r), FLOOR * rms)
+    den = np.maximum(np.abs(r), floor * rms)
     den = np.where(den > 0, den, 1.0)
     return float(np.max(np.abs(g - r) / den))
 

@@ -38,8 +38,10 @@ def check_full(w: inputs.ScanWorkload, softplus=True, drop=(), **kw):
     torch.cuda.synchronize()
     ro, rs = oracle_full(cpu, softplus=softplus)
     tol = TOL[inputs.DTYPES[w.dtype]]
-    e_out, e_state = rel_err(to_np(out), ro), rel_err(to_np(last), rs)
-    record(f"{w.name} {kw} drop={drop}", out=e_out, state=e_state)
+    go, gs = to_np(out), to_np(last)
+    e_out, e_state = rel_err(go, ro), rel_err(gs, rs)
+    record(f"{w.name} {kw} drop={drop}", out=e_out, state=e_state,
+           out_floor_0_1=rel_err(go, ro, floor=0.1), state_floor_0_1=rel_err(gs, rs, floor=0.1))
     assert e_out <= tol and e_state <= tol, (w.name, kw, e_out, e_state)
     return e_out, e_state
 
@@ -69,6 +71,16 @@ def test_tiny_odd_lengths_and_states(dtype, L, dstate):
 def test_every_dstate(dstate):
     check_full(inputs.custom(2, 19, 100, dstate, "fp32", seed=dstate))
     check_full(inputs.custom(2, 19, 104, dstate, "bf16", seed=dstate + 100))
+
+
+@pytest.mark.parametrize("dstate", [16, 24, 32, 64])
+@pytest.mark.parametrize("seed", [0, 1, 2, 3, 4])
+def test_fp32_large_dstate_several_seeds(dstate, seed):
+    """fp32 at the 1e-4 bar with the fast-decaying states of A = -(n + 1) up
+    to n = 63 (decay exponents down to ~-20 per step), five seeds each, on
+    the tiny workload's shape and its distributions."""
+    check_full(inputs.custom(1, 64, 256, dstate, "fp32", seed=1000 * dstate + seed, d_mode="ones"))
+    check_full(inputs.custom(2, 40, 256, dstate, "fp32", seed=2000 * dstate + seed))
 
 
 def _lane_configs():

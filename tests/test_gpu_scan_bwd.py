@@ -46,9 +46,17 @@ def check_bwd(batch, dim, L, N, dtype, seed, gate=True, softplus=True, dlast=Tru
         errs[k] = rel_err(to_np(got[k]), ref[k])
     record(f"scan_bwd {batch}x{dim}x{L} N{N} {dtype} gate={gate} sp={softplus} dlast={dlast} h0={h0}", **errs)
     for k, e in errs.items():
-        tol = TOL[inputs.DTYPES[dtype]] if k in ACT_GRADS else 1e-3
-        assert e <= tol, (k, e, errs)
+        assert e <= grad_tol(k, dtype), (k, e, errs)
     return errs
+
+
+def grad_tol(name, dtype):
+    """The activation-dtype bar (1e-4 fp32, 2e-2 bf16) for every gradient of
+    fp32 inputs; with bf16 inputs the fp32 parameter gradients (sums over
+    channels and time) are held to 1e-3, stricter than the bf16 bar."""
+    if dtype == "fp32" or name in ACT_GRADS:
+        return TOL[inputs.DTYPES[dtype]]
+    return 1e-3
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
@@ -133,4 +141,4 @@ def test_bwd_benchmark_layer_sampled():
     errs.update({k: rel_err(to_np(got[k][chans]), r[k]) for k in ("dA", "dD", "ddelta_bias")})
     record("scan_bwd mamba-2.8b layer sampled channels", **errs)
     for k, e in errs.items():
-        assert e <= (TOL[torch.bfloat16] if k in ACT_GRADS else 1e-3), (k, e, errs)
+        assert e <= grad_tol(k, "bf16"), (k, e, errs)
