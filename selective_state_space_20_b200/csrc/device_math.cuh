@@ -102,16 +102,19 @@ __device__ __forceinline__ float2 silu2_f(float2 z) {
 // keeps its sign over those steps becomes an error of e / (1 - Abar) in h --
 // ex2.approx's bias of a few 2^-24 grows to ~1e-4 and beyond over a few
 // hundred steps, where a correctly rounded decay stays near 5e-5.  So with
-// fp32 activations the kernels advance a state as h + ((Abar - 1) h + b),
-// Abar - 1 from expm1_f below: its error is relative to the small change of
-// h per step, not to h, and it carries no bias.  bf16 activations keep the
-// single MUFU op per decay.
+// fp32 activations the kernels advance a state whose decay is near 1 as
+// h + ((Abar - 1) h + b), Abar - 1 from expm1_poly below: its error is
+// relative to the small change of h per step, not to h, and carries no bias.
+// A decay far from 1 (|delta A| > 1, Abar < e^-1) is used as Abar itself from
+// the MUFU exponential: such a state forgets within a step or two, so no
+// bias can build up, and fma(Abar, h, b) keeps the relative accuracy of a
+// tiny Abar h that the difference form would lose.  bf16 activations keep
+// the single MUFU op per decay.
 
-// e^x - 1 = x + x^2 P(x) on |x| <= 1, P the degree-6 Chebyshev interpolant of
+// e^x - 1 = x + x^2 P(x) for |x| <= 1, P the degree-6 Chebyshev interpolant of
 // (e^x - 1 - x) / x^2 (coefficients from fit_expm1_poly.py in this directory;
-// relative error <= 1.6e-7 in fp32 however close x is to 0); elsewhere e^x - 1
-// from the MUFU exponential, whose error is then relative to |e^x - 1| >= 0.63.
-__device__ __forceinline__ float expm1_f(float x) {
+// relative error <= 1.6e-7 in fp32 however close x is to 0).
+__device__ __forceinline__ float expm1_poly(float x) {
     float p = 2.528843470e-05f;
     p = fmaf(p, x, 2.032904158e-04f);
     p = fmaf(p, x, 1.388644800e-03f);
@@ -119,9 +122,7 @@ __device__ __forceinline__ float expm1_f(float x) {
     p = fmaf(p, x, 4.166669771e-02f);
     p = fmaf(p, x, 1.666669697e-01f);
     p = fmaf(p, x, 5.000000000e-01f);
-    float em1 = fmaf(x * x, p, x);
-    if (fabsf(x) > 1.f) em1 = __expf(x) - 1.f;
-    return em1;
+    return fmaf(x * x, p, x);
 }
 
 // softplus with CUDA's full-precision expf and log1pf (errors of an ulp or
@@ -134,26 +135,28 @@ __device__ __forceinline__ float softplus_precise(float x) {
 // One state's step h <- Abar h + b with Abar = e^x, x = delta * A * kScale.
 //   ACC = false (bf16 activations): A is pre-scaled by log2 e and Abar comes
 //     from one ex2 on the MUFU; h <- fma(Abar, h, b).
-//   ACC = true (fp32 activations): A is used as is; h <- h + fma(e^x - 1, h, b).
+//   ACC = true (fp32 activations): A is used as is; for |x| <= 1
+//     h <- h + fma(e^x - 1, h, b), else h <- fma(e^x, h, b).
 template <bool ACC>
 struct Decay {
     static constexpr float kScale = ACC ? 1.f : kLog2e;
+    __device__ __forceinline__ static bool near_one(float x) { return fabsf(x) <= 1.f; }
     __device__ __forceinline__ static float step(float x, float h, float b) {
-        if (ACC) return h + fmaf(expm1_f(x), h, b);
+        if (ACC) return near_one(x) ? h + fmaf(expm1_poly(x), h, b) : fmaf(__expf(x), h, b);
         return fmaf(ex2_mufu(x), h, b);
     }
     __device__ __forceinline__ static float2 step2(float2 x, float2 h, float2 b) {
-        if (ACC) return __fadd2_rn(h, __ffma2_rn(f2(expm1_f(x.x), expm1_f(x.y)), h, b));
+        if (ACC) return f2(step(x.x, h.x, b.x), step(x.y, h.y, b.y));
         return __ffma2_rn(f2(ex2_mufu(x.x), ex2_mufu(x.y)), h, b);
     }
     // v * Abar (the adjoint's decay in the backward pass)
     __device__ __forceinline__ static float scale(float x, float v) {
-        if (ACC) return fmaf(expm1_f(x), v, v);
+        if (ACC) return near_one(x) ? fmaf(expm1_poly(x), v, v) : __expf(x) * v;
         return ex2_mufu(x) * v;
     }
     // Abar itself
     __device__ __forceinline__ static float abar(float x) {
-        if (ACC) return 1.f + expm1_f(x);
+        if (ACC) return near_one(x) ? 1.f + expm1_poly(x) : __expf(x);
         return ex2_mufu(x);
     }
     // softplus of the step's raw value

@@ -12,20 +12,19 @@
 //
 // With bf16 activations each state-step costs three special-function ops
 // (ex2, sin, cos) instead of one, so the kernel is bound by the MUFU at a
-// third of the real scan's rate; with fp32 activations they run on the FMA
-// pipe instead.  Layout of the work as in the real static kernel: a block
+// third of the real scan's rate.  With fp32 activations the state, the decay
+// and the readout are carried in fp64 (see kF64 below).  Layout of the work as in the real static kernel: a block
 // owns one batch row and CG = 128 / R channels, R lanes per channel split the 16
 // (padded) states, tiles of 32 timesteps are copied to shared memory with
 // 16-byte cp.async into a double buffer; a prologue forms delta and delta*u
 // once per element and widens B / C to fp32 [t][n] complex pairs shared by
 // every channel of the block; partial readouts of a channel's R lanes are
 // summed with a transposed butterfly; the epilogue applies D and the gate.
-// bf16 activations take Abar from the special-function unit; fp32 ones
-// advance the state by (Abar - 1) h with Abar - 1 from FMA-pipe polynomials
-// (abar_minus_one says why).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "device_math.cuh"
 #include "internal.h"
@@ -48,18 +47,24 @@ struct CParams {
     int dstate, softplus, vec;
 };
 
+// fp32 activations carry delta, delta * u, the states and the readout in
+// fp64 (see the kernel), bf16 ones in fp32.
+template <typename T>
+using CHi = typename std::conditional<sizeof(T) == 4, double, float>::type;
+
 template <typename T, int R>
 struct CGeom {
+    using H = CHi<T>;
     static constexpr int S = kCNP / R;                  // complex states per lane
     static constexpr int CG = kCThreads / R;            // channels per block
     static constexpr int V = 16 / (int)sizeof(T);       // elements per 16 bytes
     static constexpr int TC = kCTC;
-    static constexpr int TCP = TC + 4;                  // fp32 row pitch
+    static constexpr int TCP = TC + 4;                  // delta / delta u / y row pitch (elements of H)
     static constexpr int VPR = TC / V;                  // vectors per channel row per chunk
     static constexpr int BVR = 2 * TC / V;              // vectors per B / C state row per chunk
     static constexpr int STAGE = 3 * CG * TC + 2 * kCNP * 2 * TC;  // raw elements per stage
     static constexpr size_t SMEM =
-        (size_t)2 * CG * TCP * 4 + (size_t)2 * TC * kCNP * 8 + (size_t)2 * STAGE * sizeof(T);
+        (size_t)2 * CG * TCP * sizeof(H) + (size_t)2 * TC * kCNP * 8 + (size_t)2 * STAGE * sizeof(T);
 };
 
 __device__ __forceinline__ void cpa16(void *smem, const void *gmem, bool pred) {
@@ -84,82 +89,29 @@ __device__ __forceinline__ float reduce_angle(float x) {
     return fmaf(-k, kTwoPiLo, fmaf(-k, kTwoPiHi, x));
 }
 
-// sin t, cos t and cos t - 1 on the FMA pipe (|t| < 2^21).  Quadrant q =
-// rint(2 t / pi) (adding 1.5 * 2^23 rounds to an integer held in the low
-// bits), r = t - q pi / 2 by Cody-Waite with pi / 2 split in a float head and
-// tail, so |r| <= pi / 4; sin r = r P(r^2), cos r - 1 = r^2 G(r^2), P and G
-// the degree-3 Chebyshev fits from fit_sincos_poly.py in this directory
-// (relative errors <= 9.3e-8 and 1.4e-7 in fp32); the quadrant then swaps
-// and negates the pair.  In quadrant 0, cos t - 1 is r^2 G(r^2) itself,
-// accurate however small; elsewhere |cos t - 1| >= 1 - cos(pi / 4) and c - 1
-// is.
-__device__ __forceinline__ void sincos_cm1(float t, float &s, float &c, float &cm1) {
-    constexpr float kRound = 12582912.f;  // 1.5 * 2^23
-    constexpr float kTwoOverPi = 0.636619772367581343f;
-    constexpr float kPio2Hi = 1.57079637050628662f;
-    constexpr float kPio2Lo = -4.37113900018624284e-08f;
-    const float tq = fmaf(t, kTwoOverPi, kRound);
-    const float q = tq - kRound;
-    const unsigned qi = __float_as_uint(tq);  // low bits: q mod 4
-    float r = fmaf(-q, kPio2Hi, t);
-    r = fmaf(-q, kPio2Lo, r);
-    const float r2 = r * r;
-    float ps = -1.950390433e-04f;
-    ps = fmaf(ps, r2, 8.332035504e-03f);
-    ps = fmaf(ps, r2, -1.666665077e-01f);
-    ps = fmaf(ps, r2, 1.0f);
-    const float sr = r * ps;
-    float pc = 2.446378858e-05f;
-    pc = fmaf(pc, r2, -1.388758887e-03f);
-    pc = fmaf(pc, r2, 4.166664928e-02f);
-    pc = fmaf(pc, r2, -0.5f);
-    const float cm1r = r2 * pc;
-    const float cr = fmaf(pc, r2, 1.0f);
-    const bool swap = (qi & 1u) != 0;
-    const float s0 = swap ? cr : sr, c0 = swap ? sr : cr;
-    s = __uint_as_float(__float_as_uint(s0) ^ ((qi & 2u) << 30));        // negate in quadrants 2, 3
-    c = __uint_as_float(__float_as_uint(c0) ^ (((qi + 1u) & 2u) << 30));  // negate in quadrants 1, 2
-    cm1 = (qi & 3u) == 0 ? cm1r : c - 1.f;
-}
-
-// The fp32 path's softplus is softplus_precise (device_math.cuh): a relative
-// error e in delta turns the rotation of a state with frequency Im A by
-// e * delta * Im A per step, and over the ~1 / (delta |Re A|) steps the state
-// remembers by e * Im A / |Re A| -- a factor of ~100 for the highest
-// frequencies of the usual complex initialisation.  The one-op softplus_f has
-// e up to 8.5e-7 for very negative inputs, enough to show at fp32 tolerance;
-// softplus_precise keeps e near 1e-7.
-
-// Abar - 1 for x = delta Re A, t = delta Im A, as (re, im):
-//   e^x cos t - 1 = em1 cos t + (cos t - 1),   e^x sin t = (1 + em1) sin t,
-// em1 = e^x - 1 from expm1_f (device_math.cuh: accurate relative to its own
-// size near x = 0).  The state then advances as h + (Abar - 1) h: a
-// step's error is relative to the small change of h, not to h.  A decay
-// rounded to fp32 near 1 would carry the same relative error, 2^-24 or more,
-// into h at every step, and those errors add up over the ~1 / (delta |Re A|)
-// steps a state remembers -- the limit of the plain form in fp32.
-__device__ __forceinline__ void abar_minus_one(float x, float t, float &dr, float &di) {
-    const float em1 = expm1_f(x);
-    float s, c, cm1;
-    sincos_cm1(t, s, c, cm1);
-    dr = fmaf(em1, c, cm1);
-    di = fmaf(em1, s, s);
-}
-
 template <typename T, int R>
 __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CParams p) {
     using G = CGeom<T, R>;
     constexpr int S = G::S, CG = G::CG, V = G::V, TC = G::TC, TCP = G::TCP;
     constexpr int VPR = G::VPR, BVR = G::BVR, STAGE = G::STAGE;
     constexpr int OWN = 4 / R;  // outputs per lane per 4 timesteps
-    // fp32 activations: Abar - 1 from FMA-pipe polynomials (abar_minus_one);
-    // bf16, whose tolerance is 200x looser: Abar from the special-function
-    // unit (ex2, sin, cos)
-    constexpr bool kAccurate = sizeof(T) == 4;
+    // fp32 activations (tolerance 1e-4): delta, delta * u, the states, the
+    // decay and the readout in fp64.  The complex recurrence amplifies
+    // relative errors: a relative error e in delta turns a state by
+    // e Im A / |Re A| over the ~1 / (delta |Re A|) steps it remembers (~100 e
+    // for the highest frequencies of the usual initialisation), and an error
+    // in a rotation angle or a bias in a decay adds up over those steps.
+    // Exact arithmetic with delta alone rounded once to fp32 already measures
+    // up to 4e-4 against the fp64 definition on long rows; in fp64 only the
+    // final rounding of each output to fp32 remains.  bf16 activations
+    // (tolerance 2e-2): everything in fp32, Abar from the special-function
+    // unit (ex2, sin, cos).
+    constexpr bool kF64 = sizeof(T) == 4;
+    using H = CHi<T>;
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    float *sDelta = reinterpret_cast<float *>(smem_raw);       // [CG][TCP]: delta, then y
-    float *sDu = sDelta + CG * TCP;                            // [CG][TCP]: delta * u
+    H *sDelta = reinterpret_cast<H *>(smem_raw);               // [CG][TCP]: delta, then y
+    H *sDu = sDelta + CG * TCP;                                // [CG][TCP]: delta * u
     float2 *sB = reinterpret_cast<float2 *>(sDu + CG * TCP);   // [TC][kCNP]
     float2 *sC = sB + TC * kCNP;                               // [TC][kCNP]
     T *rawBase = reinterpret_cast<T *>(sC + TC * kCNP);        // 2 stages
@@ -183,12 +135,13 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
     // ---- this thread: channel c, lane r, complex states r*S .. r*S+S-1
     const int c = tid / R, r = tid % R;
     const int64_t d = d0 + c;
-    float Are[S], Aim[S], hr[S], hi[S];
+    float Are[S], Aim[S];
+    H hr[S], hi[S];
 #pragma unroll
     for (int s = 0; s < S; ++s) {
         const int n = r * S + s;
         const bool ok = d < Dm && n < N;
-        Are[s] = ok ? __ldg(p.A + (d * N + n) * 2) * (kAccurate ? 1.f : kLog2e) : 0.f;
+        Are[s] = ok ? __ldg(p.A + (d * N + n) * 2) * (kF64 ? 1.f : kLog2e) : 0.f;
         Aim[s] = ok ? __ldg(p.A + (d * N + n) * 2 + 1) : 0.f;
         hr[s] = (ok && p.h0) ? __ldcg(p.h0 + ((b * Dm + d) * N + n) * 2) : 0.f;
         hi[s] = (ok && p.h0) ? __ldcg(p.h0 + ((b * Dm + d) * N + n) * 2 + 1) : 0.f;
@@ -261,20 +214,25 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
             float fu[V], fd[V];
             Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + pc * TC + tv * V), fu);
             Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rD + pc * TC + tv * V), fd);
+            H hd[V], hu[V];
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                float dl = fd[i] + bias;
-                if (p.softplus) dl = kAccurate ? softplus_precise(dl) : softplus_f(dl);
+                H dl;
+                if constexpr (kF64) {
+                    dl = (double)fd[i] + (double)bias;
+                    if (p.softplus) dl = fmax(dl, 0.0) + log1p(exp(-fabs(dl)));
+                } else {
+                    dl = fd[i] + bias;
+                    if (p.softplus) dl = softplus_f(dl);
+                }
                 if (tv * V + i >= tvalid) dl = 0.f;  // past the end: Abar = 1, no input
-                fd[i] = dl;
-                fu[i] = dl * fu[i];
+                hd[i] = dl;
+                hu[i] = dl * (H)fu[i];
             }
 #pragma unroll
-            for (int i = 0; i < V; i += 4) {
-                *reinterpret_cast<float4 *>(sDelta + pc * TCP + tv * V + i) =
-                    make_float4(fd[i], fd[i + 1], fd[i + 2], fd[i + 3]);
-                *reinterpret_cast<float4 *>(sDu + pc * TCP + tv * V + i) =
-                    make_float4(fu[i], fu[i + 1], fu[i + 2], fu[i + 3]);
+            for (int i = 0; i < V; ++i) {
+                sDelta[pc * TCP + tv * V + i] = hd[i];
+                sDu[pc * TCP + tv * V + i] = hu[i];
             }
         }
         for (int vi = tid; vi < 2 * kCNP * BVR; vi += kCThreads) {
@@ -292,21 +250,23 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
 
         // ---- scan: thread (c, r) advances its S complex states
         {
-            float *dRow = sDelta + c * TCP;
-            const float *uRow = sDu + c * TCP;
+            H *dRow = sDelta + c * TCP;
+            const H *uRow = sDu + c * TCP;
 #pragma unroll 1
             for (int tb = 0; tb < tvalid; tb += 4) {
-                const float4 dl4 = *reinterpret_cast<const float4 *>(dRow + tb);
-                const float4 du4 = *reinterpret_cast<const float4 *>(uRow + tb);
-                const float dls[4] = {dl4.x, dl4.y, dl4.z, dl4.w};
-                const float dus[4] = {du4.x, du4.y, du4.z, du4.w};
-                float yp[4];
+                H dls[4], dus[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float dl = dls[q], du = dus[q];
+                    dls[q] = dRow[tb + q];
+                    dus[q] = uRow[tb + q];
+                }
+                H yp[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const H dl = dls[q], du = dus[q];
                     const float4 *Bt = reinterpret_cast<const float4 *>(sB + (tb + q) * kCNP + r * S);
                     const float4 *Ct = reinterpret_cast<const float4 *>(sC + (tb + q) * kCNP + r * S);
-                    float y = 0.f;
+                    H y = 0.f;
 #pragma unroll
                     for (int s2 = 0; s2 < S / 2; ++s2) {  // two complex states per 16-byte read
                         const float4 bb = Bt[s2], cc = Ct[s2];
@@ -315,12 +275,15 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
 #pragma unroll
                         for (int k = 0; k < 2; ++k) {
                             const int s = 2 * s2 + k;
-                            float nr, ni;
-                            if (kAccurate) {
-                                float dr, di;
-                                abar_minus_one(dl * Are[s], dl * Aim[s], dr, di);
-                                nr = hr[s] + fmaf(dr, hr[s], fmaf(-di, hi[s], du * br[k]));
-                                ni = hi[s] + fmaf(dr, hi[s], fmaf(di, hr[s], du * bi[k]));
+                            H nr, ni;
+                            if constexpr (kF64) {
+                                const double mag = exp(dl * (double)Are[s]);
+                                double sn, cs;
+                                sincos(dl * (double)Aim[s], &sn, &cs);
+                                const double ar = mag * cs, ai = mag * sn;
+                                nr = fma(ar, hr[s], fma(-ai, hi[s], du * (double)br[k]));
+                                ni = fma(ar, hi[s], fma(ai, hr[s], du * (double)bi[k]));
+                                y = fma((double)cr[k], nr, fma(-(double)ci[k], ni, y));
                             } else {
                                 const float mag = ex2_mufu(dl * Are[s]);
                                 float sn, cs;
@@ -328,10 +291,10 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
                                 const float ar = mag * cs, ai = mag * sn;
                                 nr = fmaf(ar, hr[s], fmaf(-ai, hi[s], du * br[k]));
                                 ni = fmaf(ar, hi[s], fmaf(ai, hr[s], du * bi[k]));
+                                y = fmaf(cr[k], nr, fmaf(-ci[k], ni, y));
                             }
                             hr[s] = nr;
                             hi[s] = ni;
-                            y = fmaf(cr[k], nr, fmaf(-ci[k], ni, y));
                         }
                     }
                     yp[q] = y;
@@ -342,18 +305,18 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
                     const bool up = (r & 2) != 0;
 #pragma unroll
                     for (int i = 0; i < 2; ++i) {
-                        const float send = up ? yp[i] : yp[i + 2];
-                        const float keep = up ? yp[i + 2] : yp[i];
+                        const H send = up ? yp[i] : yp[i + 2];
+                        const H keep = up ? yp[i + 2] : yp[i];
                         yp[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
                     }
                 }
                 if (R >= 2) {
-                    constexpr int H = R >= 4 ? 1 : 2;  // live values per lane after the round
+                    constexpr int HV = R >= 4 ? 1 : 2;  // live values per lane after the round
                     const bool up = (r & 1) != 0;
 #pragma unroll
-                    for (int i = 0; i < H; ++i) {
-                        const float send = up ? yp[i] : yp[i + H];
-                        const float keep = up ? yp[i + H] : yp[i];
+                    for (int i = 0; i < HV; ++i) {
+                        const H send = up ? yp[i] : yp[i + HV];
+                        const H keep = up ? yp[i + HV] : yp[i];
                         yp[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
                     }
                 }
@@ -376,9 +339,15 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
             if (has_z) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rZ + pc * TC + tv * V), fz);
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                float o = fmaf(Dd, fu[i], sDelta[pc * TCP + tv * V + i]);
-                if (has_z) o *= silu_f(fz[i]);
-                y[i] = o;
+                if constexpr (kF64) {
+                    double o = fma((double)Dd, (double)fu[i], sDelta[pc * TCP + tv * V + i]);
+                    if (has_z) o *= (double)fz[i] / (1.0 + exp(-(double)fz[i]));
+                    y[i] = (float)o;
+                } else {
+                    float o = fmaf(Dd, fu[i], sDelta[pc * TCP + tv * V + i]);
+                    if (has_z) o *= silu_f(fz[i]);
+                    y[i] = o;
+                }
             }
             T *dst = gout + row0 + pc * L + t;
             if (p.vec) {
@@ -397,8 +366,8 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
         for (int s = 0; s < S; ++s) {
             const int n = r * S + s;
             if (n < N) {
-                ls[2 * n] = hr[s];
-                ls[2 * n + 1] = hi[s];
+                ls[2 * n] = (float)hr[s];
+                ls[2 * n + 1] = (float)hi[s];
             }
         }
     }
