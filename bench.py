@@ -4,9 +4,12 @@
 One "step" is one fused scan launch (softplus -> discretisation -> recurrence
 -> readout -> D skip -> silu gate -> last state) over the Mamba-2.8B layer
 shape: batch 4, 5120 channels (d_model 2560, expand 2), L = 4096, N = 16,
-bf16 activations, fp32 state and arithmetic.  Inputs are synthetic and
-seeded, resident in HBM, and larger than L2 (504 MB of u/delta/z), so no L2
-flush is needed between steps.
+bf16 activations, fp32 state and arithmetic, through the C ABI's
+mamba_scan_fwd (no workspace).  Inputs are synthetic and seeded, resident in
+HBM, and larger than L2 (504 MB of u/delta/z), so no L2 flush is needed
+between steps.  Sections beside the headline time the same call on the
+Mamba-130M layer and the long-context shape, the workspace entry point, the
+decode step, the conv1d prologue, the backward and the complex mode.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -175,6 +178,62 @@ class ClockSampler:
                 "power_w_max": max(pw) if pw else None}
 
 
+class NvmlSampler:
+    """SM clock and clock-event reasons read through NVML every ~1 ms in a
+    thread: the timed region of a short run (tens of ms) is far shorter than
+    nvidia-smi's sampling period."""
+    # NVML clock-event reason bits
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device: torch.device):
+        self.samples = []
+        self.handle = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.nvml = pynvml
+        except Exception:
+            self.handle = None
+
+    def start(self):
+        if self.handle is None:
+            return
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+                self.samples.append((time.time(), sm, mx, rs))
+            except Exception:
+                return
+            time.sleep(0.001)
+
+    def stop(self):
+        self._stop.set()
+
+    def summary(self, t0, t1):
+        inside = [x for x in self.samples if t0 <= x[0] <= t1]
+        if not inside:
+            return None
+        sm = [x[1] for x in inside]
+        reasons = sorted({name for x in inside for bit, name in self.REASONS.items() if x[3] & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[2] for x in inside),
+                "sm_mhz_min": min(sm), "reasons": reasons, "samples": len(inside), "source": "nvml"}
+
+
 # ------------------------------------------------------------ distributed
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -238,7 +297,12 @@ def oracle_beside(kind: str, w, k: int = 32):
     cores = os.cpu_count() or 1
     sw = dataclasses.replace(w, dim=min(k, w.dim))
     elems = sw.batch * sw.dim * sw.seqlen
-    if kind == "backward":
+    if kind == "scan":
+        d = inputs.scan_inputs(sw)
+        t0 = time.perf_counter()
+        oracle.scan(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"], delta_bias=d["delta_bias"],
+                    nthreads=cores)
+    elif kind == "backward":
         d = inputs.scan_inputs(sw)
         g = torch.Generator().manual_seed(7)
         dout = torch.randn(sw.batch, sw.dim, sw.seqlen, generator=g)
@@ -343,9 +407,8 @@ def scan_call(ins, out, last, ws=None):
 def time_device(w, ins, steps, warmup):
     out = torch.empty_like(ins["u"])
     last = torch.empty(w.batch, w.dim, w.dstate, device=ins["u"].device)
-    ws = workspace_for(w, ins["u"].device)
     for _ in range(warmup):
-        scan_call(ins, out, last, ws)
+        scan_call(ins, out, last)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
@@ -382,6 +445,82 @@ def e2e_measure(w, dev_ins, steps):
     torch.cuda.synchronize()
     ms = s.elapsed_time(e) / steps
     return ms, h2d, d2h
+
+
+def _median_us(fn, reps, warmup=3):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in ev:
+        a.record(st)
+        fn()
+        b.record(st)
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+
+
+def scan_kernel_name(lanes, sched):
+    if sched in (binding.SCHEDULE_PERSISTENT, binding.SCHEDULE_LOCAL):
+        return "scan_fwd_pairs_kernel" if lanes > 1 else "scan_fwd_spec_kernel"
+    return "scan_fwd_kernel"
+
+
+SCHED_NAMES = {1: "static", 2: "persistent (device-wide, workspace)", 3: "local (block per SM, no workspace)"}
+
+
+def layer_measure(w, reps, oracle_k, cpu_oracle=True):
+    """One more Mamba-layer shape through mamba_scan_fwd (no workspace):
+    median CUDA-event time of `reps` launches (inputs larger than L2, or
+    re-read from L2 at most once per launch: see `l2`), Gelem/s, algorithmic
+    GB/s, the MUFU roofline, and the oracle on a fixed sample of the shape."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ins = inputs.scan_inputs(w, device=dev)
+    out = torch.empty_like(ins["u"])
+    last = torch.empty(w.batch, w.dim, w.dstate, device=dev)
+    us = _median_us(lambda: scan_call(ins, out, last), reps)
+    peaks = load_peaks()
+    mufu = MUFU_PER_CLK_PER_SM * SM_COUNT * peaks["sm_max_mhz"] * 1e6 / w.dstate / 1e9
+    gel = w.elements / (us * 1e-6) / 1e9
+    alg = algorithmic_bytes(w)
+    lanes, threads, sched = binding.mamba_scan_plan(w.batch, w.dim, w.seqlen, w.dstate, inputs.DTYPES[w.dtype],
+                                                    workspace=False)
+    kernel = scan_kernel_name(lanes, sched)
+    if binding.device_status() != 0:
+        raise SystemExit(f"{w.name}: the scan reported a timeout")
+    act_bytes = 3 * w.elements * (2 if w.dtype == "bf16" else 4)
+    sec = {"workload": w.name, "entry": "mamba_scan_fwd", "us_per_call": us, "value": gel, "unit": UNIT,
+           "reps": reps, "gbs": alg / (us * 1e-6) / 1e9,
+           "l2": "inputs larger than L2" if act_bytes > 126e6 else
+                 f"inputs {act_bytes / 1e6:.0f} MB: may stay partly in L2 between launches",
+           "launch": {"schedule": SCHED_NAMES.get(sched, sched), "lanes_per_channel": lanes,
+                      "threads_per_block": threads},
+           "roofline": {"bound": "alu", "achieved": gel, "peak": mufu, "unit": UNIT, "frac": gel / mufu,
+                        "kernel": kernel, "traffic": measured_traffic(f"{kernel} {w.name}"),
+                        "hbm": {"algorithmic_bytes_per_launch": alg, "frac": alg / (us * 1e-6) / 1e9 /
+                                peaks["hbm_gbs"]}}}
+    del ins, out, last
+    torch.cuda.empty_cache()
+    if cpu_oracle:
+        sec["cpu_oracle"] = oracle_beside("scan", w, k=oracle_k)
+    return sec
+
+
+def workspace_measure(w, ins, reps):
+    """The Mamba-2.8B layer through mamba_scan_fwd_ws (caller workspace,
+    device-wide persistent schedule) beside the headline's no-workspace call."""
+    out = torch.empty_like(ins["u"])
+    last = torch.empty(w.batch, w.dim, w.dstate, device=ins["u"].device)
+    ws = workspace_for(w, ins["u"].device)
+    us = _median_us(lambda: scan_call(ins, out, last, ws), reps)
+    if binding.workspace_status(ws) != 0:
+        raise SystemExit("persistent scan reported a timeout")
+    lanes, threads, sched = binding.mamba_scan_plan(w.batch, w.dim, w.seqlen, w.dstate, inputs.DTYPES[w.dtype])
+    return {"entry": "mamba_scan_fwd_ws", "us_per_call": us, "value": w.elements / (us * 1e-6) / 1e9,
+            "unit": UNIT, "reps": reps, "workspace_bytes": ws.numel(),
+            "launch": {"schedule": SCHED_NAMES.get(sched, sched), "lanes_per_channel": lanes,
+                       "threads_per_block": threads}}
 
 
 def decode_measure(steps=256):
@@ -592,6 +731,7 @@ def main():
     ap.add_argument("--no-conv", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-complex", action="store_true")
+    ap.add_argument("--no-layers", action="store_true", help="skip the Mamba-130M / long-context / workspace sections")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -612,8 +752,10 @@ def main():
     out, last, starts, ends, stream = time_device(w, ins, args.steps, args.warmup)
 
     clocks = ClockSampler(local)
+    nvml = NvmlSampler(dev)
     if rank == 0:
         clocks.start()
+        nvml.start()
         time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize()
@@ -621,10 +763,9 @@ def main():
     g0 = torch.cuda.Event(enable_timing=True)
     g1 = torch.cuda.Event(enable_timing=True)
     g0.record(stream)
-    ws = workspace_for(w, dev)
     for i in range(args.steps):
         starts[i].record(stream)
-        scan_call(ins, out, last, ws)
+        scan_call(ins, out, last)
         ends[i].record(stream)
     g1.record(stream)
     torch.cuda.synchronize()
@@ -634,7 +775,12 @@ def main():
     launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(total_ms, world)
     clk = clocks.summary(t_wall0, t_wall1) if rank == 0 else None
+    nvml.stop()
     clocks.stop()
+    if rank == 0:
+        fast = nvml.summary(t_wall0, t_wall1)
+        if fast:  # NVML samples inside the timed region decide; nvidia-smi's kept beside
+            clk = dict(fast, nvidia_smi=clk)
 
     ms_step = total_ms / args.steps
     elems = w.elements
@@ -644,13 +790,11 @@ def main():
     mufu_peak_gelem = MUFU_PER_CLK_PER_SM * SM_COUNT * peaks["sm_max_mhz"] * 1e6 / w.dstate / 1e9
     achieved = elems / (avg_launch_ms * 1e-3) / 1e9
     alg_bytes = algorithmic_bytes(w)
-    lanes, threads, sched = binding.mamba_scan_plan(w.batch, w.dim, w.seqlen, w.dstate, inputs.DTYPES[w.dtype])
-    if binding.workspace_status(ws) != 0:
-        raise SystemExit("persistent scan reported a timeout")
-    if sched == binding.SCHEDULE_PERSISTENT:
-        kernel = "scan_fwd_pairs_kernel" if lanes > 1 else "scan_fwd_spec_kernel"
-    else:
-        kernel = "scan_fwd_kernel"
+    lanes, threads, sched = binding.mamba_scan_plan(w.batch, w.dim, w.seqlen, w.dstate, inputs.DTYPES[w.dtype],
+                                                    workspace=False)
+    if binding.device_status() != 0:
+        raise SystemExit("the scan reported a timeout")
+    kernel = scan_kernel_name(lanes, sched)
     roof = {"bound": "alu", "achieved": achieved, "peak": mufu_peak_gelem, "unit": UNIT,
             "frac": achieved / mufu_peak_gelem,
             "traffic": measured_traffic(f"{kernel} {w.name}"),
@@ -671,7 +815,8 @@ def main():
                        "dstate": w.dstate, "act_dtype": w.dtype, "state_dtype": "f32",
                        "gate": True, "softplus": True, "emit_last_state": True,
                        "l2": "inputs larger than L2 (3 x 168 MB act tensors), no flush",
-                       "launch": {"schedule": {1: "static", 2: "persistent"}.get(sched, sched),
+                       "entry": "mamba_scan_fwd (C ABI, no workspace)",
+                       "launch": {"schedule": SCHED_NAMES.get(sched, sched),
                                   "lanes_per_channel": lanes, "threads_per_block": threads},
                        "per_rank": "independent problem of this shape (seed + rank)"},
             "gpu_launches": args.steps, "roofline": roof, "clocks": clk}
@@ -684,6 +829,9 @@ def main():
                        "ms_per_step": ms_e2e, "steps": e2e_steps,
                        "path": "mamba_scan_fwd_host: pinned host buffers in and out; copies in, scans and "
                                "copies out pipelined over 16 chunks on three streams"}
+    if rank == 0 and not args.no_layers:
+        line["with_workspace"] = workspace_measure(w, ins, reps=50)
+        line["with_workspace"]["vs_headline"] = line["with_workspace"]["us_per_call"] / (avg_launch_ms * 1e3)
     if rank == 0 and not args.no_decode:
         line["decode"] = decode_measure()
     if rank == 0 and not args.no_conv:
@@ -692,6 +840,12 @@ def main():
         line["backward"] = backward_measure()
     if rank == 0 and not args.no_complex:
         line["complex"] = complex_measure()
+    if rank == 0 and not args.no_layers:
+        del ins
+        torch.cuda.empty_cache()
+        with_oracle = world == 1 and not args.no_cpu_baseline
+        line["mamba_130m"] = layer_measure(inputs.MAMBA_130M, reps=50, oracle_k=64, cpu_oracle=with_oracle)
+        line["long_context"] = layer_measure(inputs.LONG_CONTEXT, reps=5, oracle_k=32, cpu_oracle=with_oracle)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         for key, kind in (("conv1d", "conv1d"), ("backward", "backward"), ("complex", "complex")):
             if key in line:

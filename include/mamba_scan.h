@@ -25,7 +25,8 @@
  *                     schedule), _noalloc, _init (from a given state),
  *                     _strided (any strides), _complex (complex mode),
  *                     _conv (causal conv1d + silu fused in), _host (sequences
- *                     in host memory); mamba_scan_plan, mamba_scan_workspace_size,
+ *                     in host memory); mamba_scan_plan, mamba_scan_plan_noworkspace,
+ *                     mamba_scan_workspace_size,
  *                     mamba_scan_host_scratch_size
  *   decoding          mamba_state_update (one token), mamba_conv1d_update
  *   conv1d            mamba_conv1d_fwd
@@ -59,9 +60,10 @@
  * - Calls are reentrant and thread-safe, with one exception:
  *   mamba_scan_fwd_noalloc calls share one scratch area per device, so the
  *   caller must serialise them (see there).  Library state: per device, the
- *   workspace pointer of the last persistent launch (for
- *   mamba_get_device_status) and the scratch area of mamba_scan_fwd_noalloc;
- *   process-wide, the mamba_debug_stall_group test hook (off by default).
+ *   workspace pointer of the last persistent launch and the local schedule's
+ *   timeout word (both for mamba_get_device_status), and the scratch area of
+ *   mamba_scan_fwd_noalloc; process-wide, the mamba_debug_stall_group test
+ *   hook (off by default).
  */
 #ifndef MAMBA_SCAN_H
 #define MAMBA_SCAN_H
@@ -101,20 +103,27 @@ typedef enum {
     MAMBA_SCHEDULE_AUTO = 0,
     MAMBA_SCHEDULE_STATIC = 1,     /* one block per channel group walks the whole
                                       sequence; no workspace */
-    MAMBA_SCHEDULE_PERSISTENT = 2  /* dstate <= 16: persistent warps, all
+    MAMBA_SCHEDULE_PERSISTENT = 2, /* dstate <= 16: persistent warps, all
                                       resident; 2 or 4 lanes per channel split
                                       the (channel group, sub-chunk) grid into
                                       equal contiguous shares, 1 lane per
                                       channel takes (group, time chunk) units
                                       from a ready queue; states pass between
                                       pieces through the workspace */
+    MAMBA_SCHEDULE_LOCAL = 3       /* dstate <= 16, 2 or 4 lanes per channel:
+                                      one block per SM takes whole channel
+                                      groups and splits their sub-chunks among
+                                      its own warps; states pass between
+                                      pieces through shared memory; no
+                                      workspace */
 } mamba_schedule_t;
 
 /* Optional launch tuning.  Zero fields mean "choose automatically".
  *   lanes_per_channel : threads sharing one channel's states.  Static
  *                       schedule: 1, 2, 4, 8 or 16 (the padded dstate must be
  *                       a multiple, and at most 16 states stay in one
- *                       thread).  Persistent schedule: 1, 2 or 4.
+ *                       thread).  Persistent schedule: 1, 2 or 4.  Local
+ *                       schedule: 2 or 4.
  *   threads_per_block : static schedule only: 128 or 256
  *   schedule          : a mamba_schedule_t
  *   chunk_timesteps   : persistent schedule only: timesteps per work unit
@@ -147,6 +156,13 @@ typedef struct {
  *   last_state   : fp32 (batch, dim, dstate) or NULL; receives h_{seqlen-1}.
  *   The state starts from zero.
  *
+ * Needs no workspace.  With dstate <= 16, 16-byte-aligned act tensors and
+ * seqlen a multiple of the 16-byte vector width, shapes with enough channels
+ * run the local schedule (MAMBA_SCHEDULE_LOCAL); others the static one.  A
+ * local launch whose bounded wait between warps ran out (it cannot, except
+ * under the mamba_debug_stall_group test hook) is reported by
+ * mamba_get_device_status.
+ *
  * Returns MAMBA_OK or a mamba_status_t error.
  */
 int mamba_scan_fwd(const void *u, const void *delta, const float *A,
@@ -174,6 +190,12 @@ int mamba_scan_fwd_tuned(const void *u, const void *delta, const float *A,
  * Returns MAMBA_OK or a validation error. */
 int mamba_scan_plan(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
                     int act_dtype, mamba_scan_tuning_t *plan);
+
+/* The launch configuration mamba_scan_fwd (no workspace) would pick for these
+ * sizes on the current device, with 16-byte-aligned tensors; as
+ * mamba_scan_plan otherwise. */
+int mamba_scan_plan_noworkspace(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                                int act_dtype, mamba_scan_tuning_t *plan);
 
 /* Bytes of device workspace mamba_scan_fwd_ws may use for these sizes (an
  * upper bound valid on every device); 0 when the persistent schedule never
@@ -426,10 +448,12 @@ int mamba_state_fold(const float *h_init, const double *delta_sums, const float 
 
 /* The device-side status of this process's work on the current device:
  * synchronises `stream`, then returns MAMBA_ERR_CUDA if the stream or the
- * context reports an error, MAMBA_ERR_TIMEOUT if the last persistent launch
- * on this device (any entry point that was given a workspace) gave up a
- * bounded wait -- the error word in its workspace, which must still be
- * allocated -- else MAMBA_OK.  No device code traps; this and
+ * context reports an error; MAMBA_ERR_TIMEOUT if a local-schedule launch
+ * (no workspace) on this device gave up a bounded wait since the previous
+ * call (a device word the library keeps; reading it clears it), or if the
+ * last persistent launch on this device (any entry point that was given a
+ * workspace) gave up one -- the error word in its workspace, which must
+ * still be allocated; else MAMBA_OK.  No device code traps; this and
  * mamba_scan_workspace_status are how failures surface. */
 int mamba_get_device_status(cudaStream_t stream);
 

@@ -26,11 +26,12 @@ STATUS_NAMES = {0: "MAMBA_OK", -1: "MAMBA_ERR_NULL", -2: "MAMBA_ERR_SHAPE",
                 -5: "MAMBA_ERR_CUDA", -6: "MAMBA_ERR_DEVICE", -7: "MAMBA_ERR_OVERLAP",
                 -8: "MAMBA_ERR_WORKSPACE", -9: "MAMBA_ERR_TIMEOUT"}
 MAMBA_ERR_TIMEOUT = -9
-SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT = 0, 1, 2
+SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT, SCHEDULE_LOCAL = 0, 1, 2, 3
 
 # Every function include/mamba_scan.h declares.
 EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
-            "mamba_scan_plan", "mamba_scan_workspace_size", "mamba_scan_workspace_status",
+            "mamba_scan_plan", "mamba_scan_plan_noworkspace", "mamba_scan_workspace_size",
+            "mamba_scan_workspace_status",
             "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_fwd_strided",
             "mamba_scan_fwd_complex", "mamba_delta_sum", "mamba_state_fold", "mamba_scan_fwd_conv",
             "mamba_scan_host_scratch_size", "mamba_scan_fwd_host", "mamba_debug_stall_group",
@@ -102,6 +103,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_fwd_noalloc.restype = ci
     lib.mamba_scan_plan.argtypes = [i64, i64, i64, i64, ci, ctypes.POINTER(Tuning)]
     lib.mamba_scan_plan.restype = ci
+    lib.mamba_scan_plan_noworkspace.argtypes = [i64, i64, i64, i64, ci, ctypes.POINTER(Tuning)]
+    lib.mamba_scan_plan_noworkspace.restype = ci
     lib.mamba_scan_workspace_size.argtypes = [i64, i64, i64, i64, ci]
     lib.mamba_scan_workspace_size.restype = ctypes.c_size_t
     lib.mamba_scan_workspace_status.argtypes = [vp, vp]
@@ -195,8 +198,11 @@ def mamba_scan_fwd(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
     Returns ``out`` (batch, dim, L), or ``(out, last_state)`` when
     ``return_last_state`` is set or ``last_state`` is passed.
 
-    A device workspace (``mamba_scan_workspace_size`` bytes, allocated here
-    with torch unless given) enables the persistent, load-balanced schedule;
+    Without a workspace the library picks the local schedule (one block per
+    SM splits whole channel groups among its warps, carries in shared memory)
+    or the static one.  A device workspace (``mamba_scan_workspace_size``
+    bytes; allocated here with torch when ``schedule`` is SCHEDULE_PERSISTENT
+    and none is given) enables the device-wide persistent schedule;
     ``schedule`` / ``lanes_per_channel`` / ``threads_per_block`` force a
     launch configuration (0 = automatic).
 
@@ -231,7 +237,7 @@ def mamba_scan_fwd(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
     _need(last_state, "last_state", dev, torch.float32, (batch, dim, N))
     _need(h0, "h0", dev, torch.float32, (batch, dim, N))
     lib = load_library()
-    if workspace is None and schedule != SCHEDULE_STATIC:
+    if workspace is None and schedule == SCHEDULE_PERSISTENT:
         nbytes = lib.mamba_scan_workspace_size(batch, dim, L, N, _ACT[act])
         if nbytes:
             workspace = torch.empty(nbytes, device=dev, dtype=torch.uint8)
@@ -568,12 +574,14 @@ def mamba_scan_workspace_size(batch: int, dim: int, seqlen: int, dstate: int,
 
 
 def mamba_scan_plan(batch: int, dim: int, seqlen: int, dstate: int,
-                    dtype: torch.dtype = torch.bfloat16) -> Tuple[int, int, int]:
+                    dtype: torch.dtype = torch.bfloat16, workspace: bool = True) -> Tuple[int, int, int]:
     """(lanes_per_channel, threads_per_block, schedule) the library picks for a
-    shape on the current device (given a workspace and aligned tensors)."""
+    shape on the current device, with aligned tensors and a workspace
+    (``workspace=False``: what the no-workspace call picks)."""
     t = Tuning()
-    _check("mamba_scan_plan", load_library().mamba_scan_plan(batch, dim, seqlen, dstate,
-                                                            _ACT[dtype], ctypes.byref(t)))
+    lib = load_library()
+    fn = lib.mamba_scan_plan if workspace else lib.mamba_scan_plan_noworkspace
+    _check("mamba_scan_plan", fn(batch, dim, seqlen, dstate, _ACT[dtype], ctypes.byref(t)))
     return t.lanes_per_channel, t.threads_per_block, t.schedule
 
 

@@ -66,7 +66,7 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
               const float *h0, void *out, float *last_state, int64_t batch, int64_t dim, int64_t seqlen,
               int64_t dstate, int act_dtype, const mamba_scan_tuning_t *tuning,
               void *workspace, size_t ws_bytes, cudaStream_t stream, bool launch,
-              mamba_scan_tuning_t *plan_out) {
+              mamba_scan_tuning_t *plan_out, bool plan_noworkspace = false) {
     if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
     int rc = check_sizes(batch, dim, seqlen, dstate);
     if (rc != MAMBA_OK) return rc;
@@ -113,7 +113,7 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
             return MAMBA_ERR_UNSUPPORTED;
         if (want_threads != 0 && want_threads != 128 && want_threads != 256)
             return MAMBA_ERR_UNSUPPORTED;
-        if (want_sched < MAMBA_SCHEDULE_AUTO || want_sched > MAMBA_SCHEDULE_PERSISTENT)
+        if (want_sched < MAMBA_SCHEDULE_AUTO || want_sched > MAMBA_SCHEDULE_LOCAL)
             return MAMBA_ERR_UNSUPPORTED;
     }
     int status = MAMBA_OK;
@@ -128,11 +128,35 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
     a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
 
     // Persistent schedule: needs a workspace (when launching), dstate <= 16,
-    // aligned tensors and enough channel groups to occupy every worker.
-    const bool ws_ok = !launch || (workspace != nullptr &&
+    // aligned tensors and enough channel groups to occupy every worker.  The
+    // local schedule (same kernel, no workspace) needs the same layout; it
+    // runs when no workspace is given.
+    const bool ws_ok = (!launch && !plan_noworkspace) || (workspace != nullptr &&
                                    ws_bytes >= mscan::persistent_workspace_bound(
                                                    batch, dim, seqlen, act_dtype));
     const bool supported = mscan::persistent_supported(a);
+    int local_lanes = 0;
+    if (want_sched == MAMBA_SCHEDULE_LOCAL) {
+        if (!supported || want_threads != 0 || (want_lanes != 0 && want_lanes != 2 && want_lanes != 4))
+            return MAMBA_ERR_UNSUPPORTED;
+        local_lanes = want_lanes != 0 ? want_lanes : mscan::local_choose_lanes(a, sms);
+        if (local_lanes == 0) local_lanes = 2;
+    } else if (want_sched == MAMBA_SCHEDULE_AUTO && want_lanes == 0 && want_threads == 0 &&
+               (launch || plan_noworkspace) && workspace == nullptr && supported) {
+        local_lanes = mscan::local_choose_lanes(a, sms);
+    }
+    if (local_lanes != 0) {
+        if (plan_out) {
+            plan_out->lanes_per_channel = local_lanes;
+            plan_out->threads_per_block = 32 * (local_lanes == 4 ? 12 : 8);
+            plan_out->schedule = MAMBA_SCHEDULE_LOCAL;
+            plan_out->chunk_timesteps = 0;
+        }
+        if (!launch) return MAMBA_OK;
+        note_workspace(nullptr);
+        return mscan::launch_scan_fwd_local(a, local_lanes, sms, stream) == cudaSuccess ? MAMBA_OK
+                                                                                        : MAMBA_ERR_CUDA;
+    }
     bool persist = false;
     int persist_lanes = 0;
     if (want_sched == MAMBA_SCHEDULE_PERSISTENT) {
@@ -523,6 +547,9 @@ int mamba_get_device_status(cudaStream_t stream) {
     if (sticky != cudaSuccess) return MAMBA_ERR_CUDA;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MAMBA_ERR_DEVICE;
+    const int local = mscan::local_error_take();  // block-local launches since the last call
+    if (local < 0) return MAMBA_ERR_CUDA;
+    if (local > 0) return MAMBA_ERR_TIMEOUT;
     const void *ws = (dev >= 0 && dev < kMaxDevices) ? g_last_workspace[dev] : nullptr;
     if (!ws) return MAMBA_OK;
     unsigned hdr[4] = {0, 0, 0, 0};
@@ -536,6 +563,14 @@ int mamba_scan_plan(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate, 
     return scan_impl(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 1,
                      nullptr, nullptr, nullptr, batch, dim, seqlen, dstate, act_dtype, nullptr, nullptr, 0,
                      nullptr, false, plan);
+}
+
+int mamba_scan_plan_noworkspace(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
+                                mamba_scan_tuning_t *plan) {
+    if (!plan) return MAMBA_ERR_NULL;
+    return scan_impl(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 1,
+                     nullptr, nullptr, nullptr, batch, dim, seqlen, dstate, act_dtype, nullptr, nullptr, 0,
+                     nullptr, false, plan, true);
 }
 
 int mamba_state_update(float *state, const void *u, const void *delta, const float *A,

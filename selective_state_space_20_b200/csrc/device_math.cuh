@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 namespace mscan {
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -136,14 +138,24 @@ __device__ __forceinline__ float softplus_precise(float x) {
 //   ACC = false (bf16 activations): A is pre-scaled by log2 e and Abar comes
 //     from one ex2 on the MUFU; h <- fma(Abar, h, b).
 //   ACC = true (fp32 activations): A is used as is; for |x| <= 1
-//     h <- h + fma(e^x - 1, h, b), else h <- fma(e^x, h, b).
+//     h <- h + fma(e^x - 1, h, b), else h <- fma(e^x, h, b).  The kernels keep
+//     such a state in fp64 (the double overload): in fp32, the rounding of h
+//     at every step, relative to the largest |h| the state reaches, adds up
+//     over the ~1 / (1 - Abar) steps it remembers to ~1e-4 of the typical
+//     magnitude -- the fp32 bar itself -- for a state that ends near zero.
+//     x, e^x - 1 and b stay fp32 (each rounded once per step, without bias).
 template <bool ACC>
 struct Decay {
     static constexpr float kScale = ACC ? 1.f : kLog2e;
+    // the state's type: fp64 for fp32 activations
+    using H = typename std::conditional<ACC, double, float>::type;
     __device__ __forceinline__ static bool near_one(float x) { return fabsf(x) <= 1.f; }
     __device__ __forceinline__ static float step(float x, float h, float b) {
         if (ACC) return near_one(x) ? h + fmaf(expm1_poly(x), h, b) : fmaf(__expf(x), h, b);
         return fmaf(ex2_mufu(x), h, b);
+    }
+    __device__ __forceinline__ static double step(float x, double h, float b) {
+        return near_one(x) ? h + fma((double)expm1_poly(x), h, (double)b) : fma((double)__expf(x), h, (double)b);
     }
     __device__ __forceinline__ static float2 step2(float2 x, float2 h, float2 b) {
         if (ACC) return f2(step(x.x, h.x, b.x), step(x.y, h.y, b.y));

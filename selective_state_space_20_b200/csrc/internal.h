@@ -133,4 +133,13 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
                                        void *workspace, size_t ws_bytes, int sm_count,
                                        cudaStream_t stream);
 
+// The lane-split kernel without a workspace: one block per SM takes whole
+// channel groups and splits them among its warps (dstate <= 16, the layout
+// rules of persistent_supported).  local_choose_lanes: 2 or 4, or 0 when the
+// static schedule should run.  local_error_take: 1 if a block-local launch on
+// the current device stopped waiting since the last call (then cleared).
+int local_choose_lanes(const ScanArgs &a, int sm_count);
+cudaError_t launch_scan_fwd_local(const ScanArgs &a, int lanes, int sm_count, cudaStream_t stream);
+int local_error_take();
+
 }  // namespace mscan

@@ -128,6 +128,12 @@ __device__ __forceinline__ void push_unit(const Params &p, int lane, unsigned ne
 // the sub-chunk position in progress[g]; the consumer waits until progress[g]
 // reaches its first sub-chunk.  Pieces of one group run strictly one after
 // the other, so the slot is never overwritten before it has been read.
+//
+// Block-local variant (no workspace): each block takes a contiguous range of
+// whole groups and splits it the same way among its own warps; a carried
+// state then only ever passes from warp w - 1 to warp w of one block, through
+// one shared-memory slot per warp boundary (a warp publishes at most once:
+// at the end of its range, if that falls inside a group).
 struct Piece {
     int g;       // group
     int sb, se;  // sub-chunks [sb, se) of the group
@@ -141,17 +147,18 @@ struct Range {
                          // sb > 0 means it continues another worker's piece
 };
 
-__device__ __forceinline__ Range worker_range(const Params &p, long long w, long long P) {
-    const long long S = p.subs_per_chain;
-    const long long T = (long long)p.n_groups * S;
+// Worker w of P over groups [g0, g0 + n_groups) of S sub-chunks each.
+__device__ __forceinline__ Range worker_range_of(long long n_groups, long long S, int g0, long long w,
+                                                 long long P) {
+    const long long T = n_groups * S;
     const long long s = w * T / P, e = (w + 1) * T / P;
     Range r;
     r.head = Piece{0, 0, 0};
     r.tail = Piece{0, 0, 0};
     r.full_b = r.full_e = 0;
     if (s >= e) return r;
-    const int cs = (int)(s / S), os = (int)(s % S);
-    const int ce = (int)(e / S), oe = (int)(e % S);
+    const int cs = g0 + (int)(s / S), os = (int)(s % S);
+    const int ce = g0 + (int)(e / S), oe = (int)(e % S);
     if (cs == ce) {  // inside one group
         r.tail = Piece{cs, os, oe};
         return r;
@@ -161,6 +168,11 @@ __device__ __forceinline__ Range worker_range(const Params &p, long long w, long
     r.full_e = ce;
     if (os > 0) r.tail = Piece{cs, os, (int)S};
     return r;
+}
+
+// Worker w of P over every group of the launch.
+__device__ __forceinline__ Range worker_range(const Params &p, long long w, long long P) {
+    return worker_range_of(p.n_groups, p.subs_per_chain, 0, w, P);
 }
 
 // Wait (lane 0 polls, bounded in time) until group g's carry covers sub-chunk

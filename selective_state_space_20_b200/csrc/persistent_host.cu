@@ -138,6 +138,65 @@ size_t persistent_workspace_bound(int64_t batch, int64_t dim, int64_t seqlen, in
     return m;
 }
 
+namespace {
+// Kernel parameters shared by both launch forms of the lane-split kernel and
+// the one-lane kernel (no workspace fields).
+persist::Params base_params(const ScanArgs &a, int lanes, int tc) {
+    persist::Params kp = {};
+    kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
+    kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias;
+    kp.out = a.out; kp.last_state = a.last_state; kp.h0 = a.h0;
+    kp.conv_w = a.conv_w; kp.conv_b = a.conv_b; kp.conv_k = a.conv_k; kp.u_out = a.u_out;
+    kp.u_bstride = a.u_bstride > 0 ? a.u_bstride : a.dim * a.seqlen;
+    kp.z_bstride = a.z_bstride > 0 ? a.z_bstride : a.dim * a.seqlen;
+    kp.dim = a.dim; kp.seqlen = a.seqlen; kp.dstate = a.dstate; kp.softplus = a.softplus;
+    kp.group_channels = group_channels(lanes);
+    kp.groups_per_batch = (int)((a.dim + kp.group_channels - 1) / kp.group_channels);
+    kp.n_groups = (int)n_groups(a.batch, a.dim, lanes);
+    kp.subs_per_chain = (int)((a.seqlen + tc - 1) / tc);
+    kp.stall_group = g_stall_group;
+    return kp;
+}
+}  // namespace
+
+// Block-local form.  Each of the min(SMs, groups) blocks takes whole groups,
+// so the slowest block holds ceil(groups / blocks) of them for its W warps.
+// Measured on B200 (Mamba layer shapes, N = 16): two lanes per channel when
+// those groups give every warp about one group or more (Mamba-2.8B: 9 groups
+// for 8 warps, 524 us); else four lanes (8-channel groups, 12 warps per
+// block) when they keep three quarters of the warps busy (Mamba-130M: 11
+// groups for 12 warps, 205 us against 240 us with two lanes); else, on rows
+// long enough for the two-phase pieces (>= 8 sub-chunks per warp), two lanes
+// again (long context: 6.35 ms against 7.38 ms with four); else the static
+// schedule, which splits states further.
+int local_choose_lanes(const ScanArgs &a, int sm_count) {
+    const int64_t g2 = n_groups(a.batch, a.dim, 2), g4 = n_groups(a.batch, a.dim, 4);
+    const int64_t w2 = local_split_warps(2), w4 = local_split_warps(4);
+    const int64_t b2 = g2 < sm_count ? g2 : sm_count, b4 = g4 < sm_count ? g4 : sm_count;
+    const int64_t per2 = (g2 + b2 - 1) / b2, per4 = (g4 + b4 - 1) / b4;  // groups of the busiest block
+    if (per2 * 10 >= w2 * 9) return 2;
+    if (per4 * 4 >= w4 * 3) return 4;
+    const int tc = sub_chunk(2, a.act);
+    if (g2 * ((a.seqlen + tc - 1) / tc) >= 8 * w2 * b2) return 2;
+    return 0;
+}
+
+cudaError_t launch_scan_fwd_local(const ScanArgs &a, int lanes, int sm_count, cudaStream_t st) {
+    if (lanes != 2 && lanes != 4) return cudaErrorInvalidValue;
+    if (a.conv_w && !a.softplus) return cudaErrorInvalidValue;
+    persist::Params kp = base_params(a, lanes, sub_chunk(lanes, a.act));
+    kp.n_chunks = 1;
+    kp.chunk_len = (int)a.seqlen;
+    kp.hdr = nullptr; kp.queue = nullptr; kp.progress = nullptr; kp.carry = nullptr;
+    return launch_local_split(kp, lanes, a.act, sm_count, st);
+}
+
+int local_error_take() {
+    unsigned v = 0;
+    if (take_local_error(&v) != 0) return -1;
+    return v != 0 ? 1 : 0;
+}
+
 cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_timesteps,
                                        void *workspace, size_t ws_bytes, int sm_count,
                                        cudaStream_t st) {
@@ -149,20 +208,8 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
     const int64_t groups = n_groups(a.batch, a.dim, lanes);
     const int tc = sub_chunk(lanes, a.act);
 
-    persist::Params kp;
-    kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
-    kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias;
-    kp.out = a.out; kp.last_state = a.last_state; kp.h0 = a.h0;
-    kp.conv_w = a.conv_w; kp.conv_b = a.conv_b; kp.conv_k = a.conv_k; kp.u_out = a.u_out;
-    kp.u_bstride = a.u_bstride > 0 ? a.u_bstride : a.dim * a.seqlen;
-    kp.z_bstride = a.z_bstride > 0 ? a.z_bstride : a.dim * a.seqlen;
     if (a.conv_w && (lanes == 1 || !a.softplus)) return cudaErrorInvalidValue;  // lane-split kernel, softplus on
-    kp.dim = a.dim; kp.seqlen = a.seqlen; kp.dstate = a.dstate; kp.softplus = a.softplus;
-    kp.group_channels = group_channels(lanes);
-    kp.groups_per_batch = (int)((a.dim + kp.group_channels - 1) / kp.group_channels);
-    kp.n_groups = (int)groups;
-    kp.subs_per_chain = (int)((a.seqlen + tc - 1) / tc);
-    kp.stall_group = g_stall_group;
+    persist::Params kp = base_params(a, lanes, tc);
     unsigned char *w = static_cast<unsigned char *>(workspace);
     kp.hdr = reinterpret_cast<unsigned *>(w);
 

@@ -22,4 +22,12 @@ int persistent_split_blocks_per_sm(int lanes);
 cudaError_t launch_persistent_split(const persist::Params &kp, int lanes, int act, int sm_count,
                                    cudaStream_t st);
 
+// The same kernel in its block-local form: one block per SM (LocalWarps
+// warps) splits whole channel groups among its warps; carries in shared
+// memory, no workspace.  take_local_error reads and clears the device word a
+// block-local launch sets when a bounded wait ran out.
+int local_split_warps(int lanes);
+cudaError_t launch_local_split(const persist::Params &kp, int lanes, int act, int sm_count, cudaStream_t st);
+int take_local_error(unsigned *flag);
+
 }  // namespace mscan

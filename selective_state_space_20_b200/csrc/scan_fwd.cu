@@ -175,7 +175,9 @@ scan_fwd_kernel(const KParams p) {
     // ---- scan identity: channel c, lane r, states r*S .. r*S+S-1
     const int c = tid / R, r = tid % R;
     const int64_t d = d0 + c;
-    float h[S], A2[S];
+    using HS = typename Dk::H;  // the state: fp64 for fp32 activations
+    HS h[S];
+    float A2[S];
 #pragma unroll
     for (int s = 0; s < S; ++s) {
         const int n = r * S + s;
@@ -336,18 +338,18 @@ scan_fwd_kernel(const KParams p) {
                 for (int q = 0; q < RB; q += 4) {
                     const float4 dl = *reinterpret_cast<const float4 *>(dRow + tb + q);
                     const float4 du = *reinterpret_cast<const float4 *>(uRow + tb + q);
-                    float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+                    HS y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
 #pragma unroll
                     for (int s = 0; s < S; ++s) {
                         const int n = r * S + s;
                         const float4 bb = *reinterpret_cast<const float4 *>(sB + n * TCP + tb + q);
                         const float4 cc = *reinterpret_cast<const float4 *>(sC + n * TCP + tb + q);
-                        h[s] = Dk::step(dl.x * A2[s], h[s], du.x * bb.x); y0 = fmaf(cc.x, h[s], y0);
-                        h[s] = Dk::step(dl.y * A2[s], h[s], du.y * bb.y); y1 = fmaf(cc.y, h[s], y1);
-                        h[s] = Dk::step(dl.z * A2[s], h[s], du.z * bb.z); y2 = fmaf(cc.z, h[s], y2);
-                        h[s] = Dk::step(dl.w * A2[s], h[s], du.w * bb.w); y3 = fmaf(cc.w, h[s], y3);
+                        h[s] = Dk::step(dl.x * A2[s], h[s], du.x * bb.x); y0 = fma((HS)cc.x, h[s], y0);
+                        h[s] = Dk::step(dl.y * A2[s], h[s], du.y * bb.y); y1 = fma((HS)cc.y, h[s], y1);
+                        h[s] = Dk::step(dl.z * A2[s], h[s], du.z * bb.z); y2 = fma((HS)cc.z, h[s], y2);
+                        h[s] = Dk::step(dl.w * A2[s], h[s], du.w * bb.w); y3 = fma((HS)cc.w, h[s], y3);
                     }
-                    yp[q] = y0; yp[q + 1] = y1; yp[q + 2] = y2; yp[q + 3] = y3;
+                    yp[q] = (float)y0; yp[q + 1] = (float)y1; yp[q + 2] = (float)y2; yp[q + 3] = (float)y3;
                 }
                 if (R > 1) transpose_reduce<R, RB>(yp, r);
                 __syncwarp();  // every lane of the channel has read dRow[tb .. tb+RB)
@@ -429,7 +431,7 @@ scan_fwd_kernel(const KParams p) {
 #pragma unroll
         for (int s = 0; s < S; ++s) {
             const int n = r * S + s;
-            if (n < N) ls[n] = h[s];
+            if (n < N) ls[n] = (float)h[s];
         }
     }
 }

@@ -13,7 +13,15 @@
 //
 // Work: the balanced split of persistent_common.cuh -- each warp runs a
 // contiguous share of the (channel group, sub-chunk) grid, at most three
-// pieces.  Per piece, per sub-chunk of TC timesteps:
+// pieces.  Two launch forms:
+//   * device-wide (LOCAL = false): every resident warp of the device takes a
+//     share of all groups; carried states pass between warps through the
+//     caller's workspace (cooperative launch, blocks of kWarps warps);
+//   * block-local (LOCAL = true): one block per SM of LocalWarps<R> warps
+//     takes a contiguous range of whole groups and splits it among its own
+//     warps, so carried states only pass between warps of one block, through
+//     shared memory -- no workspace at all.
+// Per piece, per sub-chunk of TC timesteps:
 //   1. cp.async stages the raw u / delta / z rows and the B / C rows of the
 //      next sub-chunk (double buffer) while this one is processed;
 //   2. prologue: B and C are widened to fp32 as [t][n] rows for broadcast
@@ -33,6 +41,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "device_math.cuh"
 #include "internal.h"
@@ -138,12 +148,93 @@ template <int R> struct LanesOccupancy;
 template <> struct LanesOccupancy<2> { static constexpr int kBlocks = 2; };
 template <> struct LanesOccupancy<4> { static constexpr int kBlocks = 3; };
 
-template <typename T, int R, bool SP, bool GATE, bool CONV>
-__global__ void __launch_bounds__(kWarps * 32, LanesOccupancy<R>::kBlocks)
+// Block-local form: warps per block (one block per SM, the same warps per SM
+// as the device-wide form's kBlocks x kWarps).
+template <int R> struct LocalWarps;
+template <> struct LocalWarps<2> { static constexpr int value = 8; };
+template <> struct LocalWarps<4> { static constexpr int value = 12; };
+
+template <int R, bool LOCAL>
+struct PairLaunch {
+    static constexpr int kWorkers = LOCAL ? LocalWarps<R>::value : kWarps;  // warps per block
+    static constexpr int kMinBlocks = LOCAL ? 1 : LanesOccupancy<R>::kBlocks;
+};
+
+// Block-local carries: slot w holds what warp w hands on to the next warp
+// with a non-empty share ([32 lanes][16 / R floats]), then one flag word per
+// slot (the sub-chunk position the carry covers; 0 = not yet published) and
+// the block's abort word (set by a warp whose wait ran out).
+template <int R>
+struct LocalSmem {
+    static constexpr int SLOTS = LocalWarps<R>::value * 32 * (kNS / R) * 4;
+    static constexpr int FLAGS = ((LocalWarps<R>::value + 1) * 4 + 15) / 16 * 16;
+    static constexpr int BYTES = SLOTS + FLAGS;
+};
+
+// Set by a block-local launch whose bounded wait ran out (read and cleared by
+// take_local_error).
+__device__ unsigned g_local_error;
+
+// Block-local wait (lane 0 polls the shared flag, bounded in time) until the
+// warp before has published the carry covering sub-chunk position `pos`.  A
+// wait that runs out raises the device error word and the block's abort
+// word; every other waiter of the block then gives up at once.
+__device__ __forceinline__ bool local_wait(volatile unsigned *flag, volatile unsigned *abort_word, int lane,
+                                           unsigned pos) {
+    unsigned ok = 1;
+    if (lane == 0) {
+        if (*flag != pos) {
+            unsigned long long t0, t;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+            unsigned ns = 32;
+            while (*flag != pos) {
+                asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+                if (*abort_word != 0u) {
+                    ok = 0;
+                    break;
+                }
+                if (t - t0 > 2000000000ull) {
+                    atomicOr(&g_local_error, 1u);
+                    *abort_word = 1u;
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(ns);
+                if (ns < 1024) ns <<= 1;
+            }
+        }
+        __threadfence_block();  // the slot's contents are read after the flag
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+// Block-local publish: every lane has written its part of the slot.
+__device__ __forceinline__ void local_publish(volatile unsigned *flag, int lane, unsigned pos) {
+    __syncwarp();
+    if (lane == 0) {
+        __threadfence_block();
+        *flag = pos;
+    }
+}
+
+template <typename T, int R, bool SP, bool GATE, bool CONV, bool LOCAL>
+__global__ void __launch_bounds__(PairLaunch<R, LOCAL>::kWorkers * 32, PairLaunch<R, LOCAL>::kMinBlocks)
 scan_fwd_pairs_kernel(const Params p) {
     using W = PairSmem<T, R>;
+    constexpr int kWorkers = PairLaunch<R, LOCAL>::kWorkers;
     constexpr bool ACC = sizeof(T) == 4;
     using Dk = Decay<ACC>;
+    // a lane's states as pairs: fp32 (packed x2 arithmetic) for bf16
+    // activations, fp64 for fp32 ones (Decay's note says why)
+    using HV = typename std::conditional<ACC, double2, float2>::type;
+    auto hv = [](float a, float b) {
+        HV r;
+        r.x = a;
+        r.y = b;
+        return r;
+    };
     constexpr int kTC = W::kTC, V = W::V, CPR = W::CPR, CW = W::CW;
     constexpr int S = kNS / R;   // states per lane
     constexpr int OWN = 8 / R;   // outputs per lane per block of 8 timesteps
@@ -165,6 +256,14 @@ scan_fwd_pairs_kernel(const Params p) {
     const T *gC = static_cast<const T *>(p.C);
     T *gout = static_cast<T *>(p.out);
 
+    // block-local carry slots and flags, after the warps' areas
+    float *lslots = reinterpret_cast<float *>(smem + kWorkers * W::BYTES);
+    volatile unsigned *lflags = reinterpret_cast<volatile unsigned *>(smem + kWorkers * W::BYTES + LocalSmem<R>::SLOTS);
+    if (LOCAL) {  // slot flags, then the abort word
+        for (int i = threadIdx.x; i <= kWorkers; i += blockDim.x) lflags[i] = 0u;
+        __syncthreads();
+    }
+
     const int sc = lane / R, sr = lane % R;    // scan: channel, state slice
     const int pc = lane % CW, ph = lane / CW;  // prologue: channel, timestep slice
 
@@ -176,12 +275,29 @@ scan_fwd_pairs_kernel(const Params p) {
     // This worker's share of the balanced split: head, whole groups, tail.
     // Piece: sub-chunks [sb, se) of group g, carried state in from sub-chunk
     // sb and out at se (or the final state when se is the group's end).
-    const long long n_workers = (long long)gridDim.x * kWarps;
-    const Range rg = worker_range(p, (long long)blockIdx.x * kWarps + warp, n_workers);
+    long long n_workers, scope_groups;
+    Range rg;
+    int producer = warp - 1;  // LOCAL: the warp whose share ends where this one's starts
+    if (LOCAL) {  // this block's whole groups [gb, ge), split among its warps
+        const long long G = p.n_groups, nb = gridDim.x;
+        const int gb = (int)((long long)blockIdx.x * G / nb);
+        const int ge = (int)(((long long)blockIdx.x + 1) * G / nb);
+        n_workers = kWorkers;
+        scope_groups = ge - gb;
+        rg = worker_range_of(scope_groups, p.subs_per_chain, gb, warp, n_workers);
+        // with fewer sub-chunks than warps some shares are empty: skip them
+        const long long T = scope_groups * (long long)p.subs_per_chain;
+        while (producer > 0 && ((long long)producer + 1) * T / n_workers == (long long)producer * T / n_workers)
+            --producer;
+    } else {
+        n_workers = (long long)gridDim.x * kWarps;
+        scope_groups = p.n_groups;
+        rg = worker_range(p, (long long)blockIdx.x * kWarps + warp, n_workers);
+    }
     // Shares shorter than ~0.55 of a group: waiting for the piece before
     // would chain a group's pieces end to end (the group's full length); the
     // two-phase pieces below cost ~1.8x their length but all run at once.
-    const bool two_phase = 20LL * p.n_groups < 11LL * n_workers;
+    const bool two_phase = 20LL * scope_groups < 11LL * n_workers;
     const int has_head = rg.head.se > 0 ? 1 : 0;
     const int n_pieces = has_head + (rg.full_e - rg.full_b) + (rg.tail.se > 0 ? 1 : 0);
 #pragma unroll 1
@@ -219,20 +335,37 @@ scan_fwd_pairs_kernel(const Params p) {
             }
         }
 
-        float *carry = p.carry + ((int64_t)g * 32 + lane) * S;
-        auto load_carry = [&](float2 (&hh)[S / 2]) {
+        // the carried state in (from the worker before) and out (to the one
+        // after): the group's workspace slot, or this block's shared slots
+        float *carry_in = LOCAL ? lslots + ((int64_t)(producer > 0 ? producer : 0) * 32 + lane) * S
+                                : p.carry + ((int64_t)g * 32 + lane) * S;
+        float *carry_out = LOCAL ? lslots + ((int64_t)warp * 32 + lane) * S : carry_in;
+        auto load_carry = [&](HV (&hh)[S / 2]) {
 #pragma unroll
             for (int k = 0; k < S / 4; ++k) {
-                const float4 v = __ldcg(reinterpret_cast<const float4 *>(carry) + k);  // S/4 float4
-                hh[2 * k] = make_float2(v.x, v.y);
-                hh[2 * k + 1] = make_float2(v.z, v.w);
+                const float4 v = LOCAL ? reinterpret_cast<const float4 *>(carry_in)[k]
+                                       : __ldcg(reinterpret_cast<const float4 *>(carry_in) + k);  // S/4 float4
+                hh[2 * k] = hv(v.x, v.y);
+                hh[2 * k + 1] = hv(v.z, v.w);
             }
         };
-        auto store_carry = [&](const float2 (&hh)[S / 2]) {
+        auto store_carry = [&](const HV (&hh)[S / 2]) {
 #pragma unroll
-            for (int k = 0; k < S / 4; ++k)
-                __stcg(reinterpret_cast<float4 *>(carry) + k,
-                       make_float4(hh[2 * k].x, hh[2 * k].y, hh[2 * k + 1].x, hh[2 * k + 1].y));
+            for (int k = 0; k < S / 4; ++k) {
+                const float4 v = make_float4((float)hh[2 * k].x, (float)hh[2 * k].y, (float)hh[2 * k + 1].x,
+                                             (float)hh[2 * k + 1].y);
+                if (LOCAL) reinterpret_cast<float4 *>(carry_out)[k] = v;
+                else __stcg(reinterpret_cast<float4 *>(carry_out) + k, v);
+            }
+        };
+        auto wait_carry = [&](int pos) {
+            if (LOCAL) return local_wait(lflags + (producer > 0 ? producer : 0), lflags + kWorkers, lane, (unsigned)pos);
+            return wait_progress(p, lane, g, pos);
+        };
+        auto publish_carry = [&](int pos) {
+            if (g == p.stall_group) return;  // test hook: the next piece's wait runs out
+            if (LOCAL) local_publish(lflags + warp, lane, (unsigned)pos);
+            else publish_progress(p, lane, g, pos);
         };
 
         const int64_t tb0 = (int64_t)sb * kTC;
@@ -289,7 +422,7 @@ scan_fwd_pairs_kernel(const Params p) {
         // The piece's sub-chunks.  State-only (SO) runs do the recurrence alone
         // -- no C rows, readout, gate or stores -- and sum delta into dsum;
         // full runs publish the carried state at the end when `publish_end`.
-        auto run_subs = [&](const bool SO, float2 (&h)[S / 2], double &dsum, bool publish_end) {
+        auto run_subs = [&](const bool SO, HV (&h)[S / 2], double &dsum, bool publish_end) {
         so_stage = SO;
         issue(0, 0);
         if (CONV && ph == 0) {
@@ -423,9 +556,13 @@ scan_fwd_pairs_kernel(const Params p) {
                         for (int e = 0; e < 8; ++e) s8 += dq[e].x;
                         dsum += (double)s8;
                     }
-                    float2 y2[8];
+                    float2 y2[8];  // readout partial sums: packed fp32 pairs, or
+                    double yd[8];  // fp64 with fp32 activations
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) y2[e] = make_float2(0.f, 0.f);
+                    for (int e = 0; e < 8; ++e) {
+                        y2[e] = make_float2(0.f, 0.f);
+                        yd[e] = 0.0;
+                    }
 #pragma unroll
                     for (int q = 0; q < S / 4; ++q) {
 #pragma unroll
@@ -438,9 +575,18 @@ scan_fwd_pairs_kernel(const Params p) {
                             const float2 x1 = __fmul2_rn(dl2, A2[2 * q + 1]);
                             const float2 bu0 = __fmul2_rn(du2, make_float2(bb.x, bb.y));
                             const float2 bu1 = __fmul2_rn(du2, make_float2(bb.z, bb.w));
-                            if (ACC) {
-                                h[2 * q] = Dk::step2(x0, h[2 * q], bu0);
-                                h[2 * q + 1] = Dk::step2(x1, h[2 * q + 1], bu1);
+                            if constexpr (ACC) {
+                                h[2 * q].x = Dk::step(x0.x, h[2 * q].x, bu0.x);
+                                h[2 * q].y = Dk::step(x0.y, h[2 * q].y, bu0.y);
+                                h[2 * q + 1].x = Dk::step(x1.x, h[2 * q + 1].x, bu1.x);
+                                h[2 * q + 1].y = Dk::step(x1.y, h[2 * q + 1].y, bu1.y);
+                                if (!SO) {
+                                    const float4 cc = *reinterpret_cast<const float4 *>(sC + to);
+                                    yd[e] = fma((double)cc.x, h[2 * q].x, yd[e]);
+                                    yd[e] = fma((double)cc.y, h[2 * q].y, yd[e]);
+                                    yd[e] = fma((double)cc.z, h[2 * q + 1].x, yd[e]);
+                                    yd[e] = fma((double)cc.w, h[2 * q + 1].y, yd[e]);
+                                }
                             } else {
                                 const float2 a0 = make_float2(ex2_mufu(x0.x), ex2_mufu(x0.y));
                                 // state-only runs lean harder on the MUFU (no readout or
@@ -451,11 +597,11 @@ scan_fwd_pairs_kernel(const Params p) {
                                 else a1 = make_float2(ex2_mufu(x1.x), ex2_mufu(x1.y));
                                 h[2 * q] = __ffma2_rn(a0, h[2 * q], bu0);
                                 h[2 * q + 1] = __ffma2_rn(a1, h[2 * q + 1], bu1);
-                            }
-                            if (!SO) {
-                                const float4 cc = *reinterpret_cast<const float4 *>(sC + to);
-                                y2[e] = __ffma2_rn(make_float2(cc.x, cc.y), h[2 * q], y2[e]);
-                                y2[e] = __ffma2_rn(make_float2(cc.z, cc.w), h[2 * q + 1], y2[e]);
+                                if (!SO) {
+                                    const float4 cc = *reinterpret_cast<const float4 *>(sC + to);
+                                    y2[e] = __ffma2_rn(make_float2(cc.x, cc.y), h[2 * q], y2[e]);
+                                    y2[e] = __ffma2_rn(make_float2(cc.z, cc.w), h[2 * q + 1], y2[e]);
+                                }
                             }
                         }
                     }
@@ -464,7 +610,7 @@ scan_fwd_pairs_kernel(const Params p) {
                     // complete outputs of timesteps tb + OWN sr .. + OWN - 1
                     float yv[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) yv[e] = y2[e].x + y2[e].y;
+                    for (int e = 0; e < 8; ++e) yv[e] = ACC ? (float)yd[e] : y2[e].x + y2[e].y;
                     LaneReduce<R / 2, 8>::run(yv, sr);
                     // epilogue of this lane's outputs: out = (y + D u) * silu(z),
                     // u and z read from the staged raw rows
@@ -490,7 +636,7 @@ scan_fwd_pairs_kernel(const Params p) {
             // before this tile's stores, so the release waits on less
             if (publish_end && sub + 1 == nsub && se < p.subs_per_chain) {
                 store_carry(h);
-                if (g != p.stall_group) publish_progress(p, lane, g, se);
+                publish_carry(se);
             }
             // ---- coalesced store of the output tile
 #pragma unroll
@@ -506,19 +652,18 @@ scan_fwd_pairs_kernel(const Params p) {
         };
 
         // the state before sub-chunk 0: the initial state, or zeros
-        auto load_h0 = [&](float2 (&hh)[S / 2]) {
+        auto load_h0 = [&](HV (&hh)[S / 2]) {
 #pragma unroll
             for (int k = 0; k < S / 2; ++k) {
                 const int n0 = S * sr + 2 * k;
                 const float *src = p.h0 + (b * Dm + ds) * N;
-                hh[k] = (p.h0 && ds < Dm) ? make_float2(n0 < N ? __ldcg(src + n0) : 0.f,
-                                                        n0 + 1 < N ? __ldcg(src + n0 + 1) : 0.f)
-                                          : make_float2(0.f, 0.f);
+                hh[k] = (p.h0 && ds < Dm) ? hv(n0 < N ? __ldcg(src + n0) : 0.f, n0 + 1 < N ? __ldcg(src + n0 + 1) : 0.f)
+                                          : hv(0.f, 0.f);
             }
         };
-        float2 h[S / 2];
+        HV h[S / 2];
 #pragma unroll
-        for (int k = 0; k < S / 2; ++k) h[k] = make_float2(0.f, 0.f);
+        for (int k = 0; k < S / 2; ++k) h[k] = hv(0.f, 0.f);
         double dsum = 0.0;
         if (two_phase && se < p.subs_per_chain) {
             // The piece ends inside its group and other workers' pieces of the
@@ -530,29 +675,33 @@ scan_fwd_pairs_kernel(const Params p) {
             // waits one after the other in a few steps instead of running one
             // after the other; the output run follows from h_in.
             run_subs(true, h, dsum, false);
-            float2 hin[S / 2];
+            HV hin[S / 2];
             if (sb > 0) {
-                if (!wait_progress(p, lane, g, sb)) return;
+                if (!wait_carry(sb)) return;
                 load_carry(hin);
             } else {
                 load_h0(hin);
             }
-            float2 hend[S / 2];
+            HV hend[S / 2];
 #pragma unroll
             for (int k = 0; k < S / 2; ++k) {
                 // exp(A sum(delta)): fp64 for fp32 activations, else one ex2 each
-                const float2 decay = ACC ? f2((float)exp((double)A2[k].x * dsum), (float)exp((double)A2[k].y * dsum))
-                                         : f2(ex2_mufu((float)((double)A2[k].x * dsum)),
-                                              ex2_mufu((float)((double)A2[k].y * dsum)));
-                hend[k] = __ffma2_rn(decay, hin[k], h[k]);
+                if constexpr (ACC) {
+                    hend[k].x = fma(exp((double)A2[k].x * dsum), hin[k].x, h[k].x);
+                    hend[k].y = fma(exp((double)A2[k].y * dsum), hin[k].y, h[k].y);
+                } else {
+                    const float2 decay = f2(ex2_mufu((float)((double)A2[k].x * dsum)),
+                                            ex2_mufu((float)((double)A2[k].y * dsum)));
+                    hend[k] = __ffma2_rn(decay, hin[k], h[k]);
+                }
                 h[k] = hin[k];
             }
             store_carry(hend);
-            if (g != p.stall_group) publish_progress(p, lane, g, se);
+            publish_carry(se);
             run_subs(false, h, dsum, false);
         } else {
             if (sb > 0) {
-                if (!wait_progress(p, lane, g, sb)) return;
+                if (!wait_carry(sb)) return;
                 load_carry(h);
             } else {
                 load_h0(h);
@@ -565,57 +714,67 @@ scan_fwd_pairs_kernel(const Params p) {
 #pragma unroll
             for (int k = 0; k < S / 2; ++k) {
                 const int n0 = S * sr + 2 * k;
-                if (n0 < N) ls[n0] = h[k].x;
-                if (n0 + 1 < N) ls[n0 + 1] = h[k].y;
+                if (n0 < N) ls[n0] = (float)h[k].x;
+                if (n0 + 1 < N) ls[n0 + 1] = (float)h[k].y;
             }
         }
     }
 }
 
-template <typename T, int R, bool SP, bool GATE, bool CONV = false>
+template <typename T, int R, bool SP, bool GATE, bool CONV, bool LOCAL>
 cudaError_t launch_t(const Params &kp, int sm_count, cudaStream_t st) {
-    const int smem = kWarps * PairSmem<T, R>::BYTES;
-    auto kern = scan_fwd_pairs_kernel<T, R, SP, GATE, CONV>;
+    using PL = PairLaunch<R, LOCAL>;
+    const int smem = PL::kWorkers * PairSmem<T, R>::BYTES + (LOCAL ? LocalSmem<R>::BYTES : 0);
+    auto kern = scan_fwd_pairs_kernel<T, R, SP, GATE, CONV, LOCAL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     static const int per_sm = [&] {
         int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kWarps * 32, smem) != cudaSuccess) n = 0;
-        return n < LanesOccupancy<R>::kBlocks ? n : LanesOccupancy<R>::kBlocks;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, PL::kWorkers * 32, smem) != cudaSuccess) n = 0;
+        return n < PL::kMinBlocks ? n : PL::kMinBlocks;
     }();
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    // a worker may wait on the one before it: launch them all resident at once
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(sm_count * per_sm));
-    cfg.blockDim = dim3(kWarps * 32);
+    cfg.blockDim = dim3(PL::kWorkers * 32);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    if (LOCAL) {
+        // independent blocks, one per SM, each with at least one whole group
+        const int grid = kp.n_groups < sm_count ? kp.n_groups : sm_count;
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.numAttrs = 0;
+    } else {
+        // a worker may wait on the one before it: launch them all resident at once
+        cfg.gridDim = dim3((unsigned)(sm_count * per_sm));
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
     return cudaLaunchKernelEx(&cfg, kern, kp);
 }
 
-template <int R>
+template <int R, bool LOCAL>
 cudaError_t launch_r(const Params &kp, int act, int sm_count, cudaStream_t st) {
     const bool gate = kp.z != nullptr;
+    using BF = __nv_bfloat16;
     if (kp.conv_w) {  // fused conv1d prologue: softplus on (checked by the caller)
-        if (act == kBF16) return gate ? launch_t<__nv_bfloat16, R, true, true, true>(kp, sm_count, st)
-                                      : launch_t<__nv_bfloat16, R, true, false, true>(kp, sm_count, st);
-        return gate ? launch_t<float, R, true, true, true>(kp, sm_count, st)
-                    : launch_t<float, R, true, false, true>(kp, sm_count, st);
+        if (act == kBF16) return gate ? launch_t<BF, R, true, true, true, LOCAL>(kp, sm_count, st)
+                                      : launch_t<BF, R, true, false, true, LOCAL>(kp, sm_count, st);
+        return gate ? launch_t<float, R, true, true, true, LOCAL>(kp, sm_count, st)
+                    : launch_t<float, R, true, false, true, LOCAL>(kp, sm_count, st);
     }
     if (act == kBF16) {
-        if (kp.softplus) return gate ? launch_t<__nv_bfloat16, R, true, true>(kp, sm_count, st)
-                                     : launch_t<__nv_bfloat16, R, true, false>(kp, sm_count, st);
-        return gate ? launch_t<__nv_bfloat16, R, false, true>(kp, sm_count, st)
-                    : launch_t<__nv_bfloat16, R, false, false>(kp, sm_count, st);
+        if (kp.softplus) return gate ? launch_t<BF, R, true, true, false, LOCAL>(kp, sm_count, st)
+                                     : launch_t<BF, R, true, false, false, LOCAL>(kp, sm_count, st);
+        return gate ? launch_t<BF, R, false, true, false, LOCAL>(kp, sm_count, st)
+                    : launch_t<BF, R, false, false, false, LOCAL>(kp, sm_count, st);
     }
-    if (kp.softplus) return gate ? launch_t<float, R, true, true>(kp, sm_count, st)
-                                 : launch_t<float, R, true, false>(kp, sm_count, st);
-    return gate ? launch_t<float, R, false, true>(kp, sm_count, st) : launch_t<float, R, false, false>(kp, sm_count, st);
+    if (kp.softplus) return gate ? launch_t<float, R, true, true, false, LOCAL>(kp, sm_count, st)
+                                 : launch_t<float, R, true, false, false, LOCAL>(kp, sm_count, st);
+    return gate ? launch_t<float, R, false, true, false, LOCAL>(kp, sm_count, st)
+                : launch_t<float, R, false, false, false, LOCAL>(kp, sm_count, st);
 }
 
 }  // namespace
@@ -630,8 +789,23 @@ int persistent_split_blocks_per_sm(int lanes) {
 }
 
 cudaError_t launch_persistent_split(const Params &kp, int lanes, int act, int sm_count, cudaStream_t st) {
-    if (lanes == 4) return launch_r<4>(kp, act, sm_count, st);
-    return launch_r<2>(kp, act, sm_count, st);
+    if (lanes == 4) return launch_r<4, false>(kp, act, sm_count, st);
+    return launch_r<2, false>(kp, act, sm_count, st);
+}
+
+int local_split_warps(int lanes) { return lanes == 4 ? LocalWarps<4>::value : LocalWarps<2>::value; }
+
+cudaError_t launch_local_split(const Params &kp, int lanes, int act, int sm_count, cudaStream_t st) {
+    if (lanes == 4) return launch_r<4, true>(kp, act, sm_count, st);
+    return launch_r<2, true>(kp, act, sm_count, st);
+}
+
+int take_local_error(unsigned *flag) {
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_local_error, sizeof(v)) != cudaSuccess) return -1;
+    if (v != 0 && cudaMemcpyToSymbol(g_local_error, &zero, sizeof(zero)) != cudaSuccess) return -1;
+    *flag = v;
+    return 0;
 }
 
 }  // namespace mscan

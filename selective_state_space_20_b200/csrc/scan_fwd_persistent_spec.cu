@@ -21,7 +21,8 @@
 //   * epilogue: out = (y + D u) * silu(z) from the scan's fp32 readouts and the
 //     staged u / z rows, packed and stored to global memory.
 // fp32 activations take the accurate decay and softplus of device_math.cuh
-// (Decay<true>) for all 16 states instead.
+// (Decay<true>) for all 16 states instead, with the states and the readout in
+// fp64.
 // The pair hands sub-chunks back and forth through two processed-data slots,
 // each guarded by a pair of mbarriers (full: helper -> scan, done: scan ->
 // helper).  Every wait is bounded in time; a timeout raises the error word.
@@ -34,6 +35,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "device_math.cuh"
 #include "internal.h"
@@ -401,12 +404,21 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
         return;
     }
 
-    // ---- scan warp: lane = channel, all states in registers
+    // ---- scan warp: lane = channel, all states in registers (pairs: fp32
+    // for bf16 activations, fp64 for fp32 ones; Decay's note says why)
+    constexpr bool ACC = sizeof(T) == 4;
+    using HV = typename std::conditional<ACC, double2, float2>::type;
+    auto hv = [](float a, float b) {
+        HV r;
+        r.x = a;
+        r.y = b;
+        return r;
+    };
     int cur_group = -1;
     float2 A2[kNS / 2];
-    float2 hs[kNS / 2];
+    HV hs[kNS / 2];
 #pragma unroll
-    for (int q = 0; q < kNS / 2; ++q) { A2[q] = f2(0.f, 0.f); hs[q] = f2(0.f, 0.f); }
+    for (int q = 0; q < kNS / 2; ++q) { A2[q] = f2(0.f, 0.f); hs[q] = hv(0.f, 0.f); }
     const int N = p.dstate;
     for (int k = 0;; ++k) {
         if (!mbar_wait(full + (k & 1), (k >> 1) & 1, err)) return;
@@ -431,15 +443,15 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
                     const float *src = p.h0 + (d.rowidx + lane) * N;
 #pragma unroll
                     for (int q = 0; q < kNS / 2; ++q)
-                        hs[q] = (p.h0 && dc < p.dim) ? f2(2 * q < N ? __ldcg(src + 2 * q) : 0.f,
+                        hs[q] = (p.h0 && dc < p.dim) ? hv(2 * q < N ? __ldcg(src + 2 * q) : 0.f,
                                                           2 * q + 1 < N ? __ldcg(src + 2 * q + 1) : 0.f)
-                                                     : f2(0.f, 0.f);
+                                                     : hv(0.f, 0.f);
                 } else {
 #pragma unroll
                     for (int q = 0; q < kNS / 4; ++q) {
                         const float4 v = __ldcg(reinterpret_cast<const float4 *>(carry) + q);
-                        hs[2 * q] = f2(v.x, v.y);
-                        hs[2 * q + 1] = f2(v.z, v.w);
+                        hs[2 * q] = hv(v.x, v.y);
+                        hs[2 * q + 1] = hv(v.z, v.w);
                     }
                 }
             }
@@ -452,9 +464,13 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
                 float4 dd[4];  // (delta_t, delta_t u_t, delta_t+1, delta_t+1 u_t+1)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) dd[i] = dlrow[tb / 2 + i];
-                float2 y2[8];
+                float2 y2[8];  // readout partial sums (fp64 in yd with fp32 activations)
+                double yd[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) y2[e] = f2(0.f, 0.f);
+                for (int e = 0; e < 8; ++e) {
+                    y2[e] = f2(0.f, 0.f);
+                    yd[e] = 0.0;
+                }
 #pragma unroll
                 for (int q = 0; q < kNS / 4; ++q) {
 #pragma unroll
@@ -468,38 +484,46 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
                         const float2 x1 = __fmul2_rn(f2(dl, dl), A2[2 * q + 1]);
                         const float2 bu0 = __fmul2_rn(f2(du, du), f2(bb.x, bb.y));
                         const float2 bu1 = __fmul2_rn(f2(du, du), f2(bb.z, bb.w));
-                        if (sizeof(T) == 4) {  // fp32 activations: the accurate decay
-                            hs[2 * q] = Decay<true>::step2(x0, hs[2 * q], bu0);
-                            hs[2 * q + 1] = Decay<true>::step2(x1, hs[2 * q + 1], bu1);
+                        if constexpr (ACC) {  // fp32 activations: the accurate decay, fp64 state
+                            hs[2 * q].x = Decay<true>::step(x0.x, hs[2 * q].x, bu0.x);
+                            hs[2 * q].y = Decay<true>::step(x0.y, hs[2 * q].y, bu0.y);
+                            hs[2 * q + 1].x = Decay<true>::step(x1.x, hs[2 * q + 1].x, bu1.x);
+                            hs[2 * q + 1].y = Decay<true>::step(x1.y, hs[2 * q + 1].y, bu1.y);
+                            yd[e] = fma((double)cc.x, hs[2 * q].x, yd[e]);
+                            yd[e] = fma((double)cc.y, hs[2 * q].y, yd[e]);
+                            yd[e] = fma((double)cc.z, hs[2 * q + 1].x, yd[e]);
+                            yd[e] = fma((double)cc.w, hs[2 * q + 1].y, yd[e]);
                         } else {
                             const float2 a0 = f2(ex2_mufu(x0.x), ex2_mufu(x0.y));
                             // states 14 and 15 on the FMA pipe
                             const float2 a1 = q == kNS / 4 - 1 ? ex2_poly2(x1) : f2(ex2_mufu(x1.x), ex2_mufu(x1.y));
                             hs[2 * q] = __ffma2_rn(a0, hs[2 * q], bu0);
                             hs[2 * q + 1] = __ffma2_rn(a1, hs[2 * q + 1], bu1);
+                            y2[e] = __ffma2_rn(f2(cc.x, cc.y), hs[2 * q], y2[e]);
+                            y2[e] = __ffma2_rn(f2(cc.z, cc.w), hs[2 * q + 1], y2[e]);
                         }
-                        y2[e] = __ffma2_rn(f2(cc.x, cc.y), hs[2 * q], y2[e]);
-                        y2[e] = __ffma2_rn(f2(cc.z, cc.w), hs[2 * q + 1], y2[e]);
                     }
                 }
-                yrow[tb / 4] = make_float4(y2[0].x + y2[0].y, y2[1].x + y2[1].y, y2[2].x + y2[2].y,
-                                           y2[3].x + y2[3].y);
-                yrow[tb / 4 + 1] = make_float4(y2[4].x + y2[4].y, y2[5].x + y2[5].y, y2[6].x + y2[6].y,
-                                               y2[7].x + y2[7].y);
+                float yv[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) yv[e] = ACC ? (float)yd[e] : y2[e].x + y2[e].y;
+                yrow[tb / 4] = make_float4(yv[0], yv[1], yv[2], yv[3]);
+                yrow[tb / 4 + 1] = make_float4(yv[4], yv[5], yv[6], yv[7]);
             }
             if (d.flags & kLast) {
                 if (d.j + 1 < p.n_chunks) {
 #pragma unroll
                     for (int q = 0; q < kNS / 4; ++q)
                         __stcg(reinterpret_cast<float4 *>(carry) + q,
-                               make_float4(hs[2 * q].x, hs[2 * q].y, hs[2 * q + 1].x, hs[2 * q + 1].y));
+                               make_float4((float)hs[2 * q].x, (float)hs[2 * q].y, (float)hs[2 * q + 1].x,
+                                           (float)hs[2 * q + 1].y));
                     push_unit(p, lane, (unsigned)((d.j + 1) * p.n_groups + d.g));
                 } else if (p.last_state != nullptr && dc < p.dim) {
                     float *ls = p.last_state + (d.rowidx + lane) * N;
 #pragma unroll
                     for (int q = 0; q < kNS / 2; ++q) {
-                        if (2 * q < N) ls[2 * q] = hs[q].x;
-                        if (2 * q + 1 < N) ls[2 * q + 1] = hs[q].y;
+                        if (2 * q < N) ls[2 * q] = (float)hs[q].x;
+                        if (2 * q + 1 < N) ls[2 * q + 1] = (float)hs[q].y;
                     }
                 }
             }

@@ -55,31 +55,33 @@ state_update_kernel(const SUParams p) {
     const float du = dl * ut;
     const float dl2 = dl * Dk::kScale;
     float *st = p.state + row * N;
-    float y = 0.f;
+    using HS = typename Dk::H;  // fp64 for fp32 activations
+    HS y = 0.f;
     if (NV > 0) {
 #pragma unroll
         for (int n = 0; n < N; n += 4) {
             float4 h = *reinterpret_cast<const float4 *>(st + n);
             const float4 a4 = __ldg(reinterpret_cast<const float4 *>(Ad + n));
-            float hv[4] = {h.x, h.y, h.z, h.w};
+            HS hv[4] = {h.x, h.y, h.z, h.w};
             const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 hv[i] = Dk::step(dl2 * av[i], hv[i], du * Elem<T>::load(gB + n + i));
-                y = fmaf(Elem<T>::load(gC + n + i), hv[i], y);
+                y = fma((HS)Elem<T>::load(gC + n + i), hv[i], y);
             }
-            *reinterpret_cast<float4 *>(st + n) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+            *reinterpret_cast<float4 *>(st + n) = make_float4((float)hv[0], (float)hv[1], (float)hv[2], (float)hv[3]);
         }
     } else {
         for (int n = 0; n < N; ++n) {
-            const float hn = Dk::step(dl2 * __ldg(Ad + n), st[n], du * Elem<T>::load(gB + n));
-            st[n] = hn;
-            y = fmaf(Elem<T>::load(gC + n), hn, y);
+            const HS hn = Dk::step(dl2 * __ldg(Ad + n), (HS)st[n], du * Elem<T>::load(gB + n));
+            st[n] = (float)hn;
+            y = fma((HS)Elem<T>::load(gC + n), hn, y);
         }
     }
-    if (p.D) y = fmaf(__ldg(p.D + d), ut, y);
-    if (gz) y *= silu_f(Elem<T>::load(gz + row));
-    Elem<T>::store(static_cast<T *>(p.out) + row, y);
+    float yo = (float)y;
+    if (p.D) yo = (float)fma((HS)__ldg(p.D + d), (HS)ut, y);
+    if (gz) yo *= silu_f(Elem<T>::load(gz + row));
+    Elem<T>::store(static_cast<T *>(p.out) + row, yo);
 }
 
 // Four states per lane: bf16 / fp32 loads of four consecutive B or C values.
@@ -124,20 +126,21 @@ state_update_lanes_kernel(const SUParams p) {
     const float4 a4 = __ldg(reinterpret_cast<const float4 *>(p.A + d * NV) + qi);
     const float4 b4 = Quad<T>::load(static_cast<const T *>(p.B) + b * NV + 4 * qi);
     const float4 c4 = Quad<T>::load(static_cast<const T *>(p.C) + b * NV + 4 * qi);
-    float4 hn;
-    hn.x = Dk::step(dl2 * a4.x, h4.x, du * b4.x);
-    hn.y = Dk::step(dl2 * a4.y, h4.y, du * b4.y);
-    hn.z = Dk::step(dl2 * a4.z, h4.z, du * b4.z);
-    hn.w = Dk::step(dl2 * a4.w, h4.w, du * b4.w);
-    float y = fmaf(c4.x, hn.x, fmaf(c4.y, hn.y, fmaf(c4.z, hn.z, c4.w * hn.w)));
+    using HS = typename Dk::H;  // fp64 for fp32 activations
+    const HS hx = Dk::step(dl2 * a4.x, (HS)h4.x, du * b4.x);
+    const HS hy = Dk::step(dl2 * a4.y, (HS)h4.y, du * b4.y);
+    const HS hz = Dk::step(dl2 * a4.z, (HS)h4.z, du * b4.z);
+    const HS hw = Dk::step(dl2 * a4.w, (HS)h4.w, du * b4.w);
+    HS y = fma((HS)c4.x, hx, fma((HS)c4.y, hy, fma((HS)c4.z, hz, (HS)c4.w * hw)));
 #pragma unroll
     for (int o = Q / 2; o >= 1; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
     if (!live) return;
-    *st = hn;
+    *st = make_float4((float)hx, (float)hy, (float)hz, (float)hw);
     if (qi == 0) {
-        if (p.D) y = fmaf(__ldg(p.D + d), ut, y);
-        if (gz) y *= silu_f(Elem<T>::load(gz + row));
-        Elem<T>::store(static_cast<T *>(p.out) + row, y);
+        float yo = (float)y;
+        if (p.D) yo = (float)fma((HS)__ldg(p.D + d), (HS)ut, y);
+        if (gz) yo *= silu_f(Elem<T>::load(gz + row));
+        Elem<T>::store(static_cast<T *>(p.out) + row, yo);
     }
 }
 

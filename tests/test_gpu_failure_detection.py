@@ -51,6 +51,36 @@ def test_stalled_carry_times_out_and_is_reported():
     assert rel_err(to_np(out.view(64, -1).index_select(0, idx)), ro) <= TOL[torch.bfloat16]
 
 
+@pytest.mark.parametrize("lanes", [2, 4])
+def test_local_schedule_stalled_carry_is_reported(lanes):
+    """The local schedule (no workspace) keeps its carries in shared memory;
+    when the hook stops group 0 from publishing, the next warp's bounded wait
+    runs out, the library's device word reports it (once: reading clears it),
+    and the next launch is complete and correct."""
+    w = inputs.custom(1, 64, 16384, 16, "bf16", seed=76)  # few groups, long rows: split groups
+    dev = inputs.scan_inputs(w, device="cuda")
+    lib = binding.load_library()
+    run = lambda: binding.mamba_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],  # noqa: E731
+                                         z=dev["z"], delta_bias=dev["delta_bias"], return_last_state=True,
+                                         schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=lanes)
+    assert binding.device_status() == 0
+    prev = lib.mamba_debug_stall_group(0)
+    try:
+        run()
+        status = binding.device_status()
+    finally:
+        lib.mamba_debug_stall_group(prev)
+    assert status == binding.MAMBA_ERR_TIMEOUT
+    assert binding.device_status() == 0  # read once, cleared
+    out, last = run()
+    assert binding.device_status() == 0
+    rows = [0, 17, 63]
+    from parity import oracle_rows
+    ro, rs = oracle_rows({k: v for k, v in dev.items()}, rows)
+    idx = torch.tensor(rows, device="cuda")
+    assert rel_err(to_np(out.view(64, -1).index_select(0, idx)), ro) <= TOL[torch.bfloat16]
+
+
 def _guarded(shape, dtype, device="cuda", pinned=False):
     n = 1
     for s in shape:
@@ -67,7 +97,8 @@ def _intact(buf):
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-@pytest.mark.parametrize("mode", ["persistent2", "persistent4", "persistent1", "static", "static_unaligned"])
+@pytest.mark.parametrize("mode", ["persistent2", "persistent4", "persistent1", "local2", "local4", "static",
+                                  "static_unaligned"])
 def test_scan_writes_stay_inside(dtype, mode):
     b, d, L, N = 2, 70, 336, 16
     w = inputs.custom(b, d, L, N, dtype, seed=72)
@@ -78,6 +109,8 @@ def test_scan_writes_stay_inside(dtype, mode):
     kw = {"persistent2": dict(schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=2),
           "persistent4": dict(schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=4),
           "persistent1": dict(schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=1),
+          "local2": dict(schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=2),
+          "local4": dict(schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=4),
           "static": dict(schedule=binding.SCHEDULE_STATIC),
           "static_unaligned": dict(schedule=binding.SCHEDULE_STATIC)}[mode]
     if mode == "static_unaligned":  # out one element off 16 bytes: the element path

@@ -250,6 +250,82 @@ def test_persistent_few_groups_long_sequences(lanes, dtype, shape):
                lanes_per_channel=lanes)
 
 
+# ------------------------------------------------------------ local schedule
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("shape", [(1, 32, 64), (2, 70, 336), (3, 33, 1000), (1, 1, 8),
+                                   (4, 100, 2048), (2, 64, 4096), (4, 1030, 256)])
+@pytest.mark.parametrize("dstate", [16, 5])
+@pytest.mark.parametrize("lanes", [2, 4])
+def test_local_schedule(dtype, shape, dstate, lanes):
+    """No workspace: one block per SM splits whole channel groups among its
+    warps (few groups per block: two-phase pieces; many: chained pieces)."""
+    b, d, L = shape
+    w = inputs.custom(b, d, L, dstate, dtype, seed=b * 1000 + d + L + dstate + 7)
+    cpu = inputs.scan_inputs(w)
+    ins = dev_inputs(cpu)
+    out, last = run_scan(ins, schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=lanes)
+    assert binding.device_status() == 0
+    ro, rs = oracle_full(cpu)
+    tol = TOL[inputs.DTYPES[dtype]]
+    e1, e2 = rel_err(to_np(out), ro), rel_err(to_np(last), rs)
+    record(f"local lanes={lanes} {w.name}", out=e1, state=e2)
+    assert e1 <= tol and e2 <= tol, (e1, e2)
+    out2, last2 = run_scan(ins, schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=lanes)
+    assert torch.equal(out, out2) and torch.equal(last, last2)
+
+
+@pytest.mark.parametrize("lanes", [2, 4])
+@pytest.mark.parametrize("drop,softplus", [(("z",), True), (("D", "delta_bias"), True), ((), False)])
+def test_local_optional_inputs(lanes, drop, softplus):
+    for dtype in ("fp32", "bf16"):
+        check_full(inputs.custom(2, 33, 152, 16, dtype, seed=19), softplus=softplus, drop=drop,
+                   schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=lanes)
+
+
+@pytest.mark.parametrize("lanes", [2, 4])
+def test_local_from_an_initial_state(lanes):
+    for dtype in ("fp32", "bf16"):
+        w = inputs.custom(2, 96, 1024, 16, dtype, seed=23)
+        cpu = inputs.scan_inputs(w)
+        h0 = inputs.initial_state(2, 96, 16, seed=24)
+        ins = dev_inputs(cpu)
+        out, last = binding.mamba_scan_fwd(ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"], D=ins["D"],
+                                           z=ins["z"], delta_bias=ins["delta_bias"], return_last_state=True,
+                                           h0=h0.cuda(), schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=lanes)
+        ro, rs = oracle.scan(cpu["u"], cpu["delta"], cpu["A"], cpu["B"], cpu["C"], D=cpu["D"], z=cpu["z"],
+                             delta_bias=cpu["delta_bias"], h0=h0)
+        tol = TOL[inputs.DTYPES[dtype]]
+        assert rel_err(to_np(out), ro) <= tol and rel_err(to_np(last), rs) <= tol
+
+
+def test_local_matches_device_wide_persistent():
+    """Where no piece of a group is split in either form (as many groups as
+    workers would take, every warp a whole number of groups) the two forms run
+    identical arithmetic: 148 SMs x 8 warps = 1184 groups of 16 channels."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    w = inputs.custom(2, 16 * 8 * sms // 2, 512, 16, "bf16", seed=25)
+    ins = dev_inputs(inputs.scan_inputs(w))
+    o1, s1 = run_scan(ins, schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=2)
+    o2, s2 = run_scan(ins, schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=2)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_default_call_takes_the_local_schedule():
+    """mamba_scan_fwd (no workspace) on the Mamba-2.8B layer runs the local
+    schedule; through the C ABI entry point itself, sampled rows vs the oracle."""
+    w = inputs.MAMBA_2_8B
+    cpu = inputs.scan_inputs(w)
+    ins = dev_inputs(cpu)
+    out, last = run_scan(ins)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    rows = sample_rows(w.batch, w.dim, 24, seed=3)
+    ro, rs = oracle_rows(cpu, rows)
+    idx = torch.tensor(rows, device="cuda")
+    assert rel_err(to_np(out.view(-1, w.seqlen).index_select(0, idx)), ro) <= TOL[torch.bfloat16]
+    assert rel_err(to_np(last.view(-1, w.dstate).index_select(0, idx)), rs) <= TOL[torch.bfloat16]
+
+
 def test_persistent_rejects_unsupported():
     w = inputs.custom(1, 32, 64, 32, "bf16", seed=1)  # dstate 32 > 16
     ins = dev_inputs(inputs.scan_inputs(w))

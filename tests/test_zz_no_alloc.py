@@ -42,8 +42,14 @@ def call_noalloc(lib, ins, out, last):
 
 
 def workspace_entry(ins):
+    """mamba_scan_fwd_ws with a workspace of its own and automatic tuning --
+    the call the scratch-area entry point makes with its scratch area."""
+    batch, dim, L = ins["u"].shape
+    N = ins["A"].shape[1]
+    ws = torch.empty(binding.mamba_scan_workspace_size(batch, dim, L, N, ins["u"].dtype), device="cuda",
+                     dtype=torch.uint8)
     return binding.mamba_scan_fwd(ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"], D=ins["D"],
-                                  z=ins["z"], delta_bias=ins["delta_bias"], return_last_state=True)
+                                  z=ins["z"], delta_bias=ins["delta_bias"], return_last_state=True, workspace=ws)
 
 
 def fresh_outputs(ins):
