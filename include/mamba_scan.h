@@ -30,7 +30,10 @@
  *                     mamba_scan_host_scratch_size
  *   decoding          mamba_state_update (one token), mamba_conv1d_update
  *   conv1d            mamba_conv1d_fwd
- *   backward          mamba_scan_bwd, mamba_scan_bwd_init, mamba_scan_bwd_workspace_size
+ *   backward          mamba_scan_bwd, mamba_scan_bwd_init, mamba_scan_bwd_workspace_size;
+ *                     mamba_scan_fwd_ckpt / mamba_scan_bwd_ckpt (the forward
+ *                     keeps the states the backward recomputes from),
+ *                     mamba_scan_ckpt_size
  *   sequence split    mamba_delta_sum, mamba_state_fold
  *   status            mamba_scan_workspace_status, mamba_get_device_status,
  *                     mamba_status_string, mamba_abi_version;
@@ -557,13 +560,15 @@ int mamba_state_update(float *state, const void *u, const void *delta,
  *   dD, ddelta_bias : fp32 (dim) or NULL -- written (sums over batch rows,
  *                  channels and time).
  *   workspace    : at least mamba_scan_bwd_workspace_size bytes, 16-byte
- *                  aligned, caller-owned (the states checkpointed every 8
- *                  timesteps, and per-32-channel partial sums of dB and dC).
+ *                  aligned, caller-owned (the states every 32 timesteps
+ *                  unless given, every 4th within a 32-step piece, and eight
+ *                  partial copies of dB and dC).
  *
- * dstate <= 16.  dA, dD and ddelta_bias add per-channel-group sums with
- * floating-point atomics, so they may differ in the last bits between runs;
- * du, ddelta, dz, dB and dC do not.  Returns MAMBA_OK or a mamba_status_t
- * error.
+ * The states every 32 timesteps come from a first sweep over the inputs;
+ * mamba_scan_bwd_ckpt takes them from the forward instead.  dstate <= 16.
+ * dA, dB, dC, dD and ddelta_bias add partial sums with floating-point
+ * atomics, so they may differ in the last bits between runs; du, ddelta and
+ * dz do not.  Returns MAMBA_OK or a mamba_status_t error.
  */
 int mamba_scan_bwd(const void *u, const void *delta, const float *A,
                    const void *B, const void *C, const float *D,
@@ -602,6 +607,51 @@ int mamba_scan_bwd_init(const void *u, const void *delta, const float *A,
  * or the sizes are invalid).  Pure host arithmetic. */
 size_t mamba_scan_bwd_workspace_size(int64_t batch, int64_t dim, int64_t seqlen,
                                      int64_t dstate);
+
+/* Bytes of the checkpoints mamba_scan_fwd_ckpt writes and mamba_scan_bwd_ckpt
+ * reads: the fp32 state entering every 32nd timestep, laid out [batch *
+ * ceil(dim / 32)][ceil(seqlen / 32)][32 channels][16 states] (0 for invalid
+ * sizes or dstate > 16).  Pure host arithmetic. */
+size_t mamba_scan_ckpt_size(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate);
+
+/*
+ * mamba_scan_fwd_ckpt -- mamba_scan_fwd (from the state h0, or zeros when h0
+ * is NULL) that also writes the checkpoints the backward pass recomputes
+ * from (the Mamba paper's recomputation, Section 3.3: the forward keeps a
+ * state every 32 steps, the backward recomputes the rest), so that
+ * mamba_scan_bwd_ckpt needs no sweep of its own.
+ *
+ *   ckpt, ckpt_bytes : at least mamba_scan_ckpt_size bytes, 16-byte aligned,
+ *                  written; must not overlap any other argument.
+ *   all other arguments as mamba_scan_fwd_init (h0 may be NULL).
+ *
+ * Runs the local schedule of mamba_scan_fwd (no workspace); needs dstate <=
+ * 16, 16-byte-aligned act tensors and seqlen a multiple of the 16-byte
+ * vector width, else MAMBA_ERR_UNSUPPORTED.
+ */
+int mamba_scan_fwd_ckpt(const void *u, const void *delta, const float *A, const void *B,
+                        const void *C, const float *D, const void *z, const float *delta_bias,
+                        int delta_softplus, const float *h0, void *out, float *last_state,
+                        float *ckpt, size_t ckpt_bytes, int64_t batch, int64_t dim,
+                        int64_t seqlen, int64_t dstate, int act_dtype, cudaStream_t stream);
+
+/*
+ * mamba_scan_bwd_ckpt -- mamba_scan_bwd_init (h0 may be NULL: zeros) with
+ * the states every 32 steps read from `ckpt`, as mamba_scan_fwd_ckpt wrote
+ * them for the same inputs and h0, instead of a sweep over the inputs.
+ *
+ *   ckpt         : mamba_scan_ckpt_size bytes, 16-byte aligned, read only.
+ *   dh0          : written when h0 is given (may be NULL), must be NULL
+ *                  otherwise.
+ *   all other arguments, results and errors as mamba_scan_bwd_init.
+ */
+int mamba_scan_bwd_ckpt(const void *u, const void *delta, const float *A, const void *B,
+                        const void *C, const float *D, const void *z, const float *delta_bias,
+                        int delta_softplus, const float *h0, const float *ckpt, const void *dout,
+                        const float *dlast_state, void *du, void *ddelta, float *dA, float *dB,
+                        float *dC, float *dD, void *dz, float *ddelta_bias, float *dh0,
+                        int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
+                        void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * mamba_conv1d_fwd -- the step that produces the scan's input u: a causal

@@ -36,7 +36,8 @@ EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_fwd_complex", "mamba_delta_sum", "mamba_state_fold", "mamba_scan_fwd_conv",
             "mamba_scan_host_scratch_size", "mamba_scan_fwd_host", "mamba_debug_stall_group",
             "mamba_get_device_status", "mamba_scan_bwd", "mamba_scan_bwd_init",
-            "mamba_scan_bwd_workspace_size",
+            "mamba_scan_bwd_workspace_size", "mamba_scan_ckpt_size", "mamba_scan_fwd_ckpt",
+            "mamba_scan_bwd_ckpt",
             "mamba_state_update", "mamba_conv1d_fwd",
             "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version")
 
@@ -120,6 +121,12 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_bwd_init.restype = ci
     lib.mamba_scan_bwd_workspace_size.argtypes = [i64, i64, i64, i64]
     lib.mamba_scan_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.mamba_scan_ckpt_size.argtypes = [i64, i64, i64, i64]
+    lib.mamba_scan_ckpt_size.restype = ctypes.c_size_t
+    lib.mamba_scan_fwd_ckpt.argtypes = scan_args[:9] + [fp, vp, fp, fp, ctypes.c_size_t, i64, i64, i64, i64, ci, vp]
+    lib.mamba_scan_fwd_ckpt.restype = ci
+    lib.mamba_scan_bwd_ckpt.argtypes = bwd[:9] + [fp, fp] + bwd[9:19] + [fp] + bwd[19:]
+    lib.mamba_scan_bwd_ckpt.restype = ci
     lib.mamba_conv1d_fwd.argtypes = [vp, fp, fp, ci, vp, i64, i64, i64, i64, i64, ci, vp]
     lib.mamba_conv1d_fwd.restype = ci
     lib.mamba_conv1d_update.argtypes = [fp, vp, fp, fp, ci, vp, i64, i64, i64, i64, ci, vp]
@@ -695,18 +702,63 @@ def mamba_conv1d_update(conv_state: Optional[torch.Tensor], x: torch.Tensor, wei
     return out
 
 
+def mamba_scan_ckpt_size(batch: int, dim: int, seqlen: int, dstate: int) -> int:
+    """Bytes of the checkpoints :func:`mamba_scan_fwd_ckpt` writes."""
+    return int(load_library().mamba_scan_ckpt_size(batch, dim, seqlen, dstate))
+
+
+def mamba_scan_fwd_ckpt(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                        C: torch.Tensor, D: Optional[torch.Tensor] = None, z: Optional[torch.Tensor] = None,
+                        delta_bias: Optional[torch.Tensor] = None, delta_softplus: bool = True,
+                        h0: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                        last_state: Optional[torch.Tensor] = None, ckpt: Optional[torch.Tensor] = None):
+    """:func:`mamba_scan_fwd` that also keeps the state every 32 steps for
+    the backward pass.  Returns (out, last_state, ckpt); pass ``ckpt`` to
+    :func:`mamba_scan_bwd`."""
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    dev, act = u.device, u.dtype
+    if dev.type != "cuda" or act not in _ACT:
+        raise ValueError("u must be a float32 or bfloat16 CUDA tensor")
+    for name, t in (("u", u), ("delta", delta), ("z", z)):
+        _need(t, name, dev, act, (batch, dim, L))
+    _need(B, "B", dev, act, (batch, N, L))
+    _need(C, "C", dev, act, (batch, N, L))
+    _need(A, "A", dev, torch.float32, (dim, N))
+    _need(D, "D", dev, torch.float32, (dim,))
+    _need(delta_bias, "delta_bias", dev, torch.float32, (dim,))
+    _need(h0, "h0", dev, torch.float32, (batch, dim, N))
+    lib = load_library()
+    out = torch.empty_like(u) if out is None else out
+    last_state = torch.empty(batch, dim, N, device=dev, dtype=torch.float32) if last_state is None else last_state
+    _need(out, "out", dev, act, (batch, dim, L))
+    _need(last_state, "last_state", dev, torch.float32, (batch, dim, N))
+    nbytes = lib.mamba_scan_ckpt_size(batch, dim, L, N)
+    if ckpt is None:
+        ckpt = torch.empty(max(nbytes // 4, 1), device=dev, dtype=torch.float32)
+    with torch.cuda.device(dev):
+        rc = lib.mamba_scan_fwd_ckpt(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                                     _ptr(delta_bias), int(bool(delta_softplus)), _ptr(h0), _ptr(out),
+                                     _ptr(last_state), _ptr(ckpt), ckpt.numel() * ckpt.element_size(),
+                                     batch, dim, L, N, _ACT[act], _stream(dev))
+    _check("mamba_scan_fwd_ckpt", rc)
+    return out, last_state, ckpt
+
+
 def mamba_scan_bwd(dout: torch.Tensor, u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor,
                    B: torch.Tensor, C: torch.Tensor, D: Optional[torch.Tensor] = None,
                    z: Optional[torch.Tensor] = None, delta_bias: Optional[torch.Tensor] = None,
                    delta_softplus: bool = True, dlast_state: Optional[torch.Tensor] = None,
                    workspace: Optional[torch.Tensor] = None,
-                   h0: Optional[torch.Tensor] = None) -> dict:
+                   h0: Optional[torch.Tensor] = None, ckpt: Optional[torch.Tensor] = None) -> dict:
     """Gradients of :func:`mamba_scan_fwd` for dL/dout = ``dout`` (and
     dL/dlast_state = ``dlast_state``).  Returns a dict: du, ddelta, dz (act
     dtype, like u; dz None without z), dA (dim, N), dB, dC (batch, N, L),
     dD, ddelta_bias (dim,) -- fp32 (dD / ddelta_bias None when D / the bias
     are not given) -- and dh0 (batch, dim, N) fp32 when the forward started
-    from the state ``h0`` (else None)."""
+    from the state ``h0`` (else None).  ``ckpt``: the checkpoints
+    :func:`mamba_scan_fwd_ckpt` wrote for the same inputs (and h0), which
+    spares the backward its own sweep over the inputs."""
     if u.dim() != 3:
         raise ValueError("u must be (batch, dim, L)")
     batch, dim, L = u.shape
@@ -744,8 +796,15 @@ def mamba_scan_bwd(dout: torch.Tensor, u: torch.Tensor, delta: torch.Tensor, A: 
     grads = [_ptr(dout), _ptr(dlast_state), _ptr(r["du"]), _ptr(r["ddelta"]), _ptr(r["dA"]),
              _ptr(r["dB"]), _ptr(r["dC"]), _ptr(r["dD"]), _ptr(r["dz"]), _ptr(r["ddelta_bias"])]
     tail = [batch, dim, L, N, _ACT[act], _ptr(workspace), workspace.numel(), _stream(dev)]
+    if ckpt is not None:
+        need_ck = lib.mamba_scan_ckpt_size(batch, dim, L, N)
+        if ckpt.device != dev or not ckpt.is_contiguous() or ckpt.numel() * ckpt.element_size() < need_ck:
+            raise ValueError("ckpt must be a contiguous device tensor of mamba_scan_ckpt_size bytes")
     with torch.cuda.device(dev):
-        if h0 is None:
+        if ckpt is not None:
+            fn = "mamba_scan_bwd_ckpt"
+            rc = lib.mamba_scan_bwd_ckpt(*head, _ptr(h0), _ptr(ckpt), *grads, _ptr(r["dh0"]), *tail)
+        elif h0 is None:
             fn = "mamba_scan_bwd"
             rc = lib.mamba_scan_bwd(*head, *grads, *tail)
         else:

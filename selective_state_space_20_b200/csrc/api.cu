@@ -61,6 +61,35 @@ int check_sizes(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate) {
     return MAMBA_OK;
 }
 
+// Null and aliasing rules of a dense scan: out may replace u, delta or z in
+// place; last_state may be h0 (in place); nothing else may overlap.
+int check_scan_aliases(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                       const float *D, const void *z, const float *delta_bias, const float *h0, void *out,
+                       float *last_state, int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
+                       int act_dtype) {
+    if (!u || !delta || !A || !B || !C || !out) return MAMBA_ERR_NULL;
+    const size_t es = act_size(act_dtype);
+    const size_t nx = (size_t)(batch * dim * seqlen) * es;
+    const size_t nbc = (size_t)(batch * dstate * seqlen) * es;
+    const size_t nA = (size_t)(dim * dstate) * 4, nd = (size_t)dim * 4;
+    const size_t nls = (size_t)(batch * dim * dstate) * 4;
+    if (bad_alias(out, nx, u, nx, true) || bad_alias(out, nx, delta, nx, true) ||
+        bad_alias(out, nx, z, nx, true) || bad_alias(out, nx, B, nbc, false) ||
+        bad_alias(out, nx, C, nbc, false) || bad_alias(out, nx, A, nA, false) ||
+        bad_alias(out, nx, D, nd, false) || bad_alias(out, nx, delta_bias, nd, false))
+        return MAMBA_ERR_OVERLAP;
+    if (last_state &&
+        (overlaps(last_state, nls, u, nx) || overlaps(last_state, nls, delta, nx) ||
+         overlaps(last_state, nls, z, nx) || overlaps(last_state, nls, B, nbc) ||
+         overlaps(last_state, nls, C, nbc) || overlaps(last_state, nls, A, nA) ||
+         overlaps(last_state, nls, D, nd) || overlaps(last_state, nls, delta_bias, nd) ||
+         overlaps(last_state, nls, out, nx)))
+        return MAMBA_ERR_OVERLAP;
+    if (h0 && (overlaps(h0, nls, out, nx) || bad_alias(last_state, nls, h0, nls, true)))
+        return MAMBA_ERR_OVERLAP;
+    return MAMBA_OK;
+}
+
 int scan_impl(const void *u, const void *delta, const float *A, const void *B, const void *C,
               const float *D, const void *z, const float *delta_bias, int delta_softplus,
               const float *h0, void *out, float *last_state, int64_t batch, int64_t dim, int64_t seqlen,
@@ -71,28 +100,14 @@ int scan_impl(const void *u, const void *delta, const float *A, const void *B, c
     int rc = check_sizes(batch, dim, seqlen, dstate);
     if (rc != MAMBA_OK) return rc;
     if (launch) {
-        if (!u || !delta || !A || !B || !C || !out) return MAMBA_ERR_NULL;
+        rc = check_scan_aliases(u, delta, A, B, C, D, z, delta_bias, h0, out, last_state, batch, dim, seqlen,
+                                dstate, act_dtype);
+        if (rc != MAMBA_OK) return rc;
         const size_t es = act_size(act_dtype);
         const size_t nx = (size_t)(batch * dim * seqlen) * es;
         const size_t nbc = (size_t)(batch * dstate * seqlen) * es;
         const size_t nA = (size_t)(dim * dstate) * 4, nd = (size_t)dim * 4;
         const size_t nls = (size_t)(batch * dim * dstate) * 4;
-        // out may replace u, delta or z in place; nothing else may overlap.
-        if (bad_alias(out, nx, u, nx, true) || bad_alias(out, nx, delta, nx, true) ||
-            bad_alias(out, nx, z, nx, true) || bad_alias(out, nx, B, nbc, false) ||
-            bad_alias(out, nx, C, nbc, false) || bad_alias(out, nx, A, nA, false) ||
-            bad_alias(out, nx, D, nd, false) || bad_alias(out, nx, delta_bias, nd, false))
-            return MAMBA_ERR_OVERLAP;
-        if (last_state &&
-            (overlaps(last_state, nls, u, nx) || overlaps(last_state, nls, delta, nx) ||
-             overlaps(last_state, nls, z, nx) || overlaps(last_state, nls, B, nbc) ||
-             overlaps(last_state, nls, C, nbc) || overlaps(last_state, nls, A, nA) ||
-             overlaps(last_state, nls, D, nd) || overlaps(last_state, nls, delta_bias, nd) ||
-             overlaps(last_state, nls, out, nx)))
-            return MAMBA_ERR_OVERLAP;
-        // the initial state may be the final-state output itself (in place)
-        if (h0 && (overlaps(h0, nls, out, nx) || bad_alias(last_state, nls, h0, nls, true)))
-            return MAMBA_ERR_OVERLAP;
         if (workspace) {
             if ((reinterpret_cast<uintptr_t>(workspace) & 15) != 0) return MAMBA_ERR_WORKSPACE;
             const void *ins[] = {u, delta, z, B, C, A, D, delta_bias, out, last_state, h0};
@@ -617,7 +632,7 @@ int scan_bwd_impl(const void *u, const void *delta, const float *A, const void *
                   void *ddelta, float *dA, float *dB, float *dC, float *dD, void *dz,
                   float *ddelta_bias, float *dh0, int64_t batch, int64_t dim, int64_t seqlen,
                   int64_t dstate, int act_dtype, void *workspace, size_t workspace_bytes,
-                  cudaStream_t stream) {
+                  cudaStream_t stream, const float *ckpt = nullptr) {
     if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
     int rc = check_sizes(batch, dim, seqlen, dstate);
     if (rc != MAMBA_OK) return rc;
@@ -631,12 +646,15 @@ int scan_bwd_impl(const void *u, const void *delta, const float *A, const void *
     const size_t nx = (size_t)(batch * dim * seqlen) * es, nbc = (size_t)(batch * dstate * seqlen) * es;
     const size_t nbc32 = (size_t)(batch * dstate * seqlen) * 4, nA = (size_t)(dim * dstate) * 4;
     const size_t nd = (size_t)dim * 4, ns = (size_t)(batch * dim * dstate) * 4;
-    const void *ins[] = {u, delta, z, dout, B, C, A, D, delta_bias, dlast_state, workspace, h0};
-    const size_t inb[] = {nx, nx, nx, nx, nbc, nbc, nA, nd, nd, ns, need, ns};
+    const size_t nck = ckpt ? (size_t)mscan::scan_bwd_ckpt_floats(batch, dim, seqlen) * 4 : 0;
+    if (ckpt && (reinterpret_cast<uintptr_t>(ckpt) & 15) != 0) return MAMBA_ERR_ALIGN;
+    const void *ins[] = {u, delta, z, dout, B, C, A, D, delta_bias, dlast_state, workspace, h0, ckpt};
+    const size_t inb[] = {nx, nx, nx, nx, nbc, nbc, nA, nd, nd, ns, need, ns, nck};
     void *outs[] = {du, ddelta, dz, dA, dB, dC, dD, ddelta_bias, dh0};
     const size_t outb[] = {nx, nx, nx, nA, nbc32, nbc32, nd, nd, ns};
+    if (ckpt && overlaps(ckpt, nck, workspace, need)) return MAMBA_ERR_OVERLAP;
     for (int i = 0; i < 9; ++i) {
-        for (int k = 0; k < 12; ++k)
+        for (int k = 0; k < 13; ++k)
             if (overlaps(outs[i], outb[i], ins[k], inb[k])) return MAMBA_ERR_OVERLAP;
         for (int k = 0; k < i; ++k)
             if (overlaps(outs[i], outb[i], outs[k], outb[k])) return MAMBA_ERR_OVERLAP;
@@ -651,7 +669,7 @@ int scan_bwd_impl(const void *u, const void *delta, const float *A, const void *
     a.dA = dA; a.dB = dB; a.dC = dC; a.dD = dD; a.ddelta_bias = ddelta_bias; a.dh0 = dh0;
     a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = (int)dstate;
     a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
-    return mscan::launch_scan_bwd(a, workspace, sms, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+    return mscan::launch_scan_bwd(a, workspace, ckpt, sms, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 }  // namespace
 
@@ -677,6 +695,64 @@ int mamba_scan_bwd_init(const void *u, const void *delta, const float *A, const 
     return scan_bwd_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, dout,
                          dlast_state, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, dh0, batch,
                          dim, seqlen, dstate, act_dtype, workspace, workspace_bytes, stream);
+}
+
+size_t mamba_scan_ckpt_size(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate) {
+    if (check_sizes(batch, dim, seqlen, dstate) != MAMBA_OK || dstate > 16) return 0;
+    return (size_t)mscan::scan_bwd_ckpt_floats(batch, dim, seqlen) * 4;
+}
+
+int mamba_scan_fwd_ckpt(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                        const float *D, const void *z, const float *delta_bias, int delta_softplus,
+                        const float *h0, void *out, float *last_state, float *ckpt, size_t ckpt_bytes,
+                        int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
+                        cudaStream_t stream) {
+    if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
+    int rc = check_sizes(batch, dim, seqlen, dstate);
+    if (rc != MAMBA_OK) return rc;
+    if (!ckpt) return MAMBA_ERR_NULL;
+    rc = check_scan_aliases(u, delta, A, B, C, D, z, delta_bias, h0, out, last_state, batch, dim, seqlen, dstate,
+                            act_dtype);
+    if (rc != MAMBA_OK) return rc;
+    if (dstate > 16) return MAMBA_ERR_UNSUPPORTED;
+    const size_t need = mamba_scan_ckpt_size(batch, dim, seqlen, dstate);
+    if (ckpt_bytes < need || (reinterpret_cast<uintptr_t>(ckpt) & 15) != 0) return MAMBA_ERR_WORKSPACE;
+    const size_t es = act_size(act_dtype);
+    const size_t nx = (size_t)(batch * dim * seqlen) * es, nbc = (size_t)(batch * dstate * seqlen) * es;
+    const size_t nA = (size_t)(dim * dstate) * 4, nd = (size_t)dim * 4, nls = (size_t)(batch * dim * dstate) * 4;
+    const void *all[] = {u, delta, z, B, C, A, D, delta_bias, h0, out, last_state};
+    const size_t sz[] = {nx, nx, nx, nbc, nbc, nA, nd, nd, nls, nx, nls};
+    for (int i = 0; i < 11; ++i)
+        if (overlaps(ckpt, need, all[i], sz[i])) return MAMBA_ERR_OVERLAP;
+    int status = MAMBA_OK;
+    const int sms = current_sm_count(&status);
+    if (status != MAMBA_OK) return status;
+    mscan::ScanArgs a;
+    a.u = u; a.delta = delta; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.D = D; a.delta_bias = delta_bias; a.out = out; a.last_state = last_state; a.h0 = h0;
+    a.strides = nullptr;
+    a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = (int)dstate;
+    a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
+    a.ckpt = ckpt;
+    if (!mscan::persistent_supported(a)) return MAMBA_ERR_UNSUPPORTED;
+    int lanes = mscan::local_choose_lanes(a, sms);
+    if (lanes == 0) lanes = 2;  // the block-local form covers any shape
+    note_workspace(nullptr);
+    return mscan::launch_scan_fwd_local(a, lanes, sms, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
+int mamba_scan_bwd_ckpt(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                        const float *D, const void *z, const float *delta_bias, int delta_softplus,
+                        const float *h0, const float *ckpt, const void *dout, const float *dlast_state,
+                        void *du, void *ddelta, float *dA, float *dB, float *dC, float *dD, void *dz,
+                        float *ddelta_bias, float *dh0, int64_t batch, int64_t dim, int64_t seqlen,
+                        int64_t dstate, int act_dtype, void *workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+    if (!ckpt) return MAMBA_ERR_NULL;
+    if (dh0 && !h0) return MAMBA_ERR_NULL;
+    return scan_bwd_impl(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, dout, dlast_state, du,
+                         ddelta, dA, dB, dC, dD, dz, ddelta_bias, dh0, batch, dim, seqlen, dstate, act_dtype,
+                         workspace, workspace_bytes, stream, ckpt);
 }
 
 int mamba_conv1d_fwd(const void *x, const float *weight, const float *bias, int apply_silu,

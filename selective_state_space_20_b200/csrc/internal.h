@@ -35,6 +35,9 @@ struct ScanArgs {
     void *u_out = nullptr;          // (batch, dim, L) act or null: the u it formed
     int64_t u_bstride = 0;          // batch stride of x when conv_w is set (elements); 0: dim * L
     int64_t z_bstride = 0;          // batch stride of z when conv_w is set; 0: dim * L
+    // lane-split kernel only: checkpoints for the backward pass (the state
+    // entering every scan_bwd_ckpt_interval() steps, its layout) or null
+    float *ckpt = nullptr;
     int64_t batch, dim, seqlen;
     int dstate;
     int softplus;
@@ -102,7 +105,14 @@ struct ScanBwdArgs {
     int dstate, softplus, act;
 };
 size_t scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen);
-cudaError_t launch_scan_bwd(const ScanBwdArgs &a, void *workspace, int sm_count, cudaStream_t stream);
+// Checkpoints the backward reads: the state entering every
+// scan_bwd_ckpt_interval() timesteps, fp32 [batch * ceil(dim / 32)][ceil(L /
+// interval)][32 channels][16 states].  ckpt == null: the backward writes them
+// itself (into the workspace) in a first sweep.
+int64_t scan_bwd_ckpt_floats(int64_t batch, int64_t dim, int64_t seqlen);
+int scan_bwd_ckpt_interval();
+cudaError_t launch_scan_bwd(const ScanBwdArgs &a, void *workspace, const float *ckpt, int sm_count,
+                            cudaStream_t stream);
 
 cudaError_t launch_conv1d_fwd(const Conv1dArgs &a, cudaStream_t stream);
 cudaError_t launch_conv1d_update(const Conv1dUpdateArgs &a, cudaStream_t stream);

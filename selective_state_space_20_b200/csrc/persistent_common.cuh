@@ -53,6 +53,10 @@ struct Params {
     int subs_per_chain;    // balanced schedule: sub-chunks per group (ceil(seqlen / TC))
     int stall_group;       // test hook: this group's pieces never publish their carry (-1: none)
     float *carry;          // workspace: n_groups * 32 lanes * states-per-lane floats
+    // optional: the state entering every 32nd timestep, for the backward pass
+    // ([batch * ckpt_gpb][ckpt_nsup][32 channels][16 states] fp32)
+    float *ckpt;
+    int ckpt_gpb, ckpt_nsup;
 };
 
 __device__ __forceinline__ void cp16(void *smem, const void *gmem, bool pred) {

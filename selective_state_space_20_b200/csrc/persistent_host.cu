@@ -155,6 +155,9 @@ persist::Params base_params(const ScanArgs &a, int lanes, int tc) {
     kp.n_groups = (int)n_groups(a.batch, a.dim, lanes);
     kp.subs_per_chain = (int)((a.seqlen + tc - 1) / tc);
     kp.stall_group = g_stall_group;
+    kp.ckpt = a.ckpt;
+    kp.ckpt_gpb = (int)((a.dim + 31) / 32);
+    kp.ckpt_nsup = (int)((a.seqlen + 31) / 32);
     return kp;
 }
 }  // namespace

@@ -5,36 +5,50 @@
 // y_t = C_t h_t + D u_t, out_t = y_t silu(z_t) (training the layer
 // back-propagates through the scan; the Mamba paper's hardware-aware
 // algorithm, Section 3.3, recomputes the states in the backward pass rather
-// than storing them).  With g = dL/dh_t carried backwards:
-//   dy = dout silu(z);  dz = dout y silu'(z);  dD += dy u;  du = dy D
-//   dC[n,t] += dy h_t[n];  g[n] += dy C[n,t]
-//   ddelta += g[n] (h_{t-1}[n] Abar A[n] + B[n,t] u);  dA[n] += g[n] h_{t-1}[n] Abar delta
-//   dB[n,t] += g[n] delta u;  du += g[n] delta B[n,t];  g[n] *= Abar
+// than storing them).  With g = dL/dh_t carried backwards and, per step,
+// g' = g + dy C_t (the adjoint of h_t once the step's readout is in):
+//   dy = dout silu(z);  dz = dout y silu'(z);  dD += dy u
+//   dC[n,t] += dy h_t[n];  dB[n,t] += g'[n] delta u
+//   S_B = sum_n g'[n] B[n,t];  S_A = sum_n g'[n] Abar h_{t-1}[n] A[n]
+//   du = dy D + delta S_B;  ddelta = S_A + u S_B;  dA[n] += g'[n] Abar h_{t-1}[n] delta
+//   g[n] <- Abar g'[n]   (the adjoint of h_{t-1})
 //   ddelta_raw = ddelta sigmoid(delta_raw + bias) (softplus);  dbias += ddelta_raw
 // and, when the forward started from a given state h0, dh0 = g after t = 0.
 //
 // Design.  A block of four warps takes a group of 32 channels of one batch
-// row through the whole sequence, twice: forward, storing the state every
-// kSeg timesteps in the workspace (the checkpoints), then backward segment
-// by segment from the end: each segment's inputs are staged once for the
-// block in shared memory (B and C widened to fp32 [t][n] for broadcast
-// reads; u, delta, sigmoid, z and dout per channel), its states recomputed
-// from the checkpoint into shared memory and consumed in reverse.  Four
-// lanes share a channel, four states each, so a group is four warps and
-// each SM sub-partition holds several -- the reverse sweep is a long chain of
-// dependent steps, and the warps hide each other's latency.  Per-channel
-// sums over states (the readout, ddelta, du) are shuffles among a channel's
-// lanes.  dB and dC are sums over all channels of a batch row: each warp sums
-// its 8 channels with a transposed shuffle reduction, the block adds its
-// warps in a fixed order and stores the group's partial sum; a second kernel
-// adds the groups of each batch row in a fixed order.  dA, dD and dbias are
-// summed over a group's whole sequence in registers and added once per
-// group with atomics.  fp32 activations take the accurate decay, softplus and
-// sigmoid (Decay<true> of device_math.cuh: the state and the adjoint advance
-// by (Abar - 1) x + b, Abar - 1 on the FMA pipe), bf16 ones one ex2 per decay.
+// row; in a warp, lane 4 c + r takes channel c (of 8) and states 4 r .. 4 r + 3.
+//   * States every kSup = 32 timesteps (the checkpoints) come from the forward
+//     (mamba_scan_fwd_ckpt writes them) or from a first sweep of this kernel.
+//   * The sequence is then walked backwards one 32-step super-segment at a
+//     time.  Its inputs are staged once for the block (16-byte cp.async, the
+//     next super-segment's copies issued as soon as this one's are
+//     converted); per element, delta = softplus(raw + bias), sigmoid(raw +
+//     bias), dy = dout silu(z) and the gate factor dout sigmoid(z) (1 + z (1 -
+//     sigmoid(z))) are formed once into shared memory, B and C widened once.
+//   * From the segment's checkpoint the states are recomputed over the 32
+//     steps, leaving one sub-checkpoint every kSub = 4 steps (per-group
+//     workspace, L2-resident); then each 4-step window, last first, is
+//     recomputed once more into registers -- states and decays -- and walked
+//     in reverse from them, so the reverse step evaluates no exponential.
+//   * Sums over a channel's states are shuffles among its 4 lanes; dB and dC,
+//     sums over every channel of a batch row, are summed over a warp's 8
+//     channels by a transposed shuffle reduction, over the block's warps in
+//     shared memory, and added with one atomic add per (state, step) and
+//     block into one of kRep copies (group % kRep: the blocks of a batch row
+//     walk the sequence in step and would otherwise all queue on the same
+//     addresses); a last kernel adds the copies.  dB / dC are therefore not
+//     bitwise reproducible from run to run (the atomics' order varies).  dA,
+//     dD and dbias are summed per group in registers, one atomic add each at
+//     the end.
+//   * du, ddelta_raw and dz of a super-segment are staged in shared memory and
+//     written as whole 16-byte pieces of each row.
+// fp32 activations keep states and adjoints in fp64 with the accurate decays
+// of device_math.cuh (Decay<true>), bf16 ones fp32 with one ex2 per decay.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "device_math.cuh"
 #include "internal.h"
@@ -42,47 +56,56 @@
 namespace mscan {
 namespace {
 
-constexpr int kNS = 16;       // padded states per channel (dstate <= 16)
-constexpr int kSeg = 8;       // timesteps between checkpoints
-constexpr int kWarpsBwd = 4;  // warps per block
+constexpr int kNS = 16;                  // padded states per channel (dstate <= 16)
+constexpr int kSPL = 4;                  // states per lane
+constexpr int kCPW = 8;                  // channels per warp
+constexpr int kSup = 32;                 // timesteps between checkpoints (one staged super-segment)
+constexpr int kSub = 4;                  // timesteps recomputed into registers at a time
+constexpr int kNSub = kSup / kSub;       // sub-checkpoints per super-segment
+constexpr int kRep = 8;                  // copies of dB / dC the blocks add into (group % kRep)
+constexpr int kCkCh = 32;                // channels per checkpoint group (the forward's layout)
+
+// per-channel fp32 values of a super-segment: one 16-byte record per (step,
+// channel) -- (delta, u, dy, gate factor) -- read with one load, and the
+// sigmoid of the raw step, [t][channel]
+
+// Row pitches are padded so that the accesses below are free of bank
+// conflicts: raw / output rows by 16 bytes (rows read or written 16 bytes at
+// a time by lanes of different rows, or element-wise by lanes of 8 rows).
+// The per-channel arrays are written by 32 lanes of one step (contiguous)
+// and read by lanes of 8 channels of one step (broadcast within a channel).
+// A block: WARPS warps = 8 WARPS channels of one batch row (4 or 6 warps,
+// chosen per shape so that the blocks spread evenly over the SMs).
+template <typename T, int WARPS>
+struct BwdSmem {
+    static constexpr int kCh = WARPS * kCPW;                  // channels per block
+    static constexpr int kRawRows = 4 * kCh + 2 * kNS;        // u, delta_raw, dout, z rows; B, C rows
+    static constexpr int V = 16 / (int)sizeof(T);            // elements per 16-byte copy
+    static constexpr int CPR = kSup / V;                      // copies per staged row
+    static constexpr int RP = kSup + V;                       // raw / output row pitch (elements)
+    static constexpr int RAW = kRawRows * RP * (int)sizeof(T);
+    static constexpr int SX = kSup * kCh * 16 + kSup * kCh * 4;  // records [t][c], sigmoid [t][c]
+    static constexpr int BC = kSup * 2 * kNS * 4;             // [t][B 0..15, C 16..31] fp32
+    static constexpr int RED = 2 * kSub * WARPS * 32 * 4;     // two buffers of [step][warp][slot]
+    static constexpr int OUT = 3 * kCh * RP * (int)sizeof(T); // du, ddelta_raw, dz [q][c][t]
+    static constexpr int BYTES = (RAW + 15) / 16 * 16 + SX + BC + RED + OUT;
+};
 
 struct BwdParams {
     const void *u, *delta, *B, *C, *z, *dout;
     const float *A, *D, *delta_bias, *dlast, *h0;
     void *du, *ddelta, *dz;
     float *dA, *dB, *dC, *dD, *dbias, *dh0;
-    float *ckpt;  // workspace: n_groups x n_segs x 32 lanes x kNS checkpointed states
-    float *part;  // workspace: n_groups x seqlen x 32 partial dB (lanes 0-15) / dC (16-31) sums
-    int vec;      // rows 16-byte aligned and a whole number of 16-byte chunks
+    float *ckpt;        // [batch * ckpt_g32][n_sup][32 channels][16 states]: the state entering each super-segment
+    int ckpt_g32;       // ceil(dim / 32)
+    float *rep;         // [kRep][2 (dB, dC)][batch][16][L] fp32, zeroed: the atomics' targets
+    void *subck;        // [group][kNSub][threads][4 states] (state type): sub-checkpoints
+    int ckpt_given;     // the checkpoints were written by the forward: no sweep
+    int vec;            // rows 16-byte aligned and L a whole number of 16-byte copies
     int64_t batch, dim, seqlen;
     int dstate, softplus;
-    int groups_per_batch, n_groups, n_segs;
+    int groups_per_batch, n_groups, n_sup;
 };
-
-// Lane layout.  A block of kWarpsBwd warps owns one group of 32 channels of
-// one batch row; in a warp, lane = 4 c + r takes channel c (of the warp's 8)
-// and states 4 r .. 4 r + 3.  Sums over a channel's states are shuffles
-// among its 4 lanes; sums over channels (dB, dC) are shuffles among the 8
-// lanes with the same r, then shared memory across the block's warps.
-constexpr int kCPW = 8;  // channels per warp
-constexpr int kSPL = 4;  // states per lane
-
-// Shared memory per block (floats): per warp the recomputed states after
-// each step of the segment [step][lane][4 states]; the segment's B and C rows
-// widened to fp32 [t][state] (C 16 floats after B's end, so the widening
-// stores are free of bank conflicts); per warp the channels' per-timestep
-// values [quantity][t][channel]; per warp the dB / dC partial sums [t][32].
-enum { X_U, X_DL, X_SIG, X_Z, X_DOUT, X_SGZ, X_N };  // X_SIG: sigmoid(delta_raw + bias), X_SGZ: sigmoid(z)
-constexpr int kHistW = (kSeg + 1) * 32 * kSPL;
-constexpr int kBC = 2 * kSeg * kNS + 16;
-constexpr int kXW = X_N * kSeg * kCPW;
-constexpr int kRedW = kSeg * 32;
-constexpr int kOutW = 3 * kSeg * kCPW;  // per warp: du, ddelta_raw, dz [q][t][channel]
-// raw rows in flight, per stage: 32 B / C rows and 32 x 4 (channel, quantity)
-// rows of kSeg elements, sized for fp32 (bf16 uses half)
-constexpr int kRawRows = 32 + kWarpsBwd * 32;
-constexpr int kRawStage = kRawRows * kSeg;  // elements of T per stage (room reserved as floats)
-constexpr int kBlockFloats = kWarpsBwd * (kHistW + kXW + kRedW + kOutW) + kBC + 2 * kRawStage;
 
 __device__ __forceinline__ void cp16_async(void *smem, const void *gmem, bool pred) {
     const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
@@ -90,10 +113,10 @@ __device__ __forceinline__ void cp16_async(void *smem, const void *gmem, bool pr
                  :: "r"(sa), "l"(gmem), "r"(pred ? 16 : 0) : "memory");
 }
 
-// Sum v[] over the 8 lanes that share lane & 3, transposed: afterwards
-// v[0] of lane 4 c + r holds the total of the lanes' original v[c].  Round K
-// (lane bit 16, 8, 4) halves the live values; the lane with bit K set keeps
-// the upper half.
+// Sum v[] over the 8 lanes that share lane & 3, transposed: afterwards v[0]
+// of lane 4 c + r holds the total of the lanes' original v[c].  Round K (lane
+// bit 16, 8, 4) halves the live values; the lane with bit K set keeps the
+// upper half.
 template <int K, int CNT>
 struct ChannelTranspose {
     __device__ __forceinline__ static void run(float (&v)[8], int lane) {
@@ -113,6 +136,12 @@ struct ChannelTranspose<2, CNT> {
     __device__ __forceinline__ static void run(float (&)[8], int) {}
 };
 
+template <typename X>
+__device__ __forceinline__ X quad_sum(X x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    return x + __shfl_xor_sync(0xffffffffu, x, 2);
+}
+
 // 1 / (1 + e^-x): the MUFU form for bf16 activations, CUDA's full-precision
 // expf and division for fp32 ones.
 template <bool ACC>
@@ -121,28 +150,27 @@ __device__ __forceinline__ float sigmoid(float x) {
     return __fdividef(1.f, 1.f + __expf(-x));
 }
 
-__device__ __forceinline__ float quad_sum(float x) {
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    return x + __shfl_xor_sync(0xffffffffu, x, 2);
-}
-
-template <typename T, bool SP, bool GATE>
-__global__ void __launch_bounds__(kWarpsBwd * 32, 5) scan_bwd_kernel(const BwdParams p) {
+template <typename T, bool SP, bool GATE, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, sizeof(T) == 4 ? (WARPS == 4 ? 3 : 2) : (WARPS == 4 ? 5 : 3))
+scan_bwd_kernel(const BwdParams p) {
     constexpr bool ACC = sizeof(T) == 4;
     using Dk = Decay<ACC>;
-    extern __shared__ __align__(16) float bwd_smem[];
+    using HS = typename Dk::H;  // states and adjoints: fp64 for fp32 activations
+    using SM = BwdSmem<T, WARPS>;
+    constexpr int kWarpsBwd = WARPS, kCh = SM::kCh, kRawRows = SM::kRawRows;
+    constexpr int V = SM::V, CPR = SM::CPR, RP = SM::RP;
+    extern __shared__ __align__(16) unsigned char bwd_smem[];
+    T *raw = reinterpret_cast<T *>(bwd_smem);                              // [kRawRows][RP]
+    float4 *srec = reinterpret_cast<float4 *>(bwd_smem + (SM::RAW + 15) / 16 * 16);  // [t][c]
+    float *ssig = reinterpret_cast<float *>(srec + kSup * kCh);           // [t][c]
+    float *sbc = ssig + kSup * kCh;                                        // [t][32]
+    float *red = sbc + kSup * 2 * kNS;                                     // [2][step][warp][slot]
+    T *outs = reinterpret_cast<T *>(red + 2 * kSub * kWarpsBwd * 32);      // [3][c][RP]
+
     const int tid = threadIdx.x, lane = tid & 31, wib = tid >> 5;
     const int c = lane >> 2, r = lane & 3;
-    float4 *hist = reinterpret_cast<float4 *>(bwd_smem + wib * kHistW);       // [kSeg + 1][32]
-    float *sB = bwd_smem + kWarpsBwd * kHistW;                                 // [t][n]
-    float *sC = sB + kSeg * kNS + 16;                                          // [t][n]
-    float *sxAll = sB + kBC;                                                   // [warp][q][t][c]
-    float *redAll = sxAll + kWarpsBwd * kXW;                                   // [warp][t][32]
-    float *sx = sxAll + wib * kXW;
-    float *red = redAll + wib * kRedW;
-    float *so = redAll + kWarpsBwd * kRedW + wib * kOutW;                      // [q][t][c]
-    T *rawBase = reinterpret_cast<T *>(redAll + kWarpsBwd * (kRedW + kOutW));  // [2][kRawRows][kSeg]
-    const int64_t L = p.seqlen;
+    const int cb = wib * kCPW + c;  // this lane's channel within the block
+    const int64_t L = p.seqlen, Dm = p.dim;
     const int N = p.dstate;
     const T *gu = static_cast<const T *>(p.u);
     const T *gd = static_cast<const T *>(p.delta);
@@ -150,17 +178,13 @@ __global__ void __launch_bounds__(kWarpsBwd * 32, 5) scan_bwd_kernel(const BwdPa
     const T *gB = static_cast<const T *>(p.B);
     const T *gC = static_cast<const T *>(p.C);
     const T *go = static_cast<const T *>(p.dout);
-    T *gdu = static_cast<T *>(p.du);
-    T *gdd = static_cast<T *>(p.ddelta);
-    T *gdz = static_cast<T *>(p.dz);
-    const bool vec = p.vec != 0;
+    T *gdst[3] = {static_cast<T *>(p.du), static_cast<T *>(p.ddelta), static_cast<T *>(p.dz)};
 
     for (int64_t grp = blockIdx.x; grp < p.n_groups; grp += gridDim.x) {
         const int64_t b = grp / p.groups_per_batch;
-        const int64_t d0 = (grp % p.groups_per_batch) * 32;
-        const int64_t dc = d0 + wib * kCPW + c;  // this lane's channel
-        const bool valid = dc < p.dim;
-        const int64_t row = (b * p.dim + (valid ? dc : 0)) * L;
+        const int64_t d0 = (grp % p.groups_per_batch) * kCh;
+        const int64_t dc = d0 + cb;
+        const bool valid = dc < Dm;
         float A2[kSPL], Ar[kSPL];
 #pragma unroll
         for (int i = 0; i < kSPL; ++i) {
@@ -168,223 +192,325 @@ __global__ void __launch_bounds__(kWarpsBwd * 32, 5) scan_bwd_kernel(const BwdPa
             Ar[i] = (valid && n < N) ? __ldg(p.A + dc * N + n) : 0.f;
             A2[i] = Ar[i] * Dk::kScale;
         }
-        const float bias = (valid && p.delta_bias) ? __ldg(p.delta_bias + dc) : 0.f;
         const float Dd = (valid && p.D) ? __ldg(p.D + dc) : 0.f;
-        // checkpoints: [group][segment][32 channels][16 states]; this lane's 4 states
-        float *ck = p.ckpt + grp * (int64_t)p.n_segs * 32 * kNS + (wib * kCPW + c) * kNS + kSPL * r;
+        // this lane's checkpoints (the forward's layout: 32-channel groups): + s * 32 * 16
+        float *ck = p.ckpt + ((b * p.ckpt_g32 + dc / kCkCh) * (int64_t)p.n_sup) * kCkCh * kNS + (dc % kCkCh) * kNS +
+                    kSPL * r;
+        HS *sub = static_cast<HS *>(p.subck) + (grp * kNSub * (kWarpsBwd * 32) + tid) * kSPL;  // + j * 128 * 4
 
-        // Staging of segment [t0, t0 + tn) for the whole block, in two halves.
-        // fetch: the raw rows go to a double-buffered shared area with 16-byte
-        // cp.async (element copies when rows are not 16-byte aligned), issued
-        // one segment ahead so the copies overlap the current segment's work:
-        // threads 0-31 copy a B (0-15) or C (16-31) row, every thread one
-        // (channel, quantity) row -- 0 u, 1 delta, 2 dout, 3 z.  convert: each
-        // thread, once its own copies have landed, widens its rows to fp32:
-        // B / C into [t][n], u / delta (softplus, sigmoid) / dout / z into
-        // each warp's sx[q][t][c].
-        const int fch = tid & 31, fq = tid >> 5;
-        const int64_t fd = d0 + fch;
-        const bool fok = fd < p.dim;
-        const T *fsrc = (fq == 0 ? gu : fq == 1 ? gd : fq == 2 ? go : gz) + (b * p.dim + (fok ? fd : 0)) * L;
-        const float fbias = (fok && p.delta_bias) ? __ldg(p.delta_bias + fd) : 0.f;
-        const int bwhich = tid >> 4, bn = tid & 15;
-        const T *bsrc = (bwhich ? gC : gB) + (b * N + (bn < N ? bn : 0)) * L;
-        auto fetch = [&](int64_t t0, int tn, bool full, int buf) {
-            T *raw = rawBase + buf * kRawStage;
-            auto copy_row = [&](T *dst, const T *src, bool ok) {
-                if (vec) {
-                    constexpr int V = 16 / (int)sizeof(T);
-#pragma unroll
-                    for (int q = 0; q < kSeg / V; ++q) {
-                        const bool in = ok && q * V < tn;
-                        cp16_async(dst + q * V, in ? src + q * V : src, in);
-                    }
+        // ---- staging of super-segment s: the raw rows to shared memory
+        // (16-byte cp.async, element copies for unaligned or ragged rows).
+        // Thread -> (row, copy): rows of u, delta_raw, dout, z (kCh each, the
+        // block's channels), then 16 B and 16 C rows.
+        auto fetch = [&](int s, bool full) {
+            const int64_t t0 = (int64_t)s * kSup;
+            const int tn = (L - t0) < kSup ? (int)(L - t0) : kSup;
+            for (int i = tid; i < kRawRows * CPR; i += kWarpsBwd * 32) {
+                const int row = i / CPR, cp = i % CPR;
+                const int q = row < 4 * kCh ? row / kCh : 4, rr = row < 4 * kCh ? row % kCh : row - 4 * kCh;
+                if (!full && (q == 2 || q == 3 || (q == 4 && rr >= kNS))) continue;  // sweep: u, delta, B
+                if (!GATE && q == 3) continue;
+                const T *src;
+                bool ok;
+                if (q < 4) {
+                    src = (q == 0 ? gu : q == 1 ? gd : q == 2 ? go : gz) + (b * Dm + d0 + rr) * L;
+                    ok = d0 + rr < Dm;
+                } else {
+                    src = (rr < kNS ? gB : gC) + (b * N + (rr & 15)) * L;
+                    ok = (rr & 15) < N;
+                }
+                T *dst = raw + row * RP + cp * V;
+                if (p.vec) {
+                    const bool in = ok && cp * V < tn;
+                    cp16_async(dst, in ? src + t0 + cp * V : src, in);
                 } else {
 #pragma unroll
-                    for (int s = 0; s < kSeg; ++s) dst[s] = (ok && s < tn) ? src[s] : T(0.f);
+                    for (int e = 0; e < V; ++e) dst[e] = (ok && cp * V + e < tn) ? src[t0 + cp * V + e] : T(0.f);
                 }
-            };
-            if (tid < 32) copy_row(raw + tid * kSeg, bsrc + t0, bn < N && (full || bwhich == 0));
-            if (fq < (full ? (GATE ? 4 : 3) : 2)) copy_row(raw + (32 + tid) * kSeg, fsrc + t0, fok);
+            }
             asm volatile("cp.async.commit_group;" ::: "memory");
         };
-        auto convert = [&](bool full, int buf) {
-            asm volatile("cp.async.wait_group 0;" ::: "memory");  // this thread's copies
-            const T *raw = rawBase + buf * kRawStage;
-            float f[kSeg];
-            if (tid < 32) {
-                const T *row = raw + tid * kSeg;
+        // ---- per-element values of the staged super-segment, once for the
+        // block: thread -> (channel tid % kCh, 16-byte piece of V steps), the
+        // rows read 16 bytes at a time; B / C widened to [t][n].  Past the end
+        // of the sequence delta = 0 (Abar = 1, no input) and the staged u,
+        // dout, B, C are zero, so a step there leaves every state and adjoint
+        // as it was: the loops below always run whole windows.
+        auto convert = [&](int s, bool full) {
+            const int64_t t0 = (int64_t)s * kSup;
+            const int tn = (L - t0) < kSup ? (int)(L - t0) : kSup;
+            const int cc = tid % kCh;
+            const float bias = (d0 + cc < Dm && p.delta_bias) ? __ldg(p.delta_bias + d0 + cc) : 0.f;
+            for (int piece = tid / kCh; piece < CPR; piece += (kWarpsBwd * 32) / kCh) {
+                float fu[V], fd[V], fo[V], fz[V];
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(raw + cc * RP + piece * V), fu);
+                Elem<T>::unpack(*reinterpret_cast<const uint4 *>(raw + (kCh + cc) * RP + piece * V), fd);
+                if (full) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(raw + (2 * kCh + cc) * RP + piece * V), fo);
+                if (full && GATE)
+                    Elem<T>::unpack(*reinterpret_cast<const uint4 *>(raw + (3 * kCh + cc) * RP + piece * V), fz);
 #pragma unroll
-                for (int s = 0; s < kSeg; ++s) f[s] = Elem<T>::to_f(row[s]);
-                float *dst = (bwhich ? sC : sB) + bn;
-#pragma unroll
-                for (int s = 0; s < kSeg; ++s) dst[s * kNS] = f[s];
-            }
-            if (fq < (full ? (GATE ? 4 : 3) : 2)) {
-                const T *row = raw + (32 + tid) * kSeg;
-#pragma unroll
-                for (int s = 0; s < kSeg; ++s) f[s] = Elem<T>::to_f(row[s]);
-                float *dst = sxAll + (fch >> 3) * kXW + (fch & 7);
-                if (fq == 1) {
-#pragma unroll
-                    for (int s = 0; s < kSeg; ++s) {
-                        const float x = f[s] + fbias;
-                        dst[(X_DL * kSeg + s) * kCPW] = SP ? Dk::softplus(x) : x;
-                        if (full) dst[(X_SIG * kSeg + s) * kCPW] = SP ? sigmoid<ACC>(x) : 1.f;
+                for (int e = 0; e < V; ++e) {
+                    const int t = piece * V + e;
+                    const float x = fd[e] + bias;
+                    const float dl = t >= tn ? 0.f : SP ? Dk::softplus(x) : x;
+                    float dy = 0.f, gzf = 0.f;
+                    if (full) {
+                        dy = fo[e];
+                        if (GATE) {
+                            const float sg = sigmoid<ACC>(fz[e]);
+                            dy = fo[e] * fz[e] * sg;                          // dout silu(z)
+                            gzf = fo[e] * sg * fmaf(fz[e], 1.f - sg, 1.f);    // dz = y * this
+                        }
+                        // zero past the end: those padding steps add nothing to dbias
+                        ssig[t * kCh + cc] = t >= tn ? 0.f : SP ? sigmoid<ACC>(x) : 1.f;
                     }
-                } else {
-                    const int X = fq == 0 ? X_U : fq == 2 ? X_DOUT : X_Z;
+                    srec[t * kCh + cc] = make_float4(dl, fu[e], dy, gzf);
+                }
+            }
+            {  // B and C rows (after the channels' rows): row tid % 32, 16-byte piece
+                const int row = tid & 31;
+                if (full || row < kNS) {
+                    for (int piece = tid >> 5; piece < CPR; piece += kWarpsBwd) {
+                        float f[V];
+                        Elem<T>::unpack(*reinterpret_cast<const uint4 *>(raw + (4 * kCh + row) * RP + piece * V), f);
 #pragma unroll
-                    for (int s = 0; s < kSeg; ++s) dst[(X * kSeg + s) * kCPW] = f[s];
-                    if (fq == 3) {
-#pragma unroll
-                        for (int s = 0; s < kSeg; ++s) dst[(X_SGZ * kSeg + s) * kCPW] = sigmoid<ACC>(f[s]);
+                        for (int e = 0; e < V; ++e) sbc[(piece * V + e) * 2 * kNS + row] = f[e];
                     }
                 }
             }
         };
-        // h <- the states after `tn` steps of the staged segment; into hist[1..] when asked
-        auto advance = [&](float (&h)[kSPL], int tn, bool keep) {
-#pragma unroll
-            for (int s = 0; s < kSeg; ++s) {
-                if (s >= tn) break;
-                const float dl = sx[(X_DL * kSeg + s) * kCPW + c];
-                const float du = dl * sx[(X_U * kSeg + s) * kCPW + c];
-                const float4 bb = *reinterpret_cast<const float4 *>(sB + s * kNS + kSPL * r);
-                const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+        // one forward step of this lane's states at step t of the staged segment
+        auto step = [&](HS (&h)[kSPL], int t) {
+            const float2 rec = *reinterpret_cast<const float2 *>(srec + t * kCh + cb);
+            const float dl = rec.x;
+            const float du = dl * rec.y;
+            const float4 bb = *reinterpret_cast<const float4 *>(sbc + t * 2 * kNS + kSPL * r);
+            const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+            if constexpr (ACC) {
 #pragma unroll
                 for (int i = 0; i < kSPL; ++i) h[i] = Dk::step(dl * A2[i], h[i], du * bv[i]);
-                if (keep) hist[(s + 1) * 32 + lane] = make_float4(h[0], h[1], h[2], h[3]);
+            } else {  // state pairs on the packed x2 instructions (the same roundings)
+#pragma unroll
+                for (int k = 0; k < kSPL / 2; ++k) {
+                    const float2 x = __fmul2_rn(f2(dl, dl), f2(A2[2 * k], A2[2 * k + 1]));
+                    const float2 hn = __ffma2_rn(f2(ex2_mufu(x.x), ex2_mufu(x.y)), f2(h[2 * k], h[2 * k + 1]),
+                                                 __fmul2_rn(f2(du, du), f2(bv[2 * k], bv[2 * k + 1])));
+                    h[2 * k] = hn.x;
+                    h[2 * k + 1] = hn.y;
+                }
             }
         };
-
-        // ---- forward from h0 (or zeros): checkpoints every kSeg timesteps (state before the segment)
-        float h[kSPL];
-#pragma unroll
-        for (int i = 0; i < kSPL; ++i) {
-            const int n = kSPL * r + i;
-            h[i] = (valid && p.h0 && n < N) ? __ldg(p.h0 + (b * p.dim + dc) * N + n) : 0.f;
-        }
-        auto seg_len = [&](int seg) {
-            const int64_t t0 = (int64_t)seg * kSeg;
-            return (L - t0) < kSeg ? (int)(L - t0) : kSeg;
+        auto seg_len = [&](int s) {
+            const int64_t t0 = (int64_t)s * kSup;
+            return (L - t0) < kSup ? (int)(L - t0) : kSup;
         };
-        fetch(0, seg_len(0), false, 0);
-        for (int seg = 0; seg < p.n_segs; ++seg) {
-            __stcg(reinterpret_cast<float4 *>(ck + (int64_t)seg * 32 * kNS), make_float4(h[0], h[1], h[2], h[3]));
-            __syncthreads();  // the previous segment's staging is consumed
-            convert(false, seg & 1);
-            if (seg + 1 < p.n_segs) fetch((int64_t)(seg + 1) * kSeg, seg_len(seg + 1), false, (seg + 1) & 1);
-            __syncthreads();
-            advance(h, seg_len(seg), false);
+
+        // ---- sweep (no checkpoints from the forward): the state entering
+        // every super-segment, from h0 (or zeros)
+        if (!p.ckpt_given) {
+            HS h[kSPL];
+#pragma unroll
+            for (int i = 0; i < kSPL; ++i) {
+                const int n = kSPL * r + i;
+                h[i] = (valid && p.h0 && n < N) ? (HS)__ldg(p.h0 + (b * Dm + dc) * N + n) : (HS)0.f;
+            }
+            fetch(0, false);
+            for (int s = 0; s < p.n_sup; ++s) {
+                if (valid)
+                    __stcg(reinterpret_cast<float4 *>(ck + (int64_t)s * kCkCh * kNS),
+                           make_float4((float)h[0], (float)h[1], (float)h[2], (float)h[3]));
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+                __syncthreads();  // the raw rows have landed
+                convert(s, false);
+                __syncthreads();  // converted; the raw buffer is free
+                if (s + 1 < p.n_sup) fetch(s + 1, false);
+                const int nwin = (seg_len(s) + kSub - 1) / kSub;
+                for (int j = 0; j < nwin; ++j) {
+#pragma unroll
+                    for (int w = 0; w < kSub; ++w) step(h, j * kSub + w);
+                }
+                __syncthreads();  // sx / sbc consumed
+            }
         }
 
-        // ---- reverse sweep, segment by segment from the end
-        float g[kSPL], dA_acc[kSPL];
+        // ---- reverse sweep, one super-segment at a time from the end
+        HS g[kSPL], dA_acc[kSPL];
 #pragma unroll
         for (int i = 0; i < kSPL; ++i) {
             const int n = kSPL * r + i;
-            g[i] = (valid && p.dlast && n < N) ? p.dlast[(b * p.dim + dc) * N + n] : 0.f;
+            g[i] = (valid && p.dlast && n < N) ? (HS)p.dlast[(b * Dm + dc) * N + n] : (HS)0.f;
             dA_acc[i] = 0.f;
         }
-        float dD_acc = 0.f, dbias_acc = 0.f;
+        HS dD_acc = 0.f, dbias_acc = 0.f;
         // this lane's slot of the warp's channel-summed dB / dC: lanes c < 4
         // hold dB of state 4 r + c, lanes c >= 4 dC of state 4 r + c - 4
         const int kslot = (c < 4 ? 0 : 16) + kSPL * r + (c & 3);
-        fetch((int64_t)(p.n_segs - 1) * kSeg, seg_len(p.n_segs - 1), true, (p.n_segs - 1) & 1);
-        for (int seg = p.n_segs - 1; seg >= 0; --seg) {
-            const int64_t t0 = (int64_t)seg * kSeg;
-            const int tn = seg_len(seg);
-            __syncthreads();  // staging, hist and red of the previous segment are consumed
-            convert(true, seg & 1);
-            if (seg > 0) fetch(t0 - kSeg, seg_len(seg - 1), true, (seg - 1) & 1);
+        int rbuf = 0;  // which red buffer the next window uses
+        fetch(p.n_sup - 1, true);
+        for (int s = p.n_sup - 1; s >= 0; --s) {
+            const int64_t t0 = (int64_t)s * kSup;
+            const int tn = seg_len(s);
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            __syncthreads();  // raw landed; sx, sbc, outs of the previous segment consumed
+            convert(s, true);
+            __syncthreads();  // converted; the raw buffer is free
+            if (s > 0) fetch(s - 1, true);
+            // recompute the segment from its checkpoint, one sub-checkpoint every kSub steps
             {
-                const float4 v = __ldcg(reinterpret_cast<const float4 *>(ck + (int64_t)seg * 32 * kNS));
-                h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
+                // (channels past dim have no checkpoint of the forward's: zeros)
+                const float4 v = valid ? __ldcg(reinterpret_cast<const float4 *>(ck + (int64_t)s * kCkCh * kNS))
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                HS h[kSPL] = {(HS)v.x, (HS)v.y, (HS)v.z, (HS)v.w};
+                for (int j = 0; j * kSub < tn; ++j) {
+#pragma unroll
+                    for (int i = 0; i < kSPL; ++i) sub[j * (kWarpsBwd * 32) * kSPL + i] = h[i];
+#pragma unroll
+                    for (int w = 0; w < kSub; ++w) step(h, j * kSub + w);
+                }
             }
-            __syncthreads();
-            hist[lane] = make_float4(h[0], h[1], h[2], h[3]);
-            advance(h, tn, true);
-            __syncwarp();
-            float4 hc4 = make_float4(h[0], h[1], h[2], h[3]);  // the state after the segment's last step
+            // windows of kSub steps, last first: states and decays into
+            // registers, then the reverse steps from them
+            for (int j = (tn - 1) / kSub; j >= 0; --j) {
+                const int tb = j * kSub;
+                HS hin[kSPL], hs[kSub][kSPL];
+                // the decays: Abar (bf16 activations), or Abar - 1 (from the
+                // near-zero polynomial, else the exponential) with fp32
+                // activations, so the adjoint decays with the state's accuracy
+                float ab[kSub][kSPL];
 #pragma unroll
-            for (int s = kSeg - 1; s >= 0; --s) {
-                if (s >= tn) continue;
-                const float dl = sx[(X_DL * kSeg + s) * kCPW + c];
-                const float ut = sx[(X_U * kSeg + s) * kCPW + c];
-                const float dout = sx[(X_DOUT * kSeg + s) * kCPW + c];
-                const float4 hp4 = hist[s * 32 + lane];
-                const float4 bb = *reinterpret_cast<const float4 *>(sB + s * kNS + kSPL * r);
-                const float4 cc = *reinterpret_cast<const float4 *>(sC + s * kNS + kSPL * r);
-                const float hcur[4] = {hc4.x, hc4.y, hc4.z, hc4.w}, hp[4] = {hp4.x, hp4.y, hp4.z, hp4.w};
-                const float bv[4] = {bb.x, bb.y, bb.z, bb.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
-                float yp = 0.f;
+                for (int i = 0; i < kSPL; ++i) hin[i] = sub[j * (kWarpsBwd * 32) * kSPL + i];
 #pragma unroll
-                for (int i = 0; i < kSPL; ++i) yp = fmaf(cv[i], hcur[i], yp);
-                const float y = fmaf(Dd, ut, quad_sum(yp));
-                float dy = dout;
-                if (GATE) {
-                    const float zt = sx[(X_Z * kSeg + s) * kCPW + c];
-                    const float sg = sx[(X_SGZ * kSeg + s) * kCPW + c];
-                    if (r == 0) so[(2 * kSeg + s) * kCPW + c] = dout * y * sg * fmaf(zt, 1.f - sg, 1.f);
-                    dy = dout * zt * sg;
-                }
-                dD_acc = fmaf(dy, ut, dD_acc);
-                float dut_p = 0.f, ddelta_p = 0.f;
-                float v[8];  // dB (0-3) and dC (4-7) terms of this lane's states
+                for (int w = 0; w < kSub; ++w) {
+                    {
+                        const int t = tb + w;
+                        const float2 rec = *reinterpret_cast<const float2 *>(srec + t * kCh + cb);
+                        const float dl = rec.x;
+                        const float du = dl * rec.y;
+                        const float4 bb = *reinterpret_cast<const float4 *>(sbc + t * 2 * kNS + kSPL * r);
+                        const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+                        if constexpr (ACC) {
 #pragma unroll
-                for (int i = 0; i < kSPL; ++i) {
-                    v[4 + i] = dy * hcur[i];
-                    g[i] = fmaf(dy, cv[i], g[i]);
-                    const float xa = dl * A2[i];
-                    const float ab = Dk::abar(xa);
-                    const float gha = g[i] * hp[i] * ab;
-                    ddelta_p = fmaf(gha, Ar[i], fmaf(g[i], bv[i] * ut, ddelta_p));
-                    dA_acc[i] = fmaf(gha, dl, dA_acc[i]);
-                    v[i] = g[i] * dl * ut;
-                    dut_p = fmaf(g[i] * dl, bv[i], dut_p);
-                    g[i] = ACC ? Dk::scale(xa, g[i]) : g[i] * ab;
-                }
-                ChannelTranspose<16, 8>::run(v, lane);
-                red[s * 32 + kslot] = v[0];
-                const float ddelta = quad_sum(ddelta_p);
-                const float ddraw = ddelta * sx[(X_SIG * kSeg + s) * kCPW + c];
-                dbias_acc += ddraw;
-                const float dut = fmaf(dy, Dd, quad_sum(dut_p));
-                if (r == 0) {
-                    so[(0 * kSeg + s) * kCPW + c] = dut;
-                    so[(1 * kSeg + s) * kCPW + c] = ddraw;
-                }
-                hc4 = hp4;
-            }
-            // this channel's rows of the segment: lane r = 0 du, 1 ddelta_raw,
-            // 2 dz, 16 bytes at a time where possible
-            __syncwarp();
-            if (valid && r < (GATE ? 3 : 2)) {
-                constexpr int V = 16 / (int)sizeof(T);
-                T *dst = (r == 0 ? gdu : r == 1 ? gdd : gdz) + row + t0;
-                float f[kSeg];
+                            for (int i = 0; i < kSPL; ++i) {
+                                const HS prev = w == 0 ? hin[i] : hs[w - 1][i];
+                                const float x = dl * A2[i];
+                                ab[w][i] = Dk::near_one(x) ? expm1_poly(x) : __expf(x) - 1.f;
+                                hs[w][i] = Dk::step(x, prev, du * bv[i]);
+                            }
+                        } else {
 #pragma unroll
-                for (int s = 0; s < kSeg; ++s) f[s] = so[(r * kSeg + s) * kCPW + c];
-#pragma unroll
-                for (int q = 0; q < kSeg / V; ++q) {
-                    if (vec && (q + 1) * V <= tn) {
-                        *reinterpret_cast<uint4 *>(dst + q * V) = Elem<T>::pack(f + q * V);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < V; ++e)
-                            if (q * V + e < tn) Elem<T>::store(dst + q * V + e, f[q * V + e]);
+                            for (int k = 0; k < kSPL / 2; ++k) {
+                                const float2 prev = w == 0 ? f2(hin[2 * k], hin[2 * k + 1])
+                                                           : f2(hs[w - 1][2 * k], hs[w - 1][2 * k + 1]);
+                                const float2 x = __fmul2_rn(f2(dl, dl), f2(A2[2 * k], A2[2 * k + 1]));
+                                const float2 a = f2(ex2_mufu(x.x), ex2_mufu(x.y));
+                                const float2 hn =
+                                    __ffma2_rn(a, prev, __fmul2_rn(f2(du, du), f2(bv[2 * k], bv[2 * k + 1])));
+                                ab[w][2 * k] = a.x;
+                                ab[w][2 * k + 1] = a.y;
+                                hs[w][2 * k] = hn.x;
+                                hs[w][2 * k + 1] = hn.y;
+                            }
+                        }
                     }
                 }
-            }
-            // the block's dB / dC partial sums: the warps' sums added in warp order
-            __syncthreads();
-            float *part = p.part + (grp * L + t0) * 32;
-            for (int idx = tid; idx < tn * 32; idx += kWarpsBwd * 32) {
-                float acc = 0.f;
+                float *rb = red + rbuf * (kSub * kWarpsBwd * 32);
 #pragma unroll
-                for (int w = 0; w < kWarpsBwd; ++w) acc += redAll[w * kRedW + idx];
-                __stcg(part + idx, acc);
+                for (int w = kSub - 1; w >= 0; --w) {
+                    const int t = tb + w;
+                    const float4 rec = srec[t * kCh + cb];
+                    const float dl = rec.x, ut = rec.y, dy = rec.z;
+                    const float4 bb = *reinterpret_cast<const float4 *>(sbc + t * 2 * kNS + kSPL * r);
+                    const float4 cq = *reinterpret_cast<const float4 *>(sbc + t * 2 * kNS + kNS + kSPL * r);
+                    const float bv[4] = {bb.x, bb.y, bb.z, bb.w}, cv[4] = {cq.x, cq.y, cq.z, cq.w};
+                    HS yp = 0.f, sA = 0.f, sB = 0.f;
+                    float v[8];  // dB (0-3) and dC (4-7) terms of this lane's states
+                    const float dlu = dl * ut;
+                    if constexpr (ACC) {
+#pragma unroll
+                        for (int i = 0; i < kSPL; ++i) {
+                            const HS hc = hs[w][i];
+                            const HS hp = w == 0 ? hin[i] : hs[w - 1][i];
+                            yp = fma((HS)cv[i], hc, yp);
+                            const HS gq = fma((HS)dy, (HS)cv[i], g[i]);   // g'
+                            const HS gab = fma(gq, (HS)ab[w][i], gq);     // g' + (Abar - 1) g'
+                            const HS gha = gab * hp;                      // g' Abar h_{t-1}
+                            sA = fma(gha, (HS)Ar[i], sA);
+                            sB = fma(gq, (HS)bv[i], sB);
+                            dA_acc[i] = fma(gha, (HS)dl, dA_acc[i]);
+                            v[i] = (float)gq * dlu;
+                            v[4 + i] = dy * (float)hc;
+                            g[i] = gab;
+                        }
+                    } else {  // state pairs on the packed x2 instructions
+                        float2 yp2 = f2(0.f, 0.f), sA2 = f2(0.f, 0.f), sB2 = f2(0.f, 0.f);
+#pragma unroll
+                        for (int k = 0; k < kSPL / 2; ++k) {
+                            const int i0 = 2 * k, i1 = 2 * k + 1;
+                            const float2 hc = f2(hs[w][i0], hs[w][i1]);
+                            const float2 hp = w == 0 ? f2(hin[i0], hin[i1]) : f2(hs[w - 1][i0], hs[w - 1][i1]);
+                            const float2 c2 = f2(cv[i0], cv[i1]);
+                            yp2 = __ffma2_rn(c2, hc, yp2);
+                            const float2 gq = __ffma2_rn(f2(dy, dy), c2, f2(g[i0], g[i1]));   // g'
+                            const float2 gab = __fmul2_rn(gq, f2(ab[w][i0], ab[w][i1]));
+                            const float2 gha = __fmul2_rn(gab, hp);                          // g' Abar h_{t-1}
+                            sA2 = __ffma2_rn(gha, f2(Ar[i0], Ar[i1]), sA2);
+                            sB2 = __ffma2_rn(gq, f2(bv[i0], bv[i1]), sB2);
+                            const float2 da = __ffma2_rn(gha, f2(dl, dl), f2(dA_acc[i0], dA_acc[i1]));
+                            const float2 vb = __fmul2_rn(gq, f2(dlu, dlu));
+                            const float2 vc = __fmul2_rn(f2(dy, dy), hc);
+                            dA_acc[i0] = da.x; dA_acc[i1] = da.y;
+                            v[i0] = vb.x; v[i1] = vb.y;
+                            v[4 + i0] = vc.x; v[4 + i1] = vc.y;
+                            g[i0] = gab.x; g[i1] = gab.y;
+                        }
+                        yp = yp2.x + yp2.y;
+                        sA = sA2.x + sA2.y;
+                        sB = sB2.x + sB2.y;
+                    }
+                    ChannelTranspose<16, 8>::run(v, lane);
+                    rb[(w * kWarpsBwd + wib) * 32 + kslot] = v[0];
+                    const float y = (float)quad_sum(yp) + Dd * ut;
+                    const float SA = (float)quad_sum(sA), SBs = (float)quad_sum(sB);
+                    const float ddelta = fmaf(ut, SBs, SA);
+                    const float ddraw = ddelta * ssig[t * kCh + cb];
+                    dbias_acc += (HS)ddraw;
+                    dD_acc = fma((HS)dy, (HS)ut, dD_acc);
+                    // this channel's three outputs, one lane each
+                    if (r == 0) outs[(0 * kCh + cb) * RP + t] = T(fmaf(dy, Dd, dl * SBs));
+                    if (r == 1) outs[(1 * kCh + cb) * RP + t] = T(ddraw);
+                    if (GATE && r == 2) outs[(2 * kCh + cb) * RP + t] = T(y * rec.w);
+                }
+                __syncthreads();  // the window's dB / dC terms of every warp are in rb
+                // dB / dC of the window: thread -> (step, slot), the warps summed in order
+                {
+                    const int w = tid >> 5, slot = tid & 31;
+                    const int n = slot & 15;
+                    if (w < kSub && tb + w < tn && n < N) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int k = 0; k < kWarpsBwd; ++k) acc += rb[(w * kWarpsBwd + k) * 32 + slot];
+                        atomicAdd(p.rep + (((grp % kRep) * 2 + (slot >> 4)) * p.batch + b) * (int64_t)kNS * L +
+                                      (int64_t)n * L + t0 + tb + w, acc);
+                    }
+                }
+                rbuf ^= 1;  // the next window fills the other buffer while this one is read
+            }
+            __syncthreads();  // every output of the segment is staged
+            // du, ddelta_raw, dz rows of the segment: thread -> (quantity, channel, copy)
+            for (int i = tid; i < 3 * kCh * CPR; i += kWarpsBwd * 32) {
+                const int q = i / (kCh * CPR), rem = i % (kCh * CPR);
+                const int cc = rem / CPR, cp = rem % CPR;
+                if (q == 2 && !GATE) continue;
+                if (d0 + cc >= Dm) continue;
+                T *dst = gdst[q] + (b * Dm + d0 + cc) * L + t0 + cp * V;
+                const T *srcp = outs + (q * kCh + cc) * RP + cp * V;
+                if (p.vec) {
+                    if (cp * V < tn) *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(srcp);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < V; ++e)
+                        if (cp * V + e < tn) dst[e] = srcp[e];
+                }
             }
         }
         if (valid) {
@@ -392,91 +518,135 @@ __global__ void __launch_bounds__(kWarpsBwd * 32, 5) scan_bwd_kernel(const BwdPa
             for (int i = 0; i < kSPL; ++i) {
                 const int n = kSPL * r + i;
                 if (n < N) {
-                    atomicAdd(p.dA + dc * N + n, dA_acc[i]);
-                    if (p.dh0) p.dh0[(b * p.dim + dc) * N + n] = g[i];  // dL/dh_{-1}
+                    atomicAdd(p.dA + dc * N + n, (float)dA_acc[i]);
+                    if (p.dh0) p.dh0[(b * Dm + dc) * N + n] = (float)g[i];  // dL/dh_{-1}
                 }
             }
             if (r == 0) {
-                if (p.dD) atomicAdd(p.dD + dc, dD_acc);
-                if (p.dbias) atomicAdd(p.dbias + dc, dbias_acc);
+                if (p.dD) atomicAdd(p.dD + dc, (float)dD_acc);
+                if (p.dbias) atomicAdd(p.dbias + dc, (float)dbias_acc);
             }
         }
         __syncthreads();  // before the next group reuses shared memory
     }
 }
 
-// dB[b,n,t] / dC[b,n,t] = sum over the groups of batch row b of their
-// partial sums part[g][t][n] / part[g][t][16 + n]: one block per (b, 32
-// timesteps) tile, the groups summed in registers, the tile transposed
-// through shared memory so that both the reads and the writes are coalesced.
-__global__ void __launch_bounds__(256) bwd_reduce_bc_kernel(const BwdParams p) {
-    __shared__ float tile[32][33];
-    const int64_t tiles_per_b = (p.seqlen + 31) / 32;
-    const int64_t b = blockIdx.x / tiles_per_b;
-    const int64_t t0 = (blockIdx.x % tiles_per_b) * 32;
-    const int tx = threadIdx.x & 31, ty0 = threadIdx.x >> 5;  // 8 rows per pass
-    const int N = p.dstate;
-    for (int ty = ty0; ty < 32; ty += 8) {
-        const int64_t t = t0 + ty;
+// dB / dC = the sum of the kRep copies, for states n < N: one thread per
+// (B or C, batch row, state, 4 timesteps).
+__global__ void __launch_bounds__(256) bwd_sum_copies_kernel(const BwdParams p) {
+    const int64_t L = p.seqlen, N = p.dstate;
+    const int64_t q4 = (L + 3) / 4;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= 2 * p.batch * N * q4) return;
+    const int64_t tq = i % q4, rest = i / q4;
+    const int64_t n = rest % N, wb = rest / N;  // wb = which * batch + b
+    const int64_t which = wb / p.batch, b = wb % p.batch;
+    float *dst = (which ? p.dC : p.dB) + (b * N + n) * L;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int64_t t = tq * 4 + e;
+        if (t >= L) break;
         float acc = 0.f;
-        if (t < p.seqlen) {
-            const float *src = p.part + ((b * p.groups_per_batch) * p.seqlen + t) * 32 + tx;
-            for (int gi = 0; gi < p.groups_per_batch; ++gi) acc += __ldcg(src + (int64_t)gi * p.seqlen * 32);
-        }
-        tile[ty][tx] = acc;
-    }
-    __syncthreads();
-    for (int k = ty0; k < 32; k += 8) {  // k: (B or C, state) pair; tx: timestep in the tile
-        const int n = k & 15;
-        const int64_t t = t0 + tx;
-        if (n < N && t < p.seqlen) (k < 16 ? p.dB : p.dC)[(b * N + n) * p.seqlen + t] = tile[tx][k];
+#pragma unroll
+        for (int k = 0; k < kRep; ++k) acc += __ldcg(p.rep + ((k * 2 + which) * p.batch + b) * (int64_t)kNS * L + n * L + t);
+        dst[t] = acc;
     }
 }
 
-template <typename T, bool SP, bool GATE>
-cudaError_t launch_t(const BwdParams &p, int sm_count, cudaStream_t st) {
-    auto kern = scan_bwd_kernel<T, SP, GATE>;
-    const int smem = kBlockFloats * 4;
+template <typename T, bool SP, bool GATE, int WARPS>
+cudaError_t launch_w(const BwdParams &p, int sm_count, cudaStream_t st) {
+    auto kern = scan_bwd_kernel<T, SP, GATE, WARPS>;
+    const int smem = BwdSmem<T, WARPS>::BYTES;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWarpsBwd * 32, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WARPS * 32, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
     int64_t grid = (int64_t)sm_count * per_sm;  // one block per channel group, grid-strided
     if (grid > p.n_groups) grid = p.n_groups;
-    kern<<<(unsigned)grid, kWarpsBwd * 32, smem, st>>>(p);
+    kern<<<(unsigned)grid, WARPS * 32, smem, st>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int64_t blocks = p.batch * ((p.seqlen + 31) / 32);
+    const int64_t items = 2 * p.batch * p.dstate * ((p.seqlen + 3) / 4);
+    const int64_t blocks = (items + 255) / 256;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    bwd_reduce_bc_kernel<<<(unsigned)blocks, 256, 0, st>>>(p);
+    bwd_sum_copies_kernel<<<(unsigned)blocks, 256, 0, st>>>(p);
     return cudaGetLastError();
 }
 
+template <typename T, bool SP, bool GATE>
+cudaError_t launch_t(const BwdParams &p, int warps, int sm_count, cudaStream_t st) {
+    return warps == 6 ? launch_w<T, SP, GATE, 6>(p, sm_count, st) : launch_w<T, SP, GATE, 4>(p, sm_count, st);
+}
+
 template <typename T>
-cudaError_t launch_typed(const BwdParams &p, int sm_count, cudaStream_t st) {
+cudaError_t launch_typed(const BwdParams &p, int warps, int sm_count, cudaStream_t st) {
     const bool gate = p.z != nullptr;
-    if (p.softplus) return gate ? launch_t<T, true, true>(p, sm_count, st) : launch_t<T, true, false>(p, sm_count, st);
-    return gate ? launch_t<T, false, true>(p, sm_count, st) : launch_t<T, false, false>(p, sm_count, st);
+    if (p.softplus)
+        return gate ? launch_t<T, true, true>(p, warps, sm_count, st) : launch_t<T, true, false>(p, warps, sm_count, st);
+    return gate ? launch_t<T, false, true>(p, warps, sm_count, st) : launch_t<T, false, false>(p, warps, sm_count, st);
+}
+
+// Warps per block.  A channel group's adjoint runs through the sequence in
+// order, so the groups are the units of work and the SM that holds the most
+// of them sets the time: pick the block size whose busiest SM carries the
+// fewest warps, all blocks resident (bf16: 5 blocks of 4 warps or 3 of 6 per
+// SM).  Mamba-2.8B layer: 640 groups of 32 channels (5 on some SMs: 20
+// warps) against 428 of 48 (3 per SM: 18 warps).
+int bwd_warps(int64_t batch, int64_t dim, int act, int sm_count) {
+    const int64_t g4 = batch * ((dim + 31) / 32), g6 = batch * ((dim + 47) / 48);
+    const int64_t slots4 = (int64_t)sm_count * (act == kBF16 ? 5 : 3), slots6 = (int64_t)sm_count * (act == kBF16 ? 3 : 2);
+    if (g6 > slots6 || g4 > slots4) return 4;
+    const int64_t load4 = 4 * ((g4 + sm_count - 1) / sm_count), load6 = 6 * ((g6 + sm_count - 1) / sm_count);
+    return load6 < load4 ? 6 : 4;
 }
 
 }  // namespace
 
-size_t scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen) {
-    const int64_t groups = batch * ((dim + 31) / 32);
-    const int64_t segs = (seqlen + kSeg - 1) / kSeg;
-    return (size_t)(groups * segs * 32 * kNS) * 4 + (size_t)(groups * seqlen * 32) * 4;
+int64_t scan_bwd_ckpt_floats(int64_t batch, int64_t dim, int64_t seqlen) {
+    const int64_t groups = batch * ((dim + kCkCh - 1) / kCkCh);
+    return groups * ((seqlen + kSup - 1) / kSup) * kCkCh * kNS;
 }
 
-cudaError_t launch_scan_bwd(const ScanBwdArgs &a, void *workspace, int sm_count, cudaStream_t st) {
+int scan_bwd_ckpt_interval() { return kSup; }
+
+namespace {
+struct BwdLayout {
+    size_t ck, sub, rep, bytes;  // offsets of the checkpoints, sub-checkpoints, dB / dC copies
+};
+BwdLayout bwd_layout(int64_t batch, int64_t dim, int64_t seqlen) {
+    // threads over all groups, for either block size (4 warps: 32 channels per group, 6: 48)
+    const int64_t t4 = ((dim + 31) / 32) * 128, t6 = ((dim + 47) / 48) * 192;
+    const int64_t threads = batch * (t4 > t6 ? t4 : t6);
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    BwdLayout l;
+    l.ck = 0;
+    l.sub = up((size_t)scan_bwd_ckpt_floats(batch, dim, seqlen) * 4);
+    // sub-checkpoints: per group, kNSub x (its threads) x 4 states of up to 8 bytes
+    l.rep = l.sub + up((size_t)(threads * kNSub * kSPL) * 8);
+    l.bytes = l.rep + (size_t)(kRep * 2 * batch * kNS * seqlen) * 4;
+    return l;
+}
+}  // namespace
+
+size_t scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen) {
+    return bwd_layout(batch, dim, seqlen).bytes;
+}
+
+cudaError_t launch_scan_bwd(const ScanBwdArgs &a, void *workspace, const float *ckpt, int sm_count,
+                            cudaStream_t st) {
     BwdParams p;
     p.u = a.u; p.delta = a.delta; p.B = a.B; p.C = a.C; p.z = a.z; p.dout = a.dout;
     p.A = a.A; p.D = a.D; p.delta_bias = a.delta_bias; p.dlast = a.dlast; p.h0 = a.h0;
     p.du = a.du; p.ddelta = a.ddelta; p.dz = a.dz;
     p.dA = a.dA; p.dB = a.dB; p.dC = a.dC; p.dD = a.dD; p.dbias = a.ddelta_bias; p.dh0 = a.dh0;
-    p.ckpt = static_cast<float *>(workspace);
-    p.part = p.ckpt + (size_t)((a.batch * ((a.dim + 31) / 32)) * ((a.seqlen + kSeg - 1) / kSeg)) * 32 * kNS;
+    const BwdLayout l = bwd_layout(a.batch, a.dim, a.seqlen);
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    p.ckpt = ckpt ? const_cast<float *>(ckpt) : reinterpret_cast<float *>(w + l.ck);
+    p.ckpt_given = ckpt ? 1 : 0;
+    p.subck = w + l.sub;
+    p.rep = reinterpret_cast<float *>(w + l.rep);
     {
         const int es = a.act == kBF16 ? 2 : 4, V = 16 / es;
         auto al = [](const void *q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
@@ -484,15 +654,20 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs &a, void *workspace, int sm_count,
                 al(a.du) && al(a.ddelta) && al(a.dz);
     }
     p.batch = a.batch; p.dim = a.dim; p.seqlen = a.seqlen; p.dstate = a.dstate; p.softplus = a.softplus;
-    p.groups_per_batch = (int)((a.dim + 31) / 32);
+    const int warps = bwd_warps(a.batch, a.dim, a.act, sm_count);
+    const int ch = warps * kCPW;
+    p.groups_per_batch = (int)((a.dim + ch - 1) / ch);
+    p.ckpt_g32 = (int)((a.dim + kCkCh - 1) / kCkCh);
     p.n_groups = (int)(a.batch * p.groups_per_batch);
-    p.n_segs = (int)((a.seqlen + kSeg - 1) / kSeg);
-    // the sums over channels and time accumulate into zeroed outputs
+    p.n_sup = (int)((a.seqlen + kSup - 1) / kSup);
+    // every sum over channels, time or batch rows accumulates into zeroed outputs
     cudaError_t e = cudaMemsetAsync(a.dA, 0, (size_t)(a.dim * a.dstate) * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(p.rep, 0, l.bytes - l.rep, st);
     if (e == cudaSuccess && a.dD) e = cudaMemsetAsync(a.dD, 0, (size_t)a.dim * 4, st);
     if (e == cudaSuccess && a.ddelta_bias) e = cudaMemsetAsync(a.ddelta_bias, 0, (size_t)a.dim * 4, st);
     if (e != cudaSuccess) return e;
-    return a.act == kBF16 ? launch_typed<__nv_bfloat16>(p, sm_count, st) : launch_typed<float>(p, sm_count, st);
+    return a.act == kBF16 ? launch_typed<__nv_bfloat16>(p, warps, sm_count, st)
+                          : launch_typed<float>(p, warps, sm_count, st);
 }
 
 }  // namespace mscan

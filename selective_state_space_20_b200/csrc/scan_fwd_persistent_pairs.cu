@@ -448,6 +448,16 @@ scan_fwd_pairs_kernel(const Params p) {
             const unsigned char *sbuf = base + st * W::STAGE;
             const int64_t t0 = tb0 + (int64_t)sub * kTC;
             const int tvalid = (L - t0) < kTC ? (int)(L - t0) : kTC;
+            // checkpoint for the backward pass: the state entering every 32nd step
+            if (!SO && p.ckpt != nullptr && (t0 & 31) == 0 && ds < Dm) {
+                float *dst = p.ckpt + (((b * p.ckpt_gpb + (ds >> 5)) * p.ckpt_nsup + (t0 >> 5)) * 32 + (ds & 31)) * 16 +
+                             S * sr;
+#pragma unroll
+                for (int k = 0; k < S / 4; ++k)
+                    __stcg(reinterpret_cast<float4 *>(dst) + k,
+                           make_float4((float)h[2 * k].x, (float)h[2 * k].y, (float)h[2 * k + 1].x,
+                                       (float)h[2 * k + 1].y));
+            }
 
             // ---- prologue (0), fused conv1d: this lane's PT inputs of its
             // channel and the 3 before them (from the row, or from the

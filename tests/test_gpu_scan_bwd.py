@@ -66,6 +66,15 @@ def test_bwd_matches_oracle(dtype, shape):
     check_bwd(*shape, dtype, seed=sum(shape))
 
 
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("h0", [False, True])
+def test_bwd_six_warp_blocks(dtype, h0):
+    """1 x 5120 channels: 48-channel blocks (6 warps) spread more evenly over
+    the SMs than 32-channel ones, so the kernel takes them; every gradient
+    against the oracle, with a ragged last 32-step piece."""
+    check_bwd(1, 5120, 72, 16, dtype, seed=77, h0=h0)
+
+
 @pytest.mark.parametrize("gate,softplus,dlast", [(False, True, True), (True, False, True), (True, True, False)])
 def test_bwd_flags(gate, softplus, dlast):
     for dtype in ("fp32", "bf16"):
@@ -142,3 +151,63 @@ def test_bwd_benchmark_layer_sampled():
     record("scan_bwd mamba-2.8b layer sampled channels", **errs)
     for k, e in errs.items():
         assert e <= grad_tol(k, "bf16"), (k, e, errs)
+
+
+# ------------------------------------------------ checkpoints from the forward
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("shape", [(2, 37, 104, 16), (1, 64, 256, 16), (3, 20, 40, 5), (2, 96, 512, 16),
+                                   (1, 33, 8, 16)])
+@pytest.mark.parametrize("h0", [False, True])
+def test_bwd_from_forward_checkpoints(dtype, shape, h0):
+    """mamba_scan_fwd_ckpt keeps the state every 32 steps; mamba_scan_bwd_ckpt
+    recomputes from them instead of sweeping the inputs: the forward's outputs
+    and every gradient against the oracle."""
+    batch, dim, L, N = shape
+    w = inputs.custom(batch, dim, L, N, dtype, seed=sum(shape) + 11)
+    cpu = inputs.scan_inputs(w)
+    g = torch.Generator().manual_seed(sum(shape) + 12)
+    dout = torch.randn(batch, dim, L, generator=g).to(inputs.DTYPES[dtype])
+    dl = torch.randn(batch, dim, N, generator=g)
+    hs = inputs.initial_state(batch, dim, N, seed=sum(shape) + 13) if h0 else None
+    dev = {k: (None if v is None else v.cuda()) for k, v in cpu.items()}
+    out, last, ck = binding.mamba_scan_fwd_ckpt(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],
+                                                z=dev["z"], delta_bias=dev["delta_bias"],
+                                                h0=None if hs is None else hs.cuda())
+    got = binding.mamba_scan_bwd(dout.cuda(), dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],
+                                 z=dev["z"], delta_bias=dev["delta_bias"], dlast_state=dl.cuda(),
+                                 h0=None if hs is None else hs.cuda(), ckpt=ck)
+    ro, rs = oracle.scan(cpu["u"], cpu["delta"], cpu["A"], cpu["B"], cpu["C"], D=cpu["D"], z=cpu["z"],
+                         delta_bias=cpu["delta_bias"], h0=hs)
+    tol = TOL[inputs.DTYPES[dtype]]
+    assert rel_err(to_np(out), ro) <= tol and rel_err(to_np(last), rs) <= tol
+    ref = oracle.scan_bwd(dout, cpu["u"], cpu["delta"], cpu["A"], cpu["B"], cpu["C"], D=cpu["D"], z=cpu["z"],
+                          delta_bias=cpu["delta_bias"], h0=hs, dlast=dl.double())
+    errs = {k: rel_err(to_np(got[k]), ref[k]) for k in FP32_GRADS + ACT_GRADS + (("dh0",) if h0 else ())}
+    record(f"scan_bwd from forward checkpoints {batch}x{dim}x{L} N{N} {dtype} h0={h0}", **errs)
+    for k, e in errs.items():
+        assert e <= grad_tol(k, dtype), (k, e, errs)
+
+
+def test_forward_checkpoints_hold_the_states():
+    """Entry s of the checkpoints is the state entering step 32 s: compared
+    with the final state of a scan over the first 32 s steps."""
+    w = inputs.custom(2, 70, 160, 16, "bf16", seed=91)
+    dev = inputs.scan_inputs(w, device="cuda")
+    _, _, ck = binding.mamba_scan_fwd_ckpt(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],
+                                           z=dev["z"], delta_bias=dev["delta_bias"])
+    g32 = (w.dim + 31) // 32
+    ck = ck[: w.batch * g32 * 5 * 32 * 16].view(w.batch, g32, 5, 32, 16)
+    for s in (1, 3, 4):
+        head = {k: (v[..., :32 * s].contiguous() if k in ("u", "delta", "z", "B", "C") else v) for k, v in dev.items()}
+        _, st = binding.mamba_scan_fwd(head["u"], head["delta"], head["A"], head["B"], head["C"], D=head["D"],
+                                       z=head["z"], delta_bias=head["delta_bias"], return_last_state=True)
+        flat = ck[:, :, s].reshape(w.batch, g32 * 32, 16)[:, :w.dim]
+        assert rel_err(to_np(flat), to_np(st)) <= 1e-3
+    assert torch.all(ck[:, :, 0].reshape(w.batch, g32 * 32, 16)[:, :w.dim] == 0)  # entering step 0: zeros
+
+
+def test_forward_checkpoints_reject_unsupported_layouts():
+    w = inputs.custom(1, 32, 60, 16, "bf16", seed=92)  # L not a multiple of 8
+    d = {k: (None if v is None else v.cuda()) for k, v in inputs.scan_inputs(w).items()}
+    with pytest.raises(binding.MambaError):
+        binding.mamba_scan_fwd_ckpt(d["u"], d["delta"], d["A"], d["B"], d["C"])
