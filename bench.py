@@ -652,9 +652,13 @@ def conv1d_measure(reps=20):
 def backward_measure(reps=5):
     """The scan's backward pass on the benchmark layer (Mamba-2.8B shape,
     bf16): every input gradient for a random dL/dout and dL/dlast_state.
-    The roof counts the decays the gradients need at least once (16 per
-    element, N = 16) on the MUFU; this kernel evaluates them three times
-    (checkpoint pass, segment recompute, reverse pass)."""
+    Timed two ways: from the checkpoints the forward keeps (mamba_scan_fwd_ckpt
+    then mamba_scan_bwd_ckpt, the training path; the forward's extra cost is
+    reported beside) and self-contained (mamba_scan_bwd, which sweeps the
+    inputs for its checkpoints first).  The roof counts the decays the
+    gradients need at least once (16 per element, N = 16) on the MUFU; the
+    kernel evaluates them twice from checkpoints (the 32-step recompute and
+    the 4-step window recompute), three times self-contained."""
     w = inputs.MAMBA_2_8B
     d = inputs.scan_inputs(w, device="cuda")
     g = torch.Generator(device="cuda").manual_seed(7)
@@ -662,27 +666,35 @@ def backward_measure(reps=5):
     dlast = torch.randn(w.batch, w.dim, w.dstate, generator=g, device="cuda")
     ws = torch.empty(binding.load_library().mamba_scan_bwd_workspace_size(w.batch, w.dim, w.seqlen, w.dstate),
                      device="cuda", dtype=torch.uint8)
-    run = lambda: binding.mamba_scan_bwd(dout, d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"],  # noqa: E731
-                                         z=d["z"], delta_bias=d["delta_bias"], dlast_state=dlast,
-                                         workspace=ws)
-    run()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        run()
-    e1.record()
-    torch.cuda.synchronize()
-    us = e0.elapsed_time(e1) * 1e3 / reps
+    kw = dict(D=d["D"], z=d["z"], delta_bias=d["delta_bias"])
+    out = torch.empty_like(d["u"])
+    last = torch.empty(w.batch, w.dim, w.dstate, device="cuda")
+    _, _, ck = binding.mamba_scan_fwd_ckpt(d["u"], d["delta"], d["A"], d["B"], d["C"], out=out, last_state=last, **kw)
+    bwd_ck = lambda: binding.mamba_scan_bwd(dout, d["u"], d["delta"], d["A"], d["B"], d["C"],  # noqa: E731
+                                            dlast_state=dlast, workspace=ws, ckpt=ck, **kw)
+    bwd_self = lambda: binding.mamba_scan_bwd(dout, d["u"], d["delta"], d["A"], d["B"], d["C"],  # noqa: E731
+                                              dlast_state=dlast, workspace=ws, **kw)
+    fwd = lambda: binding.mamba_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], out=out,  # noqa: E731
+                                         last_state=last, **kw)
+    fwd_ck = lambda: binding.mamba_scan_fwd_ckpt(d["u"], d["delta"], d["A"], d["B"], d["C"], out=out,  # noqa: E731
+                                                 last_state=last, ckpt=ck, **kw)
+    us = _median_us(bwd_ck, reps)
+    us_self = _median_us(bwd_self, reps)
+    us_fwd, us_fwd_ck = _median_us(fwd, 20), _median_us(fwd_ck, 20)
     peak = MUFU_PER_CLK_PER_SM * SM_COUNT * load_peaks()["sm_max_mhz"] * 1e6 / w.dstate / 1e9
     achieved = w.elements / us / 1e3
-    return {"workload": w.name, "us_per_call": us, "Gelem_per_s": achieved,
+    return {"workload": w.name, "entry": "mamba_scan_bwd_ckpt (checkpoints from mamba_scan_fwd_ckpt)",
+            "us_per_call": us, "Gelem_per_s": achieved,
             "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Gelem/s",
                          "frac": achieved / peak,
                          "traffic": measured_traffic(f"scan_bwd_kernel {w.name}"),
-                         "note": "peak = 16 decays per element once on the MUFU; the kernel evaluates them 3x "
-                                 "(checkpoint sweep, segment recompute, reverse sweep)"},
-            "reps": reps}
+                         "note": "peak = 16 decays per element once on the MUFU; from checkpoints the kernel "
+                                 "evaluates them twice (32-step recompute, 4-step window recompute)"},
+            "self_contained": {"entry": "mamba_scan_bwd", "us_per_call": us_self,
+                               "Gelem_per_s": w.elements / us_self / 1e3},
+            "forward_checkpoint_cost": {"mamba_scan_fwd_us": us_fwd, "mamba_scan_fwd_ckpt_us": us_fwd_ck,
+                                        "checkpoint_bytes": ck.numel() * 4},
+            "reps": reps, "deterministic": "du, ddelta, dz yes; dA, dB, dC, dD, dbias sum with atomics"}
 
 
 def complex_measure(reps=10):
@@ -719,6 +731,83 @@ def complex_measure(reps=10):
             "reps": reps, "l2": "inputs larger than L2, no flush"}
 
 
+def seqpar_shard(w, world, rank, device):
+    """This rank's shard of one sequence of workload ``w``: timesteps
+    [rank L / world, (rank + 1) L / world), drawn with seed + rank; the
+    per-channel parameters (A, D, bias) are the base seed's on every rank."""
+    Lr = w.seqlen // world
+    shard = inputs.scan_inputs(dataclasses.replace(w, seqlen=Lr, seed=w.seed + rank), device=device)
+    params = inputs.scan_inputs(dataclasses.replace(w, batch=1, seqlen=8), device=device)
+    for k in ("A", "D", "delta_bias"):
+        shard[k] = params[k]
+    return shard, Lr
+
+
+def seqpar_run(w, world, rank, steps, warmup, device, ops=None, group=None):
+    """Time `steps` calls of the sequence split (each rank scans its shard
+    from zero, the ranks all-gather the shard summaries, each folds the shards
+    before it and scans its shard again) after `warmup` untimed ones; returns
+    (max over ranks of the time per step in ms, elements per step of the
+    whole sequence).  ``ops`` replaces the per-shard steps (CPU stand-ins in
+    the multi-process test)."""
+    import torch.distributed as dist
+    from selective_state_space_20_b200 import seqpar
+    shard, Lr = seqpar_shard(w, world, rank, device)
+    run = lambda: seqpar.scan_sequence_parallel(shard["u"], shard["delta"], shard["A"], shard["B"],  # noqa: E731
+                                                shard["C"], D=shard["D"], z=shard["z"],
+                                                delta_bias=shard["delta_bias"], group=group, _ops=ops)
+    for _ in range(warmup):
+        run()
+    on_gpu = device.type == "cuda"
+    if on_gpu:
+        torch.cuda.synchronize()
+    dist.barrier(group)
+    if on_gpu:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        run()
+    if on_gpu:
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+    else:
+        ms = (time.perf_counter() - t0) * 1e3
+    dist.barrier(group)
+    ms = max_over_ranks(ms, world)
+    return ms / steps, w.batch * w.dim * Lr * world
+
+
+def seqpar_main(args, world, rank, local):
+    """--seqpar: the long-context layer as ONE sequence split over the ranks
+    (strong scaling: the whole job is one 1 x 2048 x 262144 scan)."""
+    if world > 1 and not torch.distributed.is_initialized():
+        raise SystemExit("--seqpar with several ranks needs the launcher's process group")
+    if world == 1 and not torch.distributed.is_initialized():  # a group of one: the exchange is trivial
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", str(29500 + os.getpid() % 1000))
+        dist.init_process_group("nccl", rank=0, world_size=1)
+    w = inputs.LONG_CONTEXT
+    dev = torch.device("cuda", torch.cuda.current_device())
+    binding.load_library()
+    ms, elems = seqpar_run(w, world, rank, args.steps, args.warmup, dev)
+    if rank == 0:
+        line = {"metric": METRIC, "value": elems / (ms * 1e-3) / 1e9, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": f"{w.name}, one sequence split over {world} ranks",
+                           "batch": w.batch, "dim": w.dim, "seqlen": w.seqlen, "dstate": w.dstate,
+                           "act_dtype": w.dtype, "seqlen_per_rank": w.seqlen // world,
+                           "exchange": "all-gather of per-shard (delta sums fp64, final states fp32) "
+                                       "through torch.distributed, then an fp64 fold",
+                           "l2": "inputs larger than L2"},
+                "gpu_launches": args.steps * (4 if world > 1 else 3)}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -732,6 +821,8 @@ def main():
     ap.add_argument("--no-bwd", action="store_true")
     ap.add_argument("--no-complex", action="store_true")
     ap.add_argument("--no-layers", action="store_true", help="skip the Mamba-130M / long-context / workspace sections")
+    ap.add_argument("--seqpar", action="store_true",
+                    help="time one long-context sequence split over the ranks (seqpar.scan_sequence_parallel)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -744,6 +835,11 @@ def main():
         return rc
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
+    if args.seqpar:
+        rc = seqpar_main(args, world, rank, local)
+        if torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+        return rc
 
     w = WORKLOAD
     dev = torch.device("cuda", torch.cuda.current_device())

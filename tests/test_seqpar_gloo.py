@@ -98,3 +98,34 @@ def test_sequence_split_matches_one_scan(world, with_h0):
     assert got.shape == ro.shape
     assert np.max(np.abs(got - ro)) <= 1e-10 * max(1.0, np.max(np.abs(ro)))
     assert np.max(np.abs(res[world - 1][1] - rs)) <= 1e-10 * max(1.0, np.max(np.abs(rs)))
+
+
+def _bench_worker(rank, world, port, q):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import bench
+    from selective_state_space_20_b200 import inputs
+    w, r, _ = bench.dist_setup()
+    wl = inputs.custom(1, 6, 64, 4, "fp32", seed=5, name="tiny split")
+    ms, elems = bench.seqpar_run(wl, w, r, steps=2, warmup=1, device=torch.device("cpu"), ops=_cpu_ops())
+    import torch.distributed as dist
+    dist.destroy_process_group()
+    q.put((r, ms, elems))
+
+
+def test_bench_sequence_split_mode_two_ranks():
+    """bench.py --seqpar's timing loop on two gloo ranks with the CPU
+    stand-ins: every rank reports the same (maximum) time per step and the
+    elements of the whole sequence."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_bench_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+        assert p.exitcode == 0
+    res = {r: (ms, el) for r, ms, el in (q.get(timeout=10) for _ in range(world))}
+    assert res[0] == res[1] and res[0][0] > 0 and res[0][1] == 1 * 6 * 64
