@@ -6,12 +6,14 @@
 //
 // The step is bound by HBM traffic: 2 * 4 * N bytes of state per channel
 // against ~N exponentials.  The main kernel gives each (batch, channel) row
-// N / 4 consecutive lanes, one 16-byte slice of the state each, so a warp's
-// state loads and stores cover whole contiguous 512-byte spans; the row's
-// readout is summed over its lanes with shuffles.  A rows are re-read by
-// every batch row and stay in L2, B and C rows are shared by all channels of a
-// batch row and stay in L1.  Other state sizes and unaligned tensors take a
-// thread-per-row kernel.  fp32 activations take the accurate decay of
+// a few lanes with two 16-byte state slices each (N = 16: two lanes), so a
+// warp's state loads and stores cover whole 32-byte sectors and the per-row
+// work (softplus, gate) is shared by fewer lanes; the row's readout is summed
+// over its lanes with shuffles.  Thread indices are 32-bit where they fit
+// (a 64-bit division by dim per thread cost ~20 % of the step).  A rows are
+// re-read by every batch row and stay in L2, B and C rows are shared by all
+// channels of a batch row and stay in L1.  Other state sizes and unaligned
+// tensors take a thread-per-row kernel.  fp32 activations take the accurate decay of
 // device_math.cuh (Decay<true>), bf16 ones one ex2 per state.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -99,57 +101,81 @@ template <> struct Quad<__nv_bfloat16> {
     }
 };
 
-// NV / 4 lanes per row (NV = dstate, a multiple of 4 up to 128); lane q of a
-// row owns states 4q .. 4q + 3.
-template <typename T, int NV>
+// NV / (4 V) = Q lanes per row (NV = dstate, a multiple of 4 up to 128);
+// lane q of a row owns the V 16-byte state slices q, q + Q, ..., so each load
+// or store instruction of a warp covers whole 32-byte sectors (a row's Q
+// lanes side by side), and a row's readout is summed over its lanes with
+// shuffles.  Every load is issued before the arithmetic.  W64: 64-bit thread
+// indices (more than 2^31 lanes).
+template <typename T, int NV, int V, bool W64>
 __global__ void __launch_bounds__(256)
 state_update_lanes_kernel(const SUParams p) {
-    constexpr int Q = NV / 4;
-    static_assert(Q >= 1 && Q <= 32 && (Q & (Q - 1)) == 0, "lanes per row: a power of two");
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const bool live = gid / Q < p.rows;
-    const int64_t row = live ? gid / Q : p.rows - 1;  // idle lanes still join the shuffles
+    constexpr int Q = NV / (4 * V);
+    static_assert(Q >= 1 && Q <= 32 && (Q & (Q - 1)) == 0 && Q * 4 * V == NV, "lanes per row: a power of two");
+    using Idx = typename std::conditional<W64, int64_t, unsigned>::type;
+    const Idx gid = (Idx)blockIdx.x * blockDim.x + threadIdx.x;
+    const Idx rows = (Idx)p.rows, dim = (Idx)p.dim;
+    const bool live = gid / Q < rows;
+    const Idx row = live ? gid / Q : rows - 1;  // idle lanes still join the shuffles
     const int qi = (int)(gid % Q);
-    const int64_t b = row / p.dim, d = row % p.dim;
-    const T *gu = static_cast<const T *>(p.u);
-    const T *gd = static_cast<const T *>(p.delta);
-    const T *gz = static_cast<const T *>(p.z);
+    const Idx b = row / dim, d = row - b * dim;
     using Dk = Decay<sizeof(T) == 4>;
+    using HS = typename Dk::H;  // fp64 for fp32 activations
 
-    float dl = Elem<T>::load(gd + row) + (p.delta_bias ? __ldg(p.delta_bias + d) : 0.f);
+    float4 h4[V], a4[V], b4[V], c4[V];
+    float4 *st = reinterpret_cast<float4 *>(p.state + (int64_t)row * NV) + qi;
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+        h4[v] = st[v * Q];
+        a4[v] = __ldg(reinterpret_cast<const float4 *>(p.A + (int64_t)d * NV) + qi + v * Q);
+        b4[v] = Quad<T>::load(static_cast<const T *>(p.B) + (int64_t)b * NV + 4 * (qi + v * Q));
+        c4[v] = Quad<T>::load(static_cast<const T *>(p.C) + (int64_t)b * NV + 4 * (qi + v * Q));
+    }
+    const float dr = Elem<T>::load(static_cast<const T *>(p.delta) + row);
+    const float ut = Elem<T>::load(static_cast<const T *>(p.u) + row);
+    const float zt = (p.z && qi == 0) ? Elem<T>::load(static_cast<const T *>(p.z) + row) : 0.f;
+    const float bias = p.delta_bias ? __ldg(p.delta_bias + d) : 0.f;
+    const float Dd = (p.D && qi == 0) ? __ldg(p.D + d) : 0.f;
+
+    float dl = dr + bias;
     if (p.softplus) dl = Dk::softplus(dl);
-    const float ut = Elem<T>::load(gu + row);
     const float du = dl * ut;
     const float dl2 = dl * Dk::kScale;
-    float4 *st = reinterpret_cast<float4 *>(p.state + row * NV) + qi;
-    const float4 h4 = *st;
-    const float4 a4 = __ldg(reinterpret_cast<const float4 *>(p.A + d * NV) + qi);
-    const float4 b4 = Quad<T>::load(static_cast<const T *>(p.B) + b * NV + 4 * qi);
-    const float4 c4 = Quad<T>::load(static_cast<const T *>(p.C) + b * NV + 4 * qi);
-    using HS = typename Dk::H;  // fp64 for fp32 activations
-    const HS hx = Dk::step(dl2 * a4.x, (HS)h4.x, du * b4.x);
-    const HS hy = Dk::step(dl2 * a4.y, (HS)h4.y, du * b4.y);
-    const HS hz = Dk::step(dl2 * a4.z, (HS)h4.z, du * b4.z);
-    const HS hw = Dk::step(dl2 * a4.w, (HS)h4.w, du * b4.w);
-    HS y = fma((HS)c4.x, hx, fma((HS)c4.y, hy, fma((HS)c4.z, hz, (HS)c4.w * hw)));
+    HS y = 0.f;
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+        const HS hx = Dk::step(dl2 * a4[v].x, (HS)h4[v].x, du * b4[v].x);
+        const HS hy = Dk::step(dl2 * a4[v].y, (HS)h4[v].y, du * b4[v].y);
+        const HS hz = Dk::step(dl2 * a4[v].z, (HS)h4[v].z, du * b4[v].z);
+        const HS hw = Dk::step(dl2 * a4[v].w, (HS)h4[v].w, du * b4[v].w);
+        y += fma((HS)c4[v].x, hx, fma((HS)c4[v].y, hy, fma((HS)c4[v].z, hz, (HS)c4[v].w * hw)));
+        h4[v] = make_float4((float)hx, (float)hy, (float)hz, (float)hw);
+    }
 #pragma unroll
     for (int o = Q / 2; o >= 1; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
     if (!live) return;
-    *st = make_float4((float)hx, (float)hy, (float)hz, (float)hw);
+#pragma unroll
+    for (int v = 0; v < V; ++v) st[v * Q] = h4[v];
     if (qi == 0) {
         float yo = (float)y;
-        if (p.D) yo = (float)fma((HS)__ldg(p.D + d), (HS)ut, y);
-        if (gz) yo *= silu_f(Elem<T>::load(gz + row));
+        if (p.D) yo = (float)fma((HS)Dd, (HS)ut, y);
+        if (p.z) yo *= silu_f(zt);
         Elem<T>::store(static_cast<T *>(p.out) + row, yo);
     }
 }
 
 template <typename T, int NV>
 static cudaError_t launch_lanes(const SUParams &kp, cudaStream_t st) {
-    const int threads = 256;
-    const int64_t blocks = (kp.rows * (NV / 4) + threads - 1) / threads;
+    constexpr int threads = 256;
+    constexpr int V = NV >= 8 ? 2 : 1;  // 16-byte state slices per lane
+    constexpr int Q = NV / (4 * V);
+    const int64_t lanes = kp.rows * Q;
+    const int64_t blocks = (lanes + threads - 1) / threads;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    state_update_lanes_kernel<T, NV><<<(unsigned)blocks, threads, 0, st>>>(kp);
+    if (blocks * threads < 0x7fffffffLL)
+        state_update_lanes_kernel<T, NV, V, false><<<(unsigned)blocks, threads, 0, st>>>(kp);
+    else
+        state_update_lanes_kernel<T, NV, V, true><<<(unsigned)blocks, threads, 0, st>>>(kp);
     return cudaGetLastError();
 }
 
@@ -176,7 +202,7 @@ static cudaError_t launch_rows(const SUParams &kp, cudaStream_t st) {
 template <typename T>
 static cudaError_t launch_typed(const SUParams &kp, cudaStream_t st) {
     auto al = [](const void *q, uintptr_t m) { return (reinterpret_cast<uintptr_t>(q) & (m - 1)) == 0; };
-    const uintptr_t bc_align = 4 * sizeof(T);  // four B / C values per lane
+    const uintptr_t bc_align = 4 * sizeof(T);  // four B / C values per load
     if (al(kp.state, 16) && al(kp.A, 16) && al(kp.B, bc_align) && al(kp.C, bc_align)) {
         if (kp.dstate == 16) return launch_lanes<T, 16>(kp, st);
         if (kp.dstate == 8) return launch_lanes<T, 8>(kp, st);
