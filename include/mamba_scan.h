@@ -280,16 +280,27 @@ typedef struct {
  *                  pointer and strides; any other overlap of out, last_state
  *                  or h0 with an input is rejected (MAMBA_ERR_OVERLAP, judged
  *                  on each tensor's address span).
- *   tuning       : NULL, or schedule AUTO / STATIC with optional lanes and
- *                  threads (the persistent schedule needs the dense layout).
+ *   tuning       : NULL, or schedule AUTO / LOCAL / STATIC with optional
+ *                  lanes and threads (PERSISTENT needs the dense layout and a
+ *                  workspace: MAMBA_ERR_UNSUPPORTED).
  *
- * Uses the static schedule.  16-byte copies are used where a tensor allows
- * them: channel-contiguous u / delta / z / out (row stride 1) with 16-byte-
- * aligned pointers, batch and time strides multiples of 8 (bf16) or 4 (fp32)
- * elements and dim a multiple of the same; time-contiguous ones likewise
- * with the row stride and seqlen; B and C likewise along time or along
- * states.  Anything else is read and written element by element (correct,
- * slower).  Other arguments, results and errors as mamba_scan_fwd.
+ * The pages' own layout -- u, delta, z and out dense (batch, seqlen, dim),
+ * i.e. strides (seqlen dim, 1, dim), and B, C dense (batch, seqlen, dstate),
+ * strides (seqlen dstate, 1, dstate) -- runs on the block-local lane-split
+ * kernel of mamba_scan_fwd (no workspace), staging each timestep's channels
+ * with 16-byte copies: results bit-equal to mamba_scan_fwd on the same values
+ * laid out densely with the same lane count.  It needs dstate <= 16, dim and
+ * dstate multiples of 8 (bf16) or 4 (fp32), 16-byte-aligned pointers, lanes
+ * 0 / 2 / 4 and no block size; schedule LOCAL insists on it
+ * (MAMBA_ERR_UNSUPPORTED otherwise), AUTO falls back to the static kernel.
+ * Every other layout, and schedule STATIC, uses the static schedule.  There
+ * 16-byte copies are used where a tensor allows them: channel-contiguous u /
+ * delta / z / out (row stride 1) with 16-byte-aligned pointers, batch and
+ * time strides multiples of 8 (bf16) or 4 (fp32) elements and dim a multiple
+ * of the same; time-contiguous ones likewise with the row stride and seqlen;
+ * B and C likewise along time or along states.  Anything else is read and
+ * written element by element (correct, slower).  Other arguments, results
+ * and errors as mamba_scan_fwd.
  */
 int mamba_scan_fwd_strided(const void *u, const void *delta, const float *A,
                            const void *B, const void *C, const float *D,

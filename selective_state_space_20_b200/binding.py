@@ -293,12 +293,16 @@ def mamba_scan_fwd_strided(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor
                            delta_softplus: bool = True, out: Optional[torch.Tensor] = None,
                            last_state: Optional[torch.Tensor] = None,
                            return_last_state: bool = False, h0: Optional[torch.Tensor] = None,
-                           lanes_per_channel: int = 0, threads_per_block: int = 0):
+                           lanes_per_channel: int = 0, threads_per_block: int = 0,
+                           schedule: int = SCHEDULE_AUTO):
     """:func:`mamba_scan_fwd` on tensors with any strides: u, delta, z (and
     out) of logical shape (batch, dim, L) and B, C of (batch, N, L), each
     laid out however it is -- e.g. ``x.transpose(1, 2)`` of a (batch, L, dim)
     activation, or a slice of a wider projection output.  ``out`` is
-    allocated channel-contiguous like u when u is.  Static schedule."""
+    allocated channel-contiguous like u when u is.  Dense (batch, L, dim)
+    activations with dense (batch, L, N) B / C run the block-local lane-split
+    kernel (SCHEDULE_AUTO or SCHEDULE_LOCAL, lanes 0 / 2 / 4, no block size
+    given); every other layout, or SCHEDULE_STATIC, the static kernel."""
     if u.dim() != 3:
         raise ValueError("u must be (batch, dim, seqlen)")
     batch, dim, L = u.shape
@@ -329,7 +333,7 @@ def mamba_scan_fwd_strided(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor
     _need(last_state, "last_state", dev, torch.float32, (batch, dim, N))
     _need(h0, "h0", dev, torch.float32, (batch, dim, N))
     st = ScanStrides(_stride3(u), _stride3(delta), _stride3(z), _stride3(out), _stride3(B), _stride3(C))
-    tun = Tuning(int(lanes_per_channel), int(threads_per_block), SCHEDULE_STATIC, 0)
+    tun = Tuning(int(lanes_per_channel), int(threads_per_block), int(schedule), 0)
     lib = load_library()
     with torch.cuda.device(dev):
         rc = lib.mamba_scan_fwd_strided(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),

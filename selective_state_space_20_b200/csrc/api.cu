@@ -267,9 +267,11 @@ int mamba_scan_fwd_strided(const void *u, const void *delta, const float *A, con
     int rc = check_sizes(batch, dim, seqlen, dstate);
     if (rc != MAMBA_OK) return rc;
     if (!u || !delta || !A || !B || !C || !out) return MAMBA_ERR_NULL;
-    int want_lanes = 0, want_threads = 0;
+    int want_lanes = 0, want_threads = 0, want_sched = MAMBA_SCHEDULE_AUTO;
     if (tuning) {
-        if (tuning->schedule != MAMBA_SCHEDULE_AUTO && tuning->schedule != MAMBA_SCHEDULE_STATIC)
+        want_sched = tuning->schedule;
+        if (want_sched != MAMBA_SCHEDULE_AUTO && want_sched != MAMBA_SCHEDULE_STATIC &&
+            want_sched != MAMBA_SCHEDULE_LOCAL)
             return MAMBA_ERR_UNSUPPORTED;
         want_lanes = tuning->lanes_per_channel;
         want_threads = tuning->threads_per_block;
@@ -331,6 +333,32 @@ int mamba_scan_fwd_strided(const void *u, const void *delta, const float *A, con
     a.strides = &ks;
     a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = (int)dstate;
     a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
+    // The pages' own layout -- (batch, L, dim) activations and (batch, L, N)
+    // B / C, each dense -- runs on the block-local lane-split kernel with
+    // channel-last staging; any other layout, or an explicit static
+    // schedule or block size, on the static kernel.
+    const mamba_stride3_t xcl{seqlen * dim, 1, dim}, bccl{seqlen * dstate, 1, dstate};
+    const bool cl_layout = same_stride(st.u, xcl) && same_stride(st.delta, xcl) && (!z || same_stride(st.z, xcl)) &&
+                           same_stride(st.out, xcl) && same_stride(st.B, bccl) && same_stride(st.C, bccl);
+    a.channels_last = true;
+    const bool cl_ok = cl_layout && mscan::channels_last_supported(a);
+    a.channels_last = false;
+    if (want_sched == MAMBA_SCHEDULE_LOCAL &&
+        (!cl_ok || want_threads != 0 || (want_lanes != 0 && want_lanes != 2 && want_lanes != 4)))
+        return MAMBA_ERR_UNSUPPORTED;
+    if (cl_ok && want_sched != MAMBA_SCHEDULE_STATIC && want_threads == 0 &&
+        (want_lanes == 0 || want_lanes == 2 || want_lanes == 4)) {
+        a.strides = nullptr;
+        a.channels_last = true;
+        int lanes = want_lanes != 0 ? want_lanes : mscan::local_choose_lanes(a, sms);
+        if (lanes == 0 && want_sched == MAMBA_SCHEDULE_LOCAL) lanes = 2;
+        if (lanes != 0) {
+            note_workspace(nullptr);
+            return mscan::launch_scan_fwd_local(a, lanes, sms, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+        }
+        a.strides = &ks;
+        a.channels_last = false;
+    }
     mscan::ScanPlan pl;
     if (mscan::make_scan_plan(a, want_lanes, want_threads, sms, &pl) != 0) return MAMBA_ERR_UNSUPPORTED;
     return mscan::launch_scan_fwd(a, pl, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;

@@ -19,6 +19,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "device_math.cuh"
 #include "internal.h"
 
@@ -40,19 +42,22 @@ __device__ __forceinline__ float load_elem(const T *p) { return Elem<T>::load(p)
 // its NT 16-byte loads first (NT x 512 bytes in flight per warp), then the
 // tiles are finished in order, each taking the inputs before a lane's chunk
 // from the lane before it, and lane 0 from lane 31 of the previous tile.
-template <typename T, int K, int NT>
+// W64: 64-bit index arithmetic (more than 2^31 threads); otherwise 32-bit,
+// whose divisions cost a fraction of the 64-bit ones.
+template <typename T, int K, int NT, bool W64>
 __global__ void __launch_bounds__(256) conv1d_tiles_kernel(const ConvParams p) {
+    using Idx = typename std::conditional<W64, int64_t, unsigned>::type;
     constexpr int V = 16 / (int)sizeof(T);  // elements per 16-byte chunk
     constexpr int TILE = 32 * V;
     const int lane = threadIdx.x & 31;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t spans_per_row = (p.seqlen + NT * TILE - 1) / (NT * TILE);
-    const int64_t row = warp / spans_per_row;
-    if (row >= p.batch * p.dim) return;  // whole warp leaves together
-    const int64_t b = row / p.dim, d = row % p.dim;
-    const int64_t span0 = (warp % spans_per_row) * (NT * TILE);
-    const T *xr = static_cast<const T *>(p.x) + b * p.x_batch_stride + d * p.seqlen;
-    T *orow = static_cast<T *>(p.out) + row * p.seqlen;
+    const Idx warp = ((Idx)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const Idx spans_per_row = ((Idx)p.seqlen + NT * TILE - 1) / (NT * TILE);
+    const Idx row = warp / spans_per_row;
+    if (row >= (Idx)(p.batch * p.dim)) return;  // whole warp leaves together
+    const Idx b = row / (Idx)p.dim, d = row - b * (Idx)p.dim;
+    const int64_t span0 = (int64_t)(warp - row * spans_per_row) * (NT * TILE);
+    const T *xr = static_cast<const T *>(p.x) + (int64_t)b * p.x_batch_stride + (int64_t)d * p.seqlen;
+    T *orow = static_cast<T *>(p.out) + (int64_t)row * p.seqlen;
 
     uint4 raw[NT];
 #pragma unroll
@@ -68,7 +73,7 @@ __global__ void __launch_bounds__(256) conv1d_tiles_kernel(const ConvParams p) {
     }
     float wk[K];
 #pragma unroll
-    for (int k = 0; k < K; ++k) wk[k] = __ldg(p.w + d * K + k);
+    for (int k = 0; k < K; ++k) wk[k] = __ldg(p.w + (int64_t)d * K + k);
     const float bias = p.bias ? __ldg(p.bias + d) : 0.f;
 
 #pragma unroll
@@ -154,11 +159,17 @@ cudaError_t launch_fwd_typed(const ConvParams &p, cudaStream_t st) {
         const int64_t warps = p.batch * p.dim * ((p.seqlen + NT * TILE - 1) / (NT * TILE));
         const int64_t blocks = (warps * 32 + threads - 1) / threads;
         if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-        switch (p.width) {
-            case 1: conv1d_tiles_kernel<T, 1, NT><<<(unsigned)blocks, threads, 0, st>>>(p); break;
-            case 2: conv1d_tiles_kernel<T, 2, NT><<<(unsigned)blocks, threads, 0, st>>>(p); break;
-            case 3: conv1d_tiles_kernel<T, 3, NT><<<(unsigned)blocks, threads, 0, st>>>(p); break;
-            default: conv1d_tiles_kernel<T, 4, NT><<<(unsigned)blocks, threads, 0, st>>>(p); break;
+        const bool w64 = blocks * threads >= 0x7fffffffLL || p.seqlen >= 0x7fffffffLL;
+        const unsigned g = (unsigned)blocks;
+        switch (p.width * 2 + (w64 ? 1 : 0)) {
+            case 2: conv1d_tiles_kernel<T, 1, NT, false><<<g, threads, 0, st>>>(p); break;
+            case 3: conv1d_tiles_kernel<T, 1, NT, true><<<g, threads, 0, st>>>(p); break;
+            case 4: conv1d_tiles_kernel<T, 2, NT, false><<<g, threads, 0, st>>>(p); break;
+            case 5: conv1d_tiles_kernel<T, 2, NT, true><<<g, threads, 0, st>>>(p); break;
+            case 6: conv1d_tiles_kernel<T, 3, NT, false><<<g, threads, 0, st>>>(p); break;
+            case 7: conv1d_tiles_kernel<T, 3, NT, true><<<g, threads, 0, st>>>(p); break;
+            case 9: conv1d_tiles_kernel<T, 4, NT, true><<<g, threads, 0, st>>>(p); break;
+            default: conv1d_tiles_kernel<T, 4, NT, false><<<g, threads, 0, st>>>(p); break;
         }
         return cudaGetLastError();
     }

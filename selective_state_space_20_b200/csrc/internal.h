@@ -38,6 +38,10 @@ struct ScanArgs {
     // lane-split kernel only: checkpoints for the backward pass (the state
     // entering every scan_bwd_ckpt_interval() steps, its layout) or null
     float *ckpt = nullptr;
+    // lane-split block-local kernel only: u / delta / z / out dense
+    // (batch, L, dim) and B / C dense (batch, L, N) -- the layout of the
+    // Keras page -- instead of (batch, dim, L) / (batch, N, L)
+    bool channels_last = false;
     int64_t batch, dim, seqlen;
     int dstate;
     int softplus;
@@ -119,6 +123,8 @@ cudaError_t launch_conv1d_update(const Conv1dUpdateArgs &a, cudaStream_t stream)
 
 // Persistent, queue-balanced scan (dstate <= 16), one or two lanes per channel.
 bool persistent_supported(const ScanArgs &a);
+// Layout and alignment rules of the channel-last block-local kernel.
+bool channels_last_supported(const ScanArgs &a);
 // Test hook: the lane-split kernel's pieces of this channel group stop
 // publishing their carried state, so the next piece's bounded wait runs out
 // (-1 turns it off).  Returns the previous value.

@@ -57,6 +57,9 @@ struct Params {
     // ([batch * ckpt_gpb][ckpt_nsup][32 channels][16 states] fp32)
     float *ckpt;
     int ckpt_gpb, ckpt_nsup;
+    // lane-split block-local kernel: u / delta / z / out as (batch, L, dim)
+    // and B / C as (batch, L, N), all dense (else (batch, dim, L) / (batch, N, L))
+    int channels_last;
 };
 
 __device__ __forceinline__ void cp16(void *smem, const void *gmem, bool pred) {

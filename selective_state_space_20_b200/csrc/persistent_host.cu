@@ -92,6 +92,19 @@ int set_stall_group(int group) {
     return prev;
 }
 
+// The channel-last form of the block-local kernel: every 16-byte copy of a
+// timestep's channels or states must be whole (dim and N multiples of 16
+// bytes of the activation type) and start aligned.
+bool channels_last_supported(const ScanArgs &a) {
+    if (a.dstate > persist::kNS) return false;
+    const int es = a.act == kBF16 ? 2 : 4;
+    if ((a.dim * es) % 16 != 0 || (a.dstate * es) % 16 != 0) return false;
+    auto al = [](const void *q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+    if (!(al(a.u) && al(a.delta) && al(a.z) && al(a.B) && al(a.C) && al(a.out))) return false;
+    const int64_t units = n_groups(a.batch, a.dim, 4) * ((a.seqlen + 15) / 16);
+    return units < ((int64_t)1 << 30);
+}
+
 bool persistent_supported(const ScanArgs &a) {
     if (a.dstate > persist::kNS) return false;
     const int es = a.act == kBF16 ? 2 : 4;
@@ -158,6 +171,7 @@ persist::Params base_params(const ScanArgs &a, int lanes, int tc) {
     kp.ckpt = a.ckpt;
     kp.ckpt_gpb = (int)((a.dim + 31) / 32);
     kp.ckpt_nsup = (int)((a.seqlen + 31) / 32);
+    kp.channels_last = a.channels_last ? 1 : 0;
     return kp;
 }
 }  // namespace

@@ -219,10 +219,11 @@ __device__ __forceinline__ void local_publish(volatile unsigned *flag, int lane,
     }
 }
 
-template <typename T, int R, bool SP, bool GATE, bool CONV, bool LOCAL>
+template <typename T, int R, bool SP, bool GATE, bool CONV, bool LOCAL, bool CL>
 __global__ void __launch_bounds__(PairLaunch<R, LOCAL>::kWorkers * 32, PairLaunch<R, LOCAL>::kMinBlocks)
 scan_fwd_pairs_kernel(const Params p) {
     using W = PairSmem<T, R>;
+    static_assert(!(CL && CONV), "the fused convolution reads the dense layout");
     constexpr int kWorkers = PairLaunch<R, LOCAL>::kWorkers;
     constexpr bool ACC = sizeof(T) == 4;
     using Dk = Decay<ACC>;
@@ -239,6 +240,23 @@ scan_fwd_pairs_kernel(const Params p) {
     constexpr int S = kNS / R;   // states per lane
     constexpr int OWN = 8 / R;   // outputs per lane per block of 8 timesteps
     constexpr int PT = kTC / R;  // prologue timesteps per lane
+    // Channel-last staging (CL: (batch, L, dim) activations, (batch, L, N) B
+    // and C).  A stage then holds, per activation tensor, kTC rows of one
+    // timestep's CW channels (CH 16-byte chunks; chunk c of row t sits at
+    // slot c ^ swz(t), so the 8 lanes of a quarter-warp that read one chunk
+    // each from consecutive rows hit distinct banks), then B and C as kTC
+    // rows of kNS states.  The prologue lane takes one timestep's channels
+    // (LPT lanes per timestep) instead of one channel's timesteps; the scan
+    // is unchanged, so results are bit-equal to the dense layout's.
+    constexpr int CH = CW * (int)sizeof(T) / 16;   // 16-byte chunks per activation row
+    constexpr int CROW = CH * 16;
+    constexpr int BCH = kNS * (int)sizeof(T) / 16;  // chunks per B / C row
+    constexpr int BROW = BCH * 16;
+    constexpr int LPT = 32 / kTC;                   // prologue lanes per timestep
+    constexpr int CL_ACT = 3 * kTC * CROW;          // B / C rows start here
+    constexpr int CL_BIAS = W::STAGE - CW * 4;      // stage 0's tail: the group's biases (fp32)
+    static_assert(!CL || (CL_ACT + 2 * kTC * BROW <= CL_BIAS && kTC * CROW <= W::OUTB), "channel-last stage");
+    auto swz = [](int t) { return (t / (8 / CH)) & (CH - 1); };
     extern __shared__ __align__(16) unsigned char smem[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -325,6 +343,10 @@ scan_fwd_pairs_kernel(const Params p) {
                 A2[k] = make_float2(a0 * Dk::kScale, a1 * Dk::kScale);
             }
             bias_p = (dp < Dm && p.delta_bias) ? __ldg(p.delta_bias + dp) : 0.f;
+            if (CL && lane < CW) {  // the prologue lane of a timestep needs every channel's bias
+                float *sbias = reinterpret_cast<float *>(base + CL_BIAS);
+                sbias[lane] = (d0 + lane < Dm && p.delta_bias) ? __ldg(p.delta_bias + d0 + lane) : 0.f;
+            }
             D_s = (ds < Dm && p.D) ? __ldg(p.D + ds) : 0.f;
             if (CONV) {  // taps right-aligned to 4: a shorter kernel sees zeros before it
                 const int K = p.conv_k;
@@ -392,8 +414,52 @@ scan_fwd_pairs_kernel(const Params p) {
             bok[i] = n < N;
             boff[i] = bc0 + (int64_t)n * L + cx * V;
         }
+        // channel-last copies: chunk q = lane + 32 i of the activation tile is
+        // (row t = q / CH, chunk c = q % CH); of the B / C tile (which, t, c)
+        constexpr int NXC = kTC * CH / 32 > 0 ? kTC * CH / 32 : 1, NBC = 2 * kTC * BCH / 32;
+        static_assert(!CL || (NXC * 32 == kTC * CH && NBC * 32 == 2 * kTC * BCH), "channel-last copy split");
+        int64_t cxoff[NXC], cboff[NBC];
+        bool cxok[NXC], cbok[NBC];
+        if (CL) {
+#pragma unroll
+            for (int i = 0; i < NXC; ++i) {
+                const int q = lane + 32 * i, t = q / CH, c = q % CH;
+                cxok[i] = d0 + c * V < Dm;
+                cxoff[i] = (b * L + t) * Dm + d0 + c * V;
+            }
+#pragma unroll
+            for (int i = 0; i < NBC; ++i) {
+                const int q = lane + 32 * i, t = (q / BCH) % kTC, c = q % BCH;
+                cbok[i] = c * V < N;
+                cboff[i] = (b * L + t) * (int64_t)N + c * V;
+            }
+        }
         bool so_stage = false;  // state-only run: no z or C rows to stage
         auto issue = [&](int sub, int st) {
+            if (CL) {
+                unsigned char *sb0 = base + st * W::STAGE;
+                const int64_t t0 = tb0 + (int64_t)sub * kTC;
+#pragma unroll
+                for (int i = 0; i < NXC; ++i) {
+                    const int q = lane + 32 * i, t = q / CH, c = q % CH;
+                    const bool ok = cxok[i] && t0 + t < L;
+                    const int64_t off = ok ? cxoff[i] + t0 * Dm : 0;
+                    unsigned char *dst = sb0 + t * CROW + ((c ^ swz(t)) * 16);
+                    cp16(dst, gu + off, ok);
+                    cp16(dst + kTC * CROW, gd + off, ok);
+                    if (GATE && !so_stage) cp16(dst + 2 * kTC * CROW, gz + off, ok);
+                }
+#pragma unroll
+                for (int i = 0; i < NBC; ++i) {
+                    const int q = lane + 32 * i, which = q / (kTC * BCH), t = (q / BCH) % kTC, c = q % BCH;
+                    const bool ok = cbok[i] && t0 + t < L;
+                    const int64_t off = ok ? cboff[i] + t0 * N : 0;
+                    if (!(so_stage && which))
+                        cp16(sb0 + CL_ACT + which * kTC * BROW + t * BROW + c * 16, (which ? gC : gB) + off, ok);
+                }
+                cp_commit();
+                return;
+            }
             unsigned char *sbuf = base + st * W::STAGE + cx * 16;
             const int64_t t0 = tb0 + (int64_t)sub * kTC;
             const bool tok = t0 + cx * V < L;
@@ -497,7 +563,19 @@ scan_fwd_pairs_kernel(const Params p) {
             // reads states 4q .. 4q+3 of B (which 0) or C (which 1) in chunk c
             // and writes them back as one 16-byte [t][4q .. 4q+3] piece per
             // timestep
-            if (!SO || lane < 16) {  // C rows only feed the readout
+            if (CL) {  // B and C rows are [t][n] already: widen to fp32
+#pragma unroll
+                for (int i = 0; i < NBC; ++i) {
+                    const int q = lane + 32 * i, which = q / (kTC * BCH), t = (q / BCH) % kTC, c = q % BCH;
+                    if (SO && which) continue;
+                    float f[V];
+                    Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sbuf + CL_ACT + which * kTC * BROW + t * BROW + c * 16), f);
+                    float *dst = bc32 + which * (W::BARR / 4) + (t / V) * (W::BLKB / 4) + (t % V) * kNS + c * V;
+#pragma unroll
+                    for (int k = 0; k < V; k += 4)
+                        *reinterpret_cast<float4 *>(dst + k) = make_float4(f[k], f[k + 1], f[k + 2], f[k + 3]);
+                }
+            } else if (!SO || lane < 16) {  // C rows only feed the readout
                 static_assert(CPR == 4, "four chunks of timesteps per sub-chunk");
                 const int which = lane >> 4, q = (lane >> 2) & 3, c = lane & 3;
                 float f[4][V];
@@ -513,8 +591,36 @@ scan_fwd_pairs_kernel(const Params p) {
             // ---- prologue (b): per element, once: delta and delta*u, stored
             // duplicated as (delta, delta, delta*u, delta*u) so the scan reads
             // both packed operand pairs with one 16-byte load
+            if (CL) {  // lane: timestep t, channel chunks h * CH / LPT ..
+                const int t = lane / LPT, h = lane % LPT;
+                const float *sbias = reinterpret_cast<const float *>(base + CL_BIAS);
 #pragma unroll
-            for (int v = 0; v < PT; v += V) {
+                for (int j = 0; j < CH / LPT; ++j) {
+                    const int c = h * (CH / LPT) + j;
+                    const unsigned char *src = sbuf + t * CROW + ((c ^ swz(t)) * 16);
+                    float fu[V], fd[V], fb[V];
+                    Elem<T>::unpack(*reinterpret_cast<const uint4 *>(src), fu);
+                    Elem<T>::unpack(*reinterpret_cast<const uint4 *>(src + kTC * CROW), fd);
+#pragma unroll
+                    for (int e = 0; e < V; e += 4) {
+                        const float4 b4 = *reinterpret_cast<const float4 *>(sbias + c * V + e);
+                        fb[e] = b4.x; fb[e + 1] = b4.y; fb[e + 2] = b4.z; fb[e + 3] = b4.w;
+                    }
+#pragma unroll
+                    for (int e = 0; e < V; e += 2) {  // channel pairs on the packed x2 instructions
+                        const int ch = c * V + e;
+                        float2 x = __fadd2_rn(f2(fd[e], fd[e + 1]), f2(fb[e], fb[e + 1]));
+                        if (SP) x = Dk::softplus2(x);
+                        if (t >= tvalid) x = f2(0.f, 0.f);  // past the end: Abar = 1, no input
+                        const float2 xu = __fmul2_rn(x, f2(fu[e], fu[e + 1]));
+                        *reinterpret_cast<float4 *>(ddu + ch * W::QUADB + t * 16) = make_float4(x.x, x.x, xu.x, xu.x);
+                        *reinterpret_cast<float4 *>(ddu + (ch + 1) * W::QUADB + t * 16) =
+                            make_float4(x.y, x.y, xu.y, xu.y);
+                    }
+                }
+            }
+#pragma unroll
+            for (int v = 0; v < (CL ? 0 : PT); v += V) {
                 const int tt = ph * PT + v;
                 float fu[V], fd[V];
                 Elem<T>::unpack(*reinterpret_cast<const uint4 *>(sbuf + (0 * CW + pc) * W::ROWB + tt * sizeof(T)), fu);
@@ -629,8 +735,22 @@ scan_fwd_pairs_kernel(const Params p) {
                     // u and z read from the staged raw rows
                     const int te = tb + OWN * sr;
                     float fu[OWN], fz[OWN], o[OWN];
-                    load_small<T, OWN>(urow + te * sizeof(T), fu);
-                    if (GATE) load_small<T, OWN>(zrow + te * sizeof(T), fz);
+                    // channel-last: rows te .. share one swizzle when its period
+                    // is a multiple of OWN rows (te is a multiple of OWN)
+                    constexpr bool kOneSlot = (8 / CH) % OWN == 0;
+                    const int slot0 = (sc / V) ^ swz(te);
+                    if (CL) {  // channel sc of rows te ..
+#pragma unroll
+                        for (int i = 0; i < OWN; ++i) {
+                            const int slot = kOneSlot ? slot0 : (sc / V) ^ swz(te + i);
+                            const unsigned char *src = sbuf + (te + i) * CROW + slot * 16 + (sc % V) * (int)sizeof(T);
+                            fu[i] = Elem<T>::to_f(*reinterpret_cast<const T *>(src));
+                            if (GATE) fz[i] = Elem<T>::to_f(*reinterpret_cast<const T *>(src + 2 * kTC * CROW));
+                        }
+                    } else {
+                        load_small<T, OWN>(urow + te * sizeof(T), fu);
+                        if (GATE) load_small<T, OWN>(zrow + te * sizeof(T), fz);
+                    }
 #pragma unroll
                     for (int i = 0; i < OWN; i += 2) {
                         const float2 uu = f2(fu[i], fu[i + 1]);
@@ -639,8 +759,18 @@ scan_fwd_pairs_kernel(const Params p) {
                         o[i] = oo.x;
                         o[i + 1] = oo.y;
                     }
-                    if (OWN == 4) store4<T>(orow + te * sizeof(T), o);
-                    else store2<T>(orow + te * sizeof(T), o);
+                    if (CL) {
+#pragma unroll
+                        for (int i = 0; i < OWN; ++i) {
+                            const int slot = kOneSlot ? slot0 : (sc / V) ^ swz(te + i);
+                            Elem<T>::store(reinterpret_cast<T *>(outt + (te + i) * CROW + slot * 16 + (sc % V) * (int)sizeof(T)),
+                                           o[i]);
+                        }
+                    } else if (OWN == 4) {
+                        store4<T>(orow + te * sizeof(T), o);
+                    } else {
+                        store2<T>(orow + te * sizeof(T), o);
+                    }
                 }
             }
             __syncwarp();
@@ -652,8 +782,17 @@ scan_fwd_pairs_kernel(const Params p) {
                 publish_carry(se);
             }
             // ---- coalesced store of the output tile
+            if (CL) {
 #pragma unroll
-            for (int i = lane; i < CW * CPR; i += 32) {
+                for (int i = 0; i < NXC; ++i) {
+                    const int q = lane + 32 * i, t = q / CH, c = q % CH;
+                    if (cxok[i] && t0 + t < L)
+                        stg16_stream(gout + cxoff[i] + t0 * Dm,
+                                     *reinterpret_cast<const uint4 *>(outt + t * CROW + ((c ^ swz(t)) * 16)));
+                }
+            }
+#pragma unroll
+            for (int i = lane; i < (CL ? 0 : CW * CPR); i += 32) {
                 const int r = i / CPR, c = i % CPR;
                 const int64_t t = t0 + c * V;
                 if (r < nrows && t < L)
@@ -734,11 +873,11 @@ scan_fwd_pairs_kernel(const Params p) {
     }
 }
 
-template <typename T, int R, bool SP, bool GATE, bool CONV, bool LOCAL>
+template <typename T, int R, bool SP, bool GATE, bool CONV, bool LOCAL, bool CL = false>
 cudaError_t launch_t(const Params &kp, int sm_count, cudaStream_t st) {
     using PL = PairLaunch<R, LOCAL>;
     const int smem = PL::kWorkers * PairSmem<T, R>::BYTES + (LOCAL ? LocalSmem<R>::BYTES : 0);
-    auto kern = scan_fwd_pairs_kernel<T, R, SP, GATE, CONV, LOCAL>;
+    auto kern = scan_fwd_pairs_kernel<T, R, SP, GATE, CONV, LOCAL, CL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     static const int per_sm = [&] {
@@ -772,6 +911,19 @@ template <int R, bool LOCAL>
 cudaError_t launch_r(const Params &kp, int act, int sm_count, cudaStream_t st) {
     const bool gate = kp.z != nullptr;
     using BF = __nv_bfloat16;
+    if (kp.channels_last) {  // block-local form only, no fused convolution
+        if (!LOCAL || kp.conv_w) return cudaErrorInvalidValue;
+        if (act == kBF16) {
+            if (kp.softplus) return gate ? launch_t<BF, R, true, true, false, true, true>(kp, sm_count, st)
+                                         : launch_t<BF, R, true, false, false, true, true>(kp, sm_count, st);
+            return gate ? launch_t<BF, R, false, true, false, true, true>(kp, sm_count, st)
+                        : launch_t<BF, R, false, false, false, true, true>(kp, sm_count, st);
+        }
+        if (kp.softplus) return gate ? launch_t<float, R, true, true, false, true, true>(kp, sm_count, st)
+                                     : launch_t<float, R, true, false, false, true, true>(kp, sm_count, st);
+        return gate ? launch_t<float, R, false, true, false, true, true>(kp, sm_count, st)
+                    : launch_t<float, R, false, false, false, true, true>(kp, sm_count, st);
+    }
     if (kp.conv_w) {  // fused conv1d prologue: softplus on (checked by the caller)
         if (act == kBF16) return gate ? launch_t<BF, R, true, true, true, LOCAL>(kp, sm_count, st)
                                       : launch_t<BF, R, true, false, true, LOCAL>(kp, sm_count, st);

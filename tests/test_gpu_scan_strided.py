@@ -113,6 +113,62 @@ def test_channels_last_matches_dense_bitwise(dtype):
     assert torch.equal(o1, o2.contiguous()) and torch.equal(s1, s2)
 
 
+def _page_layout(cpu, keep=()):
+    """The pages' layout: (batch, L, dim) activations and (batch, L, N) B / C,
+    dense, seen as (batch, dim, L) / (batch, N, L) views."""
+    return {k: (None if v is None else (_channels_last(v) if k in ("u", "delta", "z", "B", "C") else v).cuda())
+            for k, v in cpu.items()}
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("shape,dstate", [((2, 96, 336), 16), ((3, 40, 128), 8), ((1, 16, 64), 16),
+                                          ((2, 1280, 512), 16), ((1, 64, 8192), 16)],
+                         ids=["2x96x336", "3x40x128-N8", "1x16x64", "2x1280x512", "1x64x8192-two-phase"])
+@pytest.mark.parametrize("lanes", [0, 2, 4])
+def test_page_layout_on_the_local_kernel(dtype, shape, dstate, lanes):
+    """The pages' (b, l, d) layout runs the block-local lane-split kernel:
+    bit-equal to mamba_scan_fwd on the same values laid out densely with the
+    same lanes (the same scan, other staging), and within the tolerance of
+    the oracle.  The long row with few channels splits each group's sequence
+    among a block's warps (two-phase pieces)."""
+    b, d, L = shape
+    w = inputs.custom(b, d, L, dstate, dtype, seed=b + d + L + lanes)
+    cpu = inputs.scan_inputs(w)
+    dense = {k: (None if v is None else v.cuda()) for k, v in cpu.items()}
+    kw = dict(schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=lanes)
+    o1, s1 = binding.mamba_scan_fwd(dense["u"], dense["delta"], dense["A"], dense["B"], dense["C"], D=dense["D"],
+                                    z=dense["z"], delta_bias=dense["delta_bias"], return_last_state=True, **kw)
+    o2, s2 = _check(f"page layout {w.name} lanes={lanes}", cpu, _page_layout(cpu), dtype, **kw)
+    assert o2.stride(1) == 1
+    assert torch.equal(o1, o2.contiguous()) and torch.equal(s1, s2)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("lanes", [2, 4])
+def test_page_layout_ragged_length_and_optional_inputs(dtype, lanes):
+    """Lengths that are no whole number of sub-chunks or of 16-byte chunks,
+    no gate, no bias, no D (the local kernel takes any length in this
+    layout)."""
+    for L, drop in ((333, ()), (97, ("z", "delta_bias", "D")), (1000, ("z",))):
+        w = inputs.custom(2, 48, L, 16, dtype, seed=L + lanes)
+        cpu = inputs.scan_inputs(w)
+        for k in drop:
+            cpu[k] = None
+        _check(f"page layout {w.name} lanes={lanes} drop={drop}", cpu, _page_layout(cpu), dtype,
+               schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=lanes)
+
+
+def test_page_layout_local_schedule_needs_the_layout():
+    """SCHEDULE_LOCAL on a layout the local kernel cannot stage (dim not a
+    multiple of 8 bf16 values) is refused; AUTO runs the static kernel."""
+    w = inputs.custom(1, 36, 64, 16, "bf16", seed=6)
+    cpu = inputs.scan_inputs(w)
+    dev = _page_layout(cpu)
+    with pytest.raises(binding.MambaError):
+        _run(dev, schedule=binding.SCHEDULE_LOCAL)
+    _check("page layout dim 36 (static)", cpu, dev, "bf16")
+
+
 def test_in_place_and_initial_state():
     w = inputs.custom(2, 32, 256, 16, "bf16", seed=12)
     cpu = inputs.scan_inputs(w)
