@@ -83,6 +83,8 @@ KERNEL_SOURCES = {
     "scan_fwd_kernel": ("scan_fwd.cu", "device_math.cuh", "internal.h"),
     "scan_fwd_complex_kernel": ("scan_fwd_complex.cu", "device_math.cuh", "internal.h"),
     "scan_bwd_kernel": ("scan_bwd.cu", "device_math.cuh", "internal.h"),
+    "state_update_lanes_kernel": ("state_update.cu", "device_math.cuh", "internal.h"),
+    "conv1d_tiles_kernel": ("conv1d.cu", "device_math.cuh", "internal.h"),
 }
 
 
@@ -618,6 +620,7 @@ def decode_measure(steps=256):
             "hbm_frac": bytes_step / us / 1e3 / hbm, "graph_of_steps": steps,
             "note": "back-to-back steps in a CUDA graph: each step also pays for the write-back of the previous "
                     "one's state; the state (84 MB) can stay partly L2-resident",
+            "traffic": measured_traffic(f"state_update_lanes_kernel {w.name}"),
             "l2_flushed": {"us_per_step": us_cold, "GB_per_s": bytes_step / us_cold / 1e3,
                            "hbm_frac": bytes_step / us_cold / 1e3 / hbm,
                            "note": f"median of 32 steps, each after a {2 * l2 >> 20} MB read, the kernel timed "
@@ -684,7 +687,9 @@ def conv1d_measure(reps=20):
     return {"workload": f"conv1d K={K} {w.batch}x{w.dim}x{w.seqlen} {w.dtype} (x half of a 2x-wide input)",
             "us_per_call": us, "Gelem_per_s": w.elements / us / 1e3,
             "roofline": {"bound": "hbm", "achieved": nbytes / us / 1e3, "peak": hbm, "unit": "GB/s",
-                         "frac": nbytes / us / 1e3 / hbm, "algorithmic_bytes": nbytes},
+                         "frac": nbytes / us / 1e3 / hbm, "algorithmic_bytes": nbytes,
+                         "traffic": measured_traffic(f"conv1d_tiles_kernel conv1d K={K} {w.batch}x{w.dim}x{w.seqlen} "
+                                                     f"{w.dtype}")},
             "fused_with_scan": {"us_per_call": us_fused, "Gelem_per_s": w.elements / us_fused / 1e3,
                                 "separate_conv_then_scan_us": us_sep,
                                 "note": "mamba_scan_fwd_conv: u formed in the scan's prologue, never stored"},
