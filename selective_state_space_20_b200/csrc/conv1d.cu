@@ -44,7 +44,7 @@ __device__ __forceinline__ float load_elem(const T *p) { return Elem<T>::load(p)
 // from the lane before it, and lane 0 from lane 31 of the previous tile.
 // W64: 64-bit index arithmetic (more than 2^31 threads); otherwise 32-bit,
 // whose divisions cost a fraction of the 64-bit ones.
-template <typename T, int K, int NT, bool W64>
+template <typename T, int K, int NT, bool W64, bool SILU>
 __global__ void __launch_bounds__(256) conv1d_tiles_kernel(const ConvParams p) {
     using Idx = typename std::conditional<W64, int64_t, unsigned>::type;
     constexpr int V = 16 / (int)sizeof(T);  // elements per 16-byte chunk
@@ -91,11 +91,13 @@ __global__ void __launch_bounds__(256) conv1d_tiles_kernel(const ConvParams p) {
         if (t0 < p.seqlen) {  // seqlen is a whole number of chunks
             float o[V];
 #pragma unroll
-            for (int i = 0; i < V; ++i) {
-                float v = bias;
+            for (int i = 0; i < V; i += 2) {  // output pairs on the packed x2 instructions
+                float2 v = f2(bias, bias);
 #pragma unroll
-                for (int k = 0; k < K; ++k) v = fmaf(wk[k], f[i + k], v);
-                o[i] = p.silu ? silu_f(v) : v;
+                for (int k = 0; k < K; ++k) v = __ffma2_rn(f2(wk[k], wk[k]), f2(f[i + k], f[i + 1 + k]), v);
+                if (SILU) v = silu2_f(v);
+                o[i] = v.x;
+                o[i + 1] = v.y;
             }
             stg16_stream(orow + t0, Elem<T>::pack(o));
         }
@@ -148,6 +150,21 @@ __global__ void __launch_bounds__(256) conv1d_update_kernel(const ConvUpdatePara
     for (int k = 0; k < S; ++k) st[k] = in[k + 1];
 }
 
+template <typename T, int NT, bool SILU>
+cudaError_t launch_tiles(const ConvParams &p, bool w64, unsigned g, int threads, cudaStream_t st) {
+    switch (p.width * 2 + (w64 ? 1 : 0)) {
+        case 2: conv1d_tiles_kernel<T, 1, NT, false, SILU><<<g, threads, 0, st>>>(p); break;
+        case 3: conv1d_tiles_kernel<T, 1, NT, true, SILU><<<g, threads, 0, st>>>(p); break;
+        case 4: conv1d_tiles_kernel<T, 2, NT, false, SILU><<<g, threads, 0, st>>>(p); break;
+        case 5: conv1d_tiles_kernel<T, 2, NT, true, SILU><<<g, threads, 0, st>>>(p); break;
+        case 6: conv1d_tiles_kernel<T, 3, NT, false, SILU><<<g, threads, 0, st>>>(p); break;
+        case 7: conv1d_tiles_kernel<T, 3, NT, true, SILU><<<g, threads, 0, st>>>(p); break;
+        case 9: conv1d_tiles_kernel<T, 4, NT, true, SILU><<<g, threads, 0, st>>>(p); break;
+        default: conv1d_tiles_kernel<T, 4, NT, false, SILU><<<g, threads, 0, st>>>(p); break;
+    }
+    return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t launch_fwd_typed(const ConvParams &p, cudaStream_t st) {
     constexpr int V = 16 / (int)sizeof(T);
@@ -160,18 +177,8 @@ cudaError_t launch_fwd_typed(const ConvParams &p, cudaStream_t st) {
         const int64_t blocks = (warps * 32 + threads - 1) / threads;
         if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
         const bool w64 = blocks * threads >= 0x7fffffffLL || p.seqlen >= 0x7fffffffLL;
-        const unsigned g = (unsigned)blocks;
-        switch (p.width * 2 + (w64 ? 1 : 0)) {
-            case 2: conv1d_tiles_kernel<T, 1, NT, false><<<g, threads, 0, st>>>(p); break;
-            case 3: conv1d_tiles_kernel<T, 1, NT, true><<<g, threads, 0, st>>>(p); break;
-            case 4: conv1d_tiles_kernel<T, 2, NT, false><<<g, threads, 0, st>>>(p); break;
-            case 5: conv1d_tiles_kernel<T, 2, NT, true><<<g, threads, 0, st>>>(p); break;
-            case 6: conv1d_tiles_kernel<T, 3, NT, false><<<g, threads, 0, st>>>(p); break;
-            case 7: conv1d_tiles_kernel<T, 3, NT, true><<<g, threads, 0, st>>>(p); break;
-            case 9: conv1d_tiles_kernel<T, 4, NT, true><<<g, threads, 0, st>>>(p); break;
-            default: conv1d_tiles_kernel<T, 4, NT, false><<<g, threads, 0, st>>>(p); break;
-        }
-        return cudaGetLastError();
+        return p.silu ? launch_tiles<T, NT, true>(p, w64, (unsigned)blocks, threads, st)
+                      : launch_tiles<T, NT, false>(p, w64, (unsigned)blocks, threads, st);
     }
     const int64_t blocks = (p.batch * p.dim * p.seqlen + threads - 1) / threads;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;

@@ -37,10 +37,12 @@ __device__ __forceinline__ float softplus_f(float x) {
     return fmaf(w, p, fmaxf(x, 0.f));
 }
 
-// silu(z) = z / (1 + e^-z); for z < -88 the denominator overflows and the
-// quotient is 0, which is the correctly rounded fp32 limit.
+// silu(z) = z (1 / (1 + e^-z)); for z < -88 the denominator overflows and
+// the product is 0, which is the correctly rounded fp32 limit.  The same
+// operations as silu2_f below, value for value, so the scalar and the packed
+// forms give identical bits.
 __device__ __forceinline__ float silu_f(float z) {
-    return __fdividef(z, 1.f + __expf(-z));
+    return z * __fdividef(1.f, ex2_mufu(z * -kLog2e) + 1.f);
 }
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }

@@ -267,6 +267,7 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
                     const float4 *Bt = reinterpret_cast<const float4 *>(sB + (tb + q) * kCNP + r * S);
                     const float4 *Ct = reinterpret_cast<const float4 *>(sC + (tb + q) * kCNP + r * S);
                     H y = 0.f;
+                    float2 yacc = f2(0.f, 0.f);  // bf16: (sum cr nr, sum ci ni), y = .x - .y
 #pragma unroll
                     for (int s2 = 0; s2 < S / 2; ++s2) {  // two complex states per 16-byte read
                         const float4 bb = Bt[s2], cc = Ct[s2];
@@ -284,19 +285,25 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
                                 nr = fma(ar, hr[s], fma(-ai, hi[s], du * (double)br[k]));
                                 ni = fma(ar, hi[s], fma(ai, hr[s], du * (double)bi[k]));
                                 y = fma((double)cr[k], nr, fma(-(double)ci[k], ni, y));
-                            } else {
-                                const float mag = ex2_mufu(dl * Are[s]);
+                            } else {  // (re, im) pairs on the packed x2 instructions
+                                const float2 x = __fmul2_rn(f2(dl, dl), f2(Are[s], Aim[s]));
+                                const float mag = ex2_mufu(x.x);
                                 float sn, cs;
-                                sincos_mufu(reduce_angle(dl * Aim[s]), sn, cs);
-                                const float ar = mag * cs, ai = mag * sn;
-                                nr = fmaf(ar, hr[s], fmaf(-ai, hi[s], du * br[k]));
-                                ni = fmaf(ar, hi[s], fmaf(ai, hr[s], du * bi[k]));
-                                y = fmaf(cr[k], nr, fmaf(-ci[k], ni, y));
+                                sincos_mufu(reduce_angle(x.y), sn, cs);
+                                const float2 a = __fmul2_rn(f2(mag, mag), f2(cs, sn));  // (ar, ai)
+                                // (nr, ni) = (ar hr - ai hi, ar hi + ai hr) + du (br, bi)
+                                float2 nn = __ffma2_rn(f2(-a.y, a.y), f2(hi[s], hr[s]),
+                                                       __fmul2_rn(f2(du, du), f2(br[k], bi[k])));
+                                nn = __ffma2_rn(f2(a.x, a.x), f2(hr[s], hi[s]), nn);
+                                yacc = __ffma2_rn(f2(cr[k], ci[k]), nn, yacc);
+                                nr = nn.x;
+                                ni = nn.y;
                             }
                             hr[s] = nr;
                             hi[s] = ni;
                         }
                     }
+                    if constexpr (!kF64) y = yacc.x - yacc.y;
                     yp[q] = y;
                 }
                 // sum over the R lanes of the channel; lane r keeps outputs

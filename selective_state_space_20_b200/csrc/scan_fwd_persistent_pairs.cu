@@ -550,11 +550,14 @@ scan_fwd_pairs_kernel(const Params p) {
                 for (int v = 0; v < PT; v += V) {
                     float uo[V];
 #pragma unroll
-                    for (int e = 0; e < V; ++e) {
-                        float acc = cb_p;
+                    for (int e = 0; e < V; e += 2) {  // the conv1d kernel's arithmetic, pair for pair
+                        float2 acc = f2(cb_p, cb_p);
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) acc = fmaf(cw[k], xs[v + e + k], acc);
-                        uo[e] = silu_f(acc);
+                        for (int k = 0; k < 4; ++k)
+                            acc = __ffma2_rn(f2(cw[k], cw[k]), f2(xs[v + e + k], xs[v + e + 1 + k]), acc);
+                        acc = silu2_f(acc);
+                        uo[e] = acc.x;
+                        uo[e + 1] = acc.y;
                     }
                     *reinterpret_cast<uint4 *>(urw + (ph * PT + v) * sizeof(T)) = Elem<T>::pack(uo);
                 }
