@@ -238,6 +238,9 @@ class NvmlSampler:
 
 # ------------------------------------------------------------ distributed
 def dist_setup():
+    # NCCL's own log lines (its version at communicator set-up) go to stderr:
+    # stdout carries the one JSON line
+    os.environ.setdefault("NCCL_DEBUG_FILE", "/dev/stderr")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
