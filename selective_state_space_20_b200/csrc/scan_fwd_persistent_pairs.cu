@@ -38,6 +38,12 @@
 // Shared arrays are padded so that every quarter-warp access is free of bank
 // conflicts.  fp32 activations take the accurate decay and softplus of
 // device_math.cuh (Decay<true>) in place of the MUFU ones.
+// Channel-last form (CL, block-local only): the activations of the Keras
+// page's layout -- (batch, L, dim), B and C (batch, L, N) -- are staged a
+// timestep row at a time (16-byte copies of a row's channels or states), the
+// prologue lane takes one timestep's channels, and the epilogue reads and
+// writes the transposed rows; steps 2 (the quads and fp32 B / C rows) and 3
+// are unchanged, so the results equal the dense layout's bit for bit.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
