@@ -37,7 +37,9 @@
  *   sequence split    mamba_delta_sum, mamba_state_fold
  *   status            mamba_scan_workspace_status, mamba_get_device_status,
  *                     mamba_status_string, mamba_abi_version;
- *                     mamba_debug_stall_group (test hook)
+ *                     mamba_debug_stall_group (test hook); the bounds-checked
+ *                     build: mamba_bounds_checked, mamba_debug_bounds_status,
+ *                     mamba_debug_shrink_output_extent (test hook)
  *
  * Conventions for every entry point
  * ---------------------------------
@@ -65,8 +67,8 @@
  *   caller must serialise them (see there).  Library state: per device, the
  *   workspace pointer of the last persistent launch and the local schedule's
  *   timeout word (both for mamba_get_device_status), and the scratch area of
- *   mamba_scan_fwd_noalloc; process-wide, the mamba_debug_stall_group test
- *   hook (off by default).
+ *   mamba_scan_fwd_noalloc; process-wide, the mamba_debug_stall_group and
+ *   mamba_debug_shrink_output_extent test hooks (off by default).
  */
 #ifndef MAMBA_SCAN_H
 #define MAMBA_SCAN_H
@@ -97,8 +99,10 @@ typedef enum {
     MAMBA_ERR_DEVICE = -6,      /* no usable CUDA device */
     MAMBA_ERR_OVERLAP = -7,     /* an output partially overlaps an input */
     MAMBA_ERR_WORKSPACE = -8,   /* workspace too small or misaligned */
-    MAMBA_ERR_TIMEOUT = -9      /* a persistent launch gave up waiting (see
+    MAMBA_ERR_TIMEOUT = -9,     /* a persistent launch gave up waiting (see
                                    mamba_scan_workspace_status) */
+    MAMBA_ERR_BOUNDS = -10      /* bounds-checked build only: a kernel access
+                                   fell outside its tensor and was skipped */
 } mamba_status_t;
 
 /* Launch schedules of the scan. */
@@ -467,8 +471,11 @@ int mamba_state_fold(const float *h_init, const double *delta_sums, const float 
  * call (a device word the library keeps; reading it clears it), or if the
  * last persistent launch on this device (any entry point that was given a
  * workspace) gave up one -- the error word in its workspace, which must
- * still be allocated; else MAMBA_OK.  No device code traps; this and
- * mamba_scan_workspace_status are how failures surface. */
+ * still be allocated; in the bounds-checked build, MAMBA_ERR_BOUNDS (checked
+ * first) if an instrumented kernel skipped an access outside its tensor
+ * since the previous call (reading clears the record); else MAMBA_OK.  No
+ * device code traps; this and mamba_scan_workspace_status are how failures
+ * surface. */
 int mamba_get_device_status(cudaStream_t stream);
 
 /* Test hook for the failure-detection path: from the next launch on, the
@@ -480,6 +487,38 @@ int mamba_get_device_status(cudaStream_t stream);
  * No wait is unbounded and nothing faults.  group < 0 turns the hook off
  * (the default).  Process-wide; returns the previous setting. */
 int mamba_debug_stall_group(int group);
+
+/*
+ * The bounds-checked build (libmamba_scan_checked.so, compiled with
+ * MSCAN_BOUNDS_CHECK; same entry points and results).  Every launch of the
+ * lane-split scan kernel (mamba_scan_fwd, _ws, _noalloc, _init, _conv,
+ * _ckpt, the (batch, L, dim) layout of mamba_scan_fwd_strided), of the decode
+ * step (mamba_state_update) and of the conv1d kernels (mamba_conv1d_fwd,
+ * mamba_conv1d_update) carries the byte range of every pointer argument,
+ * computed from the sizes given; each global access first checks that it
+ * stays inside its range.  One that would not is skipped (a load reads
+ * zeros, a store is dropped) and the first such access is recorded: its site
+ * (the tensor: 1 A, 2 delta_bias, 3 D, 4 conv weight, 5 conv bias, 6 u / x,
+ * 7 delta, 8 z, 9 B, 10 C, 11 conv input before a piece, 12 u written by the
+ * fused conv, 13 out, 14 last_state, 15 h0, 16 checkpoints, 17 workspace
+ * carries, 18 decode state, 19 conv1d input, 20 conv1d state) and its byte
+ * offset from the tensor's start.  Nothing traps.  The static, one-lane,
+ * complex and backward kernels are not instrumented.  In the normal build the
+ * checks compile away.
+ *
+ * mamba_bounds_checked: 1 in the bounds-checked build, 0 otherwise.
+ * mamba_debug_bounds_status: 1 with the first recorded violation (site and
+ *   offset written when the pointers are not NULL), 0 without; clears the
+ *   record.  Does not synchronise: call after the work has completed.
+ *   MAMBA_ERR_CUDA if the record cannot be read.
+ * mamba_debug_shrink_output_extent: test hook -- every later launch records
+ *   its output range `bytes` short of the real one, so that the checks have a
+ *   violation to find while every access still lands in allocated memory.
+ *   Process-wide; 0 (the default) turns it off; returns the previous value.
+ */
+int mamba_bounds_checked(void);
+int mamba_debug_bounds_status(int *site, long long *offset);
+int mamba_debug_shrink_output_extent(int bytes);
 
 /* Synchronises `stream`, then reads the status a persistent launch left in
  * `workspace`: MAMBA_OK, or MAMBA_ERR_TIMEOUT if a worker stopped waiting for

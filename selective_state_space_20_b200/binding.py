@@ -24,8 +24,9 @@ MAMBA_OK = 0
 STATUS_NAMES = {0: "MAMBA_OK", -1: "MAMBA_ERR_NULL", -2: "MAMBA_ERR_SHAPE",
                 -3: "MAMBA_ERR_UNSUPPORTED", -4: "MAMBA_ERR_ALIGN",
                 -5: "MAMBA_ERR_CUDA", -6: "MAMBA_ERR_DEVICE", -7: "MAMBA_ERR_OVERLAP",
-                -8: "MAMBA_ERR_WORKSPACE", -9: "MAMBA_ERR_TIMEOUT"}
+                -8: "MAMBA_ERR_WORKSPACE", -9: "MAMBA_ERR_TIMEOUT", -10: "MAMBA_ERR_BOUNDS"}
 MAMBA_ERR_TIMEOUT = -9
+MAMBA_ERR_BOUNDS = -10
 SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT, SCHEDULE_LOCAL = 0, 1, 2, 3
 
 # Every function include/mamba_scan.h declares.
@@ -39,7 +40,8 @@ EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_bwd_workspace_size", "mamba_scan_ckpt_size", "mamba_scan_fwd_ckpt",
             "mamba_scan_bwd_ckpt",
             "mamba_state_update", "mamba_conv1d_fwd",
-            "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version")
+            "mamba_conv1d_update", "mamba_status_string", "mamba_abi_version",
+            "mamba_bounds_checked", "mamba_debug_bounds_status", "mamba_debug_shrink_output_extent")
 
 
 class MambaError(RuntimeError):
@@ -92,6 +94,12 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_get_device_status.restype = ci
     lib.mamba_debug_stall_group.argtypes = [ci]
     lib.mamba_debug_stall_group.restype = ci
+    lib.mamba_bounds_checked.argtypes = []
+    lib.mamba_bounds_checked.restype = ci
+    lib.mamba_debug_bounds_status.argtypes = [vp, vp]
+    lib.mamba_debug_bounds_status.restype = ci
+    lib.mamba_debug_shrink_output_extent.argtypes = [ci]
+    lib.mamba_debug_shrink_output_extent.restype = ci
     lib.mamba_scan_host_scratch_size.argtypes = [i64, i64, i64, i64, ci]
     lib.mamba_scan_host_scratch_size.restype = ctypes.c_size_t
     lib.mamba_scan_fwd_host.argtypes = scan_args[:9] + [fp] + scan_args[9:] + [vp, ctypes.c_size_t, vp]
@@ -570,6 +578,35 @@ def device_status(device=None) -> int:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     with torch.cuda.device(dev):
         return load_library().mamba_get_device_status(_stream(dev))
+
+
+def load_checked_library() -> ctypes.CDLL:
+    """The bounds-checked build of the library (built with nvcc first if it
+    is missing or older than its sources), declared like the normal one.
+    The binding keeps using the normal library; a caller that wants the
+    checked one for the binding's functions sets it in their place."""
+    with _lock:
+        if _build.CHECKED_LIB not in _checked:
+            if not _build.up_to_date(checked=True):
+                _build.build(checked=True)
+            _checked[_build.CHECKED_LIB] = _declare(ctypes.CDLL(_build.CHECKED_LIB))
+        return _checked[_build.CHECKED_LIB]
+
+
+_checked = {}
+
+
+def bounds_status(lib: Optional[ctypes.CDLL] = None):
+    """The first access outside its tensor that a bounds-checked launch
+    skipped since the previous call, as (site, byte offset), or None; clears
+    the record (the normal build always returns None).  Call after the work
+    has completed."""
+    lib = lib or load_library()
+    site, off = ctypes.c_int(0), ctypes.c_longlong(0)
+    rc = lib.mamba_debug_bounds_status(ctypes.c_void_p(ctypes.addressof(site)), ctypes.c_void_p(ctypes.addressof(off)))
+    if rc < 0:
+        _check("mamba_debug_bounds_status", rc)
+    return (site.value, off.value) if rc else None
 
 
 def workspace_status(workspace: torch.Tensor) -> int:

@@ -1,7 +1,9 @@
 """Build ``libmamba_scan.so`` (the C-ABI library) from ``csrc/`` with nvcc for
-sm_100a.  The library is built in-tree, next to this file.
+sm_100a, and on request the bounds-checked build of the same sources,
+``libmamba_scan_checked.so`` (MSCAN_BOUNDS_CHECK: see csrc/bounds.cuh).  Both
+are built in-tree, next to this file.
 
-Usage:  python -m selective_state_space_20_b200.build [--force] [--verbose]
+Usage:  python -m selective_state_space_20_b200.build [--force] [--verbose] [--checked]
 """
 from __future__ import annotations
 
@@ -20,6 +22,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libmamba_scan.so")
 STAMP = LIB + ".srchash"
 BUILD_DIR = os.path.join(HERE, "_build")
+CHECKED_LIB = os.path.join(HERE, "libmamba_scan_checked.so")
+CHECKED_FLAGS = ["-DMSCAN_BOUNDS_CHECK"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2",
@@ -42,9 +46,20 @@ def _deps():
         glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")) + [__file__]
 
 
-def source_digest() -> str:
+def _paths(checked: bool):
+    """(library, stamp, object directory) of the normal or the checked build."""
+    if checked:
+        return CHECKED_LIB, CHECKED_LIB + ".srchash", os.path.join(HERE, "_build_checked")
+    return LIB, STAMP, BUILD_DIR
+
+
+def _flags(checked: bool):
+    return NVCC_FLAGS + (CHECKED_FLAGS if checked else [])
+
+
+def source_digest(checked: bool = False) -> str:
     """Hash of every input of the build (sources, headers, flags)."""
-    flags = [f for f in NVCC_FLAGS if not os.path.isabs(f)]  # paths differ per checkout
+    flags = [f for f in _flags(checked) if not os.path.isabs(f)]  # paths differ per checkout
     h = hashlib.sha256(" ".join(flags).encode())
     for p in sorted(_deps()):
         with open(p, "rb") as fh:
@@ -52,17 +67,18 @@ def source_digest() -> str:
     return h.hexdigest()
 
 
-def up_to_date() -> bool:
+def up_to_date(checked: bool = False) -> bool:
     """True if the library exists and was built from the current sources."""
-    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
+    lib, stamp, _ = _paths(checked)
+    if not (os.path.exists(lib) and os.path.exists(stamp)):
         return False
-    with open(STAMP) as fh:
-        return fh.read().strip() == source_digest()
+    with open(stamp) as fh:
+        return fh.read().strip() == source_digest(checked)
 
 
-def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
-    cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
+def _compile(src: str, verbose: bool, checked: bool = False) -> str:
+    obj = os.path.join(_paths(checked)[2], os.path.basename(src) + ".o")
+    cmd = [nvcc()] + _flags(checked) + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
@@ -71,24 +87,26 @@ def _compile(src: str, verbose: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every ``csrc/*.cu`` and link ``libmamba_scan.so``."""
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD_DIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    """Compile every ``csrc/*.cu`` and link ``libmamba_scan.so`` (or, with
+    ``checked``, ``libmamba_scan_checked.so``)."""
+    lib, stamp, build_dir = _paths(checked)
+    if not force and up_to_date(checked):
+        return lib
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sources()
     with cf.ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
-    tmp = LIB + f".tmp{os.getpid()}"
+        objs = list(ex.map(lambda s: _compile(s, verbose, checked), srcs))
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    with open(STAMP, "w") as fh:
-        fh.write(source_digest())
-    return LIB
+    os.replace(tmp, lib)
+    with open(stamp, "w") as fh:
+        fh.write(source_digest(checked))
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, checked="--checked" in sys.argv))

@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include "mamba_scan.h"
+#include "bounds.cuh"
 #include "internal.h"
 
 namespace {
@@ -19,6 +20,26 @@ const void *g_last_workspace[kMaxDevices];
 void note_workspace(const void *ws) {
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) g_last_workspace[dev] = ws;
+}
+
+// The first recorded violation of the instrumented kernels (pairs, decode,
+// conv1d), every record cleared: 1 with it, 0 without, -1 on a read error.
+int take_bounds(int *site, long long *off) {
+    int found = 0;
+    int (*takes[])(int *, long long *) = {mscan::pairs_bounds_take, mscan::state_update_bounds_take,
+                                          mscan::conv1d_bounds_take};
+    for (auto take : takes) {
+        int s = 0;
+        long long o = 0;
+        const int r = take(&s, &o);
+        if (r < 0) return -1;
+        if (r > 0 && !found) {
+            found = 1;
+            *site = s;
+            *off = o;
+        }
+    }
+    return found;
 }
 
 int current_sm_count(int *status) {
@@ -590,6 +611,11 @@ int mamba_get_device_status(cudaStream_t stream) {
     if (sticky != cudaSuccess) return MAMBA_ERR_CUDA;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MAMBA_ERR_DEVICE;
+    int site = 0;
+    long long off = 0;
+    const int bounds = take_bounds(&site, &off);  // bounds-checked build only
+    if (bounds < 0) return MAMBA_ERR_CUDA;
+    if (bounds > 0) return MAMBA_ERR_BOUNDS;
     const int local = mscan::local_error_take();  // block-local launches since the last call
     if (local < 0) return MAMBA_ERR_CUDA;
     if (local > 0) return MAMBA_ERR_TIMEOUT;
@@ -849,11 +875,30 @@ const char *mamba_status_string(int status) {
         case MAMBA_ERR_OVERLAP: return "an output overlaps an input or the workspace";
         case MAMBA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
         case MAMBA_ERR_TIMEOUT: return "a persistent launch stopped waiting for a predecessor chunk";
+        case MAMBA_ERR_BOUNDS: return "a kernel access fell outside its tensor (bounds-checked build)";
         default: return "unknown status";
     }
 }
 
 int mamba_debug_stall_group(int group) { return mscan::set_stall_group(group < 0 ? -1 : group); }
+
+int mamba_bounds_checked(void) { return mscan::kBoundsChecked ? 1 : 0; }
+
+int mamba_debug_bounds_status(int *site, long long *offset) {
+    int s = 0;
+    long long o = 0;
+    const int r = take_bounds(&s, &o);
+    if (r < 0) return MAMBA_ERR_CUDA;
+    if (site) *site = s;
+    if (offset) *offset = o;
+    return r;
+}
+
+int mamba_debug_shrink_output_extent(int bytes) {
+    const int prev = mscan::g_out_extent_shrink;
+    mscan::g_out_extent_shrink = bytes < 0 ? 0 : bytes;
+    return prev;
+}
 
 int mamba_abi_version(void) { return (1 << 16) | 8; }
 

@@ -9,6 +9,17 @@ namespace mscan {
 
 enum ActType : int { kF32 = 0, kBF16 = 1 };
 
+// Test hook of the bounds-checked build: the output extent every launch
+// records is this many bytes short of the real one (0 in normal use).
+extern int g_out_extent_shrink;
+
+// The bounds-checked build's record of each instrumented translation unit
+// (1: a violation, its site and byte offset; cleared), 0 without one, -1 on
+// a read error.  Always 0 in the normal build.
+int pairs_bounds_take(int *site, long long *off);
+int state_update_bounds_take(int *site, long long *off);
+int conv1d_bounds_take(int *site, long long *off);
+
 // Element strides of one (batch, channel or state, time) tensor.
 struct Stride3 {
     int64_t b, d, t;

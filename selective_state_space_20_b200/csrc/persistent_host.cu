@@ -86,6 +86,8 @@ namespace {
 int g_stall_group = -1;  // test hook (mamba_debug_stall_group)
 }  // namespace
 
+int g_out_extent_shrink = 0;  // test hook (mamba_debug_shrink_output_extent)
+
 int set_stall_group(int group) {
     const int prev = g_stall_group;
     g_stall_group = group;
@@ -172,6 +174,28 @@ persist::Params base_params(const ScanArgs &a, int lanes, int tc) {
     kp.ckpt_gpb = (int)((a.dim + 31) / 32);
     kp.ckpt_nsup = (int)((a.seqlen + 31) / 32);
     kp.channels_last = a.channels_last ? 1 : 0;
+    // byte ranges of the pointer arguments (checked in the bounds-checked build)
+    const unsigned long long es = a.act == kBF16 ? 2 : 4;
+    const unsigned long long x = (unsigned long long)(a.batch * a.dim * a.seqlen) * es;
+    const unsigned long long bc = (unsigned long long)(a.batch * a.dstate * a.seqlen) * es;
+    const unsigned long long st = (unsigned long long)(a.batch * a.dim * a.dstate) * 4;
+    const unsigned long long row = (unsigned long long)(a.dim * a.seqlen) * es;
+    kp.x_u = extent_of(a.u, a.conv_w ? (unsigned long long)(a.batch - 1) * kp.u_bstride * es + row : x);
+    kp.x_delta = extent_of(a.delta, x);
+    kp.x_z = extent_of(a.z, a.conv_w ? (unsigned long long)(a.batch - 1) * kp.z_bstride * es + row : x);
+    kp.x_B = extent_of(a.B, bc);
+    kp.x_C = extent_of(a.C, bc);
+    kp.x_A = extent_of(a.A, (unsigned long long)(a.dim * a.dstate) * 4);
+    kp.x_D = extent_of(a.D, (unsigned long long)a.dim * 4);
+    kp.x_bias = extent_of(a.delta_bias, (unsigned long long)a.dim * 4);
+    kp.x_out = extent_of(a.out, x > (unsigned long long)g_out_extent_shrink ? x - g_out_extent_shrink : 0);
+    kp.x_last = extent_of(a.last_state, st);
+    kp.x_h0 = extent_of(a.h0, st);
+    kp.x_conv_w = extent_of(a.conv_w, (unsigned long long)(a.dim * a.conv_k) * 4);
+    kp.x_conv_b = extent_of(a.conv_b, (unsigned long long)a.dim * 4);
+    kp.x_u_out = extent_of(a.u_out, x);
+    kp.x_ckpt = extent_of(a.ckpt, (unsigned long long)a.batch * kp.ckpt_gpb * kp.ckpt_nsup * 32 * 16 * 4);
+    kp.x_carry = extent_of(nullptr, 0);
     return kp;
 }
 }  // namespace
@@ -239,6 +263,7 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
         kp.queue = nullptr;
         kp.progress = reinterpret_cast<unsigned *>(w + l.queue_off);
         kp.carry = reinterpret_cast<float *>(w + l.carry_off);
+        kp.x_carry = extent_of(kp.carry, l.bytes - l.carry_off);
         cudaError_t e = cudaMemsetAsync(w, 0, l.queue_off + (size_t)groups * 4, st);
         if (e != cudaSuccess) return e;
         return launch_persistent_split(kp, lanes, a.act, sm_count, st);

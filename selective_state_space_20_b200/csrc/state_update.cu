@@ -19,6 +19,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "bounds.cuh"
 #include "device_math.cuh"
 #include "internal.h"
 
@@ -32,7 +33,19 @@ struct SUParams {
     int64_t rows, dim;
     int dstate;
     int softplus;
+    // byte ranges of the pointer arguments, for the bounds-checked build
+    Extent x_state, x_u, x_delta, x_B, x_C, x_z, x_A, x_D, x_bias, x_out;
 };
+
+// Loads that the bounds-checked build tests against the tensor's range (a
+// load outside reads zero; see bounds.cuh).
+template <typename T>
+__device__ __forceinline__ float load_chk(const Extent &e, const T *q, int site) {
+    return within(e, q, sizeof(T), site) ? Elem<T>::load(q) : 0.f;
+}
+__device__ __forceinline__ float ldg_chk(const Extent &e, const float *q, int site) {
+    return within(e, q, 4, site) ? __ldg(q) : 0.f;
+}
 
 // NV > 0: dstate == NV, known at compile time, 16-byte state accesses.
 // NV == 0: any dstate, scalar accesses.
@@ -51,9 +64,10 @@ state_update_kernel(const SUParams p) {
     const float *Ad = p.A + d * N;
     using Dk = Decay<sizeof(T) == 4>;
 
-    float dl = Elem<T>::load(gd + row) + (p.delta_bias ? __ldg(p.delta_bias + d) : 0.f);
+    float dl = load_chk(p.x_delta, gd + row, kSiteDelta) +
+               (p.delta_bias ? ldg_chk(p.x_bias, p.delta_bias + d, kSiteBias) : 0.f);
     if (p.softplus) dl = Dk::softplus(dl);
-    const float ut = Elem<T>::load(gu + row);
+    const float ut = load_chk(p.x_u, gu + row, kSiteU);
     const float du = dl * ut;
     const float dl2 = dl * Dk::kScale;
     float *st = p.state + row * N;
@@ -62,28 +76,35 @@ state_update_kernel(const SUParams p) {
     if (NV > 0) {
 #pragma unroll
         for (int n = 0; n < N; n += 4) {
-            float4 h = *reinterpret_cast<const float4 *>(st + n);
-            const float4 a4 = __ldg(reinterpret_cast<const float4 *>(Ad + n));
+            const bool sok = within(p.x_state, st + n, 16, kSiteState);
+            float4 h = sok ? *reinterpret_cast<const float4 *>(st + n) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 a4 = within(p.x_A, Ad + n, 16, kSiteA) ? __ldg(reinterpret_cast<const float4 *>(Ad + n))
+                                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
             HS hv[4] = {h.x, h.y, h.z, h.w};
             const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                hv[i] = Dk::step(dl2 * av[i], hv[i], du * Elem<T>::load(gB + n + i));
-                y = fma((HS)Elem<T>::load(gC + n + i), hv[i], y);
+                hv[i] = Dk::step(dl2 * av[i], hv[i], du * load_chk(p.x_B, gB + n + i, kSiteB));
+                y = fma((HS)load_chk(p.x_C, gC + n + i, kSiteC), hv[i], y);
             }
-            *reinterpret_cast<float4 *>(st + n) = make_float4((float)hv[0], (float)hv[1], (float)hv[2], (float)hv[3]);
+            if (sok)
+                *reinterpret_cast<float4 *>(st + n) =
+                    make_float4((float)hv[0], (float)hv[1], (float)hv[2], (float)hv[3]);
         }
     } else {
         for (int n = 0; n < N; ++n) {
-            const HS hn = Dk::step(dl2 * __ldg(Ad + n), (HS)st[n], du * Elem<T>::load(gB + n));
-            st[n] = (float)hn;
-            y = fma((HS)Elem<T>::load(gC + n), hn, y);
+            const bool sok = within(p.x_state, st + n, 4, kSiteState);
+            const HS hn = Dk::step(dl2 * ldg_chk(p.x_A, Ad + n, kSiteA), (HS)(sok ? st[n] : 0.f),
+                                   du * load_chk(p.x_B, gB + n, kSiteB));
+            if (sok) st[n] = (float)hn;
+            y = fma((HS)load_chk(p.x_C, gC + n, kSiteC), hn, y);
         }
     }
     float yo = (float)y;
-    if (p.D) yo = (float)fma((HS)__ldg(p.D + d), (HS)ut, y);
-    if (gz) yo *= silu_f(Elem<T>::load(gz + row));
-    Elem<T>::store(static_cast<T *>(p.out) + row, yo);
+    if (p.D) yo = (float)fma((HS)ldg_chk(p.x_D, p.D + d, kSiteD), (HS)ut, y);
+    if (gz) yo *= silu_f(load_chk(p.x_z, gz + row, kSiteZ));
+    T *o = static_cast<T *>(p.out) + row;
+    if (within(p.x_out, o, sizeof(T), kSiteOut)) Elem<T>::store(o, yo);
 }
 
 // Four states per lane: bf16 / fp32 loads of four consecutive B or C values.
@@ -124,18 +145,22 @@ state_update_lanes_kernel(const SUParams p) {
 
     float4 h4[V], a4[V], b4[V], c4[V];
     float4 *st = reinterpret_cast<float4 *>(p.state + (int64_t)row * NV) + qi;
+    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int v = 0; v < V; ++v) {
-        h4[v] = st[v * Q];
-        a4[v] = __ldg(reinterpret_cast<const float4 *>(p.A + (int64_t)d * NV) + qi + v * Q);
-        b4[v] = Quad<T>::load(static_cast<const T *>(p.B) + (int64_t)b * NV + 4 * (qi + v * Q));
-        c4[v] = Quad<T>::load(static_cast<const T *>(p.C) + (int64_t)b * NV + 4 * (qi + v * Q));
+        const float4 *a = reinterpret_cast<const float4 *>(p.A + (int64_t)d * NV) + qi + v * Q;
+        const T *bq = static_cast<const T *>(p.B) + (int64_t)b * NV + 4 * (qi + v * Q);
+        const T *cq = static_cast<const T *>(p.C) + (int64_t)b * NV + 4 * (qi + v * Q);
+        h4[v] = within(p.x_state, st + v * Q, 16, kSiteState) ? st[v * Q] : zero4;
+        a4[v] = within(p.x_A, a, 16, kSiteA) ? __ldg(a) : zero4;
+        b4[v] = within(p.x_B, bq, 4 * sizeof(T), kSiteB) ? Quad<T>::load(bq) : zero4;
+        c4[v] = within(p.x_C, cq, 4 * sizeof(T), kSiteC) ? Quad<T>::load(cq) : zero4;
     }
-    const float dr = Elem<T>::load(static_cast<const T *>(p.delta) + row);
-    const float ut = Elem<T>::load(static_cast<const T *>(p.u) + row);
-    const float zt = (p.z && qi == 0) ? Elem<T>::load(static_cast<const T *>(p.z) + row) : 0.f;
-    const float bias = p.delta_bias ? __ldg(p.delta_bias + d) : 0.f;
-    const float Dd = (p.D && qi == 0) ? __ldg(p.D + d) : 0.f;
+    const float dr = load_chk(p.x_delta, static_cast<const T *>(p.delta) + row, kSiteDelta);
+    const float ut = load_chk(p.x_u, static_cast<const T *>(p.u) + row, kSiteU);
+    const float zt = (p.z && qi == 0) ? load_chk(p.x_z, static_cast<const T *>(p.z) + row, kSiteZ) : 0.f;
+    const float bias = p.delta_bias ? ldg_chk(p.x_bias, p.delta_bias + d, kSiteBias) : 0.f;
+    const float Dd = (p.D && qi == 0) ? ldg_chk(p.x_D, p.D + d, kSiteD) : 0.f;
 
     float dl = dr + bias;
     if (p.softplus) dl = Dk::softplus(dl);
@@ -155,12 +180,14 @@ state_update_lanes_kernel(const SUParams p) {
     for (int o = Q / 2; o >= 1; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
     if (!live) return;
 #pragma unroll
-    for (int v = 0; v < V; ++v) st[v * Q] = h4[v];
+    for (int v = 0; v < V; ++v)
+        if (within(p.x_state, st + v * Q, 16, kSiteState)) st[v * Q] = h4[v];
     if (qi == 0) {
         float yo = (float)y;
         if (p.D) yo = (float)fma((HS)Dd, (HS)ut, y);
         if (p.z) yo *= silu_f(zt);
-        Elem<T>::store(static_cast<T *>(p.out) + row, yo);
+        T *o = static_cast<T *>(p.out) + row;
+        if (within(p.x_out, o, sizeof(T), kSiteOut)) Elem<T>::store(o, yo);
     }
 }
 
@@ -213,11 +240,25 @@ static cudaError_t launch_typed(const SUParams &kp, cudaStream_t st) {
     return launch_rows<T>(kp, st);
 }
 
+MSCAN_BOUNDS_TAKE(state_update_bounds_take)
+
 cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t st) {
     SUParams kp;
     kp.state = a.state; kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
     kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias; kp.out = a.out;
     kp.rows = a.batch * a.dim; kp.dim = a.dim; kp.dstate = a.dstate; kp.softplus = a.softplus;
+    const unsigned long long es = a.act == kBF16 ? 2 : 4, rows = (unsigned long long)(a.batch * a.dim);
+    const unsigned long long xb = rows * es;
+    kp.x_state = extent_of(a.state, rows * a.dstate * 4);
+    kp.x_u = extent_of(a.u, xb);
+    kp.x_delta = extent_of(a.delta, xb);
+    kp.x_z = extent_of(a.z, xb);
+    kp.x_B = extent_of(a.B, (unsigned long long)(a.batch * a.dstate) * es);
+    kp.x_C = extent_of(a.C, (unsigned long long)(a.batch * a.dstate) * es);
+    kp.x_A = extent_of(a.A, (unsigned long long)(a.dim * a.dstate) * 4);
+    kp.x_D = extent_of(a.D, (unsigned long long)a.dim * 4);
+    kp.x_bias = extent_of(a.delta_bias, (unsigned long long)a.dim * 4);
+    kp.x_out = extent_of(a.out, xb > (unsigned long long)g_out_extent_shrink ? xb - g_out_extent_shrink : 0);
     if (a.act == kBF16) return launch_typed<__nv_bfloat16>(kp, st);
     return launch_typed<float>(kp, st);
 }

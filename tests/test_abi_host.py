@@ -282,3 +282,14 @@ def test_host_memory_scan_validation(lib):
     bad = list(args)
     bad[15] = 65
     assert lib.mamba_scan_fwd_host(*bad, vp(0x1000000), 1 << 30, None) == -3
+
+
+def test_checked_build_exports_the_same_abi():
+    """The bounds-checked build of the same sources: every declared symbol,
+    and it says which build it is (host-only calls)."""
+    checked = binding.load_checked_library()
+    for name in declared_functions():
+        assert hasattr(checked, name), f"{name} not exported by the checked build"
+    assert checked.mamba_bounds_checked() == 1
+    assert binding.load_library().mamba_bounds_checked() == 0
+    assert binding.load_library().mamba_debug_shrink_output_extent(0) == 0

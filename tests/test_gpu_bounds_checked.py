@@ -1,0 +1,219 @@
+"""The bounds-checked build (libmamba_scan_checked.so, MSCAN_BOUNDS_CHECK).
+
+Its instrumented kernels -- the lane-split scan in every form that uses it,
+the decode step, the conv1d kernels -- test every global access against the
+byte range of its tensor.  On the shapes below (ragged groups and lengths,
+N < 16, both lane counts, two-phase pieces, the device-wide and block-local
+forms, the (b, l, d) layout, the fused conv1d with u written out,
+checkpoints, initial and final states) they must record no access outside a
+tensor and give the normal build's results bit for bit.  A test hook then
+shortens the output range the launches record: the checks must report the
+output site at the first byte past the shortened range, skip that access
+(the tail of the output keeps its old contents) and leave everything else
+equal to the normal build's.  No access leaves allocated memory in any of
+these runs.
+"""
+import contextlib
+
+import pytest
+import torch
+
+from selective_state_space_20_b200 import binding, inputs
+
+pytestmark = pytest.mark.gpu
+
+SITE_OUT = 13
+
+
+@pytest.fixture(scope="module")
+def checked():
+    lib = binding.load_checked_library()
+    assert lib.mamba_bounds_checked() == 1
+    assert binding.load_library().mamba_bounds_checked() == 0
+    return lib
+
+
+@contextlib.contextmanager
+def using(lib):
+    prev = binding._lib
+    binding._lib = lib
+    try:
+        yield
+    finally:
+        binding._lib = prev
+
+
+def both(checked, fn):
+    """fn() with the normal library, then with the checked one; the checked
+    run must record no violation."""
+    ref = fn()
+    torch.cuda.synchronize()
+    with using(checked):
+        got = fn()
+        torch.cuda.synchronize()
+        assert binding.bounds_status(checked) is None
+    return ref, got
+
+
+def equal(a, b):
+    if isinstance(a, (tuple, list)):
+        return all(equal(x, y) for x, y in zip(a, b))
+    return torch.equal(a, b)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("shape,dstate,lanes", [((2, 70, 336), 16, 2), ((3, 33, 1000), 5, 4),
+                                                ((1, 64, 8192), 16, 2), ((4, 1030, 256), 16, 0)],
+                         ids=["2x70x336-R2", "3x33x1000-N5-R4", "1x64x8192-two-phase", "4x1030x256-lanes-auto"])
+def test_block_local_scan(checked, dtype, shape, dstate, lanes):
+    b, d, L = shape
+    ins = inputs.scan_inputs(inputs.custom(b, d, L, dstate, dtype, seed=b + d + L), device="cuda")
+    h0 = inputs.initial_state(b, d, dstate, seed=3, device="cuda")
+    # lanes 0: the library's choice within the block-local schedule
+    kw = dict(schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=lanes)
+    run = lambda: binding.mamba_scan_fwd(ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"], D=ins["D"],  # noqa: E731
+                                         z=ins["z"], delta_bias=ins["delta_bias"], h0=h0, return_last_state=True,
+                                         **kw)
+    ref, got = both(checked, run)
+    assert equal(ref, got)
+
+
+@pytest.mark.parametrize("lanes", [2, 4])
+def test_device_wide_scan_and_checkpoints(checked, lanes):
+    w = inputs.custom(2, 16 * 30, 512, 16, "bf16", seed=31)
+    ins = inputs.scan_inputs(w, device="cuda")
+    ws = torch.empty(binding.mamba_scan_workspace_size(w.batch, w.dim, w.seqlen, w.dstate, torch.bfloat16),
+                     device="cuda", dtype=torch.uint8)
+    run = lambda: binding.mamba_scan_fwd(ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"], D=ins["D"],  # noqa: E731
+                                         z=ins["z"], delta_bias=ins["delta_bias"], return_last_state=True,
+                                         workspace=ws, schedule=binding.SCHEDULE_PERSISTENT,
+                                         lanes_per_channel=lanes)
+    ref, got = both(checked, run)
+    assert equal(ref, got)
+    ck = lambda: binding.mamba_scan_fwd_ckpt(ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"], D=ins["D"],  # noqa: E731
+                                             z=ins["z"], delta_bias=ins["delta_bias"])
+    ref, got = both(checked, ck)
+    assert equal(ref, got)
+
+
+@pytest.mark.parametrize("lanes", [2, 4])
+def test_page_layout_and_fused_conv(checked, lanes):
+    w = inputs.custom(2, 96, 336, 16, "bf16", seed=32)
+    cpu = inputs.scan_inputs(w)
+    cl = {k: (None if v is None else (v.transpose(1, 2).contiguous().transpose(1, 2)
+                                      if k in ("u", "delta", "z", "B", "C") else v).cuda())
+          for k, v in cpu.items()}
+    run = lambda: binding.mamba_scan_fwd_strided(cl["u"], cl["delta"], cl["A"], cl["B"], cl["C"], D=cl["D"],  # noqa: E731
+                                                 z=cl["z"], delta_bias=cl["delta_bias"], return_last_state=True,
+                                                 schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=lanes)
+    ref, got = both(checked, run)
+    assert equal(ref, got)
+    ci = inputs.conv_inputs(2, 96, 512, 4, "bf16", seed=33, device="cuda")
+    ins = inputs.scan_inputs(inputs.custom(2, 96, 512, 16, "bf16", seed=34), device="cuda")
+    x, z = ci["xz"][:, :96], ci["xz"][:, 96:]
+    fused = lambda: binding.mamba_scan_fwd_conv(x, ci["weight"], ci["bias"], ins["delta"], ins["A"], ins["B"],  # noqa: E731
+                                                ins["C"], D=ins["D"], z=z, delta_bias=ins["delta_bias"],
+                                                return_last_state=True, return_u=True)
+    ref, got = both(checked, fused)
+    assert equal(ref, got)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("dstate", [16, 13, 8])
+def test_decode_step(checked, dtype, dstate):
+    d = inputs.decode_inputs(inputs.DecodeWorkload("decode test", 7, 301, dstate, 2, dtype, 1e-3, 1e-1,
+                                                   "uniform", seed=35), device="cuda", steps=2)
+    state0 = inputs.initial_state(7, 301, dstate, seed=8, device="cuda")
+
+    def run():
+        st = state0.clone()
+        outs = [binding.mamba_state_update(st, d["u"][t], d["delta"][t], d["A"], d["B"][t], d["C"][t], D=d["D"],
+                                           z=d["z"][t], delta_bias=d["delta_bias"]) for t in range(2)]
+        return outs + [st]
+
+    ref, got = both(checked, run)
+    assert equal(ref, got)
+
+
+@pytest.mark.parametrize("L", [4096, 333])
+def test_conv1d(checked, L):
+    ci = inputs.conv_inputs(3, 40, L, 4, "bf16", seed=36, device="cuda")
+    run = lambda: binding.mamba_conv1d_fwd(ci["xz"], ci["weight"], ci["bias"], dim=40)  # noqa: E731
+    ref, got = both(checked, run)
+    assert equal(ref, got)
+    state0 = torch.randn(3, 40, 3, device="cuda")
+
+    def step():
+        st = state0.clone()
+        return binding.mamba_conv1d_update(st, ci["xz"][:, :40, 0].contiguous(), ci["weight"], ci["bias"]), st
+
+    ref, got = both(checked, step)
+    assert equal(ref, got)
+
+
+def _shrunk(checked, fn, out_of, shrink):
+    """fn() with the normal library, then with the checked one and the
+    output range `shrink` bytes short; checks the violation recorded (the
+    output site, at the first byte past the range) and returns both results."""
+    ref = fn()
+    torch.cuda.synchronize()
+    with using(checked):
+        prev = checked.mamba_debug_shrink_output_extent(shrink)
+        try:
+            got = fn()
+            torch.cuda.synchronize()
+        finally:
+            checked.mamba_debug_shrink_output_extent(prev)
+        hit = binding.bounds_status(checked)
+    nbytes = out_of(ref).numel() * out_of(ref).element_size()
+    assert hit == (SITE_OUT, nbytes - shrink), (hit, nbytes)
+    return ref, got
+
+
+def test_a_short_output_range_is_reported_and_its_store_skipped(checked):
+    w = inputs.custom(2, 64, 512, 16, "bf16", seed=37)
+    ins = inputs.scan_inputs(w, device="cuda")
+    sentinel = torch.full_like(ins["u"], 7.0)
+
+    def scan():
+        out = sentinel.clone()
+        # the block-local lane-split kernel (a shape this small would otherwise
+        # take the static kernel, which is not instrumented)
+        binding.mamba_scan_fwd(ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"], D=ins["D"], z=ins["z"],
+                               delta_bias=ins["delta_bias"], out=out, schedule=binding.SCHEDULE_LOCAL)
+        return out
+
+    ref, got = _shrunk(checked, scan, lambda o: o, 16)
+    flat_r, flat_g = ref.reshape(-1), got.reshape(-1)
+    assert torch.equal(flat_g[:-8], flat_r[:-8])  # every 16-byte chunk but the last
+    assert torch.all(flat_g[-8:] == 7.0)          # the last was skipped
+
+    d = inputs.decode_inputs(inputs.DecodeWorkload("decode shrink", 4, 96, 16, 1, "bf16", 1e-3, 1e-1,
+                                                   "uniform", seed=38), device="cuda", steps=1)
+    st0 = inputs.initial_state(4, 96, 16, seed=9, device="cuda")
+
+    def step():
+        st = st0.clone()
+        out = torch.full((4, 96), 7.0, device="cuda", dtype=torch.bfloat16)
+        binding.mamba_state_update(st, d["u"][0], d["delta"][0], d["A"], d["B"][0], d["C"][0], D=d["D"],
+                                   z=d["z"][0], delta_bias=d["delta_bias"], out=out)
+        return out
+
+    ref, got = _shrunk(checked, step, lambda o: o, 2)
+    assert torch.equal(got.reshape(-1)[:-1], ref.reshape(-1)[:-1]) and got.reshape(-1)[-1] == 7.0
+
+    ci = inputs.conv_inputs(2, 32, 256, 4, "bf16", seed=39, device="cuda")
+    conv = lambda: binding.mamba_conv1d_fwd(ci["xz"], ci["weight"], ci["bias"], dim=32,  # noqa: E731
+                                            out=torch.full((2, 32, 256), 7.0, device="cuda", dtype=torch.bfloat16))
+    ref, got = _shrunk(checked, conv, lambda o: o, 16)
+    assert torch.equal(got.reshape(-1)[:-8], ref.reshape(-1)[:-8]) and torch.all(got.reshape(-1)[-8:] == 7.0)
+
+    # the device status reports it too (and reading clears the record)
+    with using(checked):
+        prev = checked.mamba_debug_shrink_output_extent(16)
+        try:
+            scan()
+        finally:
+            checked.mamba_debug_shrink_output_extent(prev)
+        assert binding.device_status() == binding.MAMBA_ERR_BOUNDS
+        assert binding.device_status() == 0 and binding.bounds_status(checked) is None
