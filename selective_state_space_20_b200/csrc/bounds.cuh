@@ -2,14 +2,14 @@
 //
 // Every kernel launch carries, for each pointer argument, the byte range it
 // may touch (an Extent, filled on the host from the sizes the caller passed).
-// In the checked build each global access of the lane-split scan kernel, the
-// decode step and the conv1d kernels first asks within(): an access that
-// would leave its range is skipped -- a load reads zeros, a store is dropped
-// -- and the first such access of the launch is recorded (site and byte
-// offset) in a word of its translation unit, which the host reads through
-// mamba_get_device_status / mamba_debug_bounds_status.  Nothing traps or
-// faults.  In the normal build within() is a constant true and the checks
-// compile away.  The static, one-lane, complex and backward kernels are not
+// In the checked build each global access of the lane-split and static scan
+// kernels, the decode step and the conv1d kernels first asks within(): an
+// access that would leave its range is skipped -- a load reads zeros, a store
+// is dropped -- and the first such access of the launch is recorded (site and
+// byte offset) in a word of its translation unit, which the host reads
+// through mamba_get_device_status / mamba_debug_bounds_status.  Nothing traps
+// or faults.  In the normal build within() is a constant true and the checks
+// compile away.  The one-lane, complex and backward kernels are not
 // instrumented.
 #pragma once
 

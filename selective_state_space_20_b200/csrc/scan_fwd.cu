@@ -46,6 +46,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "bounds.cuh"
 #include "device_math.cuh"
 #include "internal.h"
 
@@ -64,6 +65,8 @@ struct KParams {
     int softplus;
     int vec;           // u / delta / z / out: 16-byte vectors along the kernel's contiguous axis
     int bc_mode;       // B / C: 0 element copies, 1 vectors along time, 2 vectors along states
+    // byte ranges of the pointer arguments, for the bounds-checked build
+    Extent x_u, x_delta, x_z, x_B, x_C, x_A, x_D, x_bias, x_out, x_last, x_h0;
 };
 
 // ------------------------------------------------------------ geometry
@@ -181,8 +184,10 @@ scan_fwd_kernel(const KParams p) {
 #pragma unroll
     for (int s = 0; s < S; ++s) {
         const int n = r * S + s;
-        A2[s] = (d < Dm && n < N) ? __ldg(p.A + d * N + n) * Dk::kScale : 0.f;
-        h[s] = (p.h0 && d < Dm && n < N) ? __ldcg(p.h0 + (b * Dm + d) * N + n) : 0.f;
+        A2[s] = (d < Dm && n < N && within(p.x_A, p.A + d * N + n, 4, kSiteA)) ? __ldg(p.A + d * N + n) * Dk::kScale
+                                                                               : 0.f;
+        h[s] = (p.h0 && d < Dm && n < N && within(p.x_h0, p.h0 + (b * Dm + d) * N + n, 4, kSiteH0))
+                   ? __ldcg(p.h0 + (b * Dm + d) * N + n) : 0.f;
     }
 
     // ---- copy one chunk's raw tiles into stage `st`: u / delta / z as
@@ -200,18 +205,26 @@ scan_fwd_kernel(const KParams p) {
                     const int pc = vi / VPR, tv = vi % VPR;
                     const int64_t t = t0 + tv * V, dd = d0 + pc;
                     const bool ok = (dd < Dm) && (t < L);
-                    cp_async16(rU + pc * TC + tv * V, gu + (ok ? b * su.b + dd * su.d + t : 0), ok);
-                    cp_async16(rD + pc * TC + tv * V, gd + (ok ? b * sdl.b + dd * sdl.d + t : 0), ok);
-                    if (has_z) cp_async16(rZ + pc * TC + tv * V, gz + (ok ? b * sz.b + dd * sz.d + t : 0), ok);
+                    const T *pu = gu + (ok ? b * su.b + dd * su.d + t : 0), *pd = gd + (ok ? b * sdl.b + dd * sdl.d + t : 0);
+                    cp_async16(rU + pc * TC + tv * V, pu, ok && within(p.x_u, pu, 16, kSiteU));
+                    cp_async16(rD + pc * TC + tv * V, pd, ok && within(p.x_delta, pd, 16, kSiteDelta));
+                    if (has_z) {
+                        const T *pz = gz + (ok ? b * sz.b + dd * sz.d + t : 0);
+                        cp_async16(rZ + pc * TC + tv * V, pz, ok && within(p.x_z, pz, 16, kSiteZ));
+                    }
                 }
             } else {
                 for (int vi = tid; vi < TC * CVR; vi += THREADS) {
                     const int tt = vi / CVR, cv = vi % CVR;
                     const int64_t t = t0 + tt, dd = d0 + cv * V;
                     const bool ok = (dd < Dm) && (t < L);  // dim is a whole number of vectors
-                    cp_async16(rU + tt * CG + cv * V, gu + (ok ? b * su.b + t * su.t + dd : 0), ok);
-                    cp_async16(rD + tt * CG + cv * V, gd + (ok ? b * sdl.b + t * sdl.t + dd : 0), ok);
-                    if (has_z) cp_async16(rZ + tt * CG + cv * V, gz + (ok ? b * sz.b + t * sz.t + dd : 0), ok);
+                    const T *pu = gu + (ok ? b * su.b + t * su.t + dd : 0), *pd = gd + (ok ? b * sdl.b + t * sdl.t + dd : 0);
+                    cp_async16(rU + tt * CG + cv * V, pu, ok && within(p.x_u, pu, 16, kSiteU));
+                    cp_async16(rD + tt * CG + cv * V, pd, ok && within(p.x_delta, pd, 16, kSiteDelta));
+                    if (has_z) {
+                        const T *pz = gz + (ok ? b * sz.b + t * sz.t + dd : 0);
+                        cp_async16(rZ + tt * CG + cv * V, pz, ok && within(p.x_z, pz, 16, kSiteZ));
+                    }
                 }
             }
         } else {
@@ -220,9 +233,13 @@ scan_fwd_kernel(const KParams p) {
                 const int pc = CL ? e % CG : e / TC, tt = CL ? e / CG : e % TC;
                 const int64_t t = t0 + tt, dd = d0 + pc;
                 const bool ok = (dd < Dm) && (t < L);
-                rU[e] = ok ? gu[b * su.b + dd * su.d + t * su.t] : T(0.f);
-                rD[e] = ok ? gd[b * sdl.b + dd * sdl.d + t * sdl.t] : T(0.f);
-                if (has_z) rZ[e] = ok ? gz[b * sz.b + dd * sz.d + t * sz.t] : T(0.f);
+                const T *pu = gu + b * su.b + dd * su.d + t * su.t, *pd = gd + b * sdl.b + dd * sdl.d + t * sdl.t;
+                rU[e] = (ok && within(p.x_u, pu, sizeof(T), kSiteU)) ? *pu : T(0.f);
+                rD[e] = (ok && within(p.x_delta, pd, sizeof(T), kSiteDelta)) ? *pd : T(0.f);
+                if (has_z) {
+                    const T *pz = gz + b * sz.b + dd * sz.d + t * sz.t;
+                    rZ[e] = (ok && within(p.x_z, pz, sizeof(T), kSiteZ)) ? *pz : T(0.f);
+                }
             }
         }
         if (p.bc_mode == 1) {
@@ -233,7 +250,9 @@ scan_fwd_kernel(const KParams p) {
                 const bool ok = (n < N) && (t < L);
                 const Stride3 &sx = which ? sCs : sBs;
                 const int64_t off = ok ? b * sx.b + n * sx.d + t : 0;
-                cp_async16((which ? rC : rB) + n * TC + tv * V, (which ? gC : gB) + off, ok);
+                const T *src = (which ? gC : gB) + off;
+                cp_async16((which ? rC : rB) + n * TC + tv * V, src,
+                           ok && within(which ? p.x_C : p.x_B, src, 16, which ? kSiteC : kSiteB));
             }
         } else if (p.bc_mode == 2) {
             for (int vi = tid; vi < 2 * TC * NVR; vi += THREADS) {
@@ -243,7 +262,9 @@ scan_fwd_kernel(const KParams p) {
                 const bool ok = (n < N) && (t < L);  // dstate is a whole number of vectors
                 const Stride3 &sx = which ? sCs : sBs;
                 const int64_t off = ok ? b * sx.b + t * sx.t + n : 0;
-                cp_async16((which ? rC : rB) + tt * NP + n, (which ? gC : gB) + off, ok);
+                const T *src = (which ? gC : gB) + off;
+                cp_async16((which ? rC : rB) + tt * NP + n, src,
+                           ok && within(which ? p.x_C : p.x_B, src, 16, which ? kSiteC : kSiteB));
             }
         } else {
             for (int e = tid; e < 2 * NP * TC; e += THREADS) {
@@ -252,7 +273,9 @@ scan_fwd_kernel(const KParams p) {
                 const int64_t t = t0 + tt;
                 const bool ok = (n < N) && (t < L);
                 const Stride3 &sx = which ? sCs : sBs;
-                (which ? rC : rB)[rem] = ok ? (which ? gC : gB)[b * sx.b + n * sx.d + t * sx.t] : T(0.f);
+                const T *src = (which ? gC : gB) + b * sx.b + n * sx.d + t * sx.t;
+                (which ? rC : rB)[rem] =
+                    (ok && within(which ? p.x_C : p.x_B, src, sizeof(T), which ? kSiteC : kSiteB)) ? *src : T(0.f);
             }
         }
         cp_async_commit();  // an empty group when everything was copied by hand
@@ -277,7 +300,8 @@ scan_fwd_kernel(const KParams p) {
         for (int vi = tid; vi < CH_VEC; vi += THREADS) {
             const int pc = CL ? vi % CG : vi / VPR, tv = CL ? vi / CG : vi % VPR;
             const int64_t dd = d0 + pc;
-            const float bias = (dd < Dm && p.delta_bias) ? __ldg(p.delta_bias + dd) : 0.f;
+            const float bias = (dd < Dm && p.delta_bias && within(p.x_bias, p.delta_bias + dd, 4, kSiteBias))
+                                   ? __ldg(p.delta_bias + dd) : 0.f;
             float fu[V], fd[V];
             if (!CL) {
                 Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + pc * TC + tv * V), fu);
@@ -373,7 +397,7 @@ scan_fwd_kernel(const KParams p) {
                 const int64_t dd = d0 + pc;
                 const int64_t t = t0 + tv * V;
                 if (dd >= Dm || tv * V >= tvalid) continue;
-                const float Dd = p.D ? __ldg(p.D + dd) : 0.f;
+                const float Dd = (p.D && within(p.x_D, p.D + dd, 4, kSiteD)) ? __ldg(p.D + dd) : 0.f;
                 float fu[V], fz[V], y[V];
                 Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + pc * TC + tv * V), fu);
                 if (has_z) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rZ + pc * TC + tv * V), fz);
@@ -391,11 +415,12 @@ scan_fwd_kernel(const KParams p) {
                 }
                 T *dst = gout + b * so.b + dd * so.d + t * so.t;
                 if (p.vec) {
-                    stg16_stream(dst, Elem<T>::pack(y));
+                    if (within(p.x_out, dst, 16, kSiteOut)) stg16_stream(dst, Elem<T>::pack(y));
                 } else {
 #pragma unroll
                     for (int i = 0; i < V; ++i)
-                        if (tv * V + i < tvalid) Elem<T>::store(dst + i * so.t, y[i]);
+                        if (tv * V + i < tvalid && within(p.x_out, dst + i * so.t, sizeof(T), kSiteOut))
+                            Elem<T>::store(dst + i * so.t, y[i]);
                 }
             }
         } else {  // one thread per V channels of one timestep
@@ -409,18 +434,20 @@ scan_fwd_kernel(const KParams p) {
                 if (has_z) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rZ + tt * CG + cv * V), fz);
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
-                    const float Dd = (p.D && dd + i < Dm) ? __ldg(p.D + dd + i) : 0.f;
+                    const float Dd = (p.D && dd + i < Dm && within(p.x_D, p.D + dd + i, 4, kSiteD)) ? __ldg(p.D + dd + i)
+                                                                                                : 0.f;
                     float o = fmaf(Dd, fu[i], sDelta[(cv * V + i) * TCP + tt]);
                     if (has_z) o *= silu_f(fz[i]);
                     y[i] = o;
                 }
                 T *dst = gout + b * so.b + t * so.t + dd * so.d;
                 if (p.vec) {
-                    stg16_stream(dst, Elem<T>::pack(y));
+                    if (within(p.x_out, dst, 16, kSiteOut)) stg16_stream(dst, Elem<T>::pack(y));
                 } else {
 #pragma unroll
                     for (int i = 0; i < V; ++i)
-                        if (dd + i < Dm) Elem<T>::store(dst + i * so.d, y[i]);
+                        if (dd + i < Dm && within(p.x_out, dst + i * so.d, sizeof(T), kSiteOut))
+                            Elem<T>::store(dst + i * so.d, y[i]);
                 }
             }
         }
@@ -431,7 +458,7 @@ scan_fwd_kernel(const KParams p) {
 #pragma unroll
         for (int s = 0; s < S; ++s) {
             const int n = r * S + s;
-            if (n < N) ls[n] = (float)h[s];
+            if (n < N && within(p.x_last, ls + n, 4, kSiteLastState)) ls[n] = (float)h[s];
         }
     }
 }
@@ -520,6 +547,8 @@ static StaticLayout static_layout(const ScanArgs &a) {
     return r;
 }
 
+MSCAN_BOUNDS_TAKE(static_bounds_take)
+
 cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &pl, cudaStream_t st) {
     KParams kp;
     kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
@@ -530,6 +559,26 @@ cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &pl, cudaStream_t 
     kp.dstate = a.dstate; kp.softplus = a.softplus;
     const StaticLayout lay = static_layout(a);
     kp.st = lay.st; kp.vec = lay.vec; kp.bc_mode = lay.bc_mode;
+    // byte ranges (bounds-checked build): one past the last element of each strided tensor
+    const unsigned long long es = a.act == kBF16 ? 2 : 4;
+    auto span = [&](const void *q, const Stride3 &x, int64_t rows) {
+        const unsigned long long last = (unsigned long long)((a.batch - 1) * x.b + (rows - 1) * x.d +
+                                                             (a.seqlen - 1) * x.t);
+        return extent_of(q, (last + 1) * es);
+    };
+    kp.x_u = span(a.u, lay.st.u, a.dim);
+    kp.x_delta = span(a.delta, lay.st.delta, a.dim);
+    kp.x_z = span(a.z, lay.st.z, a.dim);
+    kp.x_B = span(a.B, lay.st.B, a.dstate);
+    kp.x_C = span(a.C, lay.st.C, a.dstate);
+    kp.x_out = span(a.out, lay.st.out, a.dim);
+    if (kp.x_out.bytes > (unsigned long long)g_out_extent_shrink) kp.x_out.bytes -= g_out_extent_shrink;
+    else kp.x_out.bytes = 0;
+    kp.x_A = extent_of(a.A, (unsigned long long)(a.dim * a.dstate) * 4);
+    kp.x_D = extent_of(a.D, (unsigned long long)a.dim * 4);
+    kp.x_bias = extent_of(a.delta_bias, (unsigned long long)a.dim * 4);
+    kp.x_last = extent_of(a.last_state, (unsigned long long)(a.batch * a.dim * a.dstate) * 4);
+    kp.x_h0 = extent_of(a.h0, (unsigned long long)(a.batch * a.dim * a.dstate) * 4);
 #define X(T, NP_, R_, TH_) \
     if (a.act == act_of<T>() && pl.padded_dstate == NP_ && pl.lanes == R_ && pl.threads == TH_) \
         return lay.cl ? launch_impl<T, NP_, R_, TH_, true>(kp, pl.blocks, st)   \

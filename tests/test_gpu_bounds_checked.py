@@ -1,8 +1,8 @@
 """The bounds-checked build (libmamba_scan_checked.so, MSCAN_BOUNDS_CHECK).
 
 Its instrumented kernels -- the lane-split scan in every form that uses it,
-the decode step, the conv1d kernels -- test every global access against the
-byte range of its tensor.  On the shapes below (ragged groups and lengths,
+the static scan in its staging forms, the decode step, the conv1d kernels --
+test every global access against the byte range of its tensor.  On the shapes below (ragged groups and lengths,
 N < 16, both lane counts, two-phase pieces, the device-wide and block-local
 forms, the (b, l, d) layout, the fused conv1d with u written out,
 checkpoints, initial and final states) they must record no access outside a
@@ -118,6 +118,46 @@ def test_page_layout_and_fused_conv(checked, lanes):
     assert equal(ref, got)
 
 
+def _channels_last(t):
+    return t.transpose(1, 2).contiguous().transpose(1, 2)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("case", ["dense", "dense-N40", "unaligned", "channels-last", "mixed-broadcast-B",
+                                  "odd-strides"])
+def test_static_scan(checked, dtype, case):
+    """The static kernel in its staging forms: 16-byte copies along time or
+    along channels, B / C along time or along states, element copies."""
+    b, d, L, N = (2, 40, 333, 40) if case == "dense-N40" else (2, 40, 333, 16)
+    cpu = inputs.scan_inputs(inputs.custom(b, d, L, N, dtype, seed=L + N))
+    dev = {k: (None if v is None else v.cuda()) for k, v in cpu.items()}
+    kw = dict(schedule=binding.SCHEDULE_STATIC)
+    if case == "unaligned":  # u one element off its 16-byte grid: element copies
+        buf = torch.empty(dev["u"].numel() + 1, device="cuda", dtype=dev["u"].dtype)
+        dev["u"] = buf[1:].view(dev["u"].shape)
+        dev["u"].copy_(cpu["u"].cuda())
+    if case == "channels-last":
+        dev = {k: (_channels_last(v) if k in ("u", "delta", "z", "B", "C") else v) for k, v in dev.items()}
+    if case == "mixed-broadcast-B":
+        dev["u"] = _channels_last(dev["u"])
+        dev["B"] = dev["B"][:1].expand(b, N, L)
+        dev["C"] = _channels_last(dev["C"])
+    if case == "odd-strides":  # every 3rd element of a wider buffer along time
+        wide = torch.zeros(b, d, 3 * L, device="cuda", dtype=dev["delta"].dtype)
+        wide[..., ::3] = dev["delta"]
+        dev["delta"] = wide[..., ::3]
+    if case.startswith("dense"):
+        run = lambda: binding.mamba_scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],  # noqa: E731
+                                             z=dev["z"], delta_bias=dev["delta_bias"], return_last_state=True,
+                                             **kw)
+    else:
+        run = lambda: binding.mamba_scan_fwd_strided(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"],  # noqa: E731
+                                                     D=dev["D"], z=dev["z"], delta_bias=dev["delta_bias"],
+                                                     return_last_state=True, **kw)
+    ref, got = both(checked, run)
+    assert equal(ref, got)
+
+
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 @pytest.mark.parametrize("dstate", [16, 13, 8])
 def test_decode_step(checked, dtype, dstate):
@@ -200,6 +240,17 @@ def test_a_short_output_range_is_reported_and_its_store_skipped(checked):
         return out
 
     ref, got = _shrunk(checked, step, lambda o: o, 2)
+    assert torch.equal(got.reshape(-1)[:-1], ref.reshape(-1)[:-1]) and got.reshape(-1)[-1] == 7.0
+
+    def static_scan():  # the static kernel, its scalar stores (L not a whole number of vectors)
+        ins2 = inputs.scan_inputs(inputs.custom(2, 40, 333, 16, "fp32", seed=40), device="cuda")
+        out = torch.full_like(ins2["u"], 7.0)
+        binding.mamba_scan_fwd(ins2["u"], ins2["delta"], ins2["A"], ins2["B"], ins2["C"], D=ins2["D"],
+                               z=ins2["z"], delta_bias=ins2["delta_bias"], out=out,
+                               schedule=binding.SCHEDULE_STATIC)
+        return out
+
+    ref, got = _shrunk(checked, static_scan, lambda o: o, 4)
     assert torch.equal(got.reshape(-1)[:-1], ref.reshape(-1)[:-1]) and got.reshape(-1)[-1] == 7.0
 
     ci = inputs.conv_inputs(2, 32, 256, 4, "bf16", seed=39, device="cuda")
