@@ -494,19 +494,22 @@ int mamba_debug_stall_group(int group);
  * lane-split scan kernel (mamba_scan_fwd, _ws, _noalloc, _init, _conv,
  * _ckpt, the (batch, L, dim) layout of mamba_scan_fwd_strided), of the static
  * scan kernel (any layout of mamba_scan_fwd_strided, small problems of
- * mamba_scan_fwd), of the decode step (mamba_state_update) and of the conv1d
+ * mamba_scan_fwd), of the complex mode, of the backward (mamba_scan_bwd,
+ * _init, _ckpt), of the decode step (mamba_state_update) and of the conv1d
  * kernels (mamba_conv1d_fwd, mamba_conv1d_update) carries the byte range of
- * every pointer argument,
+ * every pointer argument and workspace part,
  * computed from the sizes given; each global access first checks that it
  * stays inside its range.  One that would not is skipped (a load reads
  * zeros, a store is dropped) and the first such access is recorded: its site
  * (the tensor: 1 A, 2 delta_bias, 3 D, 4 conv weight, 5 conv bias, 6 u / x,
  * 7 delta, 8 z, 9 B, 10 C, 11 conv input before a piece, 12 u written by the
  * fused conv, 13 out, 14 last_state, 15 h0, 16 checkpoints, 17 workspace
- * carries, 18 decode state, 19 conv1d input, 20 conv1d state) and its byte
- * offset from the tensor's start.  Nothing traps.  The one-lane, complex and
- * backward kernels are not instrumented.  In the normal build the checks
- * compile away.
+ * carries, 18 decode state, 19 conv1d input, 20 conv1d state; the backward
+ * reports dout and du / ddelta / dz as 13, dlast as 14, dA / dD / dbias as
+ * 1 / 3 / 2, dB / dC as 9 / 10 and its workspace parts as 16 and 17) and its
+ * byte offset from the tensor's start.  Nothing traps.  The one-lane kernel
+ * (lanes_per_channel = 1 on request) is not instrumented.  In the normal build
+ * the checks compile away.
  *
  * mamba_bounds_checked: 1 in the bounds-checked build, 0 otherwise.
  * mamba_debug_bounds_status: 1 with the first recorded violation (site and

@@ -2,15 +2,16 @@
 //
 // Every kernel launch carries, for each pointer argument, the byte range it
 // may touch (an Extent, filled on the host from the sizes the caller passed).
-// In the checked build each global access of the lane-split and static scan
-// kernels, the decode step and the conv1d kernels first asks within(): an
-// access that would leave its range is skipped -- a load reads zeros, a store
+// In the checked build each global access of the lane-split, static and
+// complex scan kernels, the backward, the decode step and the conv1d kernels
+// first asks MSCAN_WITHIN(): an access that would leave its range is skipped -- a load reads zeros, a store
 // is dropped -- and the first such access of the launch is recorded (site and
 // byte offset) in a word of its translation unit, which the host reads
 // through mamba_get_device_status / mamba_debug_bounds_status.  Nothing traps
-// or faults.  In the normal build within() is a constant true and the checks
-// compile away.  The one-lane, complex and backward kernels are not
-// instrumented.
+// or faults.  In the normal build MSCAN_WITHIN() is the constant true, its
+// arguments are not compiled, and the launch parameters carry no ranges
+// (MSCAN_EXTENTS declares them in the checked build only).  The one-lane
+// kernel is not instrumented.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -55,6 +56,9 @@ __device__ __forceinline__ bool within(const Extent &e, const void *p, unsigned 
     return false;
 }
 
+#define MSCAN_WITHIN(e, q, n, site) ::mscan::within((e), (q), (n), (site))
+#define MSCAN_EXTENTS(...) Extent __VA_ARGS__;
+
 // Host: this translation unit's record (1 = a violation, with its site and
 // offset), cleared; -1 when the words cannot be read.
 #define MSCAN_BOUNDS_TAKE(fn)                                                                     \
@@ -69,8 +73,12 @@ __device__ __forceinline__ bool within(const Extent &e, const void *p, unsigned 
         return 1;                                                                                 \
     }
 #else
+// The normal build: no ranges in the launch parameters (their layout, and so
+// the kernels' register allocation, stays exactly as without the checks) and
+// no checks -- the macro arguments are not even compiled.
 constexpr bool kBoundsChecked = false;
-__device__ __forceinline__ constexpr bool within(const Extent &, const void *, unsigned, int) { return true; }
+#define MSCAN_WITHIN(e, q, n, site) true
+#define MSCAN_EXTENTS(...)
 #define MSCAN_BOUNDS_TAKE(fn) \
     int fn(int *, long long *) { return 0; }
 #endif

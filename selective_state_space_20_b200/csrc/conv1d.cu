@@ -34,7 +34,7 @@ struct ConvParams {
     void *out;
     int64_t batch, dim, seqlen, x_batch_stride;
     int width, silu;
-    Extent x_x, x_w, x_bias, x_out;  // byte ranges, for the bounds-checked build
+    MSCAN_EXTENTS(x_x, x_w, x_bias, x_out)  // byte ranges, for the bounds-checked build
 };
 
 template <typename T>
@@ -42,13 +42,18 @@ __device__ __forceinline__ float load_elem(const T *p) { return Elem<T>::load(p)
 
 // Loads and stores that the bounds-checked build tests against the tensor's
 // range (a load outside reads zero, a store outside is dropped).
+#ifdef MSCAN_BOUNDS_CHECK
 template <typename T>
 __device__ __forceinline__ float load_chk(const Extent &e, const T *q, int site) {
-    return within(e, q, sizeof(T), site) ? Elem<T>::load(q) : 0.f;
+    return MSCAN_WITHIN(e, q, sizeof(T), site) ? Elem<T>::load(q) : 0.f;
 }
 __device__ __forceinline__ float ldg_chk(const Extent &e, const float *q, int site) {
-    return within(e, q, 4, site) ? __ldg(q) : 0.f;
+    return MSCAN_WITHIN(e, q, 4, site) ? __ldg(q) : 0.f;
 }
+#else
+#define load_chk(e, q, site) load_elem(q)
+#define ldg_chk(e, q, site) __ldg(q)
+#endif
 
 // One warp per NT consecutive 32-chunk tiles of one row: every lane issues
 // its NT 16-byte loads first (NT x 512 bytes in flight per warp), then the
@@ -75,7 +80,7 @@ __global__ void __launch_bounds__(256) conv1d_tiles_kernel(const ConvParams p) {
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
         const int64_t t0 = span0 + j * TILE + (int64_t)lane * V;
-        raw[j] = (t0 < p.seqlen && within(p.x_x, xr + t0, 16, kSiteX)) ? ldg16_stream(xr + t0)
+        raw[j] = (t0 < p.seqlen && MSCAN_WITHIN(p.x_x, xr + t0, 16, kSiteX)) ? ldg16_stream(xr + t0)
                                                                      : make_uint4(0u, 0u, 0u, 0u);
     }
     float carry[K];  // lane 0: the K-1 inputs before the span
@@ -112,7 +117,7 @@ __global__ void __launch_bounds__(256) conv1d_tiles_kernel(const ConvParams p) {
                 o[i] = v.x;
                 o[i + 1] = v.y;
             }
-            if (within(p.x_out, orow + t0, 16, kSiteOut)) stg16_stream(orow + t0, Elem<T>::pack(o));
+            if (MSCAN_WITHIN(p.x_out, orow + t0, 16, kSiteOut)) stg16_stream(orow + t0, Elem<T>::pack(o));
         }
     }
 }
@@ -131,7 +136,7 @@ __global__ void __launch_bounds__(256) conv1d_scalar_kernel(const ConvParams p) 
         if (s >= 0) v = fmaf(ldg_chk(p.x_w, p.w + d * p.width + k, kSiteConvW), load_chk(p.x_x, xr + s, kSiteX), v);
     }
     T *o = static_cast<T *>(p.out) + i;
-    if (within(p.x_out, o, sizeof(T), kSiteOut)) Elem<T>::store(o, p.silu ? silu_f(v) : v);
+    if (MSCAN_WITHIN(p.x_out, o, sizeof(T), kSiteOut)) Elem<T>::store(o, p.silu ? silu_f(v) : v);
 }
 
 struct ConvUpdateParams {
@@ -141,7 +146,7 @@ struct ConvUpdateParams {
     void *out;
     int64_t batch, dim, x_batch_stride;
     int width, silu;
-    Extent x_state, x_x, x_w, x_bias, x_out;  // byte ranges, for the bounds-checked build
+    MSCAN_EXTENTS(x_state, x_x, x_w, x_bias, x_out)  // byte ranges, for the bounds-checked build
 };
 
 // One thread per (batch, channel): read the K-1 kept inputs and the token,
@@ -155,16 +160,16 @@ __global__ void __launch_bounds__(256) conv1d_update_kernel(const ConvUpdatePara
     float *st = p.state + row * S;
     float in[K];
 #pragma unroll
-    for (int k = 0; k < S; ++k) in[k] = within(p.x_state, st + k, 4, kSiteConvState) ? st[k] : 0.f;
+    for (int k = 0; k < S; ++k) in[k] = MSCAN_WITHIN(p.x_state, st + k, 4, kSiteConvState) ? st[k] : 0.f;
     in[S] = load_chk(p.x_x, static_cast<const T *>(p.x) + b * p.x_batch_stride + d, kSiteX);
     float v = p.bias ? ldg_chk(p.x_bias, p.bias + d, kSiteConvB) : 0.f;
 #pragma unroll
     for (int k = 0; k < K; ++k) v = fmaf(ldg_chk(p.x_w, p.w + d * K + k, kSiteConvW), in[k], v);
     T *o = static_cast<T *>(p.out) + row;
-    if (within(p.x_out, o, sizeof(T), kSiteOut)) Elem<T>::store(o, p.silu ? silu_f(v) : v);
+    if (MSCAN_WITHIN(p.x_out, o, sizeof(T), kSiteOut)) Elem<T>::store(o, p.silu ? silu_f(v) : v);
 #pragma unroll
     for (int k = 0; k < S; ++k)
-        if (within(p.x_state, st + k, 4, kSiteConvState)) st[k] = in[k + 1];
+        if (MSCAN_WITHIN(p.x_state, st + k, 4, kSiteConvState)) st[k] = in[k + 1];
 }
 
 template <typename T, int NT, bool SILU>
@@ -223,6 +228,7 @@ cudaError_t launch_conv1d_fwd(const Conv1dArgs &a, cudaStream_t st) {
     p.x = a.x; p.w = a.weight; p.bias = a.bias; p.out = a.out;
     p.batch = a.batch; p.dim = a.dim; p.seqlen = a.seqlen; p.x_batch_stride = a.x_batch_stride;
     p.width = a.width; p.silu = a.silu;
+#ifdef MSCAN_BOUNDS_CHECK
     const unsigned long long es = a.act == kBF16 ? 2 : 4;
     const unsigned long long row = (unsigned long long)(a.dim * a.seqlen) * es;
     const unsigned long long ob = (unsigned long long)a.batch * row;
@@ -230,6 +236,7 @@ cudaError_t launch_conv1d_fwd(const Conv1dArgs &a, cudaStream_t st) {
     p.x_w = extent_of(a.weight, (unsigned long long)(a.dim * a.width) * 4);
     p.x_bias = extent_of(a.bias, (unsigned long long)a.dim * 4);
     p.x_out = extent_of(a.out, ob > (unsigned long long)g_out_extent_shrink ? ob - g_out_extent_shrink : 0);
+#endif
     return a.act == kBF16 ? launch_fwd_typed<__nv_bfloat16>(p, st) : launch_fwd_typed<float>(p, st);
 }
 
@@ -238,12 +245,14 @@ cudaError_t launch_conv1d_update(const Conv1dUpdateArgs &a, cudaStream_t st) {
     p.state = a.state; p.x = a.x; p.w = a.weight; p.bias = a.bias; p.out = a.out;
     p.batch = a.batch; p.dim = a.dim; p.x_batch_stride = a.x_batch_stride;
     p.width = a.width; p.silu = a.silu;
+#ifdef MSCAN_BOUNDS_CHECK
     const unsigned long long es = a.act == kBF16 ? 2 : 4, rows = (unsigned long long)(a.batch * a.dim);
     p.x_state = extent_of(a.state, rows * (a.width - 1) * 4);
     p.x_x = extent_of(a.x, (unsigned long long)(a.batch - 1) * a.x_batch_stride * es + (unsigned long long)a.dim * es);
     p.x_w = extent_of(a.weight, (unsigned long long)(a.dim * a.width) * 4);
     p.x_bias = extent_of(a.bias, (unsigned long long)a.dim * 4);
     p.x_out = extent_of(a.out, rows * es > (unsigned long long)g_out_extent_shrink ? rows * es - g_out_extent_shrink : 0);
+#endif
     const int threads = 256;
     const int64_t blocks = (a.batch * a.dim + threads - 1) / threads;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;

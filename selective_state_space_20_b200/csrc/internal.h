@@ -18,6 +18,8 @@ extern int g_out_extent_shrink;
 // a read error.  Always 0 in the normal build.
 int pairs_bounds_take(int *site, long long *off);
 int static_bounds_take(int *site, long long *off);
+int complex_bounds_take(int *site, long long *off);
+int bwd_bounds_take(int *site, long long *off);
 int state_update_bounds_take(int *site, long long *off);
 int conv1d_bounds_take(int *site, long long *off);
 

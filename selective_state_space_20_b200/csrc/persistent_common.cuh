@@ -63,8 +63,8 @@ struct Params {
     // and B / C as (batch, L, N), all dense (else (batch, dim, L) / (batch, N, L))
     int channels_last;
     // byte ranges of the pointer arguments, for the bounds-checked build
-    Extent x_u, x_delta, x_z, x_B, x_C, x_A, x_D, x_bias, x_out, x_last, x_h0, x_conv_w, x_conv_b, x_u_out,
-        x_ckpt, x_carry;
+    MSCAN_EXTENTS(x_u, x_delta, x_z, x_B, x_C, x_A, x_D, x_bias, x_out, x_last, x_h0, x_conv_w, x_conv_b, x_u_out,
+                  x_ckpt, x_carry)
 };
 
 __device__ __forceinline__ void cp16(void *smem, const void *gmem, bool pred) {

@@ -174,6 +174,7 @@ persist::Params base_params(const ScanArgs &a, int lanes, int tc) {
     kp.ckpt_gpb = (int)((a.dim + 31) / 32);
     kp.ckpt_nsup = (int)((a.seqlen + 31) / 32);
     kp.channels_last = a.channels_last ? 1 : 0;
+#ifdef MSCAN_BOUNDS_CHECK
     // byte ranges of the pointer arguments (checked in the bounds-checked build)
     const unsigned long long es = a.act == kBF16 ? 2 : 4;
     const unsigned long long x = (unsigned long long)(a.batch * a.dim * a.seqlen) * es;
@@ -196,6 +197,7 @@ persist::Params base_params(const ScanArgs &a, int lanes, int tc) {
     kp.x_u_out = extent_of(a.u_out, x);
     kp.x_ckpt = extent_of(a.ckpt, (unsigned long long)a.batch * kp.ckpt_gpb * kp.ckpt_nsup * 32 * 16 * 4);
     kp.x_carry = extent_of(nullptr, 0);
+#endif
     return kp;
 }
 }  // namespace
@@ -263,7 +265,9 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
         kp.queue = nullptr;
         kp.progress = reinterpret_cast<unsigned *>(w + l.queue_off);
         kp.carry = reinterpret_cast<float *>(w + l.carry_off);
+#ifdef MSCAN_BOUNDS_CHECK
         kp.x_carry = extent_of(kp.carry, l.bytes - l.carry_off);
+#endif
         cudaError_t e = cudaMemsetAsync(w, 0, l.queue_off + (size_t)groups * 4, st);
         if (e != cudaSuccess) return e;
         return launch_persistent_split(kp, lanes, a.act, sm_count, st);

@@ -50,6 +50,7 @@
 
 #include <type_traits>
 
+#include "bounds.cuh"
 #include "device_math.cuh"
 #include "internal.h"
 
@@ -105,6 +106,11 @@ struct BwdParams {
     int64_t batch, dim, seqlen;
     int dstate, softplus;
     int groups_per_batch, n_groups, n_sup;
+    // byte ranges of the pointer arguments and workspace parts, for the
+    // bounds-checked build (indexed by the fetch's row kind: u, delta, dout,
+    // z, then B, C)
+    MSCAN_EXTENTS(x_in[6], x_A, x_D, x_bias, x_dlast, x_h0, x_dout3[3], x_dA, x_dB, x_dC, x_dD, x_dbias, x_dh0,
+                  x_ckpt, x_subck, x_rep)
 };
 
 __device__ __forceinline__ void cp16_async(void *smem, const void *gmem, bool pred) {
@@ -189,10 +195,10 @@ scan_bwd_kernel(const BwdParams p) {
 #pragma unroll
         for (int i = 0; i < kSPL; ++i) {
             const int n = kSPL * r + i;
-            Ar[i] = (valid && n < N) ? __ldg(p.A + dc * N + n) : 0.f;
+            Ar[i] = (valid && n < N && MSCAN_WITHIN(p.x_A, p.A + dc * N + n, 4, kSiteA)) ? __ldg(p.A + dc * N + n) : 0.f;
             A2[i] = Ar[i] * Dk::kScale;
         }
-        const float Dd = (valid && p.D) ? __ldg(p.D + dc) : 0.f;
+        const float Dd = (valid && p.D && MSCAN_WITHIN(p.x_D, p.D + dc, 4, kSiteD)) ? __ldg(p.D + dc) : 0.f;
         // this lane's checkpoints (the forward's layout: 32-channel groups): + s * 32 * 16
         float *ck = p.ckpt + ((b * p.ckpt_g32 + dc / kCkCh) * (int64_t)p.n_sup) * kCkCh * kNS + (dc % kCkCh) * kNS +
                     kSPL * r;
@@ -220,12 +226,19 @@ scan_bwd_kernel(const BwdParams p) {
                     ok = (rr & 15) < N;
                 }
                 T *dst = raw + row * RP + cp * V;
+#ifdef MSCAN_BOUNDS_CHECK
+                const int kind = q < 4 ? q : (rr < kNS ? 4 : 5);
+                const int site = kind == 0 ? kSiteU : kind == 1 ? kSiteDelta : kind == 2 ? kSiteOut
+                               : kind == 3 ? kSiteZ : kind == 4 ? kSiteB : kSiteC;
+#endif
                 if (p.vec) {
-                    const bool in = ok && cp * V < tn;
+                    const bool in = ok && cp * V < tn && MSCAN_WITHIN(p.x_in[kind], src + t0 + cp * V, 16, site);
                     cp16_async(dst, in ? src + t0 + cp * V : src, in);
                 } else {
 #pragma unroll
-                    for (int e = 0; e < V; ++e) dst[e] = (ok && cp * V + e < tn) ? src[t0 + cp * V + e] : T(0.f);
+                    for (int e = 0; e < V; ++e)
+                        dst[e] = (ok && cp * V + e < tn && MSCAN_WITHIN(p.x_in[kind], src + t0 + cp * V + e, sizeof(T), site))
+                                     ? src[t0 + cp * V + e] : T(0.f);
                 }
             }
             asm volatile("cp.async.commit_group;" ::: "memory");
@@ -240,7 +253,8 @@ scan_bwd_kernel(const BwdParams p) {
             const int64_t t0 = (int64_t)s * kSup;
             const int tn = (L - t0) < kSup ? (int)(L - t0) : kSup;
             const int cc = tid % kCh;
-            const float bias = (d0 + cc < Dm && p.delta_bias) ? __ldg(p.delta_bias + d0 + cc) : 0.f;
+            const float bias = (d0 + cc < Dm && p.delta_bias && MSCAN_WITHIN(p.x_bias, p.delta_bias + d0 + cc, 4, kSiteBias))
+                                   ? __ldg(p.delta_bias + d0 + cc) : 0.f;
             for (int piece = tid / kCh; piece < CPR; piece += (kWarpsBwd * 32) / kCh) {
                 float fu[V], fd[V], fo[V], fz[V];
                 Elem<T>::unpack(*reinterpret_cast<const uint4 *>(raw + cc * RP + piece * V), fu);
@@ -312,11 +326,12 @@ scan_bwd_kernel(const BwdParams p) {
 #pragma unroll
             for (int i = 0; i < kSPL; ++i) {
                 const int n = kSPL * r + i;
-                h[i] = (valid && p.h0 && n < N) ? (HS)__ldg(p.h0 + (b * Dm + dc) * N + n) : (HS)0.f;
+                h[i] = (valid && p.h0 && n < N && MSCAN_WITHIN(p.x_h0, p.h0 + (b * Dm + dc) * N + n, 4, kSiteH0))
+                           ? (HS)__ldg(p.h0 + (b * Dm + dc) * N + n) : (HS)0.f;
             }
             fetch(0, false);
             for (int s = 0; s < p.n_sup; ++s) {
-                if (valid)
+                if (valid && MSCAN_WITHIN(p.x_ckpt, ck + (int64_t)s * kCkCh * kNS, 16, kSiteCkpt))
                     __stcg(reinterpret_cast<float4 *>(ck + (int64_t)s * kCkCh * kNS),
                            make_float4((float)h[0], (float)h[1], (float)h[2], (float)h[3]));
                 asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -338,7 +353,8 @@ scan_bwd_kernel(const BwdParams p) {
 #pragma unroll
         for (int i = 0; i < kSPL; ++i) {
             const int n = kSPL * r + i;
-            g[i] = (valid && p.dlast && n < N) ? (HS)p.dlast[(b * Dm + dc) * N + n] : (HS)0.f;
+            g[i] = (valid && p.dlast && n < N && MSCAN_WITHIN(p.x_dlast, p.dlast + (b * Dm + dc) * N + n, 4, kSiteLastState))
+                       ? (HS)p.dlast[(b * Dm + dc) * N + n] : (HS)0.f;
             dA_acc[i] = 0.f;
         }
         HS dD_acc = 0.f, dbias_acc = 0.f;
@@ -358,12 +374,15 @@ scan_bwd_kernel(const BwdParams p) {
             // recompute the segment from its checkpoint, one sub-checkpoint every kSub steps
             {
                 // (channels past dim have no checkpoint of the forward's: zeros)
-                const float4 v = valid ? __ldcg(reinterpret_cast<const float4 *>(ck + (int64_t)s * kCkCh * kNS))
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 v = (valid && MSCAN_WITHIN(p.x_ckpt, ck + (int64_t)s * kCkCh * kNS, 16, kSiteCkpt))
+                                     ? __ldcg(reinterpret_cast<const float4 *>(ck + (int64_t)s * kCkCh * kNS))
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
                 HS h[kSPL] = {(HS)v.x, (HS)v.y, (HS)v.z, (HS)v.w};
                 for (int j = 0; j * kSub < tn; ++j) {
 #pragma unroll
-                    for (int i = 0; i < kSPL; ++i) sub[j * (kWarpsBwd * 32) * kSPL + i] = h[i];
+                    for (int i = 0; i < kSPL; ++i)
+                        if (MSCAN_WITHIN(p.x_subck, sub + j * (kWarpsBwd * 32) * kSPL + i, sizeof(HS), kSiteCarry))
+                            sub[j * (kWarpsBwd * 32) * kSPL + i] = h[i];
 #pragma unroll
                     for (int w = 0; w < kSub; ++w) step(h, j * kSub + w);
                 }
@@ -378,7 +397,9 @@ scan_bwd_kernel(const BwdParams p) {
                 // activations, so the adjoint decays with the state's accuracy
                 float ab[kSub][kSPL];
 #pragma unroll
-                for (int i = 0; i < kSPL; ++i) hin[i] = sub[j * (kWarpsBwd * 32) * kSPL + i];
+                for (int i = 0; i < kSPL; ++i)
+                    hin[i] = MSCAN_WITHIN(p.x_subck, sub + j * (kWarpsBwd * 32) * kSPL + i, sizeof(HS), kSiteCarry)
+                                 ? sub[j * (kWarpsBwd * 32) * kSPL + i] : (HS)0.f;
 #pragma unroll
                 for (int w = 0; w < kSub; ++w) {
                     {
@@ -489,8 +510,9 @@ scan_bwd_kernel(const BwdParams p) {
                         float acc = 0.f;
 #pragma unroll
                         for (int k = 0; k < kWarpsBwd; ++k) acc += rb[(w * kWarpsBwd + k) * 32 + slot];
-                        atomicAdd(p.rep + (((grp % kRep) * 2 + (slot >> 4)) * p.batch + b) * (int64_t)kNS * L +
-                                      (int64_t)n * L + t0 + tb + w, acc);
+                        float *dst = p.rep + (((grp % kRep) * 2 + (slot >> 4)) * p.batch + b) * (int64_t)kNS * L +
+                                     (int64_t)n * L + t0 + tb + w;
+                        if (MSCAN_WITHIN(p.x_rep, dst, 4, kSiteCarry)) atomicAdd(dst, acc);
                     }
                 }
                 rbuf ^= 1;  // the next window fills the other buffer while this one is read
@@ -505,11 +527,12 @@ scan_bwd_kernel(const BwdParams p) {
                 T *dst = gdst[q] + (b * Dm + d0 + cc) * L + t0 + cp * V;
                 const T *srcp = outs + (q * kCh + cc) * RP + cp * V;
                 if (p.vec) {
-                    if (cp * V < tn) *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(srcp);
+                    if (cp * V < tn && MSCAN_WITHIN(p.x_dout3[q], dst, 16, kSiteOut))
+                        *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(srcp);
                 } else {
 #pragma unroll
                     for (int e = 0; e < V; ++e)
-                        if (cp * V + e < tn) dst[e] = srcp[e];
+                        if (cp * V + e < tn && MSCAN_WITHIN(p.x_dout3[q], dst + e, sizeof(T), kSiteOut)) dst[e] = srcp[e];
                 }
             }
         }
@@ -518,13 +541,14 @@ scan_bwd_kernel(const BwdParams p) {
             for (int i = 0; i < kSPL; ++i) {
                 const int n = kSPL * r + i;
                 if (n < N) {
-                    atomicAdd(p.dA + dc * N + n, (float)dA_acc[i]);
-                    if (p.dh0) p.dh0[(b * Dm + dc) * N + n] = (float)g[i];  // dL/dh_{-1}
+                    if (MSCAN_WITHIN(p.x_dA, p.dA + dc * N + n, 4, kSiteA)) atomicAdd(p.dA + dc * N + n, (float)dA_acc[i]);
+                    if (p.dh0 && MSCAN_WITHIN(p.x_dh0, p.dh0 + (b * Dm + dc) * N + n, 4, kSiteH0))
+                        p.dh0[(b * Dm + dc) * N + n] = (float)g[i];  // dL/dh_{-1}
                 }
             }
             if (r == 0) {
-                if (p.dD) atomicAdd(p.dD + dc, (float)dD_acc);
-                if (p.dbias) atomicAdd(p.dbias + dc, (float)dbias_acc);
+                if (p.dD && MSCAN_WITHIN(p.x_dD, p.dD + dc, 4, kSiteD)) atomicAdd(p.dD + dc, (float)dD_acc);
+                if (p.dbias && MSCAN_WITHIN(p.x_dbias, p.dbias + dc, 4, kSiteBias)) atomicAdd(p.dbias + dc, (float)dbias_acc);
             }
         }
         __syncthreads();  // before the next group reuses shared memory
@@ -548,8 +572,11 @@ __global__ void __launch_bounds__(256) bwd_sum_copies_kernel(const BwdParams p) 
         if (t >= L) break;
         float acc = 0.f;
 #pragma unroll
-        for (int k = 0; k < kRep; ++k) acc += __ldcg(p.rep + ((k * 2 + which) * p.batch + b) * (int64_t)kNS * L + n * L + t);
-        dst[t] = acc;
+        for (int k = 0; k < kRep; ++k) {
+            const float *q = p.rep + ((k * 2 + which) * p.batch + b) * (int64_t)kNS * L + n * L + t;
+            acc += MSCAN_WITHIN(p.x_rep, q, 4, kSiteCarry) ? __ldcg(q) : 0.f;
+        }
+        if (MSCAN_WITHIN(which ? p.x_dC : p.x_dB, dst + t, 4, which ? kSiteC : kSiteB)) dst[t] = acc;
     }
 }
 
@@ -630,6 +657,8 @@ BwdLayout bwd_layout(int64_t batch, int64_t dim, int64_t seqlen) {
 }
 }  // namespace
 
+MSCAN_BOUNDS_TAKE(bwd_bounds_take)
+
 size_t scan_bwd_workspace_bytes(int64_t batch, int64_t dim, int64_t seqlen) {
     return bwd_layout(batch, dim, seqlen).bytes;
 }
@@ -660,6 +689,38 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs &a, void *workspace, const float *
     p.ckpt_g32 = (int)((a.dim + kCkCh - 1) / kCkCh);
     p.n_groups = (int)(a.batch * p.groups_per_batch);
     p.n_sup = (int)((a.seqlen + kSup - 1) / kSup);
+#ifdef MSCAN_BOUNDS_CHECK
+    {  // byte ranges (bounds-checked build)
+        const unsigned long long es = a.act == kBF16 ? 2 : 4;
+        const unsigned long long x = (unsigned long long)(a.batch * a.dim * a.seqlen) * es;
+        const unsigned long long bc = (unsigned long long)(a.batch * a.dstate * a.seqlen) * es;
+        const unsigned long long stb = (unsigned long long)(a.batch * a.dim * a.dstate) * 4;
+        const unsigned long long ob = x > (unsigned long long)g_out_extent_shrink ? x - g_out_extent_shrink : 0;
+        p.x_in[0] = extent_of(a.u, x);
+        p.x_in[1] = extent_of(a.delta, x);
+        p.x_in[2] = extent_of(a.dout, x);
+        p.x_in[3] = extent_of(a.z, x);
+        p.x_in[4] = extent_of(a.B, bc);
+        p.x_in[5] = extent_of(a.C, bc);
+        p.x_A = extent_of(a.A, (unsigned long long)(a.dim * a.dstate) * 4);
+        p.x_D = extent_of(a.D, (unsigned long long)a.dim * 4);
+        p.x_bias = extent_of(a.delta_bias, (unsigned long long)a.dim * 4);
+        p.x_dlast = extent_of(a.dlast, stb);
+        p.x_h0 = extent_of(a.h0, stb);
+        p.x_dout3[0] = extent_of(a.du, ob);
+        p.x_dout3[1] = extent_of(a.ddelta, ob);
+        p.x_dout3[2] = extent_of(a.dz, ob);
+        p.x_dA = extent_of(a.dA, (unsigned long long)(a.dim * a.dstate) * 4);
+        p.x_dB = extent_of(a.dB, (unsigned long long)(a.batch * a.dstate * a.seqlen) * 4);
+        p.x_dC = extent_of(a.dC, (unsigned long long)(a.batch * a.dstate * a.seqlen) * 4);
+        p.x_dD = extent_of(a.dD, (unsigned long long)a.dim * 4);
+        p.x_dbias = extent_of(a.ddelta_bias, (unsigned long long)a.dim * 4);
+        p.x_dh0 = extent_of(a.dh0, stb);
+        p.x_ckpt = extent_of(p.ckpt, (unsigned long long)scan_bwd_ckpt_floats(a.batch, a.dim, a.seqlen) * 4);
+        p.x_subck = extent_of(p.subck, l.rep - l.sub);
+        p.x_rep = extent_of(p.rep, l.bytes - l.rep);
+    }
+#endif
     // every sum over channels, time or batch rows accumulates into zeroed outputs
     cudaError_t e = cudaMemsetAsync(a.dA, 0, (size_t)(a.dim * a.dstate) * 4, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(p.rep, 0, l.bytes - l.rep, st);

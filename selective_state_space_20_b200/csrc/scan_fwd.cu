@@ -66,7 +66,7 @@ struct KParams {
     int vec;           // u / delta / z / out: 16-byte vectors along the kernel's contiguous axis
     int bc_mode;       // B / C: 0 element copies, 1 vectors along time, 2 vectors along states
     // byte ranges of the pointer arguments, for the bounds-checked build
-    Extent x_u, x_delta, x_z, x_B, x_C, x_A, x_D, x_bias, x_out, x_last, x_h0;
+    MSCAN_EXTENTS(x_u, x_delta, x_z, x_B, x_C, x_A, x_D, x_bias, x_out, x_last, x_h0)
 };
 
 // ------------------------------------------------------------ geometry
@@ -184,9 +184,9 @@ scan_fwd_kernel(const KParams p) {
 #pragma unroll
     for (int s = 0; s < S; ++s) {
         const int n = r * S + s;
-        A2[s] = (d < Dm && n < N && within(p.x_A, p.A + d * N + n, 4, kSiteA)) ? __ldg(p.A + d * N + n) * Dk::kScale
+        A2[s] = (d < Dm && n < N && MSCAN_WITHIN(p.x_A, p.A + d * N + n, 4, kSiteA)) ? __ldg(p.A + d * N + n) * Dk::kScale
                                                                                : 0.f;
-        h[s] = (p.h0 && d < Dm && n < N && within(p.x_h0, p.h0 + (b * Dm + d) * N + n, 4, kSiteH0))
+        h[s] = (p.h0 && d < Dm && n < N && MSCAN_WITHIN(p.x_h0, p.h0 + (b * Dm + d) * N + n, 4, kSiteH0))
                    ? __ldcg(p.h0 + (b * Dm + d) * N + n) : 0.f;
     }
 
@@ -206,11 +206,11 @@ scan_fwd_kernel(const KParams p) {
                     const int64_t t = t0 + tv * V, dd = d0 + pc;
                     const bool ok = (dd < Dm) && (t < L);
                     const T *pu = gu + (ok ? b * su.b + dd * su.d + t : 0), *pd = gd + (ok ? b * sdl.b + dd * sdl.d + t : 0);
-                    cp_async16(rU + pc * TC + tv * V, pu, ok && within(p.x_u, pu, 16, kSiteU));
-                    cp_async16(rD + pc * TC + tv * V, pd, ok && within(p.x_delta, pd, 16, kSiteDelta));
+                    cp_async16(rU + pc * TC + tv * V, pu, ok && MSCAN_WITHIN(p.x_u, pu, 16, kSiteU));
+                    cp_async16(rD + pc * TC + tv * V, pd, ok && MSCAN_WITHIN(p.x_delta, pd, 16, kSiteDelta));
                     if (has_z) {
                         const T *pz = gz + (ok ? b * sz.b + dd * sz.d + t : 0);
-                        cp_async16(rZ + pc * TC + tv * V, pz, ok && within(p.x_z, pz, 16, kSiteZ));
+                        cp_async16(rZ + pc * TC + tv * V, pz, ok && MSCAN_WITHIN(p.x_z, pz, 16, kSiteZ));
                     }
                 }
             } else {
@@ -219,11 +219,11 @@ scan_fwd_kernel(const KParams p) {
                     const int64_t t = t0 + tt, dd = d0 + cv * V;
                     const bool ok = (dd < Dm) && (t < L);  // dim is a whole number of vectors
                     const T *pu = gu + (ok ? b * su.b + t * su.t + dd : 0), *pd = gd + (ok ? b * sdl.b + t * sdl.t + dd : 0);
-                    cp_async16(rU + tt * CG + cv * V, pu, ok && within(p.x_u, pu, 16, kSiteU));
-                    cp_async16(rD + tt * CG + cv * V, pd, ok && within(p.x_delta, pd, 16, kSiteDelta));
+                    cp_async16(rU + tt * CG + cv * V, pu, ok && MSCAN_WITHIN(p.x_u, pu, 16, kSiteU));
+                    cp_async16(rD + tt * CG + cv * V, pd, ok && MSCAN_WITHIN(p.x_delta, pd, 16, kSiteDelta));
                     if (has_z) {
                         const T *pz = gz + (ok ? b * sz.b + t * sz.t + dd : 0);
-                        cp_async16(rZ + tt * CG + cv * V, pz, ok && within(p.x_z, pz, 16, kSiteZ));
+                        cp_async16(rZ + tt * CG + cv * V, pz, ok && MSCAN_WITHIN(p.x_z, pz, 16, kSiteZ));
                     }
                 }
             }
@@ -234,11 +234,11 @@ scan_fwd_kernel(const KParams p) {
                 const int64_t t = t0 + tt, dd = d0 + pc;
                 const bool ok = (dd < Dm) && (t < L);
                 const T *pu = gu + b * su.b + dd * su.d + t * su.t, *pd = gd + b * sdl.b + dd * sdl.d + t * sdl.t;
-                rU[e] = (ok && within(p.x_u, pu, sizeof(T), kSiteU)) ? *pu : T(0.f);
-                rD[e] = (ok && within(p.x_delta, pd, sizeof(T), kSiteDelta)) ? *pd : T(0.f);
+                rU[e] = (ok && MSCAN_WITHIN(p.x_u, pu, sizeof(T), kSiteU)) ? *pu : T(0.f);
+                rD[e] = (ok && MSCAN_WITHIN(p.x_delta, pd, sizeof(T), kSiteDelta)) ? *pd : T(0.f);
                 if (has_z) {
                     const T *pz = gz + b * sz.b + dd * sz.d + t * sz.t;
-                    rZ[e] = (ok && within(p.x_z, pz, sizeof(T), kSiteZ)) ? *pz : T(0.f);
+                    rZ[e] = (ok && MSCAN_WITHIN(p.x_z, pz, sizeof(T), kSiteZ)) ? *pz : T(0.f);
                 }
             }
         }
@@ -252,7 +252,7 @@ scan_fwd_kernel(const KParams p) {
                 const int64_t off = ok ? b * sx.b + n * sx.d + t : 0;
                 const T *src = (which ? gC : gB) + off;
                 cp_async16((which ? rC : rB) + n * TC + tv * V, src,
-                           ok && within(which ? p.x_C : p.x_B, src, 16, which ? kSiteC : kSiteB));
+                           ok && MSCAN_WITHIN(which ? p.x_C : p.x_B, src, 16, which ? kSiteC : kSiteB));
             }
         } else if (p.bc_mode == 2) {
             for (int vi = tid; vi < 2 * TC * NVR; vi += THREADS) {
@@ -264,7 +264,7 @@ scan_fwd_kernel(const KParams p) {
                 const int64_t off = ok ? b * sx.b + t * sx.t + n : 0;
                 const T *src = (which ? gC : gB) + off;
                 cp_async16((which ? rC : rB) + tt * NP + n, src,
-                           ok && within(which ? p.x_C : p.x_B, src, 16, which ? kSiteC : kSiteB));
+                           ok && MSCAN_WITHIN(which ? p.x_C : p.x_B, src, 16, which ? kSiteC : kSiteB));
             }
         } else {
             for (int e = tid; e < 2 * NP * TC; e += THREADS) {
@@ -275,7 +275,7 @@ scan_fwd_kernel(const KParams p) {
                 const Stride3 &sx = which ? sCs : sBs;
                 const T *src = (which ? gC : gB) + b * sx.b + n * sx.d + t * sx.t;
                 (which ? rC : rB)[rem] =
-                    (ok && within(which ? p.x_C : p.x_B, src, sizeof(T), which ? kSiteC : kSiteB)) ? *src : T(0.f);
+                    (ok && MSCAN_WITHIN(which ? p.x_C : p.x_B, src, sizeof(T), which ? kSiteC : kSiteB)) ? *src : T(0.f);
             }
         }
         cp_async_commit();  // an empty group when everything was copied by hand
@@ -300,7 +300,7 @@ scan_fwd_kernel(const KParams p) {
         for (int vi = tid; vi < CH_VEC; vi += THREADS) {
             const int pc = CL ? vi % CG : vi / VPR, tv = CL ? vi / CG : vi % VPR;
             const int64_t dd = d0 + pc;
-            const float bias = (dd < Dm && p.delta_bias && within(p.x_bias, p.delta_bias + dd, 4, kSiteBias))
+            const float bias = (dd < Dm && p.delta_bias && MSCAN_WITHIN(p.x_bias, p.delta_bias + dd, 4, kSiteBias))
                                    ? __ldg(p.delta_bias + dd) : 0.f;
             float fu[V], fd[V];
             if (!CL) {
@@ -397,7 +397,7 @@ scan_fwd_kernel(const KParams p) {
                 const int64_t dd = d0 + pc;
                 const int64_t t = t0 + tv * V;
                 if (dd >= Dm || tv * V >= tvalid) continue;
-                const float Dd = (p.D && within(p.x_D, p.D + dd, 4, kSiteD)) ? __ldg(p.D + dd) : 0.f;
+                const float Dd = (p.D && MSCAN_WITHIN(p.x_D, p.D + dd, 4, kSiteD)) ? __ldg(p.D + dd) : 0.f;
                 float fu[V], fz[V], y[V];
                 Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + pc * TC + tv * V), fu);
                 if (has_z) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rZ + pc * TC + tv * V), fz);
@@ -415,11 +415,11 @@ scan_fwd_kernel(const KParams p) {
                 }
                 T *dst = gout + b * so.b + dd * so.d + t * so.t;
                 if (p.vec) {
-                    if (within(p.x_out, dst, 16, kSiteOut)) stg16_stream(dst, Elem<T>::pack(y));
+                    if (MSCAN_WITHIN(p.x_out, dst, 16, kSiteOut)) stg16_stream(dst, Elem<T>::pack(y));
                 } else {
 #pragma unroll
                     for (int i = 0; i < V; ++i)
-                        if (tv * V + i < tvalid && within(p.x_out, dst + i * so.t, sizeof(T), kSiteOut))
+                        if (tv * V + i < tvalid && MSCAN_WITHIN(p.x_out, dst + i * so.t, sizeof(T), kSiteOut))
                             Elem<T>::store(dst + i * so.t, y[i]);
                 }
             }
@@ -434,7 +434,7 @@ scan_fwd_kernel(const KParams p) {
                 if (has_z) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rZ + tt * CG + cv * V), fz);
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
-                    const float Dd = (p.D && dd + i < Dm && within(p.x_D, p.D + dd + i, 4, kSiteD)) ? __ldg(p.D + dd + i)
+                    const float Dd = (p.D && dd + i < Dm && MSCAN_WITHIN(p.x_D, p.D + dd + i, 4, kSiteD)) ? __ldg(p.D + dd + i)
                                                                                                 : 0.f;
                     float o = fmaf(Dd, fu[i], sDelta[(cv * V + i) * TCP + tt]);
                     if (has_z) o *= silu_f(fz[i]);
@@ -442,11 +442,11 @@ scan_fwd_kernel(const KParams p) {
                 }
                 T *dst = gout + b * so.b + t * so.t + dd * so.d;
                 if (p.vec) {
-                    if (within(p.x_out, dst, 16, kSiteOut)) stg16_stream(dst, Elem<T>::pack(y));
+                    if (MSCAN_WITHIN(p.x_out, dst, 16, kSiteOut)) stg16_stream(dst, Elem<T>::pack(y));
                 } else {
 #pragma unroll
                     for (int i = 0; i < V; ++i)
-                        if (dd + i < Dm && within(p.x_out, dst + i * so.d, sizeof(T), kSiteOut))
+                        if (dd + i < Dm && MSCAN_WITHIN(p.x_out, dst + i * so.d, sizeof(T), kSiteOut))
                             Elem<T>::store(dst + i * so.d, y[i]);
                 }
             }
@@ -458,7 +458,7 @@ scan_fwd_kernel(const KParams p) {
 #pragma unroll
         for (int s = 0; s < S; ++s) {
             const int n = r * S + s;
-            if (n < N && within(p.x_last, ls + n, 4, kSiteLastState)) ls[n] = (float)h[s];
+            if (n < N && MSCAN_WITHIN(p.x_last, ls + n, 4, kSiteLastState)) ls[n] = (float)h[s];
         }
     }
 }
@@ -559,6 +559,7 @@ cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &pl, cudaStream_t 
     kp.dstate = a.dstate; kp.softplus = a.softplus;
     const StaticLayout lay = static_layout(a);
     kp.st = lay.st; kp.vec = lay.vec; kp.bc_mode = lay.bc_mode;
+#ifdef MSCAN_BOUNDS_CHECK
     // byte ranges (bounds-checked build): one past the last element of each strided tensor
     const unsigned long long es = a.act == kBF16 ? 2 : 4;
     auto span = [&](const void *q, const Stride3 &x, int64_t rows) {
@@ -579,6 +580,7 @@ cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &pl, cudaStream_t 
     kp.x_bias = extent_of(a.delta_bias, (unsigned long long)a.dim * 4);
     kp.x_last = extent_of(a.last_state, (unsigned long long)(a.batch * a.dim * a.dstate) * 4);
     kp.x_h0 = extent_of(a.h0, (unsigned long long)(a.batch * a.dim * a.dstate) * 4);
+#endif
 #define X(T, NP_, R_, TH_) \
     if (a.act == act_of<T>() && pl.padded_dstate == NP_ && pl.lanes == R_ && pl.threads == TH_) \
         return lay.cl ? launch_impl<T, NP_, R_, TH_, true>(kp, pl.blocks, st)   \

@@ -26,6 +26,7 @@
 
 #include <type_traits>
 
+#include "bounds.cuh"
 #include "device_math.cuh"
 #include "internal.h"
 
@@ -45,6 +46,8 @@ struct CParams {
     int64_t dim, seqlen;
     int n_groups;  // channel groups per batch row
     int dstate, softplus, vec;
+    // byte ranges of the pointer arguments, for the bounds-checked build
+    MSCAN_EXTENTS(x_u, x_delta, x_z, x_B, x_C, x_A, x_D, x_bias, x_out, x_last, x_h0)
 };
 
 // fp32 activations carry delta, delta * u, the states and the readout in
@@ -141,10 +144,12 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
     for (int s = 0; s < S; ++s) {
         const int n = r * S + s;
         const bool ok = d < Dm && n < N;
-        Are[s] = ok ? __ldg(p.A + (d * N + n) * 2) * (kF64 ? 1.f : kLog2e) : 0.f;
-        Aim[s] = ok ? __ldg(p.A + (d * N + n) * 2 + 1) : 0.f;
-        hr[s] = (ok && p.h0) ? __ldcg(p.h0 + ((b * Dm + d) * N + n) * 2) : 0.f;
-        hi[s] = (ok && p.h0) ? __ldcg(p.h0 + ((b * Dm + d) * N + n) * 2 + 1) : 0.f;
+        const bool aok = ok && MSCAN_WITHIN(p.x_A, p.A + (d * N + n) * 2, 8, kSiteA);
+        const bool hok = ok && p.h0 && MSCAN_WITHIN(p.x_h0, p.h0 + ((b * Dm + d) * N + n) * 2, 8, kSiteH0);
+        Are[s] = aok ? __ldg(p.A + (d * N + n) * 2) * (kF64 ? 1.f : kLog2e) : 0.f;
+        Aim[s] = aok ? __ldg(p.A + (d * N + n) * 2 + 1) : 0.f;
+        hr[s] = hok ? __ldcg(p.h0 + ((b * Dm + d) * N + n) * 2) : 0.f;
+        hi[s] = hok ? __ldcg(p.h0 + ((b * Dm + d) * N + n) * 2 + 1) : 0.f;
     }
 
     auto issue_loads = [&](int64_t t0, int st) {
@@ -159,9 +164,9 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
                 const int64_t t = t0 + tv * V;
                 const bool ok = (d0 + pc < Dm) && (t < L);
                 const int64_t off = ok ? row0 + pc * L + t : 0;
-                cpa16(rU + pc * TC + tv * V, gu + off, ok);
-                cpa16(rD + pc * TC + tv * V, gd + off, ok);
-                if (has_z) cpa16(rZ + pc * TC + tv * V, gz + off, ok);
+                cpa16(rU + pc * TC + tv * V, gu + off, ok && MSCAN_WITHIN(p.x_u, gu + off, 16, kSiteU));
+                cpa16(rD + pc * TC + tv * V, gd + off, ok && MSCAN_WITHIN(p.x_delta, gd + off, 16, kSiteDelta));
+                if (has_z) cpa16(rZ + pc * TC + tv * V, gz + off, ok && MSCAN_WITHIN(p.x_z, gz + off, 16, kSiteZ));
             }
             for (int vi = tid; vi < 2 * kCNP * BVR; vi += kCThreads) {
                 const int which = vi / (kCNP * BVR), rem = vi % (kCNP * BVR);
@@ -169,7 +174,8 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
                 const int64_t e = 2 * t0 + bv * V;  // element along the interleaved row
                 const bool ok = (n < N) && (e < 2 * L);
                 const int64_t off = ok ? bc0 + (int64_t)n * 2 * L + e : 0;
-                cpa16((which ? rC : rB) + n * 2 * TC + bv * V, (which ? gC : gB) + off, ok);
+                cpa16((which ? rC : rB) + n * 2 * TC + bv * V, (which ? gC : gB) + off,
+                      ok && MSCAN_WITHIN(which ? p.x_C : p.x_B, (which ? gC : gB) + off, 16, which ? kSiteC : kSiteB));
             }
         } else {
             for (int e = tid; e < CG * TC; e += kCThreads) {
@@ -177,16 +183,18 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
                 const int64_t t = t0 + tt;
                 const bool ok = (d0 + pc < Dm) && (t < L);
                 const int64_t off = row0 + pc * L + t;
-                rU[e] = ok ? gu[off] : T(0.f);
-                rD[e] = ok ? gd[off] : T(0.f);
-                if (has_z) rZ[e] = ok ? gz[off] : T(0.f);
+                rU[e] = (ok && MSCAN_WITHIN(p.x_u, gu + off, sizeof(T), kSiteU)) ? gu[off] : T(0.f);
+                rD[e] = (ok && MSCAN_WITHIN(p.x_delta, gd + off, sizeof(T), kSiteDelta)) ? gd[off] : T(0.f);
+                if (has_z) rZ[e] = (ok && MSCAN_WITHIN(p.x_z, gz + off, sizeof(T), kSiteZ)) ? gz[off] : T(0.f);
             }
             for (int e = tid; e < 2 * kCNP * 2 * TC; e += kCThreads) {
                 const int which = e / (kCNP * 2 * TC), rem = e % (kCNP * 2 * TC);
                 const int n = rem / (2 * TC), k = rem % (2 * TC);
                 const bool ok = (n < N) && (2 * t0 + k < 2 * L);
                 const int64_t off = bc0 + (int64_t)n * 2 * L + 2 * t0 + k;
-                (which ? rC : rB)[rem] = ok ? (which ? gC : gB)[off] : T(0.f);
+                (which ? rC : rB)[rem] =
+                    (ok && MSCAN_WITHIN(which ? p.x_C : p.x_B, (which ? gC : gB) + off, sizeof(T), which ? kSiteC : kSiteB))
+                        ? (which ? gC : gB)[off] : T(0.f);
             }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
@@ -210,7 +218,8 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
         for (int vi = tid; vi < CG * VPR; vi += kCThreads) {
             const int pc = vi / VPR, tv = vi % VPR;
             const int64_t dd = d0 + pc;
-            const float bias = (dd < Dm && p.delta_bias) ? __ldg(p.delta_bias + dd) : 0.f;
+            const float bias = (dd < Dm && p.delta_bias && MSCAN_WITHIN(p.x_bias, p.delta_bias + dd, 4, kSiteBias))
+                                   ? __ldg(p.delta_bias + dd) : 0.f;
             float fu[V], fd[V];
             Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + pc * TC + tv * V), fu);
             Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rD + pc * TC + tv * V), fd);
@@ -340,7 +349,7 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
             const int64_t dd = d0 + pc;
             const int64_t t = t0 + tv * V;
             if (dd >= Dm || tv * V >= tvalid) continue;
-            const float Dd = p.D ? __ldg(p.D + dd) : 0.f;
+            const float Dd = (p.D && MSCAN_WITHIN(p.x_D, p.D + dd, 4, kSiteD)) ? __ldg(p.D + dd) : 0.f;
             float fu[V], fz[V], y[V];
             Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rU + pc * TC + tv * V), fu);
             if (has_z) Elem<T>::unpack(*reinterpret_cast<const uint4 *>(rZ + pc * TC + tv * V), fz);
@@ -358,11 +367,12 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
             }
             T *dst = gout + row0 + pc * L + t;
             if (p.vec) {
-                stg16_stream(dst, Elem<T>::pack(y));
+                if (MSCAN_WITHIN(p.x_out, dst, 16, kSiteOut)) stg16_stream(dst, Elem<T>::pack(y));
             } else {
 #pragma unroll
                 for (int i = 0; i < V; ++i)
-                    if (tv * V + i < tvalid) Elem<T>::store(dst + i, y[i]);
+                    if (tv * V + i < tvalid && MSCAN_WITHIN(p.x_out, dst + i, sizeof(T), kSiteOut))
+                        Elem<T>::store(dst + i, y[i]);
             }
         }
     }
@@ -372,7 +382,7 @@ __global__ void __launch_bounds__(kCThreads) scan_fwd_complex_kernel(const CPara
 #pragma unroll
         for (int s = 0; s < S; ++s) {
             const int n = r * S + s;
-            if (n < N) {
+            if (n < N && MSCAN_WITHIN(p.x_last, ls + 2 * n, 8, kSiteLastState)) {
                 ls[2 * n] = (float)hr[s];
                 ls[2 * n + 1] = (float)hi[s];
             }
@@ -427,6 +437,8 @@ int complex_scan_lanes(int64_t batch, int64_t dim, int sm_count) {
     return best_r;
 }
 
+MSCAN_BOUNDS_TAKE(complex_bounds_take)
+
 cudaError_t launch_scan_fwd_complex(const ScanArgs &a, int lanes, cudaStream_t st) {
     CParams p;
     p.u = a.u; p.delta = a.delta; p.B = a.B; p.C = a.C; p.z = a.z;
@@ -434,6 +446,23 @@ cudaError_t launch_scan_fwd_complex(const ScanArgs &a, int lanes, cudaStream_t s
     p.out = a.out; p.last_state = a.last_state; p.h0 = a.h0;
     p.dim = a.dim; p.seqlen = a.seqlen; p.n_groups = 0;
     p.dstate = a.dstate; p.softplus = a.softplus;
+#ifdef MSCAN_BOUNDS_CHECK
+    const unsigned long long es = a.act == kBF16 ? 2 : 4;
+    const unsigned long long xb = (unsigned long long)(a.batch * a.dim * a.seqlen) * es;
+    const unsigned long long bcb = (unsigned long long)(a.batch * a.dstate * a.seqlen) * 2 * es;
+    const unsigned long long stb = (unsigned long long)(a.batch * a.dim * a.dstate) * 2 * 4;
+    p.x_u = extent_of(a.u, xb);
+    p.x_delta = extent_of(a.delta, xb);
+    p.x_z = extent_of(a.z, xb);
+    p.x_B = extent_of(a.B, bcb);
+    p.x_C = extent_of(a.C, bcb);
+    p.x_A = extent_of(a.A, (unsigned long long)(a.dim * a.dstate) * 2 * 4);
+    p.x_D = extent_of(a.D, (unsigned long long)a.dim * 4);
+    p.x_bias = extent_of(a.delta_bias, (unsigned long long)a.dim * 4);
+    p.x_out = extent_of(a.out, xb > (unsigned long long)g_out_extent_shrink ? xb - g_out_extent_shrink : 0);
+    p.x_last = extent_of(a.last_state, stb);
+    p.x_h0 = extent_of(a.h0, stb);
+#endif
     const int V = a.act == kBF16 ? 8 : 4;
     auto al = [](const void *q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
     p.vec = (a.seqlen % V == 0) && al(a.u) && al(a.delta) && al(a.z) && al(a.B) && al(a.C) && al(a.out);

@@ -344,29 +344,29 @@ scan_fwd_pairs_kernel(const Params p) {
 #pragma unroll
             for (int k = 0; k < S / 2; ++k) {
                 const int n0 = S * sr + 2 * k, n1 = n0 + 1;
-                const float a0 = (ds < Dm && n0 < N && within(p.x_A, p.A + ds * N + n0, 4, kSiteA))
+                const float a0 = (ds < Dm && n0 < N && MSCAN_WITHIN(p.x_A, p.A + ds * N + n0, 4, kSiteA))
                                      ? __ldg(p.A + ds * N + n0) : 0.f;
-                const float a1 = (ds < Dm && n1 < N && within(p.x_A, p.A + ds * N + n1, 4, kSiteA))
+                const float a1 = (ds < Dm && n1 < N && MSCAN_WITHIN(p.x_A, p.A + ds * N + n1, 4, kSiteA))
                                      ? __ldg(p.A + ds * N + n1) : 0.f;
                 A2[k] = make_float2(a0 * Dk::kScale, a1 * Dk::kScale);
             }
-            bias_p = (dp < Dm && p.delta_bias && within(p.x_bias, p.delta_bias + dp, 4, kSiteBias))
+            bias_p = (dp < Dm && p.delta_bias && MSCAN_WITHIN(p.x_bias, p.delta_bias + dp, 4, kSiteBias))
                          ? __ldg(p.delta_bias + dp) : 0.f;
             if (CL && lane < CW) {  // the prologue lane of a timestep needs every channel's bias
                 float *sbias = reinterpret_cast<float *>(base + CL_BIAS);
                 sbias[lane] = (d0 + lane < Dm && p.delta_bias &&
-                               within(p.x_bias, p.delta_bias + d0 + lane, 4, kSiteBias))
+                               MSCAN_WITHIN(p.x_bias, p.delta_bias + d0 + lane, 4, kSiteBias))
                                   ? __ldg(p.delta_bias + d0 + lane) : 0.f;
             }
-            D_s = (ds < Dm && p.D && within(p.x_D, p.D + ds, 4, kSiteD)) ? __ldg(p.D + ds) : 0.f;
+            D_s = (ds < Dm && p.D && MSCAN_WITHIN(p.x_D, p.D + ds, 4, kSiteD)) ? __ldg(p.D + ds) : 0.f;
             if (CONV) {  // taps right-aligned to 4: a shorter kernel sees zeros before it
                 const int K = p.conv_k;
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     cw[j] = (dp < Dm && j >= 4 - K &&
-                             within(p.x_conv_w, p.conv_w + dp * K + (j - (4 - K)), 4, kSiteConvW))
+                             MSCAN_WITHIN(p.x_conv_w, p.conv_w + dp * K + (j - (4 - K)), 4, kSiteConvW))
                                 ? __ldg(p.conv_w + dp * K + (j - (4 - K))) : 0.f;
-                cb_p = (dp < Dm && p.conv_b && within(p.x_conv_b, p.conv_b + dp, 4, kSiteConvB))
+                cb_p = (dp < Dm && p.conv_b && MSCAN_WITHIN(p.x_conv_b, p.conv_b + dp, 4, kSiteConvB))
                            ? __ldg(p.conv_b + dp) : 0.f;
             }
         }
@@ -380,7 +380,7 @@ scan_fwd_pairs_kernel(const Params p) {
 #pragma unroll
             for (int k = 0; k < S / 4; ++k) {
                 const float4 v = LOCAL ? reinterpret_cast<const float4 *>(carry_in)[k]
-                                 : within(p.x_carry, reinterpret_cast<const float4 *>(carry_in) + k, 16, kSiteCarry)
+                                 : MSCAN_WITHIN(p.x_carry, reinterpret_cast<const float4 *>(carry_in) + k, 16, kSiteCarry)
                                        ? __ldcg(reinterpret_cast<const float4 *>(carry_in) + k)  // S/4 float4
                                        : make_float4(0.f, 0.f, 0.f, 0.f);
                 hh[2 * k] = hv(v.x, v.y);
@@ -393,7 +393,7 @@ scan_fwd_pairs_kernel(const Params p) {
                 const float4 v = make_float4((float)hh[2 * k].x, (float)hh[2 * k].y, (float)hh[2 * k + 1].x,
                                              (float)hh[2 * k + 1].y);
                 if (LOCAL) reinterpret_cast<float4 *>(carry_out)[k] = v;
-                else if (within(p.x_carry, reinterpret_cast<float4 *>(carry_out) + k, 16, kSiteCarry))
+                else if (MSCAN_WITHIN(p.x_carry, reinterpret_cast<float4 *>(carry_out) + k, 16, kSiteCarry))
                     __stcg(reinterpret_cast<float4 *>(carry_out) + k, v);
             }
         };
@@ -462,10 +462,10 @@ scan_fwd_pairs_kernel(const Params p) {
                     const bool ok = cxok[i] && t0 + t < L;
                     const int64_t off = ok ? cxoff[i] + t0 * Dm : 0;
                     unsigned char *dst = sb0 + t * CROW + ((c ^ swz(t)) * 16);
-                    cp16(dst, gu + off, ok && within(p.x_u, gu + off, 16, kSiteU));
-                    cp16(dst + kTC * CROW, gd + off, ok && within(p.x_delta, gd + off, 16, kSiteDelta));
+                    cp16(dst, gu + off, ok && MSCAN_WITHIN(p.x_u, gu + off, 16, kSiteU));
+                    cp16(dst + kTC * CROW, gd + off, ok && MSCAN_WITHIN(p.x_delta, gd + off, 16, kSiteDelta));
                     if (GATE && !so_stage)
-                        cp16(dst + 2 * kTC * CROW, gz + off, ok && within(p.x_z, gz + off, 16, kSiteZ));
+                        cp16(dst + 2 * kTC * CROW, gz + off, ok && MSCAN_WITHIN(p.x_z, gz + off, 16, kSiteZ));
                 }
 #pragma unroll
                 for (int i = 0; i < NBC; ++i) {
@@ -474,7 +474,7 @@ scan_fwd_pairs_kernel(const Params p) {
                     const int64_t off = ok ? cboff[i] + t0 * N : 0;
                     if (!(so_stage && which))
                         cp16(sb0 + CL_ACT + which * kTC * BROW + t * BROW + c * 16, (which ? gC : gB) + off,
-                             ok && within(which ? p.x_C : p.x_B, (which ? gC : gB) + off, 16, which ? kSiteC : kSiteB));
+                             ok && MSCAN_WITHIN(which ? p.x_C : p.x_B, (which ? gC : gB) + off, 16, which ? kSiteC : kSiteB));
                 }
                 cp_commit();
                 return;
@@ -489,10 +489,10 @@ scan_fwd_pairs_kernel(const Params p) {
                     const bool ok = xok[i] && tok;
                     const int64_t off = ok ? xoff[i] + t0 : 0;
                     const T *su = gu + (ok ? uoff[i] + t0 : 0), *sz = gz + (ok ? zoff[i] + t0 : 0);
-                    cp16(sbuf + (0 * CW + r) * W::ROWB, su, ok && within(p.x_u, su, 16, kSiteU));
-                    cp16(sbuf + (1 * CW + r) * W::ROWB, gd + off, ok && within(p.x_delta, gd + off, 16, kSiteDelta));
+                    cp16(sbuf + (0 * CW + r) * W::ROWB, su, ok && MSCAN_WITHIN(p.x_u, su, 16, kSiteU));
+                    cp16(sbuf + (1 * CW + r) * W::ROWB, gd + off, ok && MSCAN_WITHIN(p.x_delta, gd + off, 16, kSiteDelta));
                     if (GATE && !so_stage)
-                        cp16(sbuf + (2 * CW + r) * W::ROWB, sz, ok && within(p.x_z, sz, 16, kSiteZ));
+                        cp16(sbuf + (2 * CW + r) * W::ROWB, sz, ok && MSCAN_WITHIN(p.x_z, sz, 16, kSiteZ));
                 }
             }
 #pragma unroll
@@ -503,7 +503,7 @@ scan_fwd_pairs_kernel(const Params p) {
                 const int64_t off = ok ? boff[i] + t0 : 0;
                 if (!(so_stage && which))
                     cp16(sbuf + (3 * CW + which * kNS + n) * W::ROWB, (which ? gC : gB) + off,
-                         ok && within(which ? p.x_C : p.x_B, (which ? gC : gB) + off, 16, which ? kSiteC : kSiteB));
+                         ok && MSCAN_WITHIN(which ? p.x_C : p.x_B, (which ? gC : gB) + off, 16, which ? kSiteC : kSiteB));
             }
             cp_commit();
         };
@@ -522,7 +522,7 @@ scan_fwd_pairs_kernel(const Params p) {
             for (int k = 0; k < 3; ++k) {
                 const int64_t t = tb0 - 3 + k;
                 const T *src = gu + b * p.u_bstride + (d0 + pc) * L + t;
-                halo[k] = (t >= 0 && pc < nrows && within(p.x_u, src, sizeof(T), kSiteHalo)) ? *src : T(0.f);
+                halo[k] = (t >= 0 && pc < nrows && MSCAN_WITHIN(p.x_u, src, sizeof(T), kSiteHalo)) ? *src : T(0.f);
             }
         }
 #pragma unroll 1
@@ -540,7 +540,7 @@ scan_fwd_pairs_kernel(const Params p) {
             const int tvalid = (L - t0) < kTC ? (int)(L - t0) : kTC;
             // checkpoint for the backward pass: the state entering every 32nd step
             if (!SO && p.ckpt != nullptr && (t0 & 31) == 0 && ds < Dm &&
-                within(p.x_ckpt,
+                MSCAN_WITHIN(p.x_ckpt,
                        p.ckpt + (((b * p.ckpt_gpb + (ds >> 5)) * p.ckpt_nsup + (t0 >> 5)) * 32 + (ds & 31)) * 16 + S * sr,
                        S * 4, kSiteCkpt)) {
                 float *dst = p.ckpt + (((b * p.ckpt_gpb + (ds >> 5)) * p.ckpt_nsup + (t0 >> 5)) * 32 + (ds & 31)) * 16 +
@@ -676,7 +676,7 @@ scan_fwd_pairs_kernel(const Params p) {
                 for (int i = lane; i < CW * CPR; i += 32) {
                     const int r = i / CPR, c = i % CPR;
                     const int64_t t = t0 + c * V;
-                    if (r < nrows && t < L && within(p.x_u_out, gu_out + row0 + r * L + t, 16, kSiteUOut))
+                    if (r < nrows && t < L && MSCAN_WITHIN(p.x_u_out, gu_out + row0 + r * L + t, 16, kSiteUOut))
                         stg16_stream(gu_out + row0 + r * L + t, *reinterpret_cast<const uint4 *>(sbuf + (0 * CW + r) * W::ROWB + c * 16));
                 }
             }
@@ -816,7 +816,7 @@ scan_fwd_pairs_kernel(const Params p) {
 #pragma unroll
                 for (int i = 0; i < NXC; ++i) {
                     const int q = lane + 32 * i, t = q / CH, c = q % CH;
-                    if (cxok[i] && t0 + t < L && within(p.x_out, gout + cxoff[i] + t0 * Dm, 16, kSiteOut))
+                    if (cxok[i] && t0 + t < L && MSCAN_WITHIN(p.x_out, gout + cxoff[i] + t0 * Dm, 16, kSiteOut))
                         stg16_stream(gout + cxoff[i] + t0 * Dm,
                                      *reinterpret_cast<const uint4 *>(outt + t * CROW + ((c ^ swz(t)) * 16)));
                 }
@@ -825,7 +825,7 @@ scan_fwd_pairs_kernel(const Params p) {
             for (int i = lane; i < (CL ? 0 : CW * CPR); i += 32) {
                 const int r = i / CPR, c = i % CPR;
                 const int64_t t = t0 + c * V;
-                if (r < nrows && t < L && within(p.x_out, gout + row0 + r * L + t, 16, kSiteOut))
+                if (r < nrows && t < L && MSCAN_WITHIN(p.x_out, gout + row0 + r * L + t, 16, kSiteOut))
                     stg16_stream(gout + row0 + r * L + t,
                                  *reinterpret_cast<const uint4 *>(outt + r * W::ROWB + c * 16));
             }
@@ -840,8 +840,8 @@ scan_fwd_pairs_kernel(const Params p) {
                 const int n0 = S * sr + 2 * k;
                 const float *src = p.h0 + (b * Dm + ds) * N;
                 hh[k] = (p.h0 && ds < Dm)
-                            ? hv((n0 < N && within(p.x_h0, src + n0, 4, kSiteH0)) ? __ldcg(src + n0) : 0.f,
-                                 (n0 + 1 < N && within(p.x_h0, src + n0 + 1, 4, kSiteH0)) ? __ldcg(src + n0 + 1) : 0.f)
+                            ? hv((n0 < N && MSCAN_WITHIN(p.x_h0, src + n0, 4, kSiteH0)) ? __ldcg(src + n0) : 0.f,
+                                 (n0 + 1 < N && MSCAN_WITHIN(p.x_h0, src + n0 + 1, 4, kSiteH0)) ? __ldcg(src + n0 + 1) : 0.f)
                                           : hv(0.f, 0.f);
             }
         };
@@ -898,8 +898,8 @@ scan_fwd_pairs_kernel(const Params p) {
 #pragma unroll
             for (int k = 0; k < S / 2; ++k) {
                 const int n0 = S * sr + 2 * k;
-                if (n0 < N && within(p.x_last, ls + n0, 4, kSiteLastState)) ls[n0] = (float)h[k].x;
-                if (n0 + 1 < N && within(p.x_last, ls + n0 + 1, 4, kSiteLastState)) ls[n0 + 1] = (float)h[k].y;
+                if (n0 < N && MSCAN_WITHIN(p.x_last, ls + n0, 4, kSiteLastState)) ls[n0] = (float)h[k].x;
+                if (n0 + 1 < N && MSCAN_WITHIN(p.x_last, ls + n0 + 1, 4, kSiteLastState)) ls[n0 + 1] = (float)h[k].y;
             }
         }
     }

@@ -34,18 +34,25 @@ struct SUParams {
     int dstate;
     int softplus;
     // byte ranges of the pointer arguments, for the bounds-checked build
-    Extent x_state, x_u, x_delta, x_B, x_C, x_z, x_A, x_D, x_bias, x_out;
+    MSCAN_EXTENTS(x_state, x_u, x_delta, x_B, x_C, x_z, x_A, x_D, x_bias, x_out)
 };
 
 // Loads that the bounds-checked build tests against the tensor's range (a
 // load outside reads zero; see bounds.cuh).
+#ifdef MSCAN_BOUNDS_CHECK
 template <typename T>
 __device__ __forceinline__ float load_chk(const Extent &e, const T *q, int site) {
-    return within(e, q, sizeof(T), site) ? Elem<T>::load(q) : 0.f;
+    return MSCAN_WITHIN(e, q, sizeof(T), site) ? Elem<T>::load(q) : 0.f;
 }
 __device__ __forceinline__ float ldg_chk(const Extent &e, const float *q, int site) {
-    return within(e, q, 4, site) ? __ldg(q) : 0.f;
+    return MSCAN_WITHIN(e, q, 4, site) ? __ldg(q) : 0.f;
 }
+#else
+template <typename T>
+__device__ __forceinline__ float load_plain(const T *q) { return Elem<T>::load(q); }
+#define load_chk(e, q, site) load_plain(q)
+#define ldg_chk(e, q, site) __ldg(q)
+#endif
 
 // NV > 0: dstate == NV, known at compile time, 16-byte state accesses.
 // NV == 0: any dstate, scalar accesses.
@@ -76,9 +83,9 @@ state_update_kernel(const SUParams p) {
     if (NV > 0) {
 #pragma unroll
         for (int n = 0; n < N; n += 4) {
-            const bool sok = within(p.x_state, st + n, 16, kSiteState);
+            const bool sok = MSCAN_WITHIN(p.x_state, st + n, 16, kSiteState);
             float4 h = sok ? *reinterpret_cast<const float4 *>(st + n) : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float4 a4 = within(p.x_A, Ad + n, 16, kSiteA) ? __ldg(reinterpret_cast<const float4 *>(Ad + n))
+            const float4 a4 = MSCAN_WITHIN(p.x_A, Ad + n, 16, kSiteA) ? __ldg(reinterpret_cast<const float4 *>(Ad + n))
                                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
             HS hv[4] = {h.x, h.y, h.z, h.w};
             const float av[4] = {a4.x, a4.y, a4.z, a4.w};
@@ -93,7 +100,7 @@ state_update_kernel(const SUParams p) {
         }
     } else {
         for (int n = 0; n < N; ++n) {
-            const bool sok = within(p.x_state, st + n, 4, kSiteState);
+            const bool sok = MSCAN_WITHIN(p.x_state, st + n, 4, kSiteState);
             const HS hn = Dk::step(dl2 * ldg_chk(p.x_A, Ad + n, kSiteA), (HS)(sok ? st[n] : 0.f),
                                    du * load_chk(p.x_B, gB + n, kSiteB));
             if (sok) st[n] = (float)hn;
@@ -104,7 +111,7 @@ state_update_kernel(const SUParams p) {
     if (p.D) yo = (float)fma((HS)ldg_chk(p.x_D, p.D + d, kSiteD), (HS)ut, y);
     if (gz) yo *= silu_f(load_chk(p.x_z, gz + row, kSiteZ));
     T *o = static_cast<T *>(p.out) + row;
-    if (within(p.x_out, o, sizeof(T), kSiteOut)) Elem<T>::store(o, yo);
+    if (MSCAN_WITHIN(p.x_out, o, sizeof(T), kSiteOut)) Elem<T>::store(o, yo);
 }
 
 // Four states per lane: bf16 / fp32 loads of four consecutive B or C values.
@@ -151,10 +158,10 @@ state_update_lanes_kernel(const SUParams p) {
         const float4 *a = reinterpret_cast<const float4 *>(p.A + (int64_t)d * NV) + qi + v * Q;
         const T *bq = static_cast<const T *>(p.B) + (int64_t)b * NV + 4 * (qi + v * Q);
         const T *cq = static_cast<const T *>(p.C) + (int64_t)b * NV + 4 * (qi + v * Q);
-        h4[v] = within(p.x_state, st + v * Q, 16, kSiteState) ? st[v * Q] : zero4;
-        a4[v] = within(p.x_A, a, 16, kSiteA) ? __ldg(a) : zero4;
-        b4[v] = within(p.x_B, bq, 4 * sizeof(T), kSiteB) ? Quad<T>::load(bq) : zero4;
-        c4[v] = within(p.x_C, cq, 4 * sizeof(T), kSiteC) ? Quad<T>::load(cq) : zero4;
+        h4[v] = MSCAN_WITHIN(p.x_state, st + v * Q, 16, kSiteState) ? st[v * Q] : zero4;
+        a4[v] = MSCAN_WITHIN(p.x_A, a, 16, kSiteA) ? __ldg(a) : zero4;
+        b4[v] = MSCAN_WITHIN(p.x_B, bq, 4 * sizeof(T), kSiteB) ? Quad<T>::load(bq) : zero4;
+        c4[v] = MSCAN_WITHIN(p.x_C, cq, 4 * sizeof(T), kSiteC) ? Quad<T>::load(cq) : zero4;
     }
     const float dr = load_chk(p.x_delta, static_cast<const T *>(p.delta) + row, kSiteDelta);
     const float ut = load_chk(p.x_u, static_cast<const T *>(p.u) + row, kSiteU);
@@ -181,13 +188,13 @@ state_update_lanes_kernel(const SUParams p) {
     if (!live) return;
 #pragma unroll
     for (int v = 0; v < V; ++v)
-        if (within(p.x_state, st + v * Q, 16, kSiteState)) st[v * Q] = h4[v];
+        if (MSCAN_WITHIN(p.x_state, st + v * Q, 16, kSiteState)) st[v * Q] = h4[v];
     if (qi == 0) {
         float yo = (float)y;
         if (p.D) yo = (float)fma((HS)Dd, (HS)ut, y);
         if (p.z) yo *= silu_f(zt);
         T *o = static_cast<T *>(p.out) + row;
-        if (within(p.x_out, o, sizeof(T), kSiteOut)) Elem<T>::store(o, yo);
+        if (MSCAN_WITHIN(p.x_out, o, sizeof(T), kSiteOut)) Elem<T>::store(o, yo);
     }
 }
 
@@ -247,6 +254,7 @@ cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t st) {
     kp.state = a.state; kp.u = a.u; kp.delta = a.delta; kp.B = a.B; kp.C = a.C; kp.z = a.z;
     kp.A = a.A; kp.D = a.D; kp.delta_bias = a.delta_bias; kp.out = a.out;
     kp.rows = a.batch * a.dim; kp.dim = a.dim; kp.dstate = a.dstate; kp.softplus = a.softplus;
+#ifdef MSCAN_BOUNDS_CHECK
     const unsigned long long es = a.act == kBF16 ? 2 : 4, rows = (unsigned long long)(a.batch * a.dim);
     const unsigned long long xb = rows * es;
     kp.x_state = extent_of(a.state, rows * a.dstate * 4);
@@ -259,6 +267,7 @@ cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t st) {
     kp.x_D = extent_of(a.D, (unsigned long long)a.dim * 4);
     kp.x_bias = extent_of(a.delta_bias, (unsigned long long)a.dim * 4);
     kp.x_out = extent_of(a.out, xb > (unsigned long long)g_out_extent_shrink ? xb - g_out_extent_shrink : 0);
+#endif
     if (a.act == kBF16) return launch_typed<__nv_bfloat16>(kp, st);
     return launch_typed<float>(kp, st);
 }

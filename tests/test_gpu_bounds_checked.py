@@ -1,8 +1,9 @@
 """The bounds-checked build (libmamba_scan_checked.so, MSCAN_BOUNDS_CHECK).
 
 Its instrumented kernels -- the lane-split scan in every form that uses it,
-the static scan in its staging forms, the decode step, the conv1d kernels --
-test every global access against the byte range of its tensor.  On the shapes below (ragged groups and lengths,
+the static scan in its staging forms, the complex mode, the backward, the
+decode step, the conv1d kernels -- test every global access against the
+byte range of its tensor.  On the shapes below (ragged groups and lengths,
 N < 16, both lane counts, two-phase pieces, the device-wide and block-local
 forms, the (b, l, d) layout, the fused conv1d with u written out,
 checkpoints, initial and final states) they must record no access outside a
@@ -188,6 +189,46 @@ def test_conv1d(checked, L):
         return binding.mamba_conv1d_update(st, ci["xz"][:, :40, 0].contiguous(), ci["weight"], ci["bias"]), st
 
     ref, got = both(checked, step)
+    assert equal(ref, got)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("shape", [(2, 70, 336), (1, 100, 1000)])
+def test_backward(checked, dtype, shape):
+    """Self-contained (its own checkpoint sweep) and from the forward's
+    checkpoints, from an initial state, with dL/dlast_state.  dA / dB / dC /
+    dD / dbias sum with atomics whose order varies, so those are compared
+    within a few ulps; du, ddelta, dz bit for bit."""
+    b, d, L = shape
+    w = inputs.custom(b, d, L, 16, dtype, seed=b + d + L + 1)
+    ins = inputs.scan_inputs(w, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(3)
+    dout = torch.randn(b, d, L, generator=g, device="cuda").to(ins["u"].dtype)
+    dlast = torch.randn(b, d, 16, generator=g, device="cuda")
+    h0 = inputs.initial_state(b, d, 16, seed=4, device="cuda")
+    kw = dict(D=ins["D"], z=ins["z"], delta_bias=ins["delta_bias"])
+    _, _, ck = binding.mamba_scan_fwd_ckpt(ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"], h0=h0, **kw)
+    for ckpt in (None, ck):
+        run = lambda: binding.mamba_scan_bwd(dout, ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"],  # noqa: E731
+                                             dlast_state=dlast, h0=h0, ckpt=ckpt, **kw)
+        ref, got = both(checked, run)
+        for k in ref:
+            if ref[k] is None:
+                continue
+            if k in ("du", "ddelta", "dz"):
+                assert torch.equal(ref[k], got[k]), k
+            else:
+                assert torch.allclose(ref[k], got[k], rtol=1e-5, atol=1e-6 * ref[k].abs().max().item()), k
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_complex_mode(checked, dtype):
+    d = inputs.complex_inputs(2, 40, 333, 16, dtype, device="cuda")
+    h0 = torch.randn(2, 40, 16, 2, device="cuda") * 0.25
+    run = lambda: binding.mamba_scan_fwd_complex(d["u"], d["delta"], d["A"], d["B"], d["C"], D=d["D"],  # noqa: E731
+                                                 z=d["z"], delta_bias=d["delta_bias"], h0=h0,
+                                                 return_last_state=True)
+    ref, got = both(checked, run)
     assert equal(ref, got)
 
 
