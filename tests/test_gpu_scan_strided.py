@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import oracle
-from parity import TOL, record, rel_err, to_np
+from parity import TOL, oracle_rows, record, rel_err, sample_rows, to_np
 from selective_state_space_20_b200 import binding, inputs
 
 pytestmark = pytest.mark.gpu
@@ -156,6 +156,44 @@ def test_page_layout_ragged_length_and_optional_inputs(dtype, lanes):
             cpu[k] = None
         _check(f"page layout {w.name} lanes={lanes} drop={drop}", cpu, _page_layout(cpu), dtype,
                schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=lanes)
+
+
+@pytest.mark.parametrize("lanes", [2, 4])
+def test_page_layout_in_place_from_a_state(lanes):
+    """The local kernel on the pages' layout writing out over u (same
+    pointer and strides) and starting from h0: bit-equal to the same call
+    with a separate output."""
+    w = inputs.custom(2, 96, 512, 16, "bf16", seed=41 + lanes)
+    cpu = inputs.scan_inputs(w)
+    h0 = inputs.initial_state(2, 96, 16, seed=5).cuda()
+    dev = _page_layout(cpu)
+    kw = dict(schedule=binding.SCHEDULE_LOCAL, lanes_per_channel=lanes)
+    ref, ref_state = _run(dev, h0=h0, **kw)
+    dev["u"] = dev["u"].clone().transpose(1, 2).contiguous().transpose(1, 2)
+    out, state = _run(dev, out=dev["u"], h0=h0, **kw)
+    assert out.data_ptr() == dev["u"].data_ptr()
+    assert torch.equal(out, ref) and torch.equal(state, ref_state)
+
+
+def test_page_layout_default_call_at_layer_size():
+    """Without a schedule the pages' layout of a Mamba-sized layer (1,280
+    lane-pair groups) takes the block-local kernel: bit-equal to the dense
+    call, sampled rows against the oracle."""
+    w = inputs.custom(4, 5120, 512, 16, "bf16", seed=43)
+    cpu = inputs.scan_inputs(w)
+    dense = {k: (None if v is None else v.cuda()) for k, v in cpu.items()}
+    o1, s1 = binding.mamba_scan_fwd(dense["u"], dense["delta"], dense["A"], dense["B"], dense["C"], D=dense["D"],
+                                    z=dense["z"], delta_bias=dense["delta_bias"], return_last_state=True)
+    assert binding.mamba_scan_plan(4, 5120, 512, 16, torch.bfloat16, workspace=False)[2] == binding.SCHEDULE_LOCAL
+    o2, s2 = _run(_page_layout(cpu))
+    assert torch.equal(o1, o2.contiguous()) and torch.equal(s1, s2)
+    rows = sample_rows(w.batch, w.dim, 8, seed=w.seed)
+    ro, rs = oracle_rows(cpu, rows)
+    idx = torch.tensor(rows, device="cuda")
+    e1 = rel_err(to_np(o2.contiguous().view(w.batch * w.dim, -1).index_select(0, idx)), ro)
+    e2 = rel_err(to_np(s2.view(w.batch * w.dim, -1).index_select(0, idx)), rs)
+    record(f"page layout default call {w.name} sampled", out=e1, state=e2)
+    assert e1 <= TOL[torch.bfloat16] and e2 <= TOL[torch.bfloat16]
 
 
 def test_page_layout_local_schedule_needs_the_layout():
