@@ -30,7 +30,10 @@
 //     workspace, L2-resident); then each 4-step window, last first, is
 //     recomputed once more into registers -- states and decays -- and walked
 //     in reverse from them, so the reverse step evaluates no exponential.
-//   * Sums over a channel's states are shuffles among its 4 lanes; dB and dC,
+//   * Sums over a channel's states (C h, S_A, S_B) are kept per step of the
+//     4-step window and summed over the channel's 4 lanes at its end,
+//     transposed: lane r then holds step r's totals and forms that step's
+//     du, ddelta_raw, dz and its dD and dbias terms.  dB and dC,
 //     sums over every channel of a batch row, are summed over a warp's 8
 //     channels by a transposed shuffle reduction, over the block's warps in
 //     shared memory, and added with one atomic add per (state, step) and
@@ -65,6 +68,8 @@ constexpr int kSub = 4;                  // timesteps recomputed into registers 
 constexpr int kNSub = kSup / kSub;       // sub-checkpoints per super-segment
 constexpr int kRep = 8;                  // copies of dB / dC the blocks add into (group % kRep)
 constexpr int kCkCh = 32;                // channels per checkpoint group (the forward's layout)
+// a window's steps are shared out one per lane of a channel for the per-step sums
+static_assert(kSub == kNS / kSPL, "one window step per lane of a channel");
 
 // per-channel fp32 values of a super-segment: one 16-byte record per (step,
 // channel) -- (delta, u, dy, gate factor) -- read with one load, and the
@@ -140,6 +145,32 @@ struct ChannelTranspose {
 template <int CNT>
 struct ChannelTranspose<2, CNT> {
     __device__ __forceinline__ static void run(float (&)[8], int) {}
+};
+
+// Sum part[w][q] over the 4 lanes of a channel (lane bits 0 and 1),
+// transposed: afterwards part[0][q] of lane r holds the total of the lanes'
+// original part[r][q].  Round K = 2 keeps steps 2, 3 in the lanes with bit 1
+// set and 0, 1 in the others; round K = 1 keeps the odd or even one.
+template <typename X>
+struct QuadTranspose {
+    __device__ __forceinline__ static void run(X (&part)[4][3], int lane) {
+        const bool up2 = (lane & 2) != 0, up1 = (lane & 1) != 0;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+                const X send = up2 ? part[i][q] : part[i + 2][q];
+                const X keep = up2 ? part[i + 2][q] : part[i][q];
+                part[i][q] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+            const X send = up1 ? part[0][q] : part[1][q];
+            const X keep = up1 ? part[1][q] : part[0][q];
+            part[0][q] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+        }
+    }
 };
 
 template <typename X>
@@ -435,6 +466,7 @@ scan_bwd_kernel(const BwdParams p) {
                     }
                 }
                 float *rb = red + rbuf * (kSub * kWarpsBwd * 32);
+                HS part[kSub][3];  // per step: this lane's share of C h, S_A, S_B
 #pragma unroll
                 for (int w = kSub - 1; w >= 0; --w) {
                     const int t = tb + w;
@@ -490,16 +522,27 @@ scan_bwd_kernel(const BwdParams p) {
                     }
                     ChannelTranspose<16, 8>::run(v, lane);
                     rb[(w * kWarpsBwd + wib) * 32 + kslot] = v[0];
-                    const float y = (float)quad_sum(yp) + Dd * ut;
-                    const float SA = (float)quad_sum(sA), SBs = (float)quad_sum(sB);
+                    part[w][0] = yp;
+                    part[w][1] = sA;
+                    part[w][2] = sB;
+                }
+                // the channel's sums over its states, transposed over the
+                // window: lane r ends with the totals of step tb + r and
+                // forms that step's outputs, dD and dbias terms
+                QuadTranspose<HS>::run(part, lane);
+                {
+                    const int t = tb + r;
+                    const float4 rec = srec[t * kCh + cb];
+                    const float dl = rec.x, ut = rec.y, dy = rec.z;
+                    const float y = (float)part[0][0] + Dd * ut;
+                    const float SA = (float)part[0][1], SBs = (float)part[0][2];
                     const float ddelta = fmaf(ut, SBs, SA);
                     const float ddraw = ddelta * ssig[t * kCh + cb];
                     dbias_acc += (HS)ddraw;
                     dD_acc = fma((HS)dy, (HS)ut, dD_acc);
-                    // this channel's three outputs, one lane each
-                    if (r == 0) outs[(0 * kCh + cb) * RP + t] = T(fmaf(dy, Dd, dl * SBs));
-                    if (r == 1) outs[(1 * kCh + cb) * RP + t] = T(ddraw);
-                    if (GATE && r == 2) outs[(2 * kCh + cb) * RP + t] = T(y * rec.w);
+                    outs[(0 * kCh + cb) * RP + t] = T(fmaf(dy, Dd, dl * SBs));
+                    outs[(1 * kCh + cb) * RP + t] = T(ddraw);
+                    if (GATE) outs[(2 * kCh + cb) * RP + t] = T(y * rec.w);
                 }
                 __syncthreads();  // the window's dB / dC terms of every warp are in rb
                 // dB / dC of the window: thread -> (step, slot), the warps summed in order
@@ -546,10 +589,13 @@ scan_bwd_kernel(const BwdParams p) {
                         p.dh0[(b * Dm + dc) * N + n] = (float)g[i];  // dL/dh_{-1}
                 }
             }
-            if (r == 0) {
-                if (p.dD && MSCAN_WITHIN(p.x_dD, p.dD + dc, 4, kSiteD)) atomicAdd(p.dD + dc, (float)dD_acc);
-                if (p.dbias && MSCAN_WITHIN(p.x_dbias, p.dbias + dc, 4, kSiteBias)) atomicAdd(p.dbias + dc, (float)dbias_acc);
-            }
+        }
+        // each lane summed dD and dbias over its step of every window
+        dD_acc = quad_sum(dD_acc);
+        dbias_acc = quad_sum(dbias_acc);
+        if (valid && r == 0) {
+            if (p.dD && MSCAN_WITHIN(p.x_dD, p.dD + dc, 4, kSiteD)) atomicAdd(p.dD + dc, (float)dD_acc);
+            if (p.dbias && MSCAN_WITHIN(p.x_dbias, p.dbias + dc, 4, kSiteBias)) atomicAdd(p.dbias + dc, (float)dbias_acc);
         }
         __syncthreads();  // before the next group reuses shared memory
     }
