@@ -492,7 +492,8 @@ int mamba_debug_stall_group(int group);
  * The bounds-checked build (libmamba_scan_checked.so, compiled with
  * MSCAN_BOUNDS_CHECK; same entry points and results).  Every launch of the
  * lane-split scan kernel (mamba_scan_fwd, _ws, _noalloc, _init, _conv,
- * _ckpt, the (batch, L, dim) layout of mamba_scan_fwd_strided), of the static
+ * _ckpt, the (batch, L, dim) layout of mamba_scan_fwd_strided), of the
+ * one-lane scan kernel (lanes_per_channel = 1 with a workspace), of the static
  * scan kernel (any layout of mamba_scan_fwd_strided, small problems of
  * mamba_scan_fwd), of the complex mode, of the backward (mamba_scan_bwd,
  * _init, _ckpt), of the decode step (mamba_state_update) and of the conv1d
@@ -507,8 +508,7 @@ int mamba_debug_stall_group(int group);
  * carries, 18 decode state, 19 conv1d input, 20 conv1d state; the backward
  * reports dout and du / ddelta / dz as 13, dlast as 14, dA / dD / dbias as
  * 1 / 3 / 2, dB / dC as 9 / 10 and its workspace parts as 16 and 17) and its
- * byte offset from the tensor's start.  Nothing traps.  The one-lane kernel
- * (lanes_per_channel = 1 on request) is not instrumented.  In the normal build
+ * byte offset from the tensor's start.  Nothing traps.  In the normal build
  * the checks compile away.
  *
  * mamba_bounds_checked: 1 in the bounds-checked build, 0 otherwise.

@@ -23,11 +23,12 @@ void note_workspace(const void *ws) {
 }
 
 // The first recorded violation of the instrumented kernels (lane-split,
-// static and complex scans, backward, decode, conv1d), every record cleared:
+// one-lane, static and complex scans, backward, decode, conv1d), every
+// record cleared:
 // 1 with it, 0 without, -1 on a read error.
 int take_bounds(int *site, long long *off) {
     int found = 0;
-    int (*takes[])(int *, long long *) = {mscan::pairs_bounds_take, mscan::static_bounds_take,
+    int (*takes[])(int *, long long *) = {mscan::pairs_bounds_take, mscan::spec_bounds_take, mscan::static_bounds_take,
                                           mscan::complex_bounds_take, mscan::bwd_bounds_take,
                                           mscan::state_update_bounds_take, mscan::conv1d_bounds_take};
     for (auto take : takes) {

@@ -2,16 +2,16 @@
 //
 // Every kernel launch carries, for each pointer argument, the byte range it
 // may touch (an Extent, filled on the host from the sizes the caller passed).
-// In the checked build each global access of the lane-split, static and
-// complex scan kernels, the backward, the decode step and the conv1d kernels
-// first asks MSCAN_WITHIN(): an access that would leave its range is skipped -- a load reads zeros, a store
+// In the checked build each global access of the scan kernels (lane-split,
+// one-lane, static, complex), the backward, the decode step and the conv1d
+// kernels first asks MSCAN_WITHIN(): an access that would leave its range is
+// skipped -- a load reads zeros, a store
 // is dropped -- and the first such access of the launch is recorded (site and
 // byte offset) in a word of its translation unit, which the host reads
 // through mamba_get_device_status / mamba_debug_bounds_status.  Nothing traps
 // or faults.  In the normal build MSCAN_WITHIN() is the constant true, its
 // arguments are not compiled, and the launch parameters carry no ranges
-// (MSCAN_EXTENTS declares them in the checked build only).  The one-lane
-// kernel is not instrumented.
+// (MSCAN_EXTENTS declares them in the checked build only).
 #pragma once
 
 #include <cuda_runtime.h>

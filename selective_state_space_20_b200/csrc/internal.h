@@ -17,6 +17,7 @@ extern int g_out_extent_shrink;
 // (1: a violation, its site and byte offset; cleared), 0 without one, -1 on
 // a read error.  Always 0 in the normal build.
 int pairs_bounds_take(int *site, long long *off);
+int spec_bounds_take(int *site, long long *off);
 int static_bounds_take(int *site, long long *off);
 int complex_bounds_take(int *site, long long *off);
 int bwd_bounds_take(int *site, long long *off);

@@ -290,6 +290,9 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
     kp.queue = reinterpret_cast<unsigned *>(w + l.queue_off);
     kp.progress = nullptr;
     kp.carry = reinterpret_cast<float *>(w + l.carry_off);
+#ifdef MSCAN_BOUNDS_CHECK
+    kp.x_carry = extent_of(kp.carry, l.bytes - l.carry_off);
+#endif
     // counters and queue entries start at zero; carries are written before read
     cudaError_t e = cudaMemsetAsync(w, 0, l.queue_off + (size_t)(l.groups * (l.chunks - 1)) * 4, st);
     if (e != cudaSuccess) return e;

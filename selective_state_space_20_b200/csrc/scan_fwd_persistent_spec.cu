@@ -263,16 +263,19 @@ struct Helper {
             for (int it = 0; it < W::CPR; ++it) {
                 const bool ok = tok && row_x[it] < nrows;
                 const long long off = ok ? base_x + off_x[it] : 0;
-                cp16(rows + (W::ROW_U + row_x[it]) * W::ROWB, gu + off, ok);
-                cp16(rows + (W::ROW_D + row_x[it]) * W::ROWB, gd + off, ok);
-                if (gz) cp16(rows + (W::ROW_Z + row_x[it]) * W::ROWB, gz + off, ok);
+                cp16(rows + (W::ROW_U + row_x[it]) * W::ROWB, gu + off, ok && MSCAN_WITHIN(p.x_u, gu + off, 16, kSiteU));
+                cp16(rows + (W::ROW_D + row_x[it]) * W::ROWB, gd + off,
+                     ok && MSCAN_WITHIN(p.x_delta, gd + off, 16, kSiteDelta));
+                if (gz)
+                    cp16(rows + (W::ROW_Z + row_x[it]) * W::ROWB, gz + off, ok && MSCAN_WITHIN(p.x_z, gz + off, 16, kSiteZ));
             }
 #pragma unroll
             for (int it = 0; it < W::CPR; ++it) {
                 const int which = (lane + 32 * it) / (kNS * W::CPR);
                 const bool ok = tok && n_bc[it] < p.dstate;
                 const long long off = ok ? base_bc + off_bc[it] : 0;
-                cp16(rows + (W::ROW_B + which * kNS + n_bc[it]) * W::ROWB, (which ? gC : gB) + off, ok);
+                cp16(rows + (W::ROW_B + which * kNS + n_bc[it]) * W::ROWB, (which ? gC : gB) + off,
+                     ok && MSCAN_WITHIN(which ? p.x_C : p.x_B, (which ? gC : gB) + off, 16, which ? kSiteC : kSiteB));
             }
         }
         cp_commit();
@@ -287,7 +290,8 @@ struct Helper {
         if (d.flags & (kEnd | kSkip)) return;
         const unsigned char *rows = raw(k) + W::HDR;
         const int dc = d.d0 + lane;
-        const float bias = (dc < p.dim && p.delta_bias) ? __ldg(p.delta_bias + dc) : 0.f;
+        const float bias = (dc < p.dim && p.delta_bias && MSCAN_WITHIN(p.x_bias, p.delta_bias + dc, 4, kSiteBias))
+                               ? __ldg(p.delta_bias + dc) : 0.f;
         float fu[kTC], fd[kTC];
         unpack_row<T>(rows + (W::ROW_U + lane) * W::ROWB, fu);
         unpack_row<T>(rows + (W::ROW_D + lane) * W::ROWB, fd);
@@ -316,7 +320,7 @@ struct Helper {
         const int dc = d.d0 + lane;
         if (dc >= p.dim) return;
         const unsigned char *rows = raw(k) + W::HDR;
-        const float Dd = p.D ? __ldg(p.D + dc) : 0.f;
+        const float Dd = (p.D && MSCAN_WITHIN(p.x_D, p.D + dc, 4, kSiteD)) ? __ldg(p.D + dc) : 0.f;
         float fu[kTC], fz[kTC], y[kTC];
         unpack_row<T>(rows + (W::ROW_U + lane) * W::ROWB, fu);
         if (GATE) unpack_row<T>(rows + (W::ROW_Z + lane) * W::ROWB, fz);
@@ -337,7 +341,8 @@ struct Helper {
         T *dst = static_cast<T *>(p.out) + (d.rowidx + lane) * p.seqlen + d.t0;
 #pragma unroll
         for (int c = 0; c < W::CPR; ++c)
-            if (c * W::V < d.tvalid) stg16_stream(dst + c * W::V, Elem<T>::pack(o + c * W::V));
+            if (c * W::V < d.tvalid && MSCAN_WITHIN(p.x_out, dst + c * W::V, 16, kSiteOut))
+                stg16_stream(dst + c * W::V, Elem<T>::pack(o + c * W::V));
     }
 };
 
@@ -434,8 +439,9 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
 #pragma unroll
                     for (int q = 0; q < kNS / 2; ++q) {
                         const int n0 = 2 * q, n1 = 2 * q + 1;
-                        const float a0 = (dc < p.dim && n0 < N) ? __ldg(p.A + (int64_t)dc * N + n0) : 0.f;
-                        const float a1 = (dc < p.dim && n1 < N) ? __ldg(p.A + (int64_t)dc * N + n1) : 0.f;
+                        const float *a = p.A + (int64_t)dc * N;
+                        const float a0 = (dc < p.dim && n0 < N && MSCAN_WITHIN(p.x_A, a + n0, 4, kSiteA)) ? __ldg(a + n0) : 0.f;
+                        const float a1 = (dc < p.dim && n1 < N && MSCAN_WITHIN(p.x_A, a + n1, 4, kSiteA)) ? __ldg(a + n1) : 0.f;
                         A2[q] = f2(a0 * Decay<sizeof(T) == 4>::kScale, a1 * Decay<sizeof(T) == 4>::kScale);
                     }
                 }
@@ -443,13 +449,17 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
                     const float *src = p.h0 + (d.rowidx + lane) * N;
 #pragma unroll
                     for (int q = 0; q < kNS / 2; ++q)
-                        hs[q] = (p.h0 && dc < p.dim) ? hv(2 * q < N ? __ldcg(src + 2 * q) : 0.f,
-                                                          2 * q + 1 < N ? __ldcg(src + 2 * q + 1) : 0.f)
-                                                     : hv(0.f, 0.f);
+                        hs[q] = (p.h0 && dc < p.dim)
+                                    ? hv((2 * q < N && MSCAN_WITHIN(p.x_h0, src + 2 * q, 4, kSiteH0)) ? __ldcg(src + 2 * q) : 0.f,
+                                         (2 * q + 1 < N && MSCAN_WITHIN(p.x_h0, src + 2 * q + 1, 4, kSiteH0))
+                                             ? __ldcg(src + 2 * q + 1) : 0.f)
+                                    : hv(0.f, 0.f);
                 } else {
 #pragma unroll
                     for (int q = 0; q < kNS / 4; ++q) {
-                        const float4 v = __ldcg(reinterpret_cast<const float4 *>(carry) + q);
+                        const float4 v = MSCAN_WITHIN(p.x_carry, reinterpret_cast<const float4 *>(carry) + q, 16, kSiteCarry)
+                                             ? __ldcg(reinterpret_cast<const float4 *>(carry) + q)
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
                         hs[2 * q] = hv(v.x, v.y);
                         hs[2 * q + 1] = hv(v.z, v.w);
                     }
@@ -514,16 +524,18 @@ __global__ void __launch_bounds__(2 * kPairs * 32, 1) scan_fwd_spec_kernel(const
                 if (d.j + 1 < p.n_chunks) {
 #pragma unroll
                     for (int q = 0; q < kNS / 4; ++q)
-                        __stcg(reinterpret_cast<float4 *>(carry) + q,
-                               make_float4((float)hs[2 * q].x, (float)hs[2 * q].y, (float)hs[2 * q + 1].x,
-                                           (float)hs[2 * q + 1].y));
+                        if (MSCAN_WITHIN(p.x_carry, reinterpret_cast<float4 *>(carry) + q, 16, kSiteCarry))
+                            __stcg(reinterpret_cast<float4 *>(carry) + q,
+                                   make_float4((float)hs[2 * q].x, (float)hs[2 * q].y, (float)hs[2 * q + 1].x,
+                                               (float)hs[2 * q + 1].y));
                     push_unit(p, lane, (unsigned)((d.j + 1) * p.n_groups + d.g));
                 } else if (p.last_state != nullptr && dc < p.dim) {
                     float *ls = p.last_state + (d.rowidx + lane) * N;
 #pragma unroll
                     for (int q = 0; q < kNS / 2; ++q) {
-                        if (2 * q < N) ls[2 * q] = (float)hs[q].x;
-                        if (2 * q + 1 < N) ls[2 * q + 1] = (float)hs[q].y;
+                        if (2 * q < N && MSCAN_WITHIN(p.x_last, ls + 2 * q, 4, kSiteLastState)) ls[2 * q] = (float)hs[q].x;
+                        if (2 * q + 1 < N && MSCAN_WITHIN(p.x_last, ls + 2 * q + 1, 4, kSiteLastState))
+                            ls[2 * q + 1] = (float)hs[q].y;
                     }
                 }
             }
@@ -544,6 +556,8 @@ cudaError_t launch_t(const Params &kp, int grid, cudaStream_t st) {
 }
 
 }  // namespace
+
+MSCAN_BOUNDS_TAKE(spec_bounds_take)
 
 int persistent_spec_sub_chunk() { return kTC; }
 int persistent_spec_pairs_per_sm() { return kPairs; }

@@ -1,9 +1,9 @@
 """The bounds-checked build (libmamba_scan_checked.so, MSCAN_BOUNDS_CHECK).
 
 Its instrumented kernels -- the lane-split scan in every form that uses it,
-the static scan in its staging forms, the complex mode, the backward, the
-decode step, the conv1d kernels -- test every global access against the
-byte range of its tensor.  On the shapes below (ragged groups and lengths,
+the one-lane scan, the static scan in its staging forms, the complex mode,
+the backward, the decode step, the conv1d kernels -- test every global
+access against the byte range of its tensor.  On the shapes below (ragged groups and lengths,
 N < 16, both lane counts, two-phase pieces, the device-wide and block-local
 forms, the (b, l, d) layout, the fused conv1d with u written out,
 checkpoints, initial and final states) they must record no access outside a
@@ -94,6 +94,26 @@ def test_device_wide_scan_and_checkpoints(checked, lanes):
     ck = lambda: binding.mamba_scan_fwd_ckpt(ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"], D=ins["D"],  # noqa: E731
                                              z=ins["z"], delta_bias=ins["delta_bias"])
     ref, got = both(checked, ck)
+    assert equal(ref, got)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("shape,dstate,chunk", [((2, 70, 1000), 16, 64), ((3, 33, 344), 5, 0)],
+                         ids=["2x70x1000-chunks64", "3x33x344-N5"])
+def test_one_lane_scan(checked, dtype, shape, dstate, chunk):
+    """The one-lane kernel (scan warp + helper warp, on request): ragged
+    channel groups and lengths, carries between chunks, h0 and last_state."""
+    b, d, L = shape
+    w = inputs.custom(b, d, L, dstate, dtype, seed=b + d + L + 1)
+    ins = inputs.scan_inputs(w, device="cuda")
+    h0 = inputs.initial_state(b, d, dstate, seed=4, device="cuda")
+    ws = torch.empty(binding.mamba_scan_workspace_size(b, d, L, dstate, ins["u"].dtype), device="cuda",
+                     dtype=torch.uint8)
+    run = lambda: binding.mamba_scan_fwd(ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"], D=ins["D"],  # noqa: E731
+                                         z=ins["z"], delta_bias=ins["delta_bias"], h0=h0, return_last_state=True,
+                                         workspace=ws, schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=1,
+                                         chunk_timesteps=chunk)
+    ref, got = both(checked, run)
     assert equal(ref, got)
 
 
@@ -259,7 +279,7 @@ def test_a_short_output_range_is_reported_and_its_store_skipped(checked):
     def scan():
         out = sentinel.clone()
         # the block-local lane-split kernel (a shape this small would otherwise
-        # take the static kernel, which is not instrumented)
+        # take the static kernel, shortened further below)
         binding.mamba_scan_fwd(ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"], D=ins["D"], z=ins["z"],
                                delta_bias=ins["delta_bias"], out=out, schedule=binding.SCHEDULE_LOCAL)
         return out
@@ -293,6 +313,19 @@ def test_a_short_output_range_is_reported_and_its_store_skipped(checked):
 
     ref, got = _shrunk(checked, static_scan, lambda o: o, 4)
     assert torch.equal(got.reshape(-1)[:-1], ref.reshape(-1)[:-1]) and got.reshape(-1)[-1] == 7.0
+
+    ws = torch.empty(binding.mamba_scan_workspace_size(w.batch, w.dim, w.seqlen, w.dstate, torch.bfloat16),
+                     device="cuda", dtype=torch.uint8)
+
+    def one_lane():  # the one-lane kernel's 16-byte stores
+        out = sentinel.clone()
+        binding.mamba_scan_fwd(ins["u"], ins["delta"], ins["A"], ins["B"], ins["C"], D=ins["D"], z=ins["z"],
+                               delta_bias=ins["delta_bias"], out=out, workspace=ws,
+                               schedule=binding.SCHEDULE_PERSISTENT, lanes_per_channel=1)
+        return out
+
+    ref, got = _shrunk(checked, one_lane, lambda o: o, 16)
+    assert torch.equal(got.reshape(-1)[:-8], ref.reshape(-1)[:-8]) and torch.all(got.reshape(-1)[-8:] == 7.0)
 
     ci = inputs.conv_inputs(2, 32, 256, 4, "bf16", seed=39, device="cuda")
     conv = lambda: binding.mamba_conv1d_fwd(ci["xz"], ci["weight"], ci["bias"], dim=32,  # noqa: E731
