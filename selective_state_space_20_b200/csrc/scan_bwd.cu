@@ -187,8 +187,13 @@ __device__ __forceinline__ float sigmoid(float x) {
     return __fdividef(1.f, 1.f + __expf(-x));
 }
 
+// Blocks per SM that shared memory allows ([fp32 activations][6 warps]; 228
+// KiB per SM, 1 KiB of it reserved per block): bf16 48 KiB (4 warps) or
+// 68.75 KiB (6); fp32 64 KiB or 91.75 KiB.  The register cap follows from it.
+constexpr int kBwdBlocksPerSM[2][2] = {{4, 3}, {3, 2}};
+
 template <typename T, bool SP, bool GATE, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32, sizeof(T) == 4 ? (WARPS == 4 ? 3 : 2) : (WARPS == 4 ? 5 : 3))
+__global__ void __launch_bounds__(WARPS * 32, kBwdBlocksPerSM[sizeof(T) == 4][WARPS == 6])
 scan_bwd_kernel(const BwdParams p) {
     constexpr bool ACC = sizeof(T) == 4;
     using Dk = Decay<ACC>;
@@ -628,6 +633,8 @@ __global__ void __launch_bounds__(256) bwd_sum_copies_kernel(const BwdParams p) 
 
 template <typename T, bool SP, bool GATE, int WARPS>
 cudaError_t launch_w(const BwdParams &p, int sm_count, cudaStream_t st) {
+    static_assert((BwdSmem<T, WARPS>::BYTES + 1024) * kBwdBlocksPerSM[sizeof(T) == 4][WARPS == 6] <= 228 * 1024,
+                  "the blocks per SM of the launch bounds fit in shared memory");
     auto kern = scan_bwd_kernel<T, SP, GATE, WARPS>;
     const int smem = BwdSmem<T, WARPS>::BYTES;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -663,16 +670,20 @@ cudaError_t launch_typed(const BwdParams &p, int warps, int sm_count, cudaStream
 
 // Warps per block.  A channel group's adjoint runs through the sequence in
 // order, so the groups are the units of work and the SM that holds the most
-// of them sets the time: pick the block size whose busiest SM carries the
-// fewest warps, all blocks resident (bf16: 5 blocks of 4 warps or 3 of 6 per
-// SM).  Mamba-2.8B layer: 640 groups of 32 channels (5 on some SMs: 20
-// warps) against 428 of 48 (3 per SM: 18 warps).
+// of them sets the time: of the block sizes whose blocks are all resident at
+// once (kBwdBlocksPerSM per SM), pick the one whose busiest SM carries the
+// fewest warps.  Mamba-2.8B layer: 640 groups of 32 channels do not fit (592
+// resident); 428 of 48 do (3 per SM: 18 warps).
 int bwd_warps(int64_t batch, int64_t dim, int act, int sm_count) {
+    const int f32 = act == kBF16 ? 0 : 1;
     const int64_t g4 = batch * ((dim + 31) / 32), g6 = batch * ((dim + 47) / 48);
-    const int64_t slots4 = (int64_t)sm_count * (act == kBF16 ? 5 : 3), slots6 = (int64_t)sm_count * (act == kBF16 ? 3 : 2);
-    if (g6 > slots6 || g4 > slots4) return 4;
-    const int64_t load4 = 4 * ((g4 + sm_count - 1) / sm_count), load6 = 6 * ((g6 + sm_count - 1) / sm_count);
-    return load6 < load4 ? 6 : 4;
+    const bool fit4 = g4 <= (int64_t)sm_count * kBwdBlocksPerSM[f32][0];
+    const bool fit6 = g6 <= (int64_t)sm_count * kBwdBlocksPerSM[f32][1];
+    if (fit4 && fit6) {
+        const int64_t load4 = 4 * ((g4 + sm_count - 1) / sm_count), load6 = 6 * ((g6 + sm_count - 1) / sm_count);
+        return load6 < load4 ? 6 : 4;
+    }
+    return fit6 ? 6 : 4;
 }
 
 }  // namespace
