@@ -173,6 +173,24 @@ struct QuadTranspose {
     }
 };
 
+// A lane's 4 states of a sub-checkpoint: one 16-byte access (fp32 states)
+// or two (fp64); the slot is 16-byte aligned.
+__device__ __forceinline__ void store4(float *q, const float (&h)[4]) {
+    *reinterpret_cast<float4 *>(q) = make_float4(h[0], h[1], h[2], h[3]);
+}
+__device__ __forceinline__ void store4(double *q, const double (&h)[4]) {
+    reinterpret_cast<double2 *>(q)[0] = make_double2(h[0], h[1]);
+    reinterpret_cast<double2 *>(q)[1] = make_double2(h[2], h[3]);
+}
+__device__ __forceinline__ void load4(const float *q, float (&h)[4]) {
+    const float4 v = *reinterpret_cast<const float4 *>(q);
+    h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
+}
+__device__ __forceinline__ void load4(const double *q, double (&h)[4]) {
+    const double2 a = reinterpret_cast<const double2 *>(q)[0], b = reinterpret_cast<const double2 *>(q)[1];
+    h[0] = a.x; h[1] = a.y; h[2] = b.x; h[3] = b.y;
+}
+
 template <typename X>
 __device__ __forceinline__ X quad_sum(X x) {
     x += __shfl_xor_sync(0xffffffffu, x, 1);
@@ -415,16 +433,22 @@ scan_bwd_kernel(const BwdParams p) {
                                      : make_float4(0.f, 0.f, 0.f, 0.f);
                 HS h[kSPL] = {(HS)v.x, (HS)v.y, (HS)v.z, (HS)v.w};
                 for (int j = 0; j * kSub < tn; ++j) {
-#pragma unroll
-                    for (int i = 0; i < kSPL; ++i)
-                        if (MSCAN_WITHIN(p.x_subck, sub + j * (kWarpsBwd * 32) * kSPL + i, sizeof(HS), kSiteCarry))
-                            sub[j * (kWarpsBwd * 32) * kSPL + i] = h[i];
+                    if (MSCAN_WITHIN(p.x_subck, sub + j * (kWarpsBwd * 32) * kSPL, kSPL * sizeof(HS), kSiteCarry))
+                        store4(sub + j * (kWarpsBwd * 32) * kSPL, h);
 #pragma unroll
                     for (int w = 0; w < kSub; ++w) step(h, j * kSub + w);
                 }
             }
             // windows of kSub steps, last first: states and decays into
-            // registers, then the reverse steps from them
+            // registers, then the reverse steps from them.  A window's
+            // sub-checkpoint (this thread's own store, in L2) is loaded one
+            // window ahead.
+            HS hnext[kSPL] = {};
+            auto load_sub = [&](int j) {
+                if (MSCAN_WITHIN(p.x_subck, sub + j * (kWarpsBwd * 32) * kSPL, kSPL * sizeof(HS), kSiteCarry))
+                    load4(sub + j * (kWarpsBwd * 32) * kSPL, hnext);
+            };
+            load_sub((tn - 1) / kSub);
             for (int j = (tn - 1) / kSub; j >= 0; --j) {
                 const int tb = j * kSub;
                 HS hin[kSPL], hs[kSub][kSPL];
@@ -433,9 +457,8 @@ scan_bwd_kernel(const BwdParams p) {
                 // activations, so the adjoint decays with the state's accuracy
                 float ab[kSub][kSPL];
 #pragma unroll
-                for (int i = 0; i < kSPL; ++i)
-                    hin[i] = MSCAN_WITHIN(p.x_subck, sub + j * (kWarpsBwd * 32) * kSPL + i, sizeof(HS), kSiteCarry)
-                                 ? sub[j * (kWarpsBwd * 32) * kSPL + i] : (HS)0.f;
+                for (int i = 0; i < kSPL; ++i) hin[i] = hnext[i];
+                if (j > 0) load_sub(j - 1);
 #pragma unroll
                 for (int w = 0; w < kSub; ++w) {
                     {
