@@ -420,6 +420,12 @@ scan_bwd_kernel(const BwdParams p) {
         for (int s = p.n_sup - 1; s >= 0; --s) {
             const int64_t t0 = (int64_t)s * kSup;
             const int tn = seg_len(s);
+            // the segment's checkpoint, loaded before the staging work that
+            // hides its latency (channels past dim have no checkpoint of the
+            // forward's: zeros)
+            const float4 ckv = (valid && MSCAN_WITHIN(p.x_ckpt, ck + (int64_t)s * kCkCh * kNS, 16, kSiteCkpt))
+                                   ? __ldcg(reinterpret_cast<const float4 *>(ck + (int64_t)s * kCkCh * kNS))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
             asm volatile("cp.async.wait_group 0;" ::: "memory");
             __syncthreads();  // raw landed; sx, sbc, outs of the previous segment consumed
             convert(s, true);
@@ -427,11 +433,7 @@ scan_bwd_kernel(const BwdParams p) {
             if (s > 0) fetch(s - 1, true);
             // recompute the segment from its checkpoint, one sub-checkpoint every kSub steps
             {
-                // (channels past dim have no checkpoint of the forward's: zeros)
-                const float4 v = (valid && MSCAN_WITHIN(p.x_ckpt, ck + (int64_t)s * kCkCh * kNS, 16, kSiteCkpt))
-                                     ? __ldcg(reinterpret_cast<const float4 *>(ck + (int64_t)s * kCkCh * kNS))
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-                HS h[kSPL] = {(HS)v.x, (HS)v.y, (HS)v.z, (HS)v.w};
+                HS h[kSPL] = {(HS)ckv.x, (HS)ckv.y, (HS)ckv.z, (HS)ckv.w};
                 for (int j = 0; j * kSub < tn; ++j) {
                     if (MSCAN_WITHIN(p.x_subck, sub + j * (kWarpsBwd * 32) * kSPL, kSPL * sizeof(HS), kSiteCarry))
                         store4(sub + j * (kWarpsBwd * 32) * kSPL, h);
