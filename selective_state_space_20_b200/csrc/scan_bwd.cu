@@ -447,8 +447,12 @@ scan_bwd_kernel(const BwdParams p) {
             // window ahead.
             HS hnext[kSPL] = {};
             auto load_sub = [&](int j) {
-                if (MSCAN_WITHIN(p.x_subck, sub + j * (kWarpsBwd * 32) * kSPL, kSPL * sizeof(HS), kSiteCarry))
+                if (MSCAN_WITHIN(p.x_subck, sub + j * (kWarpsBwd * 32) * kSPL, kSPL * sizeof(HS), kSiteCarry)) {
                     load4(sub + j * (kWarpsBwd * 32) * kSPL, hnext);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kSPL; ++i) hnext[i] = (HS)0.f;
+                }
             };
             load_sub((tn - 1) / kSub);
             for (int j = (tn - 1) / kSub; j >= 0; --j) {
