@@ -253,6 +253,44 @@ int mamba_scan_fwd_init(const void *u, const void *delta, const float *A,
                         const mamba_scan_tuning_t *tuning, void *workspace,
                         size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * mamba_scan_state -- the final state of the scan alone: last_state =
+ * h_{L-1} of the recurrence of mamba_scan_fwd_init (steps a2-a4 and a7 of the
+ * S6 forward), without the readout, gate or outputs.  This is what one shard
+ * of a sequence split over several GPUs contributes before the exchange
+ * (its state from a zero start; the shards are then folded with
+ * mamba_state_fold), and the way to advance a state over a prompt whose
+ * outputs are not wanted.
+ *
+ *   u, delta     : act (batch, dim, seqlen), as mamba_scan_fwd.
+ *   A            : fp32 (dim, dstate); delta_bias fp32 (dim) or NULL.
+ *   B            : act (batch, dstate, seqlen).  C, D and z take no part.
+ *   h0           : fp32 (batch, dim, dstate) or NULL (zeros); may be
+ *                  last_state exactly (advanced in place).
+ *   last_state   : fp32 (batch, dim, dstate), required, written.
+ *   workspace    : NULL (block-local lane-split kernel, no workspace) or at
+ *                  least mamba_scan_workspace_size bytes, 16-byte aligned
+ *                  (device-wide form).
+ *
+ * The lane-split kernel runs every piece of each channel group's sequence
+ * state-only from a zero start (no C rows, readout, gate or stores; delta
+ * summed in fp64) and combines it with the state before the piece as
+ * exp(A sum(delta)) h_in + h_piece: about three quarters of a full scan.
+ * Results agree with mamba_scan_fwd_init's last_state within the tolerance,
+ * not bit for bit (the pieces are combined in another order).
+ * Requires dstate <= 16 and 16-byte aligned rows of a whole number of
+ * 16-byte vectors (as the lane-split schedules): else MAMBA_ERR_UNSUPPORTED.
+ * Errors: MAMBA_ERR_NULL, MAMBA_ERR_SHAPE, MAMBA_ERR_OVERLAP (last_state over
+ * an input, a workspace over anything), MAMBA_ERR_WORKSPACE (misaligned or
+ * small), MAMBA_ERR_CUDA.
+ */
+int mamba_scan_state(const void *u, const void *delta, const float *A,
+                     const void *B, const float *delta_bias, int delta_softplus,
+                     const float *h0, float *last_state, int64_t batch,
+                     int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
+                     void *workspace, size_t workspace_bytes,
+                     cudaStream_t stream);
+
 /* Element strides of one sequence tensor: along the batch, along its rows
  * (channels for u / delta / z / out, states for B / C) and along time. */
 typedef struct {
@@ -492,7 +530,8 @@ int mamba_debug_stall_group(int group);
  * The bounds-checked build (libmamba_scan_checked.so, compiled with
  * MSCAN_BOUNDS_CHECK; same entry points and results).  Every launch of the
  * lane-split scan kernel (mamba_scan_fwd, _ws, _noalloc, _init, _conv,
- * _ckpt, the (batch, L, dim) layout of mamba_scan_fwd_strided), of the
+ * _ckpt, the (batch, L, dim) layout of mamba_scan_fwd_strided,
+ * mamba_scan_state), of the
  * one-lane scan kernel (lanes_per_channel = 1 with a workspace), of the static
  * scan kernel (any layout of mamba_scan_fwd_strided, small problems of
  * mamba_scan_fwd), of the complex mode, of the backward (mamba_scan_bwd,

@@ -25,6 +25,7 @@ STATUS_NAMES = {0: "MAMBA_OK", -1: "MAMBA_ERR_NULL", -2: "MAMBA_ERR_SHAPE",
                 -3: "MAMBA_ERR_UNSUPPORTED", -4: "MAMBA_ERR_ALIGN",
                 -5: "MAMBA_ERR_CUDA", -6: "MAMBA_ERR_DEVICE", -7: "MAMBA_ERR_OVERLAP",
                 -8: "MAMBA_ERR_WORKSPACE", -9: "MAMBA_ERR_TIMEOUT", -10: "MAMBA_ERR_BOUNDS"}
+MAMBA_ERR_UNSUPPORTED = -3
 MAMBA_ERR_TIMEOUT = -9
 MAMBA_ERR_BOUNDS = -10
 SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT, SCHEDULE_LOCAL = 0, 1, 2, 3
@@ -33,7 +34,7 @@ SCHEDULE_AUTO, SCHEDULE_STATIC, SCHEDULE_PERSISTENT, SCHEDULE_LOCAL = 0, 1, 2, 3
 EXPORTED = ("mamba_scan_fwd", "mamba_scan_fwd_tuned", "mamba_scan_fwd_ws",
             "mamba_scan_plan", "mamba_scan_plan_noworkspace", "mamba_scan_workspace_size",
             "mamba_scan_workspace_status",
-            "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_fwd_strided",
+            "mamba_scan_fwd_noalloc", "mamba_scan_fwd_init", "mamba_scan_state", "mamba_scan_fwd_strided",
             "mamba_scan_fwd_complex", "mamba_delta_sum", "mamba_state_fold", "mamba_scan_fwd_conv",
             "mamba_scan_host_scratch_size", "mamba_scan_fwd_host", "mamba_debug_stall_group",
             "mamba_get_device_status", "mamba_scan_bwd", "mamba_scan_bwd_init",
@@ -80,6 +81,9 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.mamba_scan_fwd_init.argtypes = scan_args[:9] + [fp] + scan_args[9:] + [
         ctypes.POINTER(Tuning), vp, ctypes.c_size_t, vp]
     lib.mamba_scan_fwd_init.restype = ci
+    lib.mamba_scan_state.argtypes = [vp, vp, fp, vp, fp, ci, fp, fp, i64, i64, i64, i64, ci, vp, ctypes.c_size_t,
+                                     vp]
+    lib.mamba_scan_state.restype = ci
     lib.mamba_scan_fwd_strided.argtypes = scan_args[:9] + [fp] + scan_args[9:] + [
         ctypes.POINTER(ScanStrides), ctypes.POINTER(Tuning), vp]
     lib.mamba_scan_fwd_strided.restype = ci
@@ -521,6 +525,46 @@ def mamba_scan_fwd_host(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor, B
                                      scratch.numel(), _stream(dev))
     _check("mamba_scan_fwd_host", rc)
     return (out, last_state) if want_state else out
+
+
+def mamba_scan_state(u: torch.Tensor, delta: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                     delta_bias: Optional[torch.Tensor] = None, delta_softplus: bool = True,
+                     h0: Optional[torch.Tensor] = None, last_state: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The final state of the scan alone (no readout, gate or outputs):
+    u, delta (batch, dim, L), B (batch, N, L) in the activation dtype; A
+    (dim, N) fp32; h0 / the returned last_state (batch, dim, N) fp32.  Raises
+    MambaError (MAMBA_ERR_UNSUPPORTED) where the lane-split kernel cannot run
+    (dstate > 16, rows not whole 16-byte vectors)."""
+    if u.dim() != 3:
+        raise ValueError("u must be (batch, dim, seqlen)")
+    batch, dim, L = u.shape
+    N = A.shape[1] if A.dim() == 2 else -1
+    dev, act = u.device, u.dtype
+    if dev.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    if act not in _ACT:
+        raise TypeError(f"unsupported activation dtype {act}")
+    _need(delta, "delta", dev, act, (batch, dim, L))
+    _need(A, "A", dev, torch.float32, (dim, N))
+    _need(B, "B", dev, act, (batch, N, L))
+    _need(delta_bias, "delta_bias", dev, torch.float32, (dim,))
+    _need(h0, "h0", dev, torch.float32, (batch, dim, N))
+    if last_state is None:
+        last_state = torch.empty((batch, dim, N), device=dev, dtype=torch.float32)
+    _need(last_state, "last_state", dev, torch.float32, (batch, dim, N))
+    ws_bytes = 0
+    if workspace is not None:
+        if workspace.device != dev:
+            raise ValueError("workspace must be on the tensors' device")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    lib = load_library()
+    with torch.cuda.device(dev):
+        rc = lib.mamba_scan_state(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(delta_bias),
+                                  int(bool(delta_softplus)), _ptr(h0), _ptr(last_state), batch, dim, L, N,
+                                  _ACT[act], _ptr(workspace), ws_bytes, _stream(dev))
+    _check("mamba_scan_state", rc)
+    return last_state
 
 
 def mamba_delta_sum(delta: torch.Tensor, delta_bias: Optional[torch.Tensor] = None,

@@ -592,6 +592,57 @@ int mamba_scan_fwd_init(const void *u, const void *delta, const float *A, const 
                      stream, true, nullptr);
 }
 
+int mamba_scan_state(const void *u, const void *delta, const float *A, const void *B,
+                     const float *delta_bias, int delta_softplus, const float *h0, float *last_state,
+                     int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate, int act_dtype,
+                     void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return MAMBA_ERR_UNSUPPORTED;
+    int rc = check_sizes(batch, dim, seqlen, dstate);
+    if (rc != MAMBA_OK) return rc;
+    if (!u || !delta || !A || !B || !last_state) return MAMBA_ERR_NULL;
+    const size_t es = act_size(act_dtype);
+    const size_t nx = (size_t)(batch * dim * seqlen) * es;
+    const size_t nbc = (size_t)(batch * dstate * seqlen) * es;
+    const size_t nA = (size_t)(dim * dstate) * 4, nd = (size_t)dim * 4;
+    const size_t nls = (size_t)(batch * dim * dstate) * 4;
+    if (overlaps(last_state, nls, u, nx) || overlaps(last_state, nls, delta, nx) ||
+        overlaps(last_state, nls, B, nbc) || overlaps(last_state, nls, A, nA) ||
+        overlaps(last_state, nls, delta_bias, nd) || bad_alias(last_state, nls, h0, nls, true))
+        return MAMBA_ERR_OVERLAP;
+    if (workspace) {
+        if ((reinterpret_cast<uintptr_t>(workspace) & 15) != 0) return MAMBA_ERR_WORKSPACE;
+        const void *ins[] = {u, delta, B, A, delta_bias, last_state, h0};
+        const size_t sz[] = {nx, nx, nbc, nA, nd, nls, nls};
+        for (int i = 0; i < 7; ++i)
+            if (overlaps(workspace, workspace_bytes, ins[i], sz[i])) return MAMBA_ERR_OVERLAP;
+        if (workspace_bytes < mscan::persistent_workspace_bound(batch, dim, seqlen, act_dtype))
+            return MAMBA_ERR_WORKSPACE;
+    }
+    int status = MAMBA_OK;
+    const int sms = current_sm_count(&status);
+    if (status != MAMBA_OK) return status;
+    mscan::ScanArgs a;
+    a.u = u; a.delta = delta; a.B = B; a.C = nullptr; a.z = nullptr;
+    a.A = A; a.D = nullptr; a.delta_bias = delta_bias; a.out = nullptr; a.last_state = last_state; a.h0 = h0;
+    a.strides = nullptr;
+    a.state_only = true;
+    a.batch = batch; a.dim = dim; a.seqlen = seqlen; a.dstate = (int)dstate;
+    a.softplus = delta_softplus ? 1 : 0; a.act = act_dtype;
+    // the lane-split kernel only: dstate <= 16, 16-byte aligned rows
+    if (!mscan::persistent_supported(a)) return MAMBA_ERR_UNSUPPORTED;
+    if (workspace) {
+        int lanes = mscan::persistent_choose_lanes(a, sms);
+        if (lanes != 2 && lanes != 4) lanes = 2;
+        note_workspace(workspace);
+        return mscan::launch_scan_fwd_persistent(a, lanes, 0, workspace, workspace_bytes, sms, stream) == cudaSuccess
+                   ? MAMBA_OK : MAMBA_ERR_CUDA;
+    }
+    int lanes = mscan::local_choose_lanes(a, sms);
+    if (lanes == 0) lanes = 2;
+    note_workspace(nullptr);
+    return mscan::launch_scan_fwd_local(a, lanes, sms, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
 size_t mamba_scan_workspace_size(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
                                  int act_dtype) {
     if (act_dtype != MAMBA_F32 && act_dtype != MAMBA_BF16) return 0;

@@ -57,6 +57,9 @@ struct ScanArgs {
     // (batch, L, dim) and B / C dense (batch, L, N) -- the layout of the
     // Keras page -- instead of (batch, dim, L) / (batch, N, L)
     bool channels_last = false;
+    // lane-split kernel only: the final state alone -- no C, D, z, readout,
+    // gate or out (dense layout, no conv, no checkpoints)
+    bool state_only = false;
     int64_t batch, dim, seqlen;
     int dstate;
     int softplus;

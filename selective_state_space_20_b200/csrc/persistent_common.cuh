@@ -62,6 +62,8 @@ struct Params {
     // lane-split block-local kernel: u / delta / z / out as (batch, L, dim)
     // and B / C as (batch, L, N), all dense (else (batch, dim, L) / (batch, N, L))
     int channels_last;
+    // lane-split kernel: the final state alone (no C, readout, gate or out)
+    int state_only;
     // byte ranges of the pointer arguments, for the bounds-checked build
     MSCAN_EXTENTS(x_u, x_delta, x_z, x_B, x_C, x_A, x_D, x_bias, x_out, x_last, x_h0, x_conv_w, x_conv_b, x_u_out,
                   x_ckpt, x_carry)

@@ -174,6 +174,7 @@ persist::Params base_params(const ScanArgs &a, int lanes, int tc) {
     kp.ckpt_gpb = (int)((a.dim + 31) / 32);
     kp.ckpt_nsup = (int)((a.seqlen + 31) / 32);
     kp.channels_last = a.channels_last ? 1 : 0;
+    kp.state_only = a.state_only ? 1 : 0;
 #ifdef MSCAN_BOUNDS_CHECK
     // byte ranges of the pointer arguments (checked in the bounds-checked build)
     const unsigned long long es = a.act == kBF16 ? 2 : 4;
@@ -224,9 +225,16 @@ int local_choose_lanes(const ScanArgs &a, int sm_count) {
     return 0;
 }
 
+// The final state alone runs on the dense layout without the fused conv1d or
+// checkpoints.
+static bool state_only_ok(const ScanArgs &a) {
+    return !a.state_only || (!a.conv_w && !a.ckpt && !a.channels_last);
+}
+
 cudaError_t launch_scan_fwd_local(const ScanArgs &a, int lanes, int sm_count, cudaStream_t st) {
     if (lanes != 2 && lanes != 4) return cudaErrorInvalidValue;
     if (a.conv_w && !a.softplus) return cudaErrorInvalidValue;
+    if (!state_only_ok(a)) return cudaErrorInvalidValue;
     persist::Params kp = base_params(a, lanes, sub_chunk(lanes, a.act));
     kp.n_chunks = 1;
     kp.chunk_len = (int)a.seqlen;
@@ -252,6 +260,7 @@ cudaError_t launch_scan_fwd_persistent(const ScanArgs &a, int lanes, int chunk_t
     const int tc = sub_chunk(lanes, a.act);
 
     if (a.conv_w && (lanes == 1 || !a.softplus)) return cudaErrorInvalidValue;  // lane-split kernel, softplus on
+    if (a.state_only && (lanes == 1 || !state_only_ok(a))) return cudaErrorInvalidValue;
     persist::Params kp = base_params(a, lanes, tc);
     unsigned char *w = static_cast<unsigned char *>(workspace);
     kp.hdr = reinterpret_cast<unsigned *>(w);

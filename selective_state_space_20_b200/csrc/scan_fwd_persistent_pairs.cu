@@ -849,7 +849,7 @@ scan_fwd_pairs_kernel(const Params p) {
 #pragma unroll
         for (int k = 0; k < S / 2; ++k) h[k] = hv(0.f, 0.f);
         double dsum = 0.0;
-        if (two_phase && se < p.subs_per_chain) {
+        if ((two_phase && se < p.subs_per_chain) || p.state_only) {
             // The piece ends inside its group and other workers' pieces of the
             // group wait for its end state.  Get that state first with a
             // state-only run from a zero start, while the worker before it is
@@ -857,7 +857,9 @@ scan_fwd_pairs_kernel(const Params p) {
             // piece starts the group): end = exp(A sum(delta)) h_in + local
             // end, published at once.  The pieces of a group thus finish their
             // waits one after the other in a few steps instead of running one
-            // after the other; the output run follows from h_in.
+            // after the other; the output run follows from h_in.  A launch for
+            // the final state alone (state_only) takes this path for every
+            // piece and stops after the end state.
             run_subs(true, h, dsum, false);
             HV hin[S / 2];
             if (sb > 0) {
@@ -878,11 +880,13 @@ scan_fwd_pairs_kernel(const Params p) {
                                             ex2_mufu((float)((double)A2[k].y * dsum)));
                     hend[k] = __ffma2_rn(decay, hin[k], h[k]);
                 }
-                h[k] = hin[k];
+                h[k] = p.state_only ? hend[k] : hin[k];
             }
-            store_carry(hend);
-            publish_carry(se);
-            run_subs(false, h, dsum, false);
+            if (se < p.subs_per_chain) {
+                store_carry(hend);
+                publish_carry(se);
+            }
+            if (!p.state_only) run_subs(false, h, dsum, false);
         } else {
             if (sb > 0) {
                 if (!wait_carry(sb)) return;

@@ -5,8 +5,9 @@ Rank r of a process group holds timesteps [r * L_r, (r + 1) * L_r) of every
 a shard's initial state h to exp(A * S) (.) h + h_local (S the shard's sum of
 delta per row, h_local its final state from a zero start), so:
 
-1. each rank scans its shard from zero, keeping only the final state, and
-   sums its delta (:func:`shard_summary`);
+1. each rank runs its shard from zero for the final state alone (the
+   state-only scan: no readout or outputs) and sums its delta
+   (:func:`shard_summary`);
 2. the ranks all-gather those summaries (one small collective:
    batch * dim * (dstate + 2) words per rank);
 3. each rank folds the summaries of the ranks before it into its true
@@ -30,11 +31,19 @@ from . import binding
 def shard_summary(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
                   workspace=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """(delta sum (batch, dim) fp64, final state from zero (batch, dim, N)
-    fp32) of this rank's shard."""
-    out = torch.empty_like(u)
-    _, h_local = binding.mamba_scan_fwd(u, delta, A, B, C, D=D, z=z, delta_bias=delta_bias,
-                                        delta_softplus=delta_softplus, out=out,
-                                        return_last_state=True, workspace=workspace)
+    fp32) of this rank's shard.  The state comes from the state-only scan;
+    where its kernel cannot run (dstate > 16, rows not whole 16-byte
+    vectors) from a full scan whose outputs are dropped."""
+    try:
+        h_local = binding.mamba_scan_state(u, delta, A, B, delta_bias=delta_bias, delta_softplus=delta_softplus,
+                                           workspace=workspace)
+    except binding.MambaError as e:
+        if e.code != binding.MAMBA_ERR_UNSUPPORTED:
+            raise
+        out = torch.empty_like(u)
+        _, h_local = binding.mamba_scan_fwd(u, delta, A, B, C, D=D, z=z, delta_bias=delta_bias,
+                                            delta_softplus=delta_softplus, out=out,
+                                            return_last_state=True, workspace=workspace)
     sums = binding.mamba_delta_sum(delta, delta_bias, delta_softplus)
     return sums, h_local
 

@@ -293,3 +293,25 @@ def test_checked_build_exports_the_same_abi():
     assert checked.mamba_bounds_checked() == 1
     assert binding.load_library().mamba_bounds_checked() == 0
     assert binding.load_library().mamba_debug_shrink_output_extent(0) == 0
+
+
+def test_scan_state_validation(lib):
+    vp = ctypes.c_void_p
+    P = [vp(0x1000000 * (i + 1)) for i in range(8)]
+    ws_n = lib.mamba_scan_workspace_size(2, 8, 64, 16, 1)
+    # u delta A B bias softplus h0 last_state batch dim L N act ws wsb stream
+    ok = [P[0], P[1], P[2], P[3], None, 1, None, P[4], 2, 8, 64, 16, 1, None, 0, None]
+    names = ["u", "delta", "A", "B", "bias", "sp", "h0", "last", "batch", "dim", "L", "N", "act", "ws", "wsb"]
+
+    def call(**kw):
+        a = list(ok)
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return lib.mamba_scan_state(*a)
+    assert call(u=None) == -1 and call(B=None) == -1 and call(last=None) == -1
+    assert call(batch=0) == -2 and call(act=2) == -3
+    assert call(last=vp(0x2000000 + 64)) == -7            # last_state inside delta
+    assert call(h0=vp(0x5000000 + 4)) == -7               # h0 overlaps last_state, not exactly
+    assert call(ws=vp(0x7000008), wsb=ws_n) == -8         # misaligned workspace
+    assert call(ws=vp(0x7000000), wsb=ws_n - 16) == -8    # small workspace
+    assert call(ws=vp(0x1000000 + 256), wsb=ws_n) == -7   # workspace over u

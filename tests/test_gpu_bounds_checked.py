@@ -98,6 +98,22 @@ def test_device_wide_scan_and_checkpoints(checked, lanes):
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("with_ws", [False, True])
+def test_state_only_scan(checked, dtype, with_ws):
+    """The lane-split kernel run for the final state alone: C, z and out are
+    not passed, so any access to them would leave its (empty) range."""
+    w = inputs.custom(3, 70, 1000, 16, dtype, seed=36)
+    ins = inputs.scan_inputs(w, device="cuda")
+    h0 = inputs.initial_state(3, 70, 16, seed=8, device="cuda")
+    ws = torch.empty(binding.mamba_scan_workspace_size(3, 70, 1000, 16, ins["u"].dtype), device="cuda",
+                     dtype=torch.uint8) if with_ws else None
+    run = lambda: binding.mamba_scan_state(ins["u"], ins["delta"], ins["A"], ins["B"],  # noqa: E731
+                                           delta_bias=ins["delta_bias"], h0=h0, workspace=ws)
+    ref, got = both(checked, run)
+    assert equal(ref, got)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 @pytest.mark.parametrize("shape,dstate,chunk", [((2, 70, 1000), 16, 64), ((3, 33, 344), 5, 0)],
                          ids=["2x70x1000-chunks64", "3x33x344-N5"])
 def test_one_lane_scan(checked, dtype, shape, dstate, chunk):
