@@ -794,9 +794,10 @@ def seqpar_shard(w, world, rank, device):
 
 
 def seqpar_run(w, world, rank, steps, warmup, device, ops=None, group=None):
-    """Time `steps` calls of the sequence split (each rank scans its shard
-    from zero, the ranks all-gather the shard summaries, each folds the shards
-    before it and scans its shard again) after `warmup` untimed ones; returns
+    """Time `steps` calls of the sequence split (each rank runs its shard
+    from zero for its final state alone, the ranks all-gather the shard
+    summaries, each folds the shards before it and scans its shard from the
+    result) after `warmup` untimed ones; returns
     (max over ranks of the time per step in ms, elements per step of the
     whole sequence).  ``ops`` replaces the per-shard steps (CPU stand-ins in
     the multi-process test)."""

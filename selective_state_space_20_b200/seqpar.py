@@ -14,8 +14,9 @@ delta per row, h_local its final state from a zero start), so:
    initial state (:func:`shard_initial_state`);
 4. each rank scans its shard again from that state (:func:`shard_outputs`).
 
-The exchange happens once per call, between two full scans of the shard;
-there is nothing to overlap it with, and its size is independent of L.
+The exchange happens once per call, between the state-only pass and the
+full scan of the shard; there is nothing to overlap it with, and its size is
+independent of L.
 Every step runs in the library's kernels; torch.distributed carries the
 exchange.
 """
