@@ -133,12 +133,21 @@ struct ChannelTranspose {
     __device__ __forceinline__ static void run(float (&v)[8], int lane) {
         constexpr int HALF = CNT / 2;
         const bool upper = (lane & K) != 0;
+        float recv[HALF], keep[HALF];
 #pragma unroll
         for (int i = 0; i < HALF; ++i) {
             const float send = upper ? v[i] : v[i + HALF];
-            const float keep = upper ? v[i + HALF] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, K);
+            keep[i] = upper ? v[i + HALF] : v[i];
+            recv[i] = __shfl_xor_sync(0xffffffffu, send, K);
         }
+        // the sums two at a time on the packed x2 add
+#pragma unroll
+        for (int i = 0; i + 1 < HALF; i += 2) {
+            const float2 s2 = __fadd2_rn(f2(keep[i], keep[i + 1]), f2(recv[i], recv[i + 1]));
+            v[i] = s2.x;
+            v[i + 1] = s2.y;
+        }
+        if (HALF & 1) v[HALF - 1] = keep[HALF - 1] + recv[HALF - 1];
         ChannelTranspose<K / 2, HALF>::run(v, lane);
     }
 };
@@ -155,20 +164,32 @@ template <typename X>
 struct QuadTranspose {
     __device__ __forceinline__ static void run(X (&part)[4][3], int lane) {
         const bool up2 = (lane & 2) != 0, up1 = (lane & 1) != 0;
+        X keep[2][3], recv[2][3];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
 #pragma unroll
             for (int q = 0; q < 3; ++q) {
                 const X send = up2 ? part[i][q] : part[i + 2][q];
-                const X keep = up2 ? part[i + 2][q] : part[i][q];
-                part[i][q] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                keep[i][q] = up2 ? part[i + 2][q] : part[i][q];
+                recv[i][q] = __shfl_xor_sync(0xffffffffu, send, 2);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+            if constexpr (std::is_same<X, float>::value) {  // steps 0 and 1 on one packed x2 add
+                const float2 s2 = __fadd2_rn(f2(keep[0][q], keep[1][q]), f2(recv[0][q], recv[1][q]));
+                part[0][q] = s2.x;
+                part[1][q] = s2.y;
+            } else {
+                part[0][q] = keep[0][q] + recv[0][q];
+                part[1][q] = keep[1][q] + recv[1][q];
             }
         }
 #pragma unroll
         for (int q = 0; q < 3; ++q) {
             const X send = up1 ? part[0][q] : part[1][q];
-            const X keep = up1 ? part[1][q] : part[0][q];
-            part[0][q] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+            const X keep1 = up1 ? part[1][q] : part[0][q];
+            part[0][q] = keep1 + __shfl_xor_sync(0xffffffffu, send, 1);
         }
     }
 };
