@@ -225,11 +225,12 @@ __device__ __forceinline__ void local_publish(volatile unsigned *flag, int lane,
     }
 }
 
-template <typename T, int R, bool SP, bool GATE, bool CONV, bool LOCAL, bool CL>
+template <typename T, int R, bool SP, bool GATE, bool CONV, bool LOCAL, bool CL, bool UNR>
 __global__ void __launch_bounds__(PairLaunch<R, LOCAL>::kWorkers * 32, PairLaunch<R, LOCAL>::kMinBlocks)
 scan_fwd_pairs_kernel(const Params p) {
     using W = PairSmem<T, R>;
     static_assert(!(CL && CONV), "the fused convolution reads the dense layout");
+    static_assert(!UNR || (R == 2 && !CONV && !CL), "the unrolled form fits the registers of lane pairs only");
     constexpr int kWorkers = PairLaunch<R, LOCAL>::kWorkers;
     constexpr bool ACC = sizeof(T) == 4;
     using Dk = Decay<ACC>;
@@ -245,6 +246,7 @@ scan_fwd_pairs_kernel(const Params p) {
     constexpr int kTC = W::kTC, V = W::V, CPR = W::CPR, CW = W::CW;
     constexpr int S = kNS / R;   // states per lane
     constexpr int OWN = 8 / R;   // outputs per lane per block of 8 timesteps
+    constexpr int kBlkUnroll = UNR ? kTC / 8 : 1;  // blocks of 8 timesteps in flight
     constexpr int PT = kTC / R;  // prologue timesteps per lane
     // Channel-last staging (CL: (batch, L, dim) activations, (batch, L, N) B
     // and C).  A stage then holds, per activation tensor, kTC rows of one
@@ -688,7 +690,14 @@ scan_fwd_pairs_kernel(const Params p) {
                 const unsigned char *zrow = sbuf + (2 * CW + sc) * W::ROWB;
                 unsigned char *orow = outt + sc * W::ROWB;
                 const float *sB0 = bc32 + S * sr;
-#pragma unroll 1
+                // UNR: the sub-chunk's blocks unrolled, so one block's readout,
+                // combine and epilogue overlap the next one's decays (Mamba-2.8B
+                // layer 527 -> 508 us, same results).  Launched only where no
+                // piece is two-phase: with warps running state-only and full
+                // pieces side by side it is slower (long context 6.5 -> 6.8 ms
+                // block-local, 5.8 -> 6.7 ms device-wide), and other forms
+                // (four lanes, fused conv1d, channel-last) would spill.
+#pragma unroll kBlkUnroll
                 for (int tb = 0; tb < kTC; tb += 8) {
                     const float *sB = sB0 + (tb / V) * (W::BLKB / 4);
                     const float *sC = sB + W::BARR / 4;
@@ -909,11 +918,11 @@ scan_fwd_pairs_kernel(const Params p) {
     }
 }
 
-template <typename T, int R, bool SP, bool GATE, bool CONV, bool LOCAL, bool CL = false>
+template <typename T, int R, bool SP, bool GATE, bool CONV, bool LOCAL, bool CL = false, bool UNR = false>
 cudaError_t launch_t(const Params &kp, int sm_count, cudaStream_t st) {
     using PL = PairLaunch<R, LOCAL>;
     const int smem = PL::kWorkers * PairSmem<T, R>::BYTES + (LOCAL ? LocalSmem<R>::BYTES : 0);
-    auto kern = scan_fwd_pairs_kernel<T, R, SP, GATE, CONV, LOCAL, CL>;
+    auto kern = scan_fwd_pairs_kernel<T, R, SP, GATE, CONV, LOCAL, CL, UNR>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     static const int per_sm = [&] {
@@ -943,6 +952,20 @@ cudaError_t launch_t(const Params &kp, int sm_count, cudaStream_t st) {
     return cudaLaunchKernelEx(&cfg, kern, kp);
 }
 
+// Whether any worker of the launch gets a share short enough for two-phase
+// pieces (the kernel's own test: 20 groups < 11 workers in its scope) -- in
+// the block-local form, the block with the fewest whole groups.
+template <int R, bool LOCAL>
+bool has_two_phase(const Params &kp, int sm_count) {
+    using PL = PairLaunch<R, LOCAL>;
+    const long long G = kp.n_groups;
+    if (LOCAL) {
+        const long long nb = G < sm_count ? G : sm_count;
+        return 20LL * (G / nb) < 11LL * PL::kWorkers;
+    }
+    return 20LL * G < 11LL * (long long)sm_count * PL::kMinBlocks * PL::kWorkers;
+}
+
 template <int R, bool LOCAL>
 cudaError_t launch_r(const Params &kp, int act, int sm_count, cudaStream_t st) {
     const bool gate = kp.z != nullptr;
@@ -967,6 +990,12 @@ cudaError_t launch_r(const Params &kp, int act, int sm_count, cudaStream_t st) {
                     : launch_t<float, R, true, false, true, LOCAL>(kp, sm_count, st);
     }
     if (act == kBF16) {
+        if (R == 2 && !kp.state_only && !has_two_phase<R, LOCAL>(kp, sm_count)) {  // the unrolled form
+            if (kp.softplus) return gate ? launch_t<BF, 2, true, true, false, LOCAL, false, true>(kp, sm_count, st)
+                                         : launch_t<BF, 2, true, false, false, LOCAL, false, true>(kp, sm_count, st);
+            return gate ? launch_t<BF, 2, false, true, false, LOCAL, false, true>(kp, sm_count, st)
+                        : launch_t<BF, 2, false, false, false, LOCAL, false, true>(kp, sm_count, st);
+        }
         if (kp.softplus) return gate ? launch_t<BF, R, true, true, false, LOCAL>(kp, sm_count, st)
                                      : launch_t<BF, R, true, false, false, LOCAL>(kp, sm_count, st);
         return gate ? launch_t<BF, R, false, true, false, LOCAL>(kp, sm_count, st)

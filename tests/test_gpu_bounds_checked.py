@@ -64,8 +64,10 @@ def equal(a, b):
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 @pytest.mark.parametrize("shape,dstate,lanes", [((2, 70, 336), 16, 2), ((3, 33, 1000), 5, 4),
-                                                ((1, 64, 8192), 16, 2), ((4, 1030, 256), 16, 0)],
-                         ids=["2x70x336-R2", "3x33x1000-N5-R4", "1x64x8192-two-phase", "4x1030x256-lanes-auto"])
+                                                ((1, 64, 8192), 16, 2), ((4, 1030, 256), 16, 0),
+                                                ((4, 2960, 96), 16, 2)],
+                         ids=["2x70x336-R2", "3x33x1000-N5-R4", "1x64x8192-two-phase", "4x1030x256-lanes-auto",
+                              "4x2960x96-unrolled"])
 def test_block_local_scan(checked, dtype, shape, dstate, lanes):
     b, d, L = shape
     ins = inputs.scan_inputs(inputs.custom(b, d, L, dstate, dtype, seed=b + d + L), device="cuda")
