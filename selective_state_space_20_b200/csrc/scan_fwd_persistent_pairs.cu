@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(PairLaunch<R, LOCAL>::kWorkers * 32, PairLaunc
 scan_fwd_pairs_kernel(const Params p) {
     using W = PairSmem<T, R>;
     static_assert(!(CL && CONV), "the fused convolution reads the dense layout");
-    static_assert(!UNR || (R == 2 && !CONV && !CL), "the unrolled form fits the registers of lane pairs only");
+    static_assert(!UNR || (R == 2 && !CL), "the unrolled form fits the registers of lane pairs only");
     constexpr int kWorkers = PairLaunch<R, LOCAL>::kWorkers;
     constexpr bool ACC = sizeof(T) == 4;
     using Dk = Decay<ACC>;
@@ -246,7 +246,9 @@ scan_fwd_pairs_kernel(const Params p) {
     constexpr int kTC = W::kTC, V = W::V, CPR = W::CPR, CW = W::CW;
     constexpr int S = kNS / R;   // states per lane
     constexpr int OWN = 8 / R;   // outputs per lane per block of 8 timesteps
-    constexpr int kBlkUnroll = UNR ? kTC / 8 : 1;  // blocks of 8 timesteps in flight
+    // blocks of 8 timesteps in flight (the fused conv1d's prologue leaves
+    // registers for two)
+    constexpr int kBlkUnroll = UNR ? (CONV ? 2 : kTC / 8) : 1;
     constexpr int PT = kTC / R;  // prologue timesteps per lane
     // Channel-last staging (CL: (batch, L, dim) activations, (batch, L, N) B
     // and C).  A stage then holds, per activation tensor, kTC rows of one
@@ -984,6 +986,9 @@ cudaError_t launch_r(const Params &kp, int act, int sm_count, cudaStream_t st) {
                     : launch_t<float, R, false, false, false, true, true>(kp, sm_count, st);
     }
     if (kp.conv_w) {  // fused conv1d prologue: softplus on (checked by the caller)
+        if (act == kBF16 && R == 2 && !has_two_phase<R, LOCAL>(kp, sm_count))
+            return gate ? launch_t<BF, 2, true, true, true, LOCAL, false, true>(kp, sm_count, st)
+                        : launch_t<BF, 2, true, false, true, LOCAL, false, true>(kp, sm_count, st);
         if (act == kBF16) return gate ? launch_t<BF, R, true, true, true, LOCAL>(kp, sm_count, st)
                                       : launch_t<BF, R, true, false, true, LOCAL>(kp, sm_count, st);
         return gate ? launch_t<float, R, true, true, true, LOCAL>(kp, sm_count, st)
