@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(PairLaunch<R, LOCAL>::kWorkers * 32, PairLaunc
 scan_fwd_pairs_kernel(const Params p) {
     using W = PairSmem<T, R>;
     static_assert(!(CL && CONV), "the fused convolution reads the dense layout");
-    static_assert(!UNR || (R == 2 && !CL), "the unrolled form fits the registers of lane pairs only");
+    static_assert(!UNR || R == 2, "the unrolled form fits the registers of lane pairs only");
     constexpr int kWorkers = PairLaunch<R, LOCAL>::kWorkers;
     constexpr bool ACC = sizeof(T) == 4;
     using Dk = Decay<ACC>;
@@ -694,11 +694,11 @@ scan_fwd_pairs_kernel(const Params p) {
                 const float *sB0 = bc32 + S * sr;
                 // UNR: the sub-chunk's blocks unrolled, so one block's readout,
                 // combine and epilogue overlap the next one's decays (Mamba-2.8B
-                // layer 527 -> 508 us, same results).  Launched only where no
+                // layer 527 -> 510 us, same results).  Launched only where no
                 // piece is two-phase: with warps running state-only and full
                 // pieces side by side it is slower (long context 6.5 -> 6.8 ms
-                // block-local, 5.8 -> 6.7 ms device-wide), and other forms
-                // (four lanes, fused conv1d, channel-last) would spill.
+                // block-local, 5.8 -> 6.7 ms device-wide); four lanes per
+                // channel would spill.
 #pragma unroll kBlkUnroll
                 for (int tb = 0; tb < kTC; tb += 8) {
                     const float *sB = sB0 + (tb / V) * (W::BLKB / 4);
@@ -974,6 +974,10 @@ cudaError_t launch_r(const Params &kp, int act, int sm_count, cudaStream_t st) {
     using BF = __nv_bfloat16;
     if (kp.channels_last) {  // block-local form only, no fused convolution
         if (!LOCAL || kp.conv_w) return cudaErrorInvalidValue;
+        // unrolled (with the gate: without it the channel-last form would spill)
+        if (act == kBF16 && R == 2 && gate && !kp.state_only && !has_two_phase<R, LOCAL>(kp, sm_count))
+            return kp.softplus ? launch_t<BF, 2, true, true, false, true, true, true>(kp, sm_count, st)
+                               : launch_t<BF, 2, false, true, false, true, true, true>(kp, sm_count, st);
         if (act == kBF16) {
             if (kp.softplus) return gate ? launch_t<BF, R, true, true, false, true, true>(kp, sm_count, st)
                                          : launch_t<BF, R, true, false, false, true, true>(kp, sm_count, st);
