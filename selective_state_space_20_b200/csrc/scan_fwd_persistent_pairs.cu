@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(PairLaunch<R, LOCAL>::kWorkers * 32, PairLaunc
 scan_fwd_pairs_kernel(const Params p) {
     using W = PairSmem<T, R>;
     static_assert(!(CL && CONV), "the fused convolution reads the dense layout");
-    static_assert(!UNR || R == 2, "the unrolled form fits the registers of lane pairs only");
+    static_assert(!UNR || R == 2 || (!CONV && !CL), "the unrolled form of four lanes: dense layout, no fused conv1d");
     constexpr int kWorkers = PairLaunch<R, LOCAL>::kWorkers;
     constexpr bool ACC = sizeof(T) == 4;
     using Dk = Decay<ACC>;
@@ -246,9 +246,9 @@ scan_fwd_pairs_kernel(const Params p) {
     constexpr int kTC = W::kTC, V = W::V, CPR = W::CPR, CW = W::CW;
     constexpr int S = kNS / R;   // states per lane
     constexpr int OWN = 8 / R;   // outputs per lane per block of 8 timesteps
-    // blocks of 8 timesteps in flight (the fused conv1d's prologue leaves
-    // registers for two)
-    constexpr int kBlkUnroll = UNR ? (CONV ? 2 : kTC / 8) : 1;
+    // blocks of 8 timesteps in flight (the fused conv1d's prologue, and the
+    // register cap of 12 warps with four lanes, leave room for two)
+    constexpr int kBlkUnroll = UNR ? ((CONV || R == 4) ? 2 : kTC / 8) : 1;
     constexpr int PT = kTC / R;  // prologue timesteps per lane
     // Channel-last staging (CL: (batch, L, dim) activations, (batch, L, N) B
     // and C).  A stage then holds, per activation tensor, kTC rows of one
@@ -999,11 +999,14 @@ cudaError_t launch_r(const Params &kp, int act, int sm_count, cudaStream_t st) {
                     : launch_t<float, R, true, false, true, LOCAL>(kp, sm_count, st);
     }
     if (act == kBF16) {
-        if (R == 2 && !kp.state_only && !has_two_phase<R, LOCAL>(kp, sm_count)) {  // the unrolled form
-            if (kp.softplus) return gate ? launch_t<BF, 2, true, true, false, LOCAL, false, true>(kp, sm_count, st)
-                                         : launch_t<BF, 2, true, false, false, LOCAL, false, true>(kp, sm_count, st);
-            return gate ? launch_t<BF, 2, false, true, false, LOCAL, false, true>(kp, sm_count, st)
-                        : launch_t<BF, 2, false, false, false, LOCAL, false, true>(kp, sm_count, st);
+        // the unrolled form (four lanes: with the gate only, else it would spill)
+        if (!kp.state_only && (R == 2 || gate) && !has_two_phase<R, LOCAL>(kp, sm_count)) {
+            if (gate)
+                return kp.softplus ? launch_t<BF, R, true, true, false, LOCAL, false, true>(kp, sm_count, st)
+                                   : launch_t<BF, R, false, true, false, LOCAL, false, true>(kp, sm_count, st);
+            if constexpr (R == 2)
+                return kp.softplus ? launch_t<BF, 2, true, false, false, LOCAL, false, true>(kp, sm_count, st)
+                                   : launch_t<BF, 2, false, false, false, LOCAL, false, true>(kp, sm_count, st);
         }
         if (kp.softplus) return gate ? launch_t<BF, R, true, true, false, LOCAL>(kp, sm_count, st)
                                      : launch_t<BF, R, true, false, false, LOCAL>(kp, sm_count, st);
