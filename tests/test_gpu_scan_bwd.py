@@ -188,10 +188,11 @@ def test_bwd_from_forward_checkpoints(dtype, shape, h0):
         assert e <= grad_tol(k, dtype), (k, e, errs)
 
 
-def test_forward_checkpoints_hold_the_states():
+@pytest.mark.parametrize("batch,dim", [(2, 70), (4, 2960)])  # the second: 740 groups, the unrolled form
+def test_forward_checkpoints_hold_the_states(batch, dim):
     """Entry s of the checkpoints is the state entering step 32 s: compared
     with the final state of a scan over the first 32 s steps."""
-    w = inputs.custom(2, 70, 160, 16, "bf16", seed=91)
+    w = inputs.custom(batch, dim, 160, 16, "bf16", seed=91)
     dev = inputs.scan_inputs(w, device="cuda")
     _, _, ck = binding.mamba_scan_fwd_ckpt(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],
                                            z=dev["z"], delta_bias=dev["delta_bias"])
